@@ -1,0 +1,213 @@
+"""Seeded synthetic inputs for the TTT scan (shared by the oracle tests, the CUDA tests and the bench).
+
+This module holds no arithmetic of the TTT method.  It draws the tensors the method takes as
+inputs, with the shapes and value distributions of the workloads on the TTT pages (the
+``TTTLinear.__init__`` listing on the nanhubrain/jiafeimiao pages for W0 ~ N(0, 0.02) and
+b0 = 0; the 125M / 1B layer shapes from ``TTT_STANDARD_CONFIGS``), and hands out the exact
+bits: fp32 arrays, or bf16 bit patterns (uint16) rounded to nearest-even from fp32 draws.
+
+Every element depends only on (seed, tensor tag, flat element index), so any chain's slice
+can be regenerated without drawing the whole tensor (see ``synth.c``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "synth.c")
+_LIB_PATH = os.path.join(_HERE, "libsynth.so")
+
+# Tensor tags: one independent stream per tensor.
+TAG = {
+    "XQ": 1, "XK": 2, "XV": 3, "LR": 4, "W0": 5, "LNW": 6, "LNB": 7,
+    "W1": 8, "W2": 9, "B0": 10, "B1": 11, "B2": 12,
+}
+
+SEED_BASE = 0x77170000
+
+
+def build(force: bool = False) -> str:
+    """Compile the generator (gcc, OpenMP).  Returns the shared-library path."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def _get_lib():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        u64, i64, dbl = ctypes.c_uint64, ctypes.c_int64, ctypes.c_double
+        fptr = ctypes.POINTER(ctypes.c_float)
+        lib.synth_stream_key.argtypes = [u64, u64]
+        lib.synth_stream_key.restype = u64
+        lib.synth_draw_u64.argtypes = [u64, u64]
+        lib.synth_draw_u64.restype = u64
+        lib.synth_normal_f32.argtypes = [u64, u64, i64, dbl, dbl, fptr]
+        lib.synth_normal_f32.restype = None
+        lib.synth_logistic_normal_f32.argtypes = [u64, u64, i64, dbl, fptr]
+        lib.synth_logistic_normal_f32.restype = None
+        _lib = lib
+    return _lib
+
+
+def stream_key(seed: int, tag: int) -> int:
+    return int(_get_lib().synth_stream_key(seed, tag))
+
+
+def normal(seed: int, tag: int, n: int, first: int = 0, mean: float = 0.0, std: float = 1.0) -> np.ndarray:
+    """n fp32 values mean + std*N(0,1), elements [first, first+n) of stream (seed, tag)."""
+    out = np.empty(n, dtype=np.float32)
+    if n:
+        _get_lib().synth_normal_f32(stream_key(seed, tag), first, n, mean, std,
+                                    out.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return out
+
+
+def logistic_normal(seed: int, tag: int, n: int, first: int = 0, denom: float = 1.0) -> np.ndarray:
+    """n fp32 values sigmoid(N(0,1)) / denom."""
+    out = np.empty(n, dtype=np.float32)
+    if n:
+        _get_lib().synth_logistic_normal_f32(stream_key(seed, tag), first, n, denom,
+                                             out.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    return out
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16 (nearest, ties to even); returns the uint16 bit patterns."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounded = (b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp32."""
+    return (np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+@dataclass
+class Workload:
+    """Shapes and distributions of one synthetic workload.
+
+    kind: "linear" (TTT-Linear prefill), "mlp" (TTT-MLP prefill) or "decode".
+    dtype: "f32" or "bf16" for XQ/XK/XV (and out); state and lr are always fp32.
+    x_std: std of XQ/XK/XV; ln: "unit" (ln_w=1, ln_b=0) or "random" (1+N(0,.1), N(0,.1)).
+    """
+    name: str
+    kind: str
+    B: int
+    H: int
+    L: int
+    d: int = 64
+    K: int = 16
+    dtype: str = "bf16"
+    x_std: float = 0.125
+    ln: str = "random"
+    hidden: int = 256
+    seed: int = SEED_BASE
+    eps: float = 1e-6
+    decode_steps: int = 0
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def chains(self) -> int:
+        return self.B * self.H
+
+
+def workload(index: int, **overrides) -> Workload:
+    """The five workloads of the TTT scan (layer shapes from TTT_STANDARD_CONFIGS)."""
+    seed = SEED_BASE + index
+    presets = {
+        0: Workload("ttt_linear_fp32_B1_H2_L64", "linear", B=1, H=2, L=64, dtype="f32",
+                    x_std=1.0 / 8.0, ln="unit", seed=seed),
+        1: Workload("ttt_linear_125m_B16_H12_L2048", "linear", B=16, H=12, L=2048, seed=seed),
+        2: Workload("ttt_linear_1b_B8_H32_L8192", "linear", B=8, H=32, L=8192, seed=seed),
+        3: Workload("ttt_mlp_B8_H32_L2048_h256", "mlp", B=8, H=32, L=2048, seed=seed),
+        4: Workload("ttt_linear_decode_B128_H32_prefill2048", "decode", B=128, H=32, L=2048,
+                    decode_steps=1024, seed=seed),
+    }
+    w = presets[index]
+    for k, v in overrides.items():
+        setattr(w, k, v)
+    return w
+
+
+def _x_tensor(w: Workload, tag: str, L: int | None = None, chains=None):
+    """[B,H,L,d] activations; returns fp32 values and (bf16 bits or None)."""
+    L = w.L if L is None else L
+    per = L * w.d
+    if chains is None:
+        vals = normal(w.seed, TAG[tag], w.chains * per, 0, 0.0, w.x_std).reshape(w.B, w.H, L, w.d)
+    else:
+        vals = np.stack([normal(w.seed, TAG[tag], per, c * per, 0.0, w.x_std) for c in chains])
+        vals = vals.reshape(len(chains), L, w.d)
+    if w.dtype == "bf16":
+        bits = f32_to_bf16_bits(vals)
+        return bf16_bits_to_f32(bits).reshape(vals.shape), bits.reshape(vals.shape)
+    return vals, None
+
+
+def linear_inputs(w: Workload, L: int | None = None, chains=None) -> dict:
+    """Inputs of ttt_linear_forward (and of a decode run over the same token stream).
+
+    Returns a dict of numpy arrays: XQ, XK, XV as fp32 values ([B,H,L,d], or [n,L,d] for a
+    chain subset), XQ_bits/XK_bits/XV_bits (uint16 bf16 patterns, bf16 workloads only),
+    lr [B,H,L] fp32 = sigmoid(N(0,1))/d, W0 [H,d,d] ~ N(0, 0.02), b0 [H,d] = 0,
+    ln_w, ln_b [H,d].  Values of a chain are identical whether drawn alone or in full.
+    """
+    L = w.L if L is None else L
+    out = {}
+    for t in ("XQ", "XK", "XV"):
+        vals, bits = _x_tensor(w, t, L, chains)
+        out[t] = vals
+        if bits is not None:
+            out[t + "_bits"] = bits
+    if chains is None:
+        out["lr"] = logistic_normal(w.seed, TAG["LR"], w.chains * L, 0, float(w.d)).reshape(w.B, w.H, L)
+    else:
+        out["lr"] = np.stack([logistic_normal(w.seed, TAG["LR"], L, c * L, float(w.d)) for c in chains])
+    out.update(state_inputs(w))
+    return out
+
+
+def state_inputs(w: Workload) -> dict:
+    """Per-head initial state and LayerNorm parameters."""
+    H, d = w.H, w.d
+    out = {}
+    if w.kind == "mlp":
+        h = w.hidden
+        out["W1"] = normal(w.seed, TAG["W1"], H * d * h, 0, 0.0, 0.02).reshape(H, d, h)
+        out["b1"] = np.zeros((H, h), np.float32)
+        out["W2"] = normal(w.seed, TAG["W2"], H * h * d, 0, 0.0, 0.02).reshape(H, h, d)
+        out["b2"] = np.zeros((H, d), np.float32)
+    else:
+        out["W0"] = normal(w.seed, TAG["W0"], H * d * d, 0, 0.0, 0.02).reshape(H, d, d)
+        out["b0"] = np.zeros((H, d), np.float32)
+    if w.ln == "unit":
+        out["ln_w"] = np.ones((H, d), np.float32)
+        out["ln_b"] = np.zeros((H, d), np.float32)
+    else:
+        out["ln_w"] = normal(w.seed, TAG["LNW"], H * d, 0, 1.0, 0.1).reshape(H, d)
+        out["ln_b"] = normal(w.seed, TAG["LNB"], H * d, 0, 0.0, 0.1).reshape(H, d)
+    return out
+
+
+def random_bias(w: Workload, tag: str, shape, std: float = 0.02) -> np.ndarray:
+    """A non-zero bias draw, for tests that must exercise the bias path."""
+    n = int(np.prod(shape))
+    return normal(w.seed, TAG[tag], n, 0, 0.0, std).reshape(shape)
+
+
+def chain_index(b: int, h: int, H: int) -> int:
+    return b * H + h
