@@ -1,0 +1,484 @@
+"""Benchmark of the TTT scan on B200: TTT layer tokens/s and the fraction of the per-layer roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,mlp,decode]
+
+One step = one ttt_linear_forward over the 1B-layer workload (B=8, H=32, L=8200, d=64, K=16,
+bf16 activations, fp32 state): every row of the path at once -- the partition, 512 full
+mini-batches, the 8-token remainder, the tail grads.  Tokens per step = B * L.  Inputs come from
+the seeded generator (synth/), resident in HBM before timing; they are 806 MB per step, larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same workload on its own GPU (the
+chains are independent; there is no exchange), `value` counts all ranks' tokens over the
+slowest rank's device time ("scaling": "weak").
+
+The JSON line also carries: `e2e` (the same call from pinned HOST buffers with the copies timed),
+`roofline` (the scan kernel's algorithmic bytes / its CUDA-event time vs the measured HBM copy
+bandwidth), `cpu_baseline` (the CPU oracle on a bounded sample, rank 0 at N=1), `clocks`
+(NVML samples taken during the timed region) and `rows` (the TTT-MLP prefill and the decode
+step, each timed the same way).  `--impl reference` times the oracle instead, as the reference
+arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+D = 64
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------------------------
+# algorithmic work (bytes that must cross HBM, tensor FLOPs) of one call
+# ---------------------------------------------------------------------------------------------
+def linear_bytes(B, H, L, tail_grads=True):
+    """Reads: XQ, XK, XV (bf16), lr (fp32), W0/b0 and ln_w/ln_b per head.  Writes: out (bf16),
+    W_last/b_last per chain, and the tail grads when requested."""
+    chains = B * H
+    per_token = 3 * D * 2 + 4 + D * 2
+    state = (D * D + D) * 4
+    return chains * L * per_token + H * state + H * 2 * D * 4 + chains * state * (2 if tail_grads else 1)
+
+
+def linear_flops(B, H, L, K=16):
+    """Dense Z = XK W, XQ W and the rank-K update (3 x 2 K d^2 per mini-batch) plus the
+    lower-triangular XQ XK^T, (eta*A) g and tril(eta) g (3 x 2 d K(K+1)/2)."""
+    n_mb = L // K + (1 if L % K else 0)
+    return B * H * n_mb * (3 * 2 * K * D * D + 3 * 2 * D * K * (K + 1) // 2)
+
+
+def mlp_bytes(B, H, L, hid=256):
+    chains = B * H
+    state = (2 * D * hid + hid + D) * 4
+    return chains * L * (3 * D * 2 + 4 + D * 2) + H * state + H * 2 * D * 4 + chains * state
+
+
+def mlp_flops(B, H, L, hid=256, K=16):
+    n_mb = L // K + (1 if L % K else 0)
+    dense = 7 * 2 * K * D * hid                  # Z1, XQ W1, Z2, Xbar2 W2, g2 W2^T, two updates
+    tri = 2 * (K * (K + 1) // 2) * (2 * D + 2 * hid)  # Attn1, Attn2, M1 g1, M2 g2
+    return B * H * n_mb * (dense + tri)
+
+
+def decode_bytes(B, H, commit_fraction=1.0 / 16):
+    """Per step and chain: read W, b, W_grad, b_grad; write W_grad, b_grad (and W, b on the
+    commit step, once per K steps); tokens xq, xk, xv, lr in, out out (bf16)."""
+    state = (D * D + D) * 4
+    return B * H * (3 * state + commit_fraction * state + 3 * D * 2 + 4 + D * 2)
+
+
+# ---------------------------------------------------------------------------------------------
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    return HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_traffic(kernel_src: str, key: str):
+    """dram bytes per launch from the committed ncu summary, if the kernel source is unchanged
+    since the counters were taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "test_rnn_layers_b200", "csrc", kernel_src)
+    if not os.path.exists(path) or not os.path.exists(src):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(key)
+    if not rec:
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return rec.get("dram_bytes_per_launch") if rec.get("source_sha256") == digest else None
+
+
+class ClockSampler:
+    """NVML samples of SM clock and clock-event reasons on one GPU, in a thread (read-only)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self.index = device_index
+        self._stop = threading.Event()
+        self._thread = None
+        self.active = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+            self.max_mhz = None
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, reasons, self.active))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+        return False
+
+    def summary(self):
+        busy = [s for s in self.samples if s[3]]
+        if not busy:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mask = 0
+        for s in busy:
+            mask |= s[2]
+        reasons = sorted(n for bit, n in self.REASONS.items() if mask & bit and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(s[1] for s in busy), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(busy)}
+
+
+# ---------------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(step, K, W, world, sampler=None):
+    """W untimed steps, then exactly K steps between CUDA events on the current stream, with a
+    barrier and a device synchronise on both sides; returns ms per step (max over ranks)."""
+    import torch
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.active = True
+    e0.record(s)
+    for _ in range(K):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.active = False
+    barrier(world)
+    torch.cuda.synchronize()
+    return max_over_ranks(world, e0.elapsed_time(e1) / K)
+
+
+def dev_act(x, name):
+    import torch
+    bits = np.ascontiguousarray(x[name + "_bits"]).view(np.int16)
+    return torch.from_numpy(bits).cuda().view(torch.bfloat16)
+
+
+def dev_f32(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+# ---------------------------------------------------------------------------------------------
+def bench_linear(args, world, rank, local, peaks):
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    w = synth.workload(2, L=8200)
+    x = synth.linear_inputs(w, values=False)
+    XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
+    lr, W0, b0, lnw, lnb = (dev_f32(x[k]) for k in ("lr", "W0", "b0", "ln_w", "ln_b"))
+    B, H, L = w.B, w.H, w.L
+    out = torch.empty_like(XQ)
+    Wl, bl = torch.empty(B, H, D, D, device="cuda"), torch.empty(B, H, D, device="cuda")
+    Wg, bg = torch.empty(B, H, D, D, device="cuda"), torch.empty(B, H, D, device="cuda")
+
+    def step():
+        ttt.ttt_linear_forward(XQ, XK, XV, lr, W0, b0, lnw, lnb, mini_batch=w.K, eps=w.eps, out=out,
+                               W_last=Wl, b_last=bl, W_grad_tail=Wg, b_grad_tail=bg, tail_grads=True)
+
+    with ClockSampler(local) as clk:
+        ms = time_steps(step, args.steps, args.warmup, world, clk)
+    ttt.ttt_device_status()  # raises if a kernel gave up on a bounded wait
+    tokens = B * L
+    value = world * tokens / (ms / 1e3)
+    hbm, tf_burst, _, which = peaks
+    nbytes = linear_bytes(B, H, L)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    traffic = kernel_traffic("linear_tc.cu", "linear_tc_kernel@1b_B8_H32_L8200")
+
+    # end to end through the public call from pinned host buffers
+    host_in = {n: t.cpu().pin_memory() for n, t in (("XQ", XQ), ("XK", XK), ("XV", XV), ("lr", lr))}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in (("out", out), ("W", Wl), ("b", bl))}
+    dev_in = {n: torch.empty_like(t, device="cuda") for n, t in host_in.items()}
+
+    def e2e_step():
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        ttt.ttt_linear_forward(dev_in["XQ"], dev_in["XK"], dev_in["XV"], dev_in["lr"], W0, b0, lnw, lnb,
+                               mini_batch=w.K, eps=w.eps, out=out, W_last=Wl, b_last=bl, W_grad_tail=Wg,
+                               b_grad_tail=bg, tail_grads=True)
+        host_out["out"].copy_(out, non_blocking=True)
+        host_out["W"].copy_(Wl, non_blocking=True)
+        host_out["b"].copy_(bl, non_blocking=True)
+
+    e2e_K = max(3, min(args.steps, 10))
+    e2e_ms = time_steps(e2e_step, e2e_K, 2, world)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    line = {
+        "metric": "TTT layer tokens/sec (1B shapes, B200) and % of per-layer roofline",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, synth/)",
+        "config": {"workload": "ttt_linear_prefill_1b_layer", "B": B, "H": H, "L": L, "d": D,
+                   "mini_batch": w.K, "chains_per_gpu": B * H, "global_batch": B * world,
+                   "activations": "bf16 [B,H,L,d]", "state": "fp32",
+                   "l2": f"inputs larger than L2 ({3 * B * H * L * D * 2 / 1e6:.0f} MB read per step), no flush",
+                   "parallelism": f"independent chains, {world} GPU(s), no collective"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "kernel": "linear_tc_kernel", "achieved": round(achieved, 1),
+                     "peak": hbm, "peak_source": f"{which} hbm_gbs", "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "algorithmic_bytes": nbytes,
+                     "traffic": traffic,
+                     "tensor_tflops": round(linear_flops(B, H, L) / (ms / 1e3) / 1e12, 2),
+                     "tensor_frac_of_bf16_peak": round(linear_flops(B, H, L) / (ms / 1e3) / 1e12 / tf_burst, 4)},
+        "e2e": {"value": round(world * tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+def bench_mlp(args, world, peaks):
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    w = synth.workload(3)
+    x = synth.linear_inputs(w, values=False)
+    XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
+    t = {k: dev_f32(x[k]) for k in ("lr", "W1", "b1", "W2", "b2", "ln_w", "ln_b")}
+    out = torch.empty_like(XQ)
+
+    def step():
+        ttt.ttt_mlp_forward(XQ, XK, XV, t["lr"], t["W1"], t["b1"], t["W2"], t["b2"], t["ln_w"], t["ln_b"],
+                            mini_batch=w.K, eps=w.eps, out=out)
+
+    K = max(3, min(args.steps, 10))
+    ms = time_steps(step, K, 3, world)
+    flops = mlp_flops(w.B, w.H, w.L)
+    hbm, tf_burst, _, which = peaks
+    tfl = flops / (ms / 1e3) / 1e12
+    return {"workload": "ttt_mlp_prefill_B8_H32_L2048_h256", "value": round(world * w.B * w.L / (ms / 1e3), 1),
+            "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": K, "gpu_launches": K,
+            "roofline": {"bound": "tensor", "achieved": round(tfl, 2), "peak": tf_burst,
+                         "peak_source": f"{which} bf16_tflops", "unit": "TFLOP/s",
+                         "frac": round(tfl / tf_burst, 4), "algorithmic_flops": flops,
+                         "hbm_frac": round(mlp_bytes(w.B, w.H, w.L) / (ms / 1e3) / 1e9 / hbm, 4)}}
+
+
+def bench_decode(args, world, peaks):
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    w = synth.workload(4, decode_steps=64)
+    x = synth.linear_inputs(w, values=False, t1=w.L)
+    _, W, b, Wg, bg = ttt.ttt_linear_forward(dev_act(x, "XQ"), dev_act(x, "XK"), dev_act(x, "XV"),
+                                             dev_f32(x["lr"]), dev_f32(x["W0"]), dev_f32(x["b0"]),
+                                             dev_f32(x["ln_w"]), dev_f32(x["ln_b"]), eps=w.eps, tail_grads=True)
+    lnw, lnb = dev_f32(x["ln_w"]), dev_f32(x["ln_b"])
+    del x
+    toks = synth.linear_inputs(w, values=False, t0=w.L, t1=w.L + w.decode_steps)
+    XQ, XK, XV = (dev_act(toks, n) for n in ("XQ", "XK", "XV"))
+    lr = dev_f32(toks["lr"])
+    out = torch.empty(w.B, w.H, D, dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    xs = [(XQ[:, :, i].contiguous(), XK[:, :, i].contiguous(), XV[:, :, i].contiguous(), lr[:, :, i].contiguous())
+          for i in range(w.decode_steps)]
+    pos = [w.L]
+
+    def one(i):
+        q, k, v, l = xs[i % w.decode_steps]
+        ttt.ttt_linear_decode_step(q, k, v, l, lnw, lnb, W, b, Wg, bg, seqlen_offset=pos[0], eps=w.eps, out=out)
+        pos[0] += 1
+
+    # each timed step starts with a cold L2 (the 133 MB state is about the L2 size): flush, then time it
+    K = max(16, args.steps)
+    for i in range(3):
+        one(i)
+    s = torch.cuda.current_stream()
+    total = 0.0
+    for i in range(K):
+        flush.fill_(float(i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        one(i)
+        e1.record(s)
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    ms = max_over_ranks(world, total / K)
+    hbm = peaks[0]
+    nbytes = decode_bytes(w.B, w.H)
+    return {"workload": "ttt_linear_decode_B128_H32_after_prefill2048", "value": round(world * w.B / (ms / 1e3), 1),
+            "unit": "tokens/s", "ms_per_step": round(ms, 5), "steps": K, "gpu_launches": K,
+            "l2": "flushed (256 MB write) before every timed step",
+            "roofline": {"bound": "hbm", "achieved": round(nbytes / (ms / 1e3) / 1e9, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(nbytes / (ms / 1e3) / 1e9 / hbm, 4),
+                         "algorithmic_bytes": int(nbytes)}}
+
+
+def cpu_baseline(seconds_target=12.0, chains_max=64):
+    """The oracle (fp64, single-threaded, as written) on a bounded sample of the 1B workload."""
+    import oracle
+    w = synth.workload(2, L=8200)
+    o = oracle.default()
+    done, tokens, t_total = 0, 0, 0.0
+    chains = []
+    while done < chains_max and t_total < seconds_target:
+        c = (done * 37) % w.chains
+        xs = synth.linear_inputs(w, chains=[c])
+        t0 = time.perf_counter()
+        o.linear_forward(xs["XQ"], xs["XK"], xs["XV"], xs["lr"], xs["W0"], xs["b0"], xs["ln_w"], xs["ln_b"],
+                         w.K, w.eps, chains=[c])
+        t_total += time.perf_counter() - t0
+        done += 1
+        tokens += w.L
+        chains.append(c)
+    return {"value": round(tokens / t_total, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} of {w.chains} chains of the 1B workload (L={w.L} each), fp64 oracle, "
+                      f"{t_total:.1f} s of CPU time"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the same workload and metric; each
+    step a bounded sample (4 chains of L=8200)."""
+    if rank != 0:
+        return
+    import oracle
+    w = synth.workload(2, L=8200)
+    o = oracle.default()
+    per_step = 4
+    samples = [synth.linear_inputs(w, chains=[(i * 53) % w.chains]) for i in range(per_step)]
+    ids = [(i * 53) % w.chains for i in range(per_step)]
+
+    def step():
+        for c, xs in zip(ids, samples):
+            o.linear_forward(xs["XQ"], xs["XK"], xs["XV"], xs["lr"], xs["W0"], xs["b0"], xs["ln_w"], xs["ln_b"],
+                             w.K, w.eps, chains=[c])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = per_step * w.L / dt
+    print(json.dumps({
+        "impl": "reference", "metric": "TTT layer tokens/sec (1B shapes, B200) and % of per-layer roofline",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded generator, synth/)",
+        "config": {"workload": "ttt_linear_prefill_1b_layer", "B": w.B, "H": w.H, "L": w.L, "d": D,
+                   "mini_batch": w.K, "sample_per_step": f"{per_step} chains"},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} chains of L={w.L} per step, fp64 oracle, single thread"},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rows", default="linear,mlp,decode",
+                    help="comma list: linear (the headline) plus mlp and decode rows in the same line")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, world, int(os.environ.get("RANK", "0")))
+        return
+
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    peaks = measured_peaks()
+    line = bench_linear(args, world, rank, local, peaks)
+    rows = [r.strip() for r in args.rows.split(",") if r.strip()]
+    extra = {}
+    if "mlp" in rows:
+        extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
+    if "decode" in rows:
+        extra["ttt_linear_decode"] = bench_decode(args, world, peaks)
+    if extra:
+        line["rows"] = extra
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

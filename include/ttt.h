@@ -1,0 +1,189 @@
+/*
+ * ttt.h -- C ABI of libttt.so: the TTT-Linear / TTT-MLP mini-batch test-time-training scan
+ * and the TTT-Linear cache decode step, for NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [walkthrough] "代码连连看——TTT" (jiafeimiao.top): TTTBase.forward, TTTLinear.ttt and
+ *                 compute_mini_batch (dual branch, primal branch) listings.
+ *   [explainer]   "测试时学习（TTT）原理解析：ttt-lm-pytorch如何让模型在推理时持续学习"
+ *                 (nanhubrain.csdn.net): TTTLinear.__init__ and the TTTCache section.
+ *   [readme]      the ttt-lm-pytorch README (downcodes.com mirror): TTT-Linear and TTT-MLP.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers into memory the caller owns (allocated by the
+ *    caller, e.g. PyTorch).  The library allocates no device memory and keeps no state across
+ *    calls except a thread-local last-error message and one device status word per device.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the legacy
+ *    default stream).  No call synchronises the stream, except ttt_device_status().
+ *  - A "chain" is one (batch b, head h) pair; chain index = b * H + h.
+ *  - Activations are [B, H, L, d] contiguous (the layout TTTLinear.ttt receives after the head
+ *    split), so one chain's mini-batch is one contiguous block of K * d elements.
+ *  - dtype selects the element type of XQ, XK, XV and out: TTT_F32 or TTT_BF16.  The output
+ *    takes the input dtype (the walkthrough allocates XQW_batch with the input dtype).  The
+ *    hidden state (W, b, grads), lr, token_eta, ln_w and ln_b are always float32.
+ *  - Only head dimension d = 64 is supported; mini_batch K in [1, 16].
+ *  - Return value: TTT_OK (0) or a negative TTT_ERR_* code; on error nothing has been enqueued
+ *    and ttt_last_error_message() describes the cause.  No C++ exception crosses the ABI.
+ *  - Argument errors are found on the host before any CUDA call, so they can be tested
+ *    without a GPU.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TTT_OK 0
+#define TTT_ERR_ARG (-1)         /* null required pointer, bad size, bad dtype or flag */
+#define TTT_ERR_ALIGN (-2)       /* a pointer is not aligned as documented */
+#define TTT_ERR_ALIAS (-3)       /* an output overlaps an input or another output */
+#define TTT_ERR_CUDA (-4)        /* a CUDA runtime/driver call or a launch failed */
+#define TTT_ERR_TIMEOUT (-5)     /* a bounded device-side wait expired (see ttt_device_status) */
+#define TTT_ERR_UNSUPPORTED (-6) /* valid but not implemented here (e.g. d != 64) */
+
+#define TTT_F32 0
+#define TTT_BF16 1
+
+/* flags for the forward calls */
+#define TTT_FLAG_FP32_COMPUTE 1u /* run bf16 inputs through the FFMA (fp32-compute) kernel */
+
+/* Bits of the device status word */
+#define TTT_STATUS_TIMEOUT 1u /* a kernel gave up on a bounded wait and returned early */
+
+/*
+ * ttt_partition -- split a sequence of L tokens into mini-batches of K.
+ * [walkthrough] TTTBase.forward: num_mini_batch = L // K full mini-batches run first, then
+ * reminder_len = L % K remaining tokens run as one mini-batch of size r.
+ *   L >= 0, mini_batch >= 1; n_full, rem: host pointers receiving L / K and L % K.
+ * Host-only, exact integer arithmetic.  Returns TTT_ERR_ARG on a bad argument.
+ */
+int ttt_partition(long long L, int mini_batch, long long* n_full, long long* rem);
+
+/* Static description of an error code; never NULL. */
+const char* ttt_error_string(int code);
+
+/* Message of the last failing call on this host thread ("" if none); valid until the next call. */
+const char* ttt_last_error_message(void);
+
+/*
+ * ttt_device_status -- read (and optionally clear) the status word that kernels on the CURRENT
+ * device set when a bounded wait expires.  Synchronises `stream`.  *status receives the
+ * TTT_STATUS_* bits (0 = healthy).  Returns TTT_ERR_TIMEOUT if the timeout bit was set,
+ * TTT_ERR_CUDA on a CUDA error, else TTT_OK.
+ */
+int ttt_device_status(void* stream, unsigned int* status, int clear);
+
+/*
+ * ttt_set_wait_limit -- test hook: cap on the polls of every bounded device-side wait issued
+ * by later launches from this process.  polls > 0: that cap; 0: the default (2^24 polls,
+ * far above any healthy wait); < 0: zero polls, so every bounded wait gives up at once.  This
+ * exercises the TTT_ERR_TIMEOUT path without faulting or hanging the GPU: the kernel raises
+ * the status bit, waits (with the default bound) for its own copies in flight and returns.
+ * Only the bf16 tensor-core prefill kernel has such waits.  Host-only; returns TTT_OK.
+ */
+int ttt_set_wait_limit(long long polls);
+
+/*
+ * ttt_linear_forward -- TTT-Linear prefill: the mini-batch TTT scan over L tokens of every
+ * chain ([walkthrough] TTTBase.forward, TTTLinear.ttt, compute_mini_batch).
+ *
+ * Per chain (b, h), with K = mini_batch, state (W, b) starting at (W0, b0):
+ *   for each mini-batch X of K tokens (then one tail mini-batch of r = L % K tokens):
+ *     Z = XK W + b;  g = d/dZ 1/2 ||LN(Z) - (XV - XK)||^2          (ln_fused_l2_bwd)
+ *     eta[i][j] = token_eta[i] * lr[j] for j <= i, else 0
+ *     Zbar = XQ W - (eta * tril(XQ XK^T)) g + b - tril(eta) g      (dual branch)
+ *     out  = XQ + LN(Zbar)                                         (ln_fwd, residual)
+ *     full mini-batch only: W -= (eta[K-1,:] * XK)^T g;  b -= sum_j eta[K-1,j] g_j
+ *   LN(u) = ln_w * (u - mean(u)) / sqrt(var(u) + eps) + ln_b, biased variance over d.
+ *
+ * Arguments:
+ *   XQ, XK, XV   [B,H,L,d] dtype, 16-byte aligned.  May be NULL only when L == 0.
+ *   lr           [B,H,L] float32, 4-byte aligned: the per-token learning rate (ttt_lr_eta).
+ *   token_eta    [K] float32 or NULL (= 1/(i+1), i = position inside the mini-batch).
+ *   W0, b0       float32, 16-byte aligned: [H,d,d] and [H,d] shared over the batch when
+ *                w0_batch_stride == 0 (the walkthrough tiles W1, b1 over B), or [B,H,d,d] and
+ *                [B,H,d] per chain when w0_batch_stride == H*d*d (a continuation).
+ *                W is indexed W[a][c]: Z[c] = sum_a XK[a] W[a][c] + b[c].
+ *   ln_w, ln_b   [H,d] float32: the per-head LayerNorm affine parameters (ttt_norm_*).
+ *   B, H, L, d   sizes: B, H >= 1; L >= 0; d == 64.  L == 0 copies the state only.
+ *   mini_batch   K in [1, 16].
+ *   eps          LayerNorm epsilon, > 0.
+ *   dtype        TTT_F32 or TTT_BF16.
+ *   flags        0 or TTT_FLAG_FP32_COMPUTE.  bf16 inputs run on the tensor-core kernel
+ *                (bf16 operands, fp32 accumulation and fp32 state) unless the flag asks for the
+ *                FFMA kernel; fp32 inputs always run on the FFMA kernel.
+ * Outputs (device, caller-allocated):
+ *   out          [B,H,L,d] dtype, 16-byte aligned (may be NULL when L == 0).
+ *   W_last, b_last  [B,H,d,d], [B,H,d] float32: the state after the last FULL mini-batch (the
+ *                tail's params are dropped, as TTTBase.forward does).  W_last may be the same
+ *                pointer as W0 (and b_last as b0) for an in-place update when the state is
+ *                per chain; no other overlap is allowed.
+ *   W_grad_tail, b_grad_tail  NULL, or [B,H,d,d], [B,H,d] float32 receiving the tail's
+ *                un-scaled grad sums sum_{j<r} lr_j XK_j^T g_j and sum_{j<r} lr_j g_j (zeros when
+ *                r == 0): with W_last/b_last they form the TTTCache state for decoding on.
+ */
+int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const float* lr,
+                       const float* token_eta, const float* W0, const float* b0,
+                       long long w0_batch_stride, const float* ln_w, const float* ln_b, int B,
+                       int H, long long L, int d, int mini_batch, float eps, int dtype,
+                       unsigned int flags, void* out, float* W_last, float* b_last,
+                       float* W_grad_tail, float* b_grad_tail, void* stream);
+
+/*
+ * ttt_mlp_forward -- TTT-MLP prefill ([readme]: the hidden state is a two-layer MLP;
+ * [walkthrough]: "TTTMLP is two TTTLinear stacked").  The state is
+ *   f(x) = gelu(x W1 + b1) W2 + b2,  gelu = tanh form, W1 [d,hid], W2 [hid,d],
+ * and each mini-batch takes the layer-wise dual update of ttt_linear_forward:
+ *   Z1 = XK W1 + b1, X2 = gelu(Z1), Z2 = X2 W2 + b2, g2 = d/dZ2 1/2||LN(Z2) - (XV - XK)||^2,
+ *   g1 = (g2 W2^T) * gelu'(Z1);
+ *   Zbar1 = XQ W1 - (eta * tril(XQ XK^T)) g1 + b1 - tril(eta) g1;  Xbar2 = gelu(Zbar1);
+ *   Zbar2 = Xbar2 W2 - (eta * tril(Xbar2 X2^T)) g2 + b2 - tril(eta) g2;  out = XQ + LN(Zbar2);
+ *   full mini-batch: W1 -= (eta[K-1,:] * XK)^T g1, W2 -= (eta[K-1,:] * X2)^T g2, biases alike.
+ * Arguments as ttt_linear_forward, with hidden == 256 (= 4 d), states W1_0 [H,d,hid],
+ * b1_0 [H,hid], W2_0 [H,hid,d], b2_0 [H,d] (w0_batch_stride 0), or per chain [B,H,...]
+ * (w0_batch_stride == H*d*hid), and outputs W1_last, b1_last, W2_last, b2_last per chain.
+ * The tail's params are dropped as in TTT-Linear; no tail grads are reported.
+ */
+int ttt_mlp_forward(const void* XQ, const void* XK, const void* XV, const float* lr,
+                    const float* token_eta, const float* W1_0, const float* b1_0,
+                    const float* W2_0, const float* b2_0, long long w0_batch_stride,
+                    const float* ln_w, const float* ln_b, int B, int H, long long L, int d,
+                    int hidden, int mini_batch, float eps, int dtype, unsigned int flags,
+                    void* out, float* W1_last, float* b1_last, float* W2_last, float* b2_last,
+                    void* stream);
+
+/*
+ * ttt_linear_decode_step -- one new token per chain through the TTTCache state
+ * ([walkthrough] TTTLinear.ttt: decoding reads the params from the cache and, the mini-batch
+ * not being a multiple of K, takes the primal branch so the grads can be stored;
+ * [explainer] TTTCache: last states + grads, seqlen_offset, mini_batch_size).
+ * With p = seqlen_offset % K (every chain shares one offset) and t = token_eta[p] (default
+ * 1/(p+1)):
+ *   z = xk W + b;  g = d/dz 1/2||LN(z) - (xv - xk)||^2;
+ *   W_grad += lr xk^T g;  b_grad += lr g;
+ *   out = xq + LN(xq (W - t W_grad) + (b - t b_grad));
+ *   if p == K-1: W -= t W_grad; b -= t b_grad; W_grad = 0; b_grad = 0   (commit)
+ * W, b hold the state committed at the last mini-batch boundary; W_grad, b_grad the
+ * lr-weighted grad sums of the tokens since.  After ttt_linear_forward over L tokens, the
+ * cache is (W_last, b_last, W_grad_tail, b_grad_tail) with seqlen_offset = L.
+ * Arguments:
+ *   xq, xk, xv  [B,H,d] dtype, 16-byte aligned;  lr [B,H] float32;  token_eta [K] or NULL.
+ *   ln_w, ln_b  [H,d] float32.
+ *   W, b, W_grad, b_grad  [B,H,d,d], [B,H,d], [B,H,d,d], [B,H,d] float32, 16-byte aligned,
+ *               read and written in place (the caller's cache).
+ *   seqlen_offset >= 0: absolute position of this token.  The caller advances it by one.
+ *   out         [B,H,d] dtype.
+ */
+int ttt_linear_decode_step(const void* xq, const void* xk, const void* xv, const float* lr,
+                           const float* token_eta, const float* ln_w, const float* ln_b,
+                           float* W, float* b, float* W_grad, float* b_grad, int B, int H,
+                           int d, int mini_batch, long long seqlen_offset, float eps, int dtype,
+                           void* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H_ */

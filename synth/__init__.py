@@ -143,40 +143,59 @@ def workload(index: int, **overrides) -> Workload:
     return w
 
 
-def _x_tensor(w: Workload, tag: str, L: int | None = None, chains=None):
-    """[B,H,L,d] activations; returns fp32 values and (bf16 bits or None)."""
-    L = w.L if L is None else L
-    per = L * w.d
-    if chains is None:
-        vals = normal(w.seed, TAG[tag], w.chains * per, 0, 0.0, w.x_std).reshape(w.B, w.H, L, w.d)
-    else:
-        vals = np.stack([normal(w.seed, TAG[tag], per, c * per, 0.0, w.x_std) for c in chains])
-        vals = vals.reshape(len(chains), L, w.d)
+def stream_length(w: Workload) -> int:
+    """Tokens per chain in the workload's stream: the prefill, then the decode tokens."""
+    return w.L + w.decode_steps
+
+
+def _window(w: Workload, tag: str, per_token: int, t0: int, t1: int, chains, draw) -> np.ndarray:
+    """Tokens [t0, t1) of every listed chain of a [chains, stream_length, per_token] stream."""
+    Ltot = stream_length(w)
+    ids = range(w.chains) if chains is None else chains
+    if chains is None and t0 == 0 and t1 == Ltot:
+        return draw(w.seed, TAG[tag], w.chains * Ltot * per_token, 0).reshape(w.chains, Ltot, per_token)
+    n = (t1 - t0) * per_token
+    out = np.empty((len(ids), t1 - t0, per_token), np.float32)
+    for i, c in enumerate(ids):
+        out[i] = draw(w.seed, TAG[tag], n, (c * Ltot + t0) * per_token).reshape(t1 - t0, per_token)
+    return out
+
+
+def _x_tensor(w: Workload, tag: str, t0: int, t1: int, chains=None, values: bool = True):
+    """Activations of tokens [t0, t1): fp32 values (None when values is False and the workload
+    is bf16) and bf16 bit patterns (None for fp32 workloads); [B,H,T,d] or [n,T,d]."""
+    vals = _window(w, tag, w.d, t0, t1, chains,
+                   lambda seed, tag_, n, first: normal(seed, tag_, n, first, 0.0, w.x_std))
+    shape = (w.B, w.H, t1 - t0, w.d) if chains is None else (len(chains), t1 - t0, w.d)
+    vals = vals.reshape(shape)
     if w.dtype == "bf16":
-        bits = f32_to_bf16_bits(vals)
-        return bf16_bits_to_f32(bits).reshape(vals.shape), bits.reshape(vals.shape)
+        bits = f32_to_bf16_bits(vals).reshape(shape)
+        del vals
+        return (bf16_bits_to_f32(bits).reshape(shape) if values else None), bits
     return vals, None
 
 
-def linear_inputs(w: Workload, L: int | None = None, chains=None) -> dict:
-    """Inputs of ttt_linear_forward (and of a decode run over the same token stream).
+def linear_inputs(w: Workload, chains=None, values: bool = True, t0: int = 0, t1: int | None = None) -> dict:
+    """Inputs of ttt_linear_forward / ttt_mlp_forward / the decode steps, for tokens [t0, t1) of
+    each chain's stream of stream_length(w) tokens (default: the whole stream).
 
-    Returns a dict of numpy arrays: XQ, XK, XV as fp32 values ([B,H,L,d], or [n,L,d] for a
-    chain subset), XQ_bits/XK_bits/XV_bits (uint16 bf16 patterns, bf16 workloads only),
-    lr [B,H,L] fp32 = sigmoid(N(0,1))/d, W0 [H,d,d] ~ N(0, 0.02), b0 [H,d] = 0,
-    ln_w, ln_b [H,d].  Values of a chain are identical whether drawn alone or in full.
+    Returns a dict of numpy arrays: XQ, XK, XV as fp32 values ([B,H,T,d], or [n,T,d] for a
+    chain subset; omitted for bf16 workloads when values is False, to save host memory),
+    XQ_bits/XK_bits/XV_bits (uint16 bf16 patterns, bf16 workloads only),
+    lr [B,H,T] fp32 = sigmoid(N(0,1))/d, and the per-head state and LayerNorm parameters
+    (state_inputs).  A chain's values are identical whether drawn alone, in a window or in full.
     """
-    L = w.L if L is None else L
+    t1 = stream_length(w) if t1 is None else t1
     out = {}
     for t in ("XQ", "XK", "XV"):
-        vals, bits = _x_tensor(w, t, L, chains)
-        out[t] = vals
+        vals, bits = _x_tensor(w, t, t0, t1, chains, values)
+        if vals is not None:
+            out[t] = vals
         if bits is not None:
             out[t + "_bits"] = bits
-    if chains is None:
-        out["lr"] = logistic_normal(w.seed, TAG["LR"], w.chains * L, 0, float(w.d)).reshape(w.B, w.H, L)
-    else:
-        out["lr"] = np.stack([logistic_normal(w.seed, TAG["LR"], L, c * L, float(w.d)) for c in chains])
+    lr = _window(w, "LR", 1, t0, t1, chains,
+                 lambda seed, tag_, n, first: logistic_normal(seed, tag_, n, first, float(w.d)))
+    out["lr"] = lr.reshape((w.B, w.H, t1 - t0) if chains is None else (len(chains), t1 - t0))
     out.update(state_inputs(w))
     return out
 

@@ -1,0 +1,229 @@
+"""Python binding of libttt.so: the TTT-Linear / TTT-MLP scan and the decode step on B200.
+
+Argument marshalling only -- every step of the computation runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream.  The functions carry the C-ABI names
+(include/ttt.h); each checks the tensors it is handed, allocates missing outputs with torch,
+calls the library and raises TTTError on a non-zero return code.
+
+If libttt.so is missing this module raises on first use: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libttt.so")
+
+TTT_OK = 0
+TTT_ERR_ARG = -1
+TTT_ERR_ALIGN = -2
+TTT_ERR_ALIAS = -3
+TTT_ERR_CUDA = -4
+TTT_ERR_TIMEOUT = -5
+TTT_ERR_UNSUPPORTED = -6
+TTT_F32 = 0
+TTT_BF16 = 1
+TTT_FLAG_FP32_COMPUTE = 1
+TTT_STATUS_TIMEOUT = 1
+
+EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
+           "ttt_set_wait_limit", "ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step")
+
+
+class TTTError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"[{code}] {message}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libttt.so with its signatures declared (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m test_rnn_layers_b200.build` "
+                               "(there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, ll, i, u, f = (ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
+                               ctypes.c_uint, ctypes.c_float)
+        L.ttt_partition.argtypes = [ll, i, ctypes.POINTER(ll), ctypes.POINTER(ll)]
+        L.ttt_error_string.argtypes = [i]
+        L.ttt_error_string.restype = ctypes.c_char_p
+        L.ttt_last_error_message.argtypes = []
+        L.ttt_last_error_message.restype = ctypes.c_char_p
+        L.ttt_device_status.argtypes = [vp, ctypes.POINTER(u), i]
+        L.ttt_set_wait_limit.argtypes = [ll]
+        L.ttt_linear_forward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
+                                         vp, fp, fp, fp, fp, vp]
+        L.ttt_mlp_forward.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, i, f, i,
+                                      u, vp, fp, fp, fp, fp, vp]
+        L.ttt_linear_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f, i,
+                                             vp, vp]
+        for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
+                     "ttt_mlp_forward", "ttt_linear_decode_step"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != TTT_OK:
+        raise TTTError(rc, lib().ttt_last_error_message().decode() or lib().ttt_error_string(rc).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TTT_F32
+    if t.dtype == torch.bfloat16:
+        return TTT_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+
+
+def _need(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def ttt_partition(L: int, mini_batch: int):
+    """(n_full, rem) = (L // K, L % K), computed by the library (host-only)."""
+    n, r = ctypes.c_longlong(), ctypes.c_longlong()
+    _check(lib().ttt_partition(L, mini_batch, ctypes.byref(n), ctypes.byref(r)))
+    return n.value, r.value
+
+
+def ttt_set_wait_limit(polls: int = 0):
+    """Cap the polls of bounded device waits of later launches (0 = default).  A test hook."""
+    _check(lib().ttt_set_wait_limit(polls))
+
+
+def ttt_device_status(clear: bool = True, stream=None) -> int:
+    """Synchronise the stream and return the device status bits; raises TTTError on a timeout."""
+    v = ctypes.c_uint()
+    _check(lib().ttt_device_status(_stream(stream), ctypes.byref(v), 1 if clear else 0))
+    return v.value
+
+
+def ttt_linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
+                       token_eta=None, out=None, W_last=None, b_last=None, W_grad_tail=None,
+                       b_grad_tail=None, tail_grads: bool = False, flags: int = 0, stream=None):
+    """TTT-Linear prefill over [B,H,L,64] activations (see include/ttt.h).
+
+    W0/b0: [H,64,64]/[H,64] shared over the batch, or [B,H,64,64]/[B,H,64] per chain.
+    Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail).
+    """
+    _need(XQ, "XQ")
+    B, H, L, d = XQ.shape
+    dt = XQ.dtype
+    for n, t in (("XK", XK), ("XV", XV)):
+        _need(t, n, dt, XQ.shape)
+    _need(lr, "lr", torch.float32, (B, H, L))
+    per_chain = W0.dim() == 4
+    _need(W0, "W0", torch.float32, (B, H, d, d) if per_chain else (H, d, d))
+    _need(b0, "b0", torch.float32, (B, H, d) if per_chain else (H, d))
+    _need(ln_w, "ln_w", torch.float32, (H, d))
+    _need(ln_b, "ln_b", torch.float32, (H, d))
+    if token_eta is not None:
+        _need(token_eta, "token_eta", torch.float32, (mini_batch,))
+    dev = XQ.device
+    out = torch.empty_like(XQ) if out is None else _need(out, "out", dt, XQ.shape)
+    W_last = torch.empty((B, H, d, d), device=dev) if W_last is None else _need(W_last, "W_last", torch.float32, (B, H, d, d))
+    b_last = torch.empty((B, H, d), device=dev) if b_last is None else _need(b_last, "b_last", torch.float32, (B, H, d))
+    if tail_grads:
+        W_grad_tail = torch.empty((B, H, d, d), device=dev) if W_grad_tail is None else W_grad_tail
+        b_grad_tail = torch.empty((B, H, d), device=dev) if b_grad_tail is None else b_grad_tail
+    rc = lib().ttt_linear_forward(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
+                                  H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
+                                  eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last),
+                                  _ptr(W_grad_tail), _ptr(b_grad_tail), _stream(stream))
+    _check(rc)
+    if tail_grads:
+        return out, W_last, b_last, W_grad_tail, b_grad_tail
+    return out, W_last, b_last
+
+
+def ttt_mlp_forward(XQ, XK, XV, lr, W1, b1, W2, b2, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
+                    token_eta=None, out=None, flags: int = 0, stream=None):
+    """TTT-MLP prefill; states W1 [H,64,256], b1 [H,256], W2 [H,256,64], b2 [H,64] (or per chain).
+
+    Returns (out, W1_last, b1_last, W2_last, b2_last).
+    """
+    _need(XQ, "XQ")
+    B, H, L, d = XQ.shape
+    dt = XQ.dtype
+    for n, t in (("XK", XK), ("XV", XV)):
+        _need(t, n, dt, XQ.shape)
+    _need(lr, "lr", torch.float32, (B, H, L))
+    hid = W1.shape[-1]
+    per_chain = W1.dim() == 4
+    pre = (B, H) if per_chain else (H,)
+    _need(W1, "W1", torch.float32, pre + (d, hid))
+    _need(b1, "b1", torch.float32, pre + (hid,))
+    _need(W2, "W2", torch.float32, pre + (hid, d))
+    _need(b2, "b2", torch.float32, pre + (d,))
+    _need(ln_w, "ln_w", torch.float32, (H, d))
+    _need(ln_b, "ln_b", torch.float32, (H, d))
+    if token_eta is not None:
+        _need(token_eta, "token_eta", torch.float32, (mini_batch,))
+    dev = XQ.device
+    out = torch.empty_like(XQ) if out is None else _need(out, "out", dt, XQ.shape)
+    W1l = torch.empty((B, H, d, hid), device=dev)
+    b1l = torch.empty((B, H, hid), device=dev)
+    W2l = torch.empty((B, H, hid, d), device=dev)
+    b2l = torch.empty((B, H, d), device=dev)
+    rc = lib().ttt_mlp_forward(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W1), _ptr(b1),
+                               _ptr(W2), _ptr(b2), H * d * hid if per_chain else 0, _ptr(ln_w), _ptr(ln_b),
+                               B, H, L, d, hid, mini_batch, eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W1l),
+                               _ptr(b1l), _ptr(W2l), _ptr(b2l), _stream(stream))
+    _check(rc)
+    return out, W1l, b1l, W2l, b2l
+
+
+def ttt_linear_decode_step(xq, xk, xv, lr, ln_w, ln_b, W, b, W_grad, b_grad, seqlen_offset: int,
+                           mini_batch: int = 16, eps: float = 1e-6, token_eta=None, out=None, stream=None):
+    """One decode token per chain ([B,H,64] inputs) through the cache state (W, b, W_grad, b_grad),
+    which is updated in place.  Returns out [B,H,64]."""
+    _need(xq, "xq")
+    B, H, d = xq.shape
+    dt = xq.dtype
+    for n, t in (("xk", xk), ("xv", xv)):
+        _need(t, n, dt, xq.shape)
+    _need(lr, "lr", torch.float32, (B, H))
+    _need(ln_w, "ln_w", torch.float32, (H, d))
+    _need(ln_b, "ln_b", torch.float32, (H, d))
+    _need(W, "W", torch.float32, (B, H, d, d))
+    _need(b, "b", torch.float32, (B, H, d))
+    _need(W_grad, "W_grad", torch.float32, (B, H, d, d))
+    _need(b_grad, "b_grad", torch.float32, (B, H, d))
+    if token_eta is not None:
+        _need(token_eta, "token_eta", torch.float32, (mini_batch,))
+    out = torch.empty_like(xq) if out is None else _need(out, "out", dt, xq.shape)
+    rc = lib().ttt_linear_decode_step(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(lr), _ptr(token_eta), _ptr(ln_w),
+                                      _ptr(ln_b), _ptr(W), _ptr(b), _ptr(W_grad), _ptr(b_grad), B, H, d,
+                                      mini_batch, seqlen_offset, eps, _dtype_code(xq), _ptr(out), _stream(stream))
+    _check(rc)
+    return out

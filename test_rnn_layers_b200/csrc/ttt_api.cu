@@ -1,0 +1,359 @@
+// ttt_api.cu -- the extern "C" boundary of libttt.so (declared in include/ttt.h).
+//
+// Argument checks run on the host before any CUDA call; each entry point then picks a kernel
+// and enqueues it on the caller's stream.  No device memory is allocated here.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/ttt.h"
+#include "ttt_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<long long> g_wait_limit{0};
+constexpr long long kDefaultWaitPolls = 1ll << 24;
+constexpr int kD = 64;
+constexpr int kHidden = 256;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int ok() {
+    g_last_error.clear();
+    return TTT_OK;
+}
+
+bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+// A byte range [p, p + n) of one argument, for the overlap checks.
+struct Span {
+    const char* name;
+    const void* p;
+    size_t n;
+};
+
+bool overlaps(const Span& x, const Span& y) {
+    if (!x.p || !y.p || x.n == 0 || y.n == 0) return false;
+    auto a = reinterpret_cast<uintptr_t>(x.p), b = reinterpret_cast<uintptr_t>(y.p);
+    return a < b + y.n && b < a + x.n;
+}
+
+// outputs must not overlap inputs or each other; `same_ok` lists (output, input) index pairs
+// allowed to be the SAME buffer (identical pointer and size: an in-place state update).
+int check_aliasing(const Span* in, int nin, const Span* out, int nout,
+                   const int (*same_ok)[2] = nullptr, int nsame = 0) {
+    for (int o = 0; o < nout; ++o) {
+        for (int i = 0; i < nin; ++i) {
+            if (!overlaps(out[o], in[i])) continue;
+            bool allowed = false;
+            for (int k = 0; k < nsame; ++k)
+                if (same_ok[k][0] == o && same_ok[k][1] == i && out[o].p == in[i].p && out[o].n == in[i].n)
+                    allowed = true;
+            if (!allowed)
+                return fail(TTT_ERR_ALIAS, "output %s overlaps input %s", out[o].name, in[i].name);
+        }
+        for (int p = o + 1; p < nout; ++p)
+            if (overlaps(out[o], out[p]))
+                return fail(TTT_ERR_ALIAS, "outputs %s and %s overlap", out[o].name, out[p].name);
+    }
+    return TTT_OK;
+}
+
+unsigned int* status_word();  // device address of the status word of the current device
+
+// polls per bounded device wait: the default, a caller's cap, or 0 polls (give up at once)
+long long wait_limit() {
+    long long v = g_wait_limit.load();
+    return v == 0 ? kDefaultWaitPolls : (v < 0 ? 0 : v);
+}
+
+// ---- driver entry point for tensor-map encoding (no link-time libcuda dependency) ----------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [chains, L, 64] bf16 viewed 3-D; box {64, K, 1}; 128-byte swizzle; out-of-range rows read 0.
+int encode_act_map(CUtensorMap* map, const void* base, long long chains, long long L, int K,
+                   const char* name) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return fail(TTT_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(chains)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(L) * kD * 2};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(K), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TTT_ERR_CUDA, "tensor map for %s: cuTensorMapEncodeTiled error %d", name, (int)r);
+    return TTT_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(TTT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Common checks of the prefill entry points.
+int check_common(int B, int H, long long L, int d, int K, float eps, int dtype, unsigned int flags) {
+    if (B < 1 || H < 1) return fail(TTT_ERR_ARG, "B and H must be >= 1 (got %d, %d)", B, H);
+    if (static_cast<long long>(B) * H > (1ll << 31) - 1) return fail(TTT_ERR_ARG, "B*H too large");
+    if (L < 0) return fail(TTT_ERR_ARG, "L must be >= 0 (got %lld)", L);
+    if (L > (1ll << 31) - 1) return fail(TTT_ERR_ARG, "L too large (%lld)", L);
+    if (d != kD) return fail(TTT_ERR_UNSUPPORTED, "only head dim d = 64 is supported (got %d)", d);
+    if (K < 1 || K > 16) return fail(TTT_ERR_ARG, "mini_batch must be in [1, 16] (got %d)", K);
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(TTT_ERR_ARG, "eps must be finite and > 0");
+    if (dtype != TTT_F32 && dtype != TTT_BF16) return fail(TTT_ERR_ARG, "dtype must be TTT_F32 or TTT_BF16");
+    if (flags & ~TTT_FLAG_FP32_COMPUTE) return fail(TTT_ERR_ARG, "unknown flags 0x%x", flags);
+    return TTT_OK;
+}
+
+}  // namespace
+
+// The status word.  Kernels OR TTT_STATUS_* bits into it; ttt_device_status reads it.
+__device__ unsigned int g_ttt_status;
+
+namespace {
+unsigned int* status_word() {
+    static std::mutex mu;
+    static unsigned int* ptrs[256] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_ttt_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<unsigned int*>(p);
+    }
+    return ptrs[dev];
+}
+}  // namespace
+
+extern "C" {
+
+int ttt_partition(long long L, int mini_batch, long long* n_full, long long* rem) {
+    if (!n_full || !rem) return fail(TTT_ERR_ARG, "n_full and rem must be non-null");
+    if (L < 0) return fail(TTT_ERR_ARG, "L must be >= 0 (got %lld)", L);
+    if (mini_batch < 1) return fail(TTT_ERR_ARG, "mini_batch must be >= 1 (got %d)", mini_batch);
+    *n_full = L / mini_batch;
+    *rem = L % mini_batch;
+    return ok();
+}
+
+const char* ttt_error_string(int code) {
+    switch (code) {
+        case TTT_OK: return "ok";
+        case TTT_ERR_ARG: return "invalid argument";
+        case TTT_ERR_ALIGN: return "misaligned pointer";
+        case TTT_ERR_ALIAS: return "output overlaps another buffer";
+        case TTT_ERR_CUDA: return "CUDA error";
+        case TTT_ERR_TIMEOUT: return "device-side wait timed out";
+        case TTT_ERR_UNSUPPORTED: return "unsupported configuration";
+        default: return "unknown error code";
+    }
+}
+
+const char* ttt_last_error_message(void) { return g_last_error.c_str(); }
+
+int ttt_set_wait_limit(long long polls) {
+    g_wait_limit.store(polls);
+    return ok();
+}
+
+int ttt_device_status(void* stream, unsigned int* status, int clear) {
+    if (!status) return fail(TTT_ERR_ARG, "status must be non-null");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned int* word = status_word();
+    if (!word) return fail(TTT_ERR_CUDA, "no device status word on the current device");
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(word, 0, sizeof(unsigned int), st);
+    if (e == cudaSuccess && clear) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+    *status = v;
+    if (v & TTT_STATUS_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a kernel gave up on a bounded wait");
+    return ok();
+}
+
+int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const float* lr,
+                       const float* token_eta, const float* W0, const float* b0,
+                       long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                       long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                       void* out, float* W_last, float* b_last, float* W_grad_tail,
+                       float* b_grad_tail, void* stream) {
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
+    if (rc) return rc;
+    const long long chains = static_cast<long long>(B) * H;
+    const long long per_head = static_cast<long long>(kD) * kD;
+    if (w0_batch_stride != 0 && w0_batch_stride != H * per_head)
+        return fail(TTT_ERR_ARG, "w0_batch_stride must be 0 or H*d*d (got %lld)", w0_batch_stride);
+    if (!W0 || !b0 || !ln_w || !ln_b || !W_last || !b_last)
+        return fail(TTT_ERR_ARG, "W0, b0, ln_w, ln_b, W_last and b_last must be non-null");
+    if (L > 0 && (!XQ || !XK || !XV || !lr || !out))
+        return fail(TTT_ERR_ARG, "XQ, XK, XV, lr and out must be non-null when L > 0");
+    const void* a16[] = {XQ, XK, XV, out, W0, b0, W_last, b_last, W_grad_tail, b_grad_tail};
+    const char* n16[] = {"XQ", "XK", "XV", "out", "W0", "b0", "W_last", "b_last", "W_grad_tail", "b_grad_tail"};
+    for (int i = 0; i < 10; ++i)
+        if (a16[i] && !aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "%s must be 16-byte aligned", n16[i]);
+    const void* a4[] = {lr, token_eta, ln_w, ln_b};
+    const char* n4[] = {"lr", "token_eta", "ln_w", "ln_b"};
+    for (int i = 0; i < 4; ++i)
+        if (a4[i] && !aligned(a4[i], 4)) return fail(TTT_ERR_ALIGN, "%s must be 4-byte aligned", n4[i]);
+
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t act = static_cast<size_t>(chains) * L * kD * esz;
+    const long long wrows = w0_batch_stride ? chains : H;
+    Span in[] = {{"XQ", XQ, act}, {"XK", XK, act}, {"XV", XV, act}, {"lr", lr, static_cast<size_t>(chains * L) * 4},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
+                 {"W0", W0, static_cast<size_t>(wrows * per_head) * 4}, {"b0", b0, static_cast<size_t>(wrows * kD) * 4},
+                 {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    Span outs[] = {{"out", out, act}, {"W_last", W_last, static_cast<size_t>(chains * per_head) * 4},
+                   {"b_last", b_last, static_cast<size_t>(chains * kD) * 4},
+                   {"W_grad_tail", W_grad_tail, static_cast<size_t>(chains * per_head) * 4},
+                   {"b_grad_tail", b_grad_tail, static_cast<size_t>(chains * kD) * 4}};
+    const int same_ok[2][2] = {{1, 5}, {2, 6}};  // W_last == W0, b_last == b0 (per-chain state)
+    rc = check_aliasing(in, 9, outs, 5, same_ok, 2);
+    if (rc) return rc;
+
+    ttt::LinearArgs a{};
+    a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
+    a.W0 = W0; a.b0 = b0; a.w0_chain_stride = w0_batch_stride ? per_head : 0;
+    a.ln_w = ln_w; a.ln_b = ln_b; a.B = B; a.H = H; a.L = L; a.K = mini_batch;
+    a.n_full = L / mini_batch; a.rem = L % mini_batch; a.eps = eps;
+    a.out = out; a.W_last = W_last; a.b_last = b_last; a.W_grad_tail = W_grad_tail; a.b_grad_tail = b_grad_tail;
+    a.status = status_word();
+    a.wait_limit = wait_limit();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    cudaError_t e;
+    if (L == 0) {
+        e = ttt::launch_linear_state_copy(a, st);
+    } else if (dtype == TTT_F32 || (flags & TTT_FLAG_FP32_COMPUTE)) {
+        e = ttt::launch_linear_simt(a, dtype, st);
+    } else {
+        ttt::LinearMaps maps;
+        if ((rc = encode_act_map(&maps.xq, XQ, chains, L, mini_batch, "XQ"))) return rc;
+        if ((rc = encode_act_map(&maps.xk, XK, chains, L, mini_batch, "XK"))) return rc;
+        if ((rc = encode_act_map(&maps.xv, XV, chains, L, mini_batch, "XV"))) return rc;
+        if ((rc = encode_act_map(&maps.out, out, chains, L, mini_batch, "out"))) return rc;
+        e = ttt::launch_linear_tc(a, maps, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward launch");
+    return ok();
+}
+
+int ttt_mlp_forward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                    const float* W1_0, const float* b1_0, const float* W2_0, const float* b2_0,
+                    long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H, long long L,
+                    int d, int hidden, int mini_batch, float eps, int dtype, unsigned int flags, void* out,
+                    float* W1_last, float* b1_last, float* W2_last, float* b2_last, void* stream) {
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
+    if (rc) return rc;
+    if (hidden != kHidden) return fail(TTT_ERR_UNSUPPORTED, "only hidden = 256 is supported (got %d)", hidden);
+    const long long chains = static_cast<long long>(B) * H;
+    const long long per_head = static_cast<long long>(kD) * kHidden;
+    if (w0_batch_stride != 0 && w0_batch_stride != H * per_head)
+        return fail(TTT_ERR_ARG, "w0_batch_stride must be 0 or H*d*hidden (got %lld)", w0_batch_stride);
+    if (!W1_0 || !b1_0 || !W2_0 || !b2_0 || !ln_w || !ln_b || !W1_last || !b1_last || !W2_last || !b2_last)
+        return fail(TTT_ERR_ARG, "state, LayerNorm and state-output pointers must be non-null");
+    if (L > 0 && (!XQ || !XK || !XV || !lr || !out))
+        return fail(TTT_ERR_ARG, "XQ, XK, XV, lr and out must be non-null when L > 0");
+    const void* a16[] = {XQ, XK, XV, out, W1_0, b1_0, W2_0, b2_0, W1_last, b1_last, W2_last, b2_last};
+    for (int i = 0; i < 12; ++i)
+        if (a16[i] && !aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "tensor argument %d must be 16-byte aligned", i);
+    const void* a4[] = {lr, token_eta, ln_w, ln_b};
+    for (int i = 0; i < 4; ++i)
+        if (a4[i] && !aligned(a4[i], 4)) return fail(TTT_ERR_ALIGN, "lr/token_eta/ln_w/ln_b must be 4-byte aligned");
+
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t act = static_cast<size_t>(chains) * L * kD * esz;
+    const long long rows = w0_batch_stride ? chains : H;
+    Span in[] = {{"XQ", XQ, act}, {"XK", XK, act}, {"XV", XV, act}, {"lr", lr, static_cast<size_t>(chains * L) * 4},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
+                 {"W1_0", W1_0, static_cast<size_t>(rows * per_head) * 4}, {"b1_0", b1_0, static_cast<size_t>(rows * kHidden) * 4},
+                 {"W2_0", W2_0, static_cast<size_t>(rows * per_head) * 4}, {"b2_0", b2_0, static_cast<size_t>(rows * kD) * 4},
+                 {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    Span outs[] = {{"out", out, act}, {"W1_last", W1_last, static_cast<size_t>(chains * per_head) * 4},
+                   {"b1_last", b1_last, static_cast<size_t>(chains * kHidden) * 4},
+                   {"W2_last", W2_last, static_cast<size_t>(chains * per_head) * 4},
+                   {"b2_last", b2_last, static_cast<size_t>(chains * kD) * 4}};
+    const int same_ok[4][2] = {{1, 5}, {2, 6}, {3, 7}, {4, 8}};
+    rc = check_aliasing(in, 11, outs, 5, same_ok, 4);
+    if (rc) return rc;
+
+    ttt::MlpArgs a{};
+    a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
+    a.W1_0 = W1_0; a.b1_0 = b1_0; a.W2_0 = W2_0; a.b2_0 = b2_0;
+    a.w0_chain_stride = w0_batch_stride ? per_head : 0;
+    a.ln_w = ln_w; a.ln_b = ln_b; a.B = B; a.H = H; a.L = L; a.K = mini_batch;
+    a.n_full = L / mini_batch; a.rem = L % mini_batch; a.eps = eps; a.out = out;
+    a.W1_last = W1_last; a.b1_last = b1_last; a.W2_last = W2_last; a.b2_last = b2_last;
+    a.status = status_word();
+    a.wait_limit = wait_limit();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = L == 0 ? ttt::launch_mlp_state_copy(a, st) : ttt::launch_mlp_simt(a, dtype, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_mlp_forward launch");
+    return ok();
+}
+
+int ttt_linear_decode_step(const void* xq, const void* xk, const void* xv, const float* lr,
+                           const float* token_eta, const float* ln_w, const float* ln_b, float* W, float* b,
+                           float* W_grad, float* b_grad, int B, int H, int d, int mini_batch,
+                           long long seqlen_offset, float eps, int dtype, void* out, void* stream) {
+    int rc = check_common(B, H, 1, d, mini_batch, eps, dtype, 0);
+    if (rc) return rc;
+    if (seqlen_offset < 0) return fail(TTT_ERR_ARG, "seqlen_offset must be >= 0");
+    if (!xq || !xk || !xv || !lr || !ln_w || !ln_b || !W || !b || !W_grad || !b_grad || !out)
+        return fail(TTT_ERR_ARG, "all tensor arguments except token_eta must be non-null");
+    const void* a16[] = {xq, xk, xv, out, W, b, W_grad, b_grad};
+    for (int i = 0; i < 8; ++i)
+        if (!aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "tensor argument %d must be 16-byte aligned", i);
+    const void* a4[] = {lr, token_eta, ln_w, ln_b};
+    for (int i = 0; i < 4; ++i)
+        if (a4[i] && !aligned(a4[i], 4)) return fail(TTT_ERR_ALIGN, "lr/token_eta/ln_w/ln_b must be 4-byte aligned");
+    const long long chains = static_cast<long long>(B) * H;
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t vec = static_cast<size_t>(chains) * kD * esz;
+    const size_t mat = static_cast<size_t>(chains) * kD * kD * 4, bv = static_cast<size_t>(chains) * kD * 4;
+    Span in[] = {{"xq", xq, vec}, {"xk", xk, vec}, {"xv", xv, vec}, {"lr", lr, static_cast<size_t>(chains) * 4},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
+                 {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    Span outs[] = {{"out", out, vec}, {"W", W, mat}, {"b", b, bv}, {"W_grad", W_grad, mat}, {"b_grad", b_grad, bv}};
+    rc = check_aliasing(in, 7, outs, 5);
+    if (rc) return rc;
+
+    ttt::DecodeArgs a{};
+    a.xq = xq; a.xk = xk; a.xv = xv; a.lr = lr; a.token_eta = token_eta; a.ln_w = ln_w; a.ln_b = ln_b;
+    a.W = W; a.b = b; a.W_grad = W_grad; a.b_grad = b_grad; a.B = B; a.H = H; a.K = mini_batch;
+    a.p = static_cast<int>(seqlen_offset % mini_batch); a.eps = eps; a.out = out;
+    cudaError_t e = ttt::launch_decode(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_decode_step launch");
+    return ok();
+}
+
+}  // extern "C"

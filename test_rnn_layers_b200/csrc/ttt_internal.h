@@ -1,0 +1,96 @@
+// ttt_internal.h -- launch arguments and launcher prototypes shared between the C-ABI layer
+// (ttt_api.cu) and the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ttt {
+
+// Arguments of one TTT-Linear prefill launch (all pointers device pointers).
+struct LinearArgs {
+    const void* XQ;
+    const void* XK;
+    const void* XV;
+    const float* lr;
+    const float* token_eta;   // [K] or nullptr -> 1/(i+1)
+    const float* W0;
+    const float* b0;
+    long long w0_chain_stride;  // elements between consecutive chains' W0 (0: per head only)
+    const float* ln_w;
+    const float* ln_b;
+    int B, H;
+    long long L;
+    int K;
+    long long n_full, rem;
+    float eps;
+    void* out;
+    float* W_last;
+    float* b_last;
+    float* W_grad_tail;
+    float* b_grad_tail;
+    unsigned int* status;     // device status word
+    long long wait_limit;     // polls per bounded wait
+};
+
+struct MlpArgs {
+    const void* XQ;
+    const void* XK;
+    const void* XV;
+    const float* lr;
+    const float* token_eta;
+    const float* W1_0;
+    const float* b1_0;
+    const float* W2_0;
+    const float* b2_0;
+    long long w0_chain_stride;  // elements between chains' W1_0 / W2_0 (0: per head only)
+    const float* ln_w;
+    const float* ln_b;
+    int B, H;
+    long long L;
+    int K;
+    long long n_full, rem;
+    float eps;
+    void* out;
+    float* W1_last;
+    float* b1_last;
+    float* W2_last;
+    float* b2_last;
+    unsigned int* status;
+    long long wait_limit;
+};
+
+struct DecodeArgs {
+    const void* xq;
+    const void* xk;
+    const void* xv;
+    const float* lr;
+    const float* token_eta;
+    const float* ln_w;
+    const float* ln_b;
+    float* W;
+    float* b;
+    float* W_grad;
+    float* b_grad;
+    int B, H, K;
+    int p;          // position inside the mini-batch: seqlen_offset % K
+    float eps;
+    void* out;
+};
+
+// Tensor maps of the bf16 tensor-core prefill kernel: [B*H, L, 64] bf16 viewed 3-D,
+// box {64, K, 1}, 128-byte swizzle.
+struct LinearMaps {
+    CUtensorMap xq, xk, xv, out;
+};
+
+// launchers (return cudaSuccess or the launch error)
+cudaError_t launch_linear_simt(const LinearArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t s);
+cudaError_t launch_linear_state_copy(const LinearArgs& a, cudaStream_t s);
+cudaError_t launch_mlp_simt(const MlpArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_mlp_state_copy(const MlpArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t s);
+
+}  // namespace ttt

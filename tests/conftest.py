@@ -19,3 +19,12 @@ def pytest_configure(config):
 def orc():
     import oracle
     return oracle.default()
+
+
+@pytest.fixture(scope="session")
+def libttt():
+    """The CUDA library, built in-tree for sm_100a if it is missing (nvcc needs no GPU)."""
+    from test_rnn_layers_b200 import build
+    build.build()
+    import test_rnn_layers_b200 as ttt
+    return ttt

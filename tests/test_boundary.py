@@ -1,0 +1,128 @@
+"""The C-ABI boundary on the host: the library loads, exports what include/ttt.h declares, and
+rejects bad arguments with the documented codes before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ttt.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttt_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for f in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_partition",
+              "ttt_error_string", "ttt_last_error_message", "ttt_device_status", "ttt_set_wait_limit"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(libttt):
+    lib = ctypes.CDLL(libttt.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(libttt.EXPORTS) <= set(declared_functions())
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 16])
+@pytest.mark.parametrize("L", [0, 1, 15, 16, 17, 31, 8192, 8200])
+def test_partition_bit_exact_against_oracle(libttt, orc, L, K):
+    assert libttt.ttt_partition(L, K) == orc.partition(L, K)
+
+
+def test_partition_rejects_bad_arguments(libttt):
+    for L, K in ((-1, 16), (10, 0), (10, -3)):
+        with pytest.raises(libttt.TTTError) as e:
+            libttt.ttt_partition(L, K)
+        assert e.value.code == libttt.TTT_ERR_ARG
+
+
+def test_error_strings(libttt):
+    lib = libttt.lib()
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.ttt_error_string(code)
+    assert lib.ttt_error_string(-99) == b"unknown error code"
+
+
+# --- host-side argument validation of the compute entry points (nothing is launched) ----------
+A = 1 << 20  # fake, 16-byte aligned "device addresses": validation never dereferences them
+
+
+def _fwd(lib, **kw):
+    args = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W0=5 * A, b0=6 * A, stride=0, lnw=7 * A,
+                lnb=8 * A, B=2, H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, flags=0, out=9 * A,
+                Wl=10 * A, bl=11 * A, Wg=None, bg=None)
+    args.update(kw)
+    return lib.ttt_linear_forward(args["XQ"], args["XK"], args["XV"], args["lr"], args["te"], args["W0"],
+                                  args["b0"], args["stride"], args["lnw"], args["lnb"], args["B"], args["H"],
+                                  args["L"], args["d"], args["K"], args["eps"], args["dtype"], args["flags"],
+                                  args["out"], args["Wl"], args["bl"], args["Wg"], args["bg"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), -1), (dict(H=-1), -1), (dict(L=-5), -1), (dict(K=0), -1), (dict(K=17), -1),
+    (dict(eps=0.0), -1), (dict(eps=float("nan")), -1), (dict(dtype=7), -1), (dict(flags=8), -1),
+    (dict(d=32), -6), (dict(XQ=None), -1), (dict(W0=None), -1), (dict(out=None), -1),
+    (dict(stride=5), -1), (dict(XK=2 * A + 2), -2), (dict(out=9 * A + 8), -2), (dict(lr=4 * A + 1), -2),
+    (dict(out=A), -3), (dict(Wl=5 * A), -3), (dict(bl=10 * A + 64), -3), (dict(Wg=10 * A), -3),
+])
+def test_linear_forward_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _fwd(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
+def test_linear_forward_L0_allows_null_activations_but_checks_state(libttt):
+    lib = libttt.lib()
+    assert _fwd(lib, L=0, XQ=None, XK=None, XV=None, lr=None, out=None, W0=None) == -1
+
+
+def test_decode_rejects(libttt):
+    lib = libttt.lib()
+
+    def call(**kw):
+        a = dict(xq=A, xk=2 * A, xv=3 * A, lr=4 * A, te=None, lnw=5 * A, lnb=6 * A, W=7 * A, b=8 * A,
+                 Wg=9 * A, bg=10 * A, B=2, H=2, d=64, K=16, off=3, eps=1e-6, dtype=1, out=11 * A)
+        a.update(kw)
+        return lib.ttt_linear_decode_step(a["xq"], a["xk"], a["xv"], a["lr"], a["te"], a["lnw"], a["lnb"],
+                                          a["W"], a["b"], a["Wg"], a["bg"], a["B"], a["H"], a["d"], a["K"],
+                                          a["off"], a["eps"], a["dtype"], a["out"], None)
+    assert call(off=-1) == -1
+    assert call(W=None) == -1
+    assert call(d=48) == -6
+    assert call(W=7 * A + 4) == -2
+    assert call(out=A) == -3
+    assert call(Wg=7 * A) == -3
+
+
+def test_mlp_rejects(libttt):
+    lib = libttt.lib()
+
+    def call(**kw):
+        a = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W1=5 * A, b1=6 * A, W2=7 * A, b2=8 * A,
+                 stride=0, lnw=9 * A, lnb=10 * A, B=1, H=2, L=32, d=64, hid=256, K=16, eps=1e-6, dtype=1,
+                 flags=0, out=11 * A, W1l=12 * A, b1l=13 * A, W2l=14 * A, b2l=15 * A)
+        a.update(kw)
+        return lib.ttt_mlp_forward(a["XQ"], a["XK"], a["XV"], a["lr"], a["te"], a["W1"], a["b1"], a["W2"],
+                                   a["b2"], a["stride"], a["lnw"], a["lnb"], a["B"], a["H"], a["L"], a["d"],
+                                   a["hid"], a["K"], a["eps"], a["dtype"], a["flags"], a["out"], a["W1l"],
+                                   a["b1l"], a["W2l"], a["b2l"], None)
+    assert call(hid=128) == -6
+    assert call(W2=None) == -1
+    assert call(out=3 * A) == -3
+    assert call(b2l=15 * A + 4) == -2
+
+
+def test_binding_refuses_cpu_tensors(libttt):
+    import torch
+    x = torch.zeros(1, 1, 16, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        libttt.ttt_linear_forward(x, x, x, torch.zeros(1, 1, 16), torch.zeros(1, 64, 64), torch.zeros(1, 64),
+                                  torch.ones(1, 64), torch.zeros(1, 64))

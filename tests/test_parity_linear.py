@@ -1,0 +1,216 @@
+"""TTT-Linear prefill through the C-ABI on the GPU, element by element against the oracle.
+
+Tolerances (max relative L2 error per chain and per tensor, the norm ||gpu-ref|| / ||ref||):
+  * fp32 inputs (FFMA kernel, fp32 compute):          1e-5 on out, W_last, b_last.
+  * bf16 inputs, tensor-core kernel (bf16 operands,
+    fp32 accumulation, fp32 state):                   1e-2 on out, W_last, b_last, tail grads.
+  * bf16 inputs with TTT_FLAG_FP32_COMPUTE:          1e-5 on W_last/b_last; out is stored in
+    bf16, whose rounding alone is up to 2^-9 relative per element, so out takes 4e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import chain_slice, dev_act, dev_f32, rel_l2, sample_chains, to_np
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 1e-2
+TOL_BF16_OUT_FP32_COMPUTE = 4e-3
+
+
+def gpu_linear(ttt, x, w, K=None, flags=0, token_eta=None, per_chain_state=None):
+    XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
+    W0 = dev_f32(x["W0"] if per_chain_state is None else per_chain_state[0])
+    b0 = dev_f32(x["b0"] if per_chain_state is None else per_chain_state[1])
+    te = None if token_eta is None else dev_f32(token_eta)
+    res = ttt.ttt_linear_forward(XQ, XK, XV, dev_f32(x["lr"]), W0, b0, dev_f32(x["ln_w"]), dev_f32(x["ln_b"]),
+                                 mini_batch=K or w.K, eps=w.eps, token_eta=te, tail_grads=True, flags=flags)
+    torch.cuda.synchronize()
+    return res
+
+
+def oracle_linear(x, w, chains=None, K=None, token_eta=None, state_per_chain=False):
+    return oracle.default().linear_forward(x["XQ"], x["XK"], x["XV"], x["lr"], x["W0"], x["b0"], x["ln_w"],
+                                           x["ln_b"], K or w.K, w.eps, token_eta, chains=chains,
+                                           state_per_chain=state_per_chain)
+
+
+def compare(res, ref, tol, tol_out=None, what=""):
+    out, Wl, bl, Wg, bg = res
+    errs = {
+        "out": rel_l2(to_np(out).reshape(-1, *out.shape[2:]), ref["out"]),
+        "W_last": rel_l2(to_np(Wl).reshape(-1, 64, 64), ref["W_last"]),
+        "b_last": rel_l2(to_np(bl).reshape(-1, 64), ref["b_last"]),
+        "W_grad_tail": rel_l2(to_np(Wg).reshape(-1, 64, 64), ref["W_grad_tail"]),
+        "b_grad_tail": rel_l2(to_np(bg).reshape(-1, 64), ref["b_grad_tail"]),
+    }
+    for k, e in errs.items():
+        t = tol_out if (k == "out" and tol_out is not None) else tol
+        assert e <= t, f"{what} {k}: max rel L2 {e:.3e} > {t:.0e}  (all: {errs})"
+    return errs
+
+
+def compare_sampled(res, ref, chains, tol, tol_out=None, what=""):
+    H = res[0].shape[1]
+    picked = tuple(torch.from_numpy(chain_slice(t, chains, H)) for t in res)
+    sliced = tuple(p.reshape(len(chains), 1, *p.shape[1:]) for p in picked)
+    return compare(sliced, ref, tol, tol_out, what)
+
+
+def test_fp32_config_B1_H2_L64(libttt):
+    w = synth.workload(0)
+    x = synth.linear_inputs(w)
+    compare(gpu_linear(libttt, x, w), oracle_linear(x, w), TOL_F32, what="fp32 B1 H2 L64")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("K,L", [(16, 1), (16, 15), (16, 16), (16, 17), (16, 50), (1, 9), (2, 7), (3, 20),
+                                 (8, 40), (15, 47)])
+def test_ragged_and_mini_batch_sizes(libttt, dtype, K, L):
+    w = synth.workload(1, B=1, H=2, L=L, K=K, dtype=dtype, seed=0x1234 + 17 * K + L)
+    x = synth.linear_inputs(w)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    compare(gpu_linear(libttt, x, w), oracle_linear(x, w), tol, what=f"{dtype} K={K} L={L}")
+
+
+def test_bf16_several_tiles_and_tail(libttt):
+    # 2 x 12 chains, 19 full mini-batches and a tail of 7 (the 125M layer's heads)
+    w = synth.workload(1, B=2, H=12, L=16 * 19 + 7)
+    x = synth.linear_inputs(w)
+    compare(gpu_linear(libttt, x, w), oracle_linear(x, w), TOL_BF16, what="bf16 B2 H12 L311")
+
+
+def test_bf16_fp32_compute_flag(libttt):
+    w = synth.workload(1, B=1, H=3, L=16 * 40 + 3)
+    x = synth.linear_inputs(w)
+    res = gpu_linear(libttt, x, w, flags=libttt.TTT_FLAG_FP32_COMPUTE)
+    compare(res, oracle_linear(x, w), TOL_F32, TOL_BF16_OUT_FP32_COMPUTE, what="bf16 via fp32 compute")
+
+
+def test_token_eta_table(libttt):
+    w = synth.workload(1, B=1, H=2, L=16 * 6 + 5)
+    x = synth.linear_inputs(w)
+    te = np.linspace(1.0, 0.3, 16).astype(np.float32)
+    for dtype, tol in (("bf16", TOL_BF16), ("f32", TOL_F32)):
+        w.dtype = dtype
+        xx = synth.linear_inputs(w)
+        compare(gpu_linear(libttt, xx, w, token_eta=te), oracle_linear(xx, w, token_eta=te.astype(np.float64)),
+                tol, what=f"token_eta {dtype}")
+
+
+def test_L0_copies_state(libttt):
+    w = synth.workload(1, B=2, H=3, L=0)
+    x = synth.linear_inputs(w)
+    out, Wl, bl, Wg, bg = gpu_linear(libttt, x, w)
+    assert out.numel() == 0
+    assert np.array_equal(to_np(Wl), np.broadcast_to(x["W0"], (2, 3, 64, 64)))
+    assert not to_np(Wg).any() and not to_np(bg).any()
+
+
+def test_per_chain_state_in_place(libttt):
+    """A continuation: W0/b0 per chain, W_last written over W0 in place."""
+    w = synth.workload(1, B=2, H=2, L=16 * 5 + 2)
+    x = synth.linear_inputs(w)
+    rng = np.random.default_rng(3)
+    W0 = (np.broadcast_to(x["W0"], (2, 2, 64, 64)) + rng.normal(0, 0.01, (2, 2, 64, 64))).astype(np.float32)
+    b0 = rng.normal(0, 0.05, (2, 2, 64)).astype(np.float32)
+    Wd, bd = dev_f32(W0), dev_f32(b0)
+    out, Wl, bl = libttt.ttt_linear_forward(dev_act(x, "XQ"), dev_act(x, "XK"), dev_act(x, "XV"),
+                                            dev_f32(x["lr"]), Wd, bd, dev_f32(x["ln_w"]), dev_f32(x["ln_b"]),
+                                            eps=w.eps, W_last=Wd, b_last=bd)
+    torch.cuda.synchronize()
+    assert Wl.data_ptr() == Wd.data_ptr()
+    xo = dict(x, W0=W0, b0=b0)
+    ref = oracle_linear(xo, w, state_per_chain=True)
+    assert rel_l2(to_np(out).reshape(4, -1, 64), ref["out"]) <= TOL_BF16
+    assert rel_l2(to_np(Wd).reshape(4, 64, 64), ref["W_last"]) <= TOL_BF16
+    assert rel_l2(to_np(bd).reshape(4, 64), ref["b_last"]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_split_and_carry_is_bit_exact(libttt, dtype):
+    """Running [0, L1) then [L1, L) from (W_last, b_last) gives the same bits as one pass."""
+    w = synth.workload(1, B=2, H=2, L=16 * 23 + 5, dtype=dtype)
+    x = synth.linear_inputs(w)
+    L1 = 16 * 9
+    whole = gpu_linear(libttt, x, w)
+    first = synth.linear_inputs(w)
+    second = {}
+    for k in ("XQ", "XK", "XV", "XQ_bits", "XK_bits", "XV_bits"):
+        if k in first:
+            second[k] = np.ascontiguousarray(first[k][:, :, L1:])
+            first[k] = np.ascontiguousarray(first[k][:, :, :L1])
+    second["lr"] = np.ascontiguousarray(first["lr"][:, :, L1:])
+    first["lr"] = np.ascontiguousarray(first["lr"][:, :, :L1])
+    for k in ("ln_w", "ln_b"):
+        second[k] = first[k]
+    a = gpu_linear(libttt, first, w)
+    b = gpu_linear(libttt, second, w, per_chain_state=(to_np(a[1]).astype(np.float32), to_np(a[2]).astype(np.float32)))
+    assert torch.equal(torch.cat([a[0], b[0]], dim=2), whole[0])
+    assert torch.equal(b[1], whole[1]) and torch.equal(b[2], whole[2])
+    assert torch.equal(b[3], whole[3]) and torch.equal(b[4], whole[4])
+
+
+def test_deterministic(libttt):
+    w = synth.workload(1, B=2, H=4, L=16 * 12 + 3)
+    x = synth.linear_inputs(w)
+    r1, r2 = gpu_linear(libttt, x, w), gpu_linear(libttt, x, w)
+    for a, b in zip(r1, r2):
+        assert torch.equal(a, b)
+
+
+def test_125m_layer_full_size_sampled(libttt):
+    """The 125M layer at full size (B=16, H=12, L=2048): GPU on all chains, oracle on a sample."""
+    w = synth.workload(1)
+    x = synth.linear_inputs(w, values=False)
+    res = gpu_linear(libttt, x, w)
+    chains = sample_chains(w.chains, 4)
+    ref = oracle_linear(synth.linear_inputs(w, chains=chains), w, chains=chains)
+    compare_sampled(res, ref, chains, TOL_BF16, what="125m full")
+
+
+def test_1b_layer_full_size_with_tail_sampled(libttt):
+    """The 1B layer at full size with the remainder (B=8, H=32, L=8200): the bench's launch."""
+    w = synth.workload(2, L=8200)
+    x = synth.linear_inputs(w, values=False)
+    res = gpu_linear(libttt, x, w)
+    assert all(torch.isfinite(t.float()).all() for t in res)
+    chains = sample_chains(w.chains, 5)
+    ref = oracle_linear(synth.linear_inputs(w, chains=chains), w, chains=chains)
+    compare_sampled(res, ref, chains, TOL_BF16, what="1b full L=8200")
+
+
+def test_misaligned_device_pointer_is_rejected(libttt):
+    w = synth.workload(1, B=1, H=1, L=32)
+    x = synth.linear_inputs(w)
+    XQ = dev_act(x, "XQ")
+    flat = torch.empty(XQ.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    shifted = flat[1:].view_as(XQ)
+    shifted.copy_(XQ)
+    with pytest.raises(libttt.TTTError) as e:
+        libttt.ttt_linear_forward(shifted, dev_act(x, "XK"), dev_act(x, "XV"), dev_f32(x["lr"]), dev_f32(x["W0"]),
+                                  dev_f32(x["b0"]), dev_f32(x["ln_w"]), dev_f32(x["ln_b"]))
+    assert e.value.code == libttt.TTT_ERR_ALIGN
+
+
+def test_bounded_wait_timeout_reports_and_recovers(libttt):
+    """Every bounded wait gives up at once: the kernel flags the status word and returns; the
+    host reads TTT_ERR_TIMEOUT; the context stays usable and the next call is correct."""
+    w = synth.workload(1, B=1, H=2, L=16 * 8)
+    x = synth.linear_inputs(w)
+    libttt.ttt_device_status(clear=True)
+    libttt.ttt_set_wait_limit(-1)
+    try:
+        gpu_linear(libttt, x, w)
+        with pytest.raises(libttt.TTTError) as e:
+            libttt.ttt_device_status(clear=True)
+        assert e.value.code == libttt.TTT_ERR_TIMEOUT
+    finally:
+        libttt.ttt_set_wait_limit(0)
+    assert libttt.ttt_device_status(clear=True) == 0
+    compare(gpu_linear(libttt, x, w), oracle_linear(x, w), TOL_BF16, what="after timeout")
+    assert libttt.ttt_device_status() == 0
