@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
+from test_rnn_layers_b200.shard import aggregate_tokens_per_s  # noqa: E402
 
 D = 64
 HBM_FALLBACK_GBS = 6650.0
@@ -187,13 +188,8 @@ def barrier(world):
 
 
 def max_over_ranks(world, v):
-    if world == 1:
-        return v
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from test_rnn_layers_b200.shard import max_over_ranks as _max
+    return _max(v) if world > 1 else v
 
 
 def time_steps(step, K, W, world, sampler=None):
@@ -254,7 +250,7 @@ def bench_linear(args, world, rank, local, peaks):
         ms = time_steps(step, args.steps, args.warmup, world, clk)
     ttt.ttt_device_status()  # raises if a kernel gave up on a bounded wait
     tokens = B * L
-    value = world * tokens / (ms / 1e3)
+    value = aggregate_tokens_per_s(tokens, world, ms)
     hbm, tf_burst, _, which = peaks
     nbytes = linear_bytes(B, H, L)
     achieved = nbytes / (ms / 1e3) / 1e9
