@@ -377,7 +377,7 @@ def bench_decode(args, world, peaks):
                          "algorithmic_bytes": int(nbytes)}}
 
 
-def cpu_baseline(seconds_target=12.0, chains_max=64):
+def cpu_baseline(seconds_target=12.0, chains_max=256):
     """The oracle (fp64, single-threaded, as written) on a bounded sample of the 1B workload."""
     import oracle
     w = synth.workload(2, L=8200)

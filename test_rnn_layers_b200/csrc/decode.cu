@@ -6,162 +6,229 @@
 //   z = xk W + b, g = ln_fused_l2_bwd(z, xv - xk), W_grad += lr xk^T g, b_grad += lr g,
 //   out = xq + LN(xq (W - t W_grad) + b - t b_grad), and at p = K-1 the state commits.
 //
-// The step is a few matrix-vector products per chain: it is bound by the state traffic
-// (read W and W_grad, write W_grad, and W on a commit), so it runs on the FFMA pipes with
-// 16-byte coalesced loads.  xq W_bar is formed without materialising W_bar:
+// The step is a few matrix-vector products per chain, bound by the state traffic (read W and
+// W_grad, write W_grad, and W on a commit).  xq W_bar is formed without materialising W_bar:
 //   xq W_bar = xq W - t (xq W_grad_old + lr (xq . xk) g).
+// Persistent CTAs walk the chains with a stride; each CTA streams the next chain's W, W_grad,
+// b, b_grad and tokens into one of two shared-memory buffers with bulk async copies (an
+// mbarrier per buffer, bounded waits) while it computes the current chain from the other, so
+// HBM stays busy through the serial LayerNorm part.  The new W_grad (and W) leave by coalesced
+// 16-byte stores straight from registers.
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
 
 namespace ttt {
 namespace {
 
-constexpr int kThreads = 256;          // 16 column groups of 4 x 16 row groups of 4
+constexpr int kThreads = 256;           // 16 column groups of 4 x 16 row groups of 4
 constexpr int kRowGroups = kThreads / 16;
+constexpr int kBufs = 2;
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
-    __shared__ float sx[3][TTT_D];                      // xq, xk, xv
-    __shared__ float4 part[3][kRowGroups][TTT_D / 4];   // partial xk W, xq W, xq W_grad
-    __shared__ float sz[TTT_D], sqw[TTT_D], sqg[TTT_D], sg[TTT_D];
-    __shared__ float sqk;
+struct __align__(16) DecSmem {
+    float W[kBufs][TTT_D * TTT_D];
+    float G[kBufs][TTT_D * TTT_D];
+    float b[kBufs][TTT_D];
+    float gb[kBufs][TTT_D];
+    T x[kBufs][3][TTT_D];                 // xq, xk, xv
+    float lr[kBufs][4];
+    float4 part[3][kRowGroups][TTT_D / 4];  // partial xk W, xq W, xq W_grad
+    float sz[TTT_D], sqw[TTT_D], sqg[TTT_D], sg[TTT_D];
+    float sqk;
+    uint64_t full[kBufs];
+    int fail;
+};
 
+template <typename T>
+__device__ __forceinline__ void issue_chain(DecSmem<T>& s, const DecodeArgs& a, long long c, int bi) {
+    const uint32_t bytes = 2u * TTT_D * TTT_D * 4 + 2u * TTT_D * 4 + 3u * TTT_D * sizeof(T);
+    mbar_arrive_expect_tx(&s.full[bi], bytes);
+    bulk_load(s.W[bi], a.W + c * TTT_D * TTT_D, TTT_D * TTT_D * 4, &s.full[bi]);
+    bulk_load(s.G[bi], a.W_grad + c * TTT_D * TTT_D, TTT_D * TTT_D * 4, &s.full[bi]);
+    bulk_load(s.b[bi], a.b + c * TTT_D, TTT_D * 4, &s.full[bi]);
+    bulk_load(s.gb[bi], a.b_grad + c * TTT_D, TTT_D * 4, &s.full[bi]);
+    bulk_load(s.x[bi][0], static_cast<const T*>(a.xq) + c * TTT_D, TTT_D * sizeof(T), &s.full[bi]);
+    bulk_load(s.x[bi][1], static_cast<const T*>(a.xk) + c * TTT_D, TTT_D * sizeof(T), &s.full[bi]);
+    bulk_load(s.x[bi][2], static_cast<const T*>(a.xv) + c * TTT_D, TTT_D * sizeof(T), &s.full[bi]);
+    cp_async_4(&s.lr[bi][0], a.lr + c);
+    cp_async_mbar_arrive_noinc(&s.full[bi]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    DecSmem<T>& s = *reinterpret_cast<DecSmem<T>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long long chain = blockIdx.x;
-    const int h = static_cast<int>(chain % a.H);
     const int cg = tid & 15;        // columns 4cg .. 4cg+3
     const int rg = tid >> 4;        // rows rg, rg+16, rg+32, rg+48
-
-    float* W = a.W + chain * TTT_D * TTT_D;
-    float* Wg = a.W_grad + chain * TTT_D * TTT_D;
-    float4 w[4], G[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        int row = rg + 16 * k;
-        w[k] = *reinterpret_cast<const float4*>(W + row * TTT_D + 4 * cg);
-        G[k] = *reinterpret_cast<const float4*>(Wg + row * TTT_D + 4 * cg);
-    }
-    if (tid < 3 * TTT_D) {
-        int which = tid / TTT_D, c = tid % TTT_D;
-        const T* src = static_cast<const T*>(which == 0 ? a.xq : which == 1 ? a.xk : a.xv);
-        sx[which][c] = to_f32(src[chain * TTT_D + c]);
-    }
-    __syncthreads();
-
-    float4 pk = make_float4(0, 0, 0, 0), pq = pk, pg = pk;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        int row = rg + 16 * k;
-        float xk = sx[1][row], xq = sx[0][row];
-        pk.x = fmaf(xk, w[k].x, pk.x); pk.y = fmaf(xk, w[k].y, pk.y);
-        pk.z = fmaf(xk, w[k].z, pk.z); pk.w = fmaf(xk, w[k].w, pk.w);
-        pq.x = fmaf(xq, w[k].x, pq.x); pq.y = fmaf(xq, w[k].y, pq.y);
-        pq.z = fmaf(xq, w[k].z, pq.z); pq.w = fmaf(xq, w[k].w, pq.w);
-        pg.x = fmaf(xq, G[k].x, pg.x); pg.y = fmaf(xq, G[k].y, pg.y);
-        pg.z = fmaf(xq, G[k].z, pg.z); pg.w = fmaf(xq, G[k].w, pg.w);
-    }
-    part[0][rg][cg] = pk;
-    part[1][rg][cg] = pq;
-    part[2][rg][cg] = pg;
-    __syncthreads();
-
-    const float* bst = a.b + chain * TTT_D;
-    const float* bg = a.b_grad + chain * TTT_D;
-    const float lr = a.lr[chain];
-    const float t = a.token_eta ? a.token_eta[a.p] : 1.0f / (a.p + 1);
-    if (tid < 3 * TTT_D) {
-        int which = tid / TTT_D, c = tid % TTT_D;
-        const float* pp = reinterpret_cast<const float*>(&part[which][0][0]);
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < kRowGroups; ++r) acc += pp[r * TTT_D + c];
-        if (which == 0) sz[c] = acc + bst[c];
-        else if (which == 1) sqw[c] = acc;
-        else sqg[c] = acc;
-    }
-    if (warp == 7) {
-        float v = sx[0][lane] * sx[1][lane] + sx[0][lane + 32] * sx[1][lane + 32];
-        v = warp_sum(v);
-        if (lane == 0) sqk = v;
-    }
-    __syncthreads();
-
-    const float* lnw = a.ln_w + h * TTT_D;
-    const float* lnb = a.ln_b + h * TTT_D;
-    if (warp == 0) {
-        // g = ln_fused_l2_bwd(z, xv - xk)
-        float z0 = sz[lane], z1 = sz[lane + 32];
-        float mu = warp_sum(z0 + z1) * (1.0f / TTT_D);
-        float c0 = z0 - mu, c1 = z1 - mu;
-        float rstd = 1.0f / sqrtf(warp_sum(c0 * c0 + c1 * c1) * (1.0f / TTT_D) + a.eps);
-        float xh0 = c0 * rstd, xh1 = c1 * rstd;
-        float w0 = lnw[lane], w1 = lnw[lane + 32];
-        float q0 = w0 * (w0 * xh0 + lnb[lane] - (sx[2][lane] - sx[1][lane]));
-        float q1 = w1 * (w1 * xh1 + lnb[lane + 32] - (sx[2][lane + 32] - sx[1][lane + 32]));
-        float sq = warp_sum(q0 + q1), sqx = warp_sum(q0 * xh0 + q1 * xh1);
-        float g0 = (TTT_D * q0 - sq - xh0 * sqx) * rstd * (1.0f / TTT_D);
-        float g1 = (TTT_D * q1 - sq - xh1 * sqx) * rstd * (1.0f / TTT_D);
-        sg[lane] = g0;
-        sg[lane + 32] = g1;
-
-        // bias grads and the bar state
-        float gb0 = bg[lane] + lr * g0, gb1 = bg[lane + 32] + lr * g1;
-        float bb0 = bst[lane] - t * gb0, bb1 = bst[lane + 32] - t * gb1;
-        // xq W_bar + b_bar
-        float u0 = sqw[lane] - t * (sqg[lane] + lr * sqk * g0) + bb0;
-        float u1 = sqw[lane + 32] - t * (sqg[lane + 32] + lr * sqk * g1) + bb1;
-        float m2 = warp_sum(u0 + u1) * (1.0f / TTT_D);
-        float d0 = u0 - m2, d1 = u1 - m2;
-        float r2 = 1.0f / sqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.0f / TTT_D) + a.eps);
-        T* out = static_cast<T*>(a.out) + chain * TTT_D;
-        out[lane] = from_f32<T>(sx[0][lane] + w0 * d0 * r2 + lnb[lane]);
-        out[lane + 32] = from_f32<T>(sx[0][lane + 32] + w1 * d1 * r2 + lnb[lane + 32]);
-
-        const bool commit = (a.p == a.K - 1);
-        float* bsw = a.b + chain * TTT_D;
-        float* bgw = a.b_grad + chain * TTT_D;
-        if (commit) {
-            bsw[lane] = bb0;
-            bsw[lane + 32] = bb1;
-            bgw[lane] = 0.f;
-            bgw[lane + 32] = 0.f;
-        } else {
-            bgw[lane] = gb0;
-            bgw[lane + 32] = gb1;
-        }
-    }
-    __syncthreads();
-
-    // W_grad += lr xk^T g ; on commit W -= t W_grad and W_grad = 0
+    const long long chains = static_cast<long long>(a.B) * a.H;
+    const long long stride = gridDim.x;
     const bool commit = (a.p == a.K - 1);
-    float4 gv = *reinterpret_cast<const float4*>(&sg[4 * cg]);
+
+    if (tid == 0) {
+        for (int i = 0; i < kBufs; ++i) mbar_init(&s.full[i], 2);  // expect-tx arrival + lr cp.async
+        fence_mbarrier_init();
+        s.fail = 0;
+    }
+    __syncthreads();
+    int issued = 0;  // loads issued by thread 0 (the i-th goes to buffer i % 2, phase (i / 2) & 1)
+    if (tid == 0)
+        for (int i = 0; i < kBufs; ++i)
+            if (blockIdx.x + i * stride < chains) {
+                issue_chain(s, a, blockIdx.x + i * stride, i);
+                ++issued;
+            }
+
+    int bi = 0, it = 0;
+    uint32_t par = 0;
+    for (long long c = blockIdx.x; c < chains; c += stride, ++it, bi ^= 1, par ^= (bi == 0)) {
+        const int h = static_cast<int>(c % a.H);
+        if (!mbar_wait_bounded(&s.full[bi], par, a.wait_limit, a.status)) s.fail = 1;
+
+        // state of this chain into registers; partial matrix-vector products
+        float4 w[4], G[4];
+        float4 pk = make_float4(0, 0, 0, 0), pq = pk, pg = pk;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        int row = rg + 16 * k;
-        float s = lr * sx[1][row];
-        float4 n;
-        n.x = fmaf(s, gv.x, G[k].x); n.y = fmaf(s, gv.y, G[k].y);
-        n.z = fmaf(s, gv.z, G[k].z); n.w = fmaf(s, gv.w, G[k].w);
-        if (commit) {
-            float4 nw;
-            nw.x = w[k].x - t * n.x; nw.y = w[k].y - t * n.y;
-            nw.z = w[k].z - t * n.z; nw.w = w[k].w - t * n.w;
-            *reinterpret_cast<float4*>(W + row * TTT_D + 4 * cg) = nw;
-            *reinterpret_cast<float4*>(Wg + row * TTT_D + 4 * cg) = make_float4(0, 0, 0, 0);
-        } else {
-            *reinterpret_cast<float4*>(Wg + row * TTT_D + 4 * cg) = n;
+        for (int k = 0; k < 4; ++k) {
+            const int row = rg + 16 * k;
+            w[k] = *reinterpret_cast<const float4*>(&s.W[bi][row * TTT_D + 4 * cg]);
+            G[k] = *reinterpret_cast<const float4*>(&s.G[bi][row * TTT_D + 4 * cg]);
+            const float xk = to_f32(s.x[bi][1][row]), xq = to_f32(s.x[bi][0][row]);
+            pk.x = fmaf(xk, w[k].x, pk.x); pk.y = fmaf(xk, w[k].y, pk.y);
+            pk.z = fmaf(xk, w[k].z, pk.z); pk.w = fmaf(xk, w[k].w, pk.w);
+            pq.x = fmaf(xq, w[k].x, pq.x); pq.y = fmaf(xq, w[k].y, pq.y);
+            pq.z = fmaf(xq, w[k].z, pq.z); pq.w = fmaf(xq, w[k].w, pq.w);
+            pg.x = fmaf(xq, G[k].x, pg.x); pg.y = fmaf(xq, G[k].y, pg.y);
+            pg.z = fmaf(xq, G[k].z, pg.z); pg.w = fmaf(xq, G[k].w, pg.w);
+        }
+        s.part[0][rg][cg] = pk;
+        s.part[1][rg][cg] = pq;
+        s.part[2][rg][cg] = pg;
+        __syncthreads();
+        if (s.fail) break;
+
+        const float lr = s.lr[bi][0];
+        const float t = a.token_eta ? a.token_eta[a.p] : 1.0f / (a.p + 1);
+        if (tid < 3 * TTT_D) {
+            const int which = tid / TTT_D, col = tid % TTT_D;
+            const float* pp = reinterpret_cast<const float*>(&s.part[which][0][0]);
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < kRowGroups; ++r) acc += pp[r * TTT_D + col];
+            if (which == 0) s.sz[col] = acc + s.b[bi][col];
+            else if (which == 1) s.sqw[col] = acc;
+            else s.sqg[col] = acc;
+        }
+        if (warp == 7) {
+            const float v = to_f32(s.x[bi][0][lane]) * to_f32(s.x[bi][1][lane]) +
+                            to_f32(s.x[bi][0][lane + 32]) * to_f32(s.x[bi][1][lane + 32]);
+            const float r = warp_sum(v);
+            if (lane == 0) s.sqk = r;
+        }
+        __syncthreads();
+
+        const float* lnw = a.ln_w + h * TTT_D;
+        const float* lnb = a.ln_b + h * TTT_D;
+        if (warp == 0) {
+            // g = ln_fused_l2_bwd(z, xv - xk)
+            const float z0 = s.sz[lane], z1 = s.sz[lane + 32];
+            const float mu = warp_sum(z0 + z1) * (1.0f / TTT_D);
+            const float c0 = z0 - mu, c1 = z1 - mu;
+            const float rstd = rsqrtf(warp_sum(c0 * c0 + c1 * c1) * (1.0f / TTT_D) + a.eps);
+            const float xh0 = c0 * rstd, xh1 = c1 * rstd;
+            const float w0 = lnw[lane], w1 = lnw[lane + 32];
+            const float xk0 = to_f32(s.x[bi][1][lane]), xk1 = to_f32(s.x[bi][1][lane + 32]);
+            const float xq0 = to_f32(s.x[bi][0][lane]), xq1 = to_f32(s.x[bi][0][lane + 32]);
+            const float q0 = w0 * (w0 * xh0 + lnb[lane] - (to_f32(s.x[bi][2][lane]) - xk0));
+            const float q1 = w1 * (w1 * xh1 + lnb[lane + 32] - (to_f32(s.x[bi][2][lane + 32]) - xk1));
+            const float sq = warp_sum(q0 + q1), sqx = warp_sum(q0 * xh0 + q1 * xh1);
+            const float g0 = (TTT_D * q0 - sq - xh0 * sqx) * rstd * (1.0f / TTT_D);
+            const float g1 = (TTT_D * q1 - sq - xh1 * sqx) * rstd * (1.0f / TTT_D);
+            s.sg[lane] = g0;
+            s.sg[lane + 32] = g1;
+
+            // bias grads and the bar state
+            const float gb0 = s.gb[bi][lane] + lr * g0, gb1 = s.gb[bi][lane + 32] + lr * g1;
+            const float bb0 = s.b[bi][lane] - t * gb0, bb1 = s.b[bi][lane + 32] - t * gb1;
+            // xq W_bar + b_bar
+            const float u0 = s.sqw[lane] - t * (s.sqg[lane] + lr * s.sqk * g0) + bb0;
+            const float u1 = s.sqw[lane + 32] - t * (s.sqg[lane + 32] + lr * s.sqk * g1) + bb1;
+            const float m2 = warp_sum(u0 + u1) * (1.0f / TTT_D);
+            const float d0 = u0 - m2, d1 = u1 - m2;
+            const float r2 = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.0f / TTT_D) + a.eps);
+            T* out = static_cast<T*>(a.out) + c * TTT_D;
+            out[lane] = from_f32<T>(xq0 + w0 * d0 * r2 + lnb[lane]);
+            out[lane + 32] = from_f32<T>(xq1 + w1 * d1 * r2 + lnb[lane + 32]);
+
+            float* bsw = a.b + c * TTT_D;
+            float* bgw = a.b_grad + c * TTT_D;
+            if (commit) {
+                bsw[lane] = bb0;
+                bsw[lane + 32] = bb1;
+                bgw[lane] = 0.f;
+                bgw[lane + 32] = 0.f;
+            } else {
+                bgw[lane] = gb0;
+                bgw[lane + 32] = gb1;
+            }
+        }
+        __syncthreads();
+
+        // W_grad += lr xk^T g ; on commit W -= t W_grad and W_grad = 0
+        float* Wc = a.W + c * TTT_D * TTT_D;
+        float* Gc = a.W_grad + c * TTT_D * TTT_D;
+        const float4 gv = *reinterpret_cast<const float4*>(&s.sg[4 * cg]);
+        float xkr[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) xkr[k] = lr * to_f32(s.x[bi][1][rg + 16 * k]);
+        __syncthreads();  // buffer bi fully read: refill it with the chain after next
+        if (tid == 0 && c + kBufs * stride < chains) {
+            issue_chain(s, a, c + kBufs * stride, bi);
+            ++issued;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int row = rg + 16 * k;
+            float4 n;
+            n.x = fmaf(xkr[k], gv.x, G[k].x); n.y = fmaf(xkr[k], gv.y, G[k].y);
+            n.z = fmaf(xkr[k], gv.z, G[k].z); n.w = fmaf(xkr[k], gv.w, G[k].w);
+            if (commit) {
+                float4 nw;
+                nw.x = w[k].x - t * n.x; nw.y = w[k].y - t * n.y;
+                nw.z = w[k].z - t * n.z; nw.w = w[k].w - t * n.w;
+                *reinterpret_cast<float4*>(Wc + row * TTT_D + 4 * cg) = nw;
+                *reinterpret_cast<float4*>(Gc + row * TTT_D + 4 * cg) = make_float4(0, 0, 0, 0);
+            } else {
+                *reinterpret_cast<float4*>(Gc + row * TTT_D + 4 * cg) = n;
+            }
         }
     }
+    // after a failed wait, leave only once this CTA's issued copies have landed (bounded)
+    if (s.fail && tid == 0)
+        for (int j = it; j < issued; ++j)
+            mbar_wait_bounded(&s.full[j % kBufs], static_cast<uint32_t>((j / kBufs) & 1), 1ll << 24, nullptr);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st) {
-    dim3 grid(static_cast<unsigned>(a.B * a.H));
-    if (dtype == 0)
-        decode_kernel<float><<<grid, kThreads, 0, st>>>(a);
-    else
-        decode_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(a);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long chains = static_cast<long long>(a.B) * a.H;
+    const unsigned grid = static_cast<unsigned>(chains < 2ll * sms ? chains : 2ll * sms);
+    cudaError_t e;
+    if (dtype == 0) {
+        const size_t smem = sizeof(DecSmem<float>);
+        e = cudaFuncSetAttribute(decode_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        decode_kernel<float><<<grid, kThreads, smem, st>>>(a);
+    } else {
+        const size_t smem = sizeof(DecSmem<__nv_bfloat16>);
+        e = cudaFuncSetAttribute(decode_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        decode_kernel<__nv_bfloat16><<<grid, kThreads, smem, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -7,32 +7,38 @@
 //   out = XQ + LN(Zbar);  full mini-batch: W -= (eta[K-1,:] * XK)^T g,  b -= sum_j eta[K-1,j] g_j
 //
 // Design (one persistent CTA of 4 warps per (batch, head) chain, the whole sequence on chip):
-//  * The fp32 master state W^T (64x64) lives in mma.sync accumulator registers: warp w owns
-//    output features 16w..16w+15, i.e. rows 16w.. of W^T, as eight m16n8 fragments.  The
-//    accumulator layout of W^T is exactly the B-operand layout of W for Z = XK W, so each
-//    mini-batch only rounds the accumulators to bf16 pairs; the rank-K update of W is an MMA
-//    that accumulates straight into the same registers.  W never leaves the SM.
-//  * The dense contractions are m16n8k16 bf16 MMAs: Z and XQ W (16x64x64), XQ XK^T (16x16x64),
-//    M g (16x16x64) and the update (64x16x64).  g enters the B and A operands through
-//    movmatrix (register transposes), with no shared-memory round trip.
-//  * LayerNorm statistics: each thread holds 2 rows x 4 features, quads reduce with shuffles,
-//    the 4 warps merge (sum, centred sum of squares) pairs through shared memory (Chan's
-//    formula), so the loss gradient costs two 128-thread barriers per mini-batch.  The output
-//    LayerNorm of mini-batch m is finished during mini-batch m+1 and shares those barriers.
-//  * A TMA ring of kStages mini-batches (XQ, XK, XV tiles with 128-byte swizzle, box {64, K})
-//    plus cp.async for lr, tracked by one mbarrier per stage, prefetches ahead of the scan; the
-//    output tile is staged in shared memory and written back by a TMA store.  All mbarrier
-//    waits are bounded; on expiry the kernel raises the status word, drains its in-flight
-//    copies (again bounded) and returns.
+//  * State in registers.  The fp32 master W^T (64x64) lives in mma.sync accumulator fragments:
+//    warp w owns output features 16w..16w+15 (rows 16w.. of W^T, eight m16n8 tiles).  The
+//    accumulator layout of W^T is exactly the B-operand layout of W for Z = XK W, so a
+//    mini-batch only rounds the accumulators to bf16 pairs, and the rank-K update of W is an MMA
+//    accumulating straight into the same registers.  The bias b is one more fp32 accumulator
+//    column, updated by the same MMA against a column of ones and spread to the lanes that add
+//    it to Z and Zbar (in fp32) by four shuffles.  Nothing of the state round-trips memory.
+//  * Tensor cores for the dense contractions: Z and XQ W (16x64x64), XQ XK^T (16x16x64),
+//    M g (16x16x64, the two tril terms of the dual form folded into M = eta * tril(XQ XK^T + 1))
+//    and the update (64x16x64): m16n8k16 bf16 MMAs with fp32 accumulation.  g reaches the B
+//    operand of M g and the A operand of the update through movmatrix register transposes.
+//  * LayerNorm fused in registers: a thread holds 2 rows x 4 features; quads reduce by shuffles;
+//    the 4 warps' (sum, centred sum of squares) per row merge through shared memory with Chan's
+//    formula.  The loss gradient costs two 128-thread named barriers per mini-batch; the output
+//    LayerNorm of mini-batch m is finished during m+1 on the same barriers and stored straight
+//    from registers.  Shared-memory traffic is kept to the TMA tiles, the ldmatrix operand loads
+//    and a few hundred bytes of row statistics per mini-batch.
+//  * A fifth, producer warp streams the inputs: a TMA ring of kStages mini-batches (XQ, XK, XV
+//    tiles, 128-byte swizzle, box {64, K}) plus cp.async for lr, with a "full" mbarrier per stage
+//    (data landed) and an "empty" one (the four compute warps are done with it).  No multicast.
+//    Every mbarrier wait is bounded; on expiry the kernel raises the status word, drains its
+//    in-flight copies (bounded) and returns.
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
 
 namespace ttt {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 4;
+constexpr int kWarps = 4;                  // compute warps
+constexpr int kThreads = 32 * kWarps;      // compute threads (the named barriers' count)
+constexpr int kBlock = kThreads + 32;      // + the producer warp
+constexpr int kStages = 6;
 constexpr int kTileBytes = TTT_KMAX * TTT_D * 2;  // 16 rows x 128 bytes
 constexpr long long kDrainPolls = 1ll << 24;
 
@@ -40,16 +46,24 @@ struct __align__(1024) TcSmem {
     uint8_t xq[kStages][kTileBytes];
     uint8_t xk[kStages][kTileBytes];
     uint8_t xv[kStages][kTileBytes];
-    uint8_t outb[2][kTileBytes];
-    float gtail[TTT_KMAX][TTT_D];      // tail grads (fp32), only on the remainder mini-batch
+    float gtail[TTT_KMAX][TTT_D];    // g in fp32 on the remainder mini-batch (tail grads)
     float lr[kStages][TTT_KMAX];
     float te[TTT_KMAX];
-    float2 red1[kWarps][TTT_KMAX];     // Z rows: (sum, centred sum of squares) per warp
-    float2 red2[kWarps][TTT_KMAX];     // (sum q, sum q * xhat) per warp
-    float2 red3[kWarps][TTT_KMAX];     // Zbar rows of the previous mini-batch
-    uint64_t full[kStages];
-    int fail;
+    // per row, the four warps' partial statistics: [row][warp pair] = (w even: a, b, w odd: a, b)
+    float4 red1[TTT_KMAX][2];        // Z rows: (sum, centred sum of squares) over 16 features
+    float4 red2[TTT_KMAX][2];        // (sum q, sum q * xhat)
+    float4 red3[2][TTT_KMAX][2];     // Zbar rows, by mini-batch parity
+    uint64_t full[kStages];          // stage loaded (1 expect-tx arrival + 16 lr arrivals)
+    uint64_t empty[kStages];         // stage consumed (one arrival per compute warp)
+    int fail;                        // a compute warp gave up on a wait
+    int fail_m;                      // the mini-batch it gave up on
 };
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 bc2(float a) { return make_float2(a, a); }
 
 // Sum over the 4 lanes of a quad (lanes sharing rows g, g+8).
 __device__ __forceinline__ float quad_sum(float v) {
@@ -59,64 +73,104 @@ __device__ __forceinline__ float quad_sum(float v) {
 }
 
 // Per-warp row partials of a [16 x 16-feature] slice held as v[nt][0..3] (rows g and g+8):
-// returns (sum, centred sum of squares) over this warp's 16 features for each of the 2 rows.
+// (sum, centred sum of squares) over this warp's 16 features for each of the 2 rows.
 __device__ __forceinline__ void warp_row_partials(const float (&v)[2][4], float2& r0, float2& r1) {
-    float s0 = quad_sum(v[0][0] + v[0][1] + v[1][0] + v[1][1]);
-    float s1 = quad_sum(v[0][2] + v[0][3] + v[1][2] + v[1][3]);
-    float m0 = s0 * (1.0f / 16), m1 = s1 * (1.0f / 16);
-    float c0 = 0.f, c1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        float a = v[nt][0] - m0, b = v[nt][1] - m0, c = v[nt][2] - m1, d = v[nt][3] - m1;
-        c0 += a * a + b * b;
-        c1 += c * c + d * d;
-    }
-    r0 = make_float2(s0, quad_sum(c0));
-    r1 = make_float2(s1, quad_sum(c1));
+    const float2 a0 = make_float2(v[0][0], v[0][1]), a1 = make_float2(v[1][0], v[1][1]);  // row g
+    const float2 b0 = make_float2(v[0][2], v[0][3]), b1 = make_float2(v[1][2], v[1][3]);  // row g+8
+    const float2 sa = __fadd2_rn(a0, a1), sb = __fadd2_rn(b0, b1);
+    const float s0 = quad_sum(sa.x + sa.y), s1 = quad_sum(sb.x + sb.y);
+    const float2 m0 = make_float2(-s0 * (1.0f / 16), -s0 * (1.0f / 16));
+    const float2 m1 = make_float2(-s1 * (1.0f / 16), -s1 * (1.0f / 16));
+    const float2 da0 = __fadd2_rn(a0, m0), da1 = __fadd2_rn(a1, m0);
+    const float2 db0 = __fadd2_rn(b0, m1), db1 = __fadd2_rn(b1, m1);
+    const float2 ca = __ffma2_rn(da1, da1, __fmul2_rn(da0, da0));
+    const float2 cb = __ffma2_rn(db1, db1, __fmul2_rn(db0, db0));
+    r0 = make_float2(s0, quad_sum(ca.x + ca.y));
+    r1 = make_float2(s1, quad_sum(cb.x + cb.y));
 }
 
-// Merge the 4 warps' partials of one row into mean and 1/sqrt(var + eps).
-__device__ __forceinline__ void merge_row(const float2 (*red)[TTT_KMAX], int row, float eps,
-                                          float& mu, float& rstd) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) s += red[w][row].x;
-    mu = s * (1.0f / TTT_D);
-    float m2 = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        float dm = red[w][row].x * (1.0f / 16) - mu;
-        m2 += red[w][row].y + 16.0f * dm * dm;
-    }
+__device__ __forceinline__ void put_partial(float4 (*red)[2], int row, int w, float2 v) {
+    reinterpret_cast<float2*>(&red[row][w >> 1])[w & 1] = v;
+}
+
+// Merge the 4 warps' (sum, centred sum of squares) of one row: mean and 1/sqrt(var + eps).
+__device__ __forceinline__ void merge_row(const float4 (*red)[2], int row, float eps, float& mu, float& rstd) {
+    const float4 a = red[row][0], b = red[row][1];
+    mu = ((a.x + a.z) + (b.x + b.z)) * (1.0f / TTT_D);
+    const float d0 = a.x * (1.0f / 16) - mu, d1 = a.z * (1.0f / 16) - mu;
+    const float d2 = b.x * (1.0f / 16) - mu, d3 = b.z * (1.0f / 16) - mu;
+    const float m2 = (a.y + a.w) + (b.y + b.w) + 16.0f * (d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3);
     rstd = rsqrtf(m2 * (1.0f / TTT_D) + eps);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+// out rows of mini-batch mm = XQ + LN(Zbar), written straight from the accumulator layout:
+// rows g and g+8, features 16w + 8nt + 2t + {0,1} (rows past the mini-batch's end are skipped).
+__device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearArgs& a, int chain, int mm, int K,
+                                          int n_full, int g, int t, int w, const float (&zb)[2][4],
+                                          const uint32_t (&xq)[4], const float (&lw)[2][2], const float (&lb)[2][2]) {
+    float mu0, rs0, mu1, rs1;
+    merge_row(red, g, a.eps, mu0, rs0);
+    merge_row(red, g + 8, a.eps, mu1, rs1);
+    const int Km = mm < n_full ? K : static_cast<int>(a.rem);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
+                         (static_cast<long long>(chain) * a.L + static_cast<long long>(mm) * K) * TTT_D;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        // xq[2nt] = row g, xq[2nt+1] = row g+8 (A fragment order a0..a3)
+        const float2 l2 = make_float2(lw[nt][0], lw[nt][1]), b2 = make_float2(lb[nt][0], lb[nt][1]);
+        const int f = 16 * w + 8 * nt + 2 * t;
+        if (g < Km) {
+            const float2 y = fma2(l2, fma2(make_float2(zb[nt][0], zb[nt][1]), bc2(rs0), bc2(-mu0 * rs0)), b2);
+            const float2 o = add2(unpack_bf16x2(xq[2 * nt]), y);
+            *reinterpret_cast<uint32_t*>(out + g * TTT_D + f) = pack_bf16x2(o.x, o.y);
+        }
+        if (g + 8 < Km) {
+            const float2 y = fma2(l2, fma2(make_float2(zb[nt][2], zb[nt][3]), bc2(rs1), bc2(-mu1 * rs1)), b2);
+            const float2 o = add2(unpack_bf16x2(xq[2 * nt + 1]), y);
+            *reinterpret_cast<uint32_t*>(out + (g + 8) * TTT_D + f) = pack_bf16x2(o.x, o.y);
+        }
+    }
+}
+
+// Select the fragment registers of k-slice `w` (warp-uniform) without local memory.
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4][4], int w, int i) {
+    const uint32_t lo = (w & 1) ? v[1][i] : v[0][i];
+    const uint32_t hi = (w & 1) ? v[3][i] : v[2][i];
+    return (w & 2) ? hi : lo;
+}
+
+__global__ void __launch_bounds__(kBlock, 2)
 linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
-    extern __shared__ uint8_t smem_raw[];
-    TcSmem& s = *reinterpret_cast<TcSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // align by a byte offset from the shared array itself (an integer round trip of the pointer
+    // would hide the shared address space and turn every access into a generic one)
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    TcSmem& s = *reinterpret_cast<TcSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int chain = blockIdx.x;
     const int h = chain % a.H;
     const int K = a.K;
-    const long long n_mb = a.n_full + (a.rem > 0 ? 1 : 0);
+    const int n_full = static_cast<int>(a.n_full);
+    const int n_mb = n_full + (a.rem > 0 ? 1 : 0);
     const float* lr_g = a.lr + static_cast<long long>(chain) * a.L;
     const uint32_t tile_tx = static_cast<uint32_t>(K) * TTT_D * 2;
 
     // ---- set-up ------------------------------------------------------------------------------
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(&s.full[i], 1 + TTT_KMAX);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&s.full[i], 1 + TTT_KMAX);
+            mbar_init(&s.empty[i], kWarps);
+        }
         fence_mbarrier_init();
         tma_prefetch_desc(&maps.xq);
         tma_prefetch_desc(&maps.xk);
         tma_prefetch_desc(&maps.xv);
-        tma_prefetch_desc(&maps.out);
         s.fail = 0;
+        s.fail_m = 0;
     }
     // rows K..15 of every tile stay zero for the whole run (TMA writes rows < K only)
-    for (int i = tid; i < kStages * kTileBytes / 16; i += kThreads) {
+    for (int i = tid; i < kStages * kTileBytes / 16; i += kBlock) {
         reinterpret_cast<uint4*>(&s.xq[0][0])[i] = make_uint4(0, 0, 0, 0);
         reinterpret_cast<uint4*>(&s.xk[0][0])[i] = make_uint4(0, 0, 0, 0);
         reinterpret_cast<uint4*>(&s.xv[0][0])[i] = make_uint4(0, 0, 0, 0);
@@ -125,11 +179,10 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     fence_proxy_async_smem();
     __syncthreads();
 
-    // producer: warp 0 loads mini-batch mm into stage mm % kStages
-    auto issue = [&](long long mm) {
-        const int st = static_cast<int>(mm % kStages);
-        const int Kmm = mm < a.n_full ? K : static_cast<int>(a.rem);
-        const int row0 = static_cast<int>(mm * K);
+    // producer: warp 0 loads mini-batch mm into stage st
+    auto issue = [&](int mm, int st) {
+        const int Kmm = mm < n_full ? K : static_cast<int>(a.rem);
+        const int row0 = mm * K;
         if (lane == 0) {
             mbar_arrive_expect_tx(&s.full[st], 3 * tile_tx);
             tma_load_3d(&s.xq[st][0], &maps.xq, 0, row0, chain, &s.full[st]);
@@ -146,217 +199,216 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             }
         }
     };
-    long long issued = 0;
-    if (w == 0)
-        for (; issued < kStages - 1 && issued < n_mb; ++issued) issue(issued);
+    if (w == kWarps) {
+        // ---- producer warp: fill stage st with mini-batch mm once the compute warps freed it --
+        int mm = 0, pst = 0;
+        for (; mm < n_mb; ++mm, pst = (pst + 1 == kStages ? 0 : pst + 1)) {
+            // from its second use on, stage pst waits for the compute warps to release mini-batch
+            // mm - kStages: the ((mm / kStages) - 1)-th completion of empty[pst]
+            const uint32_t epar = static_cast<uint32_t>((mm / kStages - 1) & 1);
+            if (mm >= kStages && !mbar_wait_bounded_sleep(&s.empty[pst], epar, a.wait_limit, 256, a.status)) break;
+            if (*reinterpret_cast<volatile int*>(&s.fail)) break;
+            issue(mm, pst);
+        }
+        // on a failure, wait (bounded) until the loads issued but not consumed have landed
+        if (*reinterpret_cast<volatile int*>(&s.fail) || mm < n_mb) {
+            if (lane == 0) {
+                const int first = *reinterpret_cast<volatile int*>(&s.fail_m);
+                for (int k = first; k < mm; ++k)
+                    mbar_wait_bounded(&s.full[k % kStages], static_cast<uint32_t>((k / kStages) & 1),
+                                      kDrainPolls, nullptr);
+            }
+        }
+        return;
+    }
 
-    // ---- state: W^T accumulators, b, LayerNorm affine --------------------------------------
+    // ---- state --------------------------------------------------------------------------------
     const long long w0off = a.w0_chain_stride ? static_cast<long long>(chain) * a.w0_chain_stride
                                               : static_cast<long long>(h) * TTT_D * TTT_D;
     const long long b0off = a.w0_chain_stride ? static_cast<long long>(chain) * TTT_D
                                               : static_cast<long long>(h) * TTT_D;
-    float Wt[8][4];  // Wt[jt][e]: W^T[16w + g + 8(e>>1)][8jt + 2t + (e&1)]
+    float Wt[8][4];  // Wt[jt][e] = W^T[16w + g + 8(e>>1)][8jt + 2t + (e&1)]
 #pragma unroll
     for (int jt = 0; jt < 8; ++jt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
+            const int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
             Wt[jt][e] = a.W0[w0off + j * TTT_D + f];
         }
+    // bias accumulator column: Bt[0] = b[16w + g], Bt[2] = b[16w + g + 8] on lanes t == 0, zero elsewhere
+    float Bt[4] = {0.f, 0.f, 0.f, 0.f};
+    if (t == 0) {
+        Bt[0] = a.b0[b0off + 16 * w + g];
+        Bt[2] = a.b0[b0off + 16 * w + g + 8];
+    }
+    const uint32_t ones_b = (g == 0) ? pack_bf16x2(1.f, 1.f) : 0u;  // B operand: ones in column 0
     float bc[2][2], lw[2][2], lb[2][2];  // per n-tile nt, feature 16w + 8nt + 2t + e
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            int f = 16 * w + 8 * nt + 2 * t + e;
+            const int f = 16 * w + 8 * nt + 2 * t + e;
             bc[nt][e] = a.b0[b0off + f];
             lw[nt][e] = a.ln_w[h * TTT_D + f];
             lb[nt][e] = a.ln_b[h * TTT_D + f];
         }
 
+    float2 lw2[2], lb2[2];  // the same LayerNorm affine, as pairs per n-tile
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        lw2[nt] = f2(lw[nt][0], lw[nt][1]);
+        lb2[nt] = f2(lb[nt][0], lb[nt][1]);
+    }
+    const float eps = a.eps;
+    const long long wait_limit = a.wait_limit;
+    unsigned int* const status = a.status;
+    const float te_g = s.te[g], te_g8 = s.te[g + 8], te_last = s.te[K - 1];
     const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row supplied by this lane
     const int lchunk = lane >> 4;
-    float zbar_prev[2][4];
-    uint32_t xq_prev[2][2];  // bf16 pairs of XQ at this thread's output positions
+    float zbar_prev[2][4] = {};
+    uint32_t xq_prev[4] = {};  // XQ at this thread's output positions (A fragment of k-slice w)
     bool failed = false;
-    long long m = 0;
+    int m = 0, st = 0;
+    uint32_t par = 0;
 
-    for (; m < n_mb; ++m) {
-        const int st = static_cast<int>(m % kStages);
-        const uint32_t par = static_cast<uint32_t>((m / kStages) & 1);
-        const bool full_mb = m < a.n_full;
+    for (; m < n_mb; ++m, st = (st + 1 == kStages ? 0 : st + 1), par ^= (st == 0)) {
+        const bool full_mb = m < n_full;
         const int Km = full_mb ? K : static_cast<int>(a.rem);
-        if (!mbar_wait_bounded(&s.full[st], par, a.wait_limit, a.status)) s.fail = 1;
-
+        if (!mbar_wait_bounded(&s.full[st], par, wait_limit, status)) {
+            s.fail_m = m;
+            s.fail = 1;
+        }
         const uint32_t xq_s = smem_u32(&s.xq[st][0]);
         const uint32_t xk_s = smem_u32(&s.xk[st][0]);
-        const uint32_t xv_s = smem_u32(&s.xv[st][0]);
 
-        // ---- Z = XK W + b, XQW = XQ W + b, Attn = XQ XK^T -----------------------------------
-        float z[2][4], xqw[2][4], at[2][4];
+        // ---- Z = XK W + b (two accumulator chains), XQ W + b, XQ XK^T ------------------------
+        float z[2][4], z2[2][4], xqw[2][4], at[2][4];
+        uint32_t k[4][4], q[4][4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            ldmatrix_x4(xk_s + swz128(lrow, 2 * kk + lchunk), k[kk][0], k[kk][1], k[kk][2], k[kk][3]);
+            ldmatrix_x4(xq_s + swz128(lrow, 2 * kk + lchunk), q[kk][0], q[kk][1], q[kk][2], q[kk][3]);
+        }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             z[nt][0] = z[nt][2] = xqw[nt][0] = xqw[nt][2] = bc[nt][0];
             z[nt][1] = z[nt][3] = xqw[nt][1] = xqw[nt][3] = bc[nt][1];
-            at[nt][0] = at[nt][1] = at[nt][2] = at[nt][3] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) z2[nt][e] = at[nt][e] = 0.f;
         }
+        uint32_t wf[4][4];  // W as bf16 B fragments: [k-slice][n-tile 0 lo/hi, n-tile 1 lo/hi]
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            uint32_t k0, k1, k2, k3, q0, q1, q2, q3;
-            ldmatrix_x4(xk_s + swz128(lrow, 2 * kk + lchunk), k0, k1, k2, k3);
-            ldmatrix_x4(xq_s + swz128(lrow, 2 * kk + lchunk), q0, q1, q2, q3);
-            const uint32_t w00 = pack_bf16x2(Wt[2 * kk][0], Wt[2 * kk][1]);
-            const uint32_t w01 = pack_bf16x2(Wt[2 * kk + 1][0], Wt[2 * kk + 1][1]);
-            const uint32_t w10 = pack_bf16x2(Wt[2 * kk][2], Wt[2 * kk][3]);
-            const uint32_t w11 = pack_bf16x2(Wt[2 * kk + 1][2], Wt[2 * kk + 1][3]);
-            mma_bf16_16816(z[0], k0, k1, k2, k3, w00, w01);
-            mma_bf16_16816(z[1], k0, k1, k2, k3, w10, w11);
-            mma_bf16_16816(xqw[0], q0, q1, q2, q3, w00, w01);
-            mma_bf16_16816(xqw[1], q0, q1, q2, q3, w10, w11);
-            mma_bf16_16816(at[0], q0, q1, q2, q3, k0, k2);
-            mma_bf16_16816(at[1], q0, q1, q2, q3, k1, k3);
+            wf[kk][0] = pack_bf16x2(Wt[2 * kk][0], Wt[2 * kk][1]);
+            wf[kk][1] = pack_bf16x2(Wt[2 * kk + 1][0], Wt[2 * kk + 1][1]);
+            wf[kk][2] = pack_bf16x2(Wt[2 * kk][2], Wt[2 * kk][3]);
+            wf[kk][3] = pack_bf16x2(Wt[2 * kk + 1][2], Wt[2 * kk + 1][3]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            mma_bf16_16816(z[0], k[kk][0], k[kk][1], k[kk][2], k[kk][3], wf[kk][0], wf[kk][1]);
+            mma_bf16_16816(z[1], k[kk][0], k[kk][1], k[kk][2], k[kk][3], wf[kk][2], wf[kk][3]);
+            mma_bf16_16816(z2[0], k[kk + 2][0], k[kk + 2][1], k[kk + 2][2], k[kk + 2][3], wf[kk + 2][0], wf[kk + 2][1]);
+            mma_bf16_16816(z2[1], k[kk + 2][0], k[kk + 2][1], k[kk + 2][2], k[kk + 2][3], wf[kk + 2][2], wf[kk + 2][3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) z[nt][e] += z2[nt][e];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            mma_bf16_16816(xqw[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], wf[kk][0], wf[kk][1]);
+            mma_bf16_16816(xqw[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], wf[kk][2], wf[kk][3]);
+            mma_bf16_16816(at[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][0], k[kk][2]);
+            mma_bf16_16816(at[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][1], k[kk][3]);
+        }
+        // XK and XQ at this thread's own positions: the A fragment of k-slice w
+        uint32_t k_own[4], q_own[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            k_own[i] = pick4(k, w, i);
+            q_own[i] = pick4(q, w, i);
         }
 
-        // ---- LayerNorm statistics of Z (and of Zbar of the previous mini-batch) -------------
+        // ---- LayerNorm statistics of Z --------------------------------------------------------
         {
             float2 r0, r1;
             warp_row_partials(z, r0, r1);
             if (t == 0) {
-                s.red1[w][g] = r0;
-                s.red1[w][g + 8] = r1;
+                put_partial(s.red1, g, w, r0);
+                put_partial(s.red1, g + 8, w, r1);
             }
         }
-        if (tid == 0 && m >= 2) bulk_wait_group_read<1>();  // out buffer (m-1)&1 is free again
-        named_barrier_sync(1, kThreads);  // ---------------------------------------- B1
+        named_barrier_sync(1, kThreads);  // ------------------------------------------------ B1
         if (s.fail) {
             failed = true;
             break;
         }
-        if (w == 0 && issued < n_mb) issue(issued++);  // stage (m-1) % kStages is free
+        if (m > 0) store_out(s.red3[(m - 1) & 1], a, chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
 
-        // finish out of the previous mini-batch into the staging buffer
-        if (m > 0) {
-            float mu0, rs0, mu1, rs1;
-            merge_row(s.red3, g, a.eps, mu0, rs0);
-            merge_row(s.red3, g + 8, a.eps, mu1, rs1);
-            uint8_t* ob = &s.outb[(m - 1) & 1][0];
+        // ---- g = ln_fused_l2_bwd(Z, XV - XK): partial sums of q and q * xhat -----------------
+        float mu[2], rs[2];
+        merge_row(s.red1, g, eps, mu[0], rs[0]);
+        merge_row(s.red1, g + 8, eps, mu[1], rs[1]);
+        float2 xh[2][2], qv[2][2];  // [n-tile][row g / g+8], feature pairs
+        float sq[2], sqx[2];
+        {
+            float2 sq2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)}, sqx2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                float2 x0 = unpack_bf16x2(xq_prev[nt][0]), x1 = unpack_bf16x2(xq_prev[nt][1]);
-                float o00 = x0.x + lw[nt][0] * (zbar_prev[nt][0] - mu0) * rs0 + lb[nt][0];
-                float o01 = x0.y + lw[nt][1] * (zbar_prev[nt][1] - mu0) * rs0 + lb[nt][1];
-                float o10 = x1.x + lw[nt][0] * (zbar_prev[nt][2] - mu1) * rs1 + lb[nt][0];
-                float o11 = x1.y + lw[nt][1] * (zbar_prev[nt][3] - mu1) * rs1 + lb[nt][1];
-                *reinterpret_cast<uint32_t*>(ob + swz128(g, 2 * w + nt) + 4 * t) = pack_bf16x2(o00, o01);
-                *reinterpret_cast<uint32_t*>(ob + swz128(g + 8, 2 * w + nt) + 4 * t) = pack_bf16x2(o10, o11);
-            }
-            fence_proxy_async_smem();
-        }
-
-        // ---- g = ln_fused_l2_bwd(Z, XV - XK) -------------------------------------------------
-        float mu[2], rs[2];
-        merge_row(s.red1, g, a.eps, mu[0], rs[0]);
-        merge_row(s.red1, g + 8, a.eps, mu[1], rs[1]);
-        float xh[2][4], q[2][4];
-        float sq[2] = {0.f, 0.f}, sqx[2] = {0.f, 0.f};
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {  // row g (hr=0) or g+8 (hr=1)
-                const int row = g + 8 * hr;
-                float2 kv = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(
-                    &s.xk[st][0] + swz128(row, 2 * w + nt) + 4 * t));
-                float2 vv = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(
-                    &s.xv[st][0] + swz128(row, 2 * w + nt) + 4 * t));
-                float tg[2] = {vv.x - kv.x, vv.y - kv.y};
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float x = (z[nt][2 * hr + e] - mu[hr]) * rs[hr];
-                    float qq = lw[nt][e] * (lw[nt][e] * x + lb[nt][e] - tg[e]);
-                    xh[nt][2 * hr + e] = x;
-                    q[nt][2 * hr + e] = qq;
-                    sq[hr] += qq;
-                    sqx[hr] += qq * x;
+                for (int hr = 0; hr < 2; ++hr) {  // row g (hr=0) or g+8 (hr=1); A fragment order a0..a3
+                    const float2 kv = unpack_bf16x2(k_own[2 * nt + hr]);
+                    const float2 vv = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(
+                        &s.xv[st][0] + swz128(g + 8 * hr, 2 * w + nt) + 4 * t));
+                    const float2 x = fma2(f2(z[nt][2 * hr], z[nt][2 * hr + 1]), bc2(rs[hr]), bc2(-mu[hr] * rs[hr]));
+                    // q = ln_w * (ln_w * xhat + ln_b - (xv - xk))
+                    const float2 r = add2(fma2(lw2[nt], x, lb2[nt]), fma2(vv, bc2(-1.f), kv));
+                    const float2 qq = mul2(lw2[nt], r);
+                    xh[nt][hr] = x;
+                    qv[nt][hr] = qq;
+                    sq2[hr] = add2(sq2[hr], qq);
+                    sqx2[hr] = fma2(qq, x, sqx2[hr]);
                 }
             }
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                sq[hr] = quad_sum(sq2[hr].x + sq2[hr].y);
+                sqx[hr] = quad_sum(sqx2[hr].x + sqx2[hr].y);
+            }
         }
-        sq[0] = quad_sum(sq[0]); sq[1] = quad_sum(sq[1]);
-        sqx[0] = quad_sum(sqx[0]); sqx[1] = quad_sum(sqx[1]);
         if (t == 0) {
-            s.red2[w][g] = make_float2(sq[0], sqx[0]);
-            s.red2[w][g + 8] = make_float2(sq[1], sqx[1]);
+            put_partial(s.red2, g, w, f2(sq[0], sqx[0]));
+            put_partial(s.red2, g + 8, w, f2(sq[1], sqx[1]));
         }
-        named_barrier_sync(1, kThreads);  // ---------------------------------------- B2
-        if (m > 0 && tid == 0) {
-            tma_store_3d(&maps.out, 0, static_cast<int>((m - 1) * K), chain, &s.outb[(m - 1) & 1][0]);
-            bulk_commit_group();
-        }
+
+        named_barrier_sync(1, kThreads);  // ------------------------------------------------ B2
         float gg[2][4];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int row = g + 8 * hr;
-            float Sq = 0.f, Sqx = 0.f;
+            const float4 r0 = s.red2[row][0], r1 = s.red2[row][1];
+            const float Sq = (r0.x + r0.z) + (r1.x + r1.z), Sqx = (r0.y + r0.w) + (r1.y + r1.w);
+            const float sc = (row < Km) ? rs[hr] * (1.0f / TTT_D) : 0.f;
 #pragma unroll
-            for (int ww = 0; ww < kWarps; ++ww) {
-                Sq += s.red2[ww][row].x;
-                Sqx += s.red2[ww][row].y;
+            for (int nt = 0; nt < 2; ++nt) {
+                const float2 v = mul2(fma2(xh[nt][hr], bc2(-Sqx), fma2(bc2(static_cast<float>(TTT_D)), qv[nt][hr], bc2(-Sq))),
+                                      bc2(sc));
+                gg[nt][2 * hr] = v.x;
+                gg[nt][2 * hr + 1] = v.y;
             }
-            const bool valid = row < Km;
-            const float sc = rs[hr] * (1.0f / TTT_D);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float v = (TTT_D * q[nt][2 * hr + e] - Sq - xh[nt][2 * hr + e] * Sqx) * sc;
-                    gg[nt][2 * hr + e] = valid ? v : 0.f;
-                }
         }
 
-        // ---- Zbar = XQ W + b - M g ------------------------------------------------------------
         const float* lr_s = s.lr[st];
-        const float tg0 = s.te[g], tg8 = s.te[g + 8];
-        const float l0 = lr_s[2 * t], l1 = lr_s[2 * t + 1], l8 = lr_s[2 * t + 8], l9 = lr_s[2 * t + 9];
-        auto Mv = [&](float attn, float te_i, float lr_j, int i, int j) {
-            return (j <= i) ? -(te_i * lr_j * (attn + 1.0f)) : 0.f;
-        };
-        const uint32_t ma0 = pack_bf16x2(Mv(at[0][0], tg0, l0, g, 2 * t), Mv(at[0][1], tg0, l1, g, 2 * t + 1));
-        const uint32_t ma1 = pack_bf16x2(Mv(at[0][2], tg8, l0, g + 8, 2 * t), Mv(at[0][3], tg8, l1, g + 8, 2 * t + 1));
-        const uint32_t ma2 = pack_bf16x2(Mv(at[1][0], tg0, l8, g, 2 * t + 8), Mv(at[1][1], tg0, l9, g, 2 * t + 9));
-        const uint32_t ma3 = pack_bf16x2(Mv(at[1][2], tg8, l8, g + 8, 2 * t + 8), Mv(at[1][3], tg8, l9, g + 8, 2 * t + 9));
-        uint32_t gb[2][2];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            gb[nt][0] = movmatrix_trans(pack_bf16x2(gg[nt][0], gg[nt][1]));  // tokens 0-7
-            gb[nt][1] = movmatrix_trans(pack_bf16x2(gg[nt][2], gg[nt][3]));  // tokens 8-15
-        }
-        mma_bf16_16816(xqw[0], ma0, ma1, ma2, ma3, gb[0][0], gb[0][1]);
-        mma_bf16_16816(xqw[1], ma0, ma1, ma2, ma3, gb[1][0], gb[1][1]);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) zbar_prev[nt][e] = xqw[nt][e];
-            xq_prev[nt][0] = *reinterpret_cast<const uint32_t*>(&s.xq[st][0] + swz128(g, 2 * w + nt) + 4 * t);
-            xq_prev[nt][1] = *reinterpret_cast<const uint32_t*>(&s.xq[st][0] + swz128(g + 8, 2 * w + nt) + 4 * t);
-        }
-        {
-            float2 r0, r1;
-            warp_row_partials(zbar_prev, r0, r1);
-            if (t == 0) {
-                s.red3[w][g] = r0;
-                s.red3[w][g + 8] = r1;
-            }
-        }
-
-        // ---- state update -----------------------------------------------------------------------
-        const float lg0 = lr_s[g], lg8 = lr_s[g + 8];
+        // ---- state update (the loop-carried path) --------------------------------------------
         if (full_mb) {
-            const float tl = s.te[K - 1];
-            // A = (-t_{K-1} lr_tok g)^T: features x tokens, via register transposes
+            const float lg0 = -te_last * lr_s[g], lg8 = -te_last * lr_s[g + 8];
+            // A = (-t_{K-1} lr_tok g)^T: this warp's features x tokens, by register transposes
             uint32_t ua[2][2];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                ua[nt][0] = movmatrix_trans(pack_bf16x2(-tl * lg0 * gg[nt][0], -tl * lg0 * gg[nt][1]));
-                ua[nt][1] = movmatrix_trans(pack_bf16x2(-tl * lg8 * gg[nt][2], -tl * lg8 * gg[nt][3]));
+                ua[nt][0] = movmatrix_trans(pack_bf16x2(lg0 * gg[nt][0], lg0 * gg[nt][1]));
+                ua[nt][1] = movmatrix_trans(pack_bf16x2(lg8 * gg[nt][2], lg8 * gg[nt][3]));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -365,18 +417,48 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
                 mma_bf16_16816(Wt[2 * kk], ua[0][0], ua[1][0], ua[0][1], ua[1][1], r0, r1);
                 mma_bf16_16816(Wt[2 * kk + 1], ua[0][0], ua[1][0], ua[0][1], ua[1][1], r2, r3);
             }
-            // b -= t_{K-1} sum_tok lr_tok g_tok
+            mma_bf16_16816(Bt, ua[0][0], ua[1][0], ua[0][1], ua[1][1], ones_b, ones_b);  // b update
+            // spread b to the layout of Z's columns: feature 16w + 8nt + 2t + e sits in lane
+            // 4 (2t + e), register Bt[2 nt]
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                bc[0][e] = __shfl_sync(0xffffffffu, Bt[0], 4 * (2 * t + e));
+                bc[1][e] = __shfl_sync(0xffffffffu, Bt[2], 4 * (2 * t + e));
+            }
+        }
+
+        // ---- Zbar = XQ W + b - M g  (finished into out during the next mini-batch) -------------
+        {
+            const float tg0 = te_g, tg8 = te_g8;
+            const float l0 = lr_s[2 * t], l1 = lr_s[2 * t + 1], l8 = lr_s[2 * t + 8], l9 = lr_s[2 * t + 9];
+            auto Mv = [&](float attn, float te_i, float lr_j, int i, int j) {
+                return (j <= i) ? -(te_i * lr_j * (attn + 1.0f)) : 0.f;
+            };
+            const uint32_t ma0 = pack_bf16x2(Mv(at[0][0], tg0, l0, g, 2 * t), Mv(at[0][1], tg0, l1, g, 2 * t + 1));
+            const uint32_t ma1 = pack_bf16x2(Mv(at[0][2], tg8, l0, g + 8, 2 * t), Mv(at[0][3], tg8, l1, g + 8, 2 * t + 1));
+            const uint32_t ma2 = pack_bf16x2(Mv(at[1][0], tg0, l8, g, 2 * t + 8), Mv(at[1][1], tg0, l9, g, 2 * t + 9));
+            const uint32_t ma3 = pack_bf16x2(Mv(at[1][2], tg8, l8, g + 8, 2 * t + 8), Mv(at[1][3], tg8, l9, g + 8, 2 * t + 9));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const uint32_t b0 = movmatrix_trans(pack_bf16x2(gg[nt][0], gg[nt][1]));  // tokens 0-7
+                const uint32_t b1 = movmatrix_trans(pack_bf16x2(gg[nt][2], gg[nt][3]));  // tokens 8-15
+                mma_bf16_16816(xqw[nt], ma0, ma1, ma2, ma3, b0, b1);
+            }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float v = lg0 * gg[nt][e] + lg8 * gg[nt][2 + e];
-                    v += __shfl_xor_sync(0xffffffffu, v, 4);
-                    v += __shfl_xor_sync(0xffffffffu, v, 8);
-                    v += __shfl_xor_sync(0xffffffffu, v, 16);
-                    bc[nt][e] -= tl * v;
-                }
-        } else if (a.W_grad_tail || a.b_grad_tail) {
+                for (int e = 0; e < 4; ++e) zbar_prev[nt][e] = xqw[nt][e];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xq_prev[i] = q_own[i];
+            float2 r0, r1;
+            warp_row_partials(zbar_prev, r0, r1);
+            if (t == 0) {
+                put_partial(s.red3[m & 1], g, w, r0);
+                put_partial(s.red3[m & 1], g + 8, w, r1);
+            }
+        }
+
+        if (!full_mb && (a.W_grad_tail || a.b_grad_tail)) {
             // remainder: report the un-scaled grad sums in fp32
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -405,44 +487,17 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
                 a.b_grad_tail[static_cast<long long>(chain) * TTT_D + tid] = acc;
             }
         }
+        // this warp is done with stage st
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[st]);
     }
 
-    if (failed) {
-        // drain the loads still in flight (bounded), then leave
-        if (tid == 0) {
-            for (long long mm = m; mm < issued; ++mm)
-                mbar_wait_bounded(&s.full[mm % kStages], static_cast<uint32_t>((mm / kStages) & 1),
-                                  kDrainPolls, nullptr);
-            bulk_wait_group<0>();
-        }
-        __syncthreads();
-        return;
-    }
+    if (failed) return;  // the producer warp drains the loads still in flight
 
     // ---- the last mini-batch's output ---------------------------------------------------------
     if (n_mb > 0) {
-        if (tid == 0 && n_mb >= 2) bulk_wait_group_read<1>();
         named_barrier_sync(1, kThreads);
-        float mu0, rs0, mu1, rs1;
-        merge_row(s.red3, g, a.eps, mu0, rs0);
-        merge_row(s.red3, g + 8, a.eps, mu1, rs1);
-        uint8_t* ob = &s.outb[(n_mb - 1) & 1][0];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            float2 x0 = unpack_bf16x2(xq_prev[nt][0]), x1 = unpack_bf16x2(xq_prev[nt][1]);
-            float o00 = x0.x + lw[nt][0] * (zbar_prev[nt][0] - mu0) * rs0 + lb[nt][0];
-            float o01 = x0.y + lw[nt][1] * (zbar_prev[nt][1] - mu0) * rs0 + lb[nt][1];
-            float o10 = x1.x + lw[nt][0] * (zbar_prev[nt][2] - mu1) * rs1 + lb[nt][0];
-            float o11 = x1.y + lw[nt][1] * (zbar_prev[nt][3] - mu1) * rs1 + lb[nt][1];
-            *reinterpret_cast<uint32_t*>(ob + swz128(g, 2 * w + nt) + 4 * t) = pack_bf16x2(o00, o01);
-            *reinterpret_cast<uint32_t*>(ob + swz128(g + 8, 2 * w + nt) + 4 * t) = pack_bf16x2(o10, o11);
-        }
-        fence_proxy_async_smem();
-        named_barrier_sync(1, kThreads);
-        if (tid == 0) {
-            tma_store_3d(&maps.out, 0, static_cast<int>((n_mb - 1) * K), chain, ob);
-            bulk_commit_group();
-        }
+        store_out(s.red3[(n_mb - 1) & 1], a, chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
     }
 
     // ---- final state ------------------------------------------------------------------------
@@ -451,22 +506,19 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     for (int jt = 0; jt < 8; ++jt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
+            const int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
             Wl[j * TTT_D + f] = Wt[jt][e];
         }
-    if (g == 0)  // every lane group g holds the same b; lanes 0..3 of each warp write it
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + 8 * nt + 2 * t + e] = bc[nt][e];
+    if (t == 0) {
+        a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + g] = Bt[0];
+        a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + g + 8] = Bt[2];
+    }
     if (a.rem == 0) {
         if (a.W_grad_tail)
             for (int i = tid; i < TTT_D * TTT_D; i += kThreads)
                 a.W_grad_tail[static_cast<long long>(chain) * TTT_D * TTT_D + i] = 0.f;
         if (a.b_grad_tail && tid < TTT_D) a.b_grad_tail[static_cast<long long>(chain) * TTT_D + tid] = 0.f;
     }
-    if (tid == 0) bulk_wait_group<0>();
 }
 
 }  // namespace
@@ -476,7 +528,7 @@ cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaSt
     cudaError_t e = cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    linear_tc_kernel<<<static_cast<unsigned>(a.B * a.H), kThreads, smem, st>>>(a, maps);
+    linear_tc_kernel<<<static_cast<unsigned>(a.B * a.H), kBlock, smem, st>>>(a, maps);
     return cudaGetLastError();
 }
 

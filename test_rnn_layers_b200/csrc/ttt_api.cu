@@ -351,6 +351,8 @@ int ttt_linear_decode_step(const void* xq, const void* xk, const void* xv, const
     a.xq = xq; a.xk = xk; a.xv = xv; a.lr = lr; a.token_eta = token_eta; a.ln_w = ln_w; a.ln_b = ln_b;
     a.W = W; a.b = b; a.W_grad = W_grad; a.b_grad = b_grad; a.B = B; a.H = H; a.K = mini_batch;
     a.p = static_cast<int>(seqlen_offset % mini_batch); a.eps = eps; a.out = out;
+    a.status = status_word();
+    a.wait_limit = wait_limit();
     cudaError_t e = ttt::launch_decode(a, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_decode_step launch");
     return ok();

@@ -101,12 +101,51 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// One poll that may suspend the thread for up to `hint_ns` nanoseconds while the phase is
+// incomplete (for a waiter with nothing else to do, e.g. a producer warp).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: false (and the status bit raised) if the phase did not complete within
-// `limit` polls.  Never spins forever.
+// `limit` polls.  Never spins forever.  A phase that has already completed (the common case
+// for a prefetched stage) is seen by one non-blocking test; otherwise the poll loop uses
+// try_wait, which may suspend the thread for a short while per poll.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, long long limit,
                                                   unsigned int* status) {
-    for (long long i = 0; i < limit; ++i)
+    if (limit > 0 && mbar_test_wait(bar, parity)) return true;
+    for (long long i = 1; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
+    raise_status(status, 1u);
+    return false;
+}
+
+// Bounded wait of an idle waiter: each poll may sleep up to hint_ns, so few polls are issued.
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t* bar, uint32_t parity, long long limit,
+                                                        uint32_t hint_ns, unsigned int* status) {
+    for (long long i = 0; i < limit; ++i)
+        if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
     raise_status(status, 1u);
     return false;
 }
@@ -154,6 +193,15 @@ template <int N> __device__ __forceinline__ void bulk_wait_group() {
 __device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
                  ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
+// Untiled bulk copy global -> shared, completion counted in bytes on an mbarrier.  Both
+// addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // The mbarrier receives one arrival once all of this thread's earlier cp.async have landed.

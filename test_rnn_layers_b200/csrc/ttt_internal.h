@@ -77,6 +77,8 @@ struct DecodeArgs {
     int p;          // position inside the mini-batch: seqlen_offset % K
     float eps;
     void* out;
+    unsigned int* status;
+    long long wait_limit;
 };
 
 // Tensor maps of the bf16 tensor-core prefill kernel: [B*H, L, 64] bf16 viewed 3-D,

@@ -48,6 +48,7 @@ def compare(res, ref, tol, tol_out=None, what=""):
         "W_grad_tail": rel_l2(to_np(Wg).reshape(-1, 64, 64), ref["W_grad_tail"]),
         "b_grad_tail": rel_l2(to_np(bg).reshape(-1, 64), ref["b_grad_tail"]),
     }
+    print(f"[parity] {what}: " + ", ".join(f"{k}={e:.2e}" for k, e in errs.items()))
     for k, e in errs.items():
         t = tol_out if (k == "out" and tol_out is not None) else tol
         assert e <= t, f"{what} {k}: max rel L2 {e:.3e} > {t:.0e}  (all: {errs})"
