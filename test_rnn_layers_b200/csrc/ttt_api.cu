@@ -316,7 +316,19 @@ int ttt_mlp_forward(const void* XQ, const void* XK, const void* XV, const float*
     a.status = status_word();
     a.wait_limit = wait_limit();
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = L == 0 ? ttt::launch_mlp_state_copy(a, st) : ttt::launch_mlp_simt(a, dtype, st);
+    cudaError_t e;
+    if (L == 0) {
+        e = ttt::launch_mlp_state_copy(a, st);
+    } else if (dtype == TTT_F32 || (flags & TTT_FLAG_FP32_COMPUTE)) {
+        e = ttt::launch_mlp_simt(a, dtype, st);
+    } else {
+        ttt::LinearMaps maps;
+        if ((rc = encode_act_map(&maps.xq, XQ, chains, L, mini_batch, "XQ"))) return rc;
+        if ((rc = encode_act_map(&maps.xk, XK, chains, L, mini_batch, "XK"))) return rc;
+        if ((rc = encode_act_map(&maps.xv, XV, chains, L, mini_batch, "XV"))) return rc;
+        maps.out = maps.xq;
+        e = ttt::launch_mlp_tc(a, maps, st);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "ttt_mlp_forward launch");
     return ok();
 }

@@ -81,8 +81,8 @@ struct DecodeArgs {
     long long wait_limit;
 };
 
-// Tensor maps of the bf16 tensor-core prefill kernel: [B*H, L, 64] bf16 viewed 3-D,
-// box {64, K, 1}, 128-byte swizzle.
+// Tensor maps of the bf16 tensor-core prefill kernels: [B*H, L, 64] bf16 viewed 3-D,
+// box {64, K, 1}, 128-byte swizzle (the TTT-MLP kernel leaves `out` unused).
 struct LinearMaps {
     CUtensorMap xq, xk, xv, out;
 };
@@ -92,6 +92,7 @@ cudaError_t launch_linear_simt(const LinearArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t s);
 cudaError_t launch_linear_state_copy(const LinearArgs& a, cudaStream_t s);
 cudaError_t launch_mlp_simt(const MlpArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_mlp_tc(const MlpArgs& a, const LinearMaps& maps, cudaStream_t s);
 cudaError_t launch_mlp_state_copy(const MlpArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t s);
 

@@ -58,3 +58,81 @@ def test_mlp_L0(libttt):
     x = synth.linear_inputs(w)
     out, W1, b1, W2, b2 = gpu_mlp(libttt, x, w)
     assert out.numel() == 0 and np.array_equal(to_np(W2)[0], x["W2"])
+
+
+def _mlp_inputs(w):
+    x = synth.linear_inputs(w)
+    x["b1"] = synth.random_bias(w, "B1", x["b1"].shape)
+    x["b2"] = synth.random_bias(w, "B2", x["b2"].shape)
+    return x
+
+
+@pytest.mark.parametrize("L,K", [(16 * 9 + 3, 16), (8 * 7 + 5, 8), (13 * 4, 13), (3, 1), (16 * 40, 16)])
+def test_mlp_tensor_core_ragged(libttt, L, K):
+    """bf16 inputs take the tensor-core kernel: several mini-batches, a ragged tail, K < 16."""
+    w = synth.workload(3, B=2, H=2, L=L, K=K, dtype="bf16", seed=0x3B00 + L * 17 + K)
+    x = _mlp_inputs(w)
+    _check(gpu_mlp(libttt, x, w), oracle_mlp(x, w), 1e-2)
+
+
+def test_mlp_token_eta_table(libttt):
+    w = synth.workload(3, B=1, H=2, L=16 * 5 + 7, dtype="bf16")
+    x = _mlp_inputs(w)
+    te = np.linspace(1.0, 0.3, 16).astype(np.float32)
+    res = libttt.ttt_mlp_forward(dev_act(x, "XQ"), dev_act(x, "XK"), dev_act(x, "XV"), dev_f32(x["lr"]),
+                                 dev_f32(x["W1"]), dev_f32(x["b1"]), dev_f32(x["W2"]), dev_f32(x["b2"]),
+                                 dev_f32(x["ln_w"]), dev_f32(x["ln_b"]), mini_batch=w.K, eps=w.eps,
+                                 token_eta=dev_f32(te))
+    torch.cuda.synchronize()
+    ref = oracle.default().mlp_forward(x["XQ"], x["XK"], x["XV"], x["lr"], x["W1"], x["b1"], x["W2"], x["b2"],
+                                       x["ln_w"], x["ln_b"], w.K, w.eps, token_eta=te.astype(np.float64))
+    _check(res, ref, 1e-2)
+
+
+def test_mlp_per_chain_state(libttt):
+    """A continuation: per-chain initial states of shape [B,H,...]."""
+    w = synth.workload(3, B=2, H=2, L=16 * 4 + 9, dtype="bf16")
+    x = _mlp_inputs(w)
+    rng = np.random.default_rng(11)
+    st = {}
+    for k in ("W1", "b1", "W2", "b2"):
+        base = np.broadcast_to(x[k], (2,) + x[k].shape)
+        st[k] = (base + rng.normal(0, 0.01, base.shape)).astype(np.float32)
+    res = libttt.ttt_mlp_forward(dev_act(x, "XQ"), dev_act(x, "XK"), dev_act(x, "XV"), dev_f32(x["lr"]),
+                                 dev_f32(st["W1"]), dev_f32(st["b1"]), dev_f32(st["W2"]), dev_f32(st["b2"]),
+                                 dev_f32(x["ln_w"]), dev_f32(x["ln_b"]), mini_batch=w.K, eps=w.eps)
+    torch.cuda.synchronize()
+    ref = oracle.default().mlp_forward(x["XQ"], x["XK"], x["XV"], x["lr"], st["W1"], st["b1"], st["W2"],
+                                       st["b2"], x["ln_w"], x["ln_b"], w.K, w.eps, state_per_chain=True)
+    _check(res, ref, 1e-2)
+
+
+def test_mlp_fp32_compute_flag(libttt):
+    """bf16 inputs with TTT_FLAG_FP32_COMPUTE take the fp32 kernel; its bf16 output is compared at
+    bf16 resolution, its fp32 states at fp32 accuracy."""
+    w = synth.workload(3, B=1, H=2, L=16 * 3 + 5, dtype="bf16")
+    x = _mlp_inputs(w)
+    res = gpu_mlp(libttt, x, w, flags=libttt.TTT_FLAG_FP32_COMPUTE)
+    ref = oracle_mlp(x, w)
+    for k, t in zip(KEYS, res):
+        e = rel_l2(to_np(t).reshape(ref[k].shape), ref[k])
+        assert e <= (4e-3 if k == "out" else 1e-5), f"{k}: {e:.3e}"
+
+
+def test_mlp_bounded_wait_timeout_reports_and_recovers(libttt):
+    """Every bounded wait of the tensor-core kernel gives up at once: the status word reports it,
+    the context stays usable and the next call is correct."""
+    w = synth.workload(3, B=1, H=2, L=16 * 6 + 3, dtype="bf16")
+    x = _mlp_inputs(w)
+    libttt.ttt_device_status(clear=True)
+    libttt.ttt_set_wait_limit(-1)
+    try:
+        gpu_mlp(libttt, x, w)
+        with pytest.raises(libttt.TTTError) as e:
+            libttt.ttt_device_status(clear=True)
+        assert e.value.code == libttt.TTT_ERR_TIMEOUT
+    finally:
+        libttt.ttt_set_wait_limit(0)
+    assert libttt.ttt_device_status(clear=True) == 0
+    _check(gpu_mlp(libttt, x, w), oracle_mlp(x, w), 1e-2)
+    assert libttt.ttt_device_status() == 0
