@@ -1,6 +1,7 @@
 """Benchmark of the TTT scan on B200: TTT layer tokens/s and the fraction of the per-layer roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,mlp,decode]
+                    [--no-cpu-baseline] [--no-headline]
 
 One step = one ttt_linear_forward over the 1B-layer workload (B=8, H=32, L=8200, d=64, K=16,
 bf16 activations, fp32 state): every row of the path at once -- the partition, 512 full
@@ -445,6 +446,8 @@ def main():
     ap.add_argument("--rows", default="linear,mlp,decode",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-headline", action="store_true",
+                    help="profiling aid: run only the --rows rows and print them (no headline line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -458,8 +461,20 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     peaks = measured_peaks()
-    line = bench_linear(args, world, rank, local, peaks)
     rows = [r.strip() for r in args.rows.split(",") if r.strip()]
+    if args.no_headline:
+        extra = {}
+        if "mlp" in rows:
+            extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
+        if "decode" in rows:
+            extra["ttt_linear_decode"] = bench_decode(args, world, peaks)
+        if rank == 0:
+            print(json.dumps({"rows": extra}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    line = bench_linear(args, world, rank, local, peaks)
     extra = {}
     if "mlp" in rows:
         extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
