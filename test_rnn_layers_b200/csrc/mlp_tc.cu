@@ -260,6 +260,24 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     const uint32_t idC1 = tc5::idesc_bf16(128, 16, 1, 0);
     const uint32_t idUp = tc5::idesc_bf16(128, 64, 1, 1);
 
+    // Operand descriptors, built once: per MMA only a constant offset is added (the single
+    // issuing thread is otherwise the bottleneck of these small-N MMAs).
+    const uint64_t dW1k = tc5::sdesc(smem_u32(&s.W1s[0][0]), 16, 1024);     // W1^T, K-major A
+    const uint64_t dW2k = tc5::sdesc(smem_u32(&s.W2s[0]), 16, 1024);        // W2, K-major A
+    const uint64_t dW2m = tc5::sdesc(smem_u32(&s.W2s[0]), 2048, 1024);      // W2^T, MN-major A (M = 64)
+    const uint64_t dX2k = tc5::sdesc(smem_u32(&s.X2s[0]), 16, 1024);        // X2, K-major B
+    const uint64_t dX2m = tc5::sdesc(smem_u32(&s.X2s[0]), kTile, 1024);     // X2^T, MN-major A
+    const uint64_t dXB2k = tc5::sdesc(smem_u32(&s.XB2s[0]), 16, 1024);      // Xbar2, K-major B
+    const uint64_t dG1m = tc5::sdesc(smem_u32(&s.G1s[0]), kTile, 1024);     // g1^T, MN-major A
+    const uint64_t dG1Lm = tc5::sdesc(smem_u32(&s.G1Ls[0]), kTile, 1024);   // (-t lr g1)^T, MN-major A
+    const uint64_t dG2k = tc5::sdesc(smem_u32(&s.G2s[0]), 16, 1024);        // g2, K-major B
+    const uint64_t dG2m = tc5::sdesc(smem_u32(&s.G2s[0]), 2048, 1024);      // g2^T, MN-major A (M = 64)
+    const uint64_t dG2Lm = tc5::sdesc(smem_u32(&s.G2Ls[0]), kTile, 1024);   // -t lr g2, MN-major B
+    const uint64_t dM1k = tc5::sdesc(smem_u32(&s.M1s[0]), 16, 1024);        // -M1, K-major B
+    const uint64_t dM2k = tc5::sdesc(smem_u32(&s.M2s[0]), 16, 1024);        // -M2, K-major B
+    const uint64_t dSk = tc5::sdesc(smem_u32(&s.stage[0][0]), 16, 1024);    // [XK; XQ] of stage 0, K-major B
+    const uint64_t dSm = tc5::sdesc(smem_u32(&s.stage[0][0]), kTile, 1024); // XK of stage 0, MN-major B
+
     uint32_t mpar = 0;  // phase parity of mma_bar
     auto mma_wait = [&]() {
         if (!mbar_wait_bounded(&s.mma_bar, mpar, wait_limit, a.status)) s.fail = 1;
@@ -292,8 +310,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             for (int t2 = 0; t2 < 2; ++t2)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc5::mma_ss(tm + cZQ + 32 * t2, tc5::sdesc(smem_u32(&s.W1s[t2][0]) + 32 * ks, 16, 1024),
-                                tc5::sdesc(smem_u32(xk_t) + 32 * ks, 16, 1024), idZQ, ks > 0);
+                    tc5::mma_ss(tm + cZQ + 32 * t2, tc5::sdesc_add(dW1k, t2 * 16384 + 32 * ks),
+                                tc5::sdesc_add(dSk, st * 3 * kTile + 32 * ks), idZQ, ks > 0);
             tc5::commit(&s.mma_bar);
         }
         // meanwhile: -M1 = -(eta * tril(XQ XK^T + 1)) into M1s (warp 4, mma.sync)
@@ -338,8 +356,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 16; ++ks)
-                tc5::mma_ss(tm + cZ2, tc5::sdesc(smem_u32(&s.W2s[0]) + 2048 * ks, 2048, 1024),
-                            tc5::sdesc(smem_u32(&s.X2s[0]) + (ks >> 2) * kTile + 32 * (ks & 3), 16, 1024), idM64,
+                tc5::mma_ss(tm + cZ2, tc5::sdesc_add(dW2m, 2048 * ks),
+                            tc5::sdesc_add(dX2k, (ks >> 2) * kTile + 32 * (ks & 3)), idM64,
                             ks > 0);
             tc5::commit(&s.mma_bar);
         }
@@ -406,8 +424,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             for (int t2 = 0; t2 < 2; ++t2)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    tc5::mma_ss(tm + cG1 + 16 * t2, tc5::sdesc(smem_u32(&s.W2s[0]) + t2 * 16384 + 32 * ks, 16, 1024),
-                                tc5::sdesc(smem_u32(&s.G2s[0]) + 32 * ks, 16, 1024), idG1, ks > 0);
+                    tc5::mma_ss(tm + cG1 + 16 * t2, tc5::sdesc_add(dW2k, t2 * 16384 + 32 * ks),
+                                tc5::sdesc_add(dG2k, 32 * ks), idG1, ks > 0);
             tc5::commit(&s.mma_bar);
         }
         mma_wait();
@@ -434,16 +452,14 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         if (tid == 0) {
 #pragma unroll
             for (int t2 = 0; t2 < 2; ++t2)
-                tc5::mma_ss(tm + cZQ + 32 * t2 + 16, tc5::sdesc(smem_u32(&s.G1s[0]) + t2 * 2 * kTile, kTile, 1024),
-                            tc5::sdesc(smem_u32(&s.M1s[0]), 16, 1024), idC1, 1);
+                tc5::mma_ss(tm + cZQ + 32 * t2 + 16, tc5::sdesc_add(dG1m, t2 * 2 * kTile), dM1k, idC1, 1);
             if (full_mb) {
 #pragma unroll
                 for (int t2 = 0; t2 < 2; ++t2) {
                     // W1^T += (-t lr g1)^T XK ;  W2 += X2^T (-t lr g2)
-                    tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc(smem_u32(&s.G1Ls[0]) + t2 * 2 * kTile, kTile, 1024),
-                                tc5::sdesc(smem_u32(xk_t), kTile, 1024), idUp, 1);
-                    tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc(smem_u32(&s.X2s[0]) + t2 * 2 * kTile, kTile, 1024),
-                                tc5::sdesc(smem_u32(&s.G2Ls[0]), kTile, 1024), idUp, 1);
+                    tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1Lm, t2 * 2 * kTile),
+                                tc5::sdesc_add(dSm, st * 3 * kTile), idUp, 1);
+                    tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc_add(dX2m, t2 * 2 * kTile), dG2Lm, idUp, 1);
                 }
             }
             tc5::commit(&s.mma_bar);
@@ -494,10 +510,10 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         if (tid == 0) {
 #pragma unroll
             for (int ks = 0; ks < 16; ++ks)
-                tc5::mma_ss(tm + cZB2, tc5::sdesc(smem_u32(&s.W2s[0]) + 2048 * ks, 2048, 1024),
-                            tc5::sdesc(smem_u32(&s.XB2s[0]) + (ks >> 2) * kTile + 32 * (ks & 3), 16, 1024), idM64,
+                tc5::mma_ss(tm + cZB2, tc5::sdesc_add(dW2m, 2048 * ks),
+                            tc5::sdesc_add(dXB2k, (ks >> 2) * kTile + 32 * (ks & 3)), idM64,
                             ks > 0);
-            tc5::mma_ss(tm + cZB2, tc5::sdesc(smem_u32(&s.G2s[0]), 2048, 1024), tc5::sdesc(smem_u32(&s.M2s[0]), 16, 1024),
+            tc5::mma_ss(tm + cZB2, dG2m, dM2k,
                         idM64, 1);
             tc5::commit(&s.mma_bar);
         }

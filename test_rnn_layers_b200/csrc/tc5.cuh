@@ -45,6 +45,10 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t smem_addr, uint32_t lbo_bytes
            (static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor `bytes` further on: the low 14 bits hold address / 16, and every operand
+// here lies in the first 256 KB of the shared window, so the add never leaves that field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D; a_mn / b_mn select MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |

@@ -134,3 +134,43 @@ def test_decode_full_size_sampled(libttt):
         assert rel_l2(chain_slice(out, chains, w.H), ref) <= 1e-2, t
     assert rel_l2(chain_slice(W, chains, w.H), st[0]) <= 1e-2
     assert rel_l2(chain_slice(Wg, chains, w.H), st[2]) <= 1e-2
+
+
+def test_decode_bounded_wait_timeout_reports_and_recovers(libttt):
+    """Every bounded wait of the decode kernel gives up at once: the status word reports it, the
+    context stays usable and the next step (on a fresh copy of the cache) is correct."""
+    L0 = 40
+    w = synth.workload(4, B=2, H=2, L=L0, decode_steps=1, dtype="f32", seed=0x4D0E)
+    x = synth.linear_inputs(w)
+    oW, ob, oWg, obg = _oracle_cache(x, w, L0)
+    f32 = lambda a: np.asarray(a, np.float32)
+
+    def cache():
+        return (dev_f32(f32(oW).reshape(2, 2, 64, 64)), dev_f32(f32(ob).reshape(2, 2, 64)),
+                dev_f32(f32(oWg).reshape(2, 2, 64, 64)), dev_f32(f32(obg).reshape(2, 2, 64)))
+
+    args = (_tok(x, "XQ", L0), _tok(x, "XK", L0), _tok(x, "XV", L0), dev_f32(np.ascontiguousarray(x["lr"][:, :, L0])),
+            dev_f32(x["ln_w"]), dev_f32(x["ln_b"]))
+    libttt.ttt_device_status(clear=True)
+    libttt.ttt_set_wait_limit(-1)
+    try:
+        libttt.ttt_linear_decode_step(*args, *cache(), seqlen_offset=L0, eps=w.eps)
+        torch.cuda.synchronize()
+        with pytest.raises(libttt.TTTError) as e:
+            libttt.ttt_device_status(clear=True)
+        assert e.value.code == libttt.TTT_ERR_TIMEOUT
+    finally:
+        libttt.ttt_set_wait_limit(0)
+    assert libttt.ttt_device_status(clear=True) == 0
+    state = [f32(a).astype(np.float64) for a in (oW, ob, oWg, obg)]
+    out = libttt.ttt_linear_decode_step(*args, *cache(), seqlen_offset=L0, eps=w.eps)
+    o = oracle.default()
+    ref = np.empty((4, 64))
+    for c in range(4):
+        bb, hh = divmod(c, 2)
+        ref[c], _ = o.decode_chain(x["XQ"][bb, hh, L0], x["XK"][bb, hh, L0], x["XV"][bb, hh, L0],
+                                   x["lr"][bb, hh, L0], x["ln_w"][hh], x["ln_b"][hh], state[0][c], state[1][c],
+                                   state[2][c], state[3][c], w.K, L0, w.eps)
+    torch.cuda.synchronize()
+    assert rel_l2(to_np(out).reshape(-1, 64), ref) <= 1e-5
+    assert libttt.ttt_device_status() == 0
