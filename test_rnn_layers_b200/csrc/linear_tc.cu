@@ -132,13 +132,6 @@ __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearAr
     }
 }
 
-// Select the fragment registers of k-slice `w` (warp-uniform) without local memory.
-__device__ __forceinline__ uint32_t pick4(const uint32_t (&v)[4][4], int w, int i) {
-    const uint32_t lo = (w & 1) ? v[1][i] : v[0][i];
-    const uint32_t hi = (w & 1) ? v[3][i] : v[2][i];
-    return (w & 2) ? hi : lo;
-}
-
 __global__ void __launch_bounds__(kBlock, 2)
 linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // align by a byte offset from the shared array itself (an integer round trip of the pointer
@@ -262,9 +255,20 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     const float eps = a.eps;
     const long long wait_limit = a.wait_limit;
     unsigned int* const status = a.status;
-    const float te_g = s.te[g], te_g8 = s.te[g + 8], te_last = s.te[K - 1];
+    const float te_last = s.te[K - 1];
     const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row supplied by this lane
     const int lchunk = lane >> 4;
+    const uint32_t own_off = swz128(lrow, 2 * w + lchunk);  // this warp's k-slice
+    // -t_i on the lower triangle j <= i, zero above, at this lane's four (i, j) positions per
+    // n-tile: M[i][j] = c (A[i][j] + 1) with c = -t_i lr_j, one multiply and one FMA per element
+    float tmask[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = g + 8 * (e >> 1), j = 8 * nt + 2 * t + (e & 1);
+            tmask[nt][e] = (j <= i) ? -s.te[i] : 0.f;
+        }
     float zbar_prev[2][4] = {};
     uint32_t xq_prev[4] = {};  // XQ at this thread's output positions (A fragment of k-slice w)
     bool failed = false;
@@ -322,13 +326,11 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             mma_bf16_16816(at[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][0], k[kk][2]);
             mma_bf16_16816(at[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][1], k[kk][3]);
         }
-        // XK and XQ at this thread's own positions: the A fragment of k-slice w
+        // XK and XQ at this thread's own positions: the A fragment of k-slice w (one more
+        // ldmatrix each is cheaper than selecting among the four slices held in registers)
         uint32_t k_own[4], q_own[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            k_own[i] = pick4(k, w, i);
-            q_own[i] = pick4(q, w, i);
-        }
+        ldmatrix_x4(xk_s + own_off, k_own[0], k_own[1], k_own[2], k_own[3]);
+        ldmatrix_x4(xq_s + own_off, q_own[0], q_own[1], q_own[2], q_own[3]);
 
         // ---- LayerNorm statistics of Z --------------------------------------------------------
         {
@@ -429,15 +431,17 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
 
         // ---- Zbar = XQ W + b - M g  (finished into out during the next mini-batch) -------------
         {
-            const float tg0 = te_g, tg8 = te_g8;
-            const float l0 = lr_s[2 * t], l1 = lr_s[2 * t + 1], l8 = lr_s[2 * t + 8], l9 = lr_s[2 * t + 9];
-            auto Mv = [&](float attn, float te_i, float lr_j, int i, int j) {
-                return (j <= i) ? -(te_i * lr_j * (attn + 1.0f)) : 0.f;
-            };
-            const uint32_t ma0 = pack_bf16x2(Mv(at[0][0], tg0, l0, g, 2 * t), Mv(at[0][1], tg0, l1, g, 2 * t + 1));
-            const uint32_t ma1 = pack_bf16x2(Mv(at[0][2], tg8, l0, g + 8, 2 * t), Mv(at[0][3], tg8, l1, g + 8, 2 * t + 1));
-            const uint32_t ma2 = pack_bf16x2(Mv(at[1][0], tg0, l8, g, 2 * t + 8), Mv(at[1][1], tg0, l9, g, 2 * t + 9));
-            const uint32_t ma3 = pack_bf16x2(Mv(at[1][2], tg8, l8, g + 8, 2 * t + 8), Mv(at[1][3], tg8, l9, g + 8, 2 * t + 9));
+            const float2 l01 = *reinterpret_cast<const float2*>(&lr_s[2 * t]);
+            const float2 l89 = *reinterpret_cast<const float2*>(&lr_s[2 * t + 8]);
+            // M = c (A + 1), c = tmask * lr_j
+            const float2 c00 = mul2(f2(tmask[0][0], tmask[0][1]), l01), c01 = mul2(f2(tmask[0][2], tmask[0][3]), l01);
+            const float2 c10 = mul2(f2(tmask[1][0], tmask[1][1]), l89), c11 = mul2(f2(tmask[1][2], tmask[1][3]), l89);
+            const float2 m00 = fma2(c00, f2(at[0][0], at[0][1]), c00), m01 = fma2(c01, f2(at[0][2], at[0][3]), c01);
+            const float2 m10 = fma2(c10, f2(at[1][0], at[1][1]), c10), m11 = fma2(c11, f2(at[1][2], at[1][3]), c11);
+            const uint32_t ma0 = pack_bf16x2(m00.x, m00.y);
+            const uint32_t ma1 = pack_bf16x2(m01.x, m01.y);
+            const uint32_t ma2 = pack_bf16x2(m10.x, m10.y);
+            const uint32_t ma3 = pack_bf16x2(m11.x, m11.y);
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 const uint32_t b0 = movmatrix_trans(pack_bf16x2(gg[nt][0], gg[nt][1]));  // tokens 0-7
