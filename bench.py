@@ -1,7 +1,7 @@
 """Benchmark of the TTT scan on B200: TTT layer tokens/s and the fraction of the per-layer roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,mlp,decode]
-                    [--no-cpu-baseline] [--no-headline]
+                    [--no-cpu-baseline] [--no-headline] [--seq-len L]
 
 One step = one ttt_linear_forward over the 1B-layer workload (B=8, H=32, L=8200, d=64, K=16,
 bf16 activations, fp32 state): every row of the path at once -- the partition, 512 full
@@ -234,7 +234,7 @@ def bench_linear(args, world, rank, local, peaks):
     import torch
 
     import test_rnn_layers_b200 as ttt
-    w = synth.workload(2, L=8200)
+    w = synth.workload(2, L=args.seq_len)
     x = synth.linear_inputs(w, values=False)
     XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
     lr, W0, b0, lnw, lnb = (dev_f32(x[k]) for k in ("lr", "W0", "b0", "ln_w", "ln_b"))
@@ -255,7 +255,7 @@ def bench_linear(args, world, rank, local, peaks):
     hbm, tf_burst, _, which = peaks
     nbytes = linear_bytes(B, H, L)
     achieved = nbytes / (ms / 1e3) / 1e9
-    traffic = kernel_traffic("linear_tc.cu", "linear_tc_kernel@1b_B8_H32_L8200")
+    traffic = kernel_traffic("linear_tc.cu", "linear_tc_kernel@1b_B8_H32_L8200") if L == 8200 else None
 
     # end to end through the public call from pinned host buffers
     host_in = {n: t.cpu().pin_memory() for n, t in (("XQ", XQ), ("XK", XK), ("XV", XV), ("lr", lr))}
@@ -446,6 +446,8 @@ def main():
     ap.add_argument("--rows", default="linear,mlp,decode",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=8200,
+                    help="profiling aid: sequence length of the TTT-Linear workload (the headline is 8200)")
     ap.add_argument("--no-headline", action="store_true",
                     help="profiling aid: run only the --rows rows and print them (no headline line)")
     args = ap.parse_args()
