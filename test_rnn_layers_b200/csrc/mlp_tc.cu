@@ -19,8 +19,9 @@
 //    product and b1 are per-thread register work, written back in bf16 straight into the
 //    operand layouts of the next MMAs (X2 as K-major B and MN-major A, g1 and lr-scaled g1 as
 //    MN-major A).
-//  * The two LayerNorms (loss gradient on Z2, output on Zbar2) run on token rows, 8 lanes per
-//    row, after a transpose of the 64 x 16 accumulator through shared memory.
+//  * The two LayerNorms (loss gradient on Z2, output on Zbar2) run on token rows, 16 lanes per
+//    row (all 8 warps), after a transpose of the 64 x 16 accumulator through shared memory.
+//  * W1's update takes its lr scaling on the small operand: W1^T += g1^T (-t_{K-1} lr XK).
 //  * The 16 x 16 token-pair products XQ XK^T and Xbar2 X2^T are too small for tcgen05
 //    (M >= 64) and run as mma.sync m16n8k16 on the same shared-memory tiles.
 //  * One thread issues every tcgen05.mma and commits to one mbarrier; all waits are bounded.
@@ -53,7 +54,7 @@ struct __align__(1024) MlpSmem {
     uint8_t X2s[4 * kTile];             // bf16 X2     [4 hidden blocks][16 token rows x 128 B]
     uint8_t XB2s[4 * kTile];            // bf16 Xbar2
     uint8_t G1s[4 * kTile];             // bf16 g1
-    uint8_t G1Ls[4 * kTile];            // bf16 -t_{K-1} lr g1
+    uint8_t XKL[kTile];                 // bf16 -t_{K-1} lr XK [16 token rows x 128 B]
     uint8_t G2s[kTile];                 // bf16 g2 [16 token rows x 128 B (64 outputs)]
     uint8_t G2Ls[kTile];                // bf16 -t_{K-1} lr g2
     uint8_t M1s[kTile];                 // bf16 -M1, row i, cols j < 16
@@ -61,7 +62,7 @@ struct __align__(1024) MlpSmem {
     float Zt[TTT_KMAX][TTT_D];          // Z2, then Zbar2, as token rows
     float A2p[4][TTT_KMAX][TTT_KMAX];   // Xbar2 X2^T partial sums over the 4 hidden blocks
     float b2[TTT_D];
-    float b2part[4][TTT_D];
+    float b2part[8][TTT_D];
     float lr[kStages][TTT_KMAX];
     float te[TTT_KMAX];
     uint64_t full[kStages];
@@ -98,33 +99,32 @@ __device__ __forceinline__ float gelu(float x) {
     return 0.5f * x * (1.0f + tanh_fast(k * fmaf(c * x, x * x, x)));
 }
 
-// Mean and 1/sqrt(var + eps) of a 64-value row held 8 per lane by 8 lanes (Chan merges).
-__device__ __forceinline__ void row_stats8(const float (&v)[8], float eps, float& mu, float& rstd) {
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m += v[i];
-    m *= 0.125f;
+// Mean and 1/sqrt(var + eps) of a 64-value row held 4 per lane by 16 lanes (Chan merges).
+__device__ __forceinline__ void row_stats16(const float (&v)[4], float eps, float& mu, float& rstd) {
+    float m = 0.25f * ((v[0] + v[1]) + (v[2] + v[3]));
     float M2 = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) M2 = fmaf(v[i] - m, v[i] - m, M2);
+    for (int i = 0; i < 4; ++i) M2 = fmaf(v[i] - m, v[i] - m, M2);
 #pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
+    for (int off = 1; off < 16; off <<= 1) {
         const float mo = __shfl_xor_sync(0xffffffffu, m, off);
         const float M2o = __shfl_xor_sync(0xffffffffu, M2, off);
         const float dm = mo - m;
-        M2 = M2 + M2o + dm * dm * (4.0f * off);
+        M2 = M2 + M2o + dm * dm * (2.0f * off);
         m = 0.5f * (m + mo);
     }
     mu = m;
     rstd = rsqrtf(M2 * (1.0f / TTT_D) + eps);
 }
 
-__device__ __forceinline__ float sum8(float v) {
+__device__ __forceinline__ float sum16(float v) {
     v += __shfl_xor_sync(0xffffffffu, v, 1);
     v += __shfl_xor_sync(0xffffffffu, v, 2);
     v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
     return v;
 }
+
 
 // 4 consecutive bf16 of row r starting at column c (c % 4 == 0) -> floats
 __device__ __forceinline__ void ld4_bf16(const uint8_t* tile, int r, int c, float* out) {
@@ -242,14 +242,13 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     if (w == 0)
         for (int mm = 0; mm < kStages - 1 && mm < n_mb; ++mm) issue(mm, mm);
 
-    // row-phase geometry (warps 0..3): token row rr, features fa..fa+3 and fb..fb+3
-    const int rr = (tid >> 3) & 15, l8 = tid & 7;
-    const int fa = 4 * l8, fb = 32 + 4 * l8;
-    float lw[8], lb[8];
+    // row-phase geometry (all 8 warps): token row rr, features f4..f4+3 (16 lanes per row)
+    const int rr = tid >> 4, f4 = 4 * (tid & 15);
+    float lw[4], lb[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        lw[i] = a.ln_w[h * TTT_D + fa + i];     lb[i] = a.ln_b[h * TTT_D + fa + i];
-        lw[4 + i] = a.ln_w[h * TTT_D + fb + i]; lb[4 + i] = a.ln_b[h * TTT_D + fb + i];
+        lw[i] = a.ln_w[h * TTT_D + f4 + i];
+        lb[i] = a.ln_b[h * TTT_D + f4 + i];
     }
     const float tl = s.te[K - 1];
     const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row supplied by this lane
@@ -269,7 +268,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     const uint64_t dX2m = tc5::sdesc(smem_u32(&s.X2s[0]), kTile, 1024);     // X2^T, MN-major A
     const uint64_t dXB2k = tc5::sdesc(smem_u32(&s.XB2s[0]), 16, 1024);      // Xbar2, K-major B
     const uint64_t dG1m = tc5::sdesc(smem_u32(&s.G1s[0]), kTile, 1024);     // g1^T, MN-major A
-    const uint64_t dG1Lm = tc5::sdesc(smem_u32(&s.G1Ls[0]), kTile, 1024);   // (-t lr g1)^T, MN-major A
+    const uint64_t dXKLm = tc5::sdesc(smem_u32(&s.XKL[0]), kTile, 1024);    // -t lr XK, MN-major B
     const uint64_t dG2k = tc5::sdesc(smem_u32(&s.G2s[0]), 16, 1024);        // g2, K-major B
     const uint64_t dG2m = tc5::sdesc(smem_u32(&s.G2s[0]), 2048, 1024);      // g2^T, MN-major A (M = 64)
     const uint64_t dG2Lm = tc5::sdesc(smem_u32(&s.G2Ls[0]), kTile, 1024);   // -t lr g2, MN-major B
@@ -372,49 +371,42 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         }
         __syncthreads();
 
-        // (4) g2 = ln_fused_l2_bwd(Z2 + b2, XV - XK) on token rows (warps 0..3)
-        if (w < 4) {
-            float z[8], xk[8], xv[8];
+        // (4) g2 = ln_fused_l2_bwd(Z2 + b2, XV - XK) on token rows; also -t lr XK for W1's update
+        {
+            float z[4], xk[4], xv[4];
+            const float4 zz = *reinterpret_cast<const float4*>(&s.Zt[rr][f4]);
+            const float4 bb = *reinterpret_cast<const float4*>(&s.b2[f4]);
+            z[0] = zz.x + bb.x; z[1] = zz.y + bb.y; z[2] = zz.z + bb.z; z[3] = zz.w + bb.w;
+            ld4_bf16(xk_t, rr, f4, xk);
+            ld4_bf16(xv_t, rr, f4, xv);
+            float mu, rs;
+            row_stats16(z, eps, mu, rs);
+            float xh[4], qv[4], sq = 0.f, sqx = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                z[i] = s.Zt[rr][fa + i] + s.b2[fa + i];
-                z[4 + i] = s.Zt[rr][fb + i] + s.b2[fb + i];
-            }
-            ld4_bf16(xk_t, rr, fa, xk); ld4_bf16(xk_t, rr, fb, xk + 4);
-            ld4_bf16(xv_t, rr, fa, xv); ld4_bf16(xv_t, rr, fb, xv + 4);
-            float mu, rs;
-            row_stats8(z, eps, mu, rs);
-            float xh[8], qv[8], sq = 0.f, sqx = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
                 xh[i] = (z[i] - mu) * rs;
                 qv[i] = lw[i] * (fmaf(lw[i], xh[i], lb[i]) - (xv[i] - xk[i]));
                 sq += qv[i];
                 sqx = fmaf(qv[i], xh[i], sqx);
             }
-            sq = sum8(sq);
-            sqx = sum8(sqx);
+            sq = sum16(sq);
+            sqx = sum16(sqx);
             const float sc = (rr < Km) ? rs * (1.0f / TTT_D) : 0.f;
-            float g2[8];
+            float g2[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) g2[i] = fmaf(-xh[i], sqx, fmaf(static_cast<float>(TTT_D), qv[i], -sq)) * sc;
-            st4_bf16(&s.G2s[0], rr, fa, g2[0], g2[1], g2[2], g2[3]);
-            st4_bf16(&s.G2s[0], rr, fb, g2[4], g2[5], g2[6], g2[7]);
+            for (int i = 0; i < 4; ++i) g2[i] = fmaf(-xh[i], sqx, fmaf(static_cast<float>(TTT_D), qv[i], -sq)) * sc;
+            st4_bf16(&s.G2s[0], rr, f4, g2[0], g2[1], g2[2], g2[3]);
             const float ls = -tl * lr_s[rr];
-            st4_bf16(&s.G2Ls[0], rr, fa, ls * g2[0], ls * g2[1], ls * g2[2], ls * g2[3]);
-            st4_bf16(&s.G2Ls[0], rr, fb, ls * g2[4], ls * g2[5], ls * g2[6], ls * g2[7]);
-            // b2: sum over this warp's 4 token rows of lr g2
-            float bs[8];
+            st4_bf16(&s.G2Ls[0], rr, f4, ls * g2[0], ls * g2[1], ls * g2[2], ls * g2[3]);
+            st4_bf16(&s.XKL[0], rr, f4, ls * xk[0], ls * xk[1], ls * xk[2], ls * xk[3]);
+            // b2: sum over this warp's 2 token rows of lr g2
+            float bs[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 bs[i] = lr_s[rr] * g2[i];
-                bs[i] += __shfl_xor_sync(0xffffffffu, bs[i], 8);
                 bs[i] += __shfl_xor_sync(0xffffffffu, bs[i], 16);
             }
-            if (lane < 8) {
-                *reinterpret_cast<float4*>(&s.b2part[w][fa]) = make_float4(bs[0], bs[1], bs[2], bs[3]);
-                *reinterpret_cast<float4*>(&s.b2part[w][fb]) = make_float4(bs[4], bs[5], bs[6], bs[7]);
-            }
+            if (lane < 16) *reinterpret_cast<float4*>(&s.b2part[w][f4]) = make_float4(bs[0], bs[1], bs[2], bs[3]);
         }
         sync_operands();
 
@@ -437,12 +429,10 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             tc5::ld16(tc5::taddr(tm, my_lane, cG1 + 16 * mt), gr);
             tc5::wait_ld();
             uint8_t* gb = &s.G1s[(u >> 6) * kTile];
-            uint8_t* gl = &s.G1Ls[(u >> 6) * kTile];
 #pragma unroll
             for (int tt = 0; tt < 16; ++tt) {
                 const float gv = gr[tt] * dg[tt];
                 st_bf16(gb, swz(tt, u & 63), gv);
-                st_bf16(gl, swz(tt, u & 63), -tl * lr_s[tt] * gv);
                 b1sum = fmaf(lr_s[tt], gv, b1sum);
             }
         }
@@ -456,9 +446,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             if (full_mb) {
 #pragma unroll
                 for (int t2 = 0; t2 < 2; ++t2) {
-                    // W1^T += (-t lr g1)^T XK ;  W2 += X2^T (-t lr g2)
-                    tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1Lm, t2 * 2 * kTile),
-                                tc5::sdesc_add(dSm, st * 3 * kTile), idUp, 1);
+                    // W1^T += g1^T (-t lr XK) ;  W2 += X2^T (-t lr g2)
+                    tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1m, t2 * 2 * kTile), dXKLm, idUp, 1);
                     tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc_add(dX2m, t2 * 2 * kTile), dG2Lm, idUp, 1);
                 }
             }
@@ -528,25 +517,22 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         }
         __syncthreads();
 
-        // (10) out = XQ + LN(Zbar2 + b2) on token rows (warps 0..3)
-        if (w < 4) {
-            float z[8], xq[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                z[i] = s.Zt[rr][fa + i] + s.b2[fa + i];
-                z[4 + i] = s.Zt[rr][fb + i] + s.b2[fb + i];
-            }
-            ld4_bf16(xq_t, rr, fa, xq); ld4_bf16(xq_t, rr, fb, xq + 4);
+        // (10) out = XQ + LN(Zbar2 + b2) on token rows
+        {
+            float z[4], xq[4];
+            const float4 zz = *reinterpret_cast<const float4*>(&s.Zt[rr][f4]);
+            const float4 bb = *reinterpret_cast<const float4*>(&s.b2[f4]);
+            z[0] = zz.x + bb.x; z[1] = zz.y + bb.y; z[2] = zz.z + bb.z; z[3] = zz.w + bb.w;
+            ld4_bf16(xq_t, rr, f4, xq);
             float mu, rs;
-            row_stats8(z, eps, mu, rs);
+            row_stats16(z, eps, mu, rs);
             if (rr < Km) {
-                float o[8];
+                float o[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) o[i] = xq[i] + fmaf(lw[i], (z[i] - mu) * rs, lb[i]);
+                for (int i = 0; i < 4; ++i) o[i] = xq[i] + fmaf(lw[i], (z[i] - mu) * rs, lb[i]);
                 __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
                                      (static_cast<long long>(chain) * a.L + static_cast<long long>(m) * K + rr) * TTT_D;
-                *reinterpret_cast<uint2*>(out + fa) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-                *reinterpret_cast<uint2*>(out + fb) = make_uint2(pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+                *reinterpret_cast<uint2*>(out + f4) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
             }
         }
         __syncthreads();
@@ -554,7 +540,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         // (12) new state: b2, and the bf16 shadows of the updated masters
         if (full_mb) {
             if (tid < TTT_D)
-                s.b2[tid] -= tl * (s.b2part[0][tid] + s.b2part[1][tid] + s.b2part[2][tid] + s.b2part[3][tid]);
+                s.b2[tid] -= tl * (((s.b2part[0][tid] + s.b2part[1][tid]) + (s.b2part[2][tid] + s.b2part[3][tid])) +
+                                   ((s.b2part[4][tid] + s.b2part[5][tid]) + (s.b2part[6][tid] + s.b2part[7][tid])));
             const int r = u & 127;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
