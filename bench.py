@@ -13,7 +13,9 @@ Multi-GPU (torchrun, one rank per GPU): every rank runs the same workload on its
 chains are independent; there is no exchange), `value` counts all ranks' tokens over the
 slowest rank's device time ("scaling": "weak").
 
-The JSON line also carries: `e2e` (the same call from pinned HOST buffers with the copies timed),
+The JSON line also carries: `e2e` (the same scan through the host-buffer entry point
+ttt_linear_forward_host from pinned HOST buffers, every input copied in and every result copied
+out inside the timed region, the batch pipelined in chunks),
 `roofline` (the scan kernel's algorithmic bytes / its CUDA-event time vs the measured HBM copy
 bandwidth), `cpu_baseline` (the CPU oracle on a bounded sample, rank 0 at N=1), `clocks`
 (NVML samples taken during the timed region) and `rows` (the TTT-MLP prefill and the decode
@@ -257,25 +259,30 @@ def bench_linear(args, world, rank, local, peaks):
     achieved = nbytes / (ms / 1e3) / 1e9
     traffic = kernel_traffic("linear_tc.cu", "linear_tc_kernel@1b_B8_H32_L8200") if L == 8200 else None
 
-    # end to end through the public call from pinned host buffers
-    host_in = {n: t.cpu().pin_memory() for n, t in (("XQ", XQ), ("XK", XK), ("XV", XV), ("lr", lr))}
-    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in (("out", out), ("W", Wl), ("b", bl))}
-    dev_in = {n: torch.empty_like(t, device="cuda") for n, t in host_in.items()}
+    # end to end through the public host-buffer call (ttt_linear_forward_host) from pinned host
+    # buffers: every step copies all inputs in and all results out, inside the timed region
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    host_in = {"XQ": pin(XQ), "XK": pin(XK), "XV": pin(XV), "lr": pin(lr), "W0": pin(W0), "b0": pin(b0),
+               "ln_w": pin(lnw), "ln_b": pin(lnb)}
+    host_out = {"out": torch.empty(XQ.shape, dtype=XQ.dtype, pin_memory=True),
+                "W_last": torch.empty(Wl.shape, pin_memory=True), "b_last": torch.empty(bl.shape, pin_memory=True),
+                "W_grad_tail": torch.empty(Wg.shape, pin_memory=True),
+                "b_grad_tail": torch.empty(bg.shape, pin_memory=True)}
+    ws = torch.empty(ttt.ttt_linear_host_workspace_bytes(B, H, L, w.K, XQ.dtype, args.e2e_chunk),
+                     dtype=torch.uint8, device="cuda")
 
     def e2e_step():
-        for n in dev_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        ttt.ttt_linear_forward(dev_in["XQ"], dev_in["XK"], dev_in["XV"], dev_in["lr"], W0, b0, lnw, lnb,
-                               mini_batch=w.K, eps=w.eps, out=out, W_last=Wl, b_last=bl, W_grad_tail=Wg,
-                               b_grad_tail=bg, tail_grads=True)
-        host_out["out"].copy_(out, non_blocking=True)
-        host_out["W"].copy_(Wl, non_blocking=True)
-        host_out["b"].copy_(bl, non_blocking=True)
+        ttt.ttt_linear_forward_host(host_in["XQ"], host_in["XK"], host_in["XV"], host_in["lr"], host_in["W0"],
+                                    host_in["b0"], host_in["ln_w"], host_in["ln_b"], mini_batch=w.K, eps=w.eps,
+                                    out=host_out["out"], W_last=host_out["W_last"], b_last=host_out["b_last"],
+                                    W_grad_tail=host_out["W_grad_tail"], b_grad_tail=host_out["b_grad_tail"],
+                                    tail_grads=True, chunk_batches=args.e2e_chunk, workspace=ws)
 
     e2e_K = max(3, min(args.steps, 10))
     e2e_ms = time_steps(e2e_step, e2e_K, 2, world)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    del ws
 
     line = {
         "metric": "TTT layer tokens/sec (1B shapes, B200) and % of per-layer roofline",
@@ -295,7 +302,8 @@ def bench_linear(args, world, rank, local, peaks):
                      "tensor_tflops": round(linear_flops(B, H, L) / (ms / 1e3) / 1e12, 2),
                      "tensor_frac_of_bf16_peak": round(linear_flops(B, H, L) / (ms / 1e3) / 1e12 / tf_burst, 4)},
         "e2e": {"value": round(world * tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": "ttt_linear_forward_host", "chunk_batches": args.e2e_chunk},
         "clocks": clk.summary(),
     }
     return line
@@ -446,6 +454,8 @@ def main():
     ap.add_argument("--rows", default="linear,mlp,decode",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-chunk", type=int, default=1,
+                    help="batch rows per chunk of the host-buffer (e2e) call")
     ap.add_argument("--seq-len", type=int, default=8200,
                     help="profiling aid: sequence length of the TTT-Linear workload (the headline is 8200)")
     ap.add_argument("--no-headline", action="store_true",

@@ -12,7 +12,7 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers into memory the caller owns (allocated by the
- *    caller, e.g. PyTorch).  The library allocates no device memory and keeps no state across
+ *    caller, e.g. PyTorch) -- except in ttt_linear_forward_host, whose tensors are HOST buffers.  The library allocates no device memory and keeps no state across
  *    calls except a thread-local last-error message and one device status word per device.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the legacy
  *    default stream).  No call synchronises the stream, except ttt_device_status().
@@ -81,7 +81,8 @@ int ttt_device_status(void* stream, unsigned int* status, int clear);
  * far above any healthy wait); < 0: zero polls, so every bounded wait gives up at once.  This
  * exercises the TTT_ERR_TIMEOUT path without faulting or hanging the GPU: the kernel raises
  * the status bit, waits (with the default bound) for its own copies in flight and returns.
- * Only the bf16 tensor-core prefill kernel has such waits.  Host-only; returns TTT_OK.
+ * The tensor-core TTT-Linear and TTT-MLP prefill kernels and the decode kernel have such waits.
+ * Host-only; returns TTT_OK.
  */
 int ttt_set_wait_limit(long long polls);
 
@@ -130,6 +131,46 @@ int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const flo
                        int H, long long L, int d, int mini_batch, float eps, int dtype,
                        unsigned int flags, void* out, float* W_last, float* b_last,
                        float* W_grad_tail, float* b_grad_tail, void* stream);
+
+/*
+ * ttt_linear_host_workspace_bytes -- size in bytes of the device workspace that
+ * ttt_linear_forward_host needs for these sizes: the per-head parameters plus two staging sets
+ * (inputs and outputs of `chunk_batches` batch rows each, tail-grad room included).
+ * Same size rules as ttt_linear_forward; 1 <= chunk_batches <= B; w0_batch_stride 0 or H*d*d.
+ * Host-only.  Returns the byte count (> 0) or a negative TTT_ERR_* code.
+ * (No counterpart on the pages: the walkthrough's tensors are already on the device.)
+ */
+long long ttt_linear_host_workspace_bytes(int B, int H, long long L, int d, int mini_batch, int dtype,
+                                          int chunk_batches, long long w0_batch_stride);
+
+/*
+ * ttt_linear_forward_host -- ttt_linear_forward on HOST buffers: the same scan, the same
+ * arguments and results, except that
+ *   - every tensor argument (XQ, XK, XV, lr, token_eta, W0, b0, ln_w, ln_b and the outputs out,
+ *     W_last, b_last, W_grad_tail, b_grad_tail) is a HOST pointer; page-locked (pinned) memory
+ *     lets the copies run asynchronously and overlap;
+ *   - workspace is a caller-owned DEVICE buffer of at least ttt_linear_host_workspace_bytes()
+ *     bytes (same B, H, L, d, mini_batch, dtype, chunk_batches, w0_batch_stride), 256-byte
+ *     aligned; its contents on entry are irrelevant and on return undefined.
+ * The batch runs in chunks of chunk_batches batch rows (the last may be shorter): the
+ * host-to-device copies of a chunk run on a copy stream owned by the library while the chunk
+ * before it computes and its results return on `stream`, so both copy directions and the
+ * kernels overlap.  The results equal ttt_linear_forward's on the same values, bit for bit.
+ * Asynchronous on `stream`: on return everything is enqueued; the host buffers must stay valid
+ * and unchanged, and the workspace unused by anyone else, until `stream` passes this point.
+ * The library creates, once per device, one non-blocking copy stream and five events (never
+ * freed) and allocates no device memory; concurrent calls are serialised while they enqueue.
+ * (No counterpart on the pages: the walkthrough's tensors are already on the device.)
+ * Errors as ttt_linear_forward, plus TTT_ERR_ARG for a missing or too small workspace or a bad
+ * chunk_batches, TTT_ERR_ALIGN for a misaligned workspace.
+ */
+int ttt_linear_forward_host(const void* XQ, const void* XK, const void* XV, const float* lr,
+                            const float* token_eta, const float* W0, const float* b0,
+                            long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                            long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                            void* out, float* W_last, float* b_last, float* W_grad_tail,
+                            float* b_grad_tail, void* workspace, long long workspace_bytes,
+                            int chunk_batches, void* stream);
 
 /*
  * ttt_mlp_forward -- TTT-MLP prefill ([readme]: the hidden state is a two-layer MLP;

@@ -30,7 +30,8 @@ TTT_FLAG_FP32_COMPUTE = 1
 TTT_STATUS_TIMEOUT = 1
 
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
-           "ttt_set_wait_limit", "ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step")
+           "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_host_workspace_bytes",
+           "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step")
 
 
 class TTTError(RuntimeError):
@@ -61,12 +62,16 @@ def lib():
         L.ttt_set_wait_limit.argtypes = [ll]
         L.ttt_linear_forward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
                                          vp, fp, fp, fp, fp, vp]
+        L.ttt_linear_host_workspace_bytes.argtypes = [i, i, ll, i, i, i, i, ll]
+        L.ttt_linear_host_workspace_bytes.restype = ll
+        L.ttt_linear_forward_host.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
+                                              vp, fp, fp, fp, fp, vp, ll, i, vp]
         L.ttt_mlp_forward.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, i, f, i,
                                       u, vp, fp, fp, fp, fp, vp]
         L.ttt_linear_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f, i,
                                              vp, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
-                     "ttt_mlp_forward", "ttt_linear_decode_step"):
+                     "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -160,6 +165,79 @@ def ttt_linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16,
                                   H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
                                   eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last),
                                   _ptr(W_grad_tail), _ptr(b_grad_tail), _stream(stream))
+    _check(rc)
+    if tail_grads:
+        return out, W_last, b_last, W_grad_tail, b_grad_tail
+    return out, W_last, b_last
+
+
+def _need_host(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor for the host-buffer entry point")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def ttt_linear_host_workspace_bytes(B: int, H: int, L: int, mini_batch: int = 16, dtype=torch.bfloat16,
+                                    chunk_batches: int = 1, per_chain_state: bool = False, d: int = 64) -> int:
+    """Bytes of device workspace that ttt_linear_forward_host needs (host-only)."""
+    code = TTT_BF16 if dtype == torch.bfloat16 else TTT_F32
+    n = lib().ttt_linear_host_workspace_bytes(B, H, L, d, mini_batch, code, chunk_batches,
+                                              H * d * d if per_chain_state else 0)
+    if n < 0:
+        _check(int(n))
+    return int(n)
+
+
+def ttt_linear_forward_host(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
+                            token_eta=None, out=None, W_last=None, b_last=None, W_grad_tail=None,
+                            b_grad_tail=None, tail_grads: bool = False, flags: int = 0, chunk_batches: int = 1,
+                            workspace=None, stream=None):
+    """ttt_linear_forward on HOST tensors (pin them for overlap): the batch streams through the
+    GPU in chunks of `chunk_batches` batch rows, copies in both directions overlapping the scan.
+    `workspace`: a CUDA uint8 tensor of at least ttt_linear_host_workspace_bytes(...) bytes, or
+    None (allocated here).  Outputs are host tensors (pinned when allocated here).
+    Asynchronous on `stream`: synchronise before reading the outputs.
+    Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail)."""
+    _need_host(XQ, "XQ")
+    B, H, L, d = XQ.shape
+    dt = XQ.dtype
+    for n, t in (("XK", XK), ("XV", XV)):
+        _need_host(t, n, dt, XQ.shape)
+    _need_host(lr, "lr", torch.float32, (B, H, L))
+    per_chain = W0.dim() == 4
+    _need_host(W0, "W0", torch.float32, (B, H, d, d) if per_chain else (H, d, d))
+    _need_host(b0, "b0", torch.float32, (B, H, d) if per_chain else (H, d))
+    _need_host(ln_w, "ln_w", torch.float32, (H, d))
+    _need_host(ln_b, "ln_b", torch.float32, (H, d))
+    if token_eta is not None:
+        _need_host(token_eta, "token_eta", torch.float32, (mini_batch,))
+
+    def host(shape, dtype):
+        return torch.empty(shape, dtype=dtype, pin_memory=True)
+
+    out = host(XQ.shape, dt) if out is None else _need_host(out, "out", dt, XQ.shape)
+    W_last = host((B, H, d, d), torch.float32) if W_last is None else _need_host(W_last, "W_last", torch.float32, (B, H, d, d))
+    b_last = host((B, H, d), torch.float32) if b_last is None else _need_host(b_last, "b_last", torch.float32, (B, H, d))
+    if tail_grads:
+        W_grad_tail = host((B, H, d, d), torch.float32) if W_grad_tail is None else W_grad_tail
+        b_grad_tail = host((B, H, d), torch.float32) if b_grad_tail is None else b_grad_tail
+    need = ttt_linear_host_workspace_bytes(B, H, L, mini_batch, dt, chunk_batches, per_chain, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    _need(workspace, "workspace", torch.uint8)
+    rc = lib().ttt_linear_forward_host(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
+                                       H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
+                                       eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last),
+                                       _ptr(W_grad_tail), _ptr(b_grad_tail), _ptr(workspace), workspace.numel(),
+                                       chunk_batches, _stream(stream))
     _check(rc)
     if tail_grads:
         return out, W_last, b_last, W_grad_tail, b_grad_tail

@@ -151,6 +151,107 @@ unsigned int* status_word() {
     }
     return ptrs[dev];
 }
+
+// The launch part of ttt_linear_forward, on validated device pointers: pick the kernel, build
+// its arguments (and tensor maps) and enqueue it on `st`.
+int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                   const float* W0, const float* b0, long long w0_chain_stride, const float* ln_w, const float* ln_b,
+                   int B, int H, long long L, int mini_batch, float eps, int dtype, unsigned int flags, void* out,
+                   float* W_last, float* b_last, float* W_grad_tail, float* b_grad_tail, cudaStream_t st) {
+    const long long chains = static_cast<long long>(B) * H;
+    int rc;
+    ttt::LinearArgs a{};
+    a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
+    a.W0 = W0; a.b0 = b0; a.w0_chain_stride = w0_chain_stride;
+    a.ln_w = ln_w; a.ln_b = ln_b; a.B = B; a.H = H; a.L = L; a.K = mini_batch;
+    a.n_full = L / mini_batch; a.rem = L % mini_batch; a.eps = eps;
+    a.out = out; a.W_last = W_last; a.b_last = b_last; a.W_grad_tail = W_grad_tail; a.b_grad_tail = b_grad_tail;
+    a.status = status_word();
+    a.wait_limit = wait_limit();
+
+    cudaError_t e;
+    if (L == 0) {
+        e = ttt::launch_linear_state_copy(a, st);
+    } else if (dtype == TTT_F32 || (flags & TTT_FLAG_FP32_COMPUTE)) {
+        e = ttt::launch_linear_simt(a, dtype, st);
+    } else {
+        ttt::LinearMaps maps;
+        if ((rc = encode_act_map(&maps.xq, XQ, chains, L, mini_batch, "XQ"))) return rc;
+        if ((rc = encode_act_map(&maps.xk, XK, chains, L, mini_batch, "XK"))) return rc;
+        if ((rc = encode_act_map(&maps.xv, XV, chains, L, mini_batch, "XV"))) return rc;
+        if ((rc = encode_act_map(&maps.out, out, chains, L, mini_batch, "out"))) return rc;
+        e = ttt::launch_linear_tc(a, maps, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward launch");
+    return ok();
+}
+
+// ---- host-buffer entry: one copy stream and a few events per device, created on first use ----
+struct HostCtx {
+    cudaStream_t copy = nullptr;
+    cudaEvent_t start = nullptr, in[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+};
+std::mutex g_host_mu;  // held while a host-buffer call enqueues (its events are shared per device)
+HostCtx g_host_ctx[256];
+
+int host_ctx(HostCtx** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 256) return fail(TTT_ERR_CUDA, "device index %d out of range", dev);
+    HostCtx& c = g_host_ctx[dev];
+    if (!c.copy) {
+        if ((e = cudaStreamCreateWithFlags(&c.copy, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "creating the copy stream");
+        cudaEvent_t* evs[5] = {&c.start, &c.in[0], &c.in[1], &c.freed[0], &c.freed[1]};
+        for (cudaEvent_t* ev : evs)
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(e, "creating an event");
+    }
+    *out = &c;
+    return TTT_OK;
+}
+
+size_t up256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// Byte offsets inside the workspace of ttt_linear_forward_host.
+struct HostLayout {
+    size_t lnw, lnb, te, w0, b0;               // shared parameters (w0, b0: per head, when shared)
+    size_t set;                                // offset of staging set 0; set 1 follows at set + set_bytes
+    size_t set_bytes;
+    size_t xq, xk, xv, lr, w0c, b0c, out, wl, bl, wg, bg;  // offsets inside a staging set
+    size_t total;
+};
+
+HostLayout host_layout(int H, long long L, int K, int dtype, int chunk_batches, bool per_chain) {
+    HostLayout y{};
+    const size_t cc = static_cast<size_t>(chunk_batches) * H;  // chains per chunk
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t act = cc * static_cast<size_t>(L) * kD * esz;
+    const size_t st = static_cast<size_t>(kD) * kD * 4, sb = static_cast<size_t>(kD) * 4;
+    size_t o = 0;
+    y.lnw = o; o += up256(static_cast<size_t>(H) * sb);
+    y.lnb = o; o += up256(static_cast<size_t>(H) * sb);
+    y.te = o; o += up256(static_cast<size_t>(K) * 4);
+    y.w0 = o; o += per_chain ? 0 : up256(static_cast<size_t>(H) * st);
+    y.b0 = o; o += per_chain ? 0 : up256(static_cast<size_t>(H) * sb);
+    y.set = o;
+    size_t q = 0;
+    y.xq = q; q += up256(act);
+    y.xk = q; q += up256(act);
+    y.xv = q; q += up256(act);
+    y.lr = q; q += up256(cc * static_cast<size_t>(L) * 4);
+    y.w0c = q; q += per_chain ? up256(cc * st) : 0;
+    y.b0c = q; q += per_chain ? up256(cc * sb) : 0;
+    y.out = q; q += up256(act);
+    y.wl = q; q += up256(cc * st);
+    y.bl = q; q += up256(cc * sb);
+    y.wg = q; q += up256(cc * st);
+    y.bg = q; q += up256(cc * sb);
+    y.set_bytes = q;
+    y.total = o + 2 * q;
+    return y;
+}
 }  // namespace
 
 extern "C" {
@@ -240,30 +341,124 @@ int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const flo
     rc = check_aliasing(in, 9, outs, 5, same_ok, 2);
     if (rc) return rc;
 
-    ttt::LinearArgs a{};
-    a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
-    a.W0 = W0; a.b0 = b0; a.w0_chain_stride = w0_batch_stride ? per_head : 0;
-    a.ln_w = ln_w; a.ln_b = ln_b; a.B = B; a.H = H; a.L = L; a.K = mini_batch;
-    a.n_full = L / mini_batch; a.rem = L % mini_batch; a.eps = eps;
-    a.out = out; a.W_last = W_last; a.b_last = b_last; a.W_grad_tail = W_grad_tail; a.b_grad_tail = b_grad_tail;
-    a.status = status_word();
-    a.wait_limit = wait_limit();
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return enqueue_linear(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride ? per_head : 0, ln_w, ln_b, B, H, L,
+                          mini_batch, eps, dtype, flags, out, W_last, b_last, W_grad_tail, b_grad_tail,
+                          static_cast<cudaStream_t>(stream));
+}
 
-    cudaError_t e;
-    if (L == 0) {
-        e = ttt::launch_linear_state_copy(a, st);
-    } else if (dtype == TTT_F32 || (flags & TTT_FLAG_FP32_COMPUTE)) {
-        e = ttt::launch_linear_simt(a, dtype, st);
-    } else {
-        ttt::LinearMaps maps;
-        if ((rc = encode_act_map(&maps.xq, XQ, chains, L, mini_batch, "XQ"))) return rc;
-        if ((rc = encode_act_map(&maps.xk, XK, chains, L, mini_batch, "XK"))) return rc;
-        if ((rc = encode_act_map(&maps.xv, XV, chains, L, mini_batch, "XV"))) return rc;
-        if ((rc = encode_act_map(&maps.out, out, chains, L, mini_batch, "out"))) return rc;
-        e = ttt::launch_linear_tc(a, maps, st);
+long long ttt_linear_host_workspace_bytes(int B, int H, long long L, int d, int mini_batch, int dtype,
+                                          int chunk_batches, long long w0_batch_stride) {
+    int rc = check_common(B, H, L, d, mini_batch, 1e-6f, dtype, 0);
+    if (rc) return rc;
+    if (chunk_batches < 1 || chunk_batches > B)
+        return fail(TTT_ERR_ARG, "chunk_batches must be in [1, B] (got %d, B = %d)", chunk_batches, B);
+    if (w0_batch_stride != 0 && w0_batch_stride != static_cast<long long>(H) * kD * kD)
+        return fail(TTT_ERR_ARG, "w0_batch_stride must be 0 or H*d*d (got %lld)", w0_batch_stride);
+    ok();
+    return static_cast<long long>(host_layout(H, L, mini_batch, dtype, chunk_batches, w0_batch_stride != 0).total);
+}
+
+int ttt_linear_forward_host(const void* XQ, const void* XK, const void* XV, const float* lr,
+                            const float* token_eta, const float* W0, const float* b0,
+                            long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                            long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                            void* out, float* W_last, float* b_last, float* W_grad_tail,
+                            float* b_grad_tail, void* workspace, long long workspace_bytes,
+                            int chunk_batches, void* stream) {
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
+    if (rc) return rc;
+    const long long per_head = static_cast<long long>(kD) * kD;
+    const bool per_chain = w0_batch_stride != 0;
+    if (per_chain && w0_batch_stride != H * per_head)
+        return fail(TTT_ERR_ARG, "w0_batch_stride must be 0 or H*d*d (got %lld)", w0_batch_stride);
+    if (!W0 || !b0 || !ln_w || !ln_b || !W_last || !b_last)
+        return fail(TTT_ERR_ARG, "W0, b0, ln_w, ln_b, W_last and b_last must be non-null");
+    if (L > 0 && (!XQ || !XK || !XV || !lr || !out))
+        return fail(TTT_ERR_ARG, "XQ, XK, XV, lr and out must be non-null when L > 0");
+    if (chunk_batches < 1 || chunk_batches > B)
+        return fail(TTT_ERR_ARG, "chunk_batches must be in [1, B] (got %d, B = %d)", chunk_batches, B);
+    if (!workspace) return fail(TTT_ERR_ARG, "workspace must be non-null");
+    if (!aligned(workspace, 256)) return fail(TTT_ERR_ALIGN, "workspace must be 256-byte aligned");
+    const HostLayout y = host_layout(H, L, mini_batch, dtype, chunk_batches, per_chain);
+    if (workspace_bytes < static_cast<long long>(y.total))
+        return fail(TTT_ERR_ARG, "workspace too small: %lld bytes, %lld needed", workspace_bytes,
+                    static_cast<long long>(y.total));
+    const long long chains = static_cast<long long>(B) * H;
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t act = static_cast<size_t>(chains) * L * kD * esz;
+    const long long wrows = per_chain ? chains : H;
+    Span in[] = {{"XQ", XQ, act}, {"XK", XK, act}, {"XV", XV, act}, {"lr", lr, static_cast<size_t>(chains * L) * 4},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
+                 {"W0", W0, static_cast<size_t>(wrows * per_head) * 4}, {"b0", b0, static_cast<size_t>(wrows * kD) * 4},
+                 {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    Span outs[] = {{"out", out, act}, {"W_last", W_last, static_cast<size_t>(chains * per_head) * 4},
+                   {"b_last", b_last, static_cast<size_t>(chains * kD) * 4},
+                   {"W_grad_tail", W_grad_tail, static_cast<size_t>(chains * per_head) * 4},
+                   {"b_grad_tail", b_grad_tail, static_cast<size_t>(chains * kD) * 4}};
+    const int same_ok[2][2] = {{1, 5}, {2, 6}};
+    rc = check_aliasing(in, 9, outs, 5, same_ok, 2);
+    if (rc) return rc;
+
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    HostCtx* c = nullptr;
+    if ((rc = host_ctx(&c))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    const auto H2D = cudaMemcpyHostToDevice;
+    const auto D2H = cudaMemcpyDeviceToHost;
+    cudaError_t e = cudaEventRecord(c->start, st);  // the workspace is free once earlier work on st is done
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(c->copy, c->start, 0);
+    // shared parameters
+    const size_t hb = static_cast<size_t>(H) * kD * 4;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + y.lnw, ln_w, hb, H2D, c->copy);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + y.lnb, ln_b, hb, H2D, c->copy);
+    if (e == cudaSuccess && token_eta) e = cudaMemcpyAsync(ws + y.te, token_eta, static_cast<size_t>(mini_batch) * 4, H2D, c->copy);
+    if (e == cudaSuccess && !per_chain) e = cudaMemcpyAsync(ws + y.w0, W0, static_cast<size_t>(H) * per_head * 4, H2D, c->copy);
+    if (e == cudaSuccess && !per_chain) e = cudaMemcpyAsync(ws + y.b0, b0, hb, H2D, c->copy);
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward_host: parameters");
+
+    const int n_chunks = (B + chunk_batches - 1) / chunk_batches;
+    for (int ci = 0; ci < n_chunks; ++ci) {
+        const int slot = ci & 1;
+        const int bfirst = ci * chunk_batches;
+        const int bc = (B - bfirst < chunk_batches) ? B - bfirst : chunk_batches;
+        const size_t cc = static_cast<size_t>(bc) * H;                       // chains in this chunk
+        const size_t c0 = static_cast<size_t>(bfirst) * H;                   // first chain
+        const size_t a_off = c0 * static_cast<size_t>(L) * kD * esz, a_n = cc * static_cast<size_t>(L) * kD * esz;
+        const size_t l_off = c0 * static_cast<size_t>(L) * 4, l_n = cc * static_cast<size_t>(L) * 4;
+        const size_t s_off = c0 * per_head * 4, s_n = cc * per_head * 4;
+        const size_t v_off = c0 * kD * 4, v_n = cc * kD * 4;
+        char* set = ws + y.set + slot * y.set_bytes;
+        // inputs of this chunk (once the kernel two chunks back has finished reading the set)
+        if (ci >= 2) e = cudaStreamWaitEvent(c->copy, c->freed[slot], 0);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.xq, static_cast<const char*>(XQ) + a_off, a_n, H2D, c->copy);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.xk, static_cast<const char*>(XK) + a_off, a_n, H2D, c->copy);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.xv, static_cast<const char*>(XV) + a_off, a_n, H2D, c->copy);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.lr, reinterpret_cast<const char*>(lr) + l_off, l_n, H2D, c->copy);
+        if (e == cudaSuccess && per_chain) e = cudaMemcpyAsync(set + y.w0c, reinterpret_cast<const char*>(W0) + s_off, s_n, H2D, c->copy);
+        if (e == cudaSuccess && per_chain) e = cudaMemcpyAsync(set + y.b0c, reinterpret_cast<const char*>(b0) + v_off, v_n, H2D, c->copy);
+        if (e == cudaSuccess) e = cudaEventRecord(c->in[slot], c->copy);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, c->in[slot], 0);
+        if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward_host: inputs");
+        // the scan of this chunk
+        rc = enqueue_linear(set + y.xq, set + y.xk, set + y.xv, reinterpret_cast<const float*>(set + y.lr),
+                            token_eta ? reinterpret_cast<const float*>(ws + y.te) : nullptr,
+                            reinterpret_cast<const float*>(per_chain ? set + y.w0c : ws + y.w0),
+                            reinterpret_cast<const float*>(per_chain ? set + y.b0c : ws + y.b0), per_chain ? per_head : 0,
+                            reinterpret_cast<const float*>(ws + y.lnw), reinterpret_cast<const float*>(ws + y.lnb), bc, H,
+                            L, mini_batch, eps, dtype, flags, set + y.out, reinterpret_cast<float*>(set + y.wl),
+                            reinterpret_cast<float*>(set + y.bl), W_grad_tail ? reinterpret_cast<float*>(set + y.wg) : nullptr,
+                            b_grad_tail ? reinterpret_cast<float*>(set + y.bg) : nullptr, st);
+        if (rc) return rc;
+        e = cudaEventRecord(c->freed[slot], st);
+        // results of this chunk
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(static_cast<char*>(out) + a_off, set + y.out, a_n, D2H, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(reinterpret_cast<char*>(W_last) + s_off, set + y.wl, s_n, D2H, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(reinterpret_cast<char*>(b_last) + v_off, set + y.bl, v_n, D2H, st);
+        if (e == cudaSuccess && W_grad_tail) e = cudaMemcpyAsync(reinterpret_cast<char*>(W_grad_tail) + s_off, set + y.wg, s_n, D2H, st);
+        if (e == cudaSuccess && b_grad_tail) e = cudaMemcpyAsync(reinterpret_cast<char*>(b_grad_tail) + v_off, set + y.bg, v_n, D2H, st);
+        if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward_host: outputs");
     }
-    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward launch");
     return ok();
 }
 

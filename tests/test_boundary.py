@@ -19,8 +19,9 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for f in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_partition",
-              "ttt_error_string", "ttt_last_error_message", "ttt_device_status", "ttt_set_wait_limit"):
+    for f in ("ttt_linear_forward", "ttt_linear_forward_host", "ttt_linear_host_workspace_bytes",
+              "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_partition", "ttt_error_string",
+              "ttt_last_error_message", "ttt_device_status", "ttt_set_wait_limit"):
         assert f in names
 
 
@@ -126,3 +127,46 @@ def test_binding_refuses_cpu_tensors(libttt):
     with pytest.raises(ValueError, match="CUDA"):
         libttt.ttt_linear_forward(x, x, x, torch.zeros(1, 1, 16), torch.zeros(1, 64, 64), torch.zeros(1, 64),
                                   torch.ones(1, 64), torch.zeros(1, 64))
+
+
+# --- the host-buffer entry point: sizing and rejections (host-only; nothing is copied) ---------
+def _host(lib, **kw):
+    args = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W0=5 * A, b0=6 * A, stride=0, lnw=7 * A,
+                lnb=8 * A, B=2, H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, flags=0, out=9 * A,
+                Wl=10 * A, bl=11 * A, Wg=None, bg=None, ws=64 * A, wsb=1 << 40, chunk=1)
+    args.update(kw)
+    return lib.ttt_linear_forward_host(args["XQ"], args["XK"], args["XV"], args["lr"], args["te"], args["W0"],
+                                       args["b0"], args["stride"], args["lnw"], args["lnb"], args["B"], args["H"],
+                                       args["L"], args["d"], args["K"], args["eps"], args["dtype"], args["flags"],
+                                       args["out"], args["Wl"], args["bl"], args["Wg"], args["bg"], args["ws"],
+                                       args["wsb"], args["chunk"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), -1), (dict(ws=64 * A + 16), -2), (dict(wsb=1000), -1), (dict(chunk=0), -1),
+    (dict(chunk=3), -1), (dict(B=0), -1), (dict(XQ=None), -1), (dict(W0=None), -1), (dict(out=A), -3),
+    (dict(Wl=5 * A), -3), (dict(stride=5), -1), (dict(d=32), -6), (dict(K=17), -1), (dict(dtype=5), -1),
+])
+def test_linear_forward_host_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _host(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
+def test_host_workspace_bytes(libttt):
+    lib = libttt.lib()
+    n1 = lib.ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, 1, 1, 0)
+    n2 = lib.ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, 1, 2, 0)
+    n1f = lib.ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, 0, 1, 0)
+    npc = lib.ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, 1, 1, 32 * 64 * 64)
+    act = 32 * 8200 * 64 * 2  # one chunk's bf16 activations
+    assert 2 * 4 * act <= n1 < n2 < 2 * n1 + (1 << 20)
+    assert n1f > n1 and npc > n1
+    assert n1 % 256 == 0
+    # the binding reports the same number
+    import torch
+    assert libttt.ttt_linear_host_workspace_bytes(8, 32, 8200, 16, torch.bfloat16, 1) == n1
+    for args, code in (((8, 32, 8200, 64, 16, 1, 0, 0), -1), ((8, 32, 8200, 64, 16, 1, 9, 0), -1),
+                       ((8, 32, 8200, 32, 16, 1, 1, 0), -6), ((8, 32, 8200, 64, 16, 1, 1, 5), -1),
+                       ((8, 32, -1, 64, 16, 1, 1, 0), -1)):
+        assert lib.ttt_linear_host_workspace_bytes(*args) == code
