@@ -1,4 +1,5 @@
-// mlp_tc.cu -- TTT-MLP prefill on the 5th-generation tensor cores (tcgen05 + tensor memory).
+// mlp_tc.cu -- TTT-MLP prefill: fp32 masters in tensor memory, 5th-generation tensor-core
+// updates (tcgen05), warp-level MMAs for the small per-mini-batch products.
 //
 // The hidden state is the two-layer MLP f(x) = gelu(x W1 + b1) W2 + b2, d = 64 -> 256 -> 64
 // (ttt-lm-pytorch README: "TTT-MLP ... a two-layer MLP"; "代码连连看——TTT": "TTTMLP is two
@@ -11,21 +12,24 @@
 //
 // Design (one CTA of 8 warps per (batch, head) chain, the whole sequence on chip):
 //  * The fp32 masters W1^T (256 x 64) and W2 (256 x 64) live in tensor memory (hidden unit =
-//    lane, two 128-lane tiles each) and are updated by accumulating tcgen05 MMAs.  Each
-//    mini-batch refreshes their bf16 shadows in shared memory (128-byte swizzle), which are the
-//    operands of the forward MMAs: W1^T as K-major A of Z1^T | (XQ W1)^T, the W2 shadow as
-//    K-major A of (g2 W2^T)^T and, read MN-major, as the A operand W2^T of Z2^T and Zbar2^T.
-//  * Thread u of the CTA owns hidden unit u (its tensor-memory lane): GELU, GELU', the g1
-//    product and b1 are per-thread register work, written back in bf16 straight into the
-//    operand layouts of the next MMAs (X2 as K-major B and MN-major A, g1 and lr-scaled g1 as
-//    MN-major A).
+//    lane, two 128-lane tiles each, 256 columns) and take their rank-16 updates as accumulating
+//    tcgen05 MMAs: W1^T += g1^T (-t lr XK), W2 += X2^T (-t lr g2).  They are issued as soon as
+//    their operands exist and run while the warps compute the output path.  Afterwards the
+//    masters are read back (tcgen05.ld) into bf16 shadows in 128-byte-swizzled shared memory.
+//  * The per-mini-batch products involve 16 tokens, so they run as mma.sync m16n8k16 on all 8
+//    warps at once (a tcgen05 MMA needs M >= 64 and a commit/wait round trip per dependent
+//    step): warp w owns hidden units 32w..32w+31 of Z1, XQ W1, X2, g2 W2^T, g1, Zbar1, Xbar2,
+//    and outputs 8w..8w+7 of Z2 and Zbar2.  The W shadows are the B operands (ldmatrix, plain
+//    or transposed), the token tiles the A operands.
+//  * The accumulator layout of a warp's [16 tokens x 32 hidden] tiles is reused as operand
+//    layout without shared memory: as A of Xbar2 X2^T (k = hidden) directly, and as B of the
+//    same product (k = hidden, n = token) directly; g1 reaches the B operand of M1 g1 by
+//    movmatrix transposes.  X2, Xbar2 and g1 go to shared memory only where other warps or the
+//    tensor cores read them.
 //  * The two LayerNorms (loss gradient on Z2, output on Zbar2) run on token rows, 16 lanes per
-//    row (all 8 warps), after a transpose of the 64 x 16 accumulator through shared memory.
-//  * W1's update takes its lr scaling on the small operand: W1^T += g1^T (-t_{K-1} lr XK).
-//  * The 16 x 16 token-pair products XQ XK^T and Xbar2 X2^T are too small for tcgen05
-//    (M >= 64) and run as mma.sync m16n8k16 on the same shared-memory tiles.
-//  * One thread issues every tcgen05.mma and commits to one mbarrier; all waits are bounded.
-//    XQ, XK, XV tiles arrive by TMA (box {64, K}, 128-byte swizzle, no multicast) into a ring.
+//    row, after the warps' output slices meet in shared memory.
+//  * XQ, XK, XV tiles arrive by TMA (box {64, K}, 128-byte swizzle, no multicast) into a ring.
+//    One thread issues the tcgen05 MMAs and commits to one mbarrier; all waits are bounded.
 #include "tc5.cuh"
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
@@ -37,32 +41,26 @@ constexpr int kThreads = 256;
 constexpr int kHid = TTT_HIDDEN;
 constexpr int kStages = 3;
 constexpr int kTile = TTT_KMAX * 128;  // [16 rows x 128 bytes] bf16 tile
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;
 constexpr long long kDrainPolls = 1ll << 24;
-// tensor-memory columns
-constexpr uint32_t cW1 = 0;     // + 64 mt: W1^T tile mt (rows = hidden 128mt.., cols = input dim)
-constexpr uint32_t cW2 = 128;   // + 64 mt: W2 tile mt (rows = hidden, cols = output dim)
-constexpr uint32_t cZQ = 256;   // + 32 mt: Z1^T (cols 0..15) | (XQ W1)^T -> Zbar1^T (cols 16..31)
-constexpr uint32_t cG1 = 320;   // + 16 mt: (g2 W2^T)^T
-constexpr uint32_t cZ2 = 352;   // M = 64: Z2^T
-constexpr uint32_t cZB2 = 368;  // M = 64: Zbar2^T
+constexpr uint32_t cW1 = 0;    // + 64 mt: W1^T tile mt (rows = hidden 128mt.., cols = input dim)
+constexpr uint32_t cW2 = 128;  // + 64 mt: W2 tile mt (rows = hidden, cols = output dim)
 
 struct __align__(1024) MlpSmem {
-    uint8_t stage[kStages][3 * kTile];  // XK | XQ | XV (XK, XQ adjacent: the N = 32 B operand)
-    uint8_t W1s[2][128 * 128];          // bf16 W1^T shadow, K-major [tile][128 hidden rows x 128 B]
+    uint8_t stage[kStages][3 * kTile];  // XK | XQ | XV
+    uint8_t W1s[2][128 * 128];          // bf16 W1^T shadow [tile][128 hidden rows x 128 B (64 inputs)]
     uint8_t W2s[kHid * 128];            // bf16 W2 shadow [256 hidden rows x 128 B (64 outputs)]
     uint8_t X2s[4 * kTile];             // bf16 X2     [4 hidden blocks][16 token rows x 128 B]
     uint8_t XB2s[4 * kTile];            // bf16 Xbar2
     uint8_t G1s[4 * kTile];             // bf16 g1
-    uint8_t XKL[kTile];                 // bf16 -t_{K-1} lr XK [16 token rows x 128 B]
     uint8_t G2s[kTile];                 // bf16 g2 [16 token rows x 128 B (64 outputs)]
     uint8_t G2Ls[kTile];                // bf16 -t_{K-1} lr g2
-    uint8_t M1s[kTile];                 // bf16 -M1, row i, cols j < 16
-    uint8_t M2s[kTile];                 // bf16 -M2
-    float Zt[TTT_KMAX][TTT_D];          // Z2, then Zbar2, as token rows
-    float A2p[4][TTT_KMAX][TTT_KMAX];   // Xbar2 X2^T partial sums over the 4 hidden blocks
+    uint8_t XKL[kTile];                 // bf16 -t_{K-1} lr XK
+    float Zt[TTT_KMAX][TTT_D];          // Z2, then Zbar2, as token rows (b2 included)
+    float A2p[8][TTT_KMAX][TTT_KMAX];   // Xbar2 X2^T over each warp's hidden slice
+    float A2[TTT_KMAX][TTT_KMAX];       // their sum
     float b2[TTT_D];
-    float b2part[8][TTT_D];
+    float b2part[8][TTT_D];             // sum_j lr_j g2_j over each warp's two token rows
     float lr[kStages][TTT_KMAX];
     float te[TTT_KMAX];
     uint64_t full[kStages];
@@ -75,10 +73,6 @@ struct __align__(1024) MlpSmem {
 // byte offset of bf16 element (row r, col c < 64) in a [rows x 128 B] tile, 128-byte swizzle
 __device__ __forceinline__ uint32_t swz(int r, int c) {
     return static_cast<uint32_t>(r * 128 + ((((c >> 3) ^ (r & 7))) << 4) + ((c & 7) << 1));
-}
-
-__device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, float v) {
-    *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(v);
 }
 
 __device__ __forceinline__ float tanh_fast(float x) {
@@ -125,7 +119,6 @@ __device__ __forceinline__ float sum16(float v) {
     return v;
 }
 
-
 // 4 consecutive bf16 of row r starting at column c (c % 4 == 0) -> floats
 __device__ __forceinline__ void ld4_bf16(const uint8_t* tile, int r, int c, float* out) {
     const uint2 v = *reinterpret_cast<const uint2*>(tile + swz(r, c));
@@ -136,6 +129,37 @@ __device__ __forceinline__ void st4_bf16(uint8_t* tile, int r, int c, float a, f
     *reinterpret_cast<uint2*>(tile + swz(r, c)) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(d, e));
 }
 
+// [16 tokens x 32 hidden] slice of this warp: four m16n8 accumulator tiles (hidden 8nt + 2t + e,
+// rows g and g+8), written as bf16 pairs into a [4 blocks][16 x 128 B] token-row operand tile.
+__device__ __forceinline__ void store_slice(uint8_t* tiles, int w, int g, int t, const uint32_t (&p)[4][2]) {
+    uint8_t* blk = tiles + (w >> 1) * kTile;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const int c = 32 * (w & 1) + 8 * nt + 2 * t;
+        *reinterpret_cast<uint32_t*>(blk + swz(g, c)) = p[nt][0];
+        *reinterpret_cast<uint32_t*>(blk + swz(g + 8, c)) = p[nt][1];
+    }
+}
+
+// D[16 x 8] += A[16 x 256] B[256 x 8] with A a [4 blocks][16 x 128 B] token-row tile (X2 or Xbar2)
+// and B the W2 shadow's 8 output columns 8w.. (k = hidden rows, read transposed).  Two
+// accumulators (even and odd k-steps) halve the dependent chain.
+__device__ __forceinline__ void tokens_times_w2(float (&acc)[2][4], uint32_t a_tiles, uint32_t w2, int w, int lane,
+                                                int lrow, int lchunk) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {  // pairs of k-steps: hidden rows 32p .. 32p + 31
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(w2 + swz128(32 * p + lane, w), b0, b1, b2, b3);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int ks = 2 * p + hh;  // hidden 16 ks .. 16 ks + 15
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a_tiles + (ks >> 2) * kTile + swz128(lrow, 2 * (ks & 3) + lchunk), a0, a1, a2, a3);
+            mma_bf16_16816(acc[hh], a0, a1, a2, a3, hh ? b2 : b0, hh ? b3 : b1);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -143,8 +167,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int q = w & 3, mt = w >> 2;            // tensor-memory lane quarter and 128-lane tile
-    const int u = 128 * mt + 32 * q + lane;      // the hidden unit this thread owns
-    const int g = lane >> 2, t4 = lane & 3;
+    const int u = 128 * mt + 32 * q + lane;      // the hidden unit whose master rows this thread moves
+    const int g = lane >> 2, t = lane & 3;
     const int chain = blockIdx.x;
     const int h = chain % a.H;
     const int K = a.K;
@@ -169,15 +193,18 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     }
     for (int i = tid; i < kStages * 3 * kTile / 16; i += kThreads)
         reinterpret_cast<uint4*>(&s.stage[0][0])[i] = make_uint4(0, 0, 0, 0);  // rows >= K stay zero
-    for (int i = tid; i < 2 * kTile / 16; i += kThreads)
-        reinterpret_cast<uint4*>(&s.M1s[0])[i] = make_uint4(0, 0, 0, 0);
     if (tid < TTT_KMAX) s.te[tid] = a.token_eta ? (tid < K ? a.token_eta[tid] : 0.f) : 1.0f / (tid + 1);
     const long long w0off = a.w0_chain_stride ? static_cast<long long>(chain) * a.w0_chain_stride
                                               : static_cast<long long>(h) * TTT_D * kHid;
     const long long b1off = a.w0_chain_stride ? static_cast<long long>(chain) * kHid : static_cast<long long>(h) * kHid;
     const long long b2off = a.w0_chain_stride ? static_cast<long long>(chain) * TTT_D : static_cast<long long>(h) * TTT_D;
     if (tid < TTT_D) s.b2[tid] = a.b2_0[b2off + tid];
-    float b1r = a.b1_0[b1off + u];
+    // b1 at this thread's accumulator columns: hidden 32w + 8nt + 2t + e
+    float b1r[4][2];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) b1r[nt][e] = a.b1_0[b1off + 32 * w + 8 * nt + 2 * t + e];
     fence_proxy_async_smem();
     tc5::fence_before();
     __syncthreads();
@@ -253,43 +280,39 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     const float tl = s.te[K - 1];
     const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;  // ldmatrix row supplied by this lane
     const int lchunk = lane >> 4;
-    const uint32_t idZQ = tc5::idesc_bf16(128, 32, 0, 0);
-    const uint32_t idM64 = tc5::idesc_bf16(64, 16, 1, 0);
-    const uint32_t idG1 = tc5::idesc_bf16(128, 16, 0, 0);
-    const uint32_t idC1 = tc5::idesc_bf16(128, 16, 1, 0);
+    // -t_i on the lower triangle j <= i, zero above, at this lane's (i, j) positions of a 16x16
+    // accumulator: M[i][j] = c (A[i][j] + 1), c = tmask lr_j
+    float tmask[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = g + 8 * (e >> 1), j = 8 * nt + 2 * t + (e & 1);
+            tmask[nt][e] = (j <= i) ? -s.te[i] : 0.f;
+        }
     const uint32_t idUp = tc5::idesc_bf16(128, 64, 1, 1);
-
-    // Operand descriptors, built once: per MMA only a constant offset is added (the single
-    // issuing thread is otherwise the bottleneck of these small-N MMAs).
-    const uint64_t dW1k = tc5::sdesc(smem_u32(&s.W1s[0][0]), 16, 1024);     // W1^T, K-major A
-    const uint64_t dW2k = tc5::sdesc(smem_u32(&s.W2s[0]), 16, 1024);        // W2, K-major A
-    const uint64_t dW2m = tc5::sdesc(smem_u32(&s.W2s[0]), 2048, 1024);      // W2^T, MN-major A (M = 64)
-    const uint64_t dX2k = tc5::sdesc(smem_u32(&s.X2s[0]), 16, 1024);        // X2, K-major B
     const uint64_t dX2m = tc5::sdesc(smem_u32(&s.X2s[0]), kTile, 1024);     // X2^T, MN-major A
-    const uint64_t dXB2k = tc5::sdesc(smem_u32(&s.XB2s[0]), 16, 1024);      // Xbar2, K-major B
     const uint64_t dG1m = tc5::sdesc(smem_u32(&s.G1s[0]), kTile, 1024);     // g1^T, MN-major A
     const uint64_t dXKLm = tc5::sdesc(smem_u32(&s.XKL[0]), kTile, 1024);    // -t lr XK, MN-major B
-    const uint64_t dG2k = tc5::sdesc(smem_u32(&s.G2s[0]), 16, 1024);        // g2, K-major B
-    const uint64_t dG2m = tc5::sdesc(smem_u32(&s.G2s[0]), 2048, 1024);      // g2^T, MN-major A (M = 64)
     const uint64_t dG2Lm = tc5::sdesc(smem_u32(&s.G2Ls[0]), kTile, 1024);   // -t lr g2, MN-major B
-    const uint64_t dM1k = tc5::sdesc(smem_u32(&s.M1s[0]), 16, 1024);        // -M1, K-major B
-    const uint64_t dM2k = tc5::sdesc(smem_u32(&s.M2s[0]), 16, 1024);        // -M2, K-major B
-    const uint64_t dSk = tc5::sdesc(smem_u32(&s.stage[0][0]), 16, 1024);    // [XK; XQ] of stage 0, K-major B
-    const uint64_t dSm = tc5::sdesc(smem_u32(&s.stage[0][0]), kTile, 1024); // XK of stage 0, MN-major B
+    const uint32_t w1_s = smem_u32(&s.W1s[(32 * w) >> 7][0]);  // this warp's 32 hidden rows live in one tile
+    const int w1_row0 = (32 * w) & 127;
+    const uint32_t w2_s = smem_u32(&s.W2s[0]);
+    const uint32_t x2_s = smem_u32(&s.X2s[0]), xb2_s = smem_u32(&s.XB2s[0]), g2_s = smem_u32(&s.G2s[0]);
+
+    // M = c (A + 1) of a 16x16 accumulator pair, as the A operand of a 16x16x16 MMA
+    auto m_operand = [&](const float (&at)[2][4], const float* lr_s, uint32_t (&ma)[4]) {
+        const float2 l01 = *reinterpret_cast<const float2*>(&lr_s[2 * t]);
+        const float2 l89 = *reinterpret_cast<const float2*>(&lr_s[2 * t + 8]);
+        const float c00 = tmask[0][0] * l01.x, c01 = tmask[0][1] * l01.y, c02 = tmask[0][2] * l01.x, c03 = tmask[0][3] * l01.y;
+        const float c10 = tmask[1][0] * l89.x, c11 = tmask[1][1] * l89.y, c12 = tmask[1][2] * l89.x, c13 = tmask[1][3] * l89.y;
+        ma[0] = pack_bf16x2(fmaf(c00, at[0][0], c00), fmaf(c01, at[0][1], c01));
+        ma[1] = pack_bf16x2(fmaf(c02, at[0][2], c02), fmaf(c03, at[0][3], c03));
+        ma[2] = pack_bf16x2(fmaf(c10, at[1][0], c10), fmaf(c11, at[1][1], c11));
+        ma[3] = pack_bf16x2(fmaf(c12, at[1][2], c12), fmaf(c13, at[1][3], c13));
+    };
 
     uint32_t mpar = 0;  // phase parity of mma_bar
-    auto mma_wait = [&]() {
-        if (!mbar_wait_bounded(&s.mma_bar, mpar, wait_limit, a.status)) s.fail = 1;
-        mpar ^= 1;
-        tc5::fence_after();
-    };
-    auto sync_operands = [&]() {  // generic-proxy smem writes -> visible to the tensor cores
-        fence_proxy_async_smem();
-        tc5::fence_before();
-        __syncthreads();
-        tc5::fence_after();
-    };
-
     int st = 0;
     uint32_t par = 0;
     int m_stop = n_mb;  // first mini-batch whose loads may still be in flight (failure path)
@@ -302,81 +325,68 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         uint8_t* xq_t = &s.stage[st][kTile];
         const uint8_t* xv_t = &s.stage[st][2 * kTile];
         const float* lr_s = s.lr[st];
+        const uint32_t xk_s = smem_u32(xk_t), xq_s = smem_u32(xq_t);
 
-        // (1) Z1^T | (XQ W1)^T = W1^T [XK; XQ]^T
-        if (tid == 0) {
+        // (1) Z1 = XK W1 + b1, XQ W1 + b1 on this warp's 32 hidden units; XQ XK^T
+        float z1[4][4], zb1[4][4], at1[2][4];
 #pragma unroll
-            for (int t2 = 0; t2 < 2; ++t2)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc5::mma_ss(tm + cZQ + 32 * t2, tc5::sdesc_add(dW1k, t2 * 16384 + 32 * ks),
-                                tc5::sdesc_add(dSk, st * 3 * kTile + 32 * ks), idZQ, ks > 0);
-            tc5::commit(&s.mma_bar);
+        for (int nt = 0; nt < 4; ++nt) {
+            z1[nt][0] = z1[nt][2] = zb1[nt][0] = zb1[nt][2] = b1r[nt][0];
+            z1[nt][1] = z1[nt][3] = zb1[nt][1] = zb1[nt][3] = b1r[nt][1];
         }
-        // meanwhile: -M1 = -(eta * tril(XQ XK^T + 1)) into M1s (warp 4, mma.sync)
-        if (w == 4) {
-            float at[2][4] = {};
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                uint32_t k0, k1, k2, k3, q0, q1, q2, q3;
-                ldmatrix_x4(smem_u32(xk_t) + swz128(lrow, 2 * kk + lchunk), k0, k1, k2, k3);
-                ldmatrix_x4(smem_u32(xq_t) + swz128(lrow, 2 * kk + lchunk), q0, q1, q2, q3);
-                mma_bf16_16816(at[0], q0, q1, q2, q3, k0, k2);
-                mma_bf16_16816(at[1], q0, q1, q2, q3, k1, k3);
+        for (int e = 0; e < 4; ++e) at1[0][e] = at1[1][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t k0, k1, k2, k3, q0, q1, q2, q3;
+            ldmatrix_x4(xk_s + swz128(lrow, 2 * kk + lchunk), k0, k1, k2, k3);
+            ldmatrix_x4(xq_s + swz128(lrow, 2 * kk + lchunk), q0, q1, q2, q3);
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {  // hidden 32w + 16hb .. + 15: n-tiles 2hb, 2hb + 1
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(w1_s + swz128(w1_row0 + 16 * hb + lrow, 2 * kk + lchunk), b0, b1, b2, b3);
+                mma_bf16_16816(z1[2 * hb], k0, k1, k2, k3, b0, b2);
+                mma_bf16_16816(z1[2 * hb + 1], k0, k1, k2, k3, b1, b3);
+                mma_bf16_16816(zb1[2 * hb], q0, q1, q2, q3, b0, b2);
+                mma_bf16_16816(zb1[2 * hb + 1], q0, q1, q2, q3, b1, b3);
             }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = g + 8 * (e >> 1), j = 8 * nt + 2 * t4 + (e & 1);
-                    const float mv = (j <= i) ? s.te[i] * lr_s[j] * (at[nt][e] + 1.0f) : 0.f;
-                    st_bf16(&s.M1s[0], swz(i, j), -mv);
-                }
+            mma_bf16_16816(at1[0], q0, q1, q2, q3, k0, k2);  // tokens 0-7 of XK as B
+            mma_bf16_16816(at1[1], q0, q1, q2, q3, k1, k3);  // tokens 8-15
         }
-        mma_wait();
 
-        // (2) X2 = gelu(Z1 + b1), by hidden unit; keep gelu'(Z1 + b1)
-        float dg[16];
+        // (2) X2 = gelu(Z1), keep gelu'(Z1); X2 to shared memory (A of Z2, A of W2's update)
+        float dg[4][4];
+        uint32_t x2p[4][2];  // X2 as bf16 pairs: [n-tile][row g, row g + 8]
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) gelu2(z1[nt][e], y[e], dg[nt][e]);
+            x2p[nt][0] = pack_bf16x2(y[0], y[1]);
+            x2p[nt][1] = pack_bf16x2(y[2], y[3]);
+        }
+        store_slice(&s.X2s[0], w, g, t, x2p);
+        __syncthreads();
+
+        // (3) Z2 = X2 W2 + b2 on this warp's outputs 8w..8w+7 -> token rows in Zt
         {
-            float z1[16];
-            tc5::ld16(tc5::taddr(tm, my_lane, cZQ + 32 * mt), z1);
-            tc5::wait_ld();
-            uint8_t* xb = &s.X2s[(u >> 6) * kTile];
+            float z2[2][4];
+            const float2 bb = *reinterpret_cast<const float2*>(&s.b2[8 * w + 2 * t]);
+            z2[0][0] = z2[0][2] = bb.x;
+            z2[0][1] = z2[0][3] = bb.y;
 #pragma unroll
-            for (int tt = 0; tt < 16; ++tt) {
-                float y;
-                gelu2(z1[tt] + b1r, y, dg[tt]);
-                st_bf16(xb, swz(tt, u & 63), y);
-            }
-        }
-        sync_operands();
-
-        // (3) Z2^T = W2^T X2^T (M = 64 outputs, K = 256 hidden)
-        if (tid == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 16; ++ks)
-                tc5::mma_ss(tm + cZ2, tc5::sdesc_add(dW2m, 2048 * ks),
-                            tc5::sdesc_add(dX2k, (ks >> 2) * kTile + 32 * (ks & 3)), idM64,
-                            ks > 0);
-            tc5::commit(&s.mma_bar);
-        }
-        mma_wait();
-        if (w < 4) {  // rows 16q..16q+15 of the M = 64 accumulator sit in lanes 32q..32q+15
-            float v[16];
-            tc5::ld16(tc5::taddr(tm, my_lane, cZ2), v);
-            tc5::wait_ld();
-            if (lane < 16)
-#pragma unroll
-                for (int tt = 0; tt < 16; ++tt) s.Zt[tt][16 * q + lane] = v[tt];
+            for (int e = 0; e < 4; ++e) z2[1][e] = 0.f;
+            tokens_times_w2(z2, x2_s, w2_s, w, lane, lrow, lchunk);
+            *reinterpret_cast<float2*>(&s.Zt[g][8 * w + 2 * t]) = make_float2(z2[0][0] + z2[1][0], z2[0][1] + z2[1][1]);
+            *reinterpret_cast<float2*>(&s.Zt[g + 8][8 * w + 2 * t]) = make_float2(z2[0][2] + z2[1][2], z2[0][3] + z2[1][3]);
         }
         __syncthreads();
 
-        // (4) g2 = ln_fused_l2_bwd(Z2 + b2, XV - XK) on token rows; also -t lr XK for W1's update
+        // (4) g2 = ln_fused_l2_bwd(Z2, XV - XK) on token rows; -t lr g2 and -t lr XK for the updates
         {
             float z[4], xk[4], xv[4];
             const float4 zz = *reinterpret_cast<const float4*>(&s.Zt[rr][f4]);
-            const float4 bb = *reinterpret_cast<const float4*>(&s.b2[f4]);
-            z[0] = zz.x + bb.x; z[1] = zz.y + bb.y; z[2] = zz.z + bb.z; z[3] = zz.w + bb.w;
+            z[0] = zz.x; z[1] = zz.y; z[2] = zz.z; z[3] = zz.w;
             ld4_bf16(xk_t, rr, f4, xk);
             ld4_bf16(xv_t, rr, f4, xv);
             float mu, rs;
@@ -399,7 +409,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             const float ls = -tl * lr_s[rr];
             st4_bf16(&s.G2Ls[0], rr, f4, ls * g2[0], ls * g2[1], ls * g2[2], ls * g2[3]);
             st4_bf16(&s.XKL[0], rr, f4, ls * xk[0], ls * xk[1], ls * xk[2], ls * xk[3]);
-            // b2: sum over this warp's 2 token rows of lr g2
+            // b2: sum over this warp's 2 token rows of lr g2 (the warps' sums meet at the end)
             float bs[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -408,121 +418,140 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             }
             if (lane < 16) *reinterpret_cast<float4*>(&s.b2part[w][f4]) = make_float4(bs[0], bs[1], bs[2], bs[3]);
         }
-        sync_operands();
+        __syncthreads();
 
-        // (5) (g2 W2^T)^T = W2 g2^T (M = 256 hidden in two tiles, K = 64 outputs)
-        if (tid == 0) {
+        // (5) g2 W2^T on this warp's hidden units; (6) g1 = (g2 W2^T) * gelu'(Z1)
+        float g1[4][4];
 #pragma unroll
-            for (int t2 = 0; t2 < 2; ++t2)
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc5::mma_ss(tm + cG1 + 16 * t2, tc5::sdesc_add(dW2k, t2 * 16384 + 32 * ks),
-                                tc5::sdesc_add(dG2k, 32 * ks), idG1, ks > 0);
-            tc5::commit(&s.mma_bar);
-        }
-        mma_wait();
-
-        // (6) g1 = (g2 W2^T) * gelu'(Z1 + b1), by hidden unit
-        float b1sum = 0.f;
-        {
-            float gr[16];
-            tc5::ld16(tc5::taddr(tm, my_lane, cG1 + 16 * mt), gr);
-            tc5::wait_ld();
-            uint8_t* gb = &s.G1s[(u >> 6) * kTile];
+            for (int e = 0; e < 4; ++e) g1[nt][e] = 0.f;
 #pragma unroll
-            for (int tt = 0; tt < 16; ++tt) {
-                const float gv = gr[tt] * dg[tt];
-                st_bf16(gb, swz(tt, u & 63), gv);
-                b1sum = fmaf(lr_s[tt], gv, b1sum);
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(g2_s + swz128(lrow, 2 * kk + lchunk), a0, a1, a2, a3);
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                uint32_t b0, b1, b2, b3;  // W2 rows = hidden (n), outputs = k
+                ldmatrix_x4(w2_s + swz128(32 * w + 16 * hb + lrow, 2 * kk + lchunk), b0, b1, b2, b3);
+                mma_bf16_16816(g1[2 * hb], a0, a1, a2, a3, b0, b2);
+                mma_bf16_16816(g1[2 * hb + 1], a0, a1, a2, a3, b1, b3);
             }
         }
-        sync_operands();
-
-        // (7) Zbar1^T = (XQ W1)^T - g1^T M1^T; (11) the state update on a full mini-batch
-        if (tid == 0) {
+        uint32_t g1p[4][2];
+        {
+            const float lg = lr_s[g], lg8 = lr_s[g + 8];
 #pragma unroll
-            for (int t2 = 0; t2 < 2; ++t2)
-                tc5::mma_ss(tm + cZQ + 32 * t2 + 16, tc5::sdesc_add(dG1m, t2 * 2 * kTile), dM1k, idC1, 1);
-            if (full_mb) {
+            for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
-                for (int t2 = 0; t2 < 2; ++t2) {
-                    // W1^T += g1^T (-t lr XK) ;  W2 += X2^T (-t lr g2)
-                    tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1m, t2 * 2 * kTile), dXKLm, idUp, 1);
-                    tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc_add(dX2m, t2 * 2 * kTile), dG2Lm, idUp, 1);
+                for (int e = 0; e < 4; ++e) g1[nt][e] *= dg[nt][e];
+                g1p[nt][0] = pack_bf16x2(g1[nt][0], g1[nt][1]);
+                g1p[nt][1] = pack_bf16x2(g1[nt][2], g1[nt][3]);
+                // b1 -= t_{K-1} sum_j lr_j g1_j (sum over the 16 token rows: lanes g = 0..7)
+                if (full_mb) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        float v = fmaf(lg, g1[nt][e], lg8 * g1[nt][2 + e]);
+                        v += __shfl_xor_sync(0xffffffffu, v, 4);
+                        v += __shfl_xor_sync(0xffffffffu, v, 8);
+                        v += __shfl_xor_sync(0xffffffffu, v, 16);
+                        b1r[nt][e] -= tl * v;
+                    }
                 }
             }
+        }
+        store_slice(&s.G1s[0], w, g, t, g1p);
+        // the state update on a full mini-batch, on the tensor cores while the output path runs:
+        // W1^T += g1^T (-t lr XK), W2 += X2^T (-t lr g2)
+        fence_proxy_async_smem();
+        tc5::fence_before();
+        __syncthreads();
+        tc5::fence_after();
+        if (tid == 0 && full_mb) {
+#pragma unroll
+            for (int t2 = 0; t2 < 2; ++t2) {
+                tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1m, t2 * 2 * kTile), dXKLm, idUp, 1);
+                tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc_add(dX2m, t2 * 2 * kTile), dG2Lm, idUp, 1);
+            }
             tc5::commit(&s.mma_bar);
         }
-        mma_wait();
 
-        // (8) Xbar2 = gelu(Zbar1 + b1), by hidden unit; then b1's update
+        // (7) Zbar1 = XQ W1 + b1 - M1 g1 (M1 = eta * tril(XQ XK^T + 1), g1 as B by transposes)
         {
-            float zb[16];
-            tc5::ld16(tc5::taddr(tm, my_lane, cZQ + 32 * mt + 16), zb);
-            tc5::wait_ld();
-            uint8_t* xb = &s.XB2s[(u >> 6) * kTile];
+            uint32_t ma[4];
+            m_operand(at1, lr_s, ma);
 #pragma unroll
-            for (int tt = 0; tt < 16; ++tt) st_bf16(xb, swz(tt, u & 63), gelu(zb[tt] + b1r));
-            if (full_mb) b1r -= tl * b1sum;
+            for (int nt = 0; nt < 4; ++nt)
+                mma_bf16_16816(zb1[nt], ma[0], ma[1], ma[2], ma[3], movmatrix_trans(g1p[nt][0]),
+                               movmatrix_trans(g1p[nt][1]));
         }
-        __syncthreads();
-        // Xbar2 X2^T partial sums over hidden block w (warps 0..3, mma.sync)
-        if (w < 4) {
-            float at[2][4] = {};
-            const uint32_t xa = smem_u32(&s.XB2s[w * kTile]), xb = smem_u32(&s.X2s[w * kTile]);
+
+        // (8) Xbar2 = gelu(Zbar1); Xbar2 X2^T over this warp's hidden units, summed over warps
+        {
+            uint32_t xb2p[4][2];
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-                ldmatrix_x4(xa + swz128(lrow, 2 * kk + lchunk), a0, a1, a2, a3);
-                ldmatrix_x4(xb + swz128(lrow, 2 * kk + lchunk), b0, b1, b2, b3);
-                mma_bf16_16816(at[0], a0, a1, a2, a3, b0, b2);
-                mma_bf16_16816(at[1], a0, a1, a2, a3, b1, b3);
+            for (int nt = 0; nt < 4; ++nt) {
+                xb2p[nt][0] = pack_bf16x2(gelu(zb1[nt][0]), gelu(zb1[nt][1]));
+                xb2p[nt][1] = pack_bf16x2(gelu(zb1[nt][2]), gelu(zb1[nt][3]));
+            }
+            store_slice(&s.XB2s[0], w, g, t, xb2p);
+            float a2[2][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {  // hidden n-tiles 2kk, 2kk + 1 form one k-step
+                // A = Xbar2 (rows = tokens), B = X2 (k = hidden, n = tokens), both from accumulators
+                mma_bf16_16816(a2[0], xb2p[2 * kk][0], xb2p[2 * kk][1], xb2p[2 * kk + 1][0], xb2p[2 * kk + 1][1],
+                               x2p[2 * kk][0], x2p[2 * kk + 1][0]);
+                mma_bf16_16816(a2[1], xb2p[2 * kk][0], xb2p[2 * kk][1], xb2p[2 * kk + 1][0], xb2p[2 * kk + 1][1],
+                               x2p[2 * kk][1], x2p[2 * kk + 1][1]);
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                s.A2p[w][g][8 * nt + 2 * t4] = at[nt][0];
-                s.A2p[w][g][8 * nt + 2 * t4 + 1] = at[nt][1];
-                s.A2p[w][g + 8][8 * nt + 2 * t4] = at[nt][2];
-                s.A2p[w][g + 8][8 * nt + 2 * t4 + 1] = at[nt][3];
+                *reinterpret_cast<float2*>(&s.A2p[w][g][8 * nt + 2 * t]) = make_float2(a2[nt][0], a2[nt][1]);
+                *reinterpret_cast<float2*>(&s.A2p[w][g + 8][8 * nt + 2 * t]) = make_float2(a2[nt][2], a2[nt][3]);
             }
         }
         __syncthreads();
-        {  // -M2 = -(eta * tril(Xbar2 X2^T + 1)), one element per thread
-            const int i = tid >> 4, j = tid & 15;
-            const float a2 = s.A2p[0][i][j] + s.A2p[1][i][j] + s.A2p[2][i][j] + s.A2p[3][i][j];
-            const float mv = (j <= i) ? s.te[i] * lr_s[j] * (a2 + 1.0f) : 0.f;
-            st_bf16(&s.M2s[0], swz(i, j), -mv);
-        }
-        sync_operands();
-
-        // (9) Zbar2^T = W2^T Xbar2^T - g2^T M2^T (M = 64)
-        if (tid == 0) {
-#pragma unroll
-            for (int ks = 0; ks < 16; ++ks)
-                tc5::mma_ss(tm + cZB2, tc5::sdesc_add(dW2m, 2048 * ks),
-                            tc5::sdesc_add(dXB2k, (ks >> 2) * kTile + 32 * (ks & 3)), idM64,
-                            ks > 0);
-            tc5::mma_ss(tm + cZB2, dG2m, dM2k,
-                        idM64, 1);
-            tc5::commit(&s.mma_bar);
-        }
-        mma_wait();
-        if (w < 4) {
-            float v[16];
-            tc5::ld16(tc5::taddr(tm, my_lane, cZB2), v);
-            tc5::wait_ld();
-            if (lane < 16)
-#pragma unroll
-                for (int tt = 0; tt < 16; ++tt) s.Zt[tt][16 * q + lane] = v[tt];
+        {  // one element of the 16x16 sum per thread
+            const float* p = &s.A2p[0][0][0] + tid;
+            constexpr int kS = TTT_KMAX * TTT_KMAX;
+            (&s.A2[0][0])[tid] = ((p[0] + p[kS]) + (p[2 * kS] + p[3 * kS])) + ((p[4 * kS] + p[5 * kS]) + (p[6 * kS] + p[7 * kS]));
         }
         __syncthreads();
 
-        // (10) out = XQ + LN(Zbar2 + b2) on token rows
+        // (9) Zbar2 = Xbar2 W2 + b2 - M2 g2 on this warp's outputs -> token rows in Zt
+        {
+            float at2[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                at2[nt][0] = s.A2[g][8 * nt + 2 * t];
+                at2[nt][1] = s.A2[g][8 * nt + 2 * t + 1];
+                at2[nt][2] = s.A2[g + 8][8 * nt + 2 * t];
+                at2[nt][3] = s.A2[g + 8][8 * nt + 2 * t + 1];
+            }
+            uint32_t ma[4];
+            m_operand(at2, lr_s, ma);
+            float zb2[2][4];
+            const float2 bb = *reinterpret_cast<const float2*>(&s.b2[8 * w + 2 * t]);
+            zb2[0][0] = zb2[0][2] = bb.x;
+            zb2[0][1] = zb2[0][3] = bb.y;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) zb2[1][e] = 0.f;
+            tokens_times_w2(zb2, xb2_s, w2_s, w, lane, lrow, lchunk);
+            {
+                uint32_t b0, b1, d0, d1;  // g2 (k = tokens, n = outputs 8w..), transposed from token rows
+                ldmatrix_x4_trans(g2_s + swz128(lrow, w), b0, b1, d0, d1);
+                mma_bf16_16816(zb2[1], ma[0], ma[1], ma[2], ma[3], b0, b1);
+            }
+            *reinterpret_cast<float2*>(&s.Zt[g][8 * w + 2 * t]) = make_float2(zb2[0][0] + zb2[1][0], zb2[0][1] + zb2[1][1]);
+            *reinterpret_cast<float2*>(&s.Zt[g + 8][8 * w + 2 * t]) = make_float2(zb2[0][2] + zb2[1][2], zb2[0][3] + zb2[1][3]);
+        }
+        __syncthreads();
+
+        // (10) out = XQ + LN(Zbar2) on token rows
         {
             float z[4], xq[4];
             const float4 zz = *reinterpret_cast<const float4*>(&s.Zt[rr][f4]);
-            const float4 bb = *reinterpret_cast<const float4*>(&s.b2[f4]);
-            z[0] = zz.x + bb.x; z[1] = zz.y + bb.y; z[2] = zz.z + bb.z; z[3] = zz.w + bb.w;
+            z[0] = zz.x; z[1] = zz.y; z[2] = zz.z; z[3] = zz.w;
             ld4_bf16(xq_t, rr, f4, xq);
             float mu, rs;
             row_stats16(z, eps, mu, rs);
@@ -535,10 +564,13 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 *reinterpret_cast<uint2*>(out + f4) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
             }
         }
-        __syncthreads();
 
-        // (12) new state: b2, and the bf16 shadows of the updated masters
+        // (11) new state: b2, and the bf16 shadows of the updated masters
         if (full_mb) {
+            if (!mbar_wait_bounded(&s.mma_bar, mpar, wait_limit, a.status)) s.fail = 1;
+            mpar ^= 1;
+            tc5::fence_after();
+            __syncthreads();  // every warp is done reading the shadows
             if (tid < TTT_D)
                 s.b2[tid] -= tl * (((s.b2part[0][tid] + s.b2part[1][tid]) + (s.b2part[2][tid] + s.b2part[3][tid])) +
                                    ((s.b2part[4][tid] + s.b2part[5][tid]) + (s.b2part[6][tid] + s.b2part[7][tid])));
@@ -562,7 +594,9 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 }
             }
         }
-        sync_operands();
+        tc5::fence_before();
+        __syncthreads();
+        tc5::fence_after();
         if (s.fail) {
             m_stop = m;
             break;
@@ -585,7 +619,12 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 W2l[u * TTT_D + 16 * c + i] = v2[i];
             }
         }
-        a.b1_last[static_cast<long long>(chain) * kHid + u] = b1r;
+        if (g == 0)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                a.b1_last[static_cast<long long>(chain) * kHid + 32 * w + 8 * nt + 2 * t] = b1r[nt][0];
+                a.b1_last[static_cast<long long>(chain) * kHid + 32 * w + 8 * nt + 2 * t + 1] = b1r[nt][1];
+            }
         if (tid < TTT_D) a.b2_last[static_cast<long long>(chain) * TTT_D + tid] = s.b2[tid];
     } else if (tid == 0) {
         // A wait gave up: let the MMAs and the loads still in flight land (bounded) before the
