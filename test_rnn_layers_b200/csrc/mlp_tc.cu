@@ -182,7 +182,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     // ---- set-up --------------------------------------------------------------------------------
     if (w == 0) tc5::alloc(&s.tmem_base, kTmemCols);
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(&s.full[i], 1 + TTT_KMAX);
+        for (int i = 0; i < kStages; ++i) mbar_init(&s.full[i], 1);
         mbar_init(&s.mma_bar, 1);
         mbar_init(&s.drain_bar, 1);
         fence_mbarrier_init();
@@ -246,24 +246,28 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     __syncthreads();
     tc5::fence_after();
 
-    // producer (warp 0): mini-batch mm into stage st
+    // producer (warp 0): mini-batch mm into stage st.  lr comes by one bulk copy when its slice
+    // is 16-byte aligned and a multiple of 16 bytes (one arrival on the stage's barrier), else by
+    // plain loads of the warp before the arrival (per-lane asynchronous arrivals would serialise
+    // in the barrier unit while every other warp waits for this one)
+    const bool lr_bulk = (K % 4 == 0) && (a.L % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lr) & 15) == 0);
     auto issue = [&](int mm, int st) {
         const int Kmm = mm < n_full ? K : static_cast<int>(a.rem);
         const int row0 = mm * K;
+        const bool bulk = lr_bulk && (Kmm % 4 == 0);
+        if (!bulk) {
+            if (lane < TTT_KMAX) s.lr[st][lane] = lane < Kmm ? lr_g[row0 + lane] : 0.f;
+            __syncwarp();
+        }
         if (lane == 0) {
-            mbar_arrive_expect_tx(&s.full[st], 3 * tile_tx);
+            if (bulk)
+                for (int j = Kmm; j < TTT_KMAX; ++j) s.lr[st][j] = 0.f;
+            const uint32_t lr_tx = bulk ? static_cast<uint32_t>(Kmm) * 4 : 0u;
+            mbar_arrive_expect_tx(&s.full[st], 3 * tile_tx + lr_tx);  // (release: orders the stores above)
             tma_load_3d(&s.stage[st][0], &maps.xk, 0, row0, chain, &s.full[st]);
             tma_load_3d(&s.stage[st][kTile], &maps.xq, 0, row0, chain, &s.full[st]);
             tma_load_3d(&s.stage[st][2 * kTile], &maps.xv, 0, row0, chain, &s.full[st]);
-        }
-        if (lane < TTT_KMAX) {
-            if (lane < Kmm) {
-                cp_async_4(&s.lr[st][lane], lr_g + row0 + lane);
-                cp_async_mbar_arrive_noinc(&s.full[st]);
-            } else {
-                s.lr[st][lane] = 0.f;
-                mbar_arrive(&s.full[st]);
-            }
+            if (bulk) bulk_load(&s.lr[st][0], lr_g + row0, lr_tx, &s.full[st]);
         }
     };
     if (w == 0)
