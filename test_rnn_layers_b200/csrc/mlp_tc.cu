@@ -34,12 +34,14 @@
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
 
+#include <cuda_fp16.h>
+
 namespace ttt {
 namespace {
 
 constexpr int kThreads = 256;
 constexpr int kHid = TTT_HIDDEN;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kTile = TTT_KMAX * 128;  // [16 rows x 128 bytes] bf16 tile
 constexpr uint32_t kTmemCols = 256;
 constexpr long long kDrainPolls = 1ll << 24;
@@ -47,7 +49,7 @@ constexpr uint32_t cW1 = 0;    // + 64 mt: W1^T tile mt (rows = hidden 128mt.., 
 constexpr uint32_t cW2 = 128;  // + 64 mt: W2 tile mt (rows = hidden, cols = output dim)
 
 struct __align__(1024) MlpSmem {
-    uint8_t stage[kStages][3 * kTile];  // XK | XQ | XV
+    uint8_t stage[kStages][3 * kTile];  // XK | XQ | XV; -t_{K-1} lr XK is written over XV
     uint8_t W1s[2][128 * 128];          // bf16 W1^T shadow [tile][128 hidden rows x 128 B (64 inputs)]
     uint8_t W2s[kHid * 128];            // bf16 W2 shadow [256 hidden rows x 128 B (64 outputs)]
     uint8_t X2s[4 * kTile];             // bf16 X2     [4 hidden blocks][16 token rows x 128 B]
@@ -55,12 +57,12 @@ struct __align__(1024) MlpSmem {
     uint8_t G1s[4 * kTile];             // bf16 g1
     uint8_t G2s[kTile];                 // bf16 g2 [16 token rows x 128 B (64 outputs)]
     uint8_t G2Ls[kTile];                // bf16 -t_{K-1} lr g2
-    uint8_t XKL[kTile];                 // bf16 -t_{K-1} lr XK
-    float Zt[TTT_KMAX][TTT_D];          // Z2, then Zbar2, as token rows (b2 included)
-    float A2p[8][TTT_KMAX][TTT_KMAX];   // Xbar2 X2^T over each warp's hidden slice
+    union {                             // (disjoint lifetimes inside a mini-batch)
+        float Zt[TTT_KMAX][TTT_D];      // Z2, then Zbar2, as token rows (b2 included)
+        __half A2p[8][TTT_KMAX][TTT_KMAX];  // Xbar2 X2^T over each warp's hidden slice
+    };
     float A2[TTT_KMAX][TTT_KMAX];       // their sum
     float b2[TTT_D];
-    float b2part[8][TTT_D];             // sum_j lr_j g2_j over each warp's two token rows
     float lr[kStages][TTT_KMAX];
     float te[TTT_KMAX];
     uint64_t full[kStages];
@@ -160,7 +162,7 @@ __device__ __forceinline__ void tokens_times_w2(float (&acc)[2][4], uint32_t a_t
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     MlpSmem& s = *reinterpret_cast<MlpSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -297,7 +299,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     const uint32_t idUp = tc5::idesc_bf16(128, 64, 1, 1);
     const uint64_t dX2m = tc5::sdesc(smem_u32(&s.X2s[0]), kTile, 1024);     // X2^T, MN-major A
     const uint64_t dG1m = tc5::sdesc(smem_u32(&s.G1s[0]), kTile, 1024);     // g1^T, MN-major A
-    const uint64_t dXKLm = tc5::sdesc(smem_u32(&s.XKL[0]), kTile, 1024);    // -t lr XK, MN-major B
+    const uint64_t dXKLm = tc5::sdesc(smem_u32(&s.stage[0][2 * kTile]), kTile, 1024);  // -t lr XK of stage 0, MN-major B
     const uint64_t dG2Lm = tc5::sdesc(smem_u32(&s.G2Ls[0]), kTile, 1024);   // -t lr g2, MN-major B
     const uint32_t w1_s = smem_u32(&s.W1s[(32 * w) >> 7][0]);  // this warp's 32 hidden rows live in one tile
     const int w1_row0 = (32 * w) & 127;
@@ -328,6 +330,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         uint8_t* xk_t = &s.stage[st][0];
         uint8_t* xq_t = &s.stage[st][kTile];
         const uint8_t* xv_t = &s.stage[st][2 * kTile];
+        uint8_t* xkl_t = &s.stage[st][2 * kTile];
         const float* lr_s = s.lr[st];
         const uint32_t xk_s = smem_u32(xk_t), xq_s = smem_u32(xq_t);
 
@@ -412,15 +415,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             st4_bf16(&s.G2s[0], rr, f4, g2[0], g2[1], g2[2], g2[3]);
             const float ls = -tl * lr_s[rr];
             st4_bf16(&s.G2Ls[0], rr, f4, ls * g2[0], ls * g2[1], ls * g2[2], ls * g2[3]);
-            st4_bf16(&s.XKL[0], rr, f4, ls * xk[0], ls * xk[1], ls * xk[2], ls * xk[3]);
-            // b2: sum over this warp's 2 token rows of lr g2 (the warps' sums meet at the end)
-            float bs[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                bs[i] = lr_s[rr] * g2[i];
-                bs[i] += __shfl_xor_sync(0xffffffffu, bs[i], 16);
-            }
-            if (lane < 16) *reinterpret_cast<float4*>(&s.b2part[w][f4]) = make_float4(bs[0], bs[1], bs[2], bs[3]);
+            // each thread overwrites exactly the XV elements it has read
+            st4_bf16(xkl_t, rr, f4, ls * xk[0], ls * xk[1], ls * xk[2], ls * xk[3]);
         }
         __syncthreads();
 
@@ -474,7 +470,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         if (tid == 0 && full_mb) {
 #pragma unroll
             for (int t2 = 0; t2 < 2; ++t2) {
-                tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1m, t2 * 2 * kTile), dXKLm, idUp, 1);
+                tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1m, t2 * 2 * kTile),
+                            tc5::sdesc_add(dXKLm, st * 3 * kTile), idUp, 1);
                 tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc_add(dX2m, t2 * 2 * kTile), dG2Lm, idUp, 1);
             }
             tc5::commit(&s.mma_bar);
@@ -510,19 +507,23 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                *reinterpret_cast<float2*>(&s.A2p[w][g][8 * nt + 2 * t]) = make_float2(a2[nt][0], a2[nt][1]);
-                *reinterpret_cast<float2*>(&s.A2p[w][g + 8][8 * nt + 2 * t]) = make_float2(a2[nt][2], a2[nt][3]);
+                *reinterpret_cast<__half2*>(&s.A2p[w][g][8 * nt + 2 * t]) = __floats2half2_rn(a2[nt][0], a2[nt][1]);
+                *reinterpret_cast<__half2*>(&s.A2p[w][g + 8][8 * nt + 2 * t]) = __floats2half2_rn(a2[nt][2], a2[nt][3]);
             }
         }
         __syncthreads();
         {  // one element of the 16x16 sum per thread
-            const float* p = &s.A2p[0][0][0] + tid;
+            const __half* p = &s.A2p[0][0][0] + tid;
             constexpr int kS = TTT_KMAX * TTT_KMAX;
-            (&s.A2[0][0])[tid] = ((p[0] + p[kS]) + (p[2 * kS] + p[3 * kS])) + ((p[4 * kS] + p[5 * kS]) + (p[6 * kS] + p[7 * kS]));
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __half2float(p[i * kS]);
+            (&s.A2[0][0])[tid] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
         }
         __syncthreads();
 
         // (9) Zbar2 = Xbar2 W2 + b2 - M2 g2 on this warp's outputs -> token rows in Zt
+        float b2d[2];
         {
             float at2[2][4];
 #pragma unroll
@@ -545,6 +546,13 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 uint32_t b0, b1, d0, d1;  // g2 (k = tokens, n = outputs 8w..), transposed from token rows
                 ldmatrix_x4_trans(g2_s + swz128(lrow, w), b0, b1, d0, d1);
                 mma_bf16_16816(zb2[1], ma[0], ma[1], ma[2], ma[3], b0, b1);
+                // sum_j lr_j g2_j for b2's update: an A operand whose row 0 is lr
+                const uint32_t r0 = g == 0 ? pack_bf16x2(lr_s[2 * t], lr_s[2 * t + 1]) : 0u;
+                const uint32_t r2 = g == 0 ? pack_bf16x2(lr_s[2 * t + 8], lr_s[2 * t + 9]) : 0u;
+                float bd[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_bf16_16816(bd, r0, 0u, r2, 0u, b0, b1);
+                b2d[0] = bd[0];  // row 0, outputs 8w + 2t, 8w + 2t + 1 (lanes g == 0)
+                b2d[1] = bd[1];
             }
             *reinterpret_cast<float2*>(&s.Zt[g][8 * w + 2 * t]) = make_float2(zb2[0][0] + zb2[1][0], zb2[0][1] + zb2[1][1]);
             *reinterpret_cast<float2*>(&s.Zt[g + 8][8 * w + 2 * t]) = make_float2(zb2[0][2] + zb2[1][2], zb2[0][3] + zb2[1][3]);
@@ -575,9 +583,10 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             mpar ^= 1;
             tc5::fence_after();
             __syncthreads();  // every warp is done reading the shadows
-            if (tid < TTT_D)
-                s.b2[tid] -= tl * (((s.b2part[0][tid] + s.b2part[1][tid]) + (s.b2part[2][tid] + s.b2part[3][tid])) +
-                                   ((s.b2part[4][tid] + s.b2part[5][tid]) + (s.b2part[6][tid] + s.b2part[7][tid])));
+            if (g == 0) {
+                s.b2[8 * w + 2 * t] -= tl * b2d[0];
+                s.b2[8 * w + 2 * t + 1] -= tl * b2d[1];
+            }
             const int r = u & 127;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -652,6 +661,10 @@ cudaError_t launch_mlp_tc(const MlpArgs& a, const LinearMaps& maps, cudaStream_t
     const size_t smem = sizeof(MlpSmem) + 1024;  // + alignment slack
     cudaError_t e = cudaFuncSetAttribute(mlp_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    // two CTAs (chains) per SM: ask for the largest shared-memory carve-out
+    e = cudaFuncSetAttribute(mlp_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     mlp_tc_kernel<<<static_cast<unsigned>(a.B * a.H), kThreads, smem, st>>>(a, maps);
     return cudaGetLastError();
