@@ -136,3 +136,10 @@ def test_mlp_bounded_wait_timeout_reports_and_recovers(libttt):
     assert libttt.ttt_device_status(clear=True) == 0
     _check(gpu_mlp(libttt, x, w), oracle_mlp(x, w), 1e-2)
     assert libttt.ttt_device_status() == 0
+
+
+def test_mlp_odd_chain_count(libttt):
+    """Chains are paired per CTA; with an odd count the last pair has one chain."""
+    w = synth.workload(3, B=1, H=3, L=16 * 3 + 5, dtype="bf16", seed=0x3C01)
+    x = _mlp_inputs(w)
+    _check(gpu_mlp(libttt, x, w), oracle_mlp(x, w), 1e-2)
