@@ -1,6 +1,6 @@
 """Benchmark of the TTT scan on B200: TTT layer tokens/s and the fraction of the per-layer roofline.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,mlp,decode]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,mlp,decode,decode_hist]
                     [--no-cpu-baseline] [--no-headline] [--seq-len L]
 
 One step = one ttt_linear_forward over the 1B-layer workload (B=8, H=32, L=8200, d=64, K=16,
@@ -18,8 +18,8 @@ ttt_linear_forward_host from pinned HOST buffers, every input copied in and ever
 out inside the timed region, the batch pipelined in chunks),
 `roofline` (the scan kernel's algorithmic bytes / its CUDA-event time vs the measured HBM copy
 bandwidth), `cpu_baseline` (the CPU oracle on a bounded sample, rank 0 at N=1), `clocks`
-(NVML samples taken during the timed region) and `rows` (the TTT-MLP prefill and the decode
-step, each timed the same way).  `--impl reference` times the oracle instead, as the reference
+(NVML samples taken during the timed region) and `rows` (the TTT-MLP prefill, the decode step
+with the dense cache and with the history-format cache, each timed the same way).  `--impl reference` times the oracle instead, as the reference
 arm.
 """
 from __future__ import annotations
@@ -76,6 +76,16 @@ def mlp_flops(B, H, L, hid=256, K=16):
     dense = 7 * 2 * K * D * hid                  # Z1, XQ W1, Z2, Xbar2 W2, g2 W2^T, two updates
     tri = 2 * (K * (K + 1) // 2) * (2 * D + 2 * hid)  # Attn1, Attn2, M1 g1, M2 g2
     return B * H * n_mb * (dense + tri)
+
+
+def decode_hist_bytes(B, H, p, K=16):
+    """One step of the history-format cache at position p, per chain: read W, b, b_grad and p
+    rows of (lr xk, g); write one row and b_grad, or W, b and b_grad on the commit step; tokens
+    xq, xk, xv, lr in, out out (bf16)."""
+    state = (D * D + D) * 4
+    rows = p * 2 * D * 4
+    write = state + D * 4 if p == K - 1 else 2 * D * 4 + D * 4
+    return B * H * (state + D * 4 + rows + write + 3 * D * 2 + 4 + D * 2)
 
 
 def decode_bytes(B, H, commit_fraction=1.0 / 16):
@@ -336,7 +346,9 @@ def bench_mlp(args, world, peaks):
                          "hbm_frac": round(mlp_bytes(w.B, w.H, w.L) / (ms / 1e3) / 1e9 / hbm, 4)}}
 
 
-def bench_decode(args, world, peaks):
+def bench_decode(args, world, peaks, hist=False):
+    """The decode step, dense cache (ttt_linear_decode_step) or history-format cache
+    (ttt_linear_decode_step_hist), from the state of a 2048-token prefill."""
     import torch
 
     import test_rnn_layers_b200 as ttt
@@ -347,6 +359,9 @@ def bench_decode(args, world, peaks):
                                              dev_f32(x["ln_w"]), dev_f32(x["ln_b"]), eps=w.eps, tail_grads=True)
     lnw, lnb = dev_f32(x["ln_w"]), dev_f32(x["ln_b"])
     del x
+    if hist:  # 2048 is a mini-batch boundary: the history cache starts empty
+        del Wg
+        rows = torch.zeros(w.B, w.H, w.K, 2, D, device="cuda")
     toks = synth.linear_inputs(w, values=False, t0=w.L, t1=w.L + w.decode_steps)
     XQ, XK, XV = (dev_act(toks, n) for n in ("XQ", "XK", "XV"))
     lr = dev_f32(toks["lr"])
@@ -358,7 +373,11 @@ def bench_decode(args, world, peaks):
 
     def one(i):
         q, k, v, l = xs[i % w.decode_steps]
-        ttt.ttt_linear_decode_step(q, k, v, l, lnw, lnb, W, b, Wg, bg, seqlen_offset=pos[0], eps=w.eps, out=out)
+        if hist:
+            ttt.ttt_linear_decode_step_hist(q, k, v, l, lnw, lnb, W, b, rows, bg, seqlen_offset=pos[0], eps=w.eps,
+                                            out=out)
+        else:
+            ttt.ttt_linear_decode_step(q, k, v, l, lnw, lnb, W, b, Wg, bg, seqlen_offset=pos[0], eps=w.eps, out=out)
         pos[0] += 1
 
     # each timed step starts with a cold L2 (the 133 MB state is about the L2 size): flush, then time it
@@ -367,18 +386,23 @@ def bench_decode(args, world, peaks):
         one(i)
     s = torch.cuda.current_stream()
     total = 0.0
+    nbytes_total = 0
     for i in range(K):
         flush.fill_(float(i))
+        p = pos[0] % w.K
+        nbytes_total += decode_hist_bytes(w.B, w.H, p, w.K) if hist else decode_bytes(w.B, w.H)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
         one(i)
         e1.record(s)
         e1.synchronize()
         total += e0.elapsed_time(e1)
+    ttt.ttt_device_status()
     ms = max_over_ranks(world, total / K)
     hbm = peaks[0]
-    nbytes = decode_bytes(w.B, w.H)
-    return {"workload": "ttt_linear_decode_B128_H32_after_prefill2048", "value": round(world * w.B / (ms / 1e3), 1),
+    nbytes = nbytes_total / K
+    name = "ttt_linear_decode_hist_cache_B128_H32_after_prefill2048" if hist else "ttt_linear_decode_B128_H32_after_prefill2048"
+    return {"workload": name, "value": round(world * w.B / (ms / 1e3), 1),
             "unit": "tokens/s", "ms_per_step": round(ms, 5), "steps": K, "gpu_launches": K,
             "l2": "flushed (256 MB write) before every timed step",
             "roofline": {"bound": "hbm", "achieved": round(nbytes / (ms / 1e3) / 1e9, 1), "peak": hbm,
@@ -451,7 +475,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rows", default="linear,mlp,decode",
+    ap.add_argument("--rows", default="linear,mlp,decode,decode_hist",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=1,
@@ -480,6 +504,8 @@ def main():
             extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
         if "decode" in rows:
             extra["ttt_linear_decode"] = bench_decode(args, world, peaks)
+        if "decode_hist" in rows:
+            extra["ttt_linear_decode_hist"] = bench_decode(args, world, peaks, hist=True)
         if rank == 0:
             print(json.dumps({"rows": extra}), flush=True)
         if world > 1:
@@ -492,6 +518,8 @@ def main():
         extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
     if "decode" in rows:
         extra["ttt_linear_decode"] = bench_decode(args, world, peaks)
+    if "decode_hist" in rows:
+        extra["ttt_linear_decode_hist"] = bench_decode(args, world, peaks, hist=True)
     if extra:
         line["rows"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

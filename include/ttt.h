@@ -223,6 +223,32 @@ int ttt_linear_decode_step(const void* xq, const void* xk, const void* xv, const
                            int d, int mini_batch, long long seqlen_offset, float eps, int dtype,
                            void* out, void* stream);
 
+/*
+ * ttt_linear_decode_step_hist -- the decode step of ttt_linear_decode_step with a history-format
+ * cache.  The dense cache keeps W_grad = sum_{j<p} lr_j xk_j^T g_j (d x d per chain); this one
+ * keeps the rows that make it up, (lr_j * xk_j, g_j) for the tokens j < p of the current
+ * mini-batch, and forms xq W_grad as sum_j (xq . lr_j xk_j) g_j.  The results are those of the
+ * dense cache (up to fp32 rounding order); the state traffic per step is W, b, b_grad and p rows
+ * read, one row and b_grad written (and W, b on the commit step) instead of W and W_grad read
+ * and W_grad written.
+ * Arguments as ttt_linear_decode_step, except
+ *   hist    [B,H,K,2,d] float32 in/out (K = mini_batch), 16-byte aligned: row j of a chain holds
+ *           lr_j * xk_j (d floats) then g_j (d floats).  Rows j < p = seqlen_offset mod K are
+ *           read; row p is written (except on the commit step p = K-1, which folds the rows into
+ *           W); rows past p are neither read nor written.
+ *   b_grad  [B,H,d] float32 in/out: sum_{j<p} lr_j g_j, zeroed on the commit step.
+ * A history cache starts at a mini-batch boundary (seqlen_offset mod K == 0) with b_grad = 0;
+ * there the dense and history caches coincide (both are just W, b).
+ * Rows are read only while the p read for this call says so: all chains share seqlen_offset.
+ * (No counterpart on the pages beyond the identity W_grad = sum_j lr_j xk_j^T g_j of the primal
+ * branch in "代码连连看——TTT", compute_mini_batch.)
+ * Errors as ttt_linear_decode_step.
+ */
+int ttt_linear_decode_step_hist(const void* xq, const void* xk, const void* xv, const float* lr,
+                                const float* token_eta, const float* ln_w, const float* ln_b, float* W, float* b,
+                                float* hist, float* b_grad, int B, int H, int d, int mini_batch,
+                                long long seqlen_offset, float eps, int dtype, void* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,8 @@ TTT_STATUS_TIMEOUT = 1
 
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
            "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_host_workspace_bytes",
-           "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step")
+           "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step",
+           "ttt_linear_decode_step_hist")
 
 
 class TTTError(RuntimeError):
@@ -70,8 +71,11 @@ def lib():
                                       u, vp, fp, fp, fp, fp, vp]
         L.ttt_linear_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f, i,
                                              vp, vp]
+        L.ttt_linear_decode_step_hist.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f,
+                                                  i, vp, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
-                     "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step"):
+                     "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step",
+                     "ttt_linear_decode_step_hist"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -303,5 +307,33 @@ def ttt_linear_decode_step(xq, xk, xv, lr, ln_w, ln_b, W, b, W_grad, b_grad, seq
     rc = lib().ttt_linear_decode_step(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(lr), _ptr(token_eta), _ptr(ln_w),
                                       _ptr(ln_b), _ptr(W), _ptr(b), _ptr(W_grad), _ptr(b_grad), B, H, d,
                                       mini_batch, seqlen_offset, eps, _dtype_code(xq), _ptr(out), _stream(stream))
+    _check(rc)
+    return out
+
+
+def ttt_linear_decode_step_hist(xq, xk, xv, lr, ln_w, ln_b, W, b, hist, b_grad, seqlen_offset: int,
+                                mini_batch: int = 16, eps: float = 1e-6, token_eta=None, out=None, stream=None):
+    """One decode token per chain ([B,H,64] inputs) through a history-format cache: W [B,H,64,64],
+    b [B,H,64], hist [B,H,K,2,64] (rows (lr_j xk_j, g_j) of the current mini-batch), b_grad
+    [B,H,64], all updated in place.  Start it at a mini-batch boundary with b_grad = 0.
+    Returns out [B,H,64]."""
+    _need(xq, "xq")
+    B, H, d = xq.shape
+    dt = xq.dtype
+    for n, t in (("xk", xk), ("xv", xv)):
+        _need(t, n, dt, xq.shape)
+    _need(lr, "lr", torch.float32, (B, H))
+    _need(ln_w, "ln_w", torch.float32, (H, d))
+    _need(ln_b, "ln_b", torch.float32, (H, d))
+    _need(W, "W", torch.float32, (B, H, d, d))
+    _need(b, "b", torch.float32, (B, H, d))
+    _need(hist, "hist", torch.float32, (B, H, mini_batch, 2, d))
+    _need(b_grad, "b_grad", torch.float32, (B, H, d))
+    if token_eta is not None:
+        _need(token_eta, "token_eta", torch.float32, (mini_batch,))
+    out = torch.empty_like(xq) if out is None else _need(out, "out", dt, xq.shape)
+    rc = lib().ttt_linear_decode_step_hist(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(lr), _ptr(token_eta), _ptr(ln_w),
+                                           _ptr(ln_b), _ptr(W), _ptr(b), _ptr(hist), _ptr(b_grad), B, H, d,
+                                           mini_batch, seqlen_offset, eps, _dtype_code(xq), _ptr(out), _stream(stream))
     _check(rc)
     return out

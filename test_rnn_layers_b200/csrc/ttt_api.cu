@@ -565,4 +565,42 @@ int ttt_linear_decode_step(const void* xq, const void* xk, const void* xv, const
     return ok();
 }
 
+int ttt_linear_decode_step_hist(const void* xq, const void* xk, const void* xv, const float* lr,
+                                const float* token_eta, const float* ln_w, const float* ln_b, float* W, float* b,
+                                float* hist, float* b_grad, int B, int H, int d, int mini_batch,
+                                long long seqlen_offset, float eps, int dtype, void* out, void* stream) {
+    int rc = check_common(B, H, 1, d, mini_batch, eps, dtype, 0);
+    if (rc) return rc;
+    if (seqlen_offset < 0) return fail(TTT_ERR_ARG, "seqlen_offset must be >= 0");
+    if (!xq || !xk || !xv || !lr || !ln_w || !ln_b || !W || !b || !hist || !b_grad || !out)
+        return fail(TTT_ERR_ARG, "all tensor arguments except token_eta must be non-null");
+    const void* a16[] = {xq, xk, xv, out, W, b, hist, b_grad};
+    for (int i = 0; i < 8; ++i)
+        if (!aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "tensor argument %d must be 16-byte aligned", i);
+    const void* a4[] = {lr, token_eta, ln_w, ln_b};
+    for (int i = 0; i < 4; ++i)
+        if (a4[i] && !aligned(a4[i], 4)) return fail(TTT_ERR_ALIGN, "lr/token_eta/ln_w/ln_b must be 4-byte aligned");
+    const long long chains = static_cast<long long>(B) * H;
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t vec = static_cast<size_t>(chains) * kD * esz;
+    const size_t mat = static_cast<size_t>(chains) * kD * kD * 4, bv = static_cast<size_t>(chains) * kD * 4;
+    const size_t hv = static_cast<size_t>(chains) * mini_batch * 2 * kD * 4;
+    Span in[] = {{"xq", xq, vec}, {"xk", xk, vec}, {"xv", xv, vec}, {"lr", lr, static_cast<size_t>(chains) * 4},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
+                 {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    Span outs[] = {{"out", out, vec}, {"W", W, mat}, {"b", b, bv}, {"hist", hist, hv}, {"b_grad", b_grad, bv}};
+    rc = check_aliasing(in, 7, outs, 5);
+    if (rc) return rc;
+
+    ttt::DecodeHistArgs a{};
+    a.xq = xq; a.xk = xk; a.xv = xv; a.lr = lr; a.token_eta = token_eta; a.ln_w = ln_w; a.ln_b = ln_b;
+    a.W = W; a.b = b; a.hist = hist; a.b_grad = b_grad; a.B = B; a.H = H; a.K = mini_batch;
+    a.p = static_cast<int>(seqlen_offset % mini_batch); a.eps = eps; a.out = out;
+    a.status = status_word();
+    a.wait_limit = wait_limit();
+    cudaError_t e = ttt::launch_decode_hist(a, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_decode_step_hist launch");
+    return ok();
+}
+
 }  // extern "C"

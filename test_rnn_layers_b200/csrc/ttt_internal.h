@@ -81,6 +81,28 @@ struct DecodeArgs {
     long long wait_limit;
 };
 
+// The decode step with a history-format cache (rows (lr_j xk_j, g_j) of the current mini-batch
+// instead of the dense gradient sum).
+struct DecodeHistArgs {
+    const void* xq;
+    const void* xk;
+    const void* xv;
+    const float* lr;
+    const float* token_eta;
+    const float* ln_w;
+    const float* ln_b;
+    float* W;
+    float* b;
+    float* hist;    // [B*H][K][2][d]
+    float* b_grad;
+    int B, H, K;
+    int p;
+    float eps;
+    void* out;
+    unsigned int* status;
+    long long wait_limit;
+};
+
 // Tensor maps of the bf16 tensor-core prefill kernels: [B*H, L, 64] bf16 viewed 3-D,
 // box {64, K, 1}, 128-byte swizzle (the TTT-MLP kernel leaves `out` unused).
 struct LinearMaps {
@@ -95,5 +117,6 @@ cudaError_t launch_mlp_simt(const MlpArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_mlp_tc(const MlpArgs& a, const LinearMaps& maps, cudaStream_t s);
 cudaError_t launch_mlp_state_copy(const MlpArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_decode_hist(const DecodeHistArgs& a, int dtype, cudaStream_t s);
 
 }  // namespace ttt

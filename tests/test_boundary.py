@@ -170,3 +170,21 @@ def test_host_workspace_bytes(libttt):
                        ((8, 32, 8200, 32, 16, 1, 1, 0), -6), ((8, 32, 8200, 64, 16, 1, 1, 5), -1),
                        ((8, 32, -1, 64, 16, 1, 1, 0), -1)):
         assert lib.ttt_linear_host_workspace_bytes(*args) == code
+
+
+def test_decode_hist_rejects(libttt):
+    lib = libttt.lib()
+
+    def call(**kw):
+        args = dict(xq=A, xk=2 * A, xv=3 * A, lr=4 * A, te=None, lnw=5 * A, lnb=6 * A, W=7 * A, b=8 * A,
+                    hist=9 * A, bg=10 * A, B=2, H=3, d=64, K=16, off=5, eps=1e-6, dtype=1, out=11 * A)
+        args.update(kw)
+        return lib.ttt_linear_decode_step_hist(args["xq"], args["xk"], args["xv"], args["lr"], args["te"],
+                                               args["lnw"], args["lnb"], args["W"], args["b"], args["hist"],
+                                               args["bg"], args["B"], args["H"], args["d"], args["K"], args["off"],
+                                               args["eps"], args["dtype"], args["out"], None)
+
+    for kw, code in ((dict(hist=None), -1), (dict(off=-1), -1), (dict(hist=9 * A + 4), -2), (dict(K=0), -1),
+                     (dict(d=48), -6), (dict(hist=7 * A), -3), (dict(out=A), -3), (dict(bg=None), -1)):
+        assert call(**kw) == code, kw
+        assert lib.ttt_last_error_message()
