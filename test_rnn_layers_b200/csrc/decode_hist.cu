@@ -39,6 +39,7 @@ struct __align__(16) HistSmem {
     float lr[kBufs][4];
     float4 part[2][kRowGroups][TTT_D / 4];  // partial xk W, xq W
     float sz[TTT_D], sqw[TTT_D], sg[TTT_D];
+    float scr[TTT_D];                     // sum_{j<p} (xq . a_j) g_j
     float c[TTT_KMAX];                    // xq . a_j
     float sqk;
     uint64_t full[kBufs];
@@ -130,6 +131,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_hist_kernel(Decod
             if (which == 0) s.sz[col] = acc + s.b[bi][col];
             else s.sqw[col] = acc;
         }
+        if (tid >= 2 * TTT_D && tid < 3 * TTT_D) {  // the rows' part of xq W_grad, off warp 0's path
+            const int col = tid - 2 * TTT_D;
+            float acc = 0.f;
+            for (int j = 0; j < p; ++j) acc = fmaf(s.c[j], s.hist[bi][j][TTT_D + col], acc);
+            s.scr[col] = acc;
+        }
         if (warp == 7) {
             const float v = to_f32(s.x[bi][0][lane]) * to_f32(s.x[bi][1][lane]) +
                             to_f32(s.x[bi][0][lane + 32]) * to_f32(s.x[bi][1][lane + 32]);
@@ -160,12 +167,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_hist_kernel(Decod
             s.sg[lane] = g0;
             s.sg[lane + 32] = g1;
 
-            // xq W_grad, summed from the rows: sum_{j<p} (xq . a_j) g_j + lr (xq . xk) g
-            float cr0 = lr * s.sqk * g0, cr1 = lr * s.sqk * g1;
-            for (int j = 0; j < p; ++j) {
-                cr0 = fmaf(s.c[j], s.hist[bi][j][TTT_D + lane], cr0);
-                cr1 = fmaf(s.c[j], s.hist[bi][j][TTT_D + lane + 32], cr1);
-            }
+            // xq W_grad = sum_{j<p} (xq . a_j) g_j + lr (xq . xk) g
+            const float cr0 = fmaf(lr * s.sqk, g0, s.scr[lane]), cr1 = fmaf(lr * s.sqk, g1, s.scr[lane + 32]);
             const float gb0 = s.gb[bi][lane] + lr * g0, gb1 = s.gb[bi][lane + 32] + lr * g1;
             const float bb0 = s.b[bi][lane] - t * gb0, bb1 = s.b[bi][lane + 32] - t * gb1;
             const float u0 = s.sqw[lane] - t * cr0 + bb0, u1 = s.sqw[lane + 32] - t * cr1 + bb1;
