@@ -1,6 +1,6 @@
 """Benchmark of the TTT scan on B200: TTT layer tokens/s and the fraction of the per-layer roofline.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,mlp,decode,decode_hist]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,linear_tm,mlp,decode,decode_hist]
                     [--no-cpu-baseline] [--no-headline] [--seq-len L]
 
 One step = one ttt_linear_forward over the 1B-layer workload (B=8, H=32, L=8200, d=64, K=16,
@@ -18,9 +18,10 @@ ttt_linear_forward_host from pinned HOST buffers, every input copied in and ever
 out inside the timed region, the batch pipelined in chunks),
 `roofline` (the scan kernel's algorithmic bytes / its CUDA-event time vs the measured HBM copy
 bandwidth), `cpu_baseline` (the CPU oracle on a bounded sample, rank 0 at N=1), `clocks`
-(NVML samples taken during the timed region) and `rows` (the TTT-MLP prefill, the decode step
-with the dense cache and with the history-format cache, each timed the same way).  `--impl reference` times the oracle instead, as the reference
-arm.
+(NVML samples taken during the timed region) and `rows` (the same scan on token-major
+[B,L,H,d] activations beside the time of the permutes that layout saves, the TTT-MLP prefill,
+the decode step with the dense cache and with the history-format cache, each timed the same
+way).  `--impl reference` times the oracle instead, as the reference arm.
 """
 from __future__ import annotations
 
@@ -319,6 +320,49 @@ def bench_linear(args, world, rank, local, peaks):
     return line
 
 
+def bench_linear_token_major(args, world, peaks):
+    """The headline scan on token-major [B,L,H,d] activations (TTT_FLAG_TOKEN_MAJOR: the layout
+    the QKV projections produce and the layer returns), and beside it the time of the four
+    [B,H,L,d] <-> [B,L,H,d] copies (XQ, XK, XV in, out back) that the flag makes unnecessary."""
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    w = synth.workload(2, L=args.seq_len)
+    x = synth.linear_inputs(w, values=False)
+    XQ, XK, XV = (dev_act(x, n).transpose(1, 2).contiguous() for n in ("XQ", "XK", "XV"))
+    lr, W0, b0, lnw, lnb = (dev_f32(x[k]) for k in ("lr", "W0", "b0", "ln_w", "ln_b"))
+    B, H, L = w.B, w.H, w.L
+    out = torch.empty_like(XQ)
+    Wl, bl = torch.empty(B, H, D, D, device="cuda"), torch.empty(B, H, D, device="cuda")
+    Wg, bg = torch.empty(B, H, D, D, device="cuda"), torch.empty(B, H, D, device="cuda")
+
+    def step():
+        ttt.ttt_linear_forward(XQ, XK, XV, lr, W0, b0, lnw, lnb, mini_batch=w.K, eps=w.eps, out=out,
+                               W_last=Wl, b_last=bl, W_grad_tail=Wg, b_grad_tail=bg, tail_grads=True,
+                               token_major=True)
+
+    K = max(3, min(args.steps, 10))
+    ms = time_steps(step, K, 3, world)
+    ttt.ttt_device_status()
+    hm = [torch.empty(B, H, L, D, dtype=XQ.dtype, device="cuda") for _ in range(4)]
+
+    def permutes():  # what a head-major scan needs around it: 3 inputs in, the output back
+        for src, dst in zip((XQ, XK, XV), hm[:3]):
+            dst.copy_(src.transpose(1, 2))
+        out.copy_(hm[3].transpose(1, 2))
+
+    perm_ms = time_steps(permutes, K, 3, world)
+    hbm = peaks[0]
+    nbytes = linear_bytes(B, H, L)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"ttt_linear_prefill_1b_layer_token_major_B{B}_H{H}_L{L}", "activations": "bf16 [B,L,H,d]",
+            "value": round(world * B * L / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "steps": K, "gpu_launches": K,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "algorithmic_bytes": nbytes},
+            "replaced_permutes_ms": round(perm_ms, 4)}
+
+
 def bench_mlp(args, world, peaks):
     import torch
 
@@ -475,7 +519,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rows", default="linear,mlp,decode,decode_hist",
+    ap.add_argument("--rows", default="linear,linear_tm,mlp,decode,decode_hist",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=1,
@@ -500,6 +544,8 @@ def main():
     rows = [r.strip() for r in args.rows.split(",") if r.strip()]
     if args.no_headline:
         extra = {}
+        if "linear_tm" in rows:
+            extra["ttt_linear_prefill_token_major"] = bench_linear_token_major(args, world, peaks)
         if "mlp" in rows:
             extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
         if "decode" in rows:
@@ -514,6 +560,8 @@ def main():
         return
     line = bench_linear(args, world, rank, local, peaks)
     extra = {}
+    if "linear_tm" in rows:
+        extra["ttt_linear_prefill_token_major"] = bench_linear_token_major(args, world, peaks)
     if "mlp" in rows:
         extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
     if "decode" in rows:

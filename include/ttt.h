@@ -48,6 +48,10 @@ extern "C" {
 
 /* flags for the forward calls */
 #define TTT_FLAG_FP32_COMPUTE 1u /* run bf16 inputs through the FFMA (fp32-compute) kernel */
+/* XQ, XK, XV and out are token-major [B,L,H,d] -- the [B,L,C] (C = H*d) layout of the QKV
+ * projections and of the scan's return value in TTTBase.forward / TTTLinear.ttt -- instead of
+ * the head-major [B,H,L,d].  lr stays [B,H,L].  The arithmetic and the results are the same. */
+#define TTT_FLAG_TOKEN_MAJOR 2u
 
 /* Bits of the device status word */
 #define TTT_STATUS_TIMEOUT 1u /* a kernel gave up on a bounded wait and returned early */
@@ -112,9 +116,12 @@ int ttt_set_wait_limit(long long polls);
  *   mini_batch   K in [1, 16].
  *   eps          LayerNorm epsilon, > 0.
  *   dtype        TTT_F32 or TTT_BF16.
- *   flags        0 or TTT_FLAG_FP32_COMPUTE.  bf16 inputs run on the tensor-core kernel
- *                (bf16 operands, fp32 accumulation and fp32 state) unless the flag asks for the
- *                FFMA kernel; fp32 inputs always run on the FFMA kernel.
+ *   flags        TTT_FLAG_FP32_COMPUTE and/or TTT_FLAG_TOKEN_MAJOR, or 0.  bf16 inputs run on
+ *                the tensor-core kernel (bf16 operands, fp32 accumulation and fp32 state) unless
+ *                FP32_COMPUTE asks for the FFMA kernel; fp32 inputs always run on the FFMA
+ *                kernel.  TOKEN_MAJOR: XQ, XK, XV and out are [B,L,H,d] instead of [B,H,L,d]
+ *                (the walkthrough's [B,L,C] before its reshape/transpose and after the scan's
+ *                permute/reshape, so neither permute is needed); lr stays [B,H,L].
  * Outputs (device, caller-allocated):
  *   out          [B,H,L,d] dtype, 16-byte aligned (may be NULL when L == 0).
  *   W_last, b_last  [B,H,d,d], [B,H,d] float32: the state after the last FULL mini-batch (the

@@ -27,6 +27,7 @@ TTT_ERR_UNSUPPORTED = -6
 TTT_F32 = 0
 TTT_BF16 = 1
 TTT_FLAG_FP32_COMPUTE = 1
+TTT_FLAG_TOKEN_MAJOR = 2
 TTT_STATUS_TIMEOUT = 1
 
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
@@ -118,6 +119,17 @@ def _need(t, name, dtype=None, shape=None):
     return t
 
 
+def _act_sizes(XQ, token_major: bool):
+    """(B, H, L, d) of activations laid out [B,H,L,d], or [B,L,H,d] when token_major."""
+    if XQ.dim() != 4:
+        raise ValueError(f"XQ must be 4-D, got shape {tuple(XQ.shape)}")
+    if token_major:
+        B, L, H, d = XQ.shape
+    else:
+        B, H, L, d = XQ.shape
+    return B, H, L, d
+
+
 def ttt_partition(L: int, mini_batch: int):
     """(n_full, rem) = (L // K, L % K), computed by the library (host-only)."""
     n, r = ctypes.c_longlong(), ctypes.c_longlong()
@@ -139,14 +151,16 @@ def ttt_device_status(clear: bool = True, stream=None) -> int:
 
 def ttt_linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
                        token_eta=None, out=None, W_last=None, b_last=None, W_grad_tail=None,
-                       b_grad_tail=None, tail_grads: bool = False, flags: int = 0, stream=None):
-    """TTT-Linear prefill over [B,H,L,64] activations (see include/ttt.h).
+                       b_grad_tail=None, tail_grads: bool = False, flags: int = 0, token_major: bool = False,
+                       stream=None):
+    """TTT-Linear prefill over [B,H,L,64] activations, or [B,L,H,64] with token_major (see include/ttt.h).
 
     W0/b0: [H,64,64]/[H,64] shared over the batch, or [B,H,64,64]/[B,H,64] per chain.
     Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail).
     """
     _need(XQ, "XQ")
-    B, H, L, d = XQ.shape
+    B, H, L, d = _act_sizes(XQ, token_major)
+    flags |= TTT_FLAG_TOKEN_MAJOR if token_major else 0
     dt = XQ.dtype
     for n, t in (("XK", XK), ("XV", XV)):
         _need(t, n, dt, XQ.shape)
@@ -203,7 +217,7 @@ def ttt_linear_host_workspace_bytes(B: int, H: int, L: int, mini_batch: int = 16
 def ttt_linear_forward_host(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
                             token_eta=None, out=None, W_last=None, b_last=None, W_grad_tail=None,
                             b_grad_tail=None, tail_grads: bool = False, flags: int = 0, chunk_batches: int = 1,
-                            workspace=None, stream=None):
+                            workspace=None, token_major: bool = False, stream=None):
     """ttt_linear_forward on HOST tensors (pin them for overlap): the batch streams through the
     GPU in chunks of `chunk_batches` batch rows, copies in both directions overlapping the scan.
     `workspace`: a CUDA uint8 tensor of at least ttt_linear_host_workspace_bytes(...) bytes, or
@@ -211,7 +225,8 @@ def ttt_linear_forward_host(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int 
     Asynchronous on `stream`: synchronise before reading the outputs.
     Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail)."""
     _need_host(XQ, "XQ")
-    B, H, L, d = XQ.shape
+    B, H, L, d = _act_sizes(XQ, token_major)
+    flags |= TTT_FLAG_TOKEN_MAJOR if token_major else 0
     dt = XQ.dtype
     for n, t in (("XK", XK), ("XV", XV)):
         _need_host(t, n, dt, XQ.shape)
@@ -249,13 +264,15 @@ def ttt_linear_forward_host(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int 
 
 
 def ttt_mlp_forward(XQ, XK, XV, lr, W1, b1, W2, b2, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
-                    token_eta=None, out=None, flags: int = 0, stream=None):
+                    token_eta=None, out=None, flags: int = 0, token_major: bool = False, stream=None):
     """TTT-MLP prefill; states W1 [H,64,256], b1 [H,256], W2 [H,256,64], b2 [H,64] (or per chain).
+    Activations [B,H,L,64], or [B,L,H,64] with token_major.
 
     Returns (out, W1_last, b1_last, W2_last, b2_last).
     """
     _need(XQ, "XQ")
-    B, H, L, d = XQ.shape
+    B, H, L, d = _act_sizes(XQ, token_major)
+    flags |= TTT_FLAG_TOKEN_MAJOR if token_major else 0
     dt = XQ.dtype
     for n, t in (("XK", XK), ("XV", XV)):
         _need(t, n, dt, XQ.shape)

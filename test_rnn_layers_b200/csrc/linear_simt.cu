@@ -45,11 +45,13 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long chain = blockIdx.x;
     const int h = static_cast<int>(chain % a.H);
-    const T* XQ = static_cast<const T*>(a.XQ) + chain * a.L * TTT_D;
-    const T* XK = static_cast<const T*>(a.XK) + chain * a.L * TTT_D;
-    const T* XV = static_cast<const T*>(a.XV) + chain * a.L * TTT_D;
+    const long long aoff = (chain / a.H) * a.act_b + (chain % a.H) * a.act_h;  // token 0 of this chain
+    const long long ts = a.act_t;                                               // elements per token step
+    const T* XQ = static_cast<const T*>(a.XQ) + aoff;
+    const T* XK = static_cast<const T*>(a.XK) + aoff;
+    const T* XV = static_cast<const T*>(a.XV) + aoff;
     const float* lr = a.lr + chain * a.L;
-    T* out = static_cast<T*>(a.out) + chain * a.L * TTT_D;
+    T* out = static_cast<T*>(a.out) + aoff;
 
     const float* W0 = a.W0 + (a.w0_chain_stride ? chain * a.w0_chain_stride
                                                  : static_cast<long long>(h) * TTT_D * TTT_D);
@@ -72,7 +74,7 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
         for (int i = tid; i < TTT_KMAX * TTT_D; i += kThreads) {
             int r = i / TTT_D, c = i % TTT_D;
             bool v = r < Km;
-            long long off = (t0 + r) * TTT_D + c;
+            long long off = (t0 + r) * ts + c;
             s.xq[r][c] = v ? to_f32(XQ[off]) : 0.f;
             s.xk[r][c] = v ? to_f32(XK[off]) : 0.f;
             s.xv[r][c] = v ? to_f32(XV[off]) : 0.f;
@@ -135,9 +137,9 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
             float mu, rstd;
             row_stats(z0, z1, a.eps, mu, rstd);
             if (r < Km) {
-                out[(t0 + r) * TTT_D + lane] =
+                out[(t0 + r) * ts + lane] =
                     from_f32<T>(s.xq[r][lane] + s.lnw[lane] * (z0 - mu) * rstd + s.lnb[lane]);
-                out[(t0 + r) * TTT_D + lane + 32] = from_f32<T>(
+                out[(t0 + r) * ts + lane + 32] = from_f32<T>(
                     s.xq[r][lane + 32] + s.lnw[lane + 32] * (z1 - mu) * rstd + s.lnb[lane + 32]);
             }
         }

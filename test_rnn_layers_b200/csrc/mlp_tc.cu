@@ -70,6 +70,7 @@ struct __align__(1024) MlpSmem {
     uint64_t drain_bar;
     uint32_t tmem_base;
     int fail;
+    long long out_off;                  // element offset of this chain's token 0 in out
 };
 
 // byte offset of bf16 element (row r, col c < 64) in a [rows x 128 B] tile, 128-byte swizzle
@@ -172,7 +173,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
     const int u = 128 * mt + 32 * q + lane;      // the hidden unit whose master rows this thread moves
     const int g = lane >> 2, t = lane & 3;
     const int chain = blockIdx.x;
-    const int h = chain % a.H;
+    const int h = chain % a.H, bi = chain / a.H;
     const int K = a.K;
     const int n_full = static_cast<int>(a.n_full);
     const int n_mb = n_full + (a.rem > 0 ? 1 : 0);
@@ -192,6 +193,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         tma_prefetch_desc(&maps.xk);
         tma_prefetch_desc(&maps.xv);
         s.fail = 0;
+        s.out_off = bi * a.act_b + h * a.act_h;
     }
     for (int i = tid; i < kStages * 3 * kTile / 16; i += kThreads)
         reinterpret_cast<uint4*>(&s.stage[0][0])[i] = make_uint4(0, 0, 0, 0);  // rows >= K stay zero
@@ -266,9 +268,11 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 for (int j = Kmm; j < TTT_KMAX; ++j) s.lr[st][j] = 0.f;
             const uint32_t lr_tx = bulk ? static_cast<uint32_t>(Kmm) * 4 : 0u;
             mbar_arrive_expect_tx(&s.full[st], 3 * tile_tx + lr_tx);  // (release: orders the stores above)
-            tma_load_3d(&s.stage[st][0], &maps.xk, 0, row0, chain, &s.full[st]);
-            tma_load_3d(&s.stage[st][kTile], &maps.xq, 0, row0, chain, &s.full[st]);
-            tma_load_3d(&s.stage[st][2 * kTile], &maps.xv, 0, row0, chain, &s.full[st]);
+            // coordinates (0, token, h, b) head-major, (0, h, token, b) token-major
+            const int c1 = a.tok_major ? h : row0, c2 = a.tok_major ? row0 : h;
+            tma_load_4d(&s.stage[st][0], &maps.xk, 0, c1, c2, bi, &s.full[st]);
+            tma_load_4d(&s.stage[st][kTile], &maps.xq, 0, c1, c2, bi, &s.full[st]);
+            tma_load_4d(&s.stage[st][2 * kTile], &maps.xv, 0, c1, c2, bi, &s.full[st]);
             if (bulk) bulk_load(&s.lr[st][0], lr_g + row0, lr_tx, &s.full[st]);
         }
     };
@@ -571,8 +575,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 float o[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) o[i] = xq[i] + fmaf(lw[i], (z[i] - mu) * rs, lb[i]);
-                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
-                                     (static_cast<long long>(chain) * a.L + static_cast<long long>(m) * K + rr) * TTT_D;
+                __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + s.out_off +
+                                     (static_cast<long long>(m) * K + rr) * a.act_t;
                 *reinterpret_cast<uint2*>(out + f4) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
             }
         }

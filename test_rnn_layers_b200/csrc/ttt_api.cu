@@ -98,20 +98,35 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// [chains, L, 64] bf16 viewed 3-D; box {64, K, 1}; 128-byte swizzle; out-of-range rows read 0.
-int encode_act_map(CUtensorMap* map, const void* base, long long chains, long long L, int K,
+// XQ / XK / XV (bf16) as a 4-D tensor map with 128-byte swizzle; out-of-range rows read 0.
+// Head-major [B, H, L, 64]: dims {64, L, H, B}, box {64, K, 1, 1}.
+// Token-major [B, L, H, 64]: dims {64, H, L, B}, box {64, 1, K, 1}.
+int encode_act_map(CUtensorMap* map, const void* base, int B, int H, long long L, int K, bool tok_major,
                    const char* name) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return fail(TTT_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(chains)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(L) * kD * 2};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(K), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    const cuuint64_t row = static_cast<cuuint64_t>(kD) * 2;  // bytes of one token of one head
+    const cuuint64_t d1 = tok_major ? H : L, d2 = tok_major ? L : H;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), d1, d2, static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {row, row * d1, row * d1 * d2};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(kD), tok_major ? 1u : static_cast<cuuint32_t>(K),
+                         tok_major ? static_cast<cuuint32_t>(K) : 1u, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(TTT_ERR_CUDA, "tensor map for %s: cuTensorMapEncodeTiled error %d", name, (int)r);
     return TTT_OK;
+}
+
+// Element strides of the activations between batch rows, heads and tokens.
+template <class Args>
+void set_act_strides(Args& a, int H, long long L, bool tok_major) {
+    const long long hd = static_cast<long long>(H) * kD;
+    a.act_b = L * hd;
+    a.act_h = tok_major ? kD : L * kD;
+    a.act_t = tok_major ? hd : kD;
+    a.tok_major = tok_major ? 1 : 0;
 }
 
 int cuda_fail(cudaError_t e, const char* what) {
@@ -128,7 +143,7 @@ int check_common(int B, int H, long long L, int d, int K, float eps, int dtype, 
     if (K < 1 || K > 16) return fail(TTT_ERR_ARG, "mini_batch must be in [1, 16] (got %d)", K);
     if (!(eps > 0.f) || !std::isfinite(eps)) return fail(TTT_ERR_ARG, "eps must be finite and > 0");
     if (dtype != TTT_F32 && dtype != TTT_BF16) return fail(TTT_ERR_ARG, "dtype must be TTT_F32 or TTT_BF16");
-    if (flags & ~TTT_FLAG_FP32_COMPUTE) return fail(TTT_ERR_ARG, "unknown flags 0x%x", flags);
+    if (flags & ~(TTT_FLAG_FP32_COMPUTE | TTT_FLAG_TOKEN_MAJOR)) return fail(TTT_ERR_ARG, "unknown flags 0x%x", flags);
     return TTT_OK;
 }
 
@@ -158,7 +173,6 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
                    const float* W0, const float* b0, long long w0_chain_stride, const float* ln_w, const float* ln_b,
                    int B, int H, long long L, int mini_batch, float eps, int dtype, unsigned int flags, void* out,
                    float* W_last, float* b_last, float* W_grad_tail, float* b_grad_tail, cudaStream_t st) {
-    const long long chains = static_cast<long long>(B) * H;
     int rc;
     ttt::LinearArgs a{};
     a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
@@ -168,6 +182,8 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
     a.out = out; a.W_last = W_last; a.b_last = b_last; a.W_grad_tail = W_grad_tail; a.b_grad_tail = b_grad_tail;
     a.status = status_word();
     a.wait_limit = wait_limit();
+    const bool tm = (flags & TTT_FLAG_TOKEN_MAJOR) != 0;
+    set_act_strides(a, H, L, tm);
 
     cudaError_t e;
     if (L == 0) {
@@ -176,10 +192,9 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
         e = ttt::launch_linear_simt(a, dtype, st);
     } else {
         ttt::LinearMaps maps;
-        if ((rc = encode_act_map(&maps.xq, XQ, chains, L, mini_batch, "XQ"))) return rc;
-        if ((rc = encode_act_map(&maps.xk, XK, chains, L, mini_batch, "XK"))) return rc;
-        if ((rc = encode_act_map(&maps.xv, XV, chains, L, mini_batch, "XV"))) return rc;
-        if ((rc = encode_act_map(&maps.out, out, chains, L, mini_batch, "out"))) return rc;
+        if ((rc = encode_act_map(&maps.xq, XQ, B, H, L, mini_batch, tm, "XQ"))) return rc;
+        if ((rc = encode_act_map(&maps.xk, XK, B, H, L, mini_batch, tm, "XK"))) return rc;
+        if ((rc = encode_act_map(&maps.xv, XV, B, H, L, mini_batch, tm, "XV"))) return rc;
         e = ttt::launch_linear_tc(a, maps, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward launch");
@@ -510,6 +525,8 @@ int ttt_mlp_forward(const void* XQ, const void* XK, const void* XV, const float*
     a.W1_last = W1_last; a.b1_last = b1_last; a.W2_last = W2_last; a.b2_last = b2_last;
     a.status = status_word();
     a.wait_limit = wait_limit();
+    const bool tm = (flags & TTT_FLAG_TOKEN_MAJOR) != 0;
+    set_act_strides(a, H, L, tm);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (L == 0) {
@@ -518,10 +535,9 @@ int ttt_mlp_forward(const void* XQ, const void* XK, const void* XV, const float*
         e = ttt::launch_mlp_simt(a, dtype, st);
     } else {
         ttt::LinearMaps maps;
-        if ((rc = encode_act_map(&maps.xq, XQ, chains, L, mini_batch, "XQ"))) return rc;
-        if ((rc = encode_act_map(&maps.xk, XK, chains, L, mini_batch, "XK"))) return rc;
-        if ((rc = encode_act_map(&maps.xv, XV, chains, L, mini_batch, "XV"))) return rc;
-        maps.out = maps.xq;
+        if ((rc = encode_act_map(&maps.xq, XQ, B, H, L, mini_batch, tm, "XQ"))) return rc;
+        if ((rc = encode_act_map(&maps.xk, XK, B, H, L, mini_batch, tm, "XK"))) return rc;
+        if ((rc = encode_act_map(&maps.xv, XV, B, H, L, mini_batch, tm, "XV"))) return rc;
         e = ttt::launch_mlp_tc(a, maps, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ttt_mlp_forward launch");

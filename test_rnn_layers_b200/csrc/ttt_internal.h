@@ -25,6 +25,10 @@ struct LinearArgs {
     int K;
     long long n_full, rem;
     float eps;
+    // element strides of XQ, XK, XV and out between batch rows, heads and tokens:
+    // [B, H, L, d] (head-major): H*L*d, L*d, d;  [B, L, H, d] (token-major): L*H*d, d, H*d
+    long long act_b, act_h, act_t;
+    int tok_major;            // 1: token-major, the order of the tensor maps' coordinates
     void* out;
     float* W_last;
     float* b_last;
@@ -52,6 +56,8 @@ struct MlpArgs {
     int K;
     long long n_full, rem;
     float eps;
+    long long act_b, act_h, act_t;  // as in LinearArgs
+    int tok_major;
     void* out;
     float* W1_last;
     float* b1_last;
@@ -103,10 +109,12 @@ struct DecodeHistArgs {
     long long wait_limit;
 };
 
-// Tensor maps of the bf16 tensor-core prefill kernels: [B*H, L, 64] bf16 viewed 3-D,
-// box {64, K, 1}, 128-byte swizzle (the TTT-MLP kernel leaves `out` unused).
+// Tensor maps of XQ, XK, XV for the bf16 tensor-core prefill kernels, 4-D, 128-byte swizzle:
+// head-major dims {64, L, H, B}, box {64, K, 1, 1}, coordinates (0, token, h, b);
+// token-major dims {64, H, L, B}, box {64, 1, K, 1}, coordinates (0, h, token, b).
+// Either way a box lands in shared memory as K rows of 128 bytes; rows past L read zero.
 struct LinearMaps {
-    CUtensorMap xq, xk, xv, out;
+    CUtensorMap xq, xk, xv;
 };
 
 // launchers (return cudaSuccess or the launch error)
