@@ -25,6 +25,14 @@ def test_header_declares_the_entry_points():
         assert f in names
 
 
+def test_binding_constants_match_the_header(libttt):
+    defines = dict(re.findall(r"#define\s+(TTT_\w+)\s+\(?(-?\d+)u?\)?", open(HEADER).read()))
+    shared = [n for n in defines if hasattr(libttt, n)]
+    assert "TTT_FLAG_TOKEN_MAJOR" in shared and "TTT_ERR_ALIAS" in shared
+    for n in shared:
+        assert getattr(libttt, n) == int(defines[n]), n
+
+
 def test_library_exports_every_declared_symbol(libttt):
     lib = ctypes.CDLL(libttt.LIB_PATH)
     for name in declared_functions():
@@ -73,6 +81,9 @@ def _fwd(lib, **kw):
     (dict(d=32), -6), (dict(XQ=None), -1), (dict(W0=None), -1), (dict(out=None), -1),
     (dict(stride=5), -1), (dict(XK=2 * A + 2), -2), (dict(out=9 * A + 8), -2), (dict(lr=4 * A + 1), -2),
     (dict(out=A), -3), (dict(Wl=5 * A), -3), (dict(bl=10 * A + 64), -3), (dict(Wg=10 * A), -3),
+    (dict(flags=4), -1), (dict(flags=2 | 4), -1),
+    # TTT_FLAG_TOKEN_MAJOR (2) alone or with FP32_COMPUTE passes the flag check; the later checks still apply
+    (dict(flags=2, out=A), -3), (dict(flags=3, XK=2 * A + 2), -2), (dict(flags=2, K=0), -1),
 ])
 def test_linear_forward_rejects(libttt, kw, code):
     lib = libttt.lib()
@@ -188,3 +199,14 @@ def test_decode_hist_rejects(libttt):
                      (dict(d=48), -6), (dict(hist=7 * A), -3), (dict(out=A), -3), (dict(bg=None), -1)):
         assert call(**kw) == code, kw
         assert lib.ttt_last_error_message()
+
+
+def test_token_major_sizes_in_the_binding(libttt):
+    """The binding reads (B, H, L, d) from [B,H,L,d], or from [B,L,H,d] with token_major (host only)."""
+    import torch
+    x = torch.empty(2, 5, 3, 64)
+    assert libttt._act_sizes(x, False) == (2, 5, 3, 64)
+    assert libttt._act_sizes(x, True) == (2, 3, 5, 64)
+    with pytest.raises(ValueError):
+        libttt._act_sizes(torch.empty(2, 5, 64), False)
+    assert libttt.TTT_FLAG_TOKEN_MAJOR == 2
