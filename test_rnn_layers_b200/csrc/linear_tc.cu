@@ -25,8 +25,8 @@
 //    from registers.  Shared-memory traffic is kept to the TMA tiles, the ldmatrix operand loads
 //    and a few hundred bytes of row statistics per mini-batch.
 //  * A fifth, producer warp streams the inputs: a TMA ring of kStages mini-batches (XQ, XK, XV
-//    tiles, 128-byte swizzle, K rows of 128 bytes, from head-major [B,H,L,64] or token-major
-//    [B,L,H,64] activations alike) plus cp.async for lr, with a "full" mbarrier per stage
+//    tiles, 128-byte swizzle, K rows of 128 bytes, from head-major [B,H,L,64] (3-D map) or
+//    token-major [B,L,H,64] (4-D map) activations alike) plus cp.async for lr, with a "full" mbarrier per stage
 //    (data landed) and an "empty" one (the four compute warps are done with it).  No multicast.
 //    Every mbarrier wait is bounded; on expiry the kernel raises the status word, drains its
 //    in-flight copies (bounded) and returns.
@@ -106,6 +106,8 @@ __device__ __forceinline__ void merge_row(const float4 (*red)[2], int row, float
 
 // out rows of mini-batch mm = XQ + LN(Zbar), written straight from the accumulator layout:
 // rows g and g+8, features 16w + 8nt + 2t + {0,1} (rows past the mini-batch's end are skipped).
+// Consecutive tokens are 64 elements apart head-major, H * 64 token-major.
+template <bool kTok>
 __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearArgs& a, __nv_bfloat16* out_chain, int mm, int K,
                                           int n_full, int g, int t, int w, const float (&zb)[2][4],
                                           const uint32_t (&xq)[4], const float (&lw)[2][2], const float (&lb)[2][2]) {
@@ -113,7 +115,8 @@ __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearAr
     merge_row(red, g, a.eps, mu0, rs0);
     merge_row(red, g + 8, a.eps, mu1, rs1);
     const int Km = mm < n_full ? K : static_cast<int>(a.rem);
-    __nv_bfloat16* out = out_chain + static_cast<long long>(mm) * K * a.act_t;
+    const long long ts = kTok ? a.act_t : TTT_D;
+    __nv_bfloat16* out = out_chain + static_cast<long long>(mm) * K * ts;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
         // xq[2nt] = row g, xq[2nt+1] = row g+8 (A fragment order a0..a3)
@@ -122,16 +125,19 @@ __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearAr
         if (g < Km) {
             const float2 y = fma2(l2, fma2(make_float2(zb[nt][0], zb[nt][1]), bc2(rs0), bc2(-mu0 * rs0)), b2);
             const float2 o = add2(unpack_bf16x2(xq[2 * nt]), y);
-            *reinterpret_cast<uint32_t*>(out + g * a.act_t + f) = pack_bf16x2(o.x, o.y);
+            *reinterpret_cast<uint32_t*>(out + g * ts + f) = pack_bf16x2(o.x, o.y);
         }
         if (g + 8 < Km) {
             const float2 y = fma2(l2, fma2(make_float2(zb[nt][2], zb[nt][3]), bc2(rs1), bc2(-mu1 * rs1)), b2);
             const float2 o = add2(unpack_bf16x2(xq[2 * nt + 1]), y);
-            *reinterpret_cast<uint32_t*>(out + (g + 8) * a.act_t + f) = pack_bf16x2(o.x, o.y);
+            *reinterpret_cast<uint32_t*>(out + (g + 8) * ts + f) = pack_bf16x2(o.x, o.y);
         }
     }
 }
 
+// kTok: token-major activations ([B, L, H, 64], 4-D tensor maps) or head-major ([B, H, L, 64],
+// 3-D tensor maps over [B*H, L, 64])
+template <bool kTok>
 __global__ void __launch_bounds__(kBlock, 2)
 linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // align by a byte offset from the shared array itself (an integer round trip of the pointer
@@ -147,7 +153,8 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     const int n_full = static_cast<int>(a.n_full);
     const int n_mb = n_full + (a.rem > 0 ? 1 : 0);
     const float* lr_g = a.lr + static_cast<long long>(chain) * a.L;
-    __nv_bfloat16* const out_chain = static_cast<__nv_bfloat16*>(a.out) + bi * a.act_b + h * a.act_h;
+    __nv_bfloat16* const out_chain = static_cast<__nv_bfloat16*>(a.out) +
+                                     (kTok ? bi * a.act_b + h * a.act_h : static_cast<long long>(chain) * a.L * TTT_D);
     const uint32_t tile_tx = static_cast<uint32_t>(K) * TTT_D * 2;
 
     // ---- set-up ------------------------------------------------------------------------------
@@ -178,12 +185,16 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         const int Kmm = mm < n_full ? K : static_cast<int>(a.rem);
         const int row0 = mm * K;
         if (lane == 0) {
-            // coordinates (0, token, h, b) head-major, (0, h, token, b) token-major
-            const int c1 = a.tok_major ? h : row0, c2 = a.tok_major ? row0 : h;
             mbar_arrive_expect_tx(&s.full[st], 3 * tile_tx);
-            tma_load_4d(&s.xq[st][0], &maps.xq, 0, c1, c2, bi, &s.full[st]);
-            tma_load_4d(&s.xk[st][0], &maps.xk, 0, c1, c2, bi, &s.full[st]);
-            tma_load_4d(&s.xv[st][0], &maps.xv, 0, c1, c2, bi, &s.full[st]);
+            if constexpr (kTok) {  // coordinates (0, h, token, b)
+                tma_load_4d(&s.xq[st][0], &maps.xq, 0, h, row0, bi, &s.full[st]);
+                tma_load_4d(&s.xk[st][0], &maps.xk, 0, h, row0, bi, &s.full[st]);
+                tma_load_4d(&s.xv[st][0], &maps.xv, 0, h, row0, bi, &s.full[st]);
+            } else {               // coordinates (0, token, chain)
+                tma_load_3d(&s.xq[st][0], &maps.xq, 0, row0, chain, &s.full[st]);
+                tma_load_3d(&s.xk[st][0], &maps.xk, 0, row0, chain, &s.full[st]);
+                tma_load_3d(&s.xv[st][0], &maps.xv, 0, row0, chain, &s.full[st]);
+            }
         }
         if (lane < TTT_KMAX) {
             if (lane < Kmm) {
@@ -349,7 +360,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             failed = true;
             break;
         }
-        if (m > 0) store_out(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
+        if (m > 0) store_out<kTok>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
 
         // ---- g = ln_fused_l2_bwd(Z, XV - XK): partial sums of q and q * xhat -----------------
         float mu[2], rs[2];
@@ -504,7 +515,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // ---- the last mini-batch's output ---------------------------------------------------------
     if (n_mb > 0) {
         named_barrier_sync(1, kThreads);
-        store_out(s.red3[(n_mb - 1) & 1], a, out_chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
+        store_out<kTok>(s.red3[(n_mb - 1) & 1], a, out_chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
     }
 
     // ---- final state ------------------------------------------------------------------------
@@ -532,10 +543,10 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
 
 cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t st) {
     const size_t smem = sizeof(TcSmem) + 1024;  // + alignment slack
-    cudaError_t e = cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    auto kernel = a.tok_major ? linear_tc_kernel<true> : linear_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    linear_tc_kernel<<<static_cast<unsigned>(a.B * a.H), kBlock, smem, st>>>(a, maps);
+    kernel<<<static_cast<unsigned>(a.B * a.H), kBlock, smem, st>>>(a, maps);
     return cudaGetLastError();
 }
 

@@ -98,11 +98,11 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// XQ / XK / XV (bf16) as a 4-D tensor map with 128-byte swizzle; out-of-range rows read 0.
-// Head-major [B, H, L, 64]: dims {64, L, H, B}, box {64, K, 1, 1}.
-// Token-major [B, L, H, 64]: dims {64, H, L, B}, box {64, 1, K, 1}.
+// XQ / XK / XV (bf16) as a tensor map with 128-byte swizzle; out-of-range rows read 0.
+// Head-major [B, H, L, 64]: 4-D dims {64, L, H, B}, box {64, K, 1, 1}, or (three_d) 3-D dims
+// {64, L, B*H}, box {64, K, 1}.  Token-major [B, L, H, 64]: 4-D dims {64, H, L, B}, box {64, 1, K, 1}.
 int encode_act_map(CUtensorMap* map, const void* base, int B, int H, long long L, int K, bool tok_major,
-                   const char* name) {
+                   const char* name, bool three_d = false) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return fail(TTT_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint64_t row = static_cast<cuuint64_t>(kD) * 2;  // bytes of one token of one head
@@ -112,7 +112,12 @@ int encode_act_map(CUtensorMap* map, const void* base, int B, int H, long long L
     cuuint32_t box[4] = {static_cast<cuuint32_t>(kD), tok_major ? 1u : static_cast<cuuint32_t>(K),
                          tok_major ? static_cast<cuuint32_t>(K) : 1u, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint32_t rank = 4;
+    if (three_d && !tok_major) {  // chains (b, h) flattened: b * H + h
+        rank = 3;
+        dims[2] = static_cast<cuuint64_t>(B) * static_cast<cuuint64_t>(H);
+    }
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(TTT_ERR_CUDA, "tensor map for %s: cuTensorMapEncodeTiled error %d", name, (int)r);
@@ -192,9 +197,9 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
         e = ttt::launch_linear_simt(a, dtype, st);
     } else {
         ttt::LinearMaps maps;
-        if ((rc = encode_act_map(&maps.xq, XQ, B, H, L, mini_batch, tm, "XQ"))) return rc;
-        if ((rc = encode_act_map(&maps.xk, XK, B, H, L, mini_batch, tm, "XK"))) return rc;
-        if ((rc = encode_act_map(&maps.xv, XV, B, H, L, mini_batch, tm, "XV"))) return rc;
+        if ((rc = encode_act_map(&maps.xq, XQ, B, H, L, mini_batch, tm, "XQ", true))) return rc;
+        if ((rc = encode_act_map(&maps.xk, XK, B, H, L, mini_batch, tm, "XK", true))) return rc;
+        if ((rc = encode_act_map(&maps.xv, XV, B, H, L, mini_batch, tm, "XV", true))) return rc;
         e = ttt::launch_linear_tc(a, maps, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward launch");

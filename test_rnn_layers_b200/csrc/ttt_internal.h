@@ -109,8 +109,9 @@ struct DecodeHistArgs {
     long long wait_limit;
 };
 
-// Tensor maps of XQ, XK, XV for the bf16 tensor-core prefill kernels, 4-D, 128-byte swizzle:
-// head-major dims {64, L, H, B}, box {64, K, 1, 1}, coordinates (0, token, h, b);
+// Tensor maps of XQ, XK, XV for the bf16 tensor-core prefill kernels, 128-byte swizzle:
+// head-major 4-D dims {64, L, H, B}, box {64, K, 1, 1}, coordinates (0, token, h, b) -- or, for
+// the TTT-Linear kernel, 3-D dims {64, L, B*H}, box {64, K, 1}, coordinates (0, token, chain);
 // token-major dims {64, H, L, B}, box {64, 1, K, 1}, coordinates (0, h, token, b).
 // Either way a box lands in shared memory as K rows of 128 bytes; rows past L read zero.
 struct LinearMaps {
