@@ -28,7 +28,8 @@
 //    tensor cores read them.
 //  * The two LayerNorms (loss gradient on Z2, output on Zbar2) run on token rows, 16 lanes per
 //    row, after the warps' output slices meet in shared memory.
-//  * XQ, XK, XV tiles arrive by TMA (box {64, K}, 128-byte swizzle, no multicast) into a ring.
+//  * XQ, XK, XV tiles arrive by TMA (K rows of 128 bytes from a 4-D tensor map, head-major or
+//    token-major, 128-byte swizzle, no multicast) into a ring.
 //    One thread issues the tcgen05 MMAs and commits to one mbarrier; all waits are bounded.
 #include "tc5.cuh"
 #include "ttt_common.cuh"
