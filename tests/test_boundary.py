@@ -130,6 +130,8 @@ def test_mlp_rejects(libttt):
     assert call(W2=None) == -1
     assert call(out=3 * A) == -3
     assert call(b2l=15 * A + 4) == -2
+    assert call(flags=4) == -1
+    assert call(flags=2, out=3 * A) == -3  # token-major accepted; the overlap check still applies
 
 
 def test_binding_refuses_cpu_tensors(libttt):
@@ -210,3 +212,25 @@ def test_token_major_sizes_in_the_binding(libttt):
     with pytest.raises(ValueError):
         libttt._act_sizes(torch.empty(2, 5, 64), False)
     assert libttt.TTT_FLAG_TOKEN_MAJOR == 2
+
+
+def test_last_error_message_is_per_host_thread(libttt):
+    """Two host threads failing in different ways each read back their own message."""
+    import threading
+    lib = libttt.lib()
+    got = {}
+    barrier = threading.Barrier(2)
+
+    def worker(name, kw):
+        rc = _fwd(lib, **kw)
+        barrier.wait()  # both calls have failed before either reads its message
+        got[name] = (rc, lib.ttt_last_error_message())
+
+    threads = [threading.Thread(target=worker, args=("K", dict(K=0))),
+               threading.Thread(target=worker, args=("align", dict(XK=2 * A + 2)))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert got["K"][0] == -1 and b"mini_batch" in got["K"][1]
+    assert got["align"][0] == -2 and b"aligned" in got["align"][1]
