@@ -12,13 +12,15 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers into memory the caller owns (allocated by the
- *    caller, e.g. PyTorch) -- except in ttt_linear_forward_host, whose tensors are HOST buffers.  The library allocates no device memory and keeps no state across
- *    calls except a thread-local last-error message and one device status word per device.
+ *    caller, e.g. PyTorch) -- except in ttt_linear_forward_host, whose tensors are HOST
+ *    buffers.  The library allocates no device memory and keeps no state across calls except
+ *    a thread-local last-error message and one device status word per device.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the legacy
  *    default stream).  No call synchronises the stream, except ttt_device_status().
  *  - A "chain" is one (batch b, head h) pair; chain index = b * H + h.
  *  - Activations are [B, H, L, d] contiguous (the layout TTTLinear.ttt receives after the head
- *    split), so one chain's mini-batch is one contiguous block of K * d elements.
+ *    split), so one chain's mini-batch is one contiguous block of K * d elements -- or, for the
+ *    prefill calls with TTT_FLAG_TOKEN_MAJOR, [B, L, H, d] (the [B, L, C] of the projections).
  *  - dtype selects the element type of XQ, XK, XV and out: TTT_F32 or TTT_BF16.  The output
  *    takes the input dtype (the walkthrough allocates XQW_batch with the input dtype).  The
  *    hidden state (W, b, grads), lr, token_eta, ln_w and ln_b are always float32.

@@ -1,0 +1,57 @@
+/* Plain C99 client of include/ttt.h: the ABI is usable from C (no C++ or torch types), and the
+ * host-only calls behave as documented.  Built and run by tests/test_c_abi.py; needs no GPU
+ * (argument errors are reported before any CUDA call).  Prints one line per check; exit 0 iff
+ * every check passed. */
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "ttt.h"
+
+static int failures = 0;
+
+static void check(int ok, const char* what) {
+    printf("%s %s\n", ok ? "ok" : "FAIL", what);
+    if (!ok) ++failures;
+}
+
+int main(void) {
+    long long n = -1, r = -1;
+    check(ttt_partition(8200, 16, &n, &r) == TTT_OK && n == 512 && r == 8, "partition 8200 / 16");
+    check(ttt_partition(0, 16, &n, &r) == TTT_OK && n == 0 && r == 0, "partition 0 / 16");
+    check(ttt_partition(-1, 16, &n, &r) == TTT_ERR_ARG, "partition rejects L < 0");
+    check(ttt_partition(10, 0, &n, &r) == TTT_ERR_ARG, "partition rejects K < 1");
+    check(strlen(ttt_last_error_message()) > 0, "a failed call leaves a message");
+    check(strcmp(ttt_error_string(TTT_ERR_ALIGN), "misaligned pointer") == 0, "error string");
+
+    /* fake, 16-byte aligned device addresses: validation never dereferences them */
+    const uintptr_t A = (uintptr_t)1 << 20;
+    const void* XQ = (const void*)(1 * A);
+    const void* XK = (const void*)(2 * A);
+    const void* XV = (const void*)(3 * A);
+    const float* lr = (const float*)(4 * A);
+    const float* W0 = (const float*)(5 * A);
+    const float* b0 = (const float*)(6 * A);
+    const float* lnw = (const float*)(7 * A);
+    const float* lnb = (const float*)(8 * A);
+    void* out = (void*)(9 * A);
+    float* Wl = (float*)(10 * A);
+    float* bl = (float*)(11 * A);
+    check(ttt_linear_forward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 17, 1e-6f, TTT_BF16, 0,
+                             out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_ARG, "forward rejects K = 17");
+    check(ttt_linear_forward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 32, 16, 1e-6f, TTT_BF16, 0,
+                             out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_UNSUPPORTED, "forward rejects d = 32");
+    check(ttt_linear_forward(XQ, (const char*)XK + 2, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f,
+                             TTT_BF16, TTT_FLAG_TOKEN_MAJOR, out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_ALIGN,
+          "forward rejects a misaligned XK (token-major flag accepted)");
+    check(ttt_linear_forward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0,
+                             (void*)XQ, Wl, bl, NULL, NULL, NULL) == TTT_ERR_ALIAS, "forward rejects out == XQ");
+    check(ttt_linear_forward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 8,
+                             out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_ARG, "forward rejects unknown flags");
+
+    const long long ws = ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 1, 0);
+    check(ws > 0 && ws % 256 == 0, "host workspace size");
+    check(ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 9, 0) == TTT_ERR_ARG,
+          "host workspace rejects chunk_batches > B");
+    return failures == 0 ? 0 : 1;
+}
