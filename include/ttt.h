@@ -25,8 +25,11 @@
  *    takes the input dtype (the walkthrough allocates XQW_batch with the input dtype).  The
  *    hidden state (W, b, grads), lr, token_eta, ln_w and ln_b are always float32.
  *  - Only head dimension d = 64 is supported; mini_batch K in [1, 16].
- *  - Return value: TTT_OK (0) or a negative TTT_ERR_* code; on error nothing has been enqueued
- *    and ttt_last_error_message() describes the cause.  No C++ exception crosses the ABI.
+ *  - Return value: TTT_OK (0) or a negative TTT_ERR_* code, and ttt_last_error_message()
+ *    describes the cause.  After an argument error (every code but TTT_ERR_CUDA) nothing has been
+ *    enqueued.  TTT_ERR_CUDA from the single-launch calls also means nothing ran; only
+ *    ttt_linear_forward_host, which enqueues many copies and launches, can fail with TTT_ERR_CUDA
+ *    after part of its work is enqueued (see there).  No C++ exception crosses the ABI.
  *  - Argument errors are found on the host before any CUDA call, so they can be tested
  *    without a GPU.
  */
@@ -76,8 +79,10 @@ const char* ttt_last_error_message(void);
 /*
  * ttt_device_status -- read (and optionally clear) the status word that kernels on the CURRENT
  * device set when a bounded wait expires.  Synchronises `stream`.  *status receives the
- * TTT_STATUS_* bits (0 = healthy).  Returns TTT_ERR_TIMEOUT if the timeout bit was set,
- * TTT_ERR_CUDA on a CUDA error, else TTT_OK.
+ * TTT_STATUS_* bits (0 = healthy).  With clear != 0 the word is read and zeroed in one atomic
+ * step on the device (a one-thread kernel on `stream`), so a bit that a kernel on another
+ * stream raises meanwhile is reported by this call or the next, never lost.  Returns
+ * TTT_ERR_TIMEOUT if the timeout bit was set, TTT_ERR_CUDA on a CUDA error, else TTT_OK.
  */
 int ttt_device_status(void* stream, unsigned int* status, int clear);
 
@@ -171,7 +176,11 @@ long long ttt_linear_host_workspace_bytes(int B, int H, long long L, int d, int 
  * freed) and allocates no device memory; concurrent calls are serialised while they enqueue.
  * (No counterpart on the pages: the walkthrough's tensors are already on the device.)
  * Errors as ttt_linear_forward, plus TTT_ERR_ARG for a missing or too small workspace or a bad
- * chunk_batches, TTT_ERR_ALIGN for a misaligned workspace.
+ * chunk_batches, TTT_ERR_ALIGN for a misaligned workspace.  All of these are found before
+ * anything is enqueued.  A TTT_ERR_CUDA, however, can come after the copies and scans of earlier
+ * chunks are already enqueued on `stream` and on the copy stream: after such a failure,
+ * synchronise `stream` before reusing the workspace or the host buffers, and treat the outputs
+ * as undefined.
  */
 int ttt_linear_forward_host(const void* XQ, const void* XK, const void* XV, const float* lr,
                             const float* token_eta, const float* W0, const float* b0,

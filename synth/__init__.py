@@ -102,7 +102,8 @@ class Workload:
 
     kind: "linear" (TTT-Linear prefill), "mlp" (TTT-MLP prefill) or "decode".
     dtype: "f32" or "bf16" for XQ/XK/XV (and out); state and lr are always fp32.
-    x_std: std of XQ/XK/XV; ln: "unit" (ln_w=1, ln_b=0) or "random" (1+N(0,.1), N(0,.1)).
+    x_std: std of XQ/XK/XV; ln: "unit" (ln_w=1, ln_b=0) or "random" (1+N(0,ln_w_std),
+    N(0,ln_b_std)); w_std: std of the initial weights (W0, or W1 and W2 for TTT-MLP).
     """
     name: str
     kind: str
@@ -114,6 +115,9 @@ class Workload:
     dtype: str = "bf16"
     x_std: float = 0.125
     ln: str = "random"
+    w_std: float = 0.02
+    ln_w_std: float = 0.1
+    ln_b_std: float = 0.1
     hidden: int = 256
     seed: int = SEED_BASE
     eps: float = 1e-6
@@ -206,19 +210,19 @@ def state_inputs(w: Workload) -> dict:
     out = {}
     if w.kind == "mlp":
         h = w.hidden
-        out["W1"] = normal(w.seed, TAG["W1"], H * d * h, 0, 0.0, 0.02).reshape(H, d, h)
+        out["W1"] = normal(w.seed, TAG["W1"], H * d * h, 0, 0.0, w.w_std).reshape(H, d, h)
         out["b1"] = np.zeros((H, h), np.float32)
-        out["W2"] = normal(w.seed, TAG["W2"], H * h * d, 0, 0.0, 0.02).reshape(H, h, d)
+        out["W2"] = normal(w.seed, TAG["W2"], H * h * d, 0, 0.0, w.w_std).reshape(H, h, d)
         out["b2"] = np.zeros((H, d), np.float32)
     else:
-        out["W0"] = normal(w.seed, TAG["W0"], H * d * d, 0, 0.0, 0.02).reshape(H, d, d)
+        out["W0"] = normal(w.seed, TAG["W0"], H * d * d, 0, 0.0, w.w_std).reshape(H, d, d)
         out["b0"] = np.zeros((H, d), np.float32)
     if w.ln == "unit":
         out["ln_w"] = np.ones((H, d), np.float32)
         out["ln_b"] = np.zeros((H, d), np.float32)
     else:
-        out["ln_w"] = normal(w.seed, TAG["LNW"], H * d, 0, 1.0, 0.1).reshape(H, d)
-        out["ln_b"] = normal(w.seed, TAG["LNB"], H * d, 0, 0.0, 0.1).reshape(H, d)
+        out["ln_w"] = normal(w.seed, TAG["LNW"], H * d, 0, 1.0, w.ln_w_std).reshape(H, d)
+        out["ln_b"] = normal(w.seed, TAG["LNB"], H * d, 0, 0.0, w.ln_b_std).reshape(H, d)
     return out
 
 

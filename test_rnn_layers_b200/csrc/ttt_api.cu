@@ -154,11 +154,19 @@ int check_common(int B, int H, long long L, int d, int K, float eps, int dtype, 
 
 }  // namespace
 
-// The status word.  Kernels OR TTT_STATUS_* bits into it; ttt_device_status reads it.
+// The status word.  Kernels OR TTT_STATUS_* bits into it; ttt_device_status reads it.  A read
+// that clears takes the word with one atomic exchange into g_ttt_status_taken and copies that,
+// so a bit raised by a kernel still running on another stream is never lost between the read
+// and the clear.
 __device__ unsigned int g_ttt_status;
+__device__ unsigned int g_ttt_status_taken;
 
 namespace {
-unsigned int* status_word() {
+__global__ void status_take_kernel(unsigned int* word, unsigned int* taken) { *taken = atomicExch(word, 0u); }
+
+// Device address of a __device__ word on the current device (looked up once per device).
+template <unsigned int& kSym>
+unsigned int* device_word() {
     static std::mutex mu;
     static unsigned int* ptrs[256] = {};
     int dev = 0;
@@ -166,11 +174,13 @@ unsigned int* status_word() {
     std::lock_guard<std::mutex> lock(mu);
     if (!ptrs[dev]) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_ttt_status) != cudaSuccess) return nullptr;
+        if (cudaGetSymbolAddress(&p, kSym) != cudaSuccess) return nullptr;
         ptrs[dev] = static_cast<unsigned int*>(p);
     }
     return ptrs[dev];
 }
+
+unsigned int* status_word() { return device_word<g_ttt_status>(); }
 
 // The launch part of ttt_linear_forward, on validated device pointers: pick the kernel, build
 // its arguments (and tensor maps) and enqueue it on `st`.
@@ -310,11 +320,18 @@ int ttt_device_status(void* stream, unsigned int* status, int clear) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned int* word = status_word();
     if (!word) return fail(TTT_ERR_CUDA, "no device status word on the current device");
+    const unsigned int* src = word;
+    cudaError_t e = cudaSuccess;
+    if (clear) {  // read and clear in one atomic step on the device
+        unsigned int* taken = device_word<g_ttt_status_taken>();
+        if (!taken) return fail(TTT_ERR_CUDA, "no device status word on the current device");
+        status_take_kernel<<<1, 1, 0, st>>>(word, taken);
+        e = cudaGetLastError();
+        src = taken;
+    }
     unsigned int v = 0;
-    cudaError_t e = cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&v, src, sizeof(v), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    if (e == cudaSuccess && clear) e = cudaMemsetAsync(word, 0, sizeof(unsigned int), st);
-    if (e == cudaSuccess && clear) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
     *status = v;
     if (v & TTT_STATUS_TIMEOUT) return fail(TTT_ERR_TIMEOUT, "a kernel gave up on a bounded wait");
