@@ -454,44 +454,109 @@ def bench_decode(args, world, peaks, hist=False):
                          "algorithmic_bytes": int(nbytes)}}
 
 
-def cpu_baseline(seconds_target=12.0, chains_max=256):
-    """The oracle (fp64, single-threaded, as written) on a bounded sample of the 1B workload."""
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    """Cores this process may run on (its CPU affinity set)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_chains(w, ids):
+    """Inputs of the listed chains of a workload as float64 arrays (so the oracle's wrapper makes
+    no copies while it is timed), generated before any timing."""
+    out = []
+    for c in ids:
+        xs = synth.linear_inputs(w, chains=[c])
+        h = c % w.H
+        out.append(tuple(np.ascontiguousarray(a, np.float64) for a in
+                         (xs["XQ"][0], xs["XK"][0], xs["XV"][0], xs["lr"][0], xs["W0"][h], xs["b0"][h],
+                          xs["ln_w"][h], xs["ln_b"][h])))
+    return out
+
+
+def _time_oracle(fn, samples, threads, seconds, K, eps):
+    """Run fn(*sample, K, eps) over the samples round-robin on `threads` host threads (each call
+    single-threaded; ctypes releases the GIL) until `seconds` have passed; returns (chains done,
+    wall seconds)."""
+    done = [0] * threads
+    start = threading.Barrier(threads + 1)
+    deadline = [0.0]
+
+    def worker(i):
+        start.wait()
+        j = i
+        while True:
+            fn(*samples[j % len(samples)], K, eps)
+            done[i] += 1
+            j += threads
+            if time.perf_counter() >= deadline[0]:
+                return
+
+    ts = [threading.Thread(target=worker, args=(i,)) for i in range(threads)]
+    for t in ts:
+        t.start()
+    t0 = time.perf_counter()
+    deadline[0] = t0 + seconds
+    start.wait()
+    for t in ts:
+        t.join()
+    return sum(done), time.perf_counter() - t0
+
+
+def cpu_baseline(seconds_each=3.5):
+    """The oracle as it stands, timed on the host on a bounded sample of the 1B workload
+    (chains of L = 8200): the fp64 parity build and the float build of the same source, each on
+    one core and with the chains spread over every core this process may use (one
+    single-threaded oracle call per thread, no change to the oracle)."""
     import oracle
     w = synth.workload(2, L=8200)
-    o = oracle.default()
-    done, tokens, t_total = 0, 0, 0.0
-    chains = []
-    while done < chains_max and t_total < seconds_target:
-        c = (done * 37) % w.chains
-        xs = synth.linear_inputs(w, chains=[c])
-        t0 = time.perf_counter()
-        o.linear_forward(xs["XQ"], xs["XK"], xs["XV"], xs["lr"], xs["W0"], xs["b0"], xs["ln_w"], xs["ln_b"],
-                         w.K, w.eps, chains=[c])
-        t_total += time.perf_counter() - t0
-        done += 1
-        tokens += w.L
-        chains.append(c)
-    return {"value": round(tokens / t_total, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} of {w.chains} chains of the 1B workload (L={w.L} each), fp64 oracle, "
-                      f"{t_total:.1f} s of CPU time"}
+    n = host_cores()
+    samples = _oracle_chains(w, [(i * 37) % w.chains for i in range(8)])
+    o64, o32 = oracle.default(), oracle.OracleF32()
+    res = {}
+    for name, fn in (("f64", o64.linear_chain), ("f32", o32.linear_chain)):
+        for cores in sorted({1, n}):
+            chains, wall = _time_oracle(fn, samples, cores, seconds_each, w.K, w.eps)
+            res[f"{name}_{cores}core"] = {"value": round(chains * w.L / wall, 1), "chains": chains,
+                                          "seconds": round(wall, 2)}
+    top = res[f"f64_{n}core"]
+    return {"value": top["value"], "unit": "tokens/s", "cores": n, "kind": "oracle", "cpu_model": cpu_model(),
+            "sample": f"chains of the 1B workload (L={w.L} each) on {n} host threads for ~{seconds_each} s, "
+                      f"fp64 oracle ({top['chains']} chains); also the float build and 1 core",
+            "runs": res}
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the CPU oracle, as it stands, on the same workload and metric; each
-    step a bounded sample (4 chains of L=8200)."""
+    """The reference arm: the CPU oracle, as it stands, on the same workload and metric.  Each
+    step runs one chain (L = 8200) per host core, one single-threaded oracle call per thread."""
     if rank != 0:
         return
     import oracle
     w = synth.workload(2, L=8200)
+    n = host_cores()
     o = oracle.default()
-    per_step = 4
-    samples = [synth.linear_inputs(w, chains=[(i * 53) % w.chains]) for i in range(per_step)]
-    ids = [(i * 53) % w.chains for i in range(per_step)]
+    samples = _oracle_chains(w, [(i * 53) % w.chains for i in range(min(n, 16))])
 
     def step():
-        for c, xs in zip(ids, samples):
-            o.linear_forward(xs["XQ"], xs["XK"], xs["XV"], xs["lr"], xs["W0"], xs["b0"], xs["ln_w"], xs["ln_b"],
-                             w.K, w.eps, chains=[c])
+        ts = [threading.Thread(target=o.linear_chain, args=(*samples[i % len(samples)], w.K, w.eps))
+              for i in range(n)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
 
     for _ in range(args.warmup):
         step()
@@ -499,16 +564,18 @@ def run_reference(args, world, rank):
     for _ in range(args.steps):
         step()
     dt = (time.perf_counter() - t0) / args.steps
-    value = per_step * w.L / dt
+    value = n * w.L / dt
     print(json.dumps({
         "impl": "reference", "metric": "TTT layer tokens/sec (1B shapes, B200) and % of per-layer roofline",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded generator, synth/)",
         "config": {"workload": "ttt_linear_prefill_1b_layer", "B": w.B, "H": w.H, "L": w.L, "d": D,
-                   "mini_batch": w.K, "sample_per_step": f"{per_step} chains"},
-        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step} chains of L={w.L} per step, fp64 oracle, single thread"},
+                   "mini_batch": w.K, "sample_per_step": f"{n} chains, one per host core"},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": n, "kind": "oracle",
+                         "cpu_model": cpu_model(),
+                         "sample": f"{n} chains of L={w.L} per step, one single-threaded fp64 oracle call per "
+                                   f"host thread"},
         "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

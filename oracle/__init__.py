@@ -18,14 +18,23 @@ _SRC = os.path.join(_HERE, "ttt_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libttt_oracle.so")
 
 
-def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
-    """Compile the oracle with gcc: plain -O2, no fast-math, no FMA contraction."""
+_LIB_F32_PATH = os.path.join(_HERE, "libttt_oracle_f32.so")
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH, real: str = "double") -> str:
+    """Compile the oracle with gcc: plain -O2, no fast-math, no FMA contraction.  real="float"
+    builds the same source in single precision (timed as a CPU baseline, never a parity
+    reference)."""
     if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
         tmp = out + f".{os.getpid()}.tmp"
         subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-std=c99",
-                               "-o", tmp, src, "-lm"])
+                               f"-DORACLE_REAL={real}", "-o", tmp, src, "-lm"])
         os.replace(tmp, out)
     return out
+
+
+def build_f32(force: bool = False) -> str:
+    return build(force, _SRC, _LIB_F32_PATH, "float")
 
 
 _D = ctypes.POINTER(ctypes.c_double)
@@ -182,6 +191,32 @@ class Oracle:
                                            self._p(b2l))
         self._check(rc, "ttt_mlp_chain")
         return {"out": out, "W1_last": W1l, "b1_last": b1l, "W2_last": W2l, "b2_last": b2l}
+
+
+class OracleF32:
+    """The float build of the same oracle source: TTT-Linear chains only, for timing (the CPU
+    baseline's single-precision figure).  Not a parity reference."""
+
+    def __init__(self):
+        lib = ctypes.CDLL(build_f32())
+        F = ctypes.POINTER(ctypes.c_float)
+        lib.oracle_ttt_linear_chain.argtypes = [F, F, F, F, F, F, F, F, F, _LL, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_float, F, F, F, F, F]
+        lib.oracle_ttt_linear_chain.restype = ctypes.c_int
+        self.lib = lib
+
+    def linear_chain(self, xq, xk, xv, lr, W0, b0, ln_w, ln_b, K, eps):
+        f = lambda a: np.ascontiguousarray(a, dtype=np.float32)
+        xq, xk, xv, lr, W0, b0, ln_w, ln_b = map(f, (xq, xk, xv, lr, W0, b0, ln_w, ln_b))
+        L, d = xq.shape
+        out, W_last, b_last = np.empty((L, d), np.float32), np.empty((d, d), np.float32), np.empty(d, np.float32)
+        Wg, bg = np.empty((d, d), np.float32), np.empty(d, np.float32)
+        p = lambda a: a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+        rc = self.lib.oracle_ttt_linear_chain(p(xq), p(xk), p(xv), p(lr), None, p(W0), p(b0), p(ln_w), p(ln_b),
+                                              L, d, K, eps, p(out), p(W_last), p(b_last), p(Wg), p(bg))
+        if rc != 0:
+            raise ValueError(f"float oracle rejected its arguments (rc={rc})")
+        return {"out": out, "W_last": W_last, "b_last": b_last}
 
 
 _default = None

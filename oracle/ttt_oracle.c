@@ -1,6 +1,10 @@
 /*
  * ttt_oracle.c -- plain, slow, single-threaded CPU oracle of the TTT scan, in double.
  *
+ * The scalar type is `real`: double unless ORACLE_REAL says otherwise.  The parity build is
+ * the double one; a float build of the same source (-DORACLE_REAL=float) is only timed, as
+ * the CPU baseline's single-precision figure.
+ *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load this file:
  * only the tests, the smoke check and the bench's CPU-baseline leg use it.  It shares no
  * code, header, table or helper with the CUDA library.
@@ -38,6 +42,11 @@
 #include <stdlib.h>
 #include <string.h>
 
+#ifndef ORACLE_REAL
+#define ORACLE_REAL double
+#endif
+typedef ORACLE_REAL real;
+
 #define ORACLE_OK 0
 #define ORACLE_ERR_ARG -1
 
@@ -62,11 +71,11 @@ int oracle_partition(long long L, int K, long long* n_full, long long* rem) {
 /* ---------------------------------------------------------------------------------------- */
 
 /* mean and sigma = sqrt(biased variance + eps) of one row of d values */
-static void ln_stats(const double* z, int d, double eps, double* mu, double* sigma) {
-    double s = 0.0;
+static void ln_stats(const real* z, int d, real eps, real* mu, real* sigma) {
+    real s = 0.0;
     for (int c = 0; c < d; ++c) s += z[c];
-    double m = s / d;
-    double v = 0.0;
+    real m = s / d;
+    real v = 0.0;
     for (int c = 0; c < d; ++c) v += (z[c] - m) * (z[c] - m);
     v /= d;
     *mu = m;
@@ -74,9 +83,9 @@ static void ln_stats(const double* z, int d, double eps, double* mu, double* sig
 }
 
 /* y = ln_w * (u - mu) / sigma + ln_b */
-static void ln_forward(const double* u, const double* ln_w, const double* ln_b, int d, double eps,
-                       double* y) {
-    double mu, sigma;
+static void ln_forward(const real* u, const real* ln_w, const real* ln_b, int d, real eps,
+                       real* y) {
+    real mu, sigma;
     ln_stats(u, d, eps, &mu, &sigma);
     for (int c = 0; c < d; ++c) y[c] = ln_w[c] * (u[c] - mu) / sigma + ln_b[c];
 }
@@ -84,14 +93,14 @@ static void ln_forward(const double* u, const double* ln_w, const double* ln_b, 
 /* g = d/dz of 1/2 * || ln_w * xhat + ln_b - tgt ||^2, xhat = (z - mu) / sigma.
  * With q = ln_w * (ln_w * xhat + ln_b - tgt) (the gradient w.r.t. xhat), the LayerNorm
  * backward gives g_c = (d q_c - sum q - xhat_c * sum(q * xhat)) / (d sigma). */
-static void lnl2_grad(const double* z, const double* tgt, const double* ln_w, const double* ln_b,
-                      int d, double eps, double* xhat, double* q, double* g) {
-    double mu, sigma;
+static void lnl2_grad(const real* z, const real* tgt, const real* ln_w, const real* ln_b,
+                      int d, real eps, real* xhat, real* q, real* g) {
+    real mu, sigma;
     ln_stats(z, d, eps, &mu, &sigma);
-    double sq = 0.0, sqx = 0.0;
+    real sq = 0.0, sqx = 0.0;
     for (int c = 0; c < d; ++c) {
         xhat[c] = (z[c] - mu) / sigma;
-        double r = ln_w[c] * xhat[c] + ln_b[c] - tgt[c];
+        real r = ln_w[c] * xhat[c] + ln_b[c] - tgt[c];
         q[c] = ln_w[c] * r;
         sq += q[c];
         sqx += q[c] * xhat[c];
@@ -100,35 +109,35 @@ static void lnl2_grad(const double* z, const double* tgt, const double* ln_w, co
 }
 
 /* Exported for the gradient pins (finite differences, autograd). */
-int oracle_lnl2_grad(const double* z, const double* tgt, const double* ln_w, const double* ln_b,
-                     int d, double eps, double* g) {
+int oracle_lnl2_grad(const real* z, const real* tgt, const real* ln_w, const real* ln_b,
+                     int d, real eps, real* g) {
     if (d < 1 || !z || !tgt || !ln_w || !ln_b || !g) return ORACLE_ERR_ARG;
-    double* tmp = (double*)malloc(sizeof(double) * 2 * d);
+    real* tmp = (real*)malloc(sizeof(real) * 2 * d);
     if (!tmp) return ORACLE_ERR_ARG;
     lnl2_grad(z, tgt, ln_w, ln_b, d, eps, tmp, tmp + d, g);
     free(tmp);
     return ORACLE_OK;
 }
 
-int oracle_ln_forward(const double* u, const double* ln_w, const double* ln_b, int d, double eps,
-                      double* y) {
+int oracle_ln_forward(const real* u, const real* ln_w, const real* ln_b, int d, real eps,
+                      real* y) {
     if (d < 1 || !u || !ln_w || !ln_b || !y) return ORACLE_ERR_ARG;
     ln_forward(u, ln_w, ln_b, d, eps, y);
     return ORACLE_OK;
 }
 
 /* token_eta_i: the per-position scale of the accumulated grad (default 1/(i+1)). */
-static double token_eta_at(const double* token_eta, int i) {
-    return token_eta ? token_eta[i] : 1.0 / (double)(i + 1);
+static real token_eta_at(const real* token_eta, int i) {
+    return token_eta ? token_eta[i] : 1.0 / (real)(i + 1);
 }
 
 /* y[c] = sum_a x[a] * M[a][c] + bias[c], M is rows x cols row-major */
-static void row_times(const double* x, const double* M, const double* bias, int rows, int cols,
-                      double* y) {
+static void row_times(const real* x, const real* M, const real* bias, int rows, int cols,
+                      real* y) {
     for (int c = 0; c < cols; ++c) y[c] = bias ? bias[c] : 0.0;
     for (int a = 0; a < rows; ++a) {
-        double xa = x[a];
-        const double* Ma = M + (size_t)a * cols;
+        real xa = x[a];
+        const real* Ma = M + (size_t)a * cols;
         for (int c = 0; c < cols; ++c) y[c] += xa * Ma[c];
     }
 }
@@ -139,15 +148,15 @@ static void row_times(const double* x, const double* M, const double* bias, int 
 /* from the carried params), TTTLinear.ttt (initial params W1, b1 tiled over the batch;       */
 /* scan over mini-batches), compute_mini_batch primal branch.                                 */
 /* ---------------------------------------------------------------------------------------- */
-int oracle_ttt_linear_chain(const double* xq, const double* xk, const double* xv, /* [L][d] */
-                            const double* lr,                                     /* [L] */
-                            const double* token_eta,                              /* [K] or NULL */
-                            const double* W0, const double* b0,                   /* [d][d], [d] */
-                            const double* ln_w, const double* ln_b,               /* [d] */
-                            long long L, int d, int K, double eps,
-                            double* out,                                          /* [L][d] */
-                            double* W_last, double* b_last,                       /* [d][d], [d] */
-                            double* W_grad_tail, double* b_grad_tail)             /* nullable */
+int oracle_ttt_linear_chain(const real* xq, const real* xk, const real* xv, /* [L][d] */
+                            const real* lr,                                     /* [L] */
+                            const real* token_eta,                              /* [K] or NULL */
+                            const real* W0, const real* b0,                   /* [d][d], [d] */
+                            const real* ln_w, const real* ln_b,               /* [d] */
+                            long long L, int d, int K, real eps,
+                            real* out,                                          /* [L][d] */
+                            real* W_last, real* b_last,                       /* [d][d], [d] */
+                            real* W_grad_tail, real* b_grad_tail)             /* nullable */
 {
     if (L < 0 || d < 1 || K < 1 || !W0 || !b0 || !ln_w || !ln_b || !W_last || !b_last)
         return ORACLE_ERR_ARG;
@@ -156,27 +165,27 @@ int oracle_ttt_linear_chain(const double* xq, const double* xk, const double* xv
     oracle_partition(L, K, &n_full, &rem);
 
     size_t dd = (size_t)d * d;
-    double* W = (double*)malloc(sizeof(double) * dd);
-    double* b = (double*)malloc(sizeof(double) * d);
-    double* G = (double*)malloc(sizeof(double) * dd);   /* sum_{j<=i} lr_j xk_j^T g_j */
-    double* gb = (double*)malloc(sizeof(double) * d);   /* sum_{j<=i} lr_j g_j */
-    double* Wbar = (double*)malloc(sizeof(double) * dd);
-    double* bbar = (double*)malloc(sizeof(double) * d);
-    double* g = (double*)malloc(sizeof(double) * (size_t)K * d); /* grads of the mini-batch */
-    double* z = (double*)malloc(sizeof(double) * d);
-    double* tgt = (double*)malloc(sizeof(double) * d);
-    double* xhat = (double*)malloc(sizeof(double) * d);
-    double* q = (double*)malloc(sizeof(double) * d);
-    double* y = (double*)malloc(sizeof(double) * d);
+    real* W = (real*)malloc(sizeof(real) * dd);
+    real* b = (real*)malloc(sizeof(real) * d);
+    real* G = (real*)malloc(sizeof(real) * dd);   /* sum_{j<=i} lr_j xk_j^T g_j */
+    real* gb = (real*)malloc(sizeof(real) * d);   /* sum_{j<=i} lr_j g_j */
+    real* Wbar = (real*)malloc(sizeof(real) * dd);
+    real* bbar = (real*)malloc(sizeof(real) * d);
+    real* g = (real*)malloc(sizeof(real) * (size_t)K * d); /* grads of the mini-batch */
+    real* z = (real*)malloc(sizeof(real) * d);
+    real* tgt = (real*)malloc(sizeof(real) * d);
+    real* xhat = (real*)malloc(sizeof(real) * d);
+    real* q = (real*)malloc(sizeof(real) * d);
+    real* y = (real*)malloc(sizeof(real) * d);
     if (!W || !b || !G || !gb || !Wbar || !bbar || !g || !z || !tgt || !xhat || !q || !y) {
         free(W); free(b); free(G); free(gb); free(Wbar); free(bbar); free(g);
         free(z); free(tgt); free(xhat); free(q); free(y);
         return ORACLE_ERR_ARG;
     }
-    memcpy(W, W0, sizeof(double) * dd);
-    memcpy(b, b0, sizeof(double) * d);
-    memset(G, 0, sizeof(double) * dd);
-    memset(gb, 0, sizeof(double) * d);
+    memcpy(W, W0, sizeof(real) * dd);
+    memcpy(b, b0, sizeof(real) * d);
+    memset(G, 0, sizeof(real) * dd);
+    memset(gb, 0, sizeof(real) * d);
 
     long long n_mb = n_full + (rem > 0 ? 1 : 0);
     for (long long m = 0; m < n_mb; ++m) {
@@ -186,50 +195,50 @@ int oracle_ttt_linear_chain(const double* xq, const double* xk, const double* xv
 
         /* g_j = ln_fused_l2_bwd(xk_j W + b, xv_j - xk_j), all at the mini-batch-start state */
         for (int j = 0; j < Km; ++j) {
-            const double* xkj = xk + (size_t)(t0 + j) * d;
-            const double* xvj = xv + (size_t)(t0 + j) * d;
+            const real* xkj = xk + (size_t)(t0 + j) * d;
+            const real* xvj = xv + (size_t)(t0 + j) * d;
             row_times(xkj, W, b, d, d, z);
             for (int c = 0; c < d; ++c) tgt[c] = xvj[c] - xkj[c];
             lnl2_grad(z, tgt, ln_w, ln_b, d, eps, xhat, q, g + (size_t)j * d);
         }
 
         /* primal: accumulate lr-weighted grads token by token and evaluate at W_bar_i */
-        memset(G, 0, sizeof(double) * dd);
-        memset(gb, 0, sizeof(double) * d);
+        memset(G, 0, sizeof(real) * dd);
+        memset(gb, 0, sizeof(real) * d);
         for (int i = 0; i < Km; ++i) {
-            const double* xki = xk + (size_t)(t0 + i) * d;
-            const double* xqi = xq + (size_t)(t0 + i) * d;
-            const double* gi = g + (size_t)i * d;
-            double lri = lr[t0 + i];
+            const real* xki = xk + (size_t)(t0 + i) * d;
+            const real* xqi = xq + (size_t)(t0 + i) * d;
+            const real* gi = g + (size_t)i * d;
+            real lri = lr[t0 + i];
             for (int a = 0; a < d; ++a)
                 for (int c = 0; c < d; ++c) G[(size_t)a * d + c] += lri * xki[a] * gi[c];
             for (int c = 0; c < d; ++c) gb[c] += lri * gi[c];
 
-            double ti = token_eta_at(token_eta, i);
+            real ti = token_eta_at(token_eta, i);
             for (size_t e = 0; e < dd; ++e) Wbar[e] = W[e] - ti * G[e];
             for (int c = 0; c < d; ++c) bbar[c] = b[c] - ti * gb[c];
 
             /* out_i = xq_i + LN(xq_i W_bar_i + b_bar_i) */
             row_times(xqi, Wbar, bbar, d, d, z);
             ln_forward(z, ln_w, ln_b, d, eps, y);
-            double* oi = out + (size_t)(t0 + i) * d;
+            real* oi = out + (size_t)(t0 + i) * d;
             for (int c = 0; c < d; ++c) oi[c] = xqi[c] + y[c];
         }
         if (full) {
-            memcpy(W, Wbar, sizeof(double) * dd);
-            memcpy(b, bbar, sizeof(double) * d);
+            memcpy(W, Wbar, sizeof(real) * dd);
+            memcpy(b, bbar, sizeof(real) * d);
         }
     }
 
-    memcpy(W_last, W, sizeof(double) * dd);
-    memcpy(b_last, b, sizeof(double) * d);
+    memcpy(W_last, W, sizeof(real) * dd);
+    memcpy(b_last, b, sizeof(real) * d);
     if (W_grad_tail) {
-        if (rem > 0) memcpy(W_grad_tail, G, sizeof(double) * dd);
-        else memset(W_grad_tail, 0, sizeof(double) * dd);
+        if (rem > 0) memcpy(W_grad_tail, G, sizeof(real) * dd);
+        else memset(W_grad_tail, 0, sizeof(real) * dd);
     }
     if (b_grad_tail) {
-        if (rem > 0) memcpy(b_grad_tail, gb, sizeof(double) * d);
-        else memset(b_grad_tail, 0, sizeof(double) * d);
+        if (rem > 0) memcpy(b_grad_tail, gb, sizeof(real) * d);
+        else memset(b_grad_tail, 0, sizeof(real) * d);
     }
     free(W); free(b); free(G); free(gb); free(Wbar); free(bbar); free(g);
     free(z); free(tgt); free(xhat); free(q); free(y);
@@ -244,25 +253,25 @@ int oracle_ttt_linear_chain(const double* xq, const double* xk, const double* xv
 /* The token sits at position p = offset % K of its mini-batch; W, b are the state committed  */
 /* at the last mini-batch boundary; W_grad, b_grad hold sum_{j<p} lr_j xk_j^T g_j, ...        */
 /* ---------------------------------------------------------------------------------------- */
-int oracle_ttt_linear_decode_chain(const double* xq, const double* xk, const double* xv, /* [d] */
-                                   double lr, const double* token_eta, /* [K] or NULL */
-                                   const double* ln_w, const double* ln_b,
-                                   double* W, double* b, double* W_grad, double* b_grad,
-                                   int d, int K, long long offset, double eps, double* out,
+int oracle_ttt_linear_decode_chain(const real* xq, const real* xk, const real* xv, /* [d] */
+                                   real lr, const real* token_eta, /* [K] or NULL */
+                                   const real* ln_w, const real* ln_b,
+                                   real* W, real* b, real* W_grad, real* b_grad,
+                                   int d, int K, long long offset, real eps, real* out,
                                    int* committed) {
     if (d < 1 || K < 1 || offset < 0 || !xq || !xk || !xv || !ln_w || !ln_b || !W || !b ||
         !W_grad || !b_grad || !out)
         return ORACLE_ERR_ARG;
     int p = (int)(offset % K);
     size_t dd = (size_t)d * d;
-    double* z = (double*)malloc(sizeof(double) * d);
-    double* tgt = (double*)malloc(sizeof(double) * d);
-    double* xhat = (double*)malloc(sizeof(double) * d);
-    double* q = (double*)malloc(sizeof(double) * d);
-    double* g = (double*)malloc(sizeof(double) * d);
-    double* y = (double*)malloc(sizeof(double) * d);
-    double* Wbar = (double*)malloc(sizeof(double) * dd);
-    double* bbar = (double*)malloc(sizeof(double) * d);
+    real* z = (real*)malloc(sizeof(real) * d);
+    real* tgt = (real*)malloc(sizeof(real) * d);
+    real* xhat = (real*)malloc(sizeof(real) * d);
+    real* q = (real*)malloc(sizeof(real) * d);
+    real* g = (real*)malloc(sizeof(real) * d);
+    real* y = (real*)malloc(sizeof(real) * d);
+    real* Wbar = (real*)malloc(sizeof(real) * dd);
+    real* bbar = (real*)malloc(sizeof(real) * d);
     if (!z || !tgt || !xhat || !q || !g || !y || !Wbar || !bbar) {
         free(z); free(tgt); free(xhat); free(q); free(g); free(y); free(Wbar); free(bbar);
         return ORACLE_ERR_ARG;
@@ -273,7 +282,7 @@ int oracle_ttt_linear_decode_chain(const double* xq, const double* xk, const dou
     for (int a = 0; a < d; ++a)
         for (int c = 0; c < d; ++c) W_grad[(size_t)a * d + c] += lr * xk[a] * g[c];
     for (int c = 0; c < d; ++c) b_grad[c] += lr * g[c];
-    double tp = token_eta_at(token_eta, p);
+    real tp = token_eta_at(token_eta, p);
     for (size_t e = 0; e < dd; ++e) Wbar[e] = W[e] - tp * W_grad[e];
     for (int c = 0; c < d; ++c) bbar[c] = b[c] - tp * b_grad[c];
     row_times(xq, Wbar, bbar, d, d, z);
@@ -281,10 +290,10 @@ int oracle_ttt_linear_decode_chain(const double* xq, const double* xk, const dou
     for (int c = 0; c < d; ++c) out[c] = xq[c] + y[c];
     int commit = (p == K - 1);
     if (commit) {
-        memcpy(W, Wbar, sizeof(double) * dd);
-        memcpy(b, bbar, sizeof(double) * d);
-        memset(W_grad, 0, sizeof(double) * dd);
-        memset(b_grad, 0, sizeof(double) * d);
+        memcpy(W, Wbar, sizeof(real) * dd);
+        memcpy(b, bbar, sizeof(real) * d);
+        memset(W_grad, 0, sizeof(real) * dd);
+        memset(b_grad, 0, sizeof(real) * d);
     }
     if (committed) *committed = commit;
     free(z); free(tgt); free(xhat); free(q); free(g); free(y); free(Wbar); free(bbar);
@@ -295,20 +304,20 @@ int oracle_ttt_linear_decode_chain(const double* xq, const double* xk, const dou
 /* TTT-MLP ([readme]: the hidden state is a two-layer MLP; [walkthrough]: "TTTMLP is two     */
 /* TTTLinear stacked").  f(x) = gelu(x W1 + b1) W2 + b2 with the tanh form of GELU.           */
 /* ---------------------------------------------------------------------------------------- */
-static double gelu_tanh(double x) {
-    const double k = 0.79788456080286535588; /* sqrt(2/pi) */
-    double u = k * (x + 0.044715 * x * x * x);
+static real gelu_tanh(real x) {
+    const real k = 0.79788456080286535588; /* sqrt(2/pi) */
+    real u = k * (x + 0.044715 * x * x * x);
     return 0.5 * x * (1.0 + tanh(u));
 }
 
-static double gelu_tanh_deriv(double x) {
-    const double k = 0.79788456080286535588;
-    double u = k * (x + 0.044715 * x * x * x);
-    double th = tanh(u);
+static real gelu_tanh_deriv(real x) {
+    const real k = 0.79788456080286535588;
+    real u = k * (x + 0.044715 * x * x * x);
+    real th = tanh(u);
     return 0.5 * (1.0 + th) + 0.5 * x * (1.0 - th * th) * k * (1.0 + 3.0 * 0.044715 * x * x);
 }
 
-int oracle_gelu_tanh(const double* x, long long n, double* y, double* dy) {
+int oracle_gelu_tanh(const real* x, long long n, real* y, real* dy) {
     if (n < 0 || !x) return ORACLE_ERR_ARG;
     for (long long i = 0; i < n; ++i) {
         if (y) y[i] = gelu_tanh(x[i]);
@@ -317,14 +326,14 @@ int oracle_gelu_tanh(const double* x, long long n, double* y, double* dy) {
     return ORACLE_OK;
 }
 
-int oracle_ttt_mlp_chain(const double* xq, const double* xk, const double* xv, /* [L][d] */
-                         const double* lr, const double* token_eta,
-                         const double* W1_0, const double* b1_0, /* [d][h], [h] */
-                         const double* W2_0, const double* b2_0, /* [h][d], [d] */
-                         const double* ln_w, const double* ln_b,
-                         long long L, int d, int h, int K, double eps,
-                         double* out,
-                         double* W1_last, double* b1_last, double* W2_last, double* b2_last) {
+int oracle_ttt_mlp_chain(const real* xq, const real* xk, const real* xv, /* [L][d] */
+                         const real* lr, const real* token_eta,
+                         const real* W1_0, const real* b1_0, /* [d][h], [h] */
+                         const real* W2_0, const real* b2_0, /* [h][d], [d] */
+                         const real* ln_w, const real* ln_b,
+                         long long L, int d, int h, int K, real eps,
+                         real* out,
+                         real* W1_last, real* b1_last, real* W2_last, real* b2_last) {
     if (L < 0 || d < 1 || h < 1 || K < 1 || !W1_0 || !b1_0 || !W2_0 || !b2_0 || !ln_w || !ln_b ||
         !W1_last || !b1_last || !W2_last || !b2_last)
         return ORACLE_ERR_ARG;
@@ -333,28 +342,28 @@ int oracle_ttt_mlp_chain(const double* xq, const double* xk, const double* xv, /
     oracle_partition(L, K, &n_full, &rem);
     size_t dh = (size_t)d * h;
 
-    double* W1 = (double*)malloc(sizeof(double) * dh);
-    double* b1 = (double*)malloc(sizeof(double) * h);
-    double* W2 = (double*)malloc(sizeof(double) * dh);
-    double* b2 = (double*)malloc(sizeof(double) * d);
-    double* G1 = (double*)malloc(sizeof(double) * dh);
-    double* gb1 = (double*)malloc(sizeof(double) * h);
-    double* G2 = (double*)malloc(sizeof(double) * dh);
-    double* gb2 = (double*)malloc(sizeof(double) * d);
-    double* W1b = (double*)malloc(sizeof(double) * dh);
-    double* b1b = (double*)malloc(sizeof(double) * h);
-    double* W2b = (double*)malloc(sizeof(double) * dh);
-    double* b2b = (double*)malloc(sizeof(double) * d);
-    double* x2 = (double*)malloc(sizeof(double) * (size_t)K * h);  /* gelu(Z1_j) */
-    double* g1 = (double*)malloc(sizeof(double) * (size_t)K * h);  /* dl/dZ1_j */
-    double* g2 = (double*)malloc(sizeof(double) * (size_t)K * d);  /* dl/dZ2_j */
-    double* z1 = (double*)malloc(sizeof(double) * h);
-    double* a1 = (double*)malloc(sizeof(double) * h);
-    double* z2 = (double*)malloc(sizeof(double) * d);
-    double* tgt = (double*)malloc(sizeof(double) * d);
-    double* xhat = (double*)malloc(sizeof(double) * d);
-    double* q = (double*)malloc(sizeof(double) * d);
-    double* y = (double*)malloc(sizeof(double) * d);
+    real* W1 = (real*)malloc(sizeof(real) * dh);
+    real* b1 = (real*)malloc(sizeof(real) * h);
+    real* W2 = (real*)malloc(sizeof(real) * dh);
+    real* b2 = (real*)malloc(sizeof(real) * d);
+    real* G1 = (real*)malloc(sizeof(real) * dh);
+    real* gb1 = (real*)malloc(sizeof(real) * h);
+    real* G2 = (real*)malloc(sizeof(real) * dh);
+    real* gb2 = (real*)malloc(sizeof(real) * d);
+    real* W1b = (real*)malloc(sizeof(real) * dh);
+    real* b1b = (real*)malloc(sizeof(real) * h);
+    real* W2b = (real*)malloc(sizeof(real) * dh);
+    real* b2b = (real*)malloc(sizeof(real) * d);
+    real* x2 = (real*)malloc(sizeof(real) * (size_t)K * h);  /* gelu(Z1_j) */
+    real* g1 = (real*)malloc(sizeof(real) * (size_t)K * h);  /* dl/dZ1_j */
+    real* g2 = (real*)malloc(sizeof(real) * (size_t)K * d);  /* dl/dZ2_j */
+    real* z1 = (real*)malloc(sizeof(real) * h);
+    real* a1 = (real*)malloc(sizeof(real) * h);
+    real* z2 = (real*)malloc(sizeof(real) * d);
+    real* tgt = (real*)malloc(sizeof(real) * d);
+    real* xhat = (real*)malloc(sizeof(real) * d);
+    real* q = (real*)malloc(sizeof(real) * d);
+    real* y = (real*)malloc(sizeof(real) * d);
     void* all[] = {W1, b1, W2, b2, G1, gb1, G2, gb2, W1b, b1b, W2b, b2b, x2, g1, g2,
                    z1, a1, z2, tgt, xhat, q, y};
     int nall = (int)(sizeof(all) / sizeof(all[0]));
@@ -363,10 +372,10 @@ int oracle_ttt_mlp_chain(const double* xq, const double* xk, const double* xv, /
             for (int k = 0; k < nall; ++k) free(all[k]);
             return ORACLE_ERR_ARG;
         }
-    memcpy(W1, W1_0, sizeof(double) * dh);
-    memcpy(b1, b1_0, sizeof(double) * h);
-    memcpy(W2, W2_0, sizeof(double) * dh);
-    memcpy(b2, b2_0, sizeof(double) * d);
+    memcpy(W1, W1_0, sizeof(real) * dh);
+    memcpy(b1, b1_0, sizeof(real) * h);
+    memcpy(W2, W2_0, sizeof(real) * dh);
+    memcpy(b2, b2_0, sizeof(real) * d);
 
     long long n_mb = n_full + (rem > 0 ? 1 : 0);
     for (long long m = 0; m < n_mb; ++m) {
@@ -376,36 +385,36 @@ int oracle_ttt_mlp_chain(const double* xq, const double* xk, const double* xv, /
 
         /* forward and backward of the reconstruction loss at the mini-batch-start state */
         for (int j = 0; j < Km; ++j) {
-            const double* xkj = xk + (size_t)(t0 + j) * d;
-            const double* xvj = xv + (size_t)(t0 + j) * d;
+            const real* xkj = xk + (size_t)(t0 + j) * d;
+            const real* xvj = xv + (size_t)(t0 + j) * d;
             row_times(xkj, W1, b1, d, h, z1);
-            double* x2j = x2 + (size_t)j * h;
+            real* x2j = x2 + (size_t)j * h;
             for (int u = 0; u < h; ++u) x2j[u] = gelu_tanh(z1[u]);
             row_times(x2j, W2, b2, h, d, z2);
             for (int c = 0; c < d; ++c) tgt[c] = xvj[c] - xkj[c];
-            double* g2j = g2 + (size_t)j * d;
+            real* g2j = g2 + (size_t)j * d;
             lnl2_grad(z2, tgt, ln_w, ln_b, d, eps, xhat, q, g2j);
             /* dl/dZ1 = (dl/dZ2 W2^T) * gelu'(Z1) */
-            double* g1j = g1 + (size_t)j * h;
+            real* g1j = g1 + (size_t)j * h;
             for (int u = 0; u < h; ++u) {
-                double s = 0.0;
-                const double* W2u = W2 + (size_t)u * d;
+                real s = 0.0;
+                const real* W2u = W2 + (size_t)u * d;
                 for (int c = 0; c < d; ++c) s += g2j[c] * W2u[c];
                 g1j[u] = s * gelu_tanh_deriv(z1[u]);
             }
         }
 
-        memset(G1, 0, sizeof(double) * dh);
-        memset(gb1, 0, sizeof(double) * h);
-        memset(G2, 0, sizeof(double) * dh);
-        memset(gb2, 0, sizeof(double) * d);
+        memset(G1, 0, sizeof(real) * dh);
+        memset(gb1, 0, sizeof(real) * h);
+        memset(G2, 0, sizeof(real) * dh);
+        memset(gb2, 0, sizeof(real) * d);
         for (int i = 0; i < Km; ++i) {
-            const double* xki = xk + (size_t)(t0 + i) * d;
-            const double* xqi = xq + (size_t)(t0 + i) * d;
-            const double* x2i = x2 + (size_t)i * h;
-            const double* g1i = g1 + (size_t)i * h;
-            const double* g2i = g2 + (size_t)i * d;
-            double lri = lr[t0 + i];
+            const real* xki = xk + (size_t)(t0 + i) * d;
+            const real* xqi = xq + (size_t)(t0 + i) * d;
+            const real* x2i = x2 + (size_t)i * h;
+            const real* g1i = g1 + (size_t)i * h;
+            const real* g2i = g2 + (size_t)i * d;
+            real lri = lr[t0 + i];
             for (int a = 0; a < d; ++a)
                 for (int u = 0; u < h; ++u) G1[(size_t)a * h + u] += lri * xki[a] * g1i[u];
             for (int u = 0; u < h; ++u) gb1[u] += lri * g1i[u];
@@ -413,7 +422,7 @@ int oracle_ttt_mlp_chain(const double* xq, const double* xk, const double* xv, /
                 for (int c = 0; c < d; ++c) G2[(size_t)u * d + c] += lri * x2i[u] * g2i[c];
             for (int c = 0; c < d; ++c) gb2[c] += lri * g2i[c];
 
-            double ti = token_eta_at(token_eta, i);
+            real ti = token_eta_at(token_eta, i);
             for (size_t e = 0; e < dh; ++e) W1b[e] = W1[e] - ti * G1[e];
             for (int u = 0; u < h; ++u) b1b[u] = b1[u] - ti * gb1[u];
             for (size_t e = 0; e < dh; ++e) W2b[e] = W2[e] - ti * G2[e];
@@ -423,20 +432,20 @@ int oracle_ttt_mlp_chain(const double* xq, const double* xk, const double* xv, /
             for (int u = 0; u < h; ++u) a1[u] = gelu_tanh(z1[u]);
             row_times(a1, W2b, b2b, h, d, z2);
             ln_forward(z2, ln_w, ln_b, d, eps, y);
-            double* oi = out + (size_t)(t0 + i) * d;
+            real* oi = out + (size_t)(t0 + i) * d;
             for (int c = 0; c < d; ++c) oi[c] = xqi[c] + y[c];
         }
         if (full) {
-            memcpy(W1, W1b, sizeof(double) * dh);
-            memcpy(b1, b1b, sizeof(double) * h);
-            memcpy(W2, W2b, sizeof(double) * dh);
-            memcpy(b2, b2b, sizeof(double) * d);
+            memcpy(W1, W1b, sizeof(real) * dh);
+            memcpy(b1, b1b, sizeof(real) * h);
+            memcpy(W2, W2b, sizeof(real) * dh);
+            memcpy(b2, b2b, sizeof(real) * d);
         }
     }
-    memcpy(W1_last, W1, sizeof(double) * dh);
-    memcpy(b1_last, b1, sizeof(double) * h);
-    memcpy(W2_last, W2, sizeof(double) * dh);
-    memcpy(b2_last, b2, sizeof(double) * d);
+    memcpy(W1_last, W1, sizeof(real) * dh);
+    memcpy(b1_last, b1, sizeof(real) * h);
+    memcpy(W2_last, W2, sizeof(real) * dh);
+    memcpy(b2_last, b2, sizeof(real) * d);
     for (int k = 0; k < nall; ++k) free(all[k]);
     return ORACLE_OK;
 }

@@ -62,5 +62,16 @@ def test_reference_arm_prints_the_contract_line():
     assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] == 3 and d["value"] > 0
     assert d["config"]["workload"] == "ttt_linear_prefill_1b_layer"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["cpu_model"] and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
+
+
+def test_cpu_baseline_reports_both_precisions_and_the_cores():
+    """The bench's CPU baseline: the fp64 oracle and its float build, on 1 core and on every core
+    of the affinity set, with the CPU model (a short run)."""
+    cb = bench.cpu_baseline(seconds_each=0.3)
+    n = bench.host_cores()
+    assert cb["cores"] == n and cb["kind"] == "oracle" and cb["cpu_model"]
+    assert set(cb["runs"]) == {f"{p}_{c}core" for p in ("f64", "f32") for c in {1, n}}
+    assert cb["value"] == cb["runs"][f"f64_{n}core"]["value"] > 0
