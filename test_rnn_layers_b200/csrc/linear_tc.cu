@@ -1,4 +1,5 @@
-// linear_tc.cu -- TTT-Linear prefill, bf16 tensor-core kernel (fp32 accumulation, fp32 state).
+// linear_tc.cu -- TTT-Linear prefill on the tensor cores (bf16 activations, fp16 operands, fp32
+// accumulation, fp32 state).
 //
 // The method ("代码连连看——TTT", compute_mini_batch, dual branch), per chain and mini-batch of
 // K <= 16 tokens, state (W, b):
@@ -10,14 +11,23 @@
 //  * State in registers.  The fp32 master W^T (64x64) lives in mma.sync accumulator fragments:
 //    warp w owns output features 16w..16w+15 (rows 16w.. of W^T, eight m16n8 tiles).  The
 //    accumulator layout of W^T is exactly the B-operand layout of W for Z = XK W, so a
-//    mini-batch only rounds the accumulators to bf16 pairs, and the rank-K update of W is an MMA
+//    mini-batch only rounds the accumulators to fp16 pairs, and the rank-K update of W is an MMA
 //    accumulating straight into the same registers.  The bias b is one more fp32 accumulator
 //    column, updated by the same MMA against a column of ones and spread to the lanes that add
 //    it to Z and Zbar (in fp32) by four shuffles.  Nothing of the state round-trips memory.
 //  * Tensor cores for the dense contractions: Z and XQ W (16x64x64), XQ XK^T (16x16x64),
 //    M g (16x16x64, the two tril terms of the dual form folded into M = eta * tril(XQ XK^T + 1))
-//    and the update (64x16x64): m16n8k16 bf16 MMAs with fp32 accumulation.  g reaches the B
-//    operand of M g and the A operand of the update through movmatrix register transposes.
+//    and the update (64x16x64): m16n8k16 MMAs with fp16 operands and fp32 accumulation.  g
+//    reaches the B operand of M g and the A operand of the update through movmatrix register
+//    transposes.
+//  * Operand precision.  The state path (Z from W, the update from g) feeds back into itself for
+//    every mini-batch; with bf16 operands (8-bit significand) the rounding of W and g grows past
+//    1e-2 relative error on a few chains of the 1B-layer workload over its 512 updates, with
+//    fp16 operands (11-bit) every chain stays near 1e-3, at the same tensor throughput.  During
+//    mini-batch m the compute warps write the fp16 copy of the XQ and XK tiles of mini-batch
+//    m + 1 (one 16-byte chunk of each per thread; exact for the values bf16 inputs take up to
+//    |x| = 65504, larger ones saturate); the LayerNorm target, the residual and the tail grads
+//    read the bf16 tiles as loaded.
 //  * LayerNorm fused in registers: a thread holds 2 rows x 4 features; quads reduce by shuffles;
 //    the 4 warps' (sum, centred sum of squares) per row merge through shared memory with Chan's
 //    formula.  The loss gradient costs two 128-thread named barriers per mini-batch; the output
@@ -26,8 +36,9 @@
 //    and a few hundred bytes of row statistics per mini-batch.
 //  * A fifth, producer warp streams the inputs: a TMA ring of kStages mini-batches (XQ, XK, XV
 //    tiles, 128-byte swizzle, K rows of 128 bytes, from head-major [B,H,L,64] (3-D map) or
-//    token-major [B,L,H,64] (4-D map) activations alike) plus cp.async for lr, with a "full" mbarrier per stage
-//    (data landed) and an "empty" one (the four compute warps are done with it).  No multicast.
+//    token-major [B,L,H,64] (4-D map) activations alike) plus cp.async for lr, with a "full"
+//    mbarrier per stage (data landed; tested one mini-batch ahead) and an "empty" one (the four
+//    compute warps are done with it).  No multicast.
 //    Every mbarrier wait is bounded; on expiry the kernel raises the status word, drains its
 //    in-flight copies (bounded) and returns.
 #include "ttt_common.cuh"
@@ -47,6 +58,9 @@ struct __align__(1024) TcSmem {
     uint8_t xq[kStages][kTileBytes];
     uint8_t xk[kStages][kTileBytes];
     uint8_t xv[kStages][kTileBytes];
+    uint8_t xq16[kStages][kTileBytes];  // fp16 copies of XQ, XK (the MMA operands), same layout,
+                                        // written by the compute warps one mini-batch ahead
+    uint8_t xk16[kStages][kTileBytes];
     float gtail[TTT_KMAX][TTT_D];    // g in fp32 on the remainder mini-batch (tail grads)
     float lr[kStages][TTT_KMAX];
     float te[TTT_KMAX];
@@ -57,7 +71,6 @@ struct __align__(1024) TcSmem {
     uint64_t full[kStages];          // stage loaded (1 expect-tx arrival + 16 lr arrivals)
     uint64_t empty[kStages];         // stage consumed (one arrival per compute warp)
     int fail;                        // a compute warp gave up on a wait
-    int fail_m;                      // the mini-batch it gave up on
 };
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
@@ -65,6 +78,45 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 bc2(float a) { return make_float2(a, a); }
+
+// two floats -> fp16x2 (lo in bits [0,16)), round to nearest, magnitudes past 65504 saturate
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// bf16x2 -> fp16x2 (exact for magnitudes in fp16's range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+    return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, fp16 inputs, fp32 accumulators (in place in d[4])
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+// This thread's 16-byte chunk (of 128) of the XQ and XK tiles of a stage, converted to fp16.
+__device__ __forceinline__ void convert_chunk(uint32_t q_s, uint32_t k_s, uint32_t q16, uint32_t k16, uint32_t off) {
+    const uint4 vq = lds128(q_s + off), vk = lds128(k_s + off);
+    sts128(q16 + off, make_uint4(bf16x2_to_f16x2(vq.x), bf16x2_to_f16x2(vq.y), bf16x2_to_f16x2(vq.z),
+                                 bf16x2_to_f16x2(vq.w)));
+    sts128(k16 + off, make_uint4(bf16x2_to_f16x2(vk.x), bf16x2_to_f16x2(vk.y), bf16x2_to_f16x2(vk.z),
+                                 bf16x2_to_f16x2(vk.w)));
+}
 
 // Sum over the 4 lanes of a quad (lanes sharing rows g, g+8).
 __device__ __forceinline__ float quad_sum(float v) {
@@ -168,7 +220,6 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         tma_prefetch_desc(&maps.xk);
         tma_prefetch_desc(&maps.xv);
         s.fail = 0;
-        s.fail_m = 0;
     }
     // rows K..15 of every tile stay zero for the whole run (TMA writes rows < K only)
     for (int i = tid; i < kStages * kTileBytes / 16; i += kBlock) {
@@ -220,8 +271,8 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         // on a failure, wait (bounded) until the loads issued but not consumed have landed
         if (*reinterpret_cast<volatile int*>(&s.fail) || mm < n_mb) {
             if (lane == 0) {
-                const int first = *reinterpret_cast<volatile int*>(&s.fail_m);
-                for (int k = first; k < mm; ++k)
+                // (every load before the first ring slot still to refill may be unconsumed)
+                for (int k = mm > kStages ? mm - kStages : 0; k < mm; ++k)
                     mbar_wait_bounded(&s.full[k % kStages], static_cast<uint32_t>((k / kStages) & 1),
                                       kDrainPolls, nullptr);
             }
@@ -248,7 +299,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         Bt[0] = a.b0[b0off + 16 * w + g];
         Bt[2] = a.b0[b0off + 16 * w + g + 8];
     }
-    const uint32_t ones_b = (g == 0) ? pack_bf16x2(1.f, 1.f) : 0u;  // B operand: ones in column 0
+    const uint32_t ones_b = (g == 0) ? 0x3c003c00u : 0u;  // fp16 B operand: ones in column 0
     float bc[2][2], lw[2][2], lb[2][2];  // per n-tile nt, feature 16w + 8nt + 2t + e
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -284,6 +335,18 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             tmask[nt][e] = (j <= i) ? -s.te[i] : 0.f;
         }
     float zbar_prev[2][4] = {};
+    const uint32_t cvt_off = 16u * static_cast<uint32_t>(tid);  // this thread's chunk of a tile
+    auto stage_of = [&](int st_) {
+        return make_uint4(smem_u32(&s.xq[st_][0]), smem_u32(&s.xk[st_][0]), smem_u32(&s.xq16[st_][0]),
+                          smem_u32(&s.xk16[st_][0]));
+    };
+    // stage 0 landed and converted before the loop; stage m + 1 during mini-batch m
+    if (n_mb > 0) {
+        if (!mbar_wait_bounded(&s.full[0], 0, wait_limit, status)) s.fail = 1;
+        const uint4 sa = stage_of(0);
+        convert_chunk(sa.x, sa.y, sa.z, sa.w, cvt_off);
+    }
+    named_barrier_sync(1, kThreads);
     uint32_t xq_prev[4] = {};  // XQ at this thread's output positions (A fragment of k-slice w)
     bool failed = false;
     int m = 0, st = 0;
@@ -292,20 +355,20 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     for (; m < n_mb; ++m, st = (st + 1 == kStages ? 0 : st + 1), par ^= (st == 0)) {
         const bool full_mb = m < n_full;
         const int Km = full_mb ? K : static_cast<int>(a.rem);
-        if (!mbar_wait_bounded(&s.full[st], par, wait_limit, status)) {
-            s.fail_m = m;
-            s.fail = 1;
-        }
-        const uint32_t xq_s = smem_u32(&s.xq[st][0]);
-        const uint32_t xk_s = smem_u32(&s.xk[st][0]);
+        const int st1 = st + 1 == kStages ? 0 : st + 1;
+        const uint32_t par1 = par ^ (st1 == 0 ? 1u : 0u);
+        // the next stage: tested now, so that the test's latency hides behind the MMAs below
+        bool have_next = (m + 1 < n_mb) && mbar_test_wait(&s.full[st1], par1);
+        const uint32_t xq_s = smem_u32(&s.xq[st][0]), xk_s = smem_u32(&s.xk[st][0]);
+        const uint32_t xq16_s = smem_u32(&s.xq16[st][0]), xk16_s = smem_u32(&s.xk16[st][0]);
 
         // ---- Z = XK W + b (two accumulator chains), XQ W + b, XQ XK^T ------------------------
         float z[2][4], z2[2][4], xqw[2][4], at[2][4];
         uint32_t k[4][4], q[4][4];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            ldmatrix_x4(xk_s + swz128(lrow, 2 * kk + lchunk), k[kk][0], k[kk][1], k[kk][2], k[kk][3]);
-            ldmatrix_x4(xq_s + swz128(lrow, 2 * kk + lchunk), q[kk][0], q[kk][1], q[kk][2], q[kk][3]);
+            ldmatrix_x4(xk16_s + swz128(lrow, 2 * kk + lchunk), k[kk][0], k[kk][1], k[kk][2], k[kk][3]);
+            ldmatrix_x4(xq16_s + swz128(lrow, 2 * kk + lchunk), q[kk][0], q[kk][1], q[kk][2], q[kk][3]);
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -314,20 +377,20 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) z2[nt][e] = at[nt][e] = 0.f;
         }
-        uint32_t wf[4][4];  // W as bf16 B fragments: [k-slice][n-tile 0 lo/hi, n-tile 1 lo/hi]
+        uint32_t wf[4][4];  // W as fp16 B fragments: [k-slice][n-tile 0 lo/hi, n-tile 1 lo/hi]
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            wf[kk][0] = pack_bf16x2(Wt[2 * kk][0], Wt[2 * kk][1]);
-            wf[kk][1] = pack_bf16x2(Wt[2 * kk + 1][0], Wt[2 * kk + 1][1]);
-            wf[kk][2] = pack_bf16x2(Wt[2 * kk][2], Wt[2 * kk][3]);
-            wf[kk][3] = pack_bf16x2(Wt[2 * kk + 1][2], Wt[2 * kk + 1][3]);
+            wf[kk][0] = pack_f16x2(Wt[2 * kk][0], Wt[2 * kk][1]);
+            wf[kk][1] = pack_f16x2(Wt[2 * kk + 1][0], Wt[2 * kk + 1][1]);
+            wf[kk][2] = pack_f16x2(Wt[2 * kk][2], Wt[2 * kk][3]);
+            wf[kk][3] = pack_f16x2(Wt[2 * kk + 1][2], Wt[2 * kk + 1][3]);
         }
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
-            mma_bf16_16816(z[0], k[kk][0], k[kk][1], k[kk][2], k[kk][3], wf[kk][0], wf[kk][1]);
-            mma_bf16_16816(z[1], k[kk][0], k[kk][1], k[kk][2], k[kk][3], wf[kk][2], wf[kk][3]);
-            mma_bf16_16816(z2[0], k[kk + 2][0], k[kk + 2][1], k[kk + 2][2], k[kk + 2][3], wf[kk + 2][0], wf[kk + 2][1]);
-            mma_bf16_16816(z2[1], k[kk + 2][0], k[kk + 2][1], k[kk + 2][2], k[kk + 2][3], wf[kk + 2][2], wf[kk + 2][3]);
+            mma_f16_16816(z[0], k[kk][0], k[kk][1], k[kk][2], k[kk][3], wf[kk][0], wf[kk][1]);
+            mma_f16_16816(z[1], k[kk][0], k[kk][1], k[kk][2], k[kk][3], wf[kk][2], wf[kk][3]);
+            mma_f16_16816(z2[0], k[kk + 2][0], k[kk + 2][1], k[kk + 2][2], k[kk + 2][3], wf[kk + 2][0], wf[kk + 2][1]);
+            mma_f16_16816(z2[1], k[kk + 2][0], k[kk + 2][1], k[kk + 2][2], k[kk + 2][3], wf[kk + 2][2], wf[kk + 2][3]);
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
@@ -335,10 +398,10 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             for (int e = 0; e < 4; ++e) z[nt][e] += z2[nt][e];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_16816(xqw[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], wf[kk][0], wf[kk][1]);
-            mma_bf16_16816(xqw[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], wf[kk][2], wf[kk][3]);
-            mma_bf16_16816(at[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][0], k[kk][2]);
-            mma_bf16_16816(at[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][1], k[kk][3]);
+            mma_f16_16816(xqw[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], wf[kk][0], wf[kk][1]);
+            mma_f16_16816(xqw[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], wf[kk][2], wf[kk][3]);
+            mma_f16_16816(at[0], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][0], k[kk][2]);
+            mma_f16_16816(at[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][1], k[kk][3]);
         }
         // XK and XQ at this thread's own positions: the A fragment of k-slice w (one more
         // ldmatrix each is cheaper than selecting among the four slices held in registers)
@@ -359,6 +422,11 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         if (s.fail) {
             failed = true;
             break;
+        }
+        if (m + 1 < n_mb) {  // fp16 copy of the next stage (seen by all warps after B2)
+            if (!have_next && !mbar_wait_bounded(&s.full[st1], par1, wait_limit, status)) s.fail = 1;
+            const uint4 sa = stage_of(st1);
+            convert_chunk(sa.x, sa.y, sa.z, sa.w, cvt_off);
         }
         if (m > 0) store_out<kTok>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
 
@@ -423,17 +491,17 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             uint32_t ua[2][2];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                ua[nt][0] = movmatrix_trans(pack_bf16x2(lg0 * gg[nt][0], lg0 * gg[nt][1]));
-                ua[nt][1] = movmatrix_trans(pack_bf16x2(lg8 * gg[nt][2], lg8 * gg[nt][3]));
+                ua[nt][0] = movmatrix_trans(pack_f16x2(lg0 * gg[nt][0], lg0 * gg[nt][1]));
+                ua[nt][1] = movmatrix_trans(pack_f16x2(lg8 * gg[nt][2], lg8 * gg[nt][3]));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t r0, r1, r2, r3;  // XK as B: tokens x input dims, j-tiles 2kk and 2kk+1
-                ldmatrix_x4_trans(xk_s + swz128(lrow, 2 * kk + lchunk), r0, r1, r2, r3);
-                mma_bf16_16816(Wt[2 * kk], ua[0][0], ua[1][0], ua[0][1], ua[1][1], r0, r1);
-                mma_bf16_16816(Wt[2 * kk + 1], ua[0][0], ua[1][0], ua[0][1], ua[1][1], r2, r3);
+                ldmatrix_x4_trans(xk16_s + swz128(lrow, 2 * kk + lchunk), r0, r1, r2, r3);
+                mma_f16_16816(Wt[2 * kk], ua[0][0], ua[1][0], ua[0][1], ua[1][1], r0, r1);
+                mma_f16_16816(Wt[2 * kk + 1], ua[0][0], ua[1][0], ua[0][1], ua[1][1], r2, r3);
             }
-            mma_bf16_16816(Bt, ua[0][0], ua[1][0], ua[0][1], ua[1][1], ones_b, ones_b);  // b update
+            mma_f16_16816(Bt, ua[0][0], ua[1][0], ua[0][1], ua[1][1], ones_b, ones_b);  // b update
             // spread b to the layout of Z's columns: feature 16w + 8nt + 2t + e sits in lane
             // 4 (2t + e), register Bt[2 nt]
 #pragma unroll
@@ -452,15 +520,15 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             const float2 c10 = mul2(f2(tmask[1][0], tmask[1][1]), l89), c11 = mul2(f2(tmask[1][2], tmask[1][3]), l89);
             const float2 m00 = fma2(c00, f2(at[0][0], at[0][1]), c00), m01 = fma2(c01, f2(at[0][2], at[0][3]), c01);
             const float2 m10 = fma2(c10, f2(at[1][0], at[1][1]), c10), m11 = fma2(c11, f2(at[1][2], at[1][3]), c11);
-            const uint32_t ma0 = pack_bf16x2(m00.x, m00.y);
-            const uint32_t ma1 = pack_bf16x2(m01.x, m01.y);
-            const uint32_t ma2 = pack_bf16x2(m10.x, m10.y);
-            const uint32_t ma3 = pack_bf16x2(m11.x, m11.y);
+            const uint32_t ma0 = pack_f16x2(m00.x, m00.y);
+            const uint32_t ma1 = pack_f16x2(m01.x, m01.y);
+            const uint32_t ma2 = pack_f16x2(m10.x, m10.y);
+            const uint32_t ma3 = pack_f16x2(m11.x, m11.y);
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t b0 = movmatrix_trans(pack_bf16x2(gg[nt][0], gg[nt][1]));  // tokens 0-7
-                const uint32_t b1 = movmatrix_trans(pack_bf16x2(gg[nt][2], gg[nt][3]));  // tokens 8-15
-                mma_bf16_16816(xqw[nt], ma0, ma1, ma2, ma3, b0, b1);
+                const uint32_t b0 = movmatrix_trans(pack_f16x2(gg[nt][0], gg[nt][1]));  // tokens 0-7
+                const uint32_t b1 = movmatrix_trans(pack_f16x2(gg[nt][2], gg[nt][3]));  // tokens 8-15
+                mma_f16_16816(xqw[nt], ma0, ma1, ma2, ma3, b0, b1);
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)

@@ -17,7 +17,7 @@ _SRC = open(os.path.join(os.path.dirname(oracle.__file__), "ttt_oracle.c")).read
 MUTANTS = [
     ("drop_bias_grad", "gb[c] += lri * gi[c];", "(void)0;", 0),
     ("update_sign", "Wbar[e] = W[e] - ti * G[e];", "Wbar[e] = W[e] + ti * G[e];", 0),
-    ("token_eta_offset", "1.0 / (double)(i + 1)", "1.0 / (double)(i + 2)", 0),
+    ("token_eta_offset", "1.0 / (real)(i + 1)", "1.0 / (real)(i + 2)", 0),
     ("transposed_outer", "G[(size_t)a * d + c] += lri * xki[a] * gi[c];",
      "G[(size_t)c * d + a] += lri * xki[a] * gi[c];", 0),
     ("unbiased_variance", "v /= d;", "v /= (d - 1);", 0),
@@ -26,14 +26,14 @@ MUTANTS = [
     ("target_sign", "tgt[c] = xvj[c] - xkj[c];", "tgt[c] = xkj[c] - xvj[c];", 0),
     ("commit_tail_state", "        if (full) {\n            memcpy(W, Wbar", "        if (1) {\n            memcpy(W, Wbar", 0),
     ("drop_residual", "oi[c] = xqi[c] + y[c];", "oi[c] = y[c];", 0),
-    ("lr_index_shift", "double lri = lr[t0 + i];", "double lri = lr[t0 + (i + 1) % Km];", 0),
+    ("lr_index_shift", "real lri = lr[t0 + i];", "real lri = lr[t0 + (i + 1) % Km];", 0),
     ("grad_uses_xq", "row_times(xkj, W, b, d, d, z);", "row_times(xq + (size_t)(t0 + j) * d, W, b, d, d, z);", 0),
-    ("strict_lower_triangle", "            double ti = token_eta_at(token_eta, i);\n            for (size_t e = 0; e < dd; ++e) Wbar[e] = W[e] - ti * G[e];",
-     "            double ti = token_eta_at(token_eta, i);\n            for (size_t e = 0; e < dd; ++e) Wbar[e] = W[e] - ti * (G[e] - lri * xki[e / d] * gi[e % d]);", 0),
+    ("strict_lower_triangle", "            real ti = token_eta_at(token_eta, i);\n            for (size_t e = 0; e < dd; ++e) Wbar[e] = W[e] - ti * G[e];",
+     "            real ti = token_eta_at(token_eta, i);\n            for (size_t e = 0; e < dd; ++e) Wbar[e] = W[e] - ti * (G[e] - lri * xki[e / d] * gi[e % d]);", 0),
     ("ln_missing_bias", "y[c] = ln_w[c] * (u[c] - mu) / sigma + ln_b[c];", "y[c] = ln_w[c] * (u[c] - mu) / sigma;", 0),
     ("decode_commit_rule", "int commit = (p == K - 1);", "int commit = (p == 0);", 0),
     ("decode_position", "int p = (int)(offset % K);", "int p = (int)((offset + 1) % K);", 0),
-    ("decode_no_grad_reset", "        memset(W_grad, 0, sizeof(double) * dd);\n        memset(b_grad, 0, sizeof(double) * d);\n    }",
+    ("decode_no_grad_reset", "        memset(W_grad, 0, sizeof(real) * dd);\n        memset(b_grad, 0, sizeof(real) * d);\n    }",
      "    }", 0),
     ("gelu_deriv_factor", "(1.0 + 3.0 * 0.044715 * x * x)", "(1.0 + 0.044715 * x * x)", 0),
     ("mlp_drop_b2_grad", "gb2[c] += lri * g2i[c];", "(void)0;", 0),
