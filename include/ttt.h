@@ -191,6 +191,45 @@ int ttt_linear_forward_host(const void* XQ, const void* XK, const void* XV, cons
                             int chunk_batches, void* stream);
 
 /*
+ * ttt_linear_forward_host_static -- ttt_linear_forward_host for callers that cannot allocate
+ * device memory, using scratch built into the library instead of a caller's workspace.
+ * (No counterpart on the pages: it is a deployment variant of the host-buffer entry.)
+ *
+ * Who needs it: a caller whose device memory is all handed out in advance by another owner (a
+ * serving framework's caching pool, a fixed per-process budget), so that a cudaMalloc would fail
+ * or break that owner's accounting; a plain C host program with no device allocator of its own;
+ * a latency-sensitive caller that must not take the device-wide synchronisation that cudaMalloc
+ * and cudaFree can imply.  It allocates nothing: no cudaMalloc, no cudaFree, no library
+ * allocation, no stream or event creation.
+ *
+ * The scratch is one static device array of TTT_STATIC_SCRATCH_BYTES (32 MiB) per device that
+ * loads the library, held until the process exits.  The batch runs in chunks of as many batch
+ * rows as fit in it (the per-head parameters plus one set of staged inputs and outputs); sizes
+ * whose single batch row does not fit are rejected with TTT_ERR_ARG and a message giving the
+ * bytes needed (use ttt_linear_forward_host with a workspace for those).  Copies and kernels run
+ * one after another on `stream` (no overlap between chunks).
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.  Every call on a device
+ * shares the one array: calls that can overlap on the GPU (on different streams, or from
+ * several threads without ordering) race and corrupt each other's results -- order them on one
+ * stream.  The array keeps the last call's contents; nothing in it needs to start at zero, since
+ * each call writes every byte it reads.
+ *
+ * Arguments, results and errors as ttt_linear_forward_host, without workspace, workspace_bytes
+ * and chunk_batches.  Asynchronous on `stream`; the host buffers must stay valid and unchanged
+ * until `stream` passes this point.  A TTT_ERR_CUDA can come after earlier chunks are enqueued;
+ * synchronise `stream` before reusing the buffers after one.
+ */
+#define TTT_STATIC_SCRATCH_BYTES 33554432
+int ttt_linear_forward_host_static(const void* XQ, const void* XK, const void* XV, const float* lr,
+                                   const float* token_eta, const float* W0, const float* b0,
+                                   long long w0_batch_stride, const float* ln_w, const float* ln_b, int B,
+                                   int H, long long L, int d, int mini_batch, float eps, int dtype,
+                                   unsigned int flags, void* out, float* W_last, float* b_last,
+                                   float* W_grad_tail, float* b_grad_tail, void* stream);
+
+/*
  * ttt_mlp_forward -- TTT-MLP prefill ([readme]: the hidden state is a two-layer MLP;
  * [walkthrough]: "TTTMLP is two TTTLinear stacked").  The state is
  *   f(x) = gelu(x W1 + b1) W2 + b2,  gelu = tanh form, W1 [d,hid], W2 [hid,d],

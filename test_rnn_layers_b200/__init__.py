@@ -29,11 +29,12 @@ TTT_BF16 = 1
 TTT_FLAG_FP32_COMPUTE = 1
 TTT_FLAG_TOKEN_MAJOR = 2
 TTT_STATUS_TIMEOUT = 1
+TTT_STATIC_SCRATCH_BYTES = 33554432
 
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
            "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_host_workspace_bytes",
-           "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step",
-           "ttt_linear_decode_step_hist")
+           "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward",
+           "ttt_linear_decode_step", "ttt_linear_decode_step_hist")
 
 
 class TTTError(RuntimeError):
@@ -68,6 +69,8 @@ def lib():
         L.ttt_linear_host_workspace_bytes.restype = ll
         L.ttt_linear_forward_host.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
                                               vp, fp, fp, fp, fp, vp, ll, i, vp]
+        L.ttt_linear_forward_host_static.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i,
+                                                     u, vp, fp, fp, fp, fp, vp]
         L.ttt_mlp_forward.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, i, f, i,
                                       u, vp, fp, fp, fp, fp, vp]
         L.ttt_linear_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f, i,
@@ -75,7 +78,7 @@ def lib():
         L.ttt_linear_decode_step_hist.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f,
                                                   i, vp, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
-                     "ttt_linear_forward_host", "ttt_mlp_forward", "ttt_linear_decode_step",
+                     "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward", "ttt_linear_decode_step",
                      "ttt_linear_decode_step_hist"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -257,6 +260,50 @@ def ttt_linear_forward_host(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int 
                                        eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last),
                                        _ptr(W_grad_tail), _ptr(b_grad_tail), _ptr(workspace), workspace.numel(),
                                        chunk_batches, _stream(stream))
+    _check(rc)
+    if tail_grads:
+        return out, W_last, b_last, W_grad_tail, b_grad_tail
+    return out, W_last, b_last
+
+
+def ttt_linear_forward_host_static(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
+                                   token_eta=None, out=None, W_last=None, b_last=None, W_grad_tail=None,
+                                   b_grad_tail=None, tail_grads: bool = False, flags: int = 0,
+                                   token_major: bool = False, stream=None):
+    """ttt_linear_forward_host without a workspace: the library stages the batch through its
+    built-in device scratch (TTT_STATIC_SCRATCH_BYTES per device) and allocates nothing, for
+    callers that cannot allocate device memory.  Calls that overlap on the GPU race on that
+    scratch; order them on one stream.  Host tensors in and out (pin them for faster copies);
+    asynchronous on `stream`: synchronise before reading the outputs.
+    Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail)."""
+    _need_host(XQ, "XQ")
+    B, H, L, d = _act_sizes(XQ, token_major)
+    flags |= TTT_FLAG_TOKEN_MAJOR if token_major else 0
+    dt = XQ.dtype
+    for n, t in (("XK", XK), ("XV", XV)):
+        _need_host(t, n, dt, XQ.shape)
+    _need_host(lr, "lr", torch.float32, (B, H, L))
+    per_chain = W0.dim() == 4
+    _need_host(W0, "W0", torch.float32, (B, H, d, d) if per_chain else (H, d, d))
+    _need_host(b0, "b0", torch.float32, (B, H, d) if per_chain else (H, d))
+    _need_host(ln_w, "ln_w", torch.float32, (H, d))
+    _need_host(ln_b, "ln_b", torch.float32, (H, d))
+    if token_eta is not None:
+        _need_host(token_eta, "token_eta", torch.float32, (mini_batch,))
+
+    def host(shape, dtype):
+        return torch.empty(shape, dtype=dtype, pin_memory=True)
+
+    out = host(XQ.shape, dt) if out is None else _need_host(out, "out", dt, XQ.shape)
+    W_last = host((B, H, d, d), torch.float32) if W_last is None else _need_host(W_last, "W_last", torch.float32, (B, H, d, d))
+    b_last = host((B, H, d), torch.float32) if b_last is None else _need_host(b_last, "b_last", torch.float32, (B, H, d))
+    if tail_grads:
+        W_grad_tail = host((B, H, d, d), torch.float32) if W_grad_tail is None else W_grad_tail
+        b_grad_tail = host((B, H, d), torch.float32) if b_grad_tail is None else b_grad_tail
+    rc = lib().ttt_linear_forward_host_static(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0),
+                                              _ptr(b0), H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H,
+                                              L, d, mini_batch, eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W_last),
+                                              _ptr(b_last), _ptr(W_grad_tail), _ptr(b_grad_tail), _stream(stream))
     _check(rc)
     if tail_grads:
         return out, W_last, b_last, W_grad_tail, b_grad_tail

@@ -642,3 +642,131 @@ int ttt_linear_decode_step_hist(const void* xq, const void* xk, const void* xv, 
 }
 
 }  // extern "C"
+
+// ---- host-buffer entry that allocates nothing ---------------------------------------------------
+// The device scratch of ttt_linear_forward_host_static: one array per device that loads this
+// library, held until the process exits.  In host code its name is only a host-side stand-in;
+// the device address comes from cudaGetSymbolAddress, looked up once per device with that
+// device current.
+static __device__ __align__(256) unsigned char g_static_scratch[TTT_STATIC_SCRATCH_BYTES];
+
+namespace {
+int static_scratch(char** out) {
+    static std::mutex mu;
+    static char* ptrs[256] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 256) return fail(TTT_ERR_CUDA, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+        ptrs[dev] = static_cast<char*>(p);
+    }
+    *out = ptrs[dev];
+    return TTT_OK;
+}
+
+// Bytes of scratch for chunks of `cb` batch rows: the shared parameters and one staging set.
+size_t static_need(int H, long long L, int K, int dtype, int cb, bool per_chain) {
+    const HostLayout y = host_layout(H, L, K, dtype, cb, per_chain);
+    return y.set + y.set_bytes;
+}
+}  // namespace
+
+extern "C" int ttt_linear_forward_host_static(const void* XQ, const void* XK, const void* XV, const float* lr,
+                                              const float* token_eta, const float* W0, const float* b0,
+                                              long long w0_batch_stride, const float* ln_w, const float* ln_b, int B,
+                                              int H, long long L, int d, int mini_batch, float eps, int dtype,
+                                              unsigned int flags, void* out, float* W_last, float* b_last,
+                                              float* W_grad_tail, float* b_grad_tail, void* stream) {
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
+    if (rc) return rc;
+    const long long per_head = static_cast<long long>(kD) * kD;
+    const bool per_chain = w0_batch_stride != 0;
+    if (per_chain && w0_batch_stride != H * per_head)
+        return fail(TTT_ERR_ARG, "w0_batch_stride must be 0 or H*d*d (got %lld)", w0_batch_stride);
+    if (!W0 || !b0 || !ln_w || !ln_b || !W_last || !b_last)
+        return fail(TTT_ERR_ARG, "W0, b0, ln_w, ln_b, W_last and b_last must be non-null");
+    if (L > 0 && (!XQ || !XK || !XV || !lr || !out))
+        return fail(TTT_ERR_ARG, "XQ, XK, XV, lr and out must be non-null when L > 0");
+    // the largest chunk of batch rows whose staging fits the built-in scratch
+    const size_t cap = static_cast<size_t>(TTT_STATIC_SCRATCH_BYTES);
+    if (static_need(H, L, mini_batch, dtype, 1, per_chain) > cap)
+        return fail(TTT_ERR_ARG,
+                    "one batch row needs %zu bytes of staging; the built-in scratch holds %zu "
+                    "(use ttt_linear_forward_host with a workspace of your own)",
+                    static_need(H, L, mini_batch, dtype, 1, per_chain), cap);
+    int lo = 1, hi = B;
+    while (lo < hi) {
+        const int mid = lo + (hi - lo + 1) / 2;
+        if (static_need(H, L, mini_batch, dtype, mid, per_chain) <= cap) lo = mid; else hi = mid - 1;
+    }
+    const int cb = lo;
+    const long long chains = static_cast<long long>(B) * H;
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t act = static_cast<size_t>(chains) * L * kD * esz;
+    const long long wrows = per_chain ? chains : H;
+    Span in[] = {{"XQ", XQ, act}, {"XK", XK, act}, {"XV", XV, act}, {"lr", lr, static_cast<size_t>(chains * L) * 4},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
+                 {"W0", W0, static_cast<size_t>(wrows * per_head) * 4}, {"b0", b0, static_cast<size_t>(wrows * kD) * 4},
+                 {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    Span outs[] = {{"out", out, act}, {"W_last", W_last, static_cast<size_t>(chains * per_head) * 4},
+                   {"b_last", b_last, static_cast<size_t>(chains * kD) * 4},
+                   {"W_grad_tail", W_grad_tail, static_cast<size_t>(chains * per_head) * 4},
+                   {"b_grad_tail", b_grad_tail, static_cast<size_t>(chains * kD) * 4}};
+    const int same_ok[2][2] = {{1, 5}, {2, 6}};
+    rc = check_aliasing(in, 9, outs, 5, same_ok, 2);
+    if (rc) return rc;
+
+    char* ws = nullptr;
+    if ((rc = static_scratch(&ws))) return rc;
+    const HostLayout y = host_layout(H, L, mini_batch, dtype, cb, per_chain);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const auto H2D = cudaMemcpyHostToDevice;
+    const auto D2H = cudaMemcpyDeviceToHost;
+    // Every byte a call reads from the scratch was written earlier in the same call (parameters,
+    // then per chunk the inputs by copies and the outputs by the kernels), so nothing needs
+    // clearing.  Everything runs on `stream`, in order.
+    const size_t hb = static_cast<size_t>(H) * kD * 4;
+    cudaError_t e = cudaMemcpyAsync(ws + y.lnw, ln_w, hb, H2D, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ws + y.lnb, ln_b, hb, H2D, st);
+    if (e == cudaSuccess && token_eta) e = cudaMemcpyAsync(ws + y.te, token_eta, static_cast<size_t>(mini_batch) * 4, H2D, st);
+    if (e == cudaSuccess && !per_chain) e = cudaMemcpyAsync(ws + y.w0, W0, static_cast<size_t>(H) * per_head * 4, H2D, st);
+    if (e == cudaSuccess && !per_chain) e = cudaMemcpyAsync(ws + y.b0, b0, hb, H2D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward_host_static: parameters");
+    char* set = ws + y.set;
+    for (int bfirst = 0; bfirst < B; bfirst += cb) {
+        const int bc = (B - bfirst < cb) ? B - bfirst : cb;
+        const size_t cc = static_cast<size_t>(bc) * H, c0 = static_cast<size_t>(bfirst) * H;
+        const size_t a_off = c0 * static_cast<size_t>(L) * kD * esz, a_n = cc * static_cast<size_t>(L) * kD * esz;
+        const size_t l_off = c0 * static_cast<size_t>(L) * 4, l_n = cc * static_cast<size_t>(L) * 4;
+        const size_t s_off = c0 * per_head * 4, s_n = cc * per_head * 4;
+        const size_t v_off = c0 * kD * 4, v_n = cc * kD * 4;
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.xq, static_cast<const char*>(XQ) + a_off, a_n, H2D, st);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.xk, static_cast<const char*>(XK) + a_off, a_n, H2D, st);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.xv, static_cast<const char*>(XV) + a_off, a_n, H2D, st);
+        if (e == cudaSuccess && L > 0) e = cudaMemcpyAsync(set + y.lr, reinterpret_cast<const char*>(lr) + l_off, l_n, H2D, st);
+        if (e == cudaSuccess && per_chain) e = cudaMemcpyAsync(set + y.w0c, reinterpret_cast<const char*>(W0) + s_off, s_n, H2D, st);
+        if (e == cudaSuccess && per_chain) e = cudaMemcpyAsync(set + y.b0c, reinterpret_cast<const char*>(b0) + v_off, v_n, H2D, st);
+        if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward_host_static: inputs");
+        rc = enqueue_linear(set + y.xq, set + y.xk, set + y.xv, reinterpret_cast<const float*>(set + y.lr),
+                            token_eta ? reinterpret_cast<const float*>(ws + y.te) : nullptr,
+                            reinterpret_cast<const float*>(per_chain ? set + y.w0c : ws + y.w0),
+                            reinterpret_cast<const float*>(per_chain ? set + y.b0c : ws + y.b0), per_chain ? per_head : 0,
+                            reinterpret_cast<const float*>(ws + y.lnw), reinterpret_cast<const float*>(ws + y.lnb), bc, H,
+                            L, mini_batch, eps, dtype, flags, set + y.out, reinterpret_cast<float*>(set + y.wl),
+                            reinterpret_cast<float*>(set + y.bl), W_grad_tail ? reinterpret_cast<float*>(set + y.wg) : nullptr,
+                            b_grad_tail ? reinterpret_cast<float*>(set + y.bg) : nullptr, st);
+        if (rc) return rc;
+        if (L > 0) e = cudaMemcpyAsync(static_cast<char*>(out) + a_off, set + y.out, a_n, D2H, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(reinterpret_cast<char*>(W_last) + s_off, set + y.wl, s_n, D2H, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(reinterpret_cast<char*>(b_last) + v_off, set + y.bl, v_n, D2H, st);
+        if (e == cudaSuccess && W_grad_tail) e = cudaMemcpyAsync(reinterpret_cast<char*>(W_grad_tail) + s_off, set + y.wg, s_n, D2H, st);
+        if (e == cudaSuccess && b_grad_tail) e = cudaMemcpyAsync(reinterpret_cast<char*>(b_grad_tail) + v_off, set + y.bg, v_n, D2H, st);
+        if (e != cudaSuccess) return cuda_fail(e, "ttt_linear_forward_host_static: outputs");
+    }
+    return ok();
+}
