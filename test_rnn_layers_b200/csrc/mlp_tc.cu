@@ -31,6 +31,14 @@
 //  * XQ, XK, XV tiles arrive by TMA (K rows of 128 bytes from a 4-D tensor map, head-major or
 //    token-major, 128-byte swizzle, no multicast) into a ring.
 //    One thread issues the tcgen05 MMAs and commits to one mbarrier; all waits are bounded.
+//  * Operand precision: every tensor-core operand is fp16 (11-bit significand), with fp32
+//    accumulation.  The state path (both layers' products and updates) feeds back into itself
+//    for every mini-batch, and with bf16 operands (8-bit) a few chains of the B=8, H=32, L=2048
+//    workload end above 1e-2 relative error on b2.  The XQ and XK tiles are converted to fp16 in
+//    place (the next mini-batch's at the end of each one; exact for bf16 values of magnitude up
+//    to 65504, larger ones saturate), XV stays bf16; the W1 update scales g1 (not XK) by -t lr
+//    so that no operand falls into fp16's subnormal range.  (In place, because two CTAs of this
+//    kernel share an SM only while each needs under half of the SM's shared memory.)
 #include "tc5.cuh"
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
@@ -50,14 +58,14 @@ constexpr uint32_t cW1 = 0;    // + 64 mt: W1^T tile mt (rows = hidden 128mt.., 
 constexpr uint32_t cW2 = 128;  // + 64 mt: W2 tile mt (rows = hidden, cols = output dim)
 
 struct __align__(1024) MlpSmem {
-    uint8_t stage[kStages][3 * kTile];  // XK | XQ | XV; -t_{K-1} lr XK is written over XV
-    uint8_t W1s[2][128 * 128];          // bf16 W1^T shadow [tile][128 hidden rows x 128 B (64 inputs)]
-    uint8_t W2s[kHid * 128];            // bf16 W2 shadow [256 hidden rows x 128 B (64 outputs)]
-    uint8_t X2s[4 * kTile];             // bf16 X2     [4 hidden blocks][16 token rows x 128 B]
-    uint8_t XB2s[4 * kTile];            // bf16 Xbar2
-    uint8_t G1s[4 * kTile];             // bf16 g1
-    uint8_t G2s[kTile];                 // bf16 g2 [16 token rows x 128 B (64 outputs)]
-    uint8_t G2Ls[kTile];                // bf16 -t_{K-1} lr g2
+    uint8_t stage[kStages][3 * kTile];  // XK | XQ | XV, bf16 as loaded; XK, XQ then fp16 in place
+    uint8_t W1s[2][128 * 128];          // fp16 W1^T shadow [tile][128 hidden rows x 128 B (64 inputs)]
+    uint8_t W2s[kHid * 128];            // fp16 W2 shadow [256 hidden rows x 128 B (64 outputs)]
+    uint8_t X2s[4 * kTile];             // fp16 X2     [4 hidden blocks][16 token rows x 128 B]
+    uint8_t XB2s[4 * kTile];            // fp16 Xbar2
+    uint8_t G1s[4 * kTile];             // fp16 -t_{K-1} lr g1
+    uint8_t G2s[kTile];                 // fp16 g2 [16 token rows x 128 B (64 outputs)]
+    uint8_t G2Ls[kTile];                // fp16 -t_{K-1} lr g2
     union {                             // (disjoint lifetimes inside a mini-batch)
         float Zt[TTT_KMAX][TTT_D];      // Z2, then Zbar2, as token rows (b2 included)
         __half A2p[8][TTT_KMAX][TTT_KMAX];  // Xbar2 X2^T over each warp's hidden slice
@@ -129,8 +137,24 @@ __device__ __forceinline__ void ld4_bf16(const uint8_t* tile, int r, int c, floa
     const float2 a = unpack_bf16x2(v.x), b = unpack_bf16x2(v.y);
     out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
 }
-__device__ __forceinline__ void st4_bf16(uint8_t* tile, int r, int c, float a, float b, float d, float e) {
-    *reinterpret_cast<uint2*>(tile + swz(r, c)) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(d, e));
+__device__ __forceinline__ void st4_f16(uint8_t* tile, int r, int c, float a, float b, float d, float e) {
+    *reinterpret_cast<uint2*>(tile + swz(r, c)) = make_uint2(pack_f16x2(a, b), pack_f16x2(d, e));
+}
+
+// A stage's XK and XQ tiles from bf16 to fp16 in place: thread tid converts one 16-byte chunk,
+// of XK for tid < 128 and of XQ otherwise.
+__device__ __forceinline__ void convert_stage(uint8_t* stage, int tid) {
+    uint4* p = reinterpret_cast<uint4*>(stage + 16u * static_cast<uint32_t>(tid & 127) +
+                                        static_cast<uint32_t>(tid >> 7) * kTile);
+    const uint4 v = *p;
+    *p = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+}
+
+// 4 consecutive fp16 of row r starting at column c (c % 4 == 0) -> floats
+__device__ __forceinline__ void ld4_f16(const uint8_t* tile, int r, int c, float* out) {
+    const uint2 v = *reinterpret_cast<const uint2*>(tile + swz(r, c));
+    const float2 a = unpack_f16x2(v.x), b = unpack_f16x2(v.y);
+    out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
 }
 
 // [16 tokens x 32 hidden] slice of this warp: four m16n8 accumulator tiles (hidden 8nt + 2t + e,
@@ -159,7 +183,7 @@ __device__ __forceinline__ void tokens_times_w2(float (&acc)[2][4], uint32_t a_t
             const int ks = 2 * p + hh;  // hidden 16 ks .. 16 ks + 15
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(a_tiles + (ks >> 2) * kTile + swz128(lrow, 2 * (ks & 3) + lchunk), a0, a1, a2, a3);
-            mma_bf16_16816(acc[hh], a0, a1, a2, a3, hh ? b2 : b0, hh ? b3 : b1);
+            mma_f16_16816(acc[hh], a0, a1, a2, a3, hh ? b2 : b0, hh ? b3 : b1);
         }
     }
 }
@@ -236,10 +260,10 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             for (int half = 0; half < 2; ++half) {
                 const int cc = 16 * c + 8 * half;  // 8 columns = one 16-byte chunk
                 uint4 p1, p2;
-                p1.x = pack_bf16x2(v1[8 * half + 0], v1[8 * half + 1]); p1.y = pack_bf16x2(v1[8 * half + 2], v1[8 * half + 3]);
-                p1.z = pack_bf16x2(v1[8 * half + 4], v1[8 * half + 5]); p1.w = pack_bf16x2(v1[8 * half + 6], v1[8 * half + 7]);
-                p2.x = pack_bf16x2(v2[8 * half + 0], v2[8 * half + 1]); p2.y = pack_bf16x2(v2[8 * half + 2], v2[8 * half + 3]);
-                p2.z = pack_bf16x2(v2[8 * half + 4], v2[8 * half + 5]); p2.w = pack_bf16x2(v2[8 * half + 6], v2[8 * half + 7]);
+                p1.x = pack_f16x2(v1[8 * half + 0], v1[8 * half + 1]); p1.y = pack_f16x2(v1[8 * half + 2], v1[8 * half + 3]);
+                p1.z = pack_f16x2(v1[8 * half + 4], v1[8 * half + 5]); p1.w = pack_f16x2(v1[8 * half + 6], v1[8 * half + 7]);
+                p2.x = pack_f16x2(v2[8 * half + 0], v2[8 * half + 1]); p2.y = pack_f16x2(v2[8 * half + 2], v2[8 * half + 3]);
+                p2.z = pack_f16x2(v2[8 * half + 4], v2[8 * half + 5]); p2.w = pack_f16x2(v2[8 * half + 6], v2[8 * half + 7]);
                 *reinterpret_cast<uint4*>(&s.W1s[mt][0] + swz(r, cc)) = p1;
                 *reinterpret_cast<uint4*>(&s.W2s[0] + swz(u, cc)) = p2;
             }
@@ -301,10 +325,10 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             const int i = g + 8 * (e >> 1), j = 8 * nt + 2 * t + (e & 1);
             tmask[nt][e] = (j <= i) ? -s.te[i] : 0.f;
         }
-    const uint32_t idUp = tc5::idesc_bf16(128, 64, 1, 1);
+    const uint32_t idUp = tc5::idesc_f16(128, 64, 1, 1);
     const uint64_t dX2m = tc5::sdesc(smem_u32(&s.X2s[0]), kTile, 1024);     // X2^T, MN-major A
-    const uint64_t dG1m = tc5::sdesc(smem_u32(&s.G1s[0]), kTile, 1024);     // g1^T, MN-major A
-    const uint64_t dXKLm = tc5::sdesc(smem_u32(&s.stage[0][2 * kTile]), kTile, 1024);  // -t lr XK of stage 0, MN-major B
+    const uint64_t dG1m = tc5::sdesc(smem_u32(&s.G1s[0]), kTile, 1024);     // (-t lr g1)^T, MN-major A
+    const uint64_t dXK16m = tc5::sdesc(smem_u32(&s.stage[0][0]), kTile, 1024);  // XK (fp16) of stage 0, MN-major B
     const uint64_t dG2Lm = tc5::sdesc(smem_u32(&s.G2Ls[0]), kTile, 1024);   // -t lr g2, MN-major B
     const uint32_t w1_s = smem_u32(&s.W1s[(32 * w) >> 7][0]);  // this warp's 32 hidden rows live in one tile
     const int w1_row0 = (32 * w) & 127;
@@ -317,11 +341,18 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         const float2 l89 = *reinterpret_cast<const float2*>(&lr_s[2 * t + 8]);
         const float c00 = tmask[0][0] * l01.x, c01 = tmask[0][1] * l01.y, c02 = tmask[0][2] * l01.x, c03 = tmask[0][3] * l01.y;
         const float c10 = tmask[1][0] * l89.x, c11 = tmask[1][1] * l89.y, c12 = tmask[1][2] * l89.x, c13 = tmask[1][3] * l89.y;
-        ma[0] = pack_bf16x2(fmaf(c00, at[0][0], c00), fmaf(c01, at[0][1], c01));
-        ma[1] = pack_bf16x2(fmaf(c02, at[0][2], c02), fmaf(c03, at[0][3], c03));
-        ma[2] = pack_bf16x2(fmaf(c10, at[1][0], c10), fmaf(c11, at[1][1], c11));
-        ma[3] = pack_bf16x2(fmaf(c12, at[1][2], c12), fmaf(c13, at[1][3], c13));
+        ma[0] = pack_f16x2(fmaf(c00, at[0][0], c00), fmaf(c01, at[0][1], c01));
+        ma[1] = pack_f16x2(fmaf(c02, at[0][2], c02), fmaf(c03, at[0][3], c03));
+        ma[2] = pack_f16x2(fmaf(c10, at[1][0], c10), fmaf(c11, at[1][1], c11));
+        ma[3] = pack_f16x2(fmaf(c12, at[1][2], c12), fmaf(c13, at[1][3], c13));
     };
+
+    // the fp16 copy of stage 0 before the loop; that of mini-batch m + 1 at the end of m
+    if (n_mb > 0) {
+        if (!mbar_wait_bounded(&s.full[0], 0, wait_limit, a.status)) s.fail = 1;
+        convert_stage(&s.stage[0][0], tid);
+    }
+    __syncthreads();
 
     uint32_t mpar = 0;  // phase parity of mma_bar
     int st = 0;
@@ -332,10 +363,9 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         const int Km = full_mb ? K : static_cast<int>(a.rem);
         if (w == 0 && m + kStages - 1 < n_mb) issue(m + kStages - 1, (m + kStages - 1) % kStages);
         if (!mbar_wait_bounded(&s.full[st], par, wait_limit, a.status)) s.fail = 1;
-        uint8_t* xk_t = &s.stage[st][0];
-        uint8_t* xq_t = &s.stage[st][kTile];
-        const uint8_t* xv_t = &s.stage[st][2 * kTile];
-        uint8_t* xkl_t = &s.stage[st][2 * kTile];
+        const uint8_t* xk_t = &s.stage[st][0];  // fp16 (converted)
+        const uint8_t* xq_t = &s.stage[st][kTile];
+        const uint8_t* xv_t = &s.stage[st][2 * kTile];  // bf16
         const float* lr_s = s.lr[st];
         const uint32_t xk_s = smem_u32(xk_t), xq_s = smem_u32(xq_t);
 
@@ -357,13 +387,13 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             for (int hb = 0; hb < 2; ++hb) {  // hidden 32w + 16hb .. + 15: n-tiles 2hb, 2hb + 1
                 uint32_t b0, b1, b2, b3;
                 ldmatrix_x4(w1_s + swz128(w1_row0 + 16 * hb + lrow, 2 * kk + lchunk), b0, b1, b2, b3);
-                mma_bf16_16816(z1[2 * hb], k0, k1, k2, k3, b0, b2);
-                mma_bf16_16816(z1[2 * hb + 1], k0, k1, k2, k3, b1, b3);
-                mma_bf16_16816(zb1[2 * hb], q0, q1, q2, q3, b0, b2);
-                mma_bf16_16816(zb1[2 * hb + 1], q0, q1, q2, q3, b1, b3);
+                mma_f16_16816(z1[2 * hb], k0, k1, k2, k3, b0, b2);
+                mma_f16_16816(z1[2 * hb + 1], k0, k1, k2, k3, b1, b3);
+                mma_f16_16816(zb1[2 * hb], q0, q1, q2, q3, b0, b2);
+                mma_f16_16816(zb1[2 * hb + 1], q0, q1, q2, q3, b1, b3);
             }
-            mma_bf16_16816(at1[0], q0, q1, q2, q3, k0, k2);  // tokens 0-7 of XK as B
-            mma_bf16_16816(at1[1], q0, q1, q2, q3, k1, k3);  // tokens 8-15
+            mma_f16_16816(at1[0], q0, q1, q2, q3, k0, k2);  // tokens 0-7 of XK as B
+            mma_f16_16816(at1[1], q0, q1, q2, q3, k1, k3);  // tokens 8-15
         }
 
         // (2) X2 = gelu(Z1), keep gelu'(Z1); X2 to shared memory (A of Z2, A of W2's update)
@@ -374,8 +404,8 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             float y[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) gelu2(z1[nt][e], y[e], dg[nt][e]);
-            x2p[nt][0] = pack_bf16x2(y[0], y[1]);
-            x2p[nt][1] = pack_bf16x2(y[2], y[3]);
+            x2p[nt][0] = pack_f16x2(y[0], y[1]);
+            x2p[nt][1] = pack_f16x2(y[2], y[3]);
         }
         store_slice(&s.X2s[0], w, g, t, x2p);
         __syncthreads();
@@ -399,7 +429,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             float z[4], xk[4], xv[4];
             const float4 zz = *reinterpret_cast<const float4*>(&s.Zt[rr][f4]);
             z[0] = zz.x; z[1] = zz.y; z[2] = zz.z; z[3] = zz.w;
-            ld4_bf16(xk_t, rr, f4, xk);
+            ld4_f16(xk_t, rr, f4, xk);
             ld4_bf16(xv_t, rr, f4, xv);
             float mu, rs;
             row_stats16(z, eps, mu, rs);
@@ -417,11 +447,9 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             float g2[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) g2[i] = fmaf(-xh[i], sqx, fmaf(static_cast<float>(TTT_D), qv[i], -sq)) * sc;
-            st4_bf16(&s.G2s[0], rr, f4, g2[0], g2[1], g2[2], g2[3]);
+            st4_f16(&s.G2s[0], rr, f4, g2[0], g2[1], g2[2], g2[3]);
             const float ls = -tl * lr_s[rr];
-            st4_bf16(&s.G2Ls[0], rr, f4, ls * g2[0], ls * g2[1], ls * g2[2], ls * g2[3]);
-            // each thread overwrites exactly the XV elements it has read
-            st4_bf16(xkl_t, rr, f4, ls * xk[0], ls * xk[1], ls * xk[2], ls * xk[3]);
+            st4_f16(&s.G2Ls[0], rr, f4, ls * g2[0], ls * g2[1], ls * g2[2], ls * g2[3]);
         }
         __syncthreads();
 
@@ -439,19 +467,22 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             for (int hb = 0; hb < 2; ++hb) {
                 uint32_t b0, b1, b2, b3;  // W2 rows = hidden (n), outputs = k
                 ldmatrix_x4(w2_s + swz128(32 * w + 16 * hb + lrow, 2 * kk + lchunk), b0, b1, b2, b3);
-                mma_bf16_16816(g1[2 * hb], a0, a1, a2, a3, b0, b2);
-                mma_bf16_16816(g1[2 * hb + 1], a0, a1, a2, a3, b1, b3);
+                mma_f16_16816(g1[2 * hb], a0, a1, a2, a3, b0, b2);
+                mma_f16_16816(g1[2 * hb + 1], a0, a1, a2, a3, b1, b3);
             }
         }
-        uint32_t g1p[4][2];
+        uint32_t g1p[4][2], g1s[4][2];  // g1, and -t_{K-1} lr g1 for W1's update, as fp16 pairs
         {
             const float lg = lr_s[g], lg8 = lr_s[g + 8];
+            const float sg = -tl * lg, sg8 = -tl * lg8;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) g1[nt][e] *= dg[nt][e];
-                g1p[nt][0] = pack_bf16x2(g1[nt][0], g1[nt][1]);
-                g1p[nt][1] = pack_bf16x2(g1[nt][2], g1[nt][3]);
+                g1p[nt][0] = pack_f16x2(g1[nt][0], g1[nt][1]);
+                g1p[nt][1] = pack_f16x2(g1[nt][2], g1[nt][3]);
+                g1s[nt][0] = pack_f16x2(sg * g1[nt][0], sg * g1[nt][1]);
+                g1s[nt][1] = pack_f16x2(sg8 * g1[nt][2], sg8 * g1[nt][3]);
                 // b1 -= t_{K-1} sum_j lr_j g1_j (sum over the 16 token rows: lanes g = 0..7)
                 if (full_mb) {
 #pragma unroll
@@ -465,7 +496,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 }
             }
         }
-        store_slice(&s.G1s[0], w, g, t, g1p);
+        store_slice(&s.G1s[0], w, g, t, g1s);
         // the state update on a full mini-batch, on the tensor cores while the output path runs:
         // W1^T += g1^T (-t lr XK), W2 += X2^T (-t lr g2)
         fence_proxy_async_smem();
@@ -476,7 +507,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
 #pragma unroll
             for (int t2 = 0; t2 < 2; ++t2) {
                 tc5::mma_ss(tm + cW1 + 64 * t2, tc5::sdesc_add(dG1m, t2 * 2 * kTile),
-                            tc5::sdesc_add(dXKLm, st * 3 * kTile), idUp, 1);
+                            tc5::sdesc_add(dXK16m, st * 3 * kTile), idUp, 1);
                 tc5::mma_ss(tm + cW2 + 64 * t2, tc5::sdesc_add(dX2m, t2 * 2 * kTile), dG2Lm, idUp, 1);
             }
             tc5::commit(&s.mma_bar);
@@ -488,7 +519,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             m_operand(at1, lr_s, ma);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
-                mma_bf16_16816(zb1[nt], ma[0], ma[1], ma[2], ma[3], movmatrix_trans(g1p[nt][0]),
+                mma_f16_16816(zb1[nt], ma[0], ma[1], ma[2], ma[3], movmatrix_trans(g1p[nt][0]),
                                movmatrix_trans(g1p[nt][1]));
         }
 
@@ -497,17 +528,17 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             uint32_t xb2p[4][2];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                xb2p[nt][0] = pack_bf16x2(gelu(zb1[nt][0]), gelu(zb1[nt][1]));
-                xb2p[nt][1] = pack_bf16x2(gelu(zb1[nt][2]), gelu(zb1[nt][3]));
+                xb2p[nt][0] = pack_f16x2(gelu(zb1[nt][0]), gelu(zb1[nt][1]));
+                xb2p[nt][1] = pack_f16x2(gelu(zb1[nt][2]), gelu(zb1[nt][3]));
             }
             store_slice(&s.XB2s[0], w, g, t, xb2p);
             float a2[2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {  // hidden n-tiles 2kk, 2kk + 1 form one k-step
                 // A = Xbar2 (rows = tokens), B = X2 (k = hidden, n = tokens), both from accumulators
-                mma_bf16_16816(a2[0], xb2p[2 * kk][0], xb2p[2 * kk][1], xb2p[2 * kk + 1][0], xb2p[2 * kk + 1][1],
+                mma_f16_16816(a2[0], xb2p[2 * kk][0], xb2p[2 * kk][1], xb2p[2 * kk + 1][0], xb2p[2 * kk + 1][1],
                                x2p[2 * kk][0], x2p[2 * kk + 1][0]);
-                mma_bf16_16816(a2[1], xb2p[2 * kk][0], xb2p[2 * kk][1], xb2p[2 * kk + 1][0], xb2p[2 * kk + 1][1],
+                mma_f16_16816(a2[1], xb2p[2 * kk][0], xb2p[2 * kk][1], xb2p[2 * kk + 1][0], xb2p[2 * kk + 1][1],
                                x2p[2 * kk][1], x2p[2 * kk + 1][1]);
             }
 #pragma unroll
@@ -550,12 +581,12 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             {
                 uint32_t b0, b1, d0, d1;  // g2 (k = tokens, n = outputs 8w..), transposed from token rows
                 ldmatrix_x4_trans(g2_s + swz128(lrow, w), b0, b1, d0, d1);
-                mma_bf16_16816(zb2[1], ma[0], ma[1], ma[2], ma[3], b0, b1);
+                mma_f16_16816(zb2[1], ma[0], ma[1], ma[2], ma[3], b0, b1);
                 // sum_j lr_j g2_j for b2's update: an A operand whose row 0 is lr
-                const uint32_t r0 = g == 0 ? pack_bf16x2(lr_s[2 * t], lr_s[2 * t + 1]) : 0u;
-                const uint32_t r2 = g == 0 ? pack_bf16x2(lr_s[2 * t + 8], lr_s[2 * t + 9]) : 0u;
+                const uint32_t r0 = g == 0 ? pack_f16x2(lr_s[2 * t], lr_s[2 * t + 1]) : 0u;
+                const uint32_t r2 = g == 0 ? pack_f16x2(lr_s[2 * t + 8], lr_s[2 * t + 9]) : 0u;
                 float bd[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_bf16_16816(bd, r0, 0u, r2, 0u, b0, b1);
+                mma_f16_16816(bd, r0, 0u, r2, 0u, b0, b1);
                 b2d[0] = bd[0];  // row 0, outputs 8w + 2t, 8w + 2t + 1 (lanes g == 0)
                 b2d[1] = bd[1];
             }
@@ -569,7 +600,7 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             float z[4], xq[4];
             const float4 zz = *reinterpret_cast<const float4*>(&s.Zt[rr][f4]);
             z[0] = zz.x; z[1] = zz.y; z[2] = zz.z; z[3] = zz.w;
-            ld4_bf16(xq_t, rr, f4, xq);
+            ld4_f16(xq_t, rr, f4, xq);
             float mu, rs;
             row_stats16(z, eps, mu, rs);
             if (rr < Km) {
@@ -603,14 +634,19 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
                 for (int half = 0; half < 2; ++half) {
                     const int cc = 16 * c + 8 * half;
                     uint4 p1, p2;
-                    p1.x = pack_bf16x2(v1[8 * half + 0], v1[8 * half + 1]); p1.y = pack_bf16x2(v1[8 * half + 2], v1[8 * half + 3]);
-                    p1.z = pack_bf16x2(v1[8 * half + 4], v1[8 * half + 5]); p1.w = pack_bf16x2(v1[8 * half + 6], v1[8 * half + 7]);
-                    p2.x = pack_bf16x2(v2[8 * half + 0], v2[8 * half + 1]); p2.y = pack_bf16x2(v2[8 * half + 2], v2[8 * half + 3]);
-                    p2.z = pack_bf16x2(v2[8 * half + 4], v2[8 * half + 5]); p2.w = pack_bf16x2(v2[8 * half + 6], v2[8 * half + 7]);
+                    p1.x = pack_f16x2(v1[8 * half + 0], v1[8 * half + 1]); p1.y = pack_f16x2(v1[8 * half + 2], v1[8 * half + 3]);
+                    p1.z = pack_f16x2(v1[8 * half + 4], v1[8 * half + 5]); p1.w = pack_f16x2(v1[8 * half + 6], v1[8 * half + 7]);
+                    p2.x = pack_f16x2(v2[8 * half + 0], v2[8 * half + 1]); p2.y = pack_f16x2(v2[8 * half + 2], v2[8 * half + 3]);
+                    p2.z = pack_f16x2(v2[8 * half + 4], v2[8 * half + 5]); p2.w = pack_f16x2(v2[8 * half + 6], v2[8 * half + 7]);
                     *reinterpret_cast<uint4*>(&s.W1s[mt][0] + swz(r, cc)) = p1;
                     *reinterpret_cast<uint4*>(&s.W2s[0] + swz(u, cc)) = p2;
                 }
             }
+        }
+        if (m + 1 < n_mb) {  // fp16 copy of the next mini-batch's XK and XQ (loaded since the top of m)
+            const int st1 = st ^ 1;
+            if (!mbar_wait_bounded(&s.full[st1], par ^ (st1 == 0 ? 1u : 0u), wait_limit, a.status)) s.fail = 1;
+            convert_stage(&s.stage[st1][0], tid);
         }
         tc5::fence_before();
         __syncthreads();
