@@ -53,10 +53,12 @@ def load(path: str | None = None):
                                             _D, _D, _D, _D, _D]
     lib.oracle_ttt_linear_decode_chain.argtypes = [_D, _D, _D, dbl, _D, _D, _D, _D, _D, _D, _D,
                                                    i, i, _LL, dbl, _D, ctypes.POINTER(i)]
+    lib.oracle_rope.argtypes = [_D, _LL, i, i, dbl, i, _D]
     lib.oracle_ttt_mlp_chain.argtypes = [_D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _LL, i, i, i,
                                          dbl, _D, _D, _D, _D, _D]
     for f in ("oracle_partition", "oracle_lnl2_grad", "oracle_ln_forward", "oracle_gelu_tanh",
-              "oracle_ttt_linear_chain", "oracle_ttt_linear_decode_chain", "oracle_ttt_mlp_chain"):
+              "oracle_ttt_linear_chain", "oracle_ttt_linear_decode_chain", "oracle_ttt_mlp_chain",
+              "oracle_rope"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -105,6 +107,20 @@ class Oracle:
         y, dy = np.empty_like(x), np.empty_like(x)
         self._check(self.lib.oracle_gelu_tanh(self._p(x), x.size, self._p(y), self._p(dy)), "gelu")
         return y, dy
+
+    def rope(self, x, K, theta, half_split=False):
+        """Rotary embedding of [..., L, d] rows (position = token index mod K), float64."""
+        x = self._f64(x)
+        y = np.empty_like(x)
+        L, d = x.shape[-2], x.shape[-1]
+        flat_x, flat_y = x.reshape(-1, L, d), y.reshape(-1, L, d)
+        for c in range(flat_x.shape[0]):
+            xc = np.ascontiguousarray(flat_x[c])
+            yc = np.empty_like(xc)
+            self._check(self.lib.oracle_rope(self._p(xc), L, d, K, float(theta), 1 if half_split else 0,
+                                             self._p(yc)), "rope")
+            flat_y[c] = yc
+        return y
 
     # ---- TTT-Linear ------------------------------------------------------------------------
     def linear_chain(self, xq, xk, xv, lr, W0, b0, ln_w, ln_b, K, eps, token_eta=None):

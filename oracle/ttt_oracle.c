@@ -67,6 +67,35 @@ int oracle_partition(long long L, int K, long long* n_full, long long* rem) {
 }
 
 /* ---------------------------------------------------------------------------------------- */
+/* Rotary position embedding of XQ and XK before the scan ([walkthrough], TTTBase.forward:    */
+/* cos, sin = rotary_emb(XV, position_ids % mini_batch_size); permute_qk; apply_rotary_pos_emb; */
+/* undo_permute_qk -- the bodies are not on the pages).  Token t of a chain takes position     */
+/* p = t mod K; feature pair k (k < d/2) turns by the angle p * theta^(-2k/d) (RoFormer):       */
+/*     (x_a, x_b) -> (x_a cos - x_b sin, x_a sin + x_b cos)                                   */
+/* with (a, b) = (2k, 2k+1) -- adjacent features, the reading of permute_qk, the rotate-half  */
+/* form and undo_permute_qk composed -- or (a, b) = (k, k + d/2) when half_split is set (the   */
+/* rotate-half form alone).  x, y: [L][d]; y may equal x.                                      */
+/* ---------------------------------------------------------------------------------------- */
+int oracle_rope(const real* x, long long L, int d, int K, real theta, int half_split, real* y) {
+    if (!x || !y || L < 0 || d < 2 || (d % 2) != 0 || K < 1 || !(theta > 0)) return ORACLE_ERR_ARG;
+    const int half = d / 2;
+    for (long long t = 0; t < L; ++t) {
+        const real p = (real)(t % K);
+        const real* xr = x + (size_t)t * d;
+        real* yr = y + (size_t)t * d;
+        for (int k = 0; k < half; ++k) {
+            const real ang = p * pow(theta, -2.0 * k / d);
+            const real c = cos(ang), s = sin(ang);
+            const int ia = half_split ? k : 2 * k, ib = half_split ? k + half : 2 * k + 1;
+            const real xa = xr[ia], xb = xr[ib];
+            yr[ia] = xa * c - xb * s;
+            yr[ib] = xa * s + xb * c;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------------------- */
 /* LayerNorm pieces ([walkthrough], compute_mini_batch: ln_fused_l2_bwd and ln_fwd).          */
 /* ---------------------------------------------------------------------------------------- */
 

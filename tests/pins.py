@@ -21,6 +21,10 @@ What pins what:
     splitting a sequence at a mini-batch boundary and carrying (W, b) changes nothing;
     decode steps from a carried cache reproduce the prefill.
   * Integers: the partition equals floor division / remainder.
+  * Rotary position embedding (applied to XQ, XK before the scan): position 0 is the identity,
+    every rotated pair keeps its norm, dot products depend only on the difference of positions,
+    and a torch restatement of the rotate-half form (with the pair permutation that permute_qk /
+    undo_permute_qk perform, for the interleaved convention) gives the same values.
 """
 from __future__ import annotations
 
@@ -315,6 +319,60 @@ def pin_mlp_split_and_carry(o):
                     a["b2_last"], w, b, K, 1e-6)
     assert _rel(np.concatenate([a["out"], c["out"]]), whole["out"]) < 1e-13
     assert _rel(c["W2_last"], whole["W2_last"]) < 1e-13
+
+
+def _rope_torch(x, K, theta, interleaved):
+    """The rotate-half rotary embedding written with torch ops (cos/sin tables over positions
+    t mod K, q * cos + rotate_half(q) * sin); for the interleaved convention the features are
+    first permuted from adjacent pairs (2k, 2k+1) to halves (k, k + d/2) and back afterwards."""
+    x = torch.as_tensor(x, dtype=torch.float64)
+    L, d = x.shape[-2], x.shape[-1]
+    inv_freq = 1.0 / (theta ** (torch.arange(0, d, 2, dtype=torch.float64) / d))
+    pos = torch.arange(L, dtype=torch.float64) % K
+    freqs = torch.outer(pos, inv_freq)
+    emb = torch.cat([freqs, freqs], dim=-1)
+    cos, sin = emb.cos(), emb.sin()
+    if interleaved:
+        x = x.reshape(*x.shape[:-1], d // 2, 2).transpose(-1, -2).reshape(*x.shape[:-1], d)
+    x1, x2 = x[..., : d // 2], x[..., d // 2:]
+    y = x * cos + torch.cat([-x2, x1], dim=-1) * sin
+    if interleaved:
+        y = y.reshape(*y.shape[:-1], 2, d // 2).transpose(-1, -2).reshape(*y.shape[:-1], d)
+    return y.numpy()
+
+
+def pin_rope_position_zero_and_pair_norms(o):
+    rng = _rng(21)
+    L, d, K = 37, 16, 8
+    x = rng.normal(0, 1, (L, d))
+    for half in (False, True):
+        y = o.rope(x, K, 500.0, half)
+        assert np.array_equal(y[::K], x[::K])  # positions 0 (t = 0, K, 2K, ...) do not move
+        a = np.arange(d // 2) if half else 2 * np.arange(d // 2)
+        b = a + d // 2 if half else a + 1
+        assert np.allclose(np.hypot(y[:, a], y[:, b]), np.hypot(x[:, a], x[:, b]), rtol=1e-13, atol=0)
+        assert not np.allclose(y[1], x[1])
+
+
+def pin_rope_relative_position(o):
+    # <R(p1) q, R(p2) k> = <q, R(p2 - p1) k>: rows p1, p2 of one array against row p2 - p1 of another
+    rng = _rng(22)
+    d, K = 16, 16
+    q, k = rng.normal(0, 1, d), rng.normal(0, 1, d)
+    for half in (False, True):
+        for p1, p2 in ((3, 11), (5, 5), (0, 15)):
+            Aq, Ak, B = np.zeros((K, d)), np.zeros((K, d)), np.zeros((K, d))
+            Aq[p1], Ak[p2], B[p2 - p1] = q, k, k
+            yq, yk, yB = (o.rope(X, K, 10000.0, half) for X in (Aq, Ak, B))
+            assert abs(yq[p1] @ yk[p2] - q @ yB[p2 - p1]) < 1e-12 * (1 + abs(q @ k))
+
+
+def pin_rope_torch_restatement(o):
+    rng = _rng(23)
+    x = rng.normal(0, 1, (3, 41, 64))
+    for half in (False, True):
+        for theta in (10000.0, 37.0):
+            assert _rel(o.rope(x, 16, theta, half), _rope_torch(x, 16, theta, not half)) < 1e-13
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

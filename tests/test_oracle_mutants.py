@@ -41,6 +41,12 @@ MUTANTS = [
      "G2[(size_t)u * d + c] += lri * g1i[u] * g2i[c];", 0),
     ("mlp_no_gelu_on_query", "for (int u = 0; u < h; ++u) a1[u] = gelu_tanh(z1[u]);",
      "for (int u = 0; u < h; ++u) a1[u] = z1[u];", 0),
+    ("rope_sin_sign", "yr[ia] = xa * c - xb * s;\n            yr[ib] = xa * s + xb * c;",
+     "yr[ia] = xa * c + xb * s;\n            yr[ib] = -xa * s + xb * c;", 0),
+    ("rope_position_not_mod_K", "const real p = (real)(t % K);", "const real p = (real)t;", 0),
+    ("rope_frequency_exponent", "pow(theta, -2.0 * k / d)", "pow(theta, -1.0 * k / d)", 0),
+    ("rope_pairs_swapped", "const int ia = half_split ? k : 2 * k, ib = half_split ? k + half : 2 * k + 1;",
+     "const int ia = half_split ? 2 * k : k, ib = half_split ? 2 * k + 1 : k + half;", 0),
 ]
 
 
