@@ -363,6 +363,62 @@ def bench_linear_token_major(args, world, peaks):
             "replaced_permutes_ms": round(perm_ms, 4)}
 
 
+def bench_linear_rope(args, world, peaks, theta=10000.0):
+    """The headline scan with the rotary embedding of XQ and XK fused into its load path
+    (ttt_linear_forward_rope, pairs (2k, 2k+1), positions t mod K), and beside it the unfused way:
+    XQ and XK rotated by torch and written back in bf16 (the walkthrough's apply_rotary_pos_emb on
+    [B,H,L,d]), then the plain scan.  Also the HBM floor of any unfused pass: reading and writing
+    XQ and XK once at the measured copy bandwidth."""
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    w = synth.workload(2, L=args.seq_len)
+    x = synth.linear_inputs(w, values=False)
+    XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
+    lr, W0, b0, lnw, lnb = (dev_f32(x[k]) for k in ("lr", "W0", "b0", "ln_w", "ln_b"))
+    B, H, L = w.B, w.H, w.L
+    out = torch.empty_like(XQ)
+    Wl, bl = torch.empty(B, H, D, D, device="cuda"), torch.empty(B, H, D, device="cuda")
+    Wg, bg = torch.empty(B, H, D, D, device="cuda"), torch.empty(B, H, D, device="cuda")
+
+    def fused():
+        ttt.ttt_linear_forward_rope(XQ, XK, XV, lr, W0, b0, lnw, lnb, mini_batch=w.K, eps=w.eps, rope_theta=theta,
+                                    out=out, W_last=Wl, b_last=bl, W_grad_tail=Wg, b_grad_tail=bg, tail_grads=True)
+
+    K = max(3, min(args.steps, 10))
+    ms = time_steps(fused, K, 3, world)
+    ttt.ttt_device_status()
+    pos = (torch.arange(L, device="cuda") % w.K).float()
+    inv = 1.0 / theta ** (torch.arange(0, D, 2, device="cuda").float() / D)
+    cos, sin = torch.cos(pos[:, None] * inv), torch.sin(pos[:, None] * inv)  # [L, d/2], outside the timing
+    rq, rk = torch.empty_like(XQ), torch.empty_like(XK)
+
+    def rope_pass():
+        for src, dst in ((XQ, rq), (XK, rk)):
+            p = src.float().view(B, H, L, D // 2, 2)
+            a, b = p[..., 0], p[..., 1]
+            dst.copy_(torch.stack((a * cos - b * sin, a * sin + b * cos), -1).view(B, H, L, D))
+
+    def unfused():
+        rope_pass()
+        ttt.ttt_linear_forward(rq, rk, XV, lr, W0, b0, lnw, lnb, mini_batch=w.K, eps=w.eps, out=out, W_last=Wl,
+                               b_last=bl, W_grad_tail=Wg, b_grad_tail=bg, tail_grads=True)
+
+    rope_ms = time_steps(rope_pass, K, 3, world)
+    unfused_ms = time_steps(unfused, K, 3, world)
+    hbm = peaks[0]
+    nbytes = linear_bytes(B, H, L)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    pass_bytes = 4 * B * H * L * D * 2  # XQ, XK read and written once in bf16
+    return {"workload": f"ttt_linear_prefill_1b_layer_rope_B{B}_H{H}_L{L}", "rope": f"theta {theta:g}, pairs (2k, 2k+1)",
+            "value": round(world * B * L / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "steps": K, "gpu_launches": K,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "algorithmic_bytes": nbytes},
+            "unfused_ms": round(unfused_ms, 4), "unfused_rope_pass_ms": round(rope_ms, 4),
+            "unfused_rope_pass_hbm_floor_ms": round(pass_bytes / (hbm * 1e9) * 1e3, 4)}
+
+
 def bench_mlp(args, world, peaks):
     import torch
 
@@ -586,7 +642,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rows", default="linear,linear_tm,mlp,decode,decode_hist",
+    ap.add_argument("--rows", default="linear,linear_tm,linear_rope,mlp,decode,decode_hist",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=1,
@@ -613,6 +669,8 @@ def main():
         extra = {}
         if "linear_tm" in rows:
             extra["ttt_linear_prefill_token_major"] = bench_linear_token_major(args, world, peaks)
+        if "linear_rope" in rows:
+            extra["ttt_linear_prefill_rope"] = bench_linear_rope(args, world, peaks)
         if "mlp" in rows:
             extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
         if "decode" in rows:
@@ -629,6 +687,8 @@ def main():
     extra = {}
     if "linear_tm" in rows:
         extra["ttt_linear_prefill_token_major"] = bench_linear_token_major(args, world, peaks)
+    if "linear_rope" in rows:
+        extra["ttt_linear_prefill_rope"] = bench_linear_rope(args, world, peaks)
     if "mlp" in rows:
         extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
     if "decode" in rows:

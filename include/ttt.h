@@ -57,6 +57,9 @@ extern "C" {
  * projections and of the scan's return value in TTTBase.forward / TTTLinear.ttt -- instead of
  * the head-major [B,H,L,d].  lr stays [B,H,L].  The arithmetic and the results are the same. */
 #define TTT_FLAG_TOKEN_MAJOR 2u
+/* ttt_linear_forward_rope only: rotate the feature pairs (k, k + d/2) (the half-split rotation
+ * applied directly, without permute_qk / undo_permute_qk) instead of (2k, 2k+1). */
+#define TTT_FLAG_ROPE_HALF_SPLIT 4u
 
 /* Bits of the device status word */
 #define TTT_STATUS_TIMEOUT 1u /* a kernel gave up on a bounded wait and returned early */
@@ -124,7 +127,7 @@ int ttt_set_wait_limit(long long polls);
  *   eps          LayerNorm epsilon, > 0.
  *   dtype        TTT_F32 or TTT_BF16.
  *   flags        TTT_FLAG_FP32_COMPUTE and/or TTT_FLAG_TOKEN_MAJOR, or 0.  bf16 inputs run on
- *                the tensor-core kernel (bf16 operands, fp32 accumulation and fp32 state) unless
+ *                the tensor-core kernel (fp16 operands, fp32 accumulation and fp32 state) unless
  *                FP32_COMPUTE asks for the FFMA kernel; fp32 inputs always run on the FFMA
  *                kernel.  TOKEN_MAJOR: XQ, XK, XV and out are [B,L,H,d] instead of [B,H,L,d]
  *                (the walkthrough's [B,L,C] before its reshape/transpose and after the scan's
@@ -145,6 +148,34 @@ int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const flo
                        int H, long long L, int d, int mini_batch, float eps, int dtype,
                        unsigned int flags, void* out, float* W_last, float* b_last,
                        float* W_grad_tail, float* b_grad_tail, void* stream);
+
+/*
+ * ttt_linear_forward_rope -- ttt_linear_forward with the rotary position embedding of XQ and XK
+ * fused into the scan's load path ([walkthrough] TTTBase.forward: cos, sin = rotary_emb(XV,
+ * position_ids % mini_batch_size); permute_qk; apply_rotary_pos_emb; undo_permute_qk -- the
+ * rotation of RoFormer).  The scan sees, in place of XQ and XK (both for the contractions and
+ * for the reconstruction target XV - XK and the residual XQ + LN(Zbar)),
+ *   X'[t, 2k]   = X[t, 2k] cos(a) - X[t, 2k+1] sin(a)
+ *   X'[t, 2k+1] = X[t, 2k] sin(a) + X[t, 2k+1] cos(a),   a = (t mod K) * rope_theta^(-2k/d),
+ * for k = 0 .. d/2 - 1: the position restarts at 0 in every mini-batch (the tail mini-batch
+ * included), and the pairs (2k, 2k+1) are the net effect of permute_qk, the half-split rotation
+ * and undo_permute_qk.  With TTT_FLAG_ROPE_HALF_SPLIT the pairs are (k, k + d/2) instead.  The
+ * rotated activations exist only on chip (in fp16, the tensor-core operand type); XQ and XK in
+ * memory are not changed.  The angle is evaluated in fp32.
+ * Arguments and results are those of ttt_linear_forward, plus
+ *   rope_theta   the rotary base theta, finite and > 0 (the walkthrough does not print its value;
+ *                RoFormer's is 10000);
+ *   flags        TTT_FLAG_TOKEN_MAJOR and/or TTT_FLAG_ROPE_HALF_SPLIT, or 0;
+ * and the restrictions: dtype must be TTT_BF16 and TTT_FLAG_FP32_COMPUTE is not accepted (both
+ * TTT_ERR_UNSUPPORTED: the rotation lives in the tensor-core kernel only).  Errors otherwise as
+ * ttt_linear_forward, plus TTT_ERR_ARG for a bad rope_theta.
+ */
+int ttt_linear_forward_rope(const void* XQ, const void* XK, const void* XV, const float* lr,
+                            const float* token_eta, const float* W0, const float* b0,
+                            long long w0_batch_stride, const float* ln_w, const float* ln_b, int B,
+                            int H, long long L, int d, int mini_batch, float eps, float rope_theta,
+                            int dtype, unsigned int flags, void* out, float* W_last, float* b_last,
+                            float* W_grad_tail, float* b_grad_tail, void* stream);
 
 /*
  * ttt_linear_host_workspace_bytes -- size in bytes of the device workspace that

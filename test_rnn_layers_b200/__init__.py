@@ -28,11 +28,12 @@ TTT_F32 = 0
 TTT_BF16 = 1
 TTT_FLAG_FP32_COMPUTE = 1
 TTT_FLAG_TOKEN_MAJOR = 2
+TTT_FLAG_ROPE_HALF_SPLIT = 4
 TTT_STATUS_TIMEOUT = 1
 TTT_STATIC_SCRATCH_BYTES = 33554432
 
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
-           "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_host_workspace_bytes",
+           "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_forward_rope", "ttt_linear_host_workspace_bytes",
            "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward",
            "ttt_linear_decode_step", "ttt_linear_decode_step_hist")
 
@@ -65,6 +66,8 @@ def lib():
         L.ttt_set_wait_limit.argtypes = [ll]
         L.ttt_linear_forward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
                                          vp, fp, fp, fp, fp, vp]
+        L.ttt_linear_forward_rope.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, f, i, u,
+                                              vp, fp, fp, fp, fp, vp]
         L.ttt_linear_host_workspace_bytes.argtypes = [i, i, ll, i, i, i, i, ll]
         L.ttt_linear_host_workspace_bytes.restype = ll
         L.ttt_linear_forward_host.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
@@ -78,6 +81,7 @@ def lib():
         L.ttt_linear_decode_step_hist.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f,
                                                   i, vp, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
+                     "ttt_linear_forward_rope",
                      "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward", "ttt_linear_decode_step",
                      "ttt_linear_decode_step_hist"):
             getattr(L, name).restype = ctypes.c_int
@@ -161,6 +165,25 @@ def ttt_linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16,
     W0/b0: [H,64,64]/[H,64] shared over the batch, or [B,H,64,64]/[B,H,64] per chain.
     Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail).
     """
+    return _linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch, eps, token_eta, out, W_last, b_last,
+                           W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, None)
+
+
+def ttt_linear_forward_rope(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
+                            rope_theta: float = 10000.0, half_split: bool = False, token_eta=None, out=None,
+                            W_last=None, b_last=None, W_grad_tail=None, b_grad_tail=None,
+                            tail_grads: bool = False, flags: int = 0, token_major: bool = False, stream=None):
+    """ttt_linear_forward with the rotary embedding of XQ and XK (positions t mod K) fused into the scan.
+
+    Pairs (2k, 2k+1), or (k, k+32) with half_split; bf16 activations only (see include/ttt.h).
+    """
+    flags |= TTT_FLAG_ROPE_HALF_SPLIT if half_split else 0
+    return _linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch, eps, token_eta, out, W_last, b_last,
+                           W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, rope_theta)
+
+
+def _linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch, eps, token_eta, out, W_last, b_last,
+                    W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, rope_theta):
     _need(XQ, "XQ")
     B, H, L, d = _act_sizes(XQ, token_major)
     flags |= TTT_FLAG_TOKEN_MAJOR if token_major else 0
@@ -182,10 +205,14 @@ def ttt_linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16,
     if tail_grads:
         W_grad_tail = torch.empty((B, H, d, d), device=dev) if W_grad_tail is None else W_grad_tail
         b_grad_tail = torch.empty((B, H, d), device=dev) if b_grad_tail is None else b_grad_tail
-    rc = lib().ttt_linear_forward(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
-                                  H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
-                                  eps, _dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last),
-                                  _ptr(W_grad_tail), _ptr(b_grad_tail), _stream(stream))
+    head = (_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
+            H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch, eps)
+    tail = (_dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last), _ptr(W_grad_tail), _ptr(b_grad_tail),
+            _stream(stream))
+    if rope_theta is None:
+        rc = lib().ttt_linear_forward(*head, *tail)
+    else:
+        rc = lib().ttt_linear_forward_rope(*head, rope_theta, *tail)
     _check(rc)
     if tail_grads:
         return out, W_last, b_last, W_grad_tail, b_grad_tail

@@ -25,9 +25,20 @@
 //    1e-2 relative error on a few chains of the 1B-layer workload over its 512 updates, with
 //    fp16 operands (11-bit) every chain stays near 1e-3, at the same tensor throughput.  During
 //    mini-batch m the compute warps write the fp16 copy of the XQ and XK tiles of mini-batch
-//    m + 1 (one 16-byte chunk of each per thread; exact for the values bf16 inputs take up to
-//    |x| = 65504, larger ones saturate); the LayerNorm target, the residual and the tail grads
-//    read the bf16 tiles as loaded.
+//    m + 1 (one 16-byte chunk of each per thread; exact for bf16 magnitudes in [2^-17, 65504],
+//    larger ones saturate); the LayerNorm target, the residual and the tail grads read the bf16
+//    tiles as loaded.
+//  * Rotary position embedding (kRope, the walkthrough's TTTBase.forward: rotary_emb at
+//    position_ids % mini_batch_size, then apply_rotary_pos_emb between permute_qk and
+//    undo_permute_qk; RoFormer's rotation): XQ and XK are rotated inside that same fp16
+//    conversion, so the rotated activations never touch HBM.  A token's position inside its
+//    mini-batch is its tile row, the same in every mini-batch, so each thread keeps the cosines
+//    and sines of its one row and eight feature pairs in registers for the whole scan.  Each
+//    thread converts chunks j and j + 4 of one row of XQ or XK, which holds both partners of
+//    every pair it touches under either pair convention: (2k, 2k+1) -- the net effect of
+//    permute_qk, the half-split rotation and undo_permute_qk -- or (k, k + d/2) without the
+//    permutes.  The LayerNorm target, the residual and the tail grads then read the rotated
+//    fp16 tiles.
 //  * LayerNorm fused in registers: a thread holds 2 rows x 4 features; quads reduce by shuffles;
 //    the 4 warps' (sum, centred sum of squares) per row merge through shared memory with Chan's
 //    formula.  The loss gradient costs two 128-thread named barriers per mini-batch; the output
@@ -97,6 +108,36 @@ __device__ __forceinline__ void convert_chunk(uint32_t q_s, uint32_t k_s, uint32
                                  bf16x2_to_f16x2(vk.w)));
 }
 
+// Rotary embedding + fp16 conversion of chunks j (offset lo) and j + 4 (offset hi) of one row of
+// the XQ or XK tile at src, into the fp16 tile at dst.  (cs[n], sn[n]) are the cosine and sine of
+// pair angle n of this thread: half-split pairs (f, f + 32) for f = 8j + n (word n / 2, element
+// n % 2 of both chunks); adjacent pairs (2k, 2k+1) for k = 4j + n (word n of chunk j, n < 4) and
+// k = 4j + 12 + n (word n - 4 of chunk j + 4).  Rotation: (a, b) -> (a cos - b sin, a sin + b cos).
+__device__ __forceinline__ void rope_convert(uint32_t src, uint32_t dst, uint32_t lo, uint32_t hi,
+                                             const float (&cs)[8], const float (&sn)[8], bool half) {
+    const uint4 vl = lds128(src + lo), vh = lds128(src + hi);
+    const uint32_t wl[4] = {vl.x, vl.y, vl.z, vl.w}, wh[4] = {vh.x, vh.y, vh.z, vh.w};
+    uint32_t ol[4], oh[4];
+    if (half) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 a = unpack_bf16x2(wl[i]), b = unpack_bf16x2(wh[i]);
+            const float c0 = cs[2 * i], s0 = sn[2 * i], c1 = cs[2 * i + 1], s1 = sn[2 * i + 1];
+            ol[i] = pack_f16x2(fmaf(a.x, c0, -b.x * s0), fmaf(a.y, c1, -b.y * s1));
+            oh[i] = pack_f16x2(fmaf(a.x, s0, b.x * c0), fmaf(a.y, s1, b.y * c1));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 a = unpack_bf16x2(wl[i]), b = unpack_bf16x2(wh[i]);
+            ol[i] = pack_f16x2(fmaf(a.x, cs[i], -a.y * sn[i]), fmaf(a.x, sn[i], a.y * cs[i]));
+            oh[i] = pack_f16x2(fmaf(b.x, cs[4 + i], -b.y * sn[4 + i]), fmaf(b.x, sn[4 + i], b.y * cs[4 + i]));
+        }
+    }
+    sts128(dst + lo, make_uint4(ol[0], ol[1], ol[2], ol[3]));
+    sts128(dst + hi, make_uint4(oh[0], oh[1], oh[2], oh[3]));
+}
+
 // Sum over the 4 lanes of a quad (lanes sharing rows g, g+8).
 __device__ __forceinline__ float quad_sum(float v) {
     v += __shfl_xor_sync(0xffffffffu, v, 1);
@@ -137,8 +178,9 @@ __device__ __forceinline__ void merge_row(const float4 (*red)[2], int row, float
 
 // out rows of mini-batch mm = XQ + LN(Zbar), written straight from the accumulator layout:
 // rows g and g+8, features 16w + 8nt + 2t + {0,1} (rows past the mini-batch's end are skipped).
-// Consecutive tokens are 64 elements apart head-major, H * 64 token-major.
-template <bool kTok>
+// Consecutive tokens are 64 elements apart head-major, H * 64 token-major.  xq holds the residual
+// as fp16 pairs (kF16, the rotated XQ) or bf16 pairs (XQ as loaded).
+template <bool kTok, bool kF16>
 __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearArgs& a, __nv_bfloat16* out_chain, int mm, int K,
                                           int n_full, int g, int t, int w, const float (&zb)[2][4],
                                           const uint32_t (&xq)[4], const float (&lw)[2][2], const float (&lb)[2][2]) {
@@ -155,20 +197,20 @@ __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearAr
         const int f = 16 * w + 8 * nt + 2 * t;
         if (g < Km) {
             const float2 y = fma2(l2, fma2(make_float2(zb[nt][0], zb[nt][1]), bc2(rs0), bc2(-mu0 * rs0)), b2);
-            const float2 o = add2(unpack_bf16x2(xq[2 * nt]), y);
+            const float2 o = add2(kF16 ? unpack_f16x2(xq[2 * nt]) : unpack_bf16x2(xq[2 * nt]), y);
             *reinterpret_cast<uint32_t*>(out + g * ts + f) = pack_bf16x2(o.x, o.y);
         }
         if (g + 8 < Km) {
             const float2 y = fma2(l2, fma2(make_float2(zb[nt][2], zb[nt][3]), bc2(rs1), bc2(-mu1 * rs1)), b2);
-            const float2 o = add2(unpack_bf16x2(xq[2 * nt + 1]), y);
+            const float2 o = add2(kF16 ? unpack_f16x2(xq[2 * nt + 1]) : unpack_bf16x2(xq[2 * nt + 1]), y);
             *reinterpret_cast<uint32_t*>(out + (g + 8) * ts + f) = pack_bf16x2(o.x, o.y);
         }
     }
 }
 
 // kTok: token-major activations ([B, L, H, 64], 4-D tensor maps) or head-major ([B, H, L, 64],
-// 3-D tensor maps over [B*H, L, 64])
-template <bool kTok>
+// 3-D tensor maps over [B*H, L, 64]).  kRope: rotate XQ and XK (a.rope selects the pairs).
+template <bool kTok, bool kRope>
 __global__ void __launch_bounds__(kBlock, 2)
 linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // align by a byte offset from the shared array itself (an integer round trip of the pointer
@@ -315,15 +357,34 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         }
     float zbar_prev[2][4] = {};
     const uint32_t cvt_off = 16u * static_cast<uint32_t>(tid);  // this thread's chunk of a tile
-    auto stage_of = [&](int st_) {
-        return make_uint4(smem_u32(&s.xq[st_][0]), smem_u32(&s.xk[st_][0]), smem_u32(&s.xq16[st_][0]),
-                          smem_u32(&s.xk16[st_][0]));
+    // rotary embedding: warps 0-1 convert XQ, warps 2-3 XK; the thread's row rr takes rows rr and
+    // rr + 4 into one quarter-warp, so that its 16-byte accesses cover all 32 banks
+    const int ru = tid & 63, rr = ((ru >> 5) & 1) * 8 + ((ru >> 2) & 1) * 4 + ((ru >> 3) & 3), rj = ru & 3;
+    const uint32_t rlo = swz128(rr, rj), rhi = swz128(rr, rj + 4);
+    const bool rope_half = kRope && a.rope == 2;
+    float rcs[8], rsn[8];
+    if constexpr (kRope) {
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const int kp = rope_half ? 8 * rj + n : (n < 4 ? 4 * rj + n : 4 * rj + 12 + n);
+            // theta^(-2k/d) as the reciprocal of theta^(2k/d), the angle in fp32 at position rr
+            const float inv = 1.0f / powf(a.rope_theta, static_cast<float>(2 * kp) / TTT_D);
+            sincosf(static_cast<float>(rr) * inv, &rsn[n], &rcs[n]);
+        }
+    }
+    auto convert = [&](int st_) {
+        if constexpr (kRope) {
+            if (tid < 64) rope_convert(smem_u32(&s.xq[st_][0]), smem_u32(&s.xq16[st_][0]), rlo, rhi, rcs, rsn, rope_half);
+            else rope_convert(smem_u32(&s.xk[st_][0]), smem_u32(&s.xk16[st_][0]), rlo, rhi, rcs, rsn, rope_half);
+        } else {
+            convert_chunk(smem_u32(&s.xq[st_][0]), smem_u32(&s.xk[st_][0]), smem_u32(&s.xq16[st_][0]),
+                          smem_u32(&s.xk16[st_][0]), cvt_off);
+        }
     };
     // stage 0 landed and converted before the loop; stage m + 1 during mini-batch m
     if (n_mb > 0) {
         if (!mbar_wait_bounded(&s.full[0], 0, wait_limit, status)) s.fail = 1;
-        const uint4 sa = stage_of(0);
-        convert_chunk(sa.x, sa.y, sa.z, sa.w, cvt_off);
+        convert(0);
     }
     named_barrier_sync(1, kThreads);
     uint32_t xq_prev[4] = {};  // XQ at this thread's output positions (A fragment of k-slice w)
@@ -383,10 +444,11 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             mma_f16_16816(at[1], q[kk][0], q[kk][1], q[kk][2], q[kk][3], k[kk][1], k[kk][3]);
         }
         // XK and XQ at this thread's own positions: the A fragment of k-slice w (one more
-        // ldmatrix each is cheaper than selecting among the four slices held in registers)
+        // ldmatrix each is cheaper than selecting among the four slices held in registers);
+        // rotated, from the fp16 tiles, under kRope
         uint32_t k_own[4], q_own[4];
-        ldmatrix_x4(xk_s + own_off, k_own[0], k_own[1], k_own[2], k_own[3]);
-        ldmatrix_x4(xq_s + own_off, q_own[0], q_own[1], q_own[2], q_own[3]);
+        ldmatrix_x4((kRope ? xk16_s : xk_s) + own_off, k_own[0], k_own[1], k_own[2], k_own[3]);
+        ldmatrix_x4((kRope ? xq16_s : xq_s) + own_off, q_own[0], q_own[1], q_own[2], q_own[3]);
 
         // ---- LayerNorm statistics of Z --------------------------------------------------------
         {
@@ -404,10 +466,9 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         }
         if (m + 1 < n_mb) {  // fp16 copy of the next stage (seen by all warps after B2)
             if (!have_next && !mbar_wait_bounded(&s.full[st1], par1, wait_limit, status)) s.fail = 1;
-            const uint4 sa = stage_of(st1);
-            convert_chunk(sa.x, sa.y, sa.z, sa.w, cvt_off);
+            convert(st1);
         }
-        if (m > 0) store_out<kTok>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
+        if (m > 0) store_out<kTok, kRope>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
 
         // ---- g = ln_fused_l2_bwd(Z, XV - XK): partial sums of q and q * xhat -----------------
         float mu[2], rs[2];
@@ -421,7 +482,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {  // row g (hr=0) or g+8 (hr=1); A fragment order a0..a3
-                    const float2 kv = unpack_bf16x2(k_own[2 * nt + hr]);
+                    const float2 kv = kRope ? unpack_f16x2(k_own[2 * nt + hr]) : unpack_bf16x2(k_own[2 * nt + hr]);
                     const float2 vv = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(
                         &s.xv[st][0] + swz128(g + 8 * hr, 2 * w + nt) + 4 * t));
                     const float2 x = fma2(f2(z[nt][2 * hr], z[nt][2 * hr + 1]), bc2(rs[hr]), bc2(-mu[hr] * rs[hr]));
@@ -539,8 +600,9 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
                     const int r = i / TTT_D, c = i % TTT_D;
                     float acc = 0.f;
                     for (int j = 0; j < Km; ++j) {
-                        const float xkv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                            &s.xk[st][0] + swz128(j, r >> 3) + (r & 7) * 2));
+                        const uint32_t xo = swz128(j, r >> 3) + (r & 7) * 2;
+                        const float xkv = kRope ? __half2float(*reinterpret_cast<const __half*>(&s.xk16[st][0] + xo))
+                                                : __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&s.xk[st][0] + xo));
                         acc = fmaf(lr_s[j] * xkv, s.gtail[j][c], acc);
                     }
                     Wg[i] = acc;
@@ -562,7 +624,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // ---- the last mini-batch's output ---------------------------------------------------------
     if (n_mb > 0) {
         named_barrier_sync(1, kThreads);
-        store_out<kTok>(s.red3[(n_mb - 1) & 1], a, out_chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
+        store_out<kTok, kRope>(s.red3[(n_mb - 1) & 1], a, out_chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
     }
 
     // ---- final state ------------------------------------------------------------------------
@@ -590,7 +652,8 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
 
 cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t st) {
     const size_t smem = sizeof(TcSmem) + 1024;  // + alignment slack
-    auto kernel = a.tok_major ? linear_tc_kernel<true> : linear_tc_kernel<false>;
+    auto kernel = a.rope ? (a.tok_major ? linear_tc_kernel<true, true> : linear_tc_kernel<false, true>)
+                         : (a.tok_major ? linear_tc_kernel<true, false> : linear_tc_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(a.B * a.H), kBlock, smem, st>>>(a, maps);

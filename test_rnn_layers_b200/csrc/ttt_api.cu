@@ -187,7 +187,8 @@ unsigned int* status_word() { return device_word<g_ttt_status>(); }
 int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
                    const float* W0, const float* b0, long long w0_chain_stride, const float* ln_w, const float* ln_b,
                    int B, int H, long long L, int mini_batch, float eps, int dtype, unsigned int flags, void* out,
-                   float* W_last, float* b_last, float* W_grad_tail, float* b_grad_tail, cudaStream_t st) {
+                   float* W_last, float* b_last, float* W_grad_tail, float* b_grad_tail, cudaStream_t st,
+                   int rope = 0, float rope_theta = 0.f) {
     int rc;
     ttt::LinearArgs a{};
     a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
@@ -197,6 +198,8 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
     a.out = out; a.W_last = W_last; a.b_last = b_last; a.W_grad_tail = W_grad_tail; a.b_grad_tail = b_grad_tail;
     a.status = status_word();
     a.wait_limit = wait_limit();
+    a.rope = rope;
+    a.rope_theta = rope_theta;
     const bool tm = (flags & TTT_FLAG_TOKEN_MAJOR) != 0;
     set_act_strides(a, H, L, tm);
 
@@ -338,12 +341,14 @@ int ttt_device_status(void* stream, unsigned int* status, int clear) {
     return ok();
 }
 
-int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const float* lr,
-                       const float* token_eta, const float* W0, const float* b0,
-                       long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
-                       long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
-                       void* out, float* W_last, float* b_last, float* W_grad_tail,
-                       float* b_grad_tail, void* stream) {
+// ttt_linear_forward and ttt_linear_forward_rope: checks on the device pointers, then the launch.
+// rope: 0 none, 1 pairs (2k, 2k+1), 2 pairs (k, k + d/2); flags hold no rope bit here.
+static int linear_forward_checked(const void* XQ, const void* XK, const void* XV, const float* lr,
+                                  const float* token_eta, const float* W0, const float* b0,
+                                  long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                                  long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                                  int rope, float rope_theta, void* out, float* W_last, float* b_last,
+                                  float* W_grad_tail, float* b_grad_tail, void* stream) {
     int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
     if (rc) return rc;
     const long long chains = static_cast<long long>(B) * H;
@@ -380,7 +385,37 @@ int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const flo
 
     return enqueue_linear(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride ? per_head : 0, ln_w, ln_b, B, H, L,
                           mini_batch, eps, dtype, flags, out, W_last, b_last, W_grad_tail, b_grad_tail,
-                          static_cast<cudaStream_t>(stream));
+                          static_cast<cudaStream_t>(stream), rope, rope_theta);
+}
+
+int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const float* lr,
+                       const float* token_eta, const float* W0, const float* b0,
+                       long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                       long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                       void* out, float* W_last, float* b_last, float* W_grad_tail,
+                       float* b_grad_tail, void* stream) {
+    return linear_forward_checked(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d,
+                                  mini_batch, eps, dtype, flags, 0, 0.f, out, W_last, b_last, W_grad_tail,
+                                  b_grad_tail, stream);
+}
+
+int ttt_linear_forward_rope(const void* XQ, const void* XK, const void* XV, const float* lr,
+                            const float* token_eta, const float* W0, const float* b0,
+                            long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                            long long L, int d, int mini_batch, float eps, float rope_theta, int dtype,
+                            unsigned int flags, void* out, float* W_last, float* b_last, float* W_grad_tail,
+                            float* b_grad_tail, void* stream) {
+    if (!(rope_theta > 0.f) || !std::isfinite(rope_theta))
+        return fail(TTT_ERR_ARG, "rope_theta must be finite and > 0");
+    if (flags & TTT_FLAG_FP32_COMPUTE)
+        return fail(TTT_ERR_UNSUPPORTED, "the rotary embedding runs on the tensor-core kernel only (no FP32_COMPUTE)");
+    const unsigned int rest = flags & ~TTT_FLAG_ROPE_HALF_SPLIT;
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, rest);
+    if (rc) return rc;
+    if (dtype != TTT_BF16) return fail(TTT_ERR_UNSUPPORTED, "the rotary embedding takes bf16 activations only");
+    return linear_forward_checked(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d,
+                                  mini_batch, eps, dtype, rest, (flags & TTT_FLAG_ROPE_HALF_SPLIT) ? 2 : 1,
+                                  rope_theta, out, W_last, b_last, W_grad_tail, b_grad_tail, stream);
 }
 
 long long ttt_linear_host_workspace_bytes(int B, int H, long long L, int d, int mini_batch, int dtype,

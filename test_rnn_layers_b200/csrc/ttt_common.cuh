@@ -48,7 +48,8 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
     __half2 h = *reinterpret_cast<__half2*>(&v);
     return __half22float2(h);
 }
-// bf16x2 -> fp16x2 (exact for the magnitudes fp16 holds)
+// bf16x2 -> fp16x2: exact for magnitudes in [2^-17, 65504]; below 2^-17 the fp16 subnormal grid
+// leaves an absolute error under 2^-25, above 65504 the value saturates
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }

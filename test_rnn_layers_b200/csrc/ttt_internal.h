@@ -29,6 +29,10 @@ struct LinearArgs {
     // [B, H, L, d] (head-major): H*L*d, L*d, d;  [B, L, H, d] (token-major): L*H*d, d, H*d
     long long act_b, act_h, act_t;
     int tok_major;            // 1: token-major, the order of the tensor maps' coordinates
+    // rotary embedding of XQ and XK at position (token index mod K), tensor-core kernel only:
+    // 0 none, 1 pairs (2k, 2k+1), 2 pairs (k, k + d/2); angle of pair k = position * theta^(-2k/d)
+    int rope;
+    float rope_theta;
     void* out;
     float* W_last;
     float* b_last;

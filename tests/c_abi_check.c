@@ -49,6 +49,15 @@ int main(void) {
     check(ttt_linear_forward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 8,
                              out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_ARG, "forward rejects unknown flags");
 
+    check(ttt_linear_forward_rope(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, 0.0f, TTT_BF16,
+                                  0, out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_ARG, "rope forward rejects theta = 0");
+    check(ttt_linear_forward_rope(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, 1e4f, TTT_F32,
+                                  0, out, Wl, bl, NULL, NULL, NULL) == TTT_ERR_UNSUPPORTED,
+          "rope forward rejects fp32 activations");
+    check(ttt_linear_forward_rope(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, 1e4f, TTT_BF16,
+                                  TTT_FLAG_ROPE_HALF_SPLIT | TTT_FLAG_TOKEN_MAJOR, (void*)XK, Wl, bl, NULL, NULL,
+                                  NULL) == TTT_ERR_ALIAS, "rope forward accepts its flags, rejects out == XK");
+
     const long long ws = ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 1, 0);
     check(ws > 0 && ws % 256 == 0, "host workspace size");
     check(ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 9, 0) == TTT_ERR_ARG,

@@ -91,6 +91,31 @@ def test_linear_forward_rejects(libttt, kw, code):
     assert lib.ttt_last_error_message()
 
 
+def _fwd_rope(lib, theta=10000.0, **kw):
+    args = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W0=5 * A, b0=6 * A, stride=0, lnw=7 * A,
+                lnb=8 * A, B=2, H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, flags=0, out=9 * A,
+                Wl=10 * A, bl=11 * A, Wg=None, bg=None)
+    args.update(kw)
+    return lib.ttt_linear_forward_rope(args["XQ"], args["XK"], args["XV"], args["lr"], args["te"], args["W0"],
+                                       args["b0"], args["stride"], args["lnw"], args["lnb"], args["B"], args["H"],
+                                       args["L"], args["d"], args["K"], args["eps"], theta, args["dtype"],
+                                       args["flags"], args["out"], args["Wl"], args["bl"], args["Wg"], args["bg"],
+                                       None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(theta=0.0), -1), (dict(theta=-1.0), -1), (dict(theta=float("nan")), -1), (dict(theta=float("inf")), -1),
+    (dict(dtype=0), -6), (dict(flags=1), -6), (dict(flags=8), -1), (dict(flags=4 | 8), -1),
+    (dict(K=0), -1), (dict(d=32), -6), (dict(eps=0.0), -1), (dict(XQ=None), -1),
+    # the pair flag (4) and token-major (2) pass the flag check; the later checks still apply
+    (dict(flags=4, out=A), -3), (dict(flags=2 | 4, XK=2 * A + 2), -2), (dict(flags=2, Wl=5 * A), -3),
+])
+def test_linear_forward_rope_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _fwd_rope(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
 def test_linear_forward_L0_allows_null_activations_but_checks_state(libttt):
     lib = libttt.lib()
     assert _fwd(lib, L=0, XQ=None, XK=None, XV=None, lr=None, out=None, W0=None) == -1
