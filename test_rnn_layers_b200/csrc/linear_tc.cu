@@ -40,8 +40,13 @@
 //    permutes.  The LayerNorm target, the residual and the tail grads then read the rotated
 //    fp16 tiles.
 //  * LayerNorm fused in registers: a thread holds 2 rows x 4 features; quads reduce by shuffles;
-//    the 4 warps' (sum, centred sum of squares) per row merge through shared memory with Chan's
-//    formula.  The loss gradient costs two 128-thread named barriers per mini-batch; the output
+//    the 4 warps' (sum, sum of squares) per row merge through shared memory, and the variance is
+//    E[x^2] - mean^2 in fp32.  This one-pass form halves the shuffle depth of the statistics.  Its
+//    rounding grows with (mean / std)^2 of a row, and the scan cannot raise that ratio: the
+//    features of the LayerNorm gradient g sum to zero, so no update changes the mean over features
+//    of b or of any row of W, and a row's mean stays what W0 and b0 give it (about std / 8 for
+//    the walkthrough's initialisation, W0 ~ N(0, 0.02), b0 = 0).  The loss gradient costs two
+//    128-thread named barriers per mini-batch; the output
 //    LayerNorm of mini-batch m is finished during m+1 on the same barriers and stored straight
 //    from registers.  Shared-memory traffic is kept to the TMA tiles, the ldmatrix operand loads
 //    and a few hundred bytes of row statistics per mini-batch.
@@ -76,7 +81,7 @@ struct __align__(1024) TcSmem {
     float lr[kStages][TTT_KMAX];
     float te[TTT_KMAX];
     // per row, the four warps' partial statistics: [row][warp pair] = (w even: a, b, w odd: a, b)
-    float4 red1[TTT_KMAX][2];        // Z rows: (sum, centred sum of squares) over 16 features
+    float4 red1[TTT_KMAX][2];        // Z rows: (sum, sum of squares) over 16 features
     float4 red2[TTT_KMAX][2];        // (sum q, sum q * xhat)
     float4 red3[2][TTT_KMAX][2];     // Zbar rows, by mini-batch parity
     uint64_t full[kStages];          // stage loaded (1 expect-tx arrival + 16 lr arrivals)
@@ -99,13 +104,14 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
-// This thread's 16-byte chunk (of 128) of the XQ and XK tiles of a stage, converted to fp16.
-__device__ __forceinline__ void convert_chunk(uint32_t q_s, uint32_t k_s, uint32_t q16, uint32_t k16, uint32_t off) {
-    const uint4 vq = lds128(q_s + off), vk = lds128(k_s + off);
-    sts128(q16 + off, make_uint4(bf16x2_to_f16x2(vq.x), bf16x2_to_f16x2(vq.y), bf16x2_to_f16x2(vq.z),
-                                 bf16x2_to_f16x2(vq.w)));
-    sts128(k16 + off, make_uint4(bf16x2_to_f16x2(vk.x), bf16x2_to_f16x2(vk.y), bf16x2_to_f16x2(vk.z),
-                                 bf16x2_to_f16x2(vk.w)));
+// This thread's 16-byte chunk (of 128) of the XQ and XK tiles of a stage, converted to fp16 (plain
+// loads and stores, so that the compiler can interleave them with the output epilogue).
+__device__ __forceinline__ void convert_plain(const uint8_t* q, const uint8_t* k, uint8_t* q16, uint8_t* k16, uint32_t off) {
+    const uint4 vq = *reinterpret_cast<const uint4*>(q + off), vk = *reinterpret_cast<const uint4*>(k + off);
+    *reinterpret_cast<uint4*>(q16 + off) = make_uint4(bf16x2_to_f16x2(vq.x), bf16x2_to_f16x2(vq.y), bf16x2_to_f16x2(vq.z),
+                                                      bf16x2_to_f16x2(vq.w));
+    *reinterpret_cast<uint4*>(k16 + off) = make_uint4(bf16x2_to_f16x2(vk.x), bf16x2_to_f16x2(vk.y), bf16x2_to_f16x2(vk.z),
+                                                      bf16x2_to_f16x2(vk.w));
 }
 
 // Rotary embedding + fp16 conversion of chunks j (offset lo) and j + 4 (offset hi) of one row of
@@ -146,34 +152,36 @@ __device__ __forceinline__ float quad_sum(float v) {
 }
 
 // Per-warp row partials of a [16 x 16-feature] slice held as v[nt][0..3] (rows g and g+8):
-// (sum, centred sum of squares) over this warp's 16 features for each of the 2 rows.
+// (sum, sum of squares) over this warp's 16 features for each of the 2 rows, the two quad
+// reductions side by side.
 __device__ __forceinline__ void warp_row_partials(const float (&v)[2][4], float2& r0, float2& r1) {
     const float2 a0 = make_float2(v[0][0], v[0][1]), a1 = make_float2(v[1][0], v[1][1]);  // row g
     const float2 b0 = make_float2(v[0][2], v[0][3]), b1 = make_float2(v[1][2], v[1][3]);  // row g+8
     const float2 sa = __fadd2_rn(a0, a1), sb = __fadd2_rn(b0, b1);
-    const float s0 = quad_sum(sa.x + sa.y), s1 = quad_sum(sb.x + sb.y);
-    const float2 m0 = make_float2(-s0 * (1.0f / 16), -s0 * (1.0f / 16));
-    const float2 m1 = make_float2(-s1 * (1.0f / 16), -s1 * (1.0f / 16));
-    const float2 da0 = __fadd2_rn(a0, m0), da1 = __fadd2_rn(a1, m0);
-    const float2 db0 = __fadd2_rn(b0, m1), db1 = __fadd2_rn(b1, m1);
-    const float2 ca = __ffma2_rn(da1, da1, __fmul2_rn(da0, da0));
-    const float2 cb = __ffma2_rn(db1, db1, __fmul2_rn(db0, db0));
-    r0 = make_float2(s0, quad_sum(ca.x + ca.y));
-    r1 = make_float2(s1, quad_sum(cb.x + cb.y));
+    const float2 qa = __ffma2_rn(a1, a1, __fmul2_rn(a0, a0)), qb = __ffma2_rn(b1, b1, __fmul2_rn(b0, b0));
+    float s0 = sa.x + sa.y, s1 = sb.x + sb.y, q0 = qa.x + qa.y, q1 = qb.x + qb.y;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        q0 += __shfl_xor_sync(0xffffffffu, q0, o);
+        q1 += __shfl_xor_sync(0xffffffffu, q1, o);
+    }
+    r0 = make_float2(s0, q0);
+    r1 = make_float2(s1, q1);
 }
 
 __device__ __forceinline__ void put_partial(float4 (*red)[2], int row, int w, float2 v) {
     reinterpret_cast<float2*>(&red[row][w >> 1])[w & 1] = v;
 }
 
-// Merge the 4 warps' (sum, centred sum of squares) of one row: mean and 1/sqrt(var + eps).
+// Merge the 4 warps' (sum, sum of squares) of one row: mean and 1/sqrt(var + eps), with the
+// variance E[x^2] - mean^2 (clamped at zero against rounding).
 __device__ __forceinline__ void merge_row(const float4 (*red)[2], int row, float eps, float& mu, float& rstd) {
     const float4 a = red[row][0], b = red[row][1];
     mu = ((a.x + a.z) + (b.x + b.z)) * (1.0f / TTT_D);
-    const float d0 = a.x * (1.0f / 16) - mu, d1 = a.z * (1.0f / 16) - mu;
-    const float d2 = b.x * (1.0f / 16) - mu, d3 = b.z * (1.0f / 16) - mu;
-    const float m2 = (a.y + a.w) + (b.y + b.w) + 16.0f * (d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3);
-    rstd = rsqrtf(m2 * (1.0f / TTT_D) + eps);
+    const float ex2 = ((a.y + a.w) + (b.y + b.w)) * (1.0f / TTT_D);
+    rstd = rsqrtf(fmaxf(fmaf(-mu, mu, ex2), 0.f) + eps);
 }
 
 // out rows of mini-batch mm = XQ + LN(Zbar), written straight from the accumulator layout:
@@ -183,11 +191,12 @@ __device__ __forceinline__ void merge_row(const float4 (*red)[2], int row, float
 template <bool kTok, bool kF16>
 __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearArgs& a, __nv_bfloat16* out_chain, int mm, int K,
                                           int n_full, int g, int t, int w, const float (&zb)[2][4],
-                                          const uint32_t (&xq)[4], const float (&lw)[2][2], const float (&lb)[2][2]) {
+                                          const uint32_t (&xq)[4], const float (&lw)[2][2], const float (&lb)[2][2],
+                                          bool valid = true) {
     float mu0, rs0, mu1, rs1;
     merge_row(red, g, a.eps, mu0, rs0);
     merge_row(red, g + 8, a.eps, mu1, rs1);
-    const int Km = mm < n_full ? K : static_cast<int>(a.rem);
+    const int Km = !valid ? 0 : mm < n_full ? K : static_cast<int>(a.rem);
     const long long ts = kTok ? a.act_t : TTT_D;
     __nv_bfloat16* out = out_chain + static_cast<long long>(mm) * K * ts;
 #pragma unroll
@@ -377,8 +386,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             if (tid < 64) rope_convert(smem_u32(&s.xq[st_][0]), smem_u32(&s.xq16[st_][0]), rlo, rhi, rcs, rsn, rope_half);
             else rope_convert(smem_u32(&s.xk[st_][0]), smem_u32(&s.xk16[st_][0]), rlo, rhi, rcs, rsn, rope_half);
         } else {
-            convert_chunk(smem_u32(&s.xq[st_][0]), smem_u32(&s.xk[st_][0]), smem_u32(&s.xq16[st_][0]),
-                          smem_u32(&s.xk16[st_][0]), cvt_off);
+            convert_plain(&s.xq[st_][0], &s.xk[st_][0], &s.xq16[st_][0], &s.xk16[st_][0], cvt_off);
         }
     };
     // stage 0 landed and converted before the loop; stage m + 1 during mini-batch m
@@ -397,6 +405,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         const int Km = full_mb ? K : static_cast<int>(a.rem);
         const int st1 = st + 1 == kStages ? 0 : st + 1;
         const uint32_t par1 = par ^ (st1 == 0 ? 1u : 0u);
+        // the next stage: tested now, so that the test's latency hides behind the MMAs below
         // the next stage: tested now, so that the test's latency hides behind the MMAs below
         bool have_next = (m + 1 < n_mb) && mbar_test_wait(&s.full[st1], par1);
         const uint32_t xq_s = smem_u32(&s.xq[st][0]), xk_s = smem_u32(&s.xk[st][0]);
@@ -464,11 +473,9 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             failed = true;
             break;
         }
-        if (m + 1 < n_mb) {  // fp16 copy of the next stage (seen by all warps after B2)
-            if (!have_next && !mbar_wait_bounded(&s.full[st1], par1, wait_limit, status)) s.fail = 1;
-            convert(st1);
-        }
-        if (m > 0) store_out<kTok, kRope>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
+        if (m + 1 < n_mb && !have_next && !mbar_wait_bounded(&s.full[st1], par1, wait_limit, status)) s.fail = 1;
+        convert(st1);  // on the last mini-batch a harmless conversion of stale data
+        store_out<kTok, kRope>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb, m > 0);
 
         // ---- g = ln_fused_l2_bwd(Z, XV - XK): partial sums of q and q * xhat -----------------
         float mu[2], rs[2];

@@ -122,3 +122,26 @@ def test_decode_wide_inputs(libttt, hist):
     print(f"\n[wide inputs] decode ({'history' if hist else 'dense'} cache): out worst {worst:.2e}, "
           f"W {eW:.2e}, b {eb:.2e}")
     assert eW <= TOL and eb <= TOL
+
+
+@pytest.mark.parametrize("offset,flags", [(0.25, 0), (1.0, 0), (4.0, 1)], ids=["b0+0.25", "b0+1", "b0+4_fp32"])
+def test_linear_row_mean_offset(libttt, offset, flags):
+    """A common offset in b0 gives every row of Z and Zbar a mean of `offset` against a spread of
+    about 0.02 (mean / std up to 200).  The tensor-core kernel takes the variance in one pass,
+    E[x^2] - mean^2 in fp32, whose rounding grows with (mean / std)^2: it holds the 1e-2 bar up to
+    mean / std = 50 (offset 1) -- the scan never raises that ratio, since the features of the
+    LayerNorm gradient sum to zero and leave the feature means of W and b unchanged -- and
+    TTT_FLAG_FP32_COMPUTE (two-pass statistics) covers larger ones."""
+    w = synth.workload(1, B=2, H=4, L=16 * 64 + 5, seed=0x0FF5)
+    x = synth.linear_inputs(w)
+    x["b0"] = (x["b0"] + offset).astype(np.float32)
+    out, Wl, bl, Wg, bg = libttt.ttt_linear_forward(
+        dev_act(x, "XQ"), dev_act(x, "XK"), dev_act(x, "XV"), dev_f32(x["lr"]), dev_f32(x["W0"]), dev_f32(x["b0"]),
+        dev_f32(x["ln_w"]), dev_f32(x["ln_b"]), mini_batch=w.K, eps=w.eps, tail_grads=True, flags=flags)
+    torch.cuda.synchronize()
+    ref = oracle.default().linear_forward(x["XQ"], x["XK"], x["XV"], x["lr"], x["W0"], x["b0"], x["ln_w"],
+                                          x["ln_b"], w.K, w.eps)
+    e = _errs({n: (to_np(t).reshape(w.chains, -1), ref[n].reshape(w.chains, -1))
+               for n, t in (("out", out), ("W_last", Wl), ("b_last", bl), ("W_grad_tail", Wg), ("b_grad_tail", bg))})
+    print(f"\n[row mean offset {offset}, flags {flags}]:", {k: f"{v:.2e}" for k, v in e.items()})
+    assert max(e.values()) <= TOL, e
