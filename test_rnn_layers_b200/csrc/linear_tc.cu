@@ -95,15 +95,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 bc2(float a) { return make_float2(a, a); }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                 : "memory");
-}
 // This thread's 16-byte chunk (of 128) of the XQ and XK tiles of a stage, converted to fp16 (plain
 // loads and stores, so that the compiler can interleave them with the output epilogue).
 __device__ __forceinline__ void convert_plain(const uint8_t* q, const uint8_t* k, uint8_t* q16, uint8_t* k16, uint32_t off) {
@@ -115,33 +106,35 @@ __device__ __forceinline__ void convert_plain(const uint8_t* q, const uint8_t* k
 }
 
 // Rotary embedding + fp16 conversion of chunks j (offset lo) and j + 4 (offset hi) of one row of
-// the XQ or XK tile at src, into the fp16 tile at dst.  (cs[n], sn[n]) are the cosine and sine of
-// pair angle n of this thread: half-split pairs (f, f + 32) for f = 8j + n (word n / 2, element
-// n % 2 of both chunks); adjacent pairs (2k, 2k+1) for k = 4j + n (word n of chunk j, n < 4) and
-// k = 4j + 12 + n (word n - 4 of chunk j + 4).  Rotation: (a, b) -> (a cos - b sin, a sin + b cos).
-__device__ __forceinline__ void rope_convert(uint32_t src, uint32_t dst, uint32_t lo, uint32_t hi,
-                                             const float (&cs)[8], const float (&sn)[8], bool half) {
-    const uint4 vl = lds128(src + lo), vh = lds128(src + hi);
+// the XQ or XK tile at src, into the fp16 tile at dst (plain loads and stores, free to interleave
+// with the surrounding code).  kHalf: pairs (f, f + 32) for f = 8j + n, word n / 2 and element
+// n % 2 of both chunks, with c[i] = (cos, cos), c[4 + i] = (sin, sin) and ns[i] = (-sin, -sin) of
+// angles 2i and 2i + 1 (paired FMAs); otherwise pairs (2k, 2k+1), word n of the two chunks read
+// as one run of eight words (k = 4j + n for n < 4, 4j + 12 + n after), with c[n] = (cos, sin)
+// and ns unused (scalar FMAs: a second coefficient pair per angle would not fit the registers).
+// Rotation: (a, b) -> (a cos - b sin, a sin + b cos).
+template <bool kHalf>
+__device__ __forceinline__ void rope_convert(const uint8_t* src, uint8_t* dst, uint32_t lo, uint32_t hi,
+                                             const float2 (&c)[8], const float2 (&ns)[8]) {
+    const uint4 vl = *reinterpret_cast<const uint4*>(src + lo), vh = *reinterpret_cast<const uint4*>(src + hi);
     const uint32_t wl[4] = {vl.x, vl.y, vl.z, vl.w}, wh[4] = {vh.x, vh.y, vh.z, vh.w};
     uint32_t ol[4], oh[4];
-    if (half) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 a = unpack_bf16x2(wl[i]), b = unpack_bf16x2(wh[i]);
-            const float c0 = cs[2 * i], s0 = sn[2 * i], c1 = cs[2 * i + 1], s1 = sn[2 * i + 1];
-            ol[i] = pack_f16x2(fmaf(a.x, c0, -b.x * s0), fmaf(a.y, c1, -b.y * s1));
-            oh[i] = pack_f16x2(fmaf(a.x, s0, b.x * c0), fmaf(a.y, s1, b.y * c1));
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = unpack_bf16x2(wl[i]), y = unpack_bf16x2(wh[i]);
+        float2 u, v;
+        if constexpr (kHalf) {
+            u = __ffma2_rn(x, c[i], __fmul2_rn(y, ns[i]));
+            v = __ffma2_rn(x, c[4 + i], __fmul2_rn(y, c[i]));
+        } else {
+            u = make_float2(fmaf(x.x, c[i].x, -x.y * c[i].y), fmaf(x.x, c[i].y, x.y * c[i].x));
+            v = make_float2(fmaf(y.x, c[4 + i].x, -y.y * c[4 + i].y), fmaf(y.x, c[4 + i].y, y.y * c[4 + i].x));
         }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 a = unpack_bf16x2(wl[i]), b = unpack_bf16x2(wh[i]);
-            ol[i] = pack_f16x2(fmaf(a.x, cs[i], -a.y * sn[i]), fmaf(a.x, sn[i], a.y * cs[i]));
-            oh[i] = pack_f16x2(fmaf(b.x, cs[4 + i], -b.y * sn[4 + i]), fmaf(b.x, sn[4 + i], b.y * cs[4 + i]));
-        }
+        ol[i] = pack_f16x2(u.x, u.y);
+        oh[i] = pack_f16x2(v.x, v.y);
     }
-    sts128(dst + lo, make_uint4(ol[0], ol[1], ol[2], ol[3]));
-    sts128(dst + hi, make_uint4(oh[0], oh[1], oh[2], oh[3]));
+    *reinterpret_cast<uint4*>(dst + lo) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+    *reinterpret_cast<uint4*>(dst + hi) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
 }
 
 // Sum over the 4 lanes of a quad (lanes sharing rows g, g+8).
@@ -218,8 +211,9 @@ __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearAr
 }
 
 // kTok: token-major activations ([B, L, H, 64], 4-D tensor maps) or head-major ([B, H, L, 64],
-// 3-D tensor maps over [B*H, L, 64]).  kRope: rotate XQ and XK (a.rope selects the pairs).
-template <bool kTok, bool kRope>
+// 3-D tensor maps over [B*H, L, 64]).  kRope: rotate XQ and XK, pairs (2k, 2k+1) (1) or
+// (k, k + d/2) (2); 0: no rotation.
+template <bool kTok, int kRope>
 __global__ void __launch_bounds__(kBlock, 2)
 linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // align by a byte offset from the shared array itself (an integer round trip of the pointer
@@ -370,21 +364,32 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // rr + 4 into one quarter-warp, so that its 16-byte accesses cover all 32 banks
     const int ru = tid & 63, rr = ((ru >> 5) & 1) * 8 + ((ru >> 2) & 1) * 4 + ((ru >> 3) & 3), rj = ru & 3;
     const uint32_t rlo = swz128(rr, rj), rhi = swz128(rr, rj + 4);
-    const bool rope_half = kRope && a.rope == 2;
-    float rcs[8], rsn[8];
-    if constexpr (kRope) {
+    float2 rc[8], rn[8];  // the rotation coefficients of this thread, laid out as rope_convert reads them
+                          // (rn only for the half-split pairs)
+    if constexpr (kRope != 0) {
+        float cs[8], sn[8];
 #pragma unroll
         for (int n = 0; n < 8; ++n) {
-            const int kp = rope_half ? 8 * rj + n : (n < 4 ? 4 * rj + n : 4 * rj + 12 + n);
+            const int kp = kRope == 2 ? 8 * rj + n : (n < 4 ? 4 * rj + n : 4 * rj + 12 + n);
             // theta^(-2k/d) as the reciprocal of theta^(2k/d), the angle in fp32 at position rr
             const float inv = 1.0f / powf(a.rope_theta, static_cast<float>(2 * kp) / TTT_D);
-            sincosf(static_cast<float>(rr) * inv, &rsn[n], &rcs[n]);
+            sincosf(static_cast<float>(rr) * inv, &sn[n], &cs[n]);
+        }
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            if constexpr (kRope == 2) {
+                rc[n] = n < 4 ? f2(cs[2 * n], cs[2 * n + 1]) : f2(sn[2 * n - 8], sn[2 * n - 7]);
+                rn[n] = n < 4 ? f2(-sn[2 * n], -sn[2 * n + 1]) : f2(0.f, 0.f);
+            } else {
+                rc[n] = f2(cs[n], sn[n]);
+                rn[n] = f2(0.f, 0.f);
+            }
         }
     }
     auto convert = [&](int st_) {
-        if constexpr (kRope) {
-            if (tid < 64) rope_convert(smem_u32(&s.xq[st_][0]), smem_u32(&s.xq16[st_][0]), rlo, rhi, rcs, rsn, rope_half);
-            else rope_convert(smem_u32(&s.xk[st_][0]), smem_u32(&s.xk16[st_][0]), rlo, rhi, rcs, rsn, rope_half);
+        if constexpr (kRope != 0) {
+            if (tid < 64) rope_convert<kRope == 2>(&s.xq[st_][0], &s.xq16[st_][0], rlo, rhi, rc, rn);
+            else rope_convert<kRope == 2>(&s.xk[st_][0], &s.xk16[st_][0], rlo, rhi, rc, rn);
         } else {
             convert_plain(&s.xq[st_][0], &s.xk[st_][0], &s.xq16[st_][0], &s.xk16[st_][0], cvt_off);
         }
@@ -456,8 +461,8 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         // ldmatrix each is cheaper than selecting among the four slices held in registers);
         // rotated, from the fp16 tiles, under kRope
         uint32_t k_own[4], q_own[4];
-        ldmatrix_x4((kRope ? xk16_s : xk_s) + own_off, k_own[0], k_own[1], k_own[2], k_own[3]);
-        ldmatrix_x4((kRope ? xq16_s : xq_s) + own_off, q_own[0], q_own[1], q_own[2], q_own[3]);
+        ldmatrix_x4((kRope != 0 ? xk16_s : xk_s) + own_off, k_own[0], k_own[1], k_own[2], k_own[3]);
+        ldmatrix_x4((kRope != 0 ? xq16_s : xq_s) + own_off, q_own[0], q_own[1], q_own[2], q_own[3]);
 
         // ---- LayerNorm statistics of Z --------------------------------------------------------
         {
@@ -475,7 +480,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         }
         if (m + 1 < n_mb && !have_next && !mbar_wait_bounded(&s.full[st1], par1, wait_limit, status)) s.fail = 1;
         convert(st1);  // on the last mini-batch a harmless conversion of stale data
-        store_out<kTok, kRope>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb, m > 0);
+        store_out<kTok, kRope != 0>(s.red3[(m - 1) & 1], a, out_chain, m - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb, m > 0);
 
         // ---- g = ln_fused_l2_bwd(Z, XV - XK): partial sums of q and q * xhat -----------------
         float mu[2], rs[2];
@@ -489,7 +494,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
             for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {  // row g (hr=0) or g+8 (hr=1); A fragment order a0..a3
-                    const float2 kv = kRope ? unpack_f16x2(k_own[2 * nt + hr]) : unpack_bf16x2(k_own[2 * nt + hr]);
+                    const float2 kv = kRope != 0 ? unpack_f16x2(k_own[2 * nt + hr]) : unpack_bf16x2(k_own[2 * nt + hr]);
                     const float2 vv = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(
                         &s.xv[st][0] + swz128(g + 8 * hr, 2 * w + nt) + 4 * t));
                     const float2 x = fma2(f2(z[nt][2 * hr], z[nt][2 * hr + 1]), bc2(rs[hr]), bc2(-mu[hr] * rs[hr]));
@@ -608,7 +613,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
                     float acc = 0.f;
                     for (int j = 0; j < Km; ++j) {
                         const uint32_t xo = swz128(j, r >> 3) + (r & 7) * 2;
-                        const float xkv = kRope ? __half2float(*reinterpret_cast<const __half*>(&s.xk16[st][0] + xo))
+                        const float xkv = kRope != 0 ? __half2float(*reinterpret_cast<const __half*>(&s.xk16[st][0] + xo))
                                                 : __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&s.xk[st][0] + xo));
                         acc = fmaf(lr_s[j] * xkv, s.gtail[j][c], acc);
                     }
@@ -631,7 +636,7 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // ---- the last mini-batch's output ---------------------------------------------------------
     if (n_mb > 0) {
         named_barrier_sync(1, kThreads);
-        store_out<kTok, kRope>(s.red3[(n_mb - 1) & 1], a, out_chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
+        store_out<kTok, kRope != 0>(s.red3[(n_mb - 1) & 1], a, out_chain, n_mb - 1, K, n_full, g, t, w, zbar_prev, xq_prev, lw, lb);
     }
 
     // ---- final state ------------------------------------------------------------------------
@@ -659,8 +664,9 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
 
 cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t st) {
     const size_t smem = sizeof(TcSmem) + 1024;  // + alignment slack
-    auto kernel = a.rope ? (a.tok_major ? linear_tc_kernel<true, true> : linear_tc_kernel<false, true>)
-                         : (a.tok_major ? linear_tc_kernel<true, false> : linear_tc_kernel<false, false>);
+    auto kernel = a.rope == 2 ? (a.tok_major ? linear_tc_kernel<true, 2> : linear_tc_kernel<false, 2>)
+                : a.rope == 1 ? (a.tok_major ? linear_tc_kernel<true, 1> : linear_tc_kernel<false, 1>)
+                              : (a.tok_major ? linear_tc_kernel<true, 0> : linear_tc_kernel<false, 0>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(a.B * a.H), kBlock, smem, st>>>(a, maps);
