@@ -54,11 +54,12 @@ def load(path: str | None = None):
     lib.oracle_ttt_linear_decode_chain.argtypes = [_D, _D, _D, dbl, _D, _D, _D, _D, _D, _D, _D,
                                                    i, i, _LL, dbl, _D, ctypes.POINTER(i)]
     lib.oracle_rope.argtypes = [_D, _LL, i, i, dbl, i, _D]
+    lib.oracle_post_norm_o_proj.argtypes = [_D, _LL, i, _D, _D, dbl, _D, i, _D]
     lib.oracle_ttt_mlp_chain.argtypes = [_D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _LL, i, i, i,
                                          dbl, _D, _D, _D, _D, _D]
     for f in ("oracle_partition", "oracle_lnl2_grad", "oracle_ln_forward", "oracle_gelu_tanh",
               "oracle_ttt_linear_chain", "oracle_ttt_linear_decode_chain", "oracle_ttt_mlp_chain",
-              "oracle_rope"):
+              "oracle_rope", "oracle_post_norm_o_proj"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -120,6 +121,16 @@ class Oracle:
             self._check(self.lib.oracle_rope(self._p(xc), L, d, K, float(theta), 1 if half_split else 0,
                                              self._p(yc)), "rope")
             flat_y[c] = yc
+        return y
+
+    def post_norm_o_proj(self, x, ln_w, ln_b, eps, Wo):
+        """y = o_proj(post_norm(x)) per token: x [T, C], ln_w / ln_b [C], Wo [N, C] (out x in)."""
+        x, ln_w, ln_b, Wo = map(self._f64, (x, ln_w, ln_b, Wo))
+        T, C = x.shape
+        N = Wo.shape[0]
+        y = np.empty((T, N))
+        self._check(self.lib.oracle_post_norm_o_proj(self._p(x), T, C, self._p(ln_w), self._p(ln_b), float(eps),
+                                                     self._p(Wo), N, self._p(y)), "post_norm_o_proj")
         return y
 
     # ---- TTT-Linear ------------------------------------------------------------------------

@@ -478,3 +478,30 @@ int oracle_ttt_mlp_chain(const real* xq, const real* xk, const real* xv, /* [L][
     for (int k = 0; k < nall; ++k) free(all[k]);
     return ORACLE_OK;
 }
+
+/* ---------------------------------------------------------------------------------------- */
+/* The output side of the layer ([walkthrough] TTTBase.forward, after the concatenation of    */
+/* the mini-batch outputs): y = o_proj(post_norm(x)) per token.  post_norm is a LayerNorm over  */
+/* the C = num_heads * head_dim features of the token (affine ln_w, ln_b; biased variance, eps  */
+/* inside the square root, as every LayerNorm here), o_proj a linear map without bias,          */
+/* y[n] = sum_k LN(x)[k] * Wo[n][k], with Wo stored [N][C] (out x in).  The page names both     */
+/* modules and shows neither body; apply_gate ("Mamba only" on the page) is not applied.        */
+/* x: [T][C], y: [T][N].                                                                        */
+int oracle_post_norm_o_proj(const real* x, long long T, int C, const real* ln_w, const real* ln_b,
+                            real eps, const real* Wo, int N, real* y) {
+    if (T < 0 || C < 1 || N < 1 || !ln_w || !ln_b || !Wo || (T > 0 && (!x || !y))) return ORACLE_ERR_ARG;
+    real* u = (real*)malloc(sizeof(real) * (size_t)C);
+    if (!u) return ORACLE_ERR_ARG;
+    for (long long t = 0; t < T; ++t) {
+        ln_forward(x + (size_t)t * C, ln_w, ln_b, C, eps, u);
+        real* yt = y + (size_t)t * N;
+        for (int n = 0; n < N; ++n) {
+            const real* wn = Wo + (size_t)n * C;
+            real acc = 0.0;
+            for (int k = 0; k < C; ++k) acc += u[k] * wn[k];
+            yt[n] = acc;
+        }
+    }
+    free(u);
+    return ORACLE_OK;
+}

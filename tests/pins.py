@@ -375,4 +375,43 @@ def pin_rope_torch_restatement(o):
             assert _rel(o.rope(x, 16, theta, half), _rope_torch(x, 16, theta, not half)) < 1e-13
 
 
+def _post_norm_case(seed, T=9, C=24, N=10):
+    rng = _rng(seed)
+    x = rng.normal(0.3, 1.5, (T, C))
+    return x, 1 + rng.normal(0, 0.2, C), rng.normal(0, 0.2, C), rng.normal(0, 0.3, (N, C))
+
+
+def pin_post_norm_identity_is_layer_norm(o):
+    # o_proj = identity reduces the step to a LayerNorm over the token's C features
+    x, w, b, _ = _post_norm_case(31)
+    ref = torch.nn.functional.layer_norm(torch.as_tensor(x), (x.shape[1],), torch.as_tensor(w),
+                                         torch.as_tensor(b), eps=1e-5).numpy()
+    assert _rel(o.post_norm_o_proj(x, w, b, 1e-5, np.eye(x.shape[1])), ref) < 1e-13
+
+
+def pin_post_norm_single_entry_weight(o):
+    # a weight with one nonzero entry Wo[n0][k0] copies feature k0 of the normalised token into
+    # output n0 and nothing else (fixes the orientation of Wo)
+    x, w, b, _ = _post_norm_case(32)
+    C = x.shape[1]
+    ln = o.post_norm_o_proj(x, w, b, 1e-5, np.eye(C))
+    Wo = np.zeros((7, C))
+    Wo[5, 2] = 2.5
+    y = o.post_norm_o_proj(x, w, b, 1e-5, Wo)
+    assert np.allclose(y[:, 5], 2.5 * ln[:, 2], rtol=1e-13, atol=1e-14)
+    assert not np.delete(y, 5, axis=1).any()
+
+
+def pin_post_norm_invariances(o):
+    # linear in Wo; blind to a per-token shift of x; with ln_w = 0 every token maps to Wo ln_b
+    x, w, b, W1 = _post_norm_case(33)
+    W2 = _rng(34).normal(0, 0.3, W1.shape)
+    y1, y2 = o.post_norm_o_proj(x, w, b, 1e-5, W1), o.post_norm_o_proj(x, w, b, 1e-5, W2)
+    assert _rel(o.post_norm_o_proj(x, w, b, 1e-5, W1 + 2 * W2), y1 + 2 * y2) < 1e-13
+    shift = _rng(35).normal(0, 3, (x.shape[0], 1))
+    assert _rel(o.post_norm_o_proj(x + shift, w, b, 1e-5, W1), y1) < 1e-12
+    y0 = o.post_norm_o_proj(x, np.zeros_like(w), b, 1e-5, W1)
+    assert np.allclose(y0, np.broadcast_to(W1 @ b, y0.shape), rtol=1e-13, atol=1e-14)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -47,6 +47,12 @@ MUTANTS = [
     ("rope_frequency_exponent", "pow(theta, -2.0 * k / d)", "pow(theta, -1.0 * k / d)", 0),
     ("rope_pairs_swapped", "const int ia = half_split ? k : 2 * k, ib = half_split ? k + half : 2 * k + 1;",
      "const int ia = half_split ? 2 * k : k, ib = half_split ? 2 * k + 1 : k + half;", 0),
+    ("o_proj_transposed", "const real* wn = Wo + (size_t)n * C;\n            real acc = 0.0;\n            for (int k = 0; k < C; ++k) acc += u[k] * wn[k];",
+     "real acc = 0.0;\n            for (int k = 0; k < C && k < N; ++k) acc += u[k] * Wo[(size_t)k * C + n];", 0),
+    ("post_norm_skipped", "        ln_forward(x + (size_t)t * C, ln_w, ln_b, C, eps, u);",
+     "        for (int k = 0; k < C; ++k) u[k] = x[(size_t)t * C + k];", 0),
+    ("post_norm_no_affine", "        ln_forward(x + (size_t)t * C, ln_w, ln_b, C, eps, u);",
+     "        ln_forward(x + (size_t)t * C, ln_w, ln_b, C, eps, u);\n        for (int k = 0; k < C; ++k) u[k] = (u[k] - ln_b[k]) / ln_w[k];", 0),
 ]
 
 
