@@ -419,6 +419,46 @@ def bench_linear_rope(args, world, peaks, theta=10000.0):
             "unfused_rope_pass_hbm_floor_ms": round(pass_bytes / (hbm * 1e9) * 1e3, 4)}
 
 
+def bench_post_norm_oproj(args, world, peaks):
+    """The layer's output side at the 1B layer, Y = o_proj(post_norm(X)) for the scan's
+    token-major output ([B*L, 2048] bf16): one tcgen05 GEMM with the LayerNorm folded into its
+    epilogue (ttt_post_norm_o_proj; the weight packed once beforehand, outside the timing), and
+    beside it the unfused torch way (layer_norm, then a cuBLAS matmul)."""
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    B, L, C = 8, args.seq_len, 2048
+    T = B * L
+    d = synth.oproj_inputs(0x0B5, T, C, C, values=False)
+    bits = lambda b, shape: torch.from_numpy(np.ascontiguousarray(b).view(np.int16).reshape(shape)).cuda().view(
+        torch.bfloat16)
+    X, Wo = bits(d["X_bits"], (T, C)), bits(d["Wo_bits"], (C, C))
+    ln_w, ln_b = torch.from_numpy(d["ln_w"]).cuda(), torch.from_numpy(d["ln_b"]).cuda()
+    Wp, u, v = ttt.ttt_o_proj_prepare(Wo, ln_w, ln_b)
+    Y = torch.empty_like(X)
+
+    def fused():
+        ttt.ttt_post_norm_o_proj(X, Wp, u, v, eps=1e-6, Y=Y)
+
+    K = max(3, min(args.steps, 20))
+    ms = time_steps(fused, K, 3, world)
+    ttt.ttt_device_status()
+
+    def unfused():
+        torch.matmul(torch.nn.functional.layer_norm(X, (C,), ln_w.bfloat16(), ln_b.bfloat16(), 1e-6), Wo.t(), out=Y)
+
+    torch_ms = time_steps(unfused, K, 3, world)
+    flops = 2.0 * T * C * C
+    peak = peaks[1]
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": f"ttt_post_norm_o_proj_1b_layer_T{T}_C{C}", "value": round(world * T / (ms / 1e3), 1),
+            "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": K, "gpu_launches": K,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,
+                         "peak_source": ("measured" if peaks[3] == "measured" else "fallback") + " bf16_tflops",
+                         "unit": "TFLOP/s", "frac": round(tf / peak, 4), "algorithmic_flops": int(flops)},
+            "unfused_torch_ms": round(torch_ms, 4)}
+
+
 def bench_mlp(args, world, peaks):
     import torch
 
@@ -645,7 +685,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rows", default="linear,linear_tm,linear_rope,mlp,decode,decode_hist",
+    ap.add_argument("--rows", default="linear,linear_tm,linear_rope,oproj,mlp,decode,decode_hist",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=1,
@@ -674,6 +714,8 @@ def main():
             extra["ttt_linear_prefill_token_major"] = bench_linear_token_major(args, world, peaks)
         if "linear_rope" in rows:
             extra["ttt_linear_prefill_rope"] = bench_linear_rope(args, world, peaks)
+        if "oproj" in rows:
+            extra["ttt_post_norm_o_proj"] = bench_post_norm_oproj(args, world, peaks)
         if "mlp" in rows:
             extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
         if "decode" in rows:
@@ -692,6 +734,8 @@ def main():
         extra["ttt_linear_prefill_token_major"] = bench_linear_token_major(args, world, peaks)
     if "linear_rope" in rows:
         extra["ttt_linear_prefill_rope"] = bench_linear_rope(args, world, peaks)
+    if "oproj" in rows:
+        extra["ttt_post_norm_o_proj"] = bench_post_norm_oproj(args, world, peaks)
     if "mlp" in rows:
         extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
     if "decode" in rows:

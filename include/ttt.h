@@ -343,6 +343,58 @@ int ttt_linear_decode_step_hist(const void* xq, const void* xk, const void* xv, 
                                 float* hist, float* b_grad, int B, int H, int d, int mini_batch,
                                 long long seqlen_offset, float eps, int dtype, void* out, void* stream);
 
+/*
+ * The layer's output side: Y = o_proj(post_norm(X)) per token ([walkthrough] TTTBase.forward,
+ * after torch.cat of the mini-batch outputs: post_norm, then o_proj; apply_gate is "Mamba only"
+ * on the page and is not part of this path).  Readings, as in the oracle: post_norm is a
+ * LayerNorm over the token's C = num_heads * head_dim features (affine ln_w, ln_b; biased
+ * variance; eps inside the square root), o_proj a linear map without bias whose weight Wo is
+ * stored [N][C] (out x in, the layout of torch's nn.Linear.weight).  X is the scan's output
+ * taken token-major: [B, L, num_heads * 64] = [T, C] (ttt_linear_forward with
+ * TTT_FLAG_TOKEN_MAJOR writes exactly that), T = B * L.
+ *
+ * The LayerNorm folds into the product: y[n] = rstd (sum_k x_k Wp[n][k] - mean u[n]) + v[n],
+ * with Wp[n][k] = ln_w[k] Wo[n][k], u[n] = sum_k Wp[n][k], v[n] = sum_k ln_b[k] Wo[n][k].
+ * ttt_o_proj_prepare packs those once per weight; ttt_post_norm_o_proj then runs one
+ * tensor-core GEMM (tcgen05, fp32 accumulation in tensor memory) whose epilogue applies the
+ * token statistics, taken from the same X tiles in one pass over C (Chan's merge per 64
+ * features).  Y is rounded to bf16.  The correction subtracts mean * u[n] from the product in
+ * fp32, so its accuracy falls as a token's |mean| / std grows (the scan's output has mean near
+ * zero next to its spread).
+ *
+ * Sizes: C a positive multiple of 64, N a positive multiple of 256 (both hold for the 125M and
+ * 1B layers, C = N = 768 and 2048); T >= 0, at most 65535 * 128 tokens.
+ */
+
+/*
+ * ttt_o_proj_prepare -- pack o_proj's weight for ttt_post_norm_o_proj.
+ *   Wo           [N][C] bf16 (device), 16-byte aligned: the o_proj weight (out x in).
+ *   ln_w, ln_b   [C] float32 (device): post_norm's affine parameters.
+ *   Wp           [N][C] bf16 (device, caller-allocated), 16-byte aligned: receives ln_w[k] * Wo[n][k].
+ *   u, v         [N] float32 (device, caller-allocated): receive sum_k Wp[n][k] (of the rounded
+ *                Wp) and sum_k ln_b[k] Wo[n][k].
+ * Asynchronous on `stream`.  Errors: TTT_ERR_UNSUPPORTED for C or N outside the sizes above,
+ * TTT_ERR_ARG for a null pointer, TTT_ERR_ALIGN, TTT_ERR_ALIAS if an output overlaps an input
+ * or another output, TTT_ERR_CUDA if the launch fails.  (No counterpart on the pages: it is the
+ * one-time weight transform of the fused form above.)
+ */
+int ttt_o_proj_prepare(const void* Wo, const float* ln_w, const float* ln_b, int C, int N, void* Wp, float* u,
+                       float* v, void* stream);
+
+/*
+ * ttt_post_norm_o_proj -- Y = o_proj(post_norm(X)) for T tokens.
+ *   X            [T][C] bf16 (device), 16-byte aligned (NULL allowed when T == 0).
+ *   Wp, u, v     from ttt_o_proj_prepare for this weight and these post_norm parameters.
+ *   eps          post_norm's epsilon, finite and > 0.
+ *   Y            [T][N] bf16 (device, caller-allocated), 16-byte aligned; must not overlap the
+ *                inputs.
+ * Asynchronous on `stream`; allocates nothing.  T == 0 does nothing.  Errors as
+ * ttt_o_proj_prepare, plus TTT_ERR_ARG for a bad eps or T < 0, TTT_ERR_UNSUPPORTED for T above
+ * 65535 * 128.  The kernel's waits are bounded (see ttt_device_status).
+ */
+int ttt_post_norm_o_proj(const void* X, long long T, int C, const void* Wp, const float* u, const float* v, int N,
+                         float eps, void* Y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,6 +26,7 @@ _LIB_PATH = os.path.join(_HERE, "libsynth.so")
 TAG = {
     "XQ": 1, "XK": 2, "XV": 3, "LR": 4, "W0": 5, "LNW": 6, "LNB": 7,
     "W1": 8, "W2": 9, "B0": 10, "B1": 11, "B2": 12,
+    "ONX": 13, "ONW": 14, "ONLW": 15, "ONLB": 16,
 }
 
 SEED_BASE = 0x77170000
@@ -234,3 +235,20 @@ def random_bias(w: Workload, tag: str, shape, std: float = 0.02) -> np.ndarray:
 
 def chain_index(b: int, h: int, H: int) -> int:
     return b * H + h
+
+
+def oproj_inputs(seed: int, T: int, C: int, N: int, x_std: float = 1.0, w_std: float = 0.02,
+                 ln_w_std: float = 0.1, ln_b_std: float = 0.1, values: bool = True) -> dict:
+    """Inputs of the layer's output side (post_norm, then o_proj): X [T, C] bf16 shaped like the
+    scan's output (XQ + LN(Zbar): about unit spread per feature), the o_proj weight Wo [N, C] bf16
+    ~ N(0, w_std), post_norm's ln_w ~ 1 + N(0, ln_w_std) and ln_b ~ N(0, ln_b_std) [C] fp32.
+    Returns X_bits / Wo_bits (uint16 bf16 patterns), and X / Wo as their fp32 values when asked."""
+    x = normal(seed, TAG["ONX"], T * C, 0, 0.0, x_std).reshape(T, C)
+    wo = normal(seed, TAG["ONW"], N * C, 0, 0.0, w_std).reshape(N, C)
+    out = {"X_bits": f32_to_bf16_bits(x), "Wo_bits": f32_to_bf16_bits(wo),
+           "ln_w": normal(seed, TAG["ONLW"], C, 0, 1.0, ln_w_std),
+           "ln_b": normal(seed, TAG["ONLB"], C, 0, 0.0, ln_b_std)}
+    if values:
+        out["X"] = bf16_bits_to_f32(out["X_bits"])
+        out["Wo"] = bf16_bits_to_f32(out["Wo_bits"])
+    return out

@@ -35,7 +35,7 @@ TTT_STATIC_SCRATCH_BYTES = 33554432
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
            "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_forward_rope", "ttt_linear_host_workspace_bytes",
            "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward",
-           "ttt_linear_decode_step", "ttt_linear_decode_step_hist")
+           "ttt_linear_decode_step", "ttt_linear_decode_step_hist", "ttt_o_proj_prepare", "ttt_post_norm_o_proj")
 
 
 class TTTError(RuntimeError):
@@ -80,7 +80,10 @@ def lib():
                                              vp, vp]
         L.ttt_linear_decode_step_hist.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f,
                                                   i, vp, vp]
+        L.ttt_o_proj_prepare.argtypes = [vp, fp, fp, i, i, vp, fp, fp, vp]
+        L.ttt_post_norm_o_proj.argtypes = [vp, ll, i, vp, fp, fp, i, f, vp, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
+                     "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
                      "ttt_linear_forward_rope",
                      "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward", "ttt_linear_decode_step",
                      "ttt_linear_decode_step_hist"):
@@ -428,3 +431,38 @@ def ttt_linear_decode_step_hist(xq, xk, xv, lr, ln_w, ln_b, W, b, hist, b_grad, 
                                            mini_batch, seqlen_offset, eps, _dtype_code(xq), _ptr(out), _stream(stream))
     _check(rc)
     return out
+
+
+def ttt_o_proj_prepare(Wo, ln_w, ln_b, Wp=None, u=None, v=None, stream=None):
+    """Pack o_proj's weight Wo [N, C] (bf16, nn.Linear layout) with post_norm's ln_w, ln_b [C]:
+    returns (Wp, u, v) for ttt_post_norm_o_proj (see include/ttt.h)."""
+    _need(Wo, "Wo", torch.bfloat16)
+    if Wo.dim() != 2:
+        raise ValueError("Wo must be [N, C]")
+    N, C = Wo.shape
+    _need(ln_w, "ln_w", torch.float32, (C,))
+    _need(ln_b, "ln_b", torch.float32, (C,))
+    dev = Wo.device
+    Wp = torch.empty_like(Wo) if Wp is None else _need(Wp, "Wp", torch.bfloat16, (N, C))
+    u = torch.empty(N, device=dev) if u is None else _need(u, "u", torch.float32, (N,))
+    v = torch.empty(N, device=dev) if v is None else _need(v, "v", torch.float32, (N,))
+    _check(lib().ttt_o_proj_prepare(_ptr(Wo), _ptr(ln_w), _ptr(ln_b), C, N, _ptr(Wp), _ptr(u), _ptr(v),
+                                    _stream(stream)))
+    return Wp, u, v
+
+
+def ttt_post_norm_o_proj(X, Wp, u, v, eps: float = 1e-6, Y=None, stream=None):
+    """Y = o_proj(post_norm(X)) for X [..., C] bf16 (the token-major scan output), with (Wp, u, v)
+    from ttt_o_proj_prepare; returns Y [..., N] bf16."""
+    _need(X, "X", torch.bfloat16)
+    _need(Wp, "Wp", torch.bfloat16)
+    N, C = Wp.shape
+    if X.shape[-1] != C:
+        raise ValueError(f"X's last dimension must be C = {C}, got {tuple(X.shape)}")
+    _need(u, "u", torch.float32, (N,))
+    _need(v, "v", torch.float32, (N,))
+    T = X.numel() // C
+    Y = torch.empty((*X.shape[:-1], N), dtype=torch.bfloat16, device=X.device) if Y is None else \
+        _need(Y, "Y", torch.bfloat16, (*X.shape[:-1], N))
+    _check(lib().ttt_post_norm_o_proj(_ptr(X), T, C, _ptr(Wp), _ptr(u), _ptr(v), N, eps, _ptr(Y), _stream(stream)))
+    return Y

@@ -676,6 +676,80 @@ int ttt_linear_decode_step_hist(const void* xq, const void* xk, const void* xv, 
     return ok();
 }
 
+// ---- the layer's output side: post_norm + o_proj ---------------------------------------------
+static int check_oproj_sizes(int C, int N) {
+    if (C < 64 || C % 64 != 0) return fail(TTT_ERR_UNSUPPORTED, "C must be a positive multiple of 64 (got %d)", C);
+    if (N < 256 || N % 256 != 0) return fail(TTT_ERR_UNSUPPORTED, "N must be a positive multiple of 256 (got %d)", N);
+    if (static_cast<long long>(C) * N > (1ll << 31) - 1) return fail(TTT_ERR_ARG, "C*N too large");
+    return TTT_OK;
+}
+
+int ttt_o_proj_prepare(const void* Wo, const float* ln_w, const float* ln_b, int C, int N, void* Wp, float* u,
+                       float* v, void* stream) {
+    int rc = check_oproj_sizes(C, N);
+    if (rc) return rc;
+    if (!Wo || !ln_w || !ln_b || !Wp || !u || !v) return fail(TTT_ERR_ARG, "every pointer must be non-null");
+    if (!aligned(Wo, 16) || !aligned(Wp, 16)) return fail(TTT_ERR_ALIGN, "Wo and Wp must be 16-byte aligned");
+    const void* a4[] = {ln_w, ln_b, u, v};
+    const char* n4[] = {"ln_w", "ln_b", "u", "v"};
+    for (int i = 0; i < 4; ++i)
+        if (!aligned(a4[i], 4)) return fail(TTT_ERR_ALIGN, "%s must be 4-byte aligned", n4[i]);
+    const size_t w = static_cast<size_t>(C) * N * 2;
+    Span in[] = {{"Wo", Wo, w}, {"ln_w", ln_w, static_cast<size_t>(C) * 4}, {"ln_b", ln_b, static_cast<size_t>(C) * 4}};
+    Span outs[] = {{"Wp", Wp, w}, {"u", u, static_cast<size_t>(N) * 4}, {"v", v, static_cast<size_t>(N) * 4}};
+    if ((rc = check_aliasing(in, 3, outs, 3))) return rc;
+    cudaError_t e = ttt::launch_oproj_prepare(Wo, ln_w, ln_b, C, N, Wp, u, v, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_o_proj_prepare launch");
+    return ok();
+}
+
+// A [rows][cols] bf16 matrix as a 2-D tensor map with 128-byte swizzle and a {64, box_rows} box.
+static int encode_rows_map(CUtensorMap* map, const void* base, long long rows, int cols, int box_rows,
+                           const char* name) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return fail(TTT_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TTT_ERR_CUDA, "tensor map for %s: cuTensorMapEncodeTiled error %d", name, (int)r);
+    return TTT_OK;
+}
+
+int ttt_post_norm_o_proj(const void* X, long long T, int C, const void* Wp, const float* u, const float* v, int N,
+                         float eps, void* Y, void* stream) {
+    int rc = check_oproj_sizes(C, N);
+    if (rc) return rc;
+    if (T < 0) return fail(TTT_ERR_ARG, "T must be >= 0 (got %lld)", T);
+    if (T > 65535ll * 128) return fail(TTT_ERR_UNSUPPORTED, "T above 65535 * 128 tokens (got %lld)", T);
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(TTT_ERR_ARG, "eps must be finite and > 0");
+    if (!Wp || !u || !v) return fail(TTT_ERR_ARG, "Wp, u and v must be non-null");
+    if (T > 0 && (!X || !Y)) return fail(TTT_ERR_ARG, "X and Y must be non-null when T > 0");
+    const void* a16[] = {X, Wp, Y};
+    const char* n16[] = {"X", "Wp", "Y"};
+    for (int i = 0; i < 3; ++i)
+        if (a16[i] && !aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "%s must be 16-byte aligned", n16[i]);
+    if (!aligned(u, 4) || !aligned(v, 4)) return fail(TTT_ERR_ALIGN, "u and v must be 4-byte aligned");
+    Span in[] = {{"X", X, static_cast<size_t>(T) * C * 2}, {"Wp", Wp, static_cast<size_t>(C) * N * 2},
+                 {"u", u, static_cast<size_t>(N) * 4}, {"v", v, static_cast<size_t>(N) * 4}};
+    Span outs[] = {{"Y", Y, static_cast<size_t>(T) * N * 2}};
+    if ((rc = check_aliasing(in, 4, outs, 1))) return rc;
+    if (T == 0) return ok();
+    ttt::OprojMaps maps;
+    if ((rc = encode_rows_map(&maps.x, X, T, C, 128, "X"))) return rc;
+    if ((rc = encode_rows_map(&maps.w, Wp, N, C, 256, "Wp"))) return rc;
+    ttt::OprojArgs a{};
+    a.T = T; a.C = C; a.N = N; a.eps = eps; a.u = u; a.v = v; a.Y = Y;
+    a.status = status_word();
+    a.wait_limit = wait_limit();
+    cudaError_t e = ttt::launch_post_norm_oproj(a, maps, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ttt_post_norm_o_proj launch");
+    return ok();
+}
+
 }  // extern "C"
 
 // ---- host-buffer entry that allocates nothing ---------------------------------------------------

@@ -123,6 +123,24 @@ struct LinearMaps {
 };
 
 // launchers (return cudaSuccess or the launch error)
+// The layer's output side, Y = o_proj(post_norm(X)) (see ttt_post_norm_o_proj).
+struct OprojArgs {
+    long long T;              // tokens (rows of X and Y)
+    int C;                    // features of X (the post-norm width), a multiple of 64
+    int N;                    // outputs (rows of the packed weight), a multiple of 256
+    float eps;
+    const float* u;           // [N] sum_k Wp[n][k]
+    const float* v;           // [N] sum_k ln_b[k] Wo[n][k]
+    void* Y;                  // [T][N] bf16
+    unsigned int* status;
+    long long wait_limit;
+};
+struct OprojMaps {
+    CUtensorMap x, w;         // X [T][C] box {64, 128}; Wp [N][C] box {64, 256}; bf16, 128-byte swizzle
+};
+cudaError_t launch_oproj_prepare(const void* Wo, const float* ln_w, const float* ln_b, int C, int N, void* Wp,
+                                 float* u, float* v, cudaStream_t s);
+cudaError_t launch_post_norm_oproj(const OprojArgs& a, const OprojMaps& maps, cudaStream_t s);
 cudaError_t launch_linear_simt(const LinearArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t s);
 cudaError_t launch_linear_state_copy(const LinearArgs& a, cudaStream_t s);

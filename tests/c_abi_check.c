@@ -58,6 +58,13 @@ int main(void) {
                                   TTT_FLAG_ROPE_HALF_SPLIT | TTT_FLAG_TOKEN_MAJOR, (void*)XK, Wl, bl, NULL, NULL,
                                   NULL) == TTT_ERR_ALIAS, "rope forward accepts its flags, rejects out == XK");
 
+    check(ttt_o_proj_prepare(XQ, W0, b0, 2048, 100, out, Wl, bl, NULL) == TTT_ERR_UNSUPPORTED,
+          "o_proj prepare rejects N = 100");
+    check(ttt_post_norm_o_proj(XQ, 65600, 2048, XK, W0, b0, 2048, 0.0f, out, NULL) == TTT_ERR_ARG,
+          "post_norm o_proj rejects eps = 0");
+    check(ttt_post_norm_o_proj(NULL, 0, 2048, XK, W0, b0, 2048, 1e-6f, NULL, NULL) == TTT_OK,
+          "post_norm o_proj with T = 0 is a no-op");
+
     const long long ws = ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 1, 0);
     check(ws > 0 && ws % 256 == 0, "host workspace size");
     check(ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 9, 0) == TTT_ERR_ARG,

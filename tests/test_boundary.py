@@ -259,3 +259,43 @@ def test_last_error_message_is_per_host_thread(libttt):
         t.join()
     assert got["K"][0] == -1 and b"mini_batch" in got["K"][1]
     assert got["align"][0] == -2 and b"aligned" in got["align"][1]
+
+
+def _prep(lib, **kw):
+    a = dict(Wo=A, lnw=2 * A, lnb=3 * A, C=2048, N=2048, Wp=4 * A, u=5 * A, v=6 * A)
+    a.update(kw)
+    return lib.ttt_o_proj_prepare(a["Wo"], a["lnw"], a["lnb"], a["C"], a["N"], a["Wp"], a["u"], a["v"], None)
+
+
+def _onorm(lib, **kw):
+    a = dict(X=A, T=65600, C=2048, Wp=8 * A, u=9 * A, v=10 * A, N=2048, eps=1e-6, Y=1 << 30)
+    a.update(kw)
+    return lib.ttt_post_norm_o_proj(a["X"], a["T"], a["C"], a["Wp"], a["u"], a["v"], a["N"], a["eps"], a["Y"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(C=32), -6), (dict(C=100), -6), (dict(N=128), -6), (dict(N=300), -6), (dict(Wo=None), -1),
+    (dict(v=None), -1), (dict(Wo=A + 8), -2), (dict(Wp=4 * A + 4), -2), (dict(u=5 * A + 2), -2),
+    (dict(Wp=A + 64), -3), (dict(u=4 * A + 16), -3), (dict(v=5 * A), -3),
+])
+def test_o_proj_prepare_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _prep(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=-1), -1), (dict(T=65535 * 128 + 1), -6), (dict(C=96), -6), (dict(N=512 + 64), -6),
+    (dict(eps=0.0), -1), (dict(eps=float("inf")), -1), (dict(X=None), -1), (dict(Wp=None), -1),
+    (dict(X=A + 2), -2), (dict(Y=(1 << 30) + 8), -2), (dict(u=9 * A + 1), -2),
+    (dict(Y=A), -3), (dict(Y=8 * A - 64), -3),
+])
+def test_post_norm_o_proj_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _onorm(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
+def test_post_norm_o_proj_T0_is_a_no_op(libttt):
+    lib = libttt.lib()
+    assert _onorm(lib, T=0, X=None, Y=None) == 0
