@@ -11,19 +11,23 @@
 // the rounded Wp, so the correction matches what the MMAs multiply), and the statistics are
 // taken from the same X tiles while they stream through shared memory for the MMAs.
 //
-// Design (one CTA per 128 x 256 output tile; grid x = output tile, y = token tile, so the 8
-// CTAs of a token tile run side by side and share its X tiles through L2):
+// Design: a persistent kernel, one CTA per SM, walking 128 x 256 output tiles (output tile
+// fastest, so the CTAs at work at any moment share their X tiles through L2), four roles:
 //  * warp 0 streams X [128 tokens x 64 features] and Wp [256 outputs x 64 features] tiles by TMA
-//    (128-byte swizzle, no multicast) into a ring of kStages stages with full / empty mbarriers;
-//  * warp 1 allocates 256 tensor-memory columns and issues, from one thread, four
-//    tcgen05.mma (kind::f16, bf16 operands, M = 128, N = 256, K = 16, fp32 accumulator in
-//    tensor memory) per stage, committing each stage's MMAs to its empty barrier;
-//  * warps 2-5 (the epilogue warps) take token row r = 32 (warp % 4) + lane of every X tile as it
-//    lands and fold its 64 values into the row's (mean, centred sum of squares) with Chan's
-//    formula, then, once the last MMA has committed, read their accumulator lane back in
-//    16-column pieces (tcgen05.ld 32x32b), apply rstd (acc - mu u) + v and store bf16.
-// Every mbarrier wait is bounded; on expiry the status word is raised, the stores are skipped,
-// the tensor core and the loads in flight are drained (bounded) and tensor memory is freed.
+//    (128-byte swizzle, no multicast) into a ring of kStages stages with full / empty mbarriers,
+//    across tile boundaries;
+//  * warp 1 allocates all 512 tensor-memory columns -- two fp32 accumulators of 128 x 256 -- and
+//    issues, from one thread, four tcgen05.mma (kind::f16, bf16 operands, M = 128, N = 256,
+//    K = 16) per stage into the tile's accumulator, committing each stage to its empty barrier
+//    and each finished tile to its accumulator's full barrier;
+//  * warps 2-5 (statistics) take token row r = 32 (warp % 4) + lane of every X tile as it lands
+//    and fold its 64 values into the row's (mean, centred sum of squares) with Chan's formula,
+//    handing (mean, rstd) per row to the epilogue through a double buffer;
+//  * warps 6-9 (epilogue) read their accumulator lane back (tcgen05.ld 32x32b, 64 columns per
+//    wait), apply rstd (acc - mean u) + v and store bf16, then free the accumulator -- while the
+//    MMAs of the next tile already run into the other one.
+// Every mbarrier wait is bounded; on expiry the status word is raised, every role stops, the
+// tensor core and the loads in flight are drained (bounded) and tensor memory is freed.
 #include "tc5.cuh"
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
@@ -33,19 +37,24 @@ namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 192;                       // producer, MMA, 4 epilogue warps
+constexpr int kThreads = 320;                       // producer, MMA, 4 statistics, 4 epilogue warps
 constexpr uint32_t kTileA = kBM * kBK * 2;          // 16 KB
 constexpr uint32_t kTileB = kBN * kBK * 2;          // 32 KB
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;                 // two 256-column accumulators
 constexpr long long kDrainPolls = 1ll << 24;
 
 struct __align__(1024) OpSmem {
     uint8_t a[kStages][kTileA];
     uint8_t b[kStages][kTileB];
-    float u[kBN], v[kBN];
+    float2 stats[2][kBM];      // (mean, rstd) of the tile's rows, by accumulator buffer
+    float uv[4][2][kBN];       // the tile's u and v, one copy per epilogue warp
     uint64_t full[kStages];
-    uint64_t empty[kStages];   // the MMA commit + one arrival per epilogue warp
-    uint64_t acc_full;         // every MMA of the tile has completed
+    uint64_t empty[kStages];   // the MMA commit + one arrival per statistics warp
+    uint64_t acc_full[2];      // the tile's MMAs have completed (MMA commit)
+    uint64_t acc_empty[2];     // the epilogue has read the accumulator (4 epilogue warps)
+    uint64_t st_full[2];       // the tile's row statistics are written (4 statistics warps)
+    uint64_t st_empty[2];      // the epilogue has read them (4 epilogue warps)
+    uint64_t drain;            // teardown: every MMA issued has completed
     uint32_t tmem_base;
     int fail;
 };
@@ -84,157 +93,227 @@ __global__ void __launch_bounds__(256) oproj_prepare_kernel(const __nv_bfloat16*
     }
 }
 
-// ---- the fused GEMM ---------------------------------------------------------------------------
+
+// tcgen05.ld results are defined only after tcgen05.wait::ld; tie the registers to a point after it
+__device__ __forceinline__ void after_wait(float (&v)[16]) {
+    asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
+}
+
+// ---- the fused GEMM (persistent) ---------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
 post_norm_oproj_kernel(const OprojArgs a, const __grid_constant__ OprojMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     OpSmem& s = *reinterpret_cast<OpSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n0 = blockIdx.x * kBN;
-    const long long m0 = static_cast<long long>(blockIdx.y) * kBM;
     const int KT = a.C / kBK;
+    const int n_tiles = a.N / kBN;
+    const long long tiles = ((a.T + kBM - 1) / kBM) * n_tiles;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1 + 4);
         }
-        mbar_init(&s.acc_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.acc_full[i], 1);
+            mbar_init(&s.acc_empty[i], 4);
+            mbar_init(&s.st_full[i], 4);
+            mbar_init(&s.st_empty[i], 4);
+        }
+        mbar_init(&s.drain, 1);
         fence_mbarrier_init();
         tma_prefetch_desc(&maps.x);
         tma_prefetch_desc(&maps.w);
         s.fail = 0;
     }
     if (warp == 1) tc5::alloc(&s.tmem_base, kTmemCols);
-    for (int i = tid; i < kBN; i += kThreads) {
-        s.u[i] = a.u[n0 + i];
-        s.v[i] = a.v[n0 + i];
-    }
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
     const uint32_t tm = s.tmem_base;
     volatile int* const vfail = &s.fail;
+    const long long wl = a.wait_limit;
 
     if (warp == 0) {
-        // ---- producer: X and Wp tiles of k-chunk kc into stage kc % kStages ----------------------
+        // ---- producer: the X and Wp tiles of every k-chunk of every tile, through the ring -------
         if (lane == 0) {
-            int kc = 0;
-            for (; kc < KT; ++kc) {
-                const int st = kc % kStages;
-                if (kc >= kStages &&
-                    !mbar_wait_bounded_sleep(&s.empty[st], static_cast<uint32_t>((kc / kStages - 1) & 1), a.wait_limit,
-                                             64, a.status)) {
-                    *vfail = 1;
-                    break;
+            long long g = 0;  // chunks issued
+            for (long long tile = blockIdx.x; tile < tiles && !*vfail; tile += gridDim.x) {
+                const int m0 = static_cast<int>((tile / n_tiles) * kBM), n0 = static_cast<int>((tile % n_tiles) * kBN);
+                for (int kc = 0; kc < KT; ++kc, ++g) {
+                    const int st = static_cast<int>(g % kStages);
+                    if (g >= kStages &&
+                        !mbar_wait_bounded_sleep(&s.empty[st], static_cast<uint32_t>((g / kStages - 1) & 1), wl, 64,
+                                                 a.status)) {
+                        *vfail = 1;
+                        break;
+                    }
+                    if (*vfail) break;
+                    mbar_arrive_expect_tx(&s.full[st], kTileA + kTileB);
+                    tma_load_2d(&s.a[st][0], &maps.x, kc * kBK, m0, &s.full[st]);
+                    tma_load_2d(&s.b[st][0], &maps.w, kc * kBK, n0, &s.full[st]);
                 }
-                if (*vfail) break;
-                mbar_arrive_expect_tx(&s.full[st], kTileA + kTileB);
-                tma_load_2d(&s.a[st][0], &maps.x, kc * kBK, static_cast<int>(m0), &s.full[st]);
-                tma_load_2d(&s.b[st][0], &maps.w, kc * kBK, n0, &s.full[st]);
             }
             if (*vfail)  // wait (bounded) until the loads issued and perhaps not consumed have landed
-                for (int k = kc > kStages ? kc - kStages : 0; k < kc; ++k)
+                for (long long k = g > kStages ? g - kStages : 0; k < g; ++k)
                     mbar_wait_bounded(&s.full[k % kStages], static_cast<uint32_t>((k / kStages) & 1), kDrainPolls,
                                       nullptr);
         }
     } else if (warp == 1) {
-        // ---- MMA issue: D[128 x 256] += X[128 x 64] Wp[256 x 64]^T per stage, 4 steps of K = 16 ----
+        // ---- MMA issue into accumulator j % 2 of the j-th tile ---------------------------------------
         if (lane == 0) {
             const uint32_t idesc = tc5::idesc_bf16(kBM, kBN, 0, 0);
-            for (int kc = 0; kc < KT; ++kc) {
-                const int st = kc % kStages;
-                if (!mbar_wait_bounded(&s.full[st], static_cast<uint32_t>((kc / kStages) & 1), a.wait_limit,
-                                       a.status)) {
+            long long g = 0;
+            int j = 0;
+            for (long long tile = blockIdx.x; tile < tiles && !*vfail; tile += gridDim.x, ++j) {
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait_bounded(&s.acc_empty[buf], static_cast<uint32_t>(((j >> 1) - 1) & 1), wl,
+                                                 a.status)) {
                     *vfail = 1;
                     break;
                 }
                 tc5::fence_after();
-                const uint64_t ad = tc5::sdesc(smem_u32(&s.a[st][0]), 16, 1024);
-                const uint64_t bd = tc5::sdesc(smem_u32(&s.b[st][0]), 16, 1024);
+                const uint32_t acc = tm + static_cast<uint32_t>(buf) * kBN;
+                for (int kc = 0; kc < KT; ++kc, ++g) {
+                    const int st = static_cast<int>(g % kStages);
+                    if (!mbar_wait_bounded(&s.full[st], static_cast<uint32_t>((g / kStages) & 1), wl, a.status)) {
+                        *vfail = 1;
+                        break;
+                    }
+                    tc5::fence_after();
+                    const uint64_t ad = tc5::sdesc(smem_u32(&s.a[st][0]), 16, 1024);
+                    const uint64_t bd = tc5::sdesc(smem_u32(&s.b[st][0]), 16, 1024);
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                    tc5::mma_ss(tm, tc5::sdesc_add(ad, 32 * k), tc5::sdesc_add(bd, 32 * k), idesc,
-                                (kc | k) != 0 ? 1u : 0u);
-                tc5::commit(&s.empty[st]);
+                    for (int k = 0; k < kBK / 16; ++k)
+                        tc5::mma_ss(acc, tc5::sdesc_add(ad, 32 * k), tc5::sdesc_add(bd, 32 * k), idesc,
+                                    (kc | k) != 0 ? 1u : 0u);
+                    tc5::commit(&s.empty[st]);
+                }
+                if (*vfail) break;
+                tc5::commit(&s.acc_full[buf]);
             }
-            tc5::commit(&s.acc_full);  // once every MMA issued above has completed
+            tc5::commit(&s.drain);  // once every MMA issued above has completed
+            mbar_wait_bounded(&s.drain, 0, kDrainPolls, nullptr);
         }
         __syncwarp();
-    } else {
-        // ---- epilogue warps: row statistics while the tiles stream, then the output tile -------
-        const int q = warp & 3;            // tensor-memory lane quarter of this warp
-        const int row = 32 * q + lane;     // tile row: token m0 + row, accumulator lane row
-        float mean = 0.f, m2 = 0.f;
-        int kc = 0;
-        for (; kc < KT; ++kc) {
-            const int st = kc % kStages;
-            if (!mbar_wait_bounded(&s.full[st], static_cast<uint32_t>((kc / kStages) & 1), a.wait_limit, a.status)) {
+    } else if (warp < 6) {
+        // ---- statistics: row r = 32 (warp % 4) + lane of every X tile, Chan's merge per chunk ------
+        const int row = 32 * (warp & 3) + lane;
+        long long g = 0;
+        int j = 0;
+        for (long long tile = blockIdx.x; tile < tiles && !*vfail; tile += gridDim.x, ++j) {
+            const int buf = j & 1;
+            float mean = 0.f, m2 = 0.f;
+            bool ok = true;
+            for (int kc = 0; kc < KT; ++kc, ++g) {
+                const int st = static_cast<int>(g % kStages);
+                if (!mbar_wait_bounded(&s.full[st], static_cast<uint32_t>((g / kStages) & 1), wl, a.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* rp = &s.a[st][0] + row * 128;
+                float x[64];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 pv = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
+                    const uint32_t wv[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float2 f = unpack_bf16x2(wv[i]);
+                        x[8 * c + 2 * i] = f.x;
+                        x[8 * c + 2 * i + 1] = f.y;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.empty[st]);  // this warp is done with the stage
+                float sum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) sum += x[i];
+                const float cm = sum * (1.0f / kBK);
+                float cs = 0.f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) cs = fmaf(x[i] - cm, x[i] - cm, cs);
+                // Chan's merge of (64 kc values, mean, m2) with (64 values, cm, cs)
+                const float delta = cm - mean, inv = 1.0f / static_cast<float>(kc + 1);
+                mean = fmaf(delta, inv, mean);
+                m2 += cs + delta * delta * (static_cast<float>(kBK * kc) * inv);
+            }
+            if (ok && j >= 2)
+                ok = mbar_wait_bounded(&s.st_empty[buf], static_cast<uint32_t>(((j >> 1) - 1) & 1), wl, a.status);
+            if (!__all_sync(0xffffffffu, ok)) {
                 *vfail = 1;
                 break;
             }
-            // this row's 64 features of the chunk (8 swizzled 16-byte pieces), centred on their mean
-            const uint8_t* rp = &s.a[st][0] + row * 128;
-            float x[64];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 pv = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
-                const uint32_t wv[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = unpack_bf16x2(wv[j]);
-                    x[8 * c + 2 * j] = f.x;
-                    x[8 * c + 2 * j + 1] = f.y;
-                }
+            s.stats[buf][row] = make_float2(mean, rsqrtf(m2 * (1.0f / static_cast<float>(a.C)) + a.eps));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.st_full[buf]);
+        }
+    } else {
+        // ---- epilogue: rstd (acc - mean u) + v of every tile, from tensor memory to bf16 rows -----
+        const int q = warp & 3;              // tensor-memory lane quarter of this warp
+        const int row = 32 * q + lane;
+        int j = 0;
+        for (long long tile = blockIdx.x; tile < tiles && !*vfail; tile += gridDim.x, ++j) {
+            const int buf = j & 1;
+            const uint32_t par = static_cast<uint32_t>((j >> 1) & 1);
+            const long long m0 = (tile / n_tiles) * kBM;
+            const int n0 = static_cast<int>((tile % n_tiles) * kBN);
+            // this warp's copy of the tile's u and v (no barrier across the epilogue warps, so that
+            // a warp that gives up on a wait cannot leave the others waiting on it)
+            __syncwarp();
+            for (int i = lane; i < kBN; i += 32) {
+                s.uv[q][0][i] = a.u[n0 + i];
+                s.uv[q][1][i] = a.v[n0 + i];
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.empty[st]);  // this warp is done with the stage
-            float sum = 0.f;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) sum += x[i];
-            const float cm = sum * (1.0f / kBK);
-            float cs = 0.f;
-#pragma unroll
-            for (int i = 0; i < 64; ++i) cs = fmaf(x[i] - cm, x[i] - cm, cs);
-            // Chan's merge of (64 kc values, mean, m2) with (64 values, cm, cs)
-            const float delta = cm - mean, inv = 1.0f / static_cast<float>(kc + 1);
-            mean = fmaf(delta, inv, mean);
-            m2 += cs + delta * delta * (static_cast<float>(kBK * kc) * inv);
-        }
-        bool ok = kc == KT && mbar_wait_bounded(&s.acc_full, 0, a.wait_limit, a.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) *vfail = 1;
-        tc5::fence_after();
-        if (ok) {
-            const float rstd = rsqrtf(m2 * (1.0f / static_cast<float>(a.C)) + a.eps);
-            const float nmr = -mean * rstd;
+            bool ok = mbar_wait_bounded(&s.st_full[buf], par, wl, a.status) &&
+                      mbar_wait_bounded(&s.acc_full[buf], par, wl, a.status);
+            if (!__all_sync(0xffffffffu, ok)) {
+                *vfail = 1;
+                break;
+            }
+            tc5::fence_after();
+            const float2 st = s.stats[buf][row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.st_empty[buf]);
+            const float rstd = st.y, nmr = -st.x * st.y;
             const long long grow = m0 + row;
             __nv_bfloat16* const yrow = static_cast<__nv_bfloat16*>(a.Y) + grow * a.N + n0;
+            const float* const uu = s.uv[q][0];
+            const float* const vv = s.uv[q][1];
 #pragma unroll 1
-            for (int c16 = 0; c16 < kBN / 16; ++c16) {
-                float acc[16];
-                tc5::ld16(tc5::taddr(tm, 32 * q, 16 * c16), acc);
-                tc5::wait_ld();
-                uint32_t pk[8];
+            for (int c64 = 0; c64 < kBN / 64; ++c64) {
+                float acc[4][16];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int n = 16 * c16 + 2 * j;
-                    // rstd (acc - mu u) + v
-                    const float y0 = fmaf(rstd, acc[2 * j], fmaf(nmr, s.u[n], s.v[n]));
-                    const float y1 = fmaf(rstd, acc[2 * j + 1], fmaf(nmr, s.u[n + 1], s.v[n + 1]));
-                    pk[j] = pack_bf16x2(y0, y1);
-                }
+                for (int i = 0; i < 4; ++i)
+                    tc5::ld16(tc5::taddr(tm, 32 * q, static_cast<uint32_t>(buf) * kBN + 64 * c64 + 16 * i), acc[i]);
+                tc5::wait_ld();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) after_wait(acc[i]);
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const int n = 64 * c64 + 16 * i + 2 * jj;
+                        const float y0 = fmaf(rstd, acc[i][2 * jj], fmaf(nmr, uu[n], vv[n]));
+                        const float y1 = fmaf(rstd, acc[i][2 * jj + 1], fmaf(nmr, uu[n + 1], vv[n + 1]));
+                        pk[8 * i + jj] = pack_bf16x2(y0, y1);
+                    }
                 if (grow < a.T) {
-                    uint4* dst = reinterpret_cast<uint4*>(yrow + 16 * c16);
-                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    uint4* dst = reinterpret_cast<uint4*>(yrow + 64 * c64);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 }
             }
+            tc5::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.acc_empty[buf]);
         }
     }
 
-    // ---- teardown: every MMA has completed before tensor memory is freed ------------------------
-    if (warp == 1 && lane == 0 && *vfail) mbar_wait_bounded(&s.acc_full, 0, kDrainPolls, nullptr);
+    // ---- teardown: the MMA thread has seen every MMA complete; free tensor memory -----------------
     tc5::fence_before();
     __syncthreads();
     tc5::fence_after();
@@ -255,7 +334,10 @@ cudaError_t launch_post_norm_oproj(const OprojArgs& a, const OprojMaps& maps, cu
     cudaError_t e = cudaFuncSetAttribute(post_norm_oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const dim3 grid(static_cast<unsigned>(a.N / kBN), static_cast<unsigned>((a.T + kBM - 1) / kBM));
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long tiles = ((a.T + kBM - 1) / kBM) * (a.N / kBN);
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
     post_norm_oproj_kernel<<<grid, kThreads, smem, st>>>(a, maps);
     return cudaGetLastError();
 }
