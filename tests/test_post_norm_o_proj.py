@@ -96,3 +96,24 @@ def test_scan_then_output_side(libttt):
     xs = out.reshape(-1, C).float().cpu().numpy()
     ref = oracle.default().post_norm_o_proj(xs, d["ln_w"], d["ln_b"], 1e-6, d["Wo"])
     assert rel_l2(Y.reshape(-1, C).float().cpu().numpy(), ref) <= TOL
+
+
+def test_post_norm_o_proj_bounded_wait_timeout(libttt):
+    """Every bounded wait gives up at once: every role of the persistent kernel stops, the tensor
+    core and the loads in flight drain, tensor memory is freed, the status word says so, and the
+    next call is correct."""
+    T, C, N = 700, 512, 512
+    d = synth.oproj_inputs(0x0FB, T, C, N)
+    libttt.ttt_device_status(clear=True)
+    libttt.ttt_set_wait_limit(-1)
+    try:
+        _run(libttt, d, T, C, N)
+        with pytest.raises(libttt.TTTError) as e:
+            libttt.ttt_device_status(clear=True)
+        assert e.value.code == libttt.TTT_ERR_TIMEOUT
+    finally:
+        libttt.ttt_set_wait_limit(0)
+    assert libttt.ttt_device_status(clear=True) == 0
+    ref = oracle.default().post_norm_o_proj(d["X"], d["ln_w"], d["ln_b"], 1e-6, d["Wo"])
+    assert rel_l2(_run(libttt, d, T, C, N), ref) <= TOL
+    assert libttt.ttt_device_status() == 0
