@@ -421,9 +421,10 @@ def bench_linear_rope(args, world, peaks, theta=10000.0):
 
 def bench_post_norm_oproj(args, world, peaks):
     """The layer's output side at the 1B layer, Y = o_proj(post_norm(X)) for the scan's
-    token-major output ([B*L, 2048] bf16): one tcgen05 GEMM with the LayerNorm folded into its
-    epilogue (ttt_post_norm_o_proj; the weight packed once beforehand, outside the timing), and
-    beside it the unfused torch way (layer_norm, then a cuBLAS matmul)."""
+    token-major output ([B*L, 2048] bf16): a token-statistics pass and one tcgen05 GEMM with the
+    LayerNorm folded into its epilogue (ttt_post_norm_o_proj, two launches; the weight packed once
+    beforehand, outside the timing), and beside it the unfused torch way (layer_norm, then a cuBLAS
+    matmul)."""
     import torch
 
     import test_rnn_layers_b200 as ttt
@@ -436,9 +437,10 @@ def bench_post_norm_oproj(args, world, peaks):
     ln_w, ln_b = torch.from_numpy(d["ln_w"]).cuda(), torch.from_numpy(d["ln_b"]).cuda()
     Wp, u, v = ttt.ttt_o_proj_prepare(Wo, ln_w, ln_b)
     Y = torch.empty_like(X)
+    stats = torch.empty((T, 2), device="cuda")
 
     def fused():
-        ttt.ttt_post_norm_o_proj(X, Wp, u, v, eps=1e-6, Y=Y)
+        ttt.ttt_post_norm_o_proj(X, Wp, u, v, eps=1e-6, Y=Y, row_stats=stats)
 
     K = max(3, min(args.steps, 20))
     ms = time_steps(fused, K, 3, world)
@@ -452,7 +454,7 @@ def bench_post_norm_oproj(args, world, peaks):
     peak = peaks[1]
     tf = flops / (ms / 1e3) / 1e12
     return {"workload": f"ttt_post_norm_o_proj_1b_layer_T{T}_C{C}", "value": round(world * T / (ms / 1e3), 1),
-            "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": K, "gpu_launches": K,
+            "unit": "tokens/s", "ms_per_step": round(ms, 4), "steps": K, "gpu_launches": 2 * K,
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak,
                          "peak_source": ("measured" if peaks[3] == "measured" else "fallback") + " bf16_tflops",
                          "unit": "TFLOP/s", "frac": round(tf / peak, 4), "algorithmic_flops": int(flops)},

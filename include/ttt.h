@@ -357,8 +357,8 @@ int ttt_linear_decode_step_hist(const void* xq, const void* xk, const void* xv, 
  * with Wp[n][k] = ln_w[k] Wo[n][k], u[n] = sum_k Wp[n][k], v[n] = sum_k ln_b[k] Wo[n][k].
  * ttt_o_proj_prepare packs those once per weight; ttt_post_norm_o_proj then runs one
  * tensor-core GEMM (tcgen05, fp32 accumulation in tensor memory) whose epilogue applies the
- * token statistics, taken from the same X tiles in one pass over C (Chan's merge per 64
- * features).  Y is rounded to bf16.  The correction subtracts mean * u[n] from the product in
+ * token statistics, which a one-warp-per-token pass over X (Chan's merge of the lanes' moments)
+ * writes just before.  Y is rounded to bf16.  The correction subtracts mean * u[n] from the product in
  * fp32, so its accuracy falls as a token's |mean| / std grows (the scan's output has mean near
  * zero next to its spread).
  *
@@ -388,12 +388,15 @@ int ttt_o_proj_prepare(const void* Wo, const float* ln_w, const float* ln_b, int
  *   eps          post_norm's epsilon, finite and > 0.
  *   Y            [T][N] bf16 (device, caller-allocated), 16-byte aligned; must not overlap the
  *                inputs.
+ *   row_stats    [T][2] float32 (device, caller-allocated), 8-byte aligned: receives each token's
+ *                (mean, 1/sqrt(var + eps)) of post_norm (written by the first of the call's two
+ *                launches, read by the second); must not overlap the inputs or Y.
  * Asynchronous on `stream`; allocates nothing.  T == 0 does nothing.  Errors as
  * ttt_o_proj_prepare, plus TTT_ERR_ARG for a bad eps or T < 0, TTT_ERR_UNSUPPORTED for T above
  * 65535 * 128.  The kernel's waits are bounded (see ttt_device_status).
  */
 int ttt_post_norm_o_proj(const void* X, long long T, int C, const void* Wp, const float* u, const float* v, int N,
-                         float eps, void* Y, void* stream);
+                         float eps, void* Y, float* row_stats, void* stream);
 
 #ifdef __cplusplus
 }

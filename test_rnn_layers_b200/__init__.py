@@ -81,7 +81,7 @@ def lib():
         L.ttt_linear_decode_step_hist.argtypes = [vp, vp, vp, fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, ll, f,
                                                   i, vp, vp]
         L.ttt_o_proj_prepare.argtypes = [vp, fp, fp, i, i, vp, fp, fp, vp]
-        L.ttt_post_norm_o_proj.argtypes = [vp, ll, i, vp, fp, fp, i, f, vp, vp]
+        L.ttt_post_norm_o_proj.argtypes = [vp, ll, i, vp, fp, fp, i, f, vp, fp, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
                      "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
                      "ttt_linear_forward_rope",
@@ -451,9 +451,10 @@ def ttt_o_proj_prepare(Wo, ln_w, ln_b, Wp=None, u=None, v=None, stream=None):
     return Wp, u, v
 
 
-def ttt_post_norm_o_proj(X, Wp, u, v, eps: float = 1e-6, Y=None, stream=None):
+def ttt_post_norm_o_proj(X, Wp, u, v, eps: float = 1e-6, Y=None, row_stats=None, stream=None):
     """Y = o_proj(post_norm(X)) for X [..., C] bf16 (the token-major scan output), with (Wp, u, v)
-    from ttt_o_proj_prepare; returns Y [..., N] bf16."""
+    from ttt_o_proj_prepare; returns Y [..., N] bf16 (row_stats, [T, 2] fp32, receives each token's
+    post_norm mean and 1/sqrt(var + eps))."""
     _need(X, "X", torch.bfloat16)
     _need(Wp, "Wp", torch.bfloat16)
     N, C = Wp.shape
@@ -464,5 +465,7 @@ def ttt_post_norm_o_proj(X, Wp, u, v, eps: float = 1e-6, Y=None, stream=None):
     T = X.numel() // C
     Y = torch.empty((*X.shape[:-1], N), dtype=torch.bfloat16, device=X.device) if Y is None else \
         _need(Y, "Y", torch.bfloat16, (*X.shape[:-1], N))
-    _check(lib().ttt_post_norm_o_proj(_ptr(X), T, C, _ptr(Wp), _ptr(u), _ptr(v), N, eps, _ptr(Y), _stream(stream)))
+    row_stats = torch.empty((T, 2), device=X.device) if row_stats is None else _need(row_stats, "row_stats", torch.float32, (T, 2))
+    _check(lib().ttt_post_norm_o_proj(_ptr(X), T, C, _ptr(Wp), _ptr(u), _ptr(v), N, eps, _ptr(Y), _ptr(row_stats),
+                                      _stream(stream)))
     return Y

@@ -8,8 +8,10 @@
 //        = rstd (sum_k x_k Wp[n][k] - mu u[n]) + v[n],
 //   Wp[n][k] = gamma_k Wo[n][k] (bf16),  u[n] = sum_k Wp[n][k],  v[n] = sum_k beta_k Wo[n][k],
 // so the tensor cores multiply the raw X by a once-packed weight (oproj_prepare_kernel; u sums
-// the rounded Wp, so the correction matches what the MMAs multiply), and the statistics are
-// taken from the same X tiles while they stream through shared memory for the MMAs.
+// the rounded Wp, so the correction matches what the MMAs multiply).  The token statistics come
+// from a one-warp-per-token pass over X just before (oproj_stats_kernel: Chan's merge of the
+// lanes' two-pass moments); taking them from the GEMM's own X tiles in shared memory instead cost
+// shared-memory bandwidth that the tensor core's operand reads need (0.547 against 0.44 ms).
 //
 // Design: a persistent kernel, one CTA per SM, walking 128 x 256 output tiles (output tile
 // fastest, so the CTAs at work at any moment share their X tiles through L2), four roles:
@@ -20,12 +22,9 @@
 //    issues, from one thread, four tcgen05.mma (kind::f16, bf16 operands, M = 128, N = 256,
 //    K = 16) per stage into the tile's accumulator, committing each stage to its empty barrier
 //    and each finished tile to its accumulator's full barrier;
-//  * warps 2-5 (statistics) take token row r = 32 (warp % 4) + lane of every X tile as it lands
-//    and fold its 64 values into the row's (mean, centred sum of squares) with Chan's formula,
-//    handing (mean, rstd) per row to the epilogue through a double buffer;
-//  * warps 6-9 (epilogue) read their accumulator lane back (tcgen05.ld 32x32b, 64 columns per
-//    wait), apply rstd (acc - mean u) + v and store bf16, then free the accumulator -- while the
-//    MMAs of the next tile already run into the other one.
+//  * warps 2-5 (epilogue) read their accumulator lane back (tcgen05.ld 32x32b, 64 columns per
+//    wait), apply rstd (acc - mean u) + v with the row's statistics and store bf16, then free the
+//    accumulator -- while the MMAs of the next tile already run into the other one.
 // Every mbarrier wait is bounded; on expiry the status word is raised, every role stops, the
 // tensor core and the loads in flight are drained (bounded) and tensor memory is freed.
 #include "tc5.cuh"
@@ -37,7 +36,7 @@ namespace {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kStages = 4;
-constexpr int kThreads = 320;                       // producer, MMA, 4 statistics, 4 epilogue warps
+constexpr int kThreads = 192;                       // producer, MMA, 4 epilogue warps
 constexpr uint32_t kTileA = kBM * kBK * 2;          // 16 KB
 constexpr uint32_t kTileB = kBN * kBK * 2;          // 32 KB
 constexpr uint32_t kTmemCols = 512;                 // two 256-column accumulators
@@ -46,14 +45,11 @@ constexpr long long kDrainPolls = 1ll << 24;
 struct __align__(1024) OpSmem {
     uint8_t a[kStages][kTileA];
     uint8_t b[kStages][kTileB];
-    float2 stats[2][kBM];      // (mean, rstd) of the tile's rows, by accumulator buffer
     float uv[4][2][kBN];       // the tile's u and v, one copy per epilogue warp
     uint64_t full[kStages];
-    uint64_t empty[kStages];   // the MMA commit + one arrival per statistics warp
+    uint64_t empty[kStages];   // the MMA commit
     uint64_t acc_full[2];      // the tile's MMAs have completed (MMA commit)
     uint64_t acc_empty[2];     // the epilogue has read the accumulator (4 epilogue warps)
-    uint64_t st_full[2];       // the tile's row statistics are written (4 statistics warps)
-    uint64_t st_empty[2];      // the epilogue has read them (4 epilogue warps)
     uint64_t drain;            // teardown: every MMA issued has completed
     uint32_t tmem_base;
     int fail;
@@ -94,6 +90,82 @@ __global__ void __launch_bounds__(256) oproj_prepare_kernel(const __nv_bfloat16*
 }
 
 
+// ---- token statistics: one warp per token, (mean, rstd) over its C features -----------------
+// Each lane takes the 16-byte pieces lane, lane + 32, ... of the row, forms their mean and centred
+// sum of squares, and the warp merges the lanes' moments pairwise by Chan's formula.
+__global__ void __launch_bounds__(256) oproj_stats_kernel(const __nv_bfloat16* __restrict__ X, long long T, int C,
+                                                          float eps, float2* __restrict__ stats) {
+    const int lane = threadIdx.x & 31;
+    const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    const int pieces = C / 8;
+    for (long long t = w0; t < T; t += nw) {
+        const uint4* row = reinterpret_cast<const uint4*>(X + t * C);
+        // the first 8 pieces of this lane (all of them for C <= 2048), held in registers
+        uint4 pv[8];
+        int np = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool in = lane + 32 * i < pieces;
+            pv[i] = in ? __ldg(row + lane + 32 * i) : make_uint4(0, 0, 0, 0);
+            np += in ? 1 : 0;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t wv[4] = {pv[i].x, pv[i].y, pv[i].z, pv[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = unpack_bf16x2(wv[j]);
+                sum += f.x + f.y;
+            }
+        }
+        int n = 8 * np;
+        float mean = n ? sum / n : 0.f, m2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i >= np) break;
+            const uint32_t wv[4] = {pv[i].x, pv[i].y, pv[i].z, pv[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = unpack_bf16x2(wv[j]);
+                m2 = fmaf(f.x - mean, f.x - mean, m2);
+                m2 = fmaf(f.y - mean, f.y - mean, m2);
+            }
+        }
+        for (int p = lane + 32 * 8; p < pieces; p += 32) {  // rows wider than 2048 features
+            const uint4 q = __ldg(row + p);
+            const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = unpack_bf16x2(wv[j]);
+                const float d0 = f.x - mean;
+                mean += d0 / static_cast<float>(n + 1);
+                m2 = fmaf(d0, f.x - mean, m2);
+                ++n;
+                const float d1 = f.y - mean;
+                mean += d1 / static_cast<float>(n + 1);
+                m2 = fmaf(d1, f.y - mean, m2);
+                ++n;
+            }
+        }
+        // Chan's merge across the lanes: (n, mean, m2) pairs, xor butterfly
+        float fn = static_cast<float>(n);
+        for (int o = 16; o > 0; o >>= 1) {
+            const float on = __shfl_xor_sync(0xffffffffu, fn, o);
+            const float om = __shfl_xor_sync(0xffffffffu, mean, o);
+            const float oq = __shfl_xor_sync(0xffffffffu, m2, o);
+            const float tn = fn + on;
+            if (tn > 0.f) {
+                const float delta = om - mean;
+                mean = fmaf(delta, on / tn, mean);
+                m2 += oq + delta * delta * (fn * on / tn);
+            }
+            fn = tn;
+        }
+        if (lane == 0) stats[t] = make_float2(mean, rsqrtf(m2 / static_cast<float>(C) + eps));
+    }
+}
+
 // tcgen05.ld results are defined only after tcgen05.wait::ld; tie the registers to a point after it
 __device__ __forceinline__ void after_wait(float (&v)[16]) {
     asm volatile("" : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
@@ -113,13 +185,11 @@ post_norm_oproj_kernel(const OprojArgs a, const __grid_constant__ OprojMaps maps
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + 4);
+            mbar_init(&s.empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.acc_full[i], 1);
             mbar_init(&s.acc_empty[i], 4);
-            mbar_init(&s.st_full[i], 4);
-            mbar_init(&s.st_empty[i], 4);
         }
         mbar_init(&s.drain, 1);
         fence_mbarrier_init();
@@ -197,58 +267,6 @@ post_norm_oproj_kernel(const OprojArgs a, const __grid_constant__ OprojMaps maps
             mbar_wait_bounded(&s.drain, 0, kDrainPolls, nullptr);
         }
         __syncwarp();
-    } else if (warp < 6) {
-        // ---- statistics: row r = 32 (warp % 4) + lane of every X tile, Chan's merge per chunk ------
-        const int row = 32 * (warp & 3) + lane;
-        long long g = 0;
-        int j = 0;
-        for (long long tile = blockIdx.x; tile < tiles && !*vfail; tile += gridDim.x, ++j) {
-            const int buf = j & 1;
-            float mean = 0.f, m2 = 0.f;
-            bool ok = true;
-            for (int kc = 0; kc < KT; ++kc, ++g) {
-                const int st = static_cast<int>(g % kStages);
-                if (!mbar_wait_bounded(&s.full[st], static_cast<uint32_t>((g / kStages) & 1), wl, a.status)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t* rp = &s.a[st][0] + row * 128;
-                float x[64];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 pv = *reinterpret_cast<const uint4*>(rp + ((c ^ (row & 7)) << 4));
-                    const uint32_t wv[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = unpack_bf16x2(wv[i]);
-                        x[8 * c + 2 * i] = f.x;
-                        x[8 * c + 2 * i + 1] = f.y;
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.empty[st]);  // this warp is done with the stage
-                float sum = 0.f;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) sum += x[i];
-                const float cm = sum * (1.0f / kBK);
-                float cs = 0.f;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) cs = fmaf(x[i] - cm, x[i] - cm, cs);
-                // Chan's merge of (64 kc values, mean, m2) with (64 values, cm, cs)
-                const float delta = cm - mean, inv = 1.0f / static_cast<float>(kc + 1);
-                mean = fmaf(delta, inv, mean);
-                m2 += cs + delta * delta * (static_cast<float>(kBK * kc) * inv);
-            }
-            if (ok && j >= 2)
-                ok = mbar_wait_bounded(&s.st_empty[buf], static_cast<uint32_t>(((j >> 1) - 1) & 1), wl, a.status);
-            if (!__all_sync(0xffffffffu, ok)) {
-                *vfail = 1;
-                break;
-            }
-            s.stats[buf][row] = make_float2(mean, rsqrtf(m2 * (1.0f / static_cast<float>(a.C)) + a.eps));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.st_full[buf]);
-        }
     } else {
         // ---- epilogue: rstd (acc - mean u) + v of every tile, from tensor memory to bf16 rows -----
         const int q = warp & 3;              // tensor-memory lane quarter of this warp
@@ -267,16 +285,13 @@ post_norm_oproj_kernel(const OprojArgs a, const __grid_constant__ OprojMaps maps
                 s.uv[q][1][i] = a.v[n0 + i];
             }
             __syncwarp();
-            bool ok = mbar_wait_bounded(&s.st_full[buf], par, wl, a.status) &&
-                      mbar_wait_bounded(&s.acc_full[buf], par, wl, a.status);
+            const float2 st = row < a.T - m0 ? a.stats[m0 + row] : make_float2(0.f, 0.f);
+            const bool ok = mbar_wait_bounded(&s.acc_full[buf], par, wl, a.status);
             if (!__all_sync(0xffffffffu, ok)) {
                 *vfail = 1;
                 break;
             }
             tc5::fence_after();
-            const float2 st = s.stats[buf][row];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.st_empty[buf]);
             const float rstd = st.y, nmr = -st.x * st.y;
             const long long grow = m0 + row;
             __nv_bfloat16* const yrow = static_cast<__nv_bfloat16*>(a.Y) + grow * a.N + n0;
@@ -330,6 +345,14 @@ cudaError_t launch_oproj_prepare(const void* Wo, const float* ln_w, const float*
 }
 
 cudaError_t launch_post_norm_oproj(const OprojArgs& a, const OprojMaps& maps, cudaStream_t st) {
+    int dev0 = 0, sms0 = 148;
+    if (cudaGetDevice(&dev0) == cudaSuccess) cudaDeviceGetAttribute(&sms0, cudaDevAttrMultiProcessorCount, dev0);
+    const long long warps_needed = a.T;
+    const long long blocks = (warps_needed + 7) / 8;
+    const unsigned sgrid = static_cast<unsigned>(blocks < 16ll * sms0 ? blocks : 16ll * sms0);
+    oproj_stats_kernel<<<sgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.X), a.T, a.C, a.eps, a.stats);
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
     const size_t smem = sizeof(OpSmem) + 1024;  // + alignment slack
     cudaError_t e = cudaFuncSetAttribute(post_norm_oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

@@ -720,29 +720,31 @@ static int encode_rows_map(CUtensorMap* map, const void* base, long long rows, i
 }
 
 int ttt_post_norm_o_proj(const void* X, long long T, int C, const void* Wp, const float* u, const float* v, int N,
-                         float eps, void* Y, void* stream) {
+                         float eps, void* Y, float* row_stats, void* stream) {
     int rc = check_oproj_sizes(C, N);
     if (rc) return rc;
     if (T < 0) return fail(TTT_ERR_ARG, "T must be >= 0 (got %lld)", T);
     if (T > 65535ll * 128) return fail(TTT_ERR_UNSUPPORTED, "T above 65535 * 128 tokens (got %lld)", T);
     if (!(eps > 0.f) || !std::isfinite(eps)) return fail(TTT_ERR_ARG, "eps must be finite and > 0");
     if (!Wp || !u || !v) return fail(TTT_ERR_ARG, "Wp, u and v must be non-null");
-    if (T > 0 && (!X || !Y)) return fail(TTT_ERR_ARG, "X and Y must be non-null when T > 0");
+    if (T > 0 && (!X || !Y || !row_stats)) return fail(TTT_ERR_ARG, "X, Y and row_stats must be non-null when T > 0");
     const void* a16[] = {X, Wp, Y};
     const char* n16[] = {"X", "Wp", "Y"};
     for (int i = 0; i < 3; ++i)
         if (a16[i] && !aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "%s must be 16-byte aligned", n16[i]);
     if (!aligned(u, 4) || !aligned(v, 4)) return fail(TTT_ERR_ALIGN, "u and v must be 4-byte aligned");
+    if (row_stats && !aligned(row_stats, 8)) return fail(TTT_ERR_ALIGN, "row_stats must be 8-byte aligned");
     Span in[] = {{"X", X, static_cast<size_t>(T) * C * 2}, {"Wp", Wp, static_cast<size_t>(C) * N * 2},
                  {"u", u, static_cast<size_t>(N) * 4}, {"v", v, static_cast<size_t>(N) * 4}};
-    Span outs[] = {{"Y", Y, static_cast<size_t>(T) * N * 2}};
-    if ((rc = check_aliasing(in, 4, outs, 1))) return rc;
+    Span outs[] = {{"Y", Y, static_cast<size_t>(T) * N * 2}, {"row_stats", row_stats, static_cast<size_t>(T) * 8}};
+    if ((rc = check_aliasing(in, 4, outs, 2))) return rc;
     if (T == 0) return ok();
     ttt::OprojMaps maps;
     if ((rc = encode_rows_map(&maps.x, X, T, C, 128, "X"))) return rc;
     if ((rc = encode_rows_map(&maps.w, Wp, N, C, 256, "Wp"))) return rc;
     ttt::OprojArgs a{};
-    a.T = T; a.C = C; a.N = N; a.eps = eps; a.u = u; a.v = v; a.Y = Y;
+    a.T = T; a.C = C; a.N = N; a.eps = eps; a.u = u; a.v = v; a.X = X; a.stats = reinterpret_cast<float2*>(row_stats);
+    a.Y = Y;
     a.status = status_word();
     a.wait_limit = wait_limit();
     cudaError_t e = ttt::launch_post_norm_oproj(a, maps, static_cast<cudaStream_t>(stream));

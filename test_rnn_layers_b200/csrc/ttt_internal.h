@@ -131,6 +131,8 @@ struct OprojArgs {
     float eps;
     const float* u;           // [N] sum_k Wp[n][k]
     const float* v;           // [N] sum_k ln_b[k] Wo[n][k]
+    const void* X;            // [T][C] bf16 (the statistics pass reads it directly)
+    float2* stats;            // [T] (mean, rstd), written by the statistics pass
     void* Y;                  // [T][N] bf16
     unsigned int* status;
     long long wait_limit;

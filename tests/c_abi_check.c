@@ -60,9 +60,9 @@ int main(void) {
 
     check(ttt_o_proj_prepare(XQ, W0, b0, 2048, 100, out, Wl, bl, NULL) == TTT_ERR_UNSUPPORTED,
           "o_proj prepare rejects N = 100");
-    check(ttt_post_norm_o_proj(XQ, 65600, 2048, XK, W0, b0, 2048, 0.0f, out, NULL) == TTT_ERR_ARG,
+    check(ttt_post_norm_o_proj(XQ, 65600, 2048, XK, W0, b0, 2048, 0.0f, out, Wl, NULL) == TTT_ERR_ARG,
           "post_norm o_proj rejects eps = 0");
-    check(ttt_post_norm_o_proj(NULL, 0, 2048, XK, W0, b0, 2048, 1e-6f, NULL, NULL) == TTT_OK,
+    check(ttt_post_norm_o_proj(NULL, 0, 2048, XK, W0, b0, 2048, 1e-6f, NULL, NULL, NULL) == TTT_OK,
           "post_norm o_proj with T = 0 is a no-op");
 
     const long long ws = ttt_linear_host_workspace_bytes(8, 32, 8200, 64, 16, TTT_BF16, 1, 0);

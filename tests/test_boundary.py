@@ -268,9 +268,10 @@ def _prep(lib, **kw):
 
 
 def _onorm(lib, **kw):
-    a = dict(X=A, T=65600, C=2048, Wp=8 * A, u=9 * A, v=10 * A, N=2048, eps=1e-6, Y=1 << 30)
+    a = dict(X=A, T=65600, C=2048, Wp=8 * A, u=9 * A, v=10 * A, N=2048, eps=1e-6, Y=1 << 30, st=1 << 31)
     a.update(kw)
-    return lib.ttt_post_norm_o_proj(a["X"], a["T"], a["C"], a["Wp"], a["u"], a["v"], a["N"], a["eps"], a["Y"], None)
+    return lib.ttt_post_norm_o_proj(a["X"], a["T"], a["C"], a["Wp"], a["u"], a["v"], a["N"], a["eps"], a["Y"], a["st"],
+                                    None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -288,7 +289,8 @@ def test_o_proj_prepare_rejects(libttt, kw, code):
     (dict(T=-1), -1), (dict(T=65535 * 128 + 1), -6), (dict(C=96), -6), (dict(N=512 + 64), -6),
     (dict(eps=0.0), -1), (dict(eps=float("inf")), -1), (dict(X=None), -1), (dict(Wp=None), -1),
     (dict(X=A + 2), -2), (dict(Y=(1 << 30) + 8), -2), (dict(u=9 * A + 1), -2),
-    (dict(Y=A), -3), (dict(Y=8 * A - 64), -3),
+    (dict(Y=A), -3), (dict(Y=8 * A - 64), -3), (dict(st=None), -1), (dict(st=(1 << 31) + 4), -2),
+    (dict(st=A), -3), (dict(st=(1 << 30) + 64), -3),
 ])
 def test_post_norm_o_proj_rejects(libttt, kw, code):
     lib = libttt.lib()
@@ -298,4 +300,4 @@ def test_post_norm_o_proj_rejects(libttt, kw, code):
 
 def test_post_norm_o_proj_T0_is_a_no_op(libttt):
     lib = libttt.lib()
-    assert _onorm(lib, T=0, X=None, Y=None) == 0
+    assert _onorm(lib, T=0, X=None, Y=None, st=None) == 0
