@@ -35,10 +35,11 @@ def _run(ttt, d, T, C, N, eps=1e-6):
 
 
 @pytest.mark.parametrize("T,C,N", [(300, 768, 768), (1, 64, 256), (128, 192, 512), (129, 2048, 2048),
-                                   (1000, 2048, 256), (257, 64, 768)])
+                                   (1000, 2048, 256), (257, 64, 768), (130, 2304, 256)])
 def test_post_norm_o_proj_against_oracle(libttt, T, C, N):
     """A ragged last token tile (T not a multiple of 128), a single token, N != C, the smallest C
-    (one k-chunk) and the model widths of the 125M (768) and 1B (2048) layers."""
+    (one k-chunk), the model widths of the 125M (768) and 1B (2048) layers, and a row wider than
+    the statistics pass keeps in registers (2304 features)."""
     d = synth.oproj_inputs(0x0F0 + T + C + N, T, C, N)
     got = _run(libttt, d, T, C, N)
     ref = oracle.default().post_norm_o_proj(d["X"], d["ln_w"], d["ln_b"], 1e-6, d["Wo"])
