@@ -398,6 +398,60 @@ int ttt_o_proj_prepare(const void* Wo, const float* ln_w, const float* ln_b, int
 int ttt_post_norm_o_proj(const void* X, long long T, int C, const void* Wp, const float* u, const float* v, int N,
                          float eps, void* Y, float* row_stats, void* stream);
 
+/* ---- training: the backward of the TTT-Linear scan ----------------------------------------
+ * [walkthrough] TTTLinear.ttt hands scan_checkpoint_group_size to its scan while training, so
+ * the outer parameters learn through the scan; [readme] says training with the pure-PyTorch
+ * code is slow.  The backward below runs through the same scan on the device. */
+
+/*
+ * ttt_linear_backward_workspace_bytes -- bytes of device workspace ttt_linear_backward needs:
+ * per chain, ceil(n_full / ckpt_group) kept states and ckpt_group rebuilt states of
+ * (d*d + d) float32 each, plus (d*d + 3d) float32 of per-chain gradient shares; n_full = L / K.
+ * Host-only.  Returns the byte count (> 0) or a negative TTT_ERR_* code.
+ */
+long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, int mini_batch, int ckpt_group);
+
+/*
+ * ttt_linear_backward -- gradients of the outer inputs of ttt_linear_forward.
+ *
+ * For the forward described at ttt_linear_forward (same inputs, same tail rule), and caller
+ * gradients d_out of out, dW_last of W_last and db_last of b_last, it returns the gradients of
+ *   <d_out, out> + <dW_last, W_last> + <db_last, b_last>
+ * with respect to XQ, XK, XV, lr, W0, b0, ln_w and ln_b -- the reverse-mode derivative of the
+ * scan, through every mini-batch's loss gradient (the derivative of ln_fused_l2_bwd itself),
+ * the dual form's attention-like terms and the state updates.  token_eta and eps are constants.
+ *
+ * Scan checkpoint groups: the forward state recursion runs once over the full mini-batches and
+ * keeps every ckpt_group-th state; the backward then takes the groups from the last, rebuilds a
+ * group's states from its kept state, and steps back through the group.  ckpt_group trades
+ * workspace (above) for nothing else: the results do not depend on it.
+ *
+ * Arguments:
+ *   XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d, mini_batch,
+ *   eps, dtype   as ttt_linear_forward (head-major [B,H,L,d] only; no flags).
+ *   ckpt_group   >= 1: mini-batches per checkpoint group.
+ *   d_out        [B,H,L,d] dtype, 16-byte aligned: the gradient of out (NULL allowed if L == 0).
+ *   dW_last, db_last  [B,H,d,d], [B,H,d] float32, 16-byte aligned, or NULL (zero).
+ * Outputs (device, caller-allocated, none overlapping an input, another output or the workspace):
+ *   dXQ, dXK, dXV  [B,H,L,d] dtype, 16-byte aligned (NULL allowed if L == 0).
+ *   d_lr         [B,H,L] float32.
+ *   dW0, db0     float32: [H,d,d] and [H,d] summed over the batch when w0_batch_stride == 0 (one
+ *                initial state per head), else [B,H,d,d] and [B,H,d] per chain.
+ *   d_ln_w, d_ln_b  [H,d] float32, summed over the batch.
+ *   workspace    device buffer of at least ttt_linear_backward_workspace_bytes, 256-byte aligned;
+ *                its contents on entry do not matter and are overwritten.
+ * Computes in float32 throughout (one CTA per chain); the batch sums run in a fixed order, so
+ * results are reproducible bit for bit.  Asynchronous on `stream`; allocates nothing; has no
+ * device-side waits.  Errors as ttt_linear_forward (flags aside), plus TTT_ERR_ARG for
+ * ckpt_group < 1 or a workspace smaller than needed.
+ */
+int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                        const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
+                        const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps, int dtype,
+                        int ckpt_group, const void* d_out, const float* dW_last, const float* db_last, void* dXQ,
+                        void* dXK, void* dXV, float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b,
+                        void* workspace, long long workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,6 +27,7 @@ TAG = {
     "XQ": 1, "XK": 2, "XV": 3, "LR": 4, "W0": 5, "LNW": 6, "LNB": 7,
     "W1": 8, "W2": 9, "B0": 10, "B1": 11, "B2": 12,
     "ONX": 13, "ONW": 14, "ONLW": 15, "ONLB": 16,
+    "DO": 17, "DWL": 18, "DBL": 19,
 }
 
 SEED_BASE = 0x77170000
@@ -202,6 +203,31 @@ def linear_inputs(w: Workload, chains=None, values: bool = True, t0: int = 0, t1
                  lambda seed, tag_, n, first: logistic_normal(seed, tag_, n, first, float(w.d)))
     out["lr"] = lr.reshape((w.B, w.H, t1 - t0) if chains is None else (len(chains), t1 - t0))
     out.update(state_inputs(w))
+    return out
+
+
+def upstream_grads(w: Workload, chains=None, values: bool = True, std: float = 1.0) -> dict:
+    """Seeded gradients arriving at the scan's outputs, for its backward: d_out shaped and typed
+    like the activations (fp32 values and, for bf16 workloads, bf16 bit patterns in d_out_bits;
+    values omitted for bf16 when values is False), dW_last [B,H,d,d] and db_last [B,H,d] fp32
+    ([n,...] for a chain subset); every entry N(0, std^2).  A chain's draws do not depend on
+    which other chains are drawn."""
+    d = w.d
+    draw = lambda seed, tag_, n, first: normal(seed, tag_, n, first, 0.0, std)
+    vals = _window(w, "DO", d, 0, w.L, chains, draw)
+    shape = (w.B, w.H, w.L, d) if chains is None else (len(chains), w.L, d)
+    vals = vals.reshape(shape)
+    out = {}
+    if w.dtype == "bf16":
+        out["d_out_bits"] = f32_to_bf16_bits(vals).reshape(shape)
+        if values:
+            out["d_out"] = bf16_bits_to_f32(out["d_out_bits"]).reshape(shape)
+    else:
+        out["d_out"] = vals
+    ids = range(w.chains) if chains is None else chains
+    lead = (w.B, w.H) if chains is None else (len(chains),)
+    out["dW_last"] = np.stack([normal(w.seed, TAG["DWL"], d * d, c * d * d, 0.0, std) for c in ids]).reshape(*lead, d, d)
+    out["db_last"] = np.stack([normal(w.seed, TAG["DBL"], d, c * d, 0.0, std) for c in ids]).reshape(*lead, d)
     return out
 
 

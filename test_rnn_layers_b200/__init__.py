@@ -35,7 +35,8 @@ TTT_STATIC_SCRATCH_BYTES = 33554432
 EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_device_status",
            "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_forward_rope", "ttt_linear_host_workspace_bytes",
            "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward",
-           "ttt_linear_decode_step", "ttt_linear_decode_step_hist", "ttt_o_proj_prepare", "ttt_post_norm_o_proj")
+           "ttt_linear_decode_step", "ttt_linear_decode_step_hist", "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
+           "ttt_linear_backward_workspace_bytes", "ttt_linear_backward")
 
 
 class TTTError(RuntimeError):
@@ -82,11 +83,15 @@ def lib():
                                                   i, vp, vp]
         L.ttt_o_proj_prepare.argtypes = [vp, fp, fp, i, i, vp, fp, fp, vp]
         L.ttt_post_norm_o_proj.argtypes = [vp, ll, i, vp, fp, fp, i, f, vp, fp, vp]
+        L.ttt_linear_backward_workspace_bytes.argtypes = [i, i, ll, i, i, i]
+        L.ttt_linear_backward_workspace_bytes.restype = ll
+        L.ttt_linear_backward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, i, vp, fp,
+                                          fp, vp, vp, vp, fp, fp, fp, fp, fp, vp, ll, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
                      "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
                      "ttt_linear_forward_rope",
                      "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward", "ttt_linear_decode_step",
-                     "ttt_linear_decode_step_hist"):
+                     "ttt_linear_decode_step_hist", "ttt_linear_backward"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -469,3 +474,57 @@ def ttt_post_norm_o_proj(X, Wp, u, v, eps: float = 1e-6, Y=None, row_stats=None,
     _check(lib().ttt_post_norm_o_proj(_ptr(X), T, C, _ptr(Wp), _ptr(u), _ptr(v), N, eps, _ptr(Y), _ptr(row_stats),
                                       _stream(stream)))
     return Y
+
+
+def ttt_linear_backward_workspace_bytes(B: int, H: int, L: int, mini_batch: int = 16, ckpt_group: int = 16,
+                                        d: int = 64) -> int:
+    """Bytes of device workspace that ttt_linear_backward needs (host-only)."""
+    n = lib().ttt_linear_backward_workspace_bytes(B, H, L, d, mini_batch, ckpt_group)
+    if n < 0:
+        _check(int(n))
+    return int(n)
+
+
+def ttt_linear_backward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, d_out, dW_last=None, db_last=None,
+                        mini_batch: int = 16, eps: float = 1e-6, token_eta=None, ckpt_group: int = 16,
+                        workspace=None, stream=None):
+    """Gradients of <d_out, out> + <dW_last, W_last> + <db_last, b_last> for ttt_linear_forward's
+    inputs (head-major [B,H,L,64]; see include/ttt.h).
+
+    Returns a dict: dXQ, dXK, dXV (the activations' dtype), dlr [B,H,L], dW0/db0 (per head when W0
+    is [H,64,64], per chain when it is [B,H,64,64]), dln_w/dln_b [H,64].
+    """
+    _need(XQ, "XQ")
+    B, H, L, d = _act_sizes(XQ, False)
+    dt = XQ.dtype
+    for n, t in (("XK", XK), ("XV", XV), ("d_out", d_out)):
+        _need(t, n, dt, XQ.shape)
+    _need(lr, "lr", torch.float32, (B, H, L))
+    per_chain = W0.dim() == 4
+    _need(W0, "W0", torch.float32, (B, H, d, d) if per_chain else (H, d, d))
+    _need(b0, "b0", torch.float32, (B, H, d) if per_chain else (H, d))
+    _need(ln_w, "ln_w", torch.float32, (H, d))
+    _need(ln_b, "ln_b", torch.float32, (H, d))
+    if dW_last is not None:
+        _need(dW_last, "dW_last", torch.float32, (B, H, d, d))
+    if db_last is not None:
+        _need(db_last, "db_last", torch.float32, (B, H, d))
+    if token_eta is not None:
+        _need(token_eta, "token_eta", torch.float32, (mini_batch,))
+    dev = XQ.device
+    ws_bytes = ttt_linear_backward_workspace_bytes(B, H, L, mini_batch, ckpt_group, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    else:
+        _need(workspace, "workspace", torch.uint8)
+    g = {"dXQ": torch.empty_like(XQ), "dXK": torch.empty_like(XQ), "dXV": torch.empty_like(XQ),
+         "dlr": torch.empty((B, H, L), device=dev),
+         "dW0": torch.empty(W0.shape, device=dev), "db0": torch.empty(b0.shape, device=dev),
+         "dln_w": torch.empty((H, d), device=dev), "dln_b": torch.empty((H, d), device=dev)}
+    _check(lib().ttt_linear_backward(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
+                                     H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
+                                     eps, _dtype_code(XQ), ckpt_group, _ptr(d_out), _ptr(dW_last), _ptr(db_last),
+                                     _ptr(g["dXQ"]), _ptr(g["dXK"]), _ptr(g["dXV"]), _ptr(g["dlr"]), _ptr(g["dW0"]),
+                                     _ptr(g["db0"]), _ptr(g["dln_w"]), _ptr(g["dln_b"]), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)))
+    return g

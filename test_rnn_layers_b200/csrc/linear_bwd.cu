@@ -1,0 +1,486 @@
+// linear_bwd.cu -- backward of the TTT-Linear scan: the gradients of the outer inputs.
+//
+// The walkthrough ("代码连连看——TTT", TTTLinear.ttt) trains through the same scan as the forward,
+// passing scan_checkpoint_group_size to its scan while training: the carried state is kept every
+// G mini-batches and rebuilt inside a group when the backward reaches it.  This file is that
+// backward, per chain (b, h), for the dual form of compute_mini_batch.  Per full mini-batch of
+// K tokens at state (W, b), with t_i the token eta, e_j = t_{K-1} lr_j, tau = XV - XK:
+//   Z = XK W + b;  g = ln_fused_l2_bwd(Z, tau)   (x_hat, sigma: Z's LayerNorm statistics)
+//   M = eta * tril(XQ XK^T + 1), eta[i][j] = t_i lr_j;  Zbar = XQ W + b - M g
+//   out = XQ + LN(Zbar);  W' = W - XK^T diag(e) g;  b' = b - e^T g
+// Given dout and the adjoints (dW', db') of the state after the mini-batch:
+//   dZbar = LN backward of dout;  dXQ = dout + dZbar W^T + dA XK
+//   dM = -dZbar g^T (lower triangle);  dA = dM * eta;  dlr_j += sum_i t_i (A_ij + 1) dM_ij
+//   U = XK dW' + db';  dg = -M^T dZbar - diag(e) U;  dlr_j += -t_{K-1} sum_f g_jf U_jf
+//   dXK = -diag(e) g dW'^T + dA^T XQ - dtau + dZ W^T;  dXV = dtau
+//   (dZ, dtau, d ln_w, d ln_b) = the vector-Jacobian product of ln_fused_l2_bwd with dg
+//   dW = dW' + XQ^T dZbar + XK^T dZ;  db = db' + sum_rows (dZbar + dZ)
+// The remainder tail (K = r) has no update: its terms in dW', db' and e are absent, and it
+// starts from the state after the full mini-batches, whose adjoint is the caller's dW_last.
+//
+// Design (one CTA of 256 threads per chain, fp32 throughout):
+//  * Phase 1 runs the forward state recursion over the full mini-batches from (W0, b0) and
+//    writes every G-th state to the workspace.  Phase 2 walks the groups from the last: it
+//    rebuilds the group's states from its checkpoint into a per-chain slab, then runs the
+//    backward step for each mini-batch of the group in reverse.  Both phases run the same
+//    forward-step code, so a rebuilt state has the bits of the first.
+//  * Tiles of 16 rows x 64 features: thread (r, c0) = (tid / 16, 4 (tid % 16)) owns four
+//    consecutive features of one row, so a row's LayerNorm sums are half-warp shuffles, and
+//    every product against a 64-wide matrix is one row of shared memory times that matrix,
+//    read as float4 rows (rows padded to 68 floats).  The state and its adjoint are kept in
+//    shared memory both as [k][f] and transposed, so that XW and XW^T products read alike;
+//    each thread owns a 4 x 4 block of them in registers and republishes it after an update.
+//  * The LayerNorm statistics are two-pass (mean, then the centred sum of squares).
+#include "ttt_common.cuh"
+#include "ttt_internal.h"
+
+namespace ttt {
+namespace {
+
+constexpr int kT = 256;                          // threads per CTA
+constexpr int kS = TTT_D + 4;                    // row stride of the 64-wide arrays (floats)
+constexpr int kS16 = TTT_KMAX + 4;               // row stride of the 16 x 16 arrays
+constexpr int kState = TTT_D * TTT_D + TTT_D;    // floats of one saved state (W, then b)
+constexpr int kPart = TTT_D * TTT_D + 3 * TTT_D; // floats of one chain's shares (dW0, db0, dln_w, dln_b)
+
+struct __align__(16) BwdSmem {
+    float W[TTT_D][kS];     // the state at the current mini-batch's start, [k][f]
+    float WT[TTT_D][kS];    // its transpose, [f][k]
+    float dW[TTT_D][kS];    // the adjoint of the state after the mini-batch, [k][f]
+    float dWT[TTT_D][kS];
+    float xq[TTT_KMAX][kS];
+    float xk[TTT_KMAX][kS];
+    float g[TTT_KMAX][kS];   // the loss gradient of each token
+    float dzb[TTT_KMAX][kS]; // dZbar
+    float dz[TTT_KMAX][kS];  // dZ
+    float A[TTT_KMAX][kS16];
+    float M[TTT_KMAX][kS16];
+    float MT[TTT_KMAX][kS16];
+    float dA[TTT_KMAX][kS16];
+    float dAT[TTT_KMAX][kS16];
+    float dlr_eta[TTT_KMAX][kS16];  // t_i (A_ij + 1) dM_ij: the eta path's share of dlr_j
+    float b[TTT_D];
+    float db[TTT_D];
+    float lr[TTT_KMAX];
+    float te[TTT_KMAX];
+    float dlr_row[TTT_KMAX];        // the update path's share of dlr_j
+};
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void st4(__nv_bfloat16* p, float4 v) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+
+__device__ __forceinline__ float4 f4(float a) { return make_float4(a, a, a, a); }
+__device__ __forceinline__ float4 operator+(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+__device__ __forceinline__ float4 operator-(float4 a, float4 b) { return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w); }
+__device__ __forceinline__ float4 operator*(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+__device__ __forceinline__ float4 operator*(float4 a, float s) { return make_float4(a.x * s, a.y * s, a.z * s, a.w * s); }
+__device__ __forceinline__ float hsum4(float4 a) { return (a.x + a.y) + (a.z + a.w); }
+
+// Sum over the 16 lanes of a half-warp (the 16 threads of one tile row).
+__device__ __forceinline__ float row_sum(float v) {
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// sum_{k < N} x[k] Y[k][c0 .. c0 + 3]: one row x (16-byte aligned) times the rows of Y.
+template <int N, int kStride>
+__device__ __forceinline__ float4 row_times(const float* x, const float (*Y)[kStride], int c0) {
+    float4 acc = f4(0.f);
+#pragma unroll 2  // (full unrolling spills at 2 CTAs per SM)
+    for (int k = 0; k < N; k += 4) {
+        const float4 xv = ld4(x + k);
+        const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 y = ld4(&Y[k + j][c0]);
+            acc.x = fmaf(xs[j], y.x, acc.x);
+            acc.y = fmaf(xs[j], y.y, acc.y);
+            acc.z = fmaf(xs[j], y.z, acc.z);
+            acc.w = fmaf(xs[j], y.w, acc.w);
+        }
+    }
+    return acc;
+}
+
+// sum_f p[f] q[f] over 64 features (rows of stride kS).
+__device__ __forceinline__ float dot64(const float* p, const float* q) {
+    float acc = 0.f;
+#pragma unroll
+    for (int f = 0; f < TTT_D; f += 4) {
+        const float4 a = ld4(p + f), b = ld4(q + f);
+        acc = fmaf(a.x, b.x, acc);
+        acc = fmaf(a.y, b.y, acc);
+        acc = fmaf(a.z, b.z, acc);
+        acc = fmaf(a.w, b.w, acc);
+    }
+    return acc;
+}
+
+// LayerNorm statistics of a row whose four features z this thread holds: x_hat and sigma.
+__device__ __forceinline__ void row_norm(float4 z, float eps, float4& xh, float& sigma) {
+    const float mu = row_sum(hsum4(z)) * (1.0f / TTT_D);
+    const float4 c = z - f4(mu);
+    const float v = row_sum(hsum4(c * c)) * (1.0f / TTT_D);
+    sigma = sqrtf(v + eps);
+    xh = make_float4(c.x / sigma, c.y / sigma, c.z / sigma, c.w / sigma);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kT, 2) linear_bwd_kernel(const LinearBwdArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    BwdSmem& s = *reinterpret_cast<BwdSmem*>(smem_raw);
+    const int tid = threadIdx.x;
+    const int r = tid >> 4, c0 = 4 * (tid & 15);  // this thread's tile row and four features
+    const int kb = 4 * (tid >> 4);                 // its 4 x 4 block of a state: rows kb.., columns c0..
+    const long long chain = blockIdx.x;
+    const int h = static_cast<int>(chain % a.H);
+    const int K = a.K;
+    const int G = a.G;
+    const long long L = a.L;
+    const float eps = a.eps;
+    const long long base = chain * L * TTT_D;
+    const T* XQ = static_cast<const T*>(a.XQ) + base;
+    const T* XK = static_cast<const T*>(a.XK) + base;
+    const T* XV = static_cast<const T*>(a.XV) + base;
+    const T* DO = static_cast<const T*>(a.d_out) + base;
+    T* dXQ = static_cast<T*>(a.dXQ) + base;
+    T* dXK = static_cast<T*>(a.dXK) + base;
+    T* dXV = static_cast<T*>(a.dXV) + base;
+    const float* lr = a.lr + chain * L;
+    float* dlr = a.d_lr + chain * L;
+    const float* lwp = a.ln_w + h * TTT_D + c0;
+    const float* lbp = a.ln_b + h * TTT_D + c0;
+    const float4 lw = make_float4(lwp[0], lwp[1], lwp[2], lwp[3]);
+    const float4 lb = make_float4(lbp[0], lbp[1], lbp[2], lbp[3]);
+
+    if (tid < TTT_KMAX) s.te[tid] = a.token_eta ? (tid < K ? a.token_eta[tid] : 0.f) : 1.0f / (tid + 1);
+    const float* W0 = a.W0 + (a.w0_chain_stride ? chain * a.w0_chain_stride : static_cast<long long>(h) * TTT_D * TTT_D);
+    const float* b0 = a.b0 + (a.w0_chain_stride ? chain * TTT_D : static_cast<long long>(h) * TTT_D);
+    float Wb[4][4];   // W[kb + i][c0 + j]
+    float dWb[4][4];  // the adjoint, same block
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 v = ld4(W0 + (kb + i) * TTT_D + c0);
+        Wb[i][0] = v.x; Wb[i][1] = v.y; Wb[i][2] = v.z; Wb[i][3] = v.w;
+    }
+    if (tid < TTT_D) s.b[tid] = b0[tid];
+
+    auto put_state = [&](bool transposed) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st4(&s.W[kb + i][c0], make_float4(Wb[i][0], Wb[i][1], Wb[i][2], Wb[i][3]));
+        if (transposed) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st4(&s.WT[c0 + j][kb], make_float4(Wb[0][j], Wb[1][j], Wb[2][j], Wb[3][j]));
+        }
+    };
+    auto put_adjoint = [&]() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st4(&s.dW[kb + i][c0], make_float4(dWb[i][0], dWb[i][1], dWb[i][2], dWb[i][3]));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) st4(&s.dWT[c0 + j][kb], make_float4(dWb[0][j], dWb[1][j], dWb[2][j], dWb[3][j]));
+    };
+    // a state in the workspace: this thread's block, and b from the threads tid < 64
+    auto save_state = [&](float* dst) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st4(dst + (kb + i) * TTT_D + c0, make_float4(Wb[i][0], Wb[i][1], Wb[i][2], Wb[i][3]));
+        if (tid < TTT_D) dst[TTT_D * TTT_D + tid] = s.b[tid];
+    };
+    auto load_state = [&](const float* src) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 v = ld4(src + (kb + i) * TTT_D + c0);
+            Wb[i][0] = v.x; Wb[i][1] = v.y; Wb[i][2] = v.z; Wb[i][3] = v.w;
+        }
+        if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
+    };
+
+    // One full mini-batch of the forward state recursion: (W, b) in Wb / s.b (W also published in
+    // s.W) becomes W - XK^T diag(e) g, b - e^T g.
+    auto fwd_step = [&](long long t0) {
+        const bool live = r < K;
+        const long long row = (t0 + r) * TTT_D + c0;
+        const float4 k4 = live ? ld4(XK + row) : f4(0.f);
+        const float4 v4 = live ? ld4(XV + row) : f4(0.f);
+        st4(&s.xk[r][c0], k4);
+        if (tid < TTT_KMAX) s.lr[tid] = tid < K ? lr[t0 + tid] : 0.f;
+        __syncthreads();
+        const float4 z = row_times<TTT_D>(s.xk[r], s.W, c0) + ld4(&s.b[c0]);
+        float4 xh;
+        float sig;
+        row_norm(z, eps, xh, sig);
+        const float4 q = lw * (lw * xh + lb - (v4 - k4));
+        const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
+        const float4 g = live ? (q - f4(mq) - xh * mqx) * (1.0f / sig) : f4(0.f);
+        st4(&s.g[r][c0], g);
+        __syncthreads();
+        const float tl = s.te[K - 1];
+        for (int i = 0; i < K; ++i) {
+            const float4 x = ld4(&s.xk[i][kb]);
+            const float4 ge = ld4(&s.g[i][c0]) * (tl * s.lr[i]);
+            const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                Wb[u][0] = fmaf(-xs[u], ge.x, Wb[u][0]);
+                Wb[u][1] = fmaf(-xs[u], ge.y, Wb[u][1]);
+                Wb[u][2] = fmaf(-xs[u], ge.z, Wb[u][2]);
+                Wb[u][3] = fmaf(-xs[u], ge.w, Wb[u][3]);
+            }
+        }
+        if (tid < TTT_D) {
+            float acc = 0.f;
+            for (int i = 0; i < K; ++i) acc = fmaf(tl * s.lr[i], s.g[i][tid], acc);
+            s.b[tid] -= acc;
+        }
+        __syncthreads();  // every read of this step's tiles and of s.W is done
+        put_state(false);
+    };
+
+    float4 dgam = f4(0.f), dbet = f4(0.f);  // this thread's shares of d ln_w, d ln_b
+
+    // The backward step of the mini-batch at t0 (Km tokens; full: it updated the state), with its
+    // start state in Wb / s.W / s.WT / s.b and the adjoint of the state after it in dWb / s.dW /
+    // s.dWT / s.db.  Leaves the adjoint of its start state there.
+    auto bwd_step = [&](long long t0, int Km, bool full) {
+        const bool live = r < Km;
+        const long long row = (t0 + r) * TTT_D + c0;
+        const float4 q4 = live ? ld4(XQ + row) : f4(0.f);
+        const float4 k4 = live ? ld4(XK + row) : f4(0.f);
+        const float4 v4 = live ? ld4(XV + row) : f4(0.f);
+        const float4 o4 = live ? ld4(DO + row) : f4(0.f);
+        st4(&s.xq[r][c0], q4);
+        st4(&s.xk[r][c0], k4);
+        if (tid < TTT_KMAX) s.lr[tid] = tid < Km ? lr[t0 + tid] : 0.f;
+        __syncthreads();  // (1)
+        // the mini-batch's forward once more: Z, its statistics, g
+        const float4 z = row_times<TTT_D>(s.xk[r], s.W, c0) + ld4(&s.b[c0]);
+        float4 xh;
+        float sig;
+        row_norm(z, eps, xh, sig);
+        const float4 res = lw * xh + lb - (v4 - k4);  // LN(Z) - (XV - XK)
+        const float4 q = lw * res;
+        const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
+        const float4 g = live ? (q - f4(mq) - xh * mqx) * (1.0f / sig) : f4(0.f);
+        st4(&s.g[r][c0], g);
+        {  // A = XQ XK^T and M = eta * tril(A + 1) at (i, j) = (r, tid % 16)
+            const int i = r, j = tid & 15;
+            const float av = dot64(s.xq[i], s.xk[j]);
+            const float m = (j <= i && i < Km) ? s.te[i] * s.lr[j] * (av + 1.0f) : 0.f;
+            s.A[i][j] = av;
+            s.M[i][j] = m;
+            s.MT[j][i] = m;
+        }
+        __syncthreads();  // (2)
+        // Zbar, and the backward of out = XQ + LN(Zbar)
+        const float4 zb = row_times<TTT_D>(s.xq[r], s.W, c0) + ld4(&s.b[c0]) - row_times<TTT_KMAX>(s.M[r], s.g, c0);
+        float4 xhb;
+        float sigb;
+        row_norm(zb, eps, xhb, sigb);
+        const float4 p = lw * o4;
+        const float mp = row_sum(hsum4(p)) * (1.0f / TTT_D), mpx = row_sum(hsum4(p * xhb)) * (1.0f / TTT_D);
+        const float4 dzb = (p - f4(mp) - xhb * mpx) * (1.0f / sigb);
+        dgam = dgam + o4 * xhb;
+        dbet = dbet + o4;
+        st4(&s.dzb[r][c0], dzb);
+        // the update's terms, read from the adjoint after the mini-batch before this step adds to it
+        float4 U = f4(0.f), V = f4(0.f);
+        if (full) {
+            U = row_times<TTT_D>(s.xk[r], s.dW, c0) + ld4(&s.db[c0]);  // XK dW' + db'
+            V = row_times<TTT_D>(s.g[r], s.dWT, c0);                   // g dW'^T
+        }
+        __syncthreads();  // (3)
+        float4 dg = f4(0.f) - row_times<TTT_KMAX>(s.MT[r], s.dzb, c0);  // -M^T dZbar
+        float4 dxk = f4(0.f);
+        float dlr_upd = 0.f;
+        if (full) {
+            const float tl = s.te[K - 1], e = tl * s.lr[r];
+            dg = dg - U * e;
+            dlr_upd = -tl * row_sum(hsum4(g * U));
+            dxk = f4(0.f) - V * e;
+        }
+        if ((tid & 15) == 0) s.dlr_row[r] = dlr_upd;
+        {  // dM = -dZbar g^T on the lower triangle: its shares of dA and of dlr
+            const int i = r, j = tid & 15;
+            const float dm = (j <= i && i < Km) ? -dot64(s.dzb[i], s.g[j]) : 0.f;
+            s.dlr_eta[i][j] = s.te[i] * (s.A[i][j] + 1.0f) * dm;
+            const float da = dm * s.te[i] * s.lr[j];
+            s.dA[i][j] = da;
+            s.dAT[j][i] = da;
+        }
+        {  // the vector-Jacobian product of g = ln_fused_l2_bwd(Z, tau) with dg
+            const float rs = 1.0f / sig;
+            const float mu = row_sum(hsum4(dg)) * (1.0f / TTT_D), mux = row_sum(hsum4(dg * xh)) * (1.0f / TTT_D);
+            const float4 w = (dg - f4(mu) - xh * mux) * rs;             // through q
+            const float4 hx = lw * lw * w - (dg * mqx + q * mux) * rs;  // through x_hat
+            const float ds = -row_sum(hsum4(dg * g)) * rs;              // through sigma's own factor
+            const float mh = row_sum(hsum4(hx)) * (1.0f / TTT_D), mhx = row_sum(hsum4(hx * xh)) * (1.0f / TTT_D);
+            const float4 dz = (hx - f4(mh) - xh * mhx) * rs + xh * (ds * (1.0f / TTT_D));
+            dgam = dgam + w * (res + lw * xh);
+            dbet = dbet + w * lw;
+            const float4 dtau = f4(0.f) - w * lw;
+            dxk = dxk - dtau;
+            if (live) st4(dXV + row, dtau);
+            st4(&s.dz[r][c0], live ? dz : f4(0.f));
+        }
+        __syncthreads();  // (4)
+        const float4 dxq = o4 + row_times<TTT_D>(s.dzb[r], s.WT, c0) + row_times<TTT_KMAX>(s.dA[r], s.xk, c0);
+        dxk = dxk + row_times<TTT_KMAX>(s.dAT[r], s.xq, c0) + row_times<TTT_D>(s.dz[r], s.WT, c0);
+        if (live) {
+            st4(dXQ + row, dxq);
+            st4(dXK + row, dxk);
+        }
+        if (tid < Km) {
+            float acc = s.dlr_row[tid];
+            for (int i = 0; i < TTT_KMAX; ++i) acc += s.dlr_eta[i][tid];
+            dlr[t0 + tid] = acc;
+        }
+        // the adjoint of the start state: dW' + XQ^T dZbar + XK^T dZ, db' + sum of the rows
+        for (int i = 0; i < Km; ++i) {
+            const float4 xa = ld4(&s.xq[i][kb]), xb = ld4(&s.xk[i][kb]);
+            const float4 ua = ld4(&s.dzb[i][c0]), ub = ld4(&s.dz[i][c0]);
+            const float as[4] = {xa.x, xa.y, xa.z, xa.w}, bs[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                dWb[u][0] = fmaf(as[u], ua.x, fmaf(bs[u], ub.x, dWb[u][0]));
+                dWb[u][1] = fmaf(as[u], ua.y, fmaf(bs[u], ub.y, dWb[u][1]));
+                dWb[u][2] = fmaf(as[u], ua.z, fmaf(bs[u], ub.z, dWb[u][2]));
+                dWb[u][3] = fmaf(as[u], ua.w, fmaf(bs[u], ub.w, dWb[u][3]));
+            }
+        }
+        if (tid < TTT_D) {
+            float acc = 0.f;
+            for (int i = 0; i < Km; ++i) acc += s.dzb[i][tid] + s.dz[i][tid];
+            s.db[tid] += acc;
+        }
+        __syncthreads();  // (5) every read of this step's tiles and adjoint copies is done
+        put_adjoint();
+    };
+
+    // ---- phase 1: the forward state recursion, a checkpoint every G full mini-batches --------
+    put_state(false);
+    __syncthreads();
+    for (long long m = 0; m < a.n_full; ++m) {
+        if (m % G == 0) save_state(a.ckpt + (chain * a.n_ckpt + m / G) * kState);
+        fwd_step(m * K);
+    }
+
+    // ---- the remainder tail, from the state after the full mini-batches -----------------------
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 v = a.dW_last ? ld4(a.dW_last + chain * TTT_D * TTT_D + (kb + i) * TTT_D + c0) : f4(0.f);
+        dWb[i][0] = v.x; dWb[i][1] = v.y; dWb[i][2] = v.z; dWb[i][3] = v.w;
+    }
+    if (tid < TTT_D) s.db[tid] = a.db_last ? a.db_last[chain * TTT_D + tid] : 0.f;
+    put_adjoint();
+    if (a.rem > 0) {
+        put_state(true);
+        __syncthreads();
+        bwd_step(a.n_full * K, static_cast<int>(a.rem), false);
+    }
+
+    // ---- phase 2: the groups from the last; rebuild each one's states, then step back ----------
+    float* const slab = a.slab + chain * G * kState;
+    for (long long c = a.n_ckpt - 1; c >= 0; --c) {
+        const long long m0 = c * G, m1 = m0 + G < a.n_full ? m0 + G : a.n_full;
+        __syncthreads();
+        load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
+        put_state(false);
+        __syncthreads();
+        for (long long m = m0; m < m1; ++m) {
+            save_state(slab + (m - m0) * kState);
+            if (m + 1 < m1) fwd_step(m * K);
+        }
+        for (long long m = m1 - 1; m >= m0; --m) {
+            __syncthreads();
+            load_state(slab + (m - m0) * kState);
+            put_state(true);
+            __syncthreads();
+            bwd_step(m * K, K, true);
+        }
+    }
+
+    // ---- this chain's shares of the shared parameters' gradients -----------------------------
+    float* part = a.part + chain * kPart;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st4(part + (kb + i) * TTT_D + c0, make_float4(dWb[i][0], dWb[i][1], dWb[i][2], dWb[i][3]));
+    __syncthreads();
+    st4(&s.g[r][c0], dgam);
+    st4(&s.dzb[r][c0], dbet);
+    __syncthreads();
+    if (tid < TTT_D) {
+        float sg = 0.f, sb = 0.f;
+        for (int i = 0; i < TTT_KMAX; ++i) {
+            sg += s.g[i][tid];
+            sb += s.dzb[i][tid];
+        }
+        part[TTT_D * TTT_D + tid] = s.db[tid];
+        part[TTT_D * TTT_D + TTT_D + tid] = sg;
+        part[TTT_D * TTT_D + 2 * TTT_D + tid] = sb;
+    }
+}
+
+// The batch sums of the chains' shares: d ln_w, d ln_b per head, and dW0, db0 per head when the
+// initial state is one per head (w0_per_chain = 0).  Fixed summation order over b.
+__global__ void linear_bwd_reduce_kernel(const float* part, int B, int H, int w0_per_chain, float* dW0, float* db0,
+                                         float* dlnw, float* dlnb) {
+    const long long n = static_cast<long long>(H) * kPart;
+    for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int h = static_cast<int>(idx / kPart), e = static_cast<int>(idx % kPart);
+        if (w0_per_chain && e < TTT_D * TTT_D + TTT_D) continue;
+        float acc = 0.f;
+        for (int b = 0; b < B; ++b) acc += part[(static_cast<long long>(b) * H + h) * kPart + e];
+        if (e < TTT_D * TTT_D) dW0[static_cast<long long>(h) * TTT_D * TTT_D + e] = acc;
+        else if (e < TTT_D * TTT_D + TTT_D) db0[h * TTT_D + e - TTT_D * TTT_D] = acc;
+        else if (e < TTT_D * TTT_D + 2 * TTT_D) dlnw[h * TTT_D + e - TTT_D * TTT_D - TTT_D] = acc;
+        else dlnb[h * TTT_D + e - TTT_D * TTT_D - 2 * TTT_D] = acc;
+    }
+}
+
+// dW0, db0 of each chain when every chain started from its own state.
+__global__ void linear_bwd_copy_kernel(const float* part, long long chains, float* dW0, float* db0) {
+    constexpr int kN = TTT_D * TTT_D + TTT_D;
+    for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < chains * kN;
+         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long c = idx / kN;
+        const int e = static_cast<int>(idx % kN);
+        const float v = part[c * kPart + e];
+        if (e < TTT_D * TTT_D) dW0[c * TTT_D * TTT_D + e] = v;
+        else db0[c * TTT_D + e - TTT_D * TTT_D] = v;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_linear_bwd(const LinearBwdArgs& a, int dtype, cudaStream_t st) {
+    const size_t smem = sizeof(BwdSmem);
+    auto kernel = dtype == 0 ? linear_bwd_kernel<float> : linear_bwd_kernel<__nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kernel<<<static_cast<unsigned>(a.B * a.H), kT, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_linear_bwd_reduce(const float* part, int B, int H, int w0_per_chain, float* dW0, float* db0,
+                                     float* d_ln_w, float* d_ln_b, cudaStream_t st) {
+    const long long n = static_cast<long long>(H) * kPart;
+    const unsigned blocks = static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    linear_bwd_reduce_kernel<<<blocks, 256, 0, st>>>(part, B, H, w0_per_chain, dW0, db0, d_ln_w, d_ln_b);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || !w0_per_chain) return e;
+    const long long chains = static_cast<long long>(B) * H;
+    const long long m = chains * (TTT_D * TTT_D + TTT_D);
+    const unsigned cb = static_cast<unsigned>((m + 255) / 256 < 8192 ? (m + 255) / 256 : 8192);
+    linear_bwd_copy_kernel<<<cb, 256, 0, st>>>(part, chains, dW0, db0);
+    return cudaGetLastError();
+}
+
+}  // namespace ttt

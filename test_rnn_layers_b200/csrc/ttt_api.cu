@@ -752,6 +752,101 @@ int ttt_post_norm_o_proj(const void* X, long long T, int C, const void* Wp, cons
     return ok();
 }
 
+// ---- the backward of the TTT-Linear scan -------------------------------------------------------
+// Workspace: [chains][n_ckpt] kept states, [chains][G] rebuilt states, [chains] gradient shares.
+struct BwdLayout {
+    long long n_ckpt;
+    size_t slab, part, total;
+};
+
+static BwdLayout bwd_layout(int B, int H, long long L, int K, int G) {
+    const long long chains = static_cast<long long>(B) * H;
+    const long long n_full = L / K;
+    const size_t state = static_cast<size_t>(kD * kD + kD) * 4;
+    BwdLayout y;
+    y.n_ckpt = (n_full + G - 1) / G;
+    y.slab = up256(static_cast<size_t>(chains * y.n_ckpt) * state);
+    y.part = y.slab + up256(static_cast<size_t>(chains) * G * state);
+    y.total = y.part + up256(static_cast<size_t>(chains) * (kD * kD + 3 * kD) * 4);
+    return y;
+}
+
+long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, int mini_batch, int ckpt_group) {
+    int rc = check_common(B, H, L, d, mini_batch, 1.0f, TTT_F32, 0);
+    if (rc) return rc;
+    if (ckpt_group < 1) return fail(TTT_ERR_ARG, "ckpt_group must be >= 1 (got %d)", ckpt_group);
+    ok();
+    return static_cast<long long>(bwd_layout(B, H, L, mini_batch, ckpt_group).total);
+}
+
+int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                        const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
+                        const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps, int dtype,
+                        int ckpt_group, const void* d_out, const float* dW_last, const float* db_last, void* dXQ,
+                        void* dXK, void* dXV, float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b,
+                        void* workspace, long long workspace_bytes, void* stream) {
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, 0);
+    if (rc) return rc;
+    if (ckpt_group < 1) return fail(TTT_ERR_ARG, "ckpt_group must be >= 1 (got %d)", ckpt_group);
+    const long long chains = static_cast<long long>(B) * H;
+    const long long per_head = static_cast<long long>(kD) * kD;
+    if (w0_batch_stride != 0 && w0_batch_stride != H * per_head)
+        return fail(TTT_ERR_ARG, "w0_batch_stride must be 0 or H*d*d (got %lld)", w0_batch_stride);
+    if (!W0 || !b0 || !ln_w || !ln_b || !dW0 || !db0 || !d_ln_w || !d_ln_b || !workspace)
+        return fail(TTT_ERR_ARG, "W0, b0, ln_w, ln_b, dW0, db0, d_ln_w, d_ln_b and workspace must be non-null");
+    if (L > 0 && (!XQ || !XK || !XV || !lr || !d_out || !dXQ || !dXK || !dXV || !d_lr))
+        return fail(TTT_ERR_ARG, "XQ, XK, XV, lr, d_out, dXQ, dXK, dXV and d_lr must be non-null when L > 0");
+    const void* a16[] = {XQ, XK, XV, d_out, dXQ, dXK, dXV, W0, b0, dW_last, db_last, dW0, db0};
+    const char* n16[] = {"XQ", "XK", "XV", "d_out", "dXQ", "dXK", "dXV", "W0", "b0", "dW_last", "db_last", "dW0", "db0"};
+    for (int i = 0; i < 13; ++i)
+        if (a16[i] && !aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "%s must be 16-byte aligned", n16[i]);
+    const void* a4[] = {lr, token_eta, ln_w, ln_b, d_lr, d_ln_w, d_ln_b};
+    const char* n4[] = {"lr", "token_eta", "ln_w", "ln_b", "d_lr", "d_ln_w", "d_ln_b"};
+    for (int i = 0; i < 7; ++i)
+        if (a4[i] && !aligned(a4[i], 4)) return fail(TTT_ERR_ALIGN, "%s must be 4-byte aligned", n4[i]);
+    if (!aligned(workspace, 256)) return fail(TTT_ERR_ALIGN, "workspace must be 256-byte aligned");
+    const BwdLayout lay = bwd_layout(B, H, L, mini_batch, ckpt_group);
+    if (workspace_bytes < 0 || static_cast<size_t>(workspace_bytes) < lay.total)
+        return fail(TTT_ERR_ARG, "workspace_bytes %lld below the %zu bytes needed", workspace_bytes, lay.total);
+
+    const size_t esz = dtype == TTT_F32 ? 4 : 2;
+    const size_t act = static_cast<size_t>(chains) * L * kD * esz;
+    const size_t tok = static_cast<size_t>(chains * L) * 4;
+    const long long wrows = w0_batch_stride ? chains : H;
+    const size_t wbytes = static_cast<size_t>(wrows * per_head) * 4, bbytes = static_cast<size_t>(wrows * kD) * 4;
+    const size_t hbytes = static_cast<size_t>(H) * kD * 4;
+    Span in[] = {{"XQ", XQ, act}, {"XK", XK, act}, {"XV", XV, act}, {"lr", lr, tok},
+                 {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4}, {"W0", W0, wbytes}, {"b0", b0, bbytes},
+                 {"ln_w", ln_w, hbytes}, {"ln_b", ln_b, hbytes}, {"d_out", d_out, act},
+                 {"dW_last", dW_last, static_cast<size_t>(chains * per_head) * 4},
+                 {"db_last", db_last, static_cast<size_t>(chains * kD) * 4}};
+    Span outs[] = {{"dXQ", dXQ, act}, {"dXK", dXK, act}, {"dXV", dXV, act}, {"d_lr", d_lr, tok},
+                   {"dW0", dW0, wbytes}, {"db0", db0, bbytes}, {"d_ln_w", d_ln_w, hbytes}, {"d_ln_b", d_ln_b, hbytes},
+                   {"workspace", workspace, lay.total}};
+    rc = check_aliasing(in, 12, outs, 9);
+    if (rc) return rc;
+
+    ttt::LinearBwdArgs a{};
+    a.XQ = XQ; a.XK = XK; a.XV = XV; a.d_out = d_out;
+    a.lr = lr; a.token_eta = token_eta; a.W0 = W0; a.b0 = b0;
+    a.w0_chain_stride = w0_batch_stride ? per_head : 0;
+    a.ln_w = ln_w; a.ln_b = ln_b; a.dW_last = dW_last; a.db_last = db_last;
+    a.B = B; a.H = H; a.K = mini_batch;
+    a.L = L; a.n_full = L / mini_batch; a.rem = L % mini_batch;
+    a.eps = eps; a.G = ckpt_group; a.n_ckpt = lay.n_ckpt;
+    a.dXQ = dXQ; a.dXK = dXK; a.dXV = dXV; a.d_lr = d_lr;
+    char* ws = static_cast<char*>(workspace);
+    a.ckpt = reinterpret_cast<float*>(ws);
+    a.slab = reinterpret_cast<float*>(ws + lay.slab);
+    a.part = reinterpret_cast<float*>(ws + lay.part);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = ttt::launch_linear_bwd(a, dtype, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    e = ttt::launch_linear_bwd_reduce(a.part, B, H, w0_batch_stride ? 1 : 0, dW0, db0, d_ln_w, d_ln_b, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward reduction launch");
+    return ok();
+}
+
 }  // extern "C"
 
 // ---- host-buffer entry that allocates nothing ---------------------------------------------------

@@ -140,6 +140,41 @@ struct OprojArgs {
 struct OprojMaps {
     CUtensorMap x, w;         // X [T][C] box {64, 128}; Wp [N][C] box {64, 256}; bf16, 128-byte swizzle
 };
+// The backward of the TTT-Linear scan (see ttt_linear_backward): one CTA per chain; fp32
+// throughout.  The workspace holds, per chain, the states kept every G mini-batches, one group's
+// rebuilt states, and the chain's shares of the gradients of the shared parameters.
+struct LinearBwdArgs {
+    const void* XQ;
+    const void* XK;
+    const void* XV;
+    const void* d_out;          // upstream gradient of out, the activations' dtype and layout
+    const float* lr;
+    const float* token_eta;     // [K] or nullptr -> 1/(i+1)
+    const float* W0;
+    const float* b0;
+    long long w0_chain_stride;  // elements between chains' W0 (0: one per head)
+    const float* ln_w;
+    const float* ln_b;
+    const float* dW_last;       // [B*H][d][d] or nullptr (zero)
+    const float* db_last;       // [B*H][d] or nullptr (zero)
+    int B, H, K;
+    long long L, n_full, rem;
+    float eps;
+    int G;                      // checkpoint group: a state is kept every G full mini-batches
+    long long n_ckpt;           // ceil(n_full / G)
+    void* dXQ;
+    void* dXK;
+    void* dXV;
+    float* d_lr;
+    float* ckpt;                // [B*H][n_ckpt][d*d + d]
+    float* slab;                // [B*H][G][d*d + d]
+    float* part;                // [B*H][d*d + 3d]: dW0, db0, d ln_w, d ln_b of each chain
+};
+cudaError_t launch_linear_bwd(const LinearBwdArgs& a, int dtype, cudaStream_t s);
+// Sum the per-chain shares over the batch: dW0/db0 per head (w0_per_chain = 0) or copied per chain,
+// d ln_w / d ln_b per head.
+cudaError_t launch_linear_bwd_reduce(const float* part, int B, int H, int w0_per_chain, float* dW0, float* db0,
+                                     float* d_ln_w, float* d_ln_b, cudaStream_t s);
 cudaError_t launch_oproj_prepare(const void* Wo, const float* ln_w, const float* ln_b, int C, int N, void* Wp,
                                  float* u, float* v, cudaStream_t s);
 cudaError_t launch_post_norm_oproj(const OprojArgs& a, const OprojMaps& maps, cudaStream_t s);
