@@ -1,6 +1,6 @@
 """Benchmark of the TTT scan on B200: TTT layer tokens/s and the fraction of the per-layer roofline.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,linear_tm,mlp,decode,decode_hist]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows linear,linear_tm,linear_rope,oproj,backward,mlp,decode,decode_hist]
                     [--no-cpu-baseline] [--no-headline] [--seq-len L]
 
 One step = one ttt_linear_forward over the 1B-layer workload (B=8, H=32, L=8200, d=64, K=16,
@@ -19,9 +19,10 @@ out inside the timed region, the batch pipelined in chunks),
 `roofline` (the scan kernel's algorithmic bytes / its CUDA-event time vs the measured HBM copy
 bandwidth), `cpu_baseline` (the CPU oracle on a bounded sample, rank 0 at N=1), `clocks`
 (NVML samples taken during the timed region) and `rows` (the same scan on token-major
-[B,L,H,d] activations beside the time of the permutes that layout saves, the TTT-MLP prefill,
-the decode step with the dense cache and with the history-format cache, each timed the same
-way).  `--impl reference` times the oracle instead, as the reference arm.
+[B,L,H,d] activations beside the time of the permutes that layout saves, the scan with the
+rotary embedding fused into its load path, the layer's output side post_norm + o_proj, the
+scan's backward with checkpoint groups, the TTT-MLP prefill, the decode step with the dense
+cache and with the history-format cache, each timed the same way).  `--impl reference` times the oracle instead, as the reference arm.
 """
 from __future__ import annotations
 
@@ -77,6 +78,29 @@ def mlp_flops(B, H, L, hid=256, K=16):
     dense = 7 * 2 * K * D * hid                  # Z1, XQ W1, Z2, Xbar2 W2, g2 W2^T, two updates
     tri = 2 * (K * (K + 1) // 2) * (2 * D + 2 * hid)  # Attn1, Attn2, M1 g1, M2 g2
     return B * H * n_mb * (dense + tri)
+
+
+def linear_bwd_bytes(B, H, L):
+    """The backward, once through: reads XQ, XK, XV, d_out (bf16) and lr per token, W0/b0 and
+    ln_w/ln_b per head, dW_last/db_last per chain; writes dXQ, dXK, dXV (bf16) and d_lr per token,
+    dW0/db0 and d ln_w / d ln_b per head."""
+    chains = B * H
+    state = (D * D + D) * 4
+    per_token = 4 * D * 2 + 4 + 3 * D * 2 + 4
+    return chains * L * per_token + 2 * H * state + chains * state + 2 * H * 2 * D * 4
+
+
+def linear_bwd_flops(B, H, L, K=16):
+    """The products the chain rule needs per mini-batch once its Z, g and Zbar are known:
+    XK dW', g dW'^T, dZbar W^T, dZ W^T, XQ^T dZbar, XK^T dZ (6 x 2 K d^2) and the lower-triangular
+    M^T dZbar, dZbar g^T, dA XK, dA^T XQ (4 x 2 d K(K+1)/2).  Rebuilding the states and the
+    forward quantities (Z, XQ W, XQ XK^T, M g, the state updates) is not counted."""
+    n_mb = L // K + (1 if L % K else 0)
+    return B * H * n_mb * (6 * 2 * K * D * D + 4 * 2 * D * K * (K + 1) // 2)
+
+
+# FP32 FMA issue peak from the unit counts: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (max clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def decode_hist_bytes(B, H, p, K=16):
@@ -461,6 +485,40 @@ def bench_post_norm_oproj(args, world, peaks):
             "unfused_torch_ms": round(torch_ms, 4)}
 
 
+def bench_linear_backward(args, world, peaks, G=16):
+    """The backward of the TTT-Linear scan at the 1B layer (ttt_linear_backward, checkpoint group
+    16): the gradients of XQ, XK, XV, lr, W0, b0, ln_w and ln_b from d_out, dW_last and db_last,
+    the inputs and upstream gradients resident in HBM (each larger than L2)."""
+    import torch
+
+    import test_rnn_layers_b200 as ttt
+    w = synth.workload(2, L=args.seq_len)
+    x, up = synth.linear_inputs(w, values=False), synth.upstream_grads(w, values=False)
+    XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
+    dout = dev_act(up, "d_out")
+    t = {k: dev_f32(x[k]) for k in ("lr", "W0", "b0", "ln_w", "ln_b")}
+    dWl, dbl = dev_f32(up["dW_last"]), dev_f32(up["db_last"])
+    del x, up
+    ws = torch.empty(ttt.ttt_linear_backward_workspace_bytes(w.B, w.H, w.L, w.K, G), dtype=torch.uint8, device="cuda")
+
+    def step():
+        ttt.ttt_linear_backward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], dout, dWl, dbl,
+                                mini_batch=w.K, eps=w.eps, ckpt_group=G, workspace=ws)
+
+    K = max(3, min(args.steps, 10))
+    ms = time_steps(step, K, 3, world)
+    flops = linear_bwd_flops(w.B, w.H, w.L)
+    tfl = flops / (ms / 1e3) / 1e12
+    hbm = peaks[0]
+    return {"workload": f"ttt_linear_backward_1b_layer_B{w.B}_H{w.H}_L{w.L}_ckpt{G}",
+            "value": round(world * w.B * w.L / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "steps": K, "gpu_launches": 2 * K, "dtype": "bf16 in/out, f32 compute",
+            "roofline": {"bound": "alu", "achieved": round(tfl, 2), "peak": round(FP32_ALU_TFLOPS, 1),
+                         "peak_source": "fp32 FMA issue rate from unit counts (148 SMs x 128 lanes x 2 x 1.965 GHz)",
+                         "unit": "TFLOP/s", "frac": round(tfl / FP32_ALU_TFLOPS, 4), "algorithmic_flops": flops,
+                         "hbm_frac": round(linear_bwd_bytes(w.B, w.H, w.L) / (ms / 1e3) / 1e9 / hbm, 4)}}
+
+
 def bench_mlp(args, world, peaks):
     import torch
 
@@ -687,7 +745,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rows", default="linear,linear_tm,linear_rope,oproj,mlp,decode,decode_hist",
+    ap.add_argument("--rows", default="linear,linear_tm,linear_rope,oproj,backward,mlp,decode,decode_hist",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-chunk", type=int, default=1,
@@ -718,6 +776,8 @@ def main():
             extra["ttt_linear_prefill_rope"] = bench_linear_rope(args, world, peaks)
         if "oproj" in rows:
             extra["ttt_post_norm_o_proj"] = bench_post_norm_oproj(args, world, peaks)
+        if "backward" in rows:
+            extra["ttt_linear_backward"] = bench_linear_backward(args, world, peaks)
         if "mlp" in rows:
             extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
         if "decode" in rows:
@@ -738,6 +798,8 @@ def main():
         extra["ttt_linear_prefill_rope"] = bench_linear_rope(args, world, peaks)
     if "oproj" in rows:
         extra["ttt_post_norm_o_proj"] = bench_post_norm_oproj(args, world, peaks)
+    if "backward" in rows:
+        extra["ttt_linear_backward"] = bench_linear_backward(args, world, peaks)
     if "mlp" in rows:
         extra["ttt_mlp_prefill"] = bench_mlp(args, world, peaks)
     if "decode" in rows:

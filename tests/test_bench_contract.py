@@ -75,3 +75,13 @@ def test_cpu_baseline_reports_both_precisions_and_the_cores():
     assert cb["cores"] == n and cb["kind"] == "oracle" and cb["cpu_model"]
     assert set(cb["runs"]) == {f"{p}_{c}core" for p in ("f64", "f32") for c in {1, n}}
     assert cb["value"] == cb["runs"][f"f64_{n}core"]["value"] > 0
+
+
+def test_backward_work_counts():
+    import bench
+    per_mb = 6 * 2 * 16 * 64 * 64 + 4 * 2 * 64 * 16 * 17 // 2
+    assert per_mb == 856064
+    assert bench.linear_bwd_flops(1, 1, 16 * 3 + 1) == 4 * per_mb     # the tail counts as a mini-batch
+    per_token = 4 * 128 + 4 + 3 * 128 + 4                             # 4 bf16 rows + lr in, 3 rows + d lr out
+    state = (64 * 64 + 64) * 4
+    assert bench.linear_bwd_bytes(2, 3, 10) == 6 * 10 * per_token + 2 * 3 * state + 6 * state + 2 * 3 * 2 * 64 * 4
