@@ -101,6 +101,8 @@ def linear_bwd_flops(B, H, L, K=16):
 
 # FP32 FMA issue peak from the unit counts: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (max clock)
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# dense TF32 tensor peak as the nominal ratio to bf16 (1.1 / 2.25 PFLOP/s) times the bf16 peak in use
+TF32_PER_BF16 = 1.1 / 2.25
 
 
 def decode_hist_bytes(B, H, p, K=16):
@@ -488,7 +490,9 @@ def bench_post_norm_oproj(args, world, peaks):
 def bench_linear_backward(args, world, peaks, G=16):
     """The backward of the TTT-Linear scan at the 1B layer (ttt_linear_backward, checkpoint group
     16): the gradients of XQ, XK, XV, lr, W0, b0, ln_w and ln_b from d_out, dW_last and db_last,
-    the inputs and upstream gradients resident in HBM (each larger than L2)."""
+    the inputs and upstream gradients resident in HBM (each larger than L2).  bf16 activations run
+    the tensor-core kernel (TF32 products), whose roofline is the larger of the HBM time of its
+    algorithmic bytes and the TF32 time of its algorithmic FLOPs: the HBM one."""
     import torch
 
     import test_rnn_layers_b200 as ttt
@@ -507,16 +511,20 @@ def bench_linear_backward(args, world, peaks, G=16):
 
     K = max(3, min(args.steps, 10))
     ms = time_steps(step, K, 3, world)
-    flops = linear_bwd_flops(w.B, w.H, w.L)
+    flops, nbytes = linear_bwd_flops(w.B, w.H, w.L), linear_bwd_bytes(w.B, w.H, w.L)
     tfl = flops / (ms / 1e3) / 1e12
-    hbm = peaks[0]
+    gbs = nbytes / (ms / 1e3) / 1e9
+    hbm, bf16_peak, _, which = peaks
+    tf32_peak = bf16_peak * TF32_PER_BF16
     return {"workload": f"ttt_linear_backward_1b_layer_B{w.B}_H{w.H}_L{w.L}_ckpt{G}",
             "value": round(world * w.B * w.L / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
-            "steps": K, "gpu_launches": 2 * K, "dtype": "bf16 in/out, f32 compute",
-            "roofline": {"bound": "alu", "achieved": round(tfl, 2), "peak": round(FP32_ALU_TFLOPS, 1),
-                         "peak_source": "fp32 FMA issue rate from unit counts (148 SMs x 128 lanes x 2 x 1.965 GHz)",
-                         "unit": "TFLOP/s", "frac": round(tfl / FP32_ALU_TFLOPS, 4), "algorithmic_flops": flops,
-                         "hbm_frac": round(linear_bwd_bytes(w.B, w.H, w.L) / (ms / 1e3) / 1e9 / hbm, 4)}}
+            "steps": K, "gpu_launches": 2 * K, "dtype": "bf16 in/out, tf32 products, f32 accumulation and state",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "peak_source": f"{which} hbm_gbs",
+                         "unit": "GB/s", "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
+                         "floor_ms": round(nbytes / hbm / 1e6, 4), "algorithmic_flops": flops,
+                         "tensor_tflops": round(tfl, 2),
+                         "tensor_frac_tf32": round(tfl / tf32_peak, 4),
+                         "tf32_peak": round(tf32_peak, 1)}}
 
 
 def bench_mlp(args, world, peaks):

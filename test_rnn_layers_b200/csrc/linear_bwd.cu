@@ -458,11 +458,431 @@ __global__ void linear_bwd_copy_kernel(const float* part, long long chains, floa
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Tensor-core form (bf16 activations).  The 16 x 64 x 64 products and the rank-16 state updates
+// run as TF32 warp MMAs (m16n8k8, fp32 accumulation): the state W and its adjoint dW live as
+// accumulators, warp w holding rows 16 (w / 2) .. +15 and columns 32 (w % 2) .. +31 of each (four
+// 16 x 8 tiles), and their copies in shared memory serve as B operands, read plain or transposed.
+// A 16 x 64 product lands in a shared result tile, warp w computing columns 8w .. 8w + 7, and the
+// row-layout threads read it back.  The LayerNorm work and the 16 x 16 products are as above.
+// ---------------------------------------------------------------------------------------------
+struct __align__(16) BwdTcSmem {
+    float W[TTT_D][kS];
+    float dW[TTT_D][kS];
+    float xq[TTT_KMAX][kS];
+    float xk[TTT_KMAX][kS];
+    float g[TTT_KMAX][kS];
+    float dzb[TTT_KMAX][kS];
+    float dz[TTT_KMAX][kS];
+    float P0[TTT_KMAX][kS];  // product results
+    float P1[TTT_KMAX][kS];
+    float P2[TTT_KMAX][kS];
+    float A[TTT_KMAX][kS16];
+    float M[TTT_KMAX][kS16];
+    float MT[TTT_KMAX][kS16];
+    float dA[TTT_KMAX][kS16];
+    float dAT[TTT_KMAX][kS16];
+    float dlr_eta[TTT_KMAX][kS16];
+    float b[TTT_D];
+    float db[TTT_D];
+    float lr[TTT_KMAX];
+    float te[TTT_KMAX];
+    float dlr_row[TTT_KMAX];
+};
+
+__device__ __forceinline__ uint32_t tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D += A B for one m16n8k8 tile, TF32 operands, fp32 accumulators in place.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// acc += sum_{k < K} X[m][k] Y(k, n0 + n) for the 16 x 8 tile at columns n0: X rows of stride kSX;
+// Y(k, n) = Ymat[k][n], or Ymat[n][k] when kTrans.  Even and odd k-steps accumulate apart (half
+// the dependent MMA latency) and meet at the end.
+template <int K, int kSX, bool kTrans>
+__device__ __forceinline__ void tc_tile(float (&acc)[4], const float (*X)[kSX], const float (*Y)[kS], int n0, int g,
+                                        int t) {
+    float odd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = tf32(X[g][k0 + t]), a1 = tf32(X[g + 8][k0 + t]);
+        const uint32_t a2 = tf32(X[g][k0 + t + 4]), a3 = tf32(X[g + 8][k0 + t + 4]);
+        const uint32_t b0 = tf32(kTrans ? Y[n0 + g][k0 + t] : Y[k0 + t][n0 + g]);
+        const uint32_t b1 = tf32(kTrans ? Y[n0 + g][k0 + t + 4] : Y[k0 + t + 4][n0 + g]);
+        if ((k0 >> 3) & 1) mma_tf32(odd, a0, a1, a2, a3, b0, b1);
+        else mma_tf32(acc, a0, a1, a2, a3, b0, b1);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += odd[e];
+}
+
+// c0 += X0 Y and c1 += X1 Y over K = 64 for the tile at columns n0, sharing Y's fragments.
+template <bool kTrans>
+__device__ __forceinline__ void tc_tile2(float (&c0)[4], float (&c1)[4], const float (*X0)[kS], const float (*X1)[kS],
+                                         const float (*Y)[kS], int n0, int g, int t) {
+#pragma unroll
+    for (int k0 = 0; k0 < TTT_D; k0 += 8) {
+        const uint32_t b0 = tf32(kTrans ? Y[n0 + g][k0 + t] : Y[k0 + t][n0 + g]);
+        const uint32_t b1 = tf32(kTrans ? Y[n0 + g][k0 + t + 4] : Y[k0 + t + 4][n0 + g]);
+        mma_tf32(c0, tf32(X0[g][k0 + t]), tf32(X0[g + 8][k0 + t]), tf32(X0[g][k0 + t + 4]), tf32(X0[g + 8][k0 + t + 4]),
+                 b0, b1);
+        mma_tf32(c1, tf32(X1[g][k0 + t]), tf32(X1[g + 8][k0 + t]), tf32(X1[g][k0 + t + 4]), tf32(X1[g + 8][k0 + t + 4]),
+                 b0, b1);
+    }
+}
+
+// A 16 x 8 accumulator tile into rows 0..15, columns n0..n0+7 of a result tile.
+__device__ __forceinline__ void put_tile(float (*P)[kS], const float (&c)[4], int n0, int g, int t) {
+    *reinterpret_cast<float2*>(&P[g][n0 + 2 * t]) = make_float2(c[0], c[1]);
+    *reinterpret_cast<float2*>(&P[g + 8][n0 + 2 * t]) = make_float2(c[2], c[3]);
+}
+
+// acc (this warp's four 16 x 8 tiles of a 64 x 64 matrix at rows m0, columns n0 + 8q) +=
+// sum_{j < 16} s_j X[j][m] Y[j][n]: the rank-16 update by the tokens of a mini-batch, with
+// s_j = scale * lr[j] (lr non-null) or 1.
+__device__ __forceinline__ void tc_rank16(float (&acc)[4][4], const float (*X)[kS], const float* lr, float scale,
+                                          const float (*Y)[kS], int m0, int n0, int g, int t) {
+#pragma unroll
+    for (int k0 = 0; k0 < TTT_KMAX; k0 += 8) {
+        float x0 = X[k0 + t][m0 + g], x1 = X[k0 + t][m0 + g + 8];
+        float x2 = X[k0 + t + 4][m0 + g], x3 = X[k0 + t + 4][m0 + g + 8];
+        if (lr) {
+            const float s0 = scale * lr[k0 + t], s1 = scale * lr[k0 + t + 4];
+            x0 *= s0;
+            x1 *= s0;
+            x2 *= s1;
+            x3 *= s1;
+        }
+        const uint32_t a0 = tf32(x0), a1 = tf32(x1), a2 = tf32(x2), a3 = tf32(x3);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            mma_tf32(acc[q], a0, a1, a2, a3, tf32(Y[k0 + t][n0 + 8 * q + g]), tf32(Y[k0 + t + 4][n0 + 8 * q + g]));
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    BwdTcSmem& s = *reinterpret_cast<BwdTcSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int r = tid >> 4, c0 = 4 * (tid & 15);       // row layout: this thread's row and four features
+    const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);    // this warp's block of a 64 x 64 matrix
+    const int nt = 8 * w;                               // this warp's columns of a 16 x 64 product
+    const long long chain = blockIdx.x;
+    const int h = static_cast<int>(chain % a.H);
+    const int K = a.K;
+    const int G = a.G;
+    const long long L = a.L;
+    const float eps = a.eps;
+    const long long base = chain * L * TTT_D;
+    const T* XQ = static_cast<const T*>(a.XQ) + base;
+    const T* XK = static_cast<const T*>(a.XK) + base;
+    const T* XV = static_cast<const T*>(a.XV) + base;
+    const T* DO = static_cast<const T*>(a.d_out) + base;
+    T* dXQ = static_cast<T*>(a.dXQ) + base;
+    T* dXK = static_cast<T*>(a.dXK) + base;
+    T* dXV = static_cast<T*>(a.dXV) + base;
+    const float* lr = a.lr + chain * L;
+    float* dlr = a.d_lr + chain * L;
+    const float* lwp = a.ln_w + h * TTT_D + c0;
+    const float* lbp = a.ln_b + h * TTT_D + c0;
+    const float4 lw = make_float4(lwp[0], lwp[1], lwp[2], lwp[3]);
+    const float4 lb = make_float4(lbp[0], lbp[1], lbp[2], lbp[3]);
+
+    if (tid < TTT_KMAX) s.te[tid] = a.token_eta ? (tid < K ? a.token_eta[tid] : 0.f) : 1.0f / (tid + 1);
+    const float* W0 = a.W0 + (a.w0_chain_stride ? chain * a.w0_chain_stride : static_cast<long long>(h) * TTT_D * TTT_D);
+    const float* b0 = a.b0 + (a.w0_chain_stride ? chain * TTT_D : static_cast<long long>(h) * TTT_D);
+
+    // this warp's tiles of a [k][f] matrix in memory <-> accumulators: tile q holds rows m0 + g
+    // (elements 0, 1) and m0 + g + 8 (elements 2, 3), columns n0 + 8q + 2t, + 1
+    auto load_acc = [&](float (&acc)[4][4], const float* src) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 u = *reinterpret_cast<const float2*>(src + (m0 + g) * TTT_D + n0 + 8 * q + 2 * t);
+            const float2 v = *reinterpret_cast<const float2*>(src + (m0 + g + 8) * TTT_D + n0 + 8 * q + 2 * t);
+            acc[q][0] = u.x; acc[q][1] = u.y; acc[q][2] = v.x; acc[q][3] = v.y;
+        }
+    };
+    auto store_acc = [&](float* dst, const float (&acc)[4][4]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            *reinterpret_cast<float2*>(dst + (m0 + g) * TTT_D + n0 + 8 * q + 2 * t) = make_float2(acc[q][0], acc[q][1]);
+            *reinterpret_cast<float2*>(dst + (m0 + g + 8) * TTT_D + n0 + 8 * q + 2 * t) = make_float2(acc[q][2], acc[q][3]);
+        }
+    };
+    auto put_acc = [&](float (*dst)[kS], const float (&acc)[4][4]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            *reinterpret_cast<float2*>(&dst[m0 + g][n0 + 8 * q + 2 * t]) = make_float2(acc[q][0], acc[q][1]);
+            *reinterpret_cast<float2*>(&dst[m0 + g + 8][n0 + 8 * q + 2 * t]) = make_float2(acc[q][2], acc[q][3]);
+        }
+    };
+    float Wacc[4][4], dWacc[4][4];
+    load_acc(Wacc, W0);
+    if (tid < TTT_D) s.b[tid] = b0[tid];
+    // a state in the workspace: each thread's sixteen accumulators (its own layout), b from tid < 64
+    auto save_state = [&](float* dst) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st4(dst + tid * 16 + 4 * q, make_float4(Wacc[q][0], Wacc[q][1], Wacc[q][2], Wacc[q][3]));
+        if (tid < TTT_D) dst[TTT_D * TTT_D + tid] = s.b[tid];
+    };
+    auto load_state = [&](const float* src) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 v = ld4(src + tid * 16 + 4 * q);
+            Wacc[q][0] = v.x; Wacc[q][1] = v.y; Wacc[q][2] = v.z; Wacc[q][3] = v.w;
+        }
+        if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
+    };
+
+    // One full mini-batch of the forward state recursion (W in Wacc and s.W, b in s.b).
+    auto fwd_step = [&](long long t0) {
+        const bool live = r < K;
+        const long long row = (t0 + r) * TTT_D + c0;
+        const float4 k4 = live ? ld4(XK + row) : f4(0.f);
+        const float4 v4 = live ? ld4(XV + row) : f4(0.f);
+        st4(&s.xk[r][c0], k4);
+        if (tid < TTT_KMAX) s.lr[tid] = tid < K ? lr[t0 + tid] : 0.f;
+        __syncthreads();
+        {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            tc_tile<TTT_D, kS, false>(c, s.xk, s.W, nt, g, t);
+            put_tile(s.P0, c, nt, g, t);
+        }
+        __syncthreads();
+        const float4 z = ld4(&s.P0[r][c0]) + ld4(&s.b[c0]);
+        float4 xh;
+        float sig;
+        row_norm(z, eps, xh, sig);
+        const float4 q = lw * (lw * xh + lb - (v4 - k4));
+        const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
+        const float4 gv = live ? (q - f4(mq) - xh * mqx) * (1.0f / sig) : f4(0.f);
+        st4(&s.g[r][c0], gv);
+        __syncthreads();
+        const float tl = s.te[K - 1];
+        tc_rank16(Wacc, s.xk, s.lr, -tl, s.g, m0, n0, g, t);
+        if (tid < TTT_D) {
+            float acc = 0.f;
+            for (int i = 0; i < K; ++i) acc = fmaf(tl * s.lr[i], s.g[i][tid], acc);
+            s.b[tid] -= acc;
+        }
+        put_acc(s.W, Wacc);  // the Z product, W's only reader, finished before the last barrier
+        __syncthreads();     // this step's reads of xk, g and lr are done
+    };
+
+    float4 dgam = f4(0.f), dbet = f4(0.f);
+
+    // The backward step of the mini-batch at t0 (as in linear_bwd_kernel), with its start state in
+    // Wacc / s.W / s.b and the adjoint after it in dWacc / s.dW / s.db.
+    auto bwd_step = [&](long long t0, int Km, bool full) {
+        const bool live = r < Km;
+        const long long row = (t0 + r) * TTT_D + c0;
+        const float4 q4 = live ? ld4(XQ + row) : f4(0.f);
+        const float4 k4 = live ? ld4(XK + row) : f4(0.f);
+        const float4 v4 = live ? ld4(XV + row) : f4(0.f);
+        const float4 o4 = live ? ld4(DO + row) : f4(0.f);
+        st4(&s.xq[r][c0], q4);
+        st4(&s.xk[r][c0], k4);
+        if (tid < TTT_KMAX) s.lr[tid] = tid < Km ? lr[t0 + tid] : 0.f;
+        __syncthreads();  // (1)
+        {  // XK W and XQ W, sharing W's fragments
+            float cz[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+            tc_tile2<false>(cz, cb, s.xk, s.xq, s.W, nt, g, t);
+            put_tile(s.P0, cz, nt, g, t);
+            put_tile(s.P1, cb, nt, g, t);
+        }
+        {  // A = XQ XK^T and M = eta * tril(A + 1) at (i, j) = (r, tid % 16)
+            const int i = r, j = tid & 15;
+            const float av = dot64(s.xq[i], s.xk[j]);
+            const float m = (j <= i && i < Km) ? s.te[i] * s.lr[j] * (av + 1.0f) : 0.f;
+            s.A[i][j] = av;
+            s.M[i][j] = m;
+            s.MT[j][i] = m;
+        }
+        __syncthreads();  // (2)
+        const float4 bb = ld4(&s.b[c0]);
+        const float4 z = ld4(&s.P0[r][c0]) + bb;
+        float4 xh;
+        float sig;
+        row_norm(z, eps, xh, sig);
+        const float4 res = lw * xh + lb - (v4 - k4);
+        const float4 q = lw * res;
+        const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
+        const float4 gv = live ? (q - f4(mq) - xh * mqx) * (1.0f / sig) : f4(0.f);
+        st4(&s.g[r][c0], gv);
+        const float4 zb0 = ld4(&s.P1[r][c0]) + bb;
+        __syncthreads();  // (3)
+        {  // M g; and the update's XK dW' and g dW'^T from the adjoint after the mini-batch
+            float cm[4] = {0.f, 0.f, 0.f, 0.f};
+            tc_tile<TTT_KMAX, kS16, false>(cm, s.M, s.g, nt, g, t);
+            put_tile(s.P0, cm, nt, g, t);
+            if (full) {
+                float cu[4] = {0.f, 0.f, 0.f, 0.f}, cv[4] = {0.f, 0.f, 0.f, 0.f};
+                tc_tile<TTT_D, kS, false>(cu, s.xk, s.dW, nt, g, t);
+                tc_tile<TTT_D, kS, true>(cv, s.g, s.dW, nt, g, t);
+                put_tile(s.P1, cu, nt, g, t);
+                put_tile(s.P2, cv, nt, g, t);
+            }
+        }
+        __syncthreads();  // (4)
+        const float4 zb = zb0 - ld4(&s.P0[r][c0]);
+        float4 xhb;
+        float sigb;
+        row_norm(zb, eps, xhb, sigb);
+        const float4 p = lw * o4;
+        const float mp = row_sum(hsum4(p)) * (1.0f / TTT_D), mpx = row_sum(hsum4(p * xhb)) * (1.0f / TTT_D);
+        st4(&s.dzb[r][c0], (p - f4(mp) - xhb * mpx) * (1.0f / sigb));
+        dgam = dgam + o4 * xhb;
+        dbet = dbet + o4;
+        const float4 U = full ? ld4(&s.P1[r][c0]) + ld4(&s.db[c0]) : f4(0.f);
+        const float4 V = full ? ld4(&s.P2[r][c0]) : f4(0.f);
+        __syncthreads();  // (5)
+        {  // M^T dZbar
+            float cg[4] = {0.f, 0.f, 0.f, 0.f};
+            tc_tile<TTT_KMAX, kS16, false>(cg, s.MT, s.dzb, nt, g, t);
+            put_tile(s.P0, cg, nt, g, t);
+        }
+        {  // dM = -dZbar g^T on the lower triangle: its shares of dA and of dlr
+            const int i = r, j = tid & 15;
+            const float dm = (j <= i && i < Km) ? -dot64(s.dzb[i], s.g[j]) : 0.f;
+            s.dlr_eta[i][j] = s.te[i] * (s.A[i][j] + 1.0f) * dm;
+            const float da = dm * s.te[i] * s.lr[j];
+            s.dA[i][j] = da;
+            s.dAT[j][i] = da;
+        }
+        __syncthreads();  // (6)
+        float4 dg = f4(0.f) - ld4(&s.P0[r][c0]);
+        float4 dxk = f4(0.f);
+        float dlr_upd = 0.f;
+        if (full) {
+            const float tl = s.te[K - 1], e = tl * s.lr[r];
+            dg = dg - U * e;
+            dlr_upd = -tl * row_sum(hsum4(gv * U));
+            dxk = f4(0.f) - V * e;
+        }
+        if ((tid & 15) == 0) s.dlr_row[r] = dlr_upd;
+        {  // the vector-Jacobian product of g = ln_fused_l2_bwd(Z, tau) with dg
+            const float rs = 1.0f / sig;
+            const float mu = row_sum(hsum4(dg)) * (1.0f / TTT_D), mux = row_sum(hsum4(dg * xh)) * (1.0f / TTT_D);
+            const float4 wq = (dg - f4(mu) - xh * mux) * rs;
+            const float4 hx = lw * lw * wq - (dg * mqx + q * mux) * rs;
+            const float ds = -row_sum(hsum4(dg * gv)) * rs;
+            const float mh = row_sum(hsum4(hx)) * (1.0f / TTT_D), mhx = row_sum(hsum4(hx * xh)) * (1.0f / TTT_D);
+            const float4 dz = (hx - f4(mh) - xh * mhx) * rs + xh * (ds * (1.0f / TTT_D));
+            dgam = dgam + wq * (res + lw * xh);
+            dbet = dbet + wq * lw;
+            const float4 dtau = f4(0.f) - wq * lw;
+            dxk = dxk - dtau;
+            if (live) st4(dXV + row, dtau);
+            st4(&s.dz[r][c0], live ? dz : f4(0.f));
+        }
+        __syncthreads();  // (7)
+        {  // dZbar W^T + dA XK and dZ W^T + dA^T XQ; the adjoint of the start state
+            float cq[4] = {0.f, 0.f, 0.f, 0.f}, ck[4] = {0.f, 0.f, 0.f, 0.f};
+            tc_tile2<true>(cq, ck, s.dzb, s.dz, s.W, nt, g, t);
+            tc_tile<TTT_KMAX, kS16, false>(cq, s.dA, s.xk, nt, g, t);
+            tc_tile<TTT_KMAX, kS16, false>(ck, s.dAT, s.xq, nt, g, t);
+            put_tile(s.P0, cq, nt, g, t);
+            put_tile(s.P1, ck, nt, g, t);
+            tc_rank16(dWacc, s.xq, nullptr, 1.f, s.dzb, m0, n0, g, t);
+            tc_rank16(dWacc, s.xk, nullptr, 1.f, s.dz, m0, n0, g, t);
+        }
+        __syncthreads();  // (8)
+        if (live) {
+            st4(dXQ + row, o4 + ld4(&s.P0[r][c0]));
+            st4(dXK + row, dxk + ld4(&s.P1[r][c0]));
+        }
+        if (tid < Km) {
+            float acc = s.dlr_row[tid];
+            for (int i = 0; i < TTT_KMAX; ++i) acc += s.dlr_eta[i][tid];
+            dlr[t0 + tid] = acc;
+        }
+        if (tid < TTT_D) {
+            float acc = 0.f;
+            for (int i = 0; i < Km; ++i) acc += s.dzb[i][tid] + s.dz[i][tid];
+            s.db[tid] += acc;
+        }
+        put_acc(s.dW, dWacc);  // s.dW's readers (the update's products) finished before barrier (4)
+    };
+
+    // ---- phase 1: the forward state recursion, a checkpoint every G full mini-batches --------
+    put_acc(s.W, Wacc);
+    __syncthreads();
+    for (long long m = 0; m < a.n_full; ++m) {
+        if (m % G == 0) save_state(a.ckpt + (chain * a.n_ckpt + m / G) * kState);
+        fwd_step(m * K);
+    }
+
+    // ---- the remainder tail, from the state after the full mini-batches -----------------------
+    if (a.dW_last) {
+        load_acc(dWacc, a.dW_last + chain * TTT_D * TTT_D);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dWacc[q][0] = dWacc[q][1] = dWacc[q][2] = dWacc[q][3] = 0.f;
+    }
+    if (tid < TTT_D) s.db[tid] = a.db_last ? a.db_last[chain * TTT_D + tid] : 0.f;
+    put_acc(s.dW, dWacc);
+    if (a.rem > 0) {
+        __syncthreads();
+        bwd_step(a.n_full * K, static_cast<int>(a.rem), false);
+    }
+
+    // ---- phase 2: the groups from the last; rebuild each one's states, then step back ----------
+    float* const slab = a.slab + chain * G * kState;
+    for (long long c = a.n_ckpt - 1; c >= 0; --c) {
+        const long long m0g = c * G, m1g = m0g + G < a.n_full ? m0g + G : a.n_full;
+        __syncthreads();
+        load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
+        put_acc(s.W, Wacc);
+        __syncthreads();
+        for (long long m = m0g; m < m1g; ++m) {
+            save_state(slab + (m - m0g) * kState);
+            if (m + 1 < m1g) fwd_step(m * K);
+        }
+        for (long long m = m1g - 1; m >= m0g; --m) {
+            __syncthreads();
+            load_state(slab + (m - m0g) * kState);
+            put_acc(s.W, Wacc);
+            __syncthreads();
+            bwd_step(m * K, K, true);
+        }
+    }
+
+    // ---- this chain's shares of the shared parameters' gradients -----------------------------
+    float* part = a.part + chain * kPart;
+    store_acc(part, dWacc);
+    __syncthreads();
+    st4(&s.g[r][c0], dgam);
+    st4(&s.dzb[r][c0], dbet);
+    __syncthreads();
+    if (tid < TTT_D) {
+        float sg = 0.f, sb = 0.f;
+        for (int i = 0; i < TTT_KMAX; ++i) {
+            sg += s.g[i][tid];
+            sb += s.dzb[i][tid];
+        }
+        part[TTT_D * TTT_D + tid] = s.db[tid];
+        part[TTT_D * TTT_D + TTT_D + tid] = sg;
+        part[TTT_D * TTT_D + 2 * TTT_D + tid] = sb;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_linear_bwd(const LinearBwdArgs& a, int dtype, cudaStream_t st) {
-    const size_t smem = sizeof(BwdSmem);
-    auto kernel = dtype == 0 ? linear_bwd_kernel<float> : linear_bwd_kernel<__nv_bfloat16>;
+    // fp32 activations: the FFMA kernel (float32 products); bf16: the tensor-core kernel
+    const size_t smem = dtype == 0 ? sizeof(BwdSmem) : sizeof(BwdTcSmem);
+    auto kernel = dtype == 0 ? linear_bwd_kernel<float> : linear_bwd_tc_kernel<__nv_bfloat16>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(a.B * a.H), kT, smem, st>>>(a);
