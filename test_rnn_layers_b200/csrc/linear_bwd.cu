@@ -67,11 +67,6 @@ struct __align__(16) BwdSmem {
 };
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ float4 ld4(const __nv_bfloat16* p) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
-    return make_float4(a.x, a.y, b.x, b.y);
-}
 __device__ __forceinline__ void st4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 __device__ __forceinline__ void st4(__nv_bfloat16* p, float4 v) {
     *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
@@ -488,7 +483,22 @@ struct __align__(16) BwdTcSmem {
     float lr[TTT_KMAX];
     float te[TTT_KMAX];
     float dlr_row[TTT_KMAX];
+    // the next step's inputs, copied in while the current step runs: [buffer][XQ, XK, XV, d_out]
+    __nv_bfloat16 stage[2][4][TTT_KMAX][TTT_D];
+    float stage_lr[2][TTT_KMAX];
 };
+
+// 16- and 4-byte cp.async with zero fill: src_bytes = size copies, 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async_16z(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_4z(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t tf32(float x) {
     uint32_t r;
@@ -645,14 +655,48 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
     };
 
-    // One full mini-batch of the forward state recursion (W in Wacc and s.W, b in s.b).
-    auto fwd_step = [&](long long t0) {
+    // The inputs of the step at t0 (Km tokens) into staging buffer buf, asynchronously: XK and XV
+    // (a forward step) or XQ, XK, XV and d_out (a backward step), rows past Km zero, and lr.
+    auto prefetch = [&](int buf, long long t0, int Km, bool bwd) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int cidx = tid + i * kT, ti = cidx >> 7;
+            if (!bwd && (ti == 0 || ti == 3)) continue;
+            const int rowc = (cidx & 127) >> 3, part = cidx & 7;
+            const bool in = rowc < Km;
+            const T* src = ti == 0 ? XQ : ti == 1 ? XK : ti == 2 ? XV : DO;
+            cp_async_16z(&s.stage[buf][ti][rowc][part * 8], in ? src + (t0 + rowc) * TTT_D + part * 8 : src,
+                         in ? 16u : 0u);
+        }
+        if (tid < TTT_KMAX) cp_async_4z(&s.stage_lr[buf][tid], tid < Km ? lr + t0 + tid : lr, tid < Km ? 4u : 0u);
+        cp_async_commit();
+    };
+    auto staged = [&](int buf, int ti) {
+        const uint2 u = *reinterpret_cast<const uint2*>(&s.stage[buf][ti][r][c0]);
+        const float2 lo = unpack_bf16x2(u.x), hi = unpack_bf16x2(u.y);
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+    };
+    // What a step prefetches for its successor: nothing (kind 0), a forward step (1) or a
+    // backward step (2) at token t0 with Km tokens.
+    struct Next {
+        int kind;
+        long long t0;
+        int Km;
+    };
+    auto start_next = [&](int buf, const Next& nx) {
+        if (nx.kind) prefetch(buf ^ 1, nx.t0, nx.Km, nx.kind == 2);
+    };
+
+    // One full mini-batch of the forward state recursion (W in Wacc and s.W, b in s.b), its inputs
+    // in staging buffer buf.
+    auto fwd_step = [&](long long t0, int buf, const Next& nx) {
         const bool live = r < K;
-        const long long row = (t0 + r) * TTT_D + c0;
-        const float4 k4 = live ? ld4(XK + row) : f4(0.f);
-        const float4 v4 = live ? ld4(XV + row) : f4(0.f);
+        cp_async_wait_all();
+        __syncthreads();  // the staged inputs have landed, and the last step's readers of the tiles are done
+        const float4 k4 = staged(buf, 1), v4 = staged(buf, 2);
         st4(&s.xk[r][c0], k4);
-        if (tid < TTT_KMAX) s.lr[tid] = tid < K ? lr[t0 + tid] : 0.f;
+        if (tid < TTT_KMAX) s.lr[tid] = s.stage_lr[buf][tid];
+        start_next(buf, nx);
         __syncthreads();
         {
             float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -683,17 +727,17 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     float4 dgam = f4(0.f), dbet = f4(0.f);
 
     // The backward step of the mini-batch at t0 (as in linear_bwd_kernel), with its start state in
-    // Wacc / s.W / s.b and the adjoint after it in dWacc / s.dW / s.db.
-    auto bwd_step = [&](long long t0, int Km, bool full) {
+    // Wacc / s.W / s.b, the adjoint after it in dWacc / s.dW / s.db, its inputs in staging buffer buf.
+    auto bwd_step = [&](long long t0, int Km, bool full, int buf, const Next& nx) {
         const bool live = r < Km;
         const long long row = (t0 + r) * TTT_D + c0;
-        const float4 q4 = live ? ld4(XQ + row) : f4(0.f);
-        const float4 k4 = live ? ld4(XK + row) : f4(0.f);
-        const float4 v4 = live ? ld4(XV + row) : f4(0.f);
-        const float4 o4 = live ? ld4(DO + row) : f4(0.f);
+        cp_async_wait_all();
+        __syncthreads();  // (0) the staged inputs have landed
+        const float4 q4 = staged(buf, 0), k4 = staged(buf, 1), v4 = staged(buf, 2), o4 = staged(buf, 3);
         st4(&s.xq[r][c0], q4);
         st4(&s.xk[r][c0], k4);
-        if (tid < TTT_KMAX) s.lr[tid] = tid < Km ? lr[t0 + tid] : 0.f;
+        if (tid < TTT_KMAX) s.lr[tid] = s.stage_lr[buf][tid];
+        start_next(buf, nx);
         __syncthreads();  // (1)
         {  // XK W and XQ W, sharing W's fragments
             float cz[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
@@ -815,12 +859,25 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         put_acc(s.dW, dWacc);  // s.dW's readers (the update's products) finished before barrier (4)
     };
 
+    // ---- the order of the steps, for the prefetch of each one's successor ----------------------
+    const long long n_full = a.n_full;
+    const int rem = static_cast<int>(a.rem);
+    auto group_first = [&](long long c) -> Next {  // the first step of group c in phase 2
+        const long long m0g = c * G, m1g = m0g + G < n_full ? m0g + G : n_full;
+        return m1g - m0g > 1 ? Next{1, m0g * K, K} : Next{2, m0g * K, K};
+    };
+    const Next after_tail = a.n_ckpt > 0 ? group_first(a.n_ckpt - 1) : Next{0, 0, 0};
+    const Next after_phase1 = rem > 0 ? Next{2, n_full * K, rem} : after_tail;
+    int buf = 0;
+
     // ---- phase 1: the forward state recursion, a checkpoint every G full mini-batches --------
     put_acc(s.W, Wacc);
-    __syncthreads();
-    for (long long m = 0; m < a.n_full; ++m) {
+    if (n_full > 0) prefetch(0, 0, K, false);
+    else if (after_phase1.kind) prefetch(0, after_phase1.t0, after_phase1.Km, after_phase1.kind == 2);
+    for (long long m = 0; m < n_full; ++m) {
         if (m % G == 0) save_state(a.ckpt + (chain * a.n_ckpt + m / G) * kState);
-        fwd_step(m * K);
+        fwd_step(m * K, buf, m + 1 < n_full ? Next{1, (m + 1) * K, K} : after_phase1);
+        buf ^= 1;
     }
 
     // ---- the remainder tail, from the state after the full mini-batches -----------------------
@@ -832,29 +889,31 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     }
     if (tid < TTT_D) s.db[tid] = a.db_last ? a.db_last[chain * TTT_D + tid] : 0.f;
     put_acc(s.dW, dWacc);
-    if (a.rem > 0) {
-        __syncthreads();
-        bwd_step(a.n_full * K, static_cast<int>(a.rem), false);
+    if (rem > 0) {
+        bwd_step(n_full * K, rem, false, buf, after_tail);
+        buf ^= 1;
     }
 
     // ---- phase 2: the groups from the last; rebuild each one's states, then step back ----------
     float* const slab = a.slab + chain * G * kState;
     for (long long c = a.n_ckpt - 1; c >= 0; --c) {
-        const long long m0g = c * G, m1g = m0g + G < a.n_full ? m0g + G : a.n_full;
+        const long long m0g = c * G, m1g = m0g + G < n_full ? m0g + G : n_full;
         __syncthreads();
         load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
         put_acc(s.W, Wacc);
-        __syncthreads();
         for (long long m = m0g; m < m1g; ++m) {
             save_state(slab + (m - m0g) * kState);
-            if (m + 1 < m1g) fwd_step(m * K);
+            if (m + 1 < m1g) {
+                fwd_step(m * K, buf, m + 2 < m1g ? Next{1, (m + 1) * K, K} : Next{2, (m1g - 1) * K, K});
+                buf ^= 1;
+            }
         }
         for (long long m = m1g - 1; m >= m0g; --m) {
             __syncthreads();
             load_state(slab + (m - m0g) * kState);
             put_acc(s.W, Wacc);
-            __syncthreads();
-            bwd_step(m * K, K, true);
+            bwd_step(m * K, K, true, buf, m > m0g ? Next{2, (m - 1) * K, K} : (c > 0 ? group_first(c - 1) : Next{0, 0, 0}));
+            buf ^= 1;
         }
     }
 
