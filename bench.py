@@ -99,8 +99,6 @@ def linear_bwd_flops(B, H, L, K=16):
     return B * H * n_mb * (6 * 2 * K * D * D + 4 * 2 * D * K * (K + 1) // 2)
 
 
-# FP32 FMA issue peak from the unit counts: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (max clock)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # dense TF32 tensor peak as the nominal ratio to bf16 (1.1 / 2.25 PFLOP/s) times the bf16 peak in use
 TF32_PER_BF16 = 1.1 / 2.25
 
