@@ -490,7 +490,10 @@ def bench_linear_backward(args, world, peaks, G=16):
     16): the gradients of XQ, XK, XV, lr, W0, b0, ln_w and ln_b from d_out, dW_last and db_last,
     the inputs and upstream gradients resident in HBM (each larger than L2).  bf16 activations run
     the tensor-core kernel (TF32 products), whose roofline is the larger of the HBM time of its
-    algorithmic bytes and the TF32 time of its algorithmic FLOPs: the HBM one."""
+    algorithmic bytes and the TF32 time of its algorithmic FLOPs: the HBM one.  Under torchrun
+    each rank runs its own batch (weak scaling) and the step ends with the one exchange data-
+    parallel training needs: the all-reduce of the shared-parameter gradients (dW0, db0, d ln_w,
+    d ln_b), NCCL."""
     import torch
 
     import test_rnn_layers_b200 as ttt
@@ -503,9 +506,13 @@ def bench_linear_backward(args, world, peaks, G=16):
     del x, up
     ws = torch.empty(ttt.ttt_linear_backward_workspace_bytes(w.B, w.H, w.L, w.K, G), dtype=torch.uint8, device="cuda")
 
+    from test_rnn_layers_b200.shard import allreduce_shared_grads
+
     def step():
-        ttt.ttt_linear_backward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], dout, dWl, dbl,
-                                mini_batch=w.K, eps=w.eps, ckpt_group=G, workspace=ws)
+        g = ttt.ttt_linear_backward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], dout, dWl, dbl,
+                                    mini_batch=w.K, eps=w.eps, ckpt_group=G, workspace=ws)
+        if world > 1:
+            allreduce_shared_grads(g)
 
     K = max(3, min(args.steps, 10))
     ms = time_steps(step, K, 3, world)
@@ -517,6 +524,8 @@ def bench_linear_backward(args, world, peaks, G=16):
     return {"workload": f"ttt_linear_backward_1b_layer_B{w.B}_H{w.H}_L{w.L}_ckpt{G}",
             "value": round(world * w.B * w.L / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "steps": K, "gpu_launches": 2 * K, "dtype": "bf16 in/out, tf32 products, f32 accumulation and state",
+            "collective": (f"all_reduce (sum, NCCL) of the shared-parameter gradients, {(w.H * (D * D + 3 * D)) * 4} "
+                           "bytes per step" if world > 1 else "none (one GPU)"),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "peak_source": f"{which} hbm_gbs",
                          "unit": "GB/s", "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
                          "floor_ms": round(nbytes / hbm / 1e6, 4), "algorithmic_flops": flops,

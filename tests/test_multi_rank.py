@@ -85,3 +85,66 @@ def test_two_gloo_ranks_shard_and_reduce():
                                             x["ln_b"], w.K, w.eps)
     assert np.array_equal(np.concatenate([o for _, _, _, o, _ in res]), whole["out"])
     assert np.array_equal(np.concatenate([W for _, _, _, _, W in res]), whole["W_last"])
+
+
+def _bwd_worker(rank, world, port, q):
+    """One rank of data-parallel training: the backward oracle on this rank's batch shard, the
+    shard's per-head sums of the shared-parameter gradients, then their all-reduce."""
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from oracle import ttt_backward
+    from test_rnn_layers_b200.shard import allreduce_shared_grads, batch_shard
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.workload(1, B=3, H=2, L=19, K=4, dtype="f32", seed=0xD158)
+        s, e = batch_shard(w.B, world, rank)
+        chains = [b * w.H + h for b in range(s, e) for h in range(w.H)]
+        x, up = synth.linear_inputs(w, chains=chains), synth.upstream_grads(w, chains=chains)
+        st = lambda a: np.stack([a[c % w.H] for c in chains])
+        r = ttt_backward.linear_backward(x["XQ"], x["XK"], x["XV"], x["lr"], st(x["W0"]), st(x["b0"]), st(x["ln_w"]),
+                                         st(x["ln_b"]), w.K, w.eps, up["d_out"], up["dW_last"], up["db_last"])
+        grads = {}
+        for n in ("dW0", "db0", "dln_w", "dln_b"):
+            acc = torch.zeros((w.H,) + r[n].shape[1:], dtype=torch.float64)
+            for i, c in enumerate(chains):
+                acc[c % w.H] += torch.from_numpy(r[n][i])
+            grads[n] = acc
+        allreduce_shared_grads(grads)
+        q.put((rank, chains, r["dXQ"], r["dlr"], {n: grads[n].numpy() for n in grads}))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_data_parallel_backward():
+    """Sharded backward + the all-reduce of the shared-parameter gradients = the whole batch's."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bwd_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort(key=lambda t: t[0])
+    import synth
+    from oracle import ttt_backward
+    w = synth.workload(1, B=3, H=2, L=19, K=4, dtype="f32", seed=0xD158)
+    ids = list(range(w.chains))
+    x, up = synth.linear_inputs(w, chains=ids), synth.upstream_grads(w, chains=ids)
+    st = lambda a: np.stack([a[c % w.H] for c in ids])
+    whole = ttt_backward.linear_backward(x["XQ"], x["XK"], x["XV"], x["lr"], st(x["W0"]), st(x["b0"]), st(x["ln_w"]),
+                                         st(x["ln_b"]), w.K, w.eps, up["d_out"], up["dW_last"], up["db_last"])
+    assert sum((c for _, c, _, _, _ in res), []) == ids
+    assert np.array_equal(np.concatenate([d for _, _, d, _, _ in res]), whole["dXQ"])
+    assert np.array_equal(np.concatenate([d for _, _, _, d, _ in res]), whole["dlr"])
+    for n in ("dW0", "db0", "dln_w", "dln_b"):
+        ref = whole[n].reshape(w.B, w.H, *whole[n].shape[1:]).sum(axis=0)
+        for _, _, _, _, g in res:  # every rank holds the same, whole-batch sums
+            np.testing.assert_allclose(g[n], ref, rtol=1e-12, atol=1e-12)
