@@ -516,6 +516,19 @@ def bench_linear_backward(args, world, peaks, G=16):
 
     K = max(3, min(args.steps, 10))
     ms = time_steps(step, K, 3, world)
+    # the same with every state kept (checkpoint group 1: 2.2 GB of workspace, no rebuild)
+    del ws
+    ws = torch.empty(ttt.ttt_linear_backward_workspace_bytes(w.B, w.H, w.L, w.K, 1), dtype=torch.uint8, device="cuda")
+
+    def step_all_states():
+        g = ttt.ttt_linear_backward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], dout, dWl, dbl,
+                                    mini_batch=w.K, eps=w.eps, ckpt_group=1, workspace=ws)
+        if world > 1:
+            allreduce_shared_grads(g)
+
+    ms_all = time_steps(step_all_states, K, 3, world)
+    ws_all = ws.numel()
+    del ws
     flops, nbytes = linear_bwd_flops(w.B, w.H, w.L), linear_bwd_bytes(w.B, w.H, w.L)
     tfl = flops / (ms / 1e3) / 1e12
     gbs = nbytes / (ms / 1e3) / 1e9
@@ -526,6 +539,8 @@ def bench_linear_backward(args, world, peaks, G=16):
             "steps": K, "gpu_launches": 2 * K, "dtype": "bf16 in/out, tf32 products, f32 accumulation and state",
             "collective": (f"all_reduce (sum, NCCL) of the shared-parameter gradients, {(w.H * (D * D + 3 * D)) * 4} "
                            "bytes per step" if world > 1 else "none (one GPU)"),
+            "every_state_kept": {"ckpt_group": 1, "ms_per_step": round(ms_all, 4),
+                                 "value": round(world * w.B * w.L / (ms_all / 1e3), 1), "workspace_bytes": ws_all},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "peak_source": f"{which} hbm_gbs",
                          "unit": "GB/s", "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
                          "floor_ms": round(nbytes / hbm / 1e6, 4), "algorithmic_flops": flops,

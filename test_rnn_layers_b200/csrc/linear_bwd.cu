@@ -106,18 +106,19 @@ __device__ __forceinline__ float4 row_times(const float* x, const float (*Y)[kSt
     return acc;
 }
 
-// sum_f p[f] q[f] over 64 features (rows of stride kS).
+// sum_f p[f] q[f] over 64 features (rows of stride kS), in two interleaved partial sums (half
+// the dependent FMA chain).
 __device__ __forceinline__ float dot64(const float* p, const float* q) {
-    float acc = 0.f;
-#pragma unroll
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
     for (int f = 0; f < TTT_D; f += 4) {
         const float4 a = ld4(p + f), b = ld4(q + f);
-        acc = fmaf(a.x, b.x, acc);
-        acc = fmaf(a.y, b.y, acc);
-        acc = fmaf(a.z, b.z, acc);
-        acc = fmaf(a.w, b.w, acc);
+        a0 = fmaf(a.x, b.x, a0);
+        a1 = fmaf(a.y, b.y, a1);
+        a0 = fmaf(a.z, b.z, a0);
+        a1 = fmaf(a.w, b.w, a1);
     }
-    return acc;
+    return a0 + a1;
 }
 
 // LayerNorm statistics of a row whose four features z this thread holds: x_hat and sigma.
@@ -126,7 +127,7 @@ __device__ __forceinline__ void row_norm(float4 z, float eps, float4& xh, float&
     const float4 c = z - f4(mu);
     const float v = row_sum(hsum4(c * c)) * (1.0f / TTT_D);
     sigma = sqrtf(v + eps);
-    xh = make_float4(c.x / sigma, c.y / sigma, c.z / sigma, c.w / sigma);
+    xh = c * (1.0f / sigma);
 }
 
 template <typename T>
