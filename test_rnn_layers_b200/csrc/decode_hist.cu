@@ -27,7 +27,7 @@ constexpr int kThreads = 256;           // 16 column groups of 4 x 16 row groups
 constexpr int kRowGroups = kThreads / 16;
 constexpr int kBufs = 2;
 constexpr int kRow = 2 * TTT_D;         // floats per history row: a_j then g_j
-constexpr int kCtasPerSm = 3;           // 3 x ~60 KB of shared memory, 80 registers: more chains in flight
+constexpr int kCtasPerSm = 4;           // 4 x ~55 KB of shared memory, 64 registers: more chains in flight
 
 template <typename T>
 struct __align__(16) HistSmem {
@@ -37,7 +37,7 @@ struct __align__(16) HistSmem {
     float gb[kBufs][TTT_D];
     T x[kBufs][3][TTT_D];                 // xq, xk, xv
     float lr[kBufs][4];
-    float4 part[2][kRowGroups][TTT_D / 4];  // partial xk W, xq W
+    float4 part[2][kRowGroups / 2][TTT_D / 4];  // partial xk W, xq W of each warp (two row groups)
     float sz[TTT_D], sqw[TTT_D], sg[TTT_D];
     float scr[TTT_D];                     // sum_{j<p} (xq . a_j) g_j
     float c[TTT_KMAX];                    // xq . a_j
@@ -108,8 +108,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_hist_kernel(Decod
             pq.x = fmaf(xq, w[k].x, pq.x); pq.y = fmaf(xq, w[k].y, pq.y);
             pq.z = fmaf(xq, w[k].z, pq.z); pq.w = fmaf(xq, w[k].w, pq.w);
         }
-        s.part[0][rg][cg] = pk;
-        s.part[1][rg][cg] = pq;
+        // the warp's two row groups (lanes l and l + 16 share columns) summed before the exchange
+        pk.x += __shfl_xor_sync(0xffffffffu, pk.x, 16); pk.y += __shfl_xor_sync(0xffffffffu, pk.y, 16);
+        pk.z += __shfl_xor_sync(0xffffffffu, pk.z, 16); pk.w += __shfl_xor_sync(0xffffffffu, pk.w, 16);
+        pq.x += __shfl_xor_sync(0xffffffffu, pq.x, 16); pq.y += __shfl_xor_sync(0xffffffffu, pq.y, 16);
+        pq.z += __shfl_xor_sync(0xffffffffu, pq.z, 16); pq.w += __shfl_xor_sync(0xffffffffu, pq.w, 16);
+        if (lane < 16) {
+            s.part[0][warp][cg] = pk;
+            s.part[1][warp][cg] = pq;
+        }
         {
             const float xq0 = to_f32(s.x[bi][0][lane]), xq1 = to_f32(s.x[bi][0][lane + 32]);
             for (int j = warp; j < p; j += kThreads / 32) {
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_hist_kernel(Decod
             const float* pp = reinterpret_cast<const float*>(&s.part[which][0][0]);
             float acc = 0.f;
 #pragma unroll
-            for (int r = 0; r < kRowGroups; ++r) acc += pp[r * TTT_D + col];
+            for (int r = 0; r < kRowGroups / 2; ++r) acc += pp[r * TTT_D + col];
             if (which == 0) s.sz[col] = acc + s.b[bi][col];
             else s.sqw[col] = acc;
         }
