@@ -18,19 +18,24 @@
 // The remainder tail (K = r) has no update: its terms in dW', db' and e are absent, and it
 // starts from the state after the full mini-batches, whose adjoint is the caller's dW_last.
 //
-// Design (one CTA of 256 threads per chain, fp32 throughout):
+// Design (one CTA of 256 threads per chain; two kernels that share this structure):
 //  * Phase 1 runs the forward state recursion over the full mini-batches from (W0, b0) and
 //    writes every G-th state to the workspace.  Phase 2 walks the groups from the last: it
 //    rebuilds the group's states from its checkpoint into a per-chain slab, then runs the
 //    backward step for each mini-batch of the group in reverse.  Both phases run the same
 //    forward-step code, so a rebuilt state has the bits of the first.
-//  * Tiles of 16 rows x 64 features: thread (r, c0) = (tid / 16, 4 (tid % 16)) owns four
-//    consecutive features of one row, so a row's LayerNorm sums are half-warp shuffles, and
-//    every product against a 64-wide matrix is one row of shared memory times that matrix,
-//    read as float4 rows (rows padded to 68 floats).  The state and its adjoint are kept in
-//    shared memory both as [k][f] and transposed, so that XW and XW^T products read alike;
-//    each thread owns a 4 x 4 block of them in registers and republishes it after an update.
-//  * The LayerNorm statistics are two-pass (mean, then the centred sum of squares).
+//  * The LayerNorm work uses a row layout: thread (r, c0) = (tid / 16, 4 (tid % 16)) owns four
+//    consecutive features of one row of a 16 x 64 tile, so a row's sums are half-warp shuffles
+//    (two-pass statistics).  The 16 x 16 products XQ XK^T and dZbar g^T are per-thread dot
+//    products.
+//  * linear_bwd_tc_kernel (bf16 activations): the 16 x 64 x 64 products and the rank-16 state
+//    updates are TF32 warp MMAs (m16n8k8, fp32 accumulation) with the state and its adjoint held
+//    as accumulators and published to shared memory as B operands; each step's input tiles are
+//    copied in one step ahead by cp.async.
+//  * linear_bwd_kernel (fp32 activations): every product is one row of a tile times a 64-wide
+//    matrix read as float4 rows, fp32 throughout; the state and its adjoint live in shared
+//    memory as [k][f] and transposed, each thread owning a 4 x 4 block of both in registers.
+//  * No waits: nothing in either kernel can hang.
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
 
