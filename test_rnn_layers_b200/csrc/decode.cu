@@ -22,6 +22,7 @@ namespace {
 
 constexpr int kThreads = 256;           // 16 column groups of 4 x 16 row groups of 4
 constexpr int kRowGroups = kThreads / 16;
+constexpr int kCtasPerSm = 3;  // 3 x ~71 KB of shared memory, 80 registers
 constexpr int kBufs = 2;
 
 template <typename T>
@@ -32,7 +33,7 @@ struct __align__(16) DecSmem {
     float gb[kBufs][TTT_D];
     T x[kBufs][3][TTT_D];                 // xq, xk, xv
     float lr[kBufs][4];
-    float4 part[3][kRowGroups][TTT_D / 4];  // partial xk W, xq W, xq W_grad
+    float4 part[3][kRowGroups / 2][TTT_D / 4];  // partial xk W, xq W, xq W_grad of each warp (two row groups)
     float sz[TTT_D], sqw[TTT_D], sqg[TTT_D], sg[TTT_D];
     float sqk;
     uint64_t full[kBufs];
@@ -55,7 +56,7 @@ __device__ __forceinline__ void issue_chain(DecSmem<T>& s, const DecodeArgs& a, 
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     DecSmem<T>& s = *reinterpret_cast<DecSmem<T>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -101,9 +102,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
             pg.x = fmaf(xq, G[k].x, pg.x); pg.y = fmaf(xq, G[k].y, pg.y);
             pg.z = fmaf(xq, G[k].z, pg.z); pg.w = fmaf(xq, G[k].w, pg.w);
         }
-        s.part[0][rg][cg] = pk;
-        s.part[1][rg][cg] = pq;
-        s.part[2][rg][cg] = pg;
+        // the warp's two row groups (lanes l and l + 16 share columns) summed before the exchange
+#pragma unroll
+        for (int o = 0; o < 3; ++o) {
+            float4& v = o == 0 ? pk : o == 1 ? pq : pg;
+            v.x += __shfl_xor_sync(0xffffffffu, v.x, 16);
+            v.y += __shfl_xor_sync(0xffffffffu, v.y, 16);
+            v.z += __shfl_xor_sync(0xffffffffu, v.z, 16);
+            v.w += __shfl_xor_sync(0xffffffffu, v.w, 16);
+        }
+        if (lane < 16) {
+            s.part[0][warp][cg] = pk;
+            s.part[1][warp][cg] = pq;
+            s.part[2][warp][cg] = pg;
+        }
         __syncthreads();
         if (s.fail) break;
 
@@ -114,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
             const float* pp = reinterpret_cast<const float*>(&s.part[which][0][0]);
             float acc = 0.f;
 #pragma unroll
-            for (int r = 0; r < kRowGroups; ++r) acc += pp[r * TTT_D + col];
+            for (int r = 0; r < kRowGroups / 2; ++r) acc += pp[r * TTT_D + col];
             if (which == 0) s.sz[col] = acc + s.b[bi][col];
             else if (which == 1) s.sqw[col] = acc;
             else s.sqg[col] = acc;
@@ -215,7 +227,8 @@ cudaError_t launch_decode(const DecodeArgs& a, int dtype, cudaStream_t st) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long chains = static_cast<long long>(a.B) * a.H;
-    const unsigned grid = static_cast<unsigned>(chains < 2ll * sms ? chains : 2ll * sms);
+    const unsigned grid = static_cast<unsigned>(chains < kCtasPerSm * static_cast<long long>(sms)
+                                                    ? chains : kCtasPerSm * static_cast<long long>(sms));
     cudaError_t e;
     if (dtype == 0) {
         const size_t smem = sizeof(DecSmem<float>);
