@@ -726,8 +726,9 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             for (int i = 0; i < K; ++i) acc = fmaf(tl * s.lr[i], s.g[i][tid], acc);
             s.b[tid] -= acc;
         }
-        put_acc(s.W, Wacc);  // the Z product, W's only reader, finished before the last barrier
-        __syncthreads();     // this step's reads of xk, g and lr are done
+        // the Z product, W's only reader, finished before the last barrier; each thread writes its own
+        // elements, and the next step rewrites xk, g and lr only after its first barrier
+        put_acc(s.W, Wacc);
     };
 
     float4 dgam = f4(0.f), dbet = f4(0.f);
@@ -904,7 +905,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     float* const slab = a.slab + chain * G * kState;
     for (long long c = a.n_ckpt - 1; c >= 0; --c) {
         const long long m0g = c * G, m1g = m0g + G < n_full ? m0g + G : n_full;
-        __syncthreads();
+        // no barrier: s.b's readers and s.W's readers of the last step passed its later barriers,
+        // and each thread rewrites only its own elements
         load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
         put_acc(s.W, Wacc);
         for (long long m = m0g; m < m1g; ++m) {
@@ -915,8 +917,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             }
         }
         for (long long m = m1g - 1; m >= m0g; --m) {
-            __syncthreads();
-            load_state(slab + (m - m0g) * kState);
+            load_state(slab + (m - m0g) * kState);  // (no barrier, as above)
             put_acc(s.W, Wacc);
             bwd_step(m * K, K, true, buf, m > m0g ? Next{2, (m - 1) * K, K} : (c > 0 ? group_first(c - 1) : Next{0, 0, 0}));
             buf ^= 1;
