@@ -126,6 +126,26 @@ __device__ __forceinline__ float dot64(const float* p, const float* q) {
     return a0 + a1;
 }
 
+// dot64 of two bf16 rows (16-byte aligned), in the same order of accumulation.
+__device__ __forceinline__ float dot64_bf16(const __nv_bfloat16* p, const __nv_bfloat16* q) {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 2
+    for (int f = 0; f < TTT_D; f += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p + f), v = *reinterpret_cast<const uint4*>(q + f);
+        const uint32_t us[4] = {u.x, u.y, u.z, u.w}, vs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; i += 2) {
+            const float2 x0 = unpack_bf16x2(us[i]), y0 = unpack_bf16x2(vs[i]);
+            const float2 x1 = unpack_bf16x2(us[i + 1]), y1 = unpack_bf16x2(vs[i + 1]);
+            a0 = fmaf(x0.x, y0.x, a0);
+            a1 = fmaf(x0.y, y0.y, a1);
+            a0 = fmaf(x1.x, y1.x, a0);
+            a1 = fmaf(x1.y, y1.y, a1);
+        }
+    }
+    return a0 + a1;
+}
+
 // LayerNorm statistics of a row whose four features z this thread holds: x_hat and sigma.
 __device__ __forceinline__ void row_norm(float4 z, float eps, float4& xh, float& sigma) {
     const float mu = row_sum(hsum4(z)) * (1.0f / TTT_D);
@@ -467,11 +487,11 @@ __global__ void linear_bwd_copy_kernel(const float* part, long long chains, floa
 // A 16 x 64 product lands in a shared result tile, warp w computing columns 8w .. 8w + 7, and the
 // row-layout threads read it back.  The LayerNorm work and the 16 x 16 products are as above.
 // ---------------------------------------------------------------------------------------------
+constexpr int kSB = TTT_D + 8;  // row stride (bf16 elements) of the staged input tiles: 144 bytes
+
 struct __align__(16) BwdTcSmem {
     float W[TTT_D][kS];
     float dW[TTT_D][kS];
-    float xq[TTT_KMAX][kS];
-    float xk[TTT_KMAX][kS];
     float g[TTT_KMAX][kS];
     float dzb[TTT_KMAX][kS];
     float dz[TTT_KMAX][kS];
@@ -486,11 +506,11 @@ struct __align__(16) BwdTcSmem {
     float dlr_eta[TTT_KMAX][kS16];
     float b[TTT_D];
     float db[TTT_D];
-    float lr[TTT_KMAX];
     float te[TTT_KMAX];
     float dlr_row[TTT_KMAX];
-    // the next step's inputs, copied in while the current step runs: [buffer][XQ, XK, XV, d_out]
-    __nv_bfloat16 stage[2][4][TTT_KMAX][TTT_D];
+    // each step's inputs, copied in while the step before runs: [buffer][XQ, XK, XV, d_out]; the
+    // MMAs and dot products read XQ and XK from here (bf16 values are exact TF32 operands)
+    __nv_bfloat16 stage[2][4][TTT_KMAX][kSB];
     float stage_lr[2][TTT_KMAX];
 };
 
@@ -521,19 +541,25 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1
                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// A TF32 operand from fp32 (rounded to nearest) or from bf16 (exact: the bits moved up).
+__device__ __forceinline__ uint32_t op32(float x) { return tf32(x); }
+__device__ __forceinline__ uint32_t op32(__nv_bfloat16 x) { return static_cast<uint32_t>(__bfloat16_as_ushort(x)) << 16; }
+__device__ __forceinline__ float f32(float x) { return x; }
+__device__ __forceinline__ float f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
 // acc += sum_{k < K} X[m][k] Y(k, n0 + n) for the 16 x 8 tile at columns n0: X rows of stride kSX;
-// Y(k, n) = Ymat[k][n], or Ymat[n][k] when kTrans.  Even and odd k-steps accumulate apart (half
-// the dependent MMA latency) and meet at the end.
-template <int K, int kSX, bool kTrans>
-__device__ __forceinline__ void tc_tile(float (&acc)[4], const float (*X)[kSX], const float (*Y)[kS], int n0, int g,
+// Y(k, n) = Ymat[k][n], or Ymat[n][k] when kTrans (rows of stride kSY).  Even and odd k-steps
+// accumulate apart (half the dependent MMA latency) and meet at the end.
+template <int K, bool kTrans, typename TX, int kSX, typename TY, int kSY>
+__device__ __forceinline__ void tc_tile(float (&acc)[4], const TX (*X)[kSX], const TY (*Y)[kSY], int n0, int g,
                                         int t) {
     float odd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k0 = 0; k0 < K; k0 += 8) {
-        const uint32_t a0 = tf32(X[g][k0 + t]), a1 = tf32(X[g + 8][k0 + t]);
-        const uint32_t a2 = tf32(X[g][k0 + t + 4]), a3 = tf32(X[g + 8][k0 + t + 4]);
-        const uint32_t b0 = tf32(kTrans ? Y[n0 + g][k0 + t] : Y[k0 + t][n0 + g]);
-        const uint32_t b1 = tf32(kTrans ? Y[n0 + g][k0 + t + 4] : Y[k0 + t + 4][n0 + g]);
+        const uint32_t a0 = op32(X[g][k0 + t]), a1 = op32(X[g + 8][k0 + t]);
+        const uint32_t a2 = op32(X[g][k0 + t + 4]), a3 = op32(X[g + 8][k0 + t + 4]);
+        const uint32_t b0 = op32(kTrans ? Y[n0 + g][k0 + t] : Y[k0 + t][n0 + g]);
+        const uint32_t b1 = op32(kTrans ? Y[n0 + g][k0 + t + 4] : Y[k0 + t + 4][n0 + g]);
         if ((k0 >> 3) & 1) mma_tf32(odd, a0, a1, a2, a3, b0, b1);
         else mma_tf32(acc, a0, a1, a2, a3, b0, b1);
     }
@@ -542,16 +568,16 @@ __device__ __forceinline__ void tc_tile(float (&acc)[4], const float (*X)[kSX], 
 }
 
 // c0 += X0 Y and c1 += X1 Y over K = 64 for the tile at columns n0, sharing Y's fragments.
-template <bool kTrans>
-__device__ __forceinline__ void tc_tile2(float (&c0)[4], float (&c1)[4], const float (*X0)[kS], const float (*X1)[kS],
+template <bool kTrans, typename TX, int kSX>
+__device__ __forceinline__ void tc_tile2(float (&c0)[4], float (&c1)[4], const TX (*X0)[kSX], const TX (*X1)[kSX],
                                          const float (*Y)[kS], int n0, int g, int t) {
 #pragma unroll
     for (int k0 = 0; k0 < TTT_D; k0 += 8) {
         const uint32_t b0 = tf32(kTrans ? Y[n0 + g][k0 + t] : Y[k0 + t][n0 + g]);
         const uint32_t b1 = tf32(kTrans ? Y[n0 + g][k0 + t + 4] : Y[k0 + t + 4][n0 + g]);
-        mma_tf32(c0, tf32(X0[g][k0 + t]), tf32(X0[g + 8][k0 + t]), tf32(X0[g][k0 + t + 4]), tf32(X0[g + 8][k0 + t + 4]),
+        mma_tf32(c0, op32(X0[g][k0 + t]), op32(X0[g + 8][k0 + t]), op32(X0[g][k0 + t + 4]), op32(X0[g + 8][k0 + t + 4]),
                  b0, b1);
-        mma_tf32(c1, tf32(X1[g][k0 + t]), tf32(X1[g + 8][k0 + t]), tf32(X1[g][k0 + t + 4]), tf32(X1[g + 8][k0 + t + 4]),
+        mma_tf32(c1, op32(X1[g][k0 + t]), op32(X1[g + 8][k0 + t]), op32(X1[g][k0 + t + 4]), op32(X1[g + 8][k0 + t + 4]),
                  b0, b1);
     }
 }
@@ -565,12 +591,13 @@ __device__ __forceinline__ void put_tile(float (*P)[kS], const float (&c)[4], in
 // acc (this warp's four 16 x 8 tiles of a 64 x 64 matrix at rows m0, columns n0 + 8q) +=
 // sum_{j < 16} s_j X[j][m] Y[j][n]: the rank-16 update by the tokens of a mini-batch, with
 // s_j = scale * lr[j] (lr non-null) or 1.
-__device__ __forceinline__ void tc_rank16(float (&acc)[4][4], const float (*X)[kS], const float* lr, float scale,
+template <typename TX, int kSX>
+__device__ __forceinline__ void tc_rank16(float (&acc)[4][4], const TX (*X)[kSX], const float* lr, float scale,
                                           const float (*Y)[kS], int m0, int n0, int g, int t) {
 #pragma unroll
     for (int k0 = 0; k0 < TTT_KMAX; k0 += 8) {
-        float x0 = X[k0 + t][m0 + g], x1 = X[k0 + t][m0 + g + 8];
-        float x2 = X[k0 + t + 4][m0 + g], x3 = X[k0 + t + 4][m0 + g + 8];
+        float x0 = f32(X[k0 + t][m0 + g]), x1 = f32(X[k0 + t][m0 + g + 8]);
+        float x2 = f32(X[k0 + t + 4][m0 + g]), x3 = f32(X[k0 + t + 4][m0 + g + 8]);
         if (lr) {
             const float s0 = scale * lr[k0 + t], s1 = scale * lr[k0 + t + 4];
             x0 *= s0;
@@ -700,13 +727,12 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         cp_async_wait_all();
         __syncthreads();  // the staged inputs have landed, and the last step's readers of the tiles are done
         const float4 k4 = staged(buf, 1), v4 = staged(buf, 2);
-        st4(&s.xk[r][c0], k4);
-        if (tid < TTT_KMAX) s.lr[tid] = s.stage_lr[buf][tid];
+        const __nv_bfloat16 (*xk)[kSB] = s.stage[buf][1];
+        const float* lrs = s.stage_lr[buf];
         start_next(buf, nx);
-        __syncthreads();
         {
             float c[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile<TTT_D, kS, false>(c, s.xk, s.W, nt, g, t);
+            tc_tile<TTT_D, false>(c, xk, s.W, nt, g, t);
             put_tile(s.P0, c, nt, g, t);
         }
         __syncthreads();
@@ -720,10 +746,10 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         st4(&s.g[r][c0], gv);
         __syncthreads();
         const float tl = s.te[K - 1];
-        tc_rank16(Wacc, s.xk, s.lr, -tl, s.g, m0, n0, g, t);
+        tc_rank16(Wacc, xk, lrs, -tl, s.g, m0, n0, g, t);
         if (tid < TTT_D) {
             float acc = 0.f;
-            for (int i = 0; i < K; ++i) acc = fmaf(tl * s.lr[i], s.g[i][tid], acc);
+            for (int i = 0; i < K; ++i) acc = fmaf(tl * lrs[i], s.g[i][tid], acc);
             s.b[tid] -= acc;
         }
         // the Z product, W's only reader, finished before the last barrier; each thread writes its own
@@ -739,23 +765,22 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const bool live = r < Km;
         const long long row = (t0 + r) * TTT_D + c0;
         cp_async_wait_all();
-        __syncthreads();  // (0) the staged inputs have landed
-        const float4 q4 = staged(buf, 0), k4 = staged(buf, 1), v4 = staged(buf, 2), o4 = staged(buf, 3);
-        st4(&s.xq[r][c0], q4);
-        st4(&s.xk[r][c0], k4);
-        if (tid < TTT_KMAX) s.lr[tid] = s.stage_lr[buf][tid];
+        __syncthreads();  // (0) the staged inputs have landed; the step reads XQ, XK and lr from them
+        const float4 k4 = staged(buf, 1), v4 = staged(buf, 2), o4 = staged(buf, 3);
+        const __nv_bfloat16 (*xq)[kSB] = s.stage[buf][0];
+        const __nv_bfloat16 (*xk)[kSB] = s.stage[buf][1];
+        const float* lrs = s.stage_lr[buf];
         start_next(buf, nx);
-        __syncthreads();  // (1)
         {  // XK W and XQ W, sharing W's fragments
             float cz[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile2<false>(cz, cb, s.xk, s.xq, s.W, nt, g, t);
+            tc_tile2<false>(cz, cb, xk, xq, s.W, nt, g, t);
             put_tile(s.P0, cz, nt, g, t);
             put_tile(s.P1, cb, nt, g, t);
         }
         {  // A = XQ XK^T and M = eta * tril(A + 1) at (i, j) = (r, tid % 16)
             const int i = r, j = tid & 15;
-            const float av = dot64(s.xq[i], s.xk[j]);
-            const float m = (j <= i && i < Km) ? s.te[i] * s.lr[j] * (av + 1.0f) : 0.f;
+            const float av = dot64_bf16(xq[i], xk[j]);
+            const float m = (j <= i && i < Km) ? s.te[i] * lrs[j] * (av + 1.0f) : 0.f;
             s.A[i][j] = av;
             s.M[i][j] = m;
             s.MT[j][i] = m;
@@ -775,12 +800,12 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         __syncthreads();  // (3)
         {  // M g; and the update's XK dW' and g dW'^T from the adjoint after the mini-batch
             float cm[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile<TTT_KMAX, kS16, false>(cm, s.M, s.g, nt, g, t);
+            tc_tile<TTT_KMAX, false>(cm, s.M, s.g, nt, g, t);
             put_tile(s.P0, cm, nt, g, t);
             if (full) {
                 float cu[4] = {0.f, 0.f, 0.f, 0.f}, cv[4] = {0.f, 0.f, 0.f, 0.f};
-                tc_tile<TTT_D, kS, false>(cu, s.xk, s.dW, nt, g, t);
-                tc_tile<TTT_D, kS, true>(cv, s.g, s.dW, nt, g, t);
+                tc_tile<TTT_D, false>(cu, xk, s.dW, nt, g, t);
+                tc_tile<TTT_D, true>(cv, s.g, s.dW, nt, g, t);
                 put_tile(s.P1, cu, nt, g, t);
                 put_tile(s.P2, cv, nt, g, t);
             }
@@ -800,14 +825,14 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         __syncthreads();  // (5)
         {  // M^T dZbar
             float cg[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile<TTT_KMAX, kS16, false>(cg, s.MT, s.dzb, nt, g, t);
+            tc_tile<TTT_KMAX, false>(cg, s.MT, s.dzb, nt, g, t);
             put_tile(s.P0, cg, nt, g, t);
         }
         {  // dM = -dZbar g^T on the lower triangle: its shares of dA and of dlr
             const int i = r, j = tid & 15;
             const float dm = (j <= i && i < Km) ? -dot64(s.dzb[i], s.g[j]) : 0.f;
             s.dlr_eta[i][j] = s.te[i] * (s.A[i][j] + 1.0f) * dm;
-            const float da = dm * s.te[i] * s.lr[j];
+            const float da = dm * s.te[i] * lrs[j];
             s.dA[i][j] = da;
             s.dAT[j][i] = da;
         }
@@ -816,7 +841,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         float4 dxk = f4(0.f);
         float dlr_upd = 0.f;
         if (full) {
-            const float tl = s.te[K - 1], e = tl * s.lr[r];
+            const float tl = s.te[K - 1], e = tl * lrs[r];
             dg = dg - U * e;
             dlr_upd = -tl * row_sum(hsum4(gv * U));
             dxk = f4(0.f) - V * e;
@@ -841,12 +866,12 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         {  // dZbar W^T + dA XK and dZ W^T + dA^T XQ; the adjoint of the start state
             float cq[4] = {0.f, 0.f, 0.f, 0.f}, ck[4] = {0.f, 0.f, 0.f, 0.f};
             tc_tile2<true>(cq, ck, s.dzb, s.dz, s.W, nt, g, t);
-            tc_tile<TTT_KMAX, kS16, false>(cq, s.dA, s.xk, nt, g, t);
-            tc_tile<TTT_KMAX, kS16, false>(ck, s.dAT, s.xq, nt, g, t);
+            tc_tile<TTT_KMAX, false>(cq, s.dA, xk, nt, g, t);
+            tc_tile<TTT_KMAX, false>(ck, s.dAT, xq, nt, g, t);
             put_tile(s.P0, cq, nt, g, t);
             put_tile(s.P1, ck, nt, g, t);
-            tc_rank16(dWacc, s.xq, nullptr, 1.f, s.dzb, m0, n0, g, t);
-            tc_rank16(dWacc, s.xk, nullptr, 1.f, s.dz, m0, n0, g, t);
+            tc_rank16(dWacc, xq, nullptr, 1.f, s.dzb, m0, n0, g, t);
+            tc_rank16(dWacc, xk, nullptr, 1.f, s.dz, m0, n0, g, t);
         }
         __syncthreads();  // (8)
         if (live) {
