@@ -105,6 +105,26 @@ __device__ __forceinline__ float gelu(float x) {
     return 0.5f * x * (1.0f + tanh_fast(k * fmaf(c * x, x * x, x)));
 }
 
+// The same for two elements at once with paired fp32 arithmetic (one FFMA2 per two FFMAs).
+__device__ __forceinline__ void gelu2_pair(float2 x, float2& y, float2& dy) {
+    const float2 k = make_float2(0.7978845608028654f, 0.7978845608028654f), c = make_float2(0.044715f, 0.044715f);
+    const float2 h = make_float2(0.5f, 0.5f), one = make_float2(1.0f, 1.0f);
+    const float2 x2 = __fmul2_rn(x, x);
+    const float2 u = __fmul2_rn(k, __ffma2_rn(__fmul2_rn(c, x), x2, x));
+    const float2 th = make_float2(tanh_fast(u.x), tanh_fast(u.y));
+    const float2 hx = __fmul2_rn(h, x), op = __fadd2_rn(one, th);
+    y = __fmul2_rn(hx, op);
+    const float2 sech2 = __ffma2_rn(__fmul2_rn(th, th), make_float2(-1.0f, -1.0f), one);
+    const float2 poly = __fmul2_rn(k, __ffma2_rn(make_float2(3.0f * 0.044715f, 3.0f * 0.044715f), x2, one));
+    dy = __ffma2_rn(__fmul2_rn(hx, sech2), poly, __fmul2_rn(h, op));
+}
+__device__ __forceinline__ float2 gelu_pair(float2 x) {
+    const float2 k = make_float2(0.7978845608028654f, 0.7978845608028654f), c = make_float2(0.044715f, 0.044715f);
+    const float2 u = __fmul2_rn(k, __ffma2_rn(__fmul2_rn(c, x), __fmul2_rn(x, x), x));
+    const float2 th = make_float2(tanh_fast(u.x), tanh_fast(u.y));
+    return __fmul2_rn(__fmul2_rn(make_float2(0.5f, 0.5f), x), __fadd2_rn(make_float2(1.0f, 1.0f), th));
+}
+
 // Mean and 1/sqrt(var + eps) of a 64-value row held 4 per lane by 16 lanes (Chan merges).
 __device__ __forceinline__ void row_stats16(const float (&v)[4], float eps, float& mu, float& rstd) {
     float m = 0.25f * ((v[0] + v[1]) + (v[2] + v[3]));
@@ -401,11 +421,12 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
         uint32_t x2p[4][2];  // X2 as bf16 pairs: [n-tile][row g, row g + 8]
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            float y[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) gelu2(z1[nt][e], y[e], dg[nt][e]);
-            x2p[nt][0] = pack_f16x2(y[0], y[1]);
-            x2p[nt][1] = pack_f16x2(y[2], y[3]);
+            float2 y0, y1, d0, d1;
+            gelu2_pair(make_float2(z1[nt][0], z1[nt][1]), y0, d0);
+            gelu2_pair(make_float2(z1[nt][2], z1[nt][3]), y1, d1);
+            dg[nt][0] = d0.x; dg[nt][1] = d0.y; dg[nt][2] = d1.x; dg[nt][3] = d1.y;
+            x2p[nt][0] = pack_f16x2(y0.x, y0.y);
+            x2p[nt][1] = pack_f16x2(y1.x, y1.y);
         }
         store_slice(&s.X2s[0], w, g, t, x2p);
         __syncthreads();
@@ -528,8 +549,10 @@ mlp_tc_kernel(const MlpArgs a, const __grid_constant__ LinearMaps maps) {
             uint32_t xb2p[4][2];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                xb2p[nt][0] = pack_f16x2(gelu(zb1[nt][0]), gelu(zb1[nt][1]));
-                xb2p[nt][1] = pack_f16x2(gelu(zb1[nt][2]), gelu(zb1[nt][3]));
+                const float2 y0 = gelu_pair(make_float2(zb1[nt][0], zb1[nt][1]));
+                const float2 y1 = gelu_pair(make_float2(zb1[nt][2], zb1[nt][3]));
+                xb2p[nt][0] = pack_f16x2(y0.x, y0.y);
+                xb2p[nt][1] = pack_f16x2(y1.x, y1.y);
             }
             store_slice(&s.XB2s[0], w, g, t, xb2p);
             float a2[2][4] = {};
