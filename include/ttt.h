@@ -440,10 +440,14 @@ long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, 
  *   d_ln_w, d_ln_b  [H,d] float32, summed over the batch.
  *   workspace    device buffer of at least ttt_linear_backward_workspace_bytes, 256-byte aligned;
  *                its contents on entry do not matter and are overwritten.
- * Computes in float32 throughout (one CTA per chain); the batch sums run in a fixed order, so
- * results are reproducible bit for bit.  Asynchronous on `stream`; allocates nothing; has no
+ * One CTA per chain.  fp32 activations compute in float32 throughout; bf16 activations run the
+ * products and state updates on the tensor cores with TF32 operands (11-bit significands, like
+ * the forward's fp16 operands) and fp32 accumulation, state and adjoint.  The batch sums run in
+ * a fixed order, so results are reproducible bit for bit.  Asynchronous on `stream`; allocates nothing; has no
  * device-side waits.  Errors as ttt_linear_forward (flags aside), plus TTT_ERR_ARG for
- * ckpt_group < 1 or a workspace smaller than needed.
+ * ckpt_group < 1 or a workspace smaller than needed.  The call makes two launches (the scan's
+ * backward, then the batch sums); a TTT_ERR_CUDA from the second comes after the first is
+ * enqueued, so synchronise `stream` before reusing the workspace or the outputs after it.
  */
 int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
                         const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
