@@ -428,12 +428,16 @@ long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, 
  *
  * Arguments:
  *   XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d, mini_batch,
- *   eps, dtype   as ttt_linear_forward (head-major [B,H,L,d] only; no flags).
+ *   eps, dtype   as ttt_linear_forward.
+ *   flags        0 or TTT_FLAG_TOKEN_MAJOR: XQ, XK, XV, d_out, dXQ, dXK and dXV are [B,L,H,d] instead
+ *                of [B,H,L,d] (lr and d_lr stay [B,H,L]); TTT_FLAG_FP32_COMPUTE is
+ *                TTT_ERR_UNSUPPORTED (fp32 activations already run in fp32).
  *   ckpt_group   >= 1: mini-batches per checkpoint group.
- *   d_out        [B,H,L,d] dtype, 16-byte aligned: the gradient of out (NULL allowed if L == 0).
+ *   d_out        [B,H,L,d] (or token-major) dtype, 16-byte aligned: the gradient of out (NULL
+ *                allowed if L == 0).
  *   dW_last, db_last  [B,H,d,d], [B,H,d] float32, 16-byte aligned, or NULL (zero).
  * Outputs (device, caller-allocated, none overlapping an input, another output or the workspace):
- *   dXQ, dXK, dXV  [B,H,L,d] dtype, 16-byte aligned (NULL allowed if L == 0).
+ *   dXQ, dXK, dXV  [B,H,L,d] (or token-major) dtype, 16-byte aligned (NULL allowed if L == 0).
  *   d_lr         [B,H,L] float32.
  *   dW0, db0     float32: [H,d,d] and [H,d] summed over the batch when w0_batch_stride == 0 (one
  *                initial state per head), else [B,H,d,d] and [B,H,d] per chain.
@@ -452,9 +456,9 @@ long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, 
 int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
                         const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
                         const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps, int dtype,
-                        int ckpt_group, const void* d_out, const float* dW_last, const float* db_last, void* dXQ,
-                        void* dXK, void* dXV, float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b,
-                        void* workspace, long long workspace_bytes, void* stream);
+                        unsigned int flags, int ckpt_group, const void* d_out, const float* dW_last,
+                        const float* db_last, void* dXQ, void* dXK, void* dXV, float* d_lr, float* dW0, float* db0,
+                        float* d_ln_w, float* d_ln_b, void* workspace, long long workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -85,7 +85,7 @@ def lib():
         L.ttt_post_norm_o_proj.argtypes = [vp, ll, i, vp, fp, fp, i, f, vp, fp, vp]
         L.ttt_linear_backward_workspace_bytes.argtypes = [i, i, ll, i, i, i]
         L.ttt_linear_backward_workspace_bytes.restype = ll
-        L.ttt_linear_backward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, i, vp, fp,
+        L.ttt_linear_backward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u, i, vp, fp,
                                           fp, vp, vp, vp, fp, fp, fp, fp, fp, vp, ll, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
                      "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
@@ -487,15 +487,15 @@ def ttt_linear_backward_workspace_bytes(B: int, H: int, L: int, mini_batch: int 
 
 def ttt_linear_backward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, d_out, dW_last=None, db_last=None,
                         mini_batch: int = 16, eps: float = 1e-6, token_eta=None, ckpt_group: int = 16,
-                        workspace=None, stream=None):
+                        token_major: bool = False, workspace=None, stream=None):
     """Gradients of <d_out, out> + <dW_last, W_last> + <db_last, b_last> for ttt_linear_forward's
-    inputs (head-major [B,H,L,64]; see include/ttt.h).
+    inputs ([B,H,L,64], or [B,L,H,64] with token_major; see include/ttt.h).
 
     Returns a dict: dXQ, dXK, dXV (the activations' dtype), dlr [B,H,L], dW0/db0 (per head when W0
     is [H,64,64], per chain when it is [B,H,64,64]), dln_w/dln_b [H,64].
     """
     _need(XQ, "XQ")
-    B, H, L, d = _act_sizes(XQ, False)
+    B, H, L, d = _act_sizes(XQ, token_major)
     dt = XQ.dtype
     for n, t in (("XK", XK), ("XV", XV), ("d_out", d_out)):
         _need(t, n, dt, XQ.shape)
@@ -523,7 +523,8 @@ def ttt_linear_backward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, d_out, dW_last=None,
          "dln_w": torch.empty((H, d), device=dev), "dln_b": torch.empty((H, d), device=dev)}
     _check(lib().ttt_linear_backward(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
                                      H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
-                                     eps, _dtype_code(XQ), ckpt_group, _ptr(d_out), _ptr(dW_last), _ptr(db_last),
+                                     eps, _dtype_code(XQ), TTT_FLAG_TOKEN_MAJOR if token_major else 0, ckpt_group,
+                                     _ptr(d_out), _ptr(dW_last), _ptr(db_last),
                                      _ptr(g["dXQ"]), _ptr(g["dXK"]), _ptr(g["dXV"]), _ptr(g["dlr"]), _ptr(g["dW0"]),
                                      _ptr(g["db0"]), _ptr(g["dln_w"]), _ptr(g["dln_b"]), _ptr(workspace),
                                      workspace.numel(), _stream(stream)))

@@ -168,7 +168,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_kernel(const LinearBwdArgs a
     const int G = a.G;
     const long long L = a.L;
     const float eps = a.eps;
-    const long long base = chain * L * TTT_D;
+    const long long base = (chain / a.H) * a.act_b + h * a.act_h;  // this chain's token 0
+    const long long ts = a.act_t;                                     // elements between its tokens
     const T* XQ = static_cast<const T*>(a.XQ) + base;
     const T* XK = static_cast<const T*>(a.XK) + base;
     const T* XV = static_cast<const T*>(a.XV) + base;
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_kernel(const LinearBwdArgs a
     // s.W) becomes W - XK^T diag(e) g, b - e^T g.
     auto fwd_step = [&](long long t0) {
         const bool live = r < K;
-        const long long row = (t0 + r) * TTT_D + c0;
+        const long long row = (t0 + r) * ts + c0;
         const float4 k4 = live ? ld4(XK + row) : f4(0.f);
         const float4 v4 = live ? ld4(XV + row) : f4(0.f);
         st4(&s.xk[r][c0], k4);
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_kernel(const LinearBwdArgs a
     // s.dWT / s.db.  Leaves the adjoint of its start state there.
     auto bwd_step = [&](long long t0, int Km, bool full) {
         const bool live = r < Km;
-        const long long row = (t0 + r) * TTT_D + c0;
+        const long long row = (t0 + r) * ts + c0;
         const float4 q4 = live ? ld4(XQ + row) : f4(0.f);
         const float4 k4 = live ? ld4(XK + row) : f4(0.f);
         const float4 v4 = live ? ld4(XV + row) : f4(0.f);
@@ -627,7 +628,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     const int G = a.G;
     const long long L = a.L;
     const float eps = a.eps;
-    const long long base = chain * L * TTT_D;
+    const long long base = (chain / a.H) * a.act_b + h * a.act_h;  // this chain's token 0
+    const long long ts = a.act_t;                                     // elements between its tokens
     const T* XQ = static_cast<const T*>(a.XQ) + base;
     const T* XK = static_cast<const T*>(a.XK) + base;
     const T* XV = static_cast<const T*>(a.XV) + base;
@@ -698,7 +700,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             const int rowc = (cidx & 127) >> 3, part = cidx & 7;
             const bool in = rowc < Km;
             const T* src = ti == 0 ? XQ : ti == 1 ? XK : ti == 2 ? XV : DO;
-            cp_async_16z(&s.stage[buf][ti][rowc][part * 8], in ? src + (t0 + rowc) * TTT_D + part * 8 : src,
+            cp_async_16z(&s.stage[buf][ti][rowc][part * 8], in ? src + (t0 + rowc) * ts + part * 8 : src,
                          in ? 16u : 0u);
         }
         if (tid < TTT_KMAX) cp_async_4z(&s.stage_lr[buf][tid], tid < Km ? lr + t0 + tid : lr, tid < Km ? 4u : 0u);
@@ -763,7 +765,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     // Wacc / s.W / s.b, the adjoint after it in dWacc / s.dW / s.db, its inputs in staging buffer buf.
     auto bwd_step = [&](long long t0, int Km, bool full, int buf, const Next& nx) {
         const bool live = r < Km;
-        const long long row = (t0 + r) * TTT_D + c0;
+        const long long row = (t0 + r) * ts + c0;
         cp_async_wait_all();
         __syncthreads();  // (0) the staged inputs have landed; the step reads XQ, XK and lr from them
         const float4 k4 = staged(buf, 1), v4 = staged(buf, 2), o4 = staged(buf, 3);

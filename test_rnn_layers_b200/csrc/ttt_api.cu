@@ -782,11 +782,13 @@ long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, 
 int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
                         const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
                         const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps, int dtype,
-                        int ckpt_group, const void* d_out, const float* dW_last, const float* db_last, void* dXQ,
-                        void* dXK, void* dXV, float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b,
-                        void* workspace, long long workspace_bytes, void* stream) {
-    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, 0);
+                        unsigned int flags, int ckpt_group, const void* d_out, const float* dW_last,
+                        const float* db_last, void* dXQ, void* dXK, void* dXV, float* d_lr, float* dW0, float* db0,
+                        float* d_ln_w, float* d_ln_b, void* workspace, long long workspace_bytes, void* stream) {
+    int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
     if (rc) return rc;
+    if (flags & TTT_FLAG_FP32_COMPUTE)
+        return fail(TTT_ERR_UNSUPPORTED, "the backward takes no TTT_FLAG_FP32_COMPUTE (fp32 activations run in fp32)");
     if (ckpt_group < 1) return fail(TTT_ERR_ARG, "ckpt_group must be >= 1 (got %d)", ckpt_group);
     const long long chains = static_cast<long long>(B) * H;
     const long long per_head = static_cast<long long>(kD) * kD;
@@ -833,6 +835,10 @@ int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const fl
     a.ln_w = ln_w; a.ln_b = ln_b; a.dW_last = dW_last; a.db_last = db_last;
     a.B = B; a.H = H; a.K = mini_batch;
     a.L = L; a.n_full = L / mini_batch; a.rem = L % mini_batch;
+    const bool tok_major = (flags & TTT_FLAG_TOKEN_MAJOR) != 0;
+    a.act_b = static_cast<long long>(H) * L * kD;
+    a.act_h = tok_major ? kD : L * kD;
+    a.act_t = tok_major ? static_cast<long long>(H) * kD : kD;
     a.eps = eps; a.G = ckpt_group; a.n_ckpt = lay.n_ckpt;
     a.dXQ = dXQ; a.dXK = dXK; a.dXV = dXV; a.d_lr = d_lr;
     char* ws = static_cast<char*>(workspace);

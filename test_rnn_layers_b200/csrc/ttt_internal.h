@@ -159,6 +159,9 @@ struct LinearBwdArgs {
     const float* db_last;       // [B*H][d] or nullptr (zero)
     int B, H, K;
     long long L, n_full, rem;
+    // element strides of XQ, XK, XV, d_out and their gradients between batch rows, heads and
+    // tokens: head-major [B, H, L, d] or token-major [B, L, H, d] (as in LinearArgs)
+    long long act_b, act_h, act_t;
     float eps;
     int G;                      // checkpoint group: a state is kept every G full mini-batches
     long long n_ckpt;           // ceil(n_full / G)

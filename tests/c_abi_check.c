@@ -75,7 +75,7 @@ int main(void) {
           "backward workspace rejects ckpt_group = 0");
     float* g[8];
     for (int i = 0; i < 8; ++i) g[i] = (float*)((uintptr_t)(12 + i) * A);  /* fake gradient outputs */
-    check(ttt_linear_backward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0, out,
+    check(ttt_linear_backward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0u, 0, out,
                               NULL, NULL, g[0], g[1], g[2], g[3], g[4], g[5], g[6], g[7], NULL, 0, NULL) == TTT_ERR_ARG,
           "backward rejects ckpt_group = 0");
     return failures == 0 ? 0 : 1;

@@ -192,3 +192,24 @@ def test_backward_1b_layer_sampled_chains(libttt):
     print("[backward 1b sampled]", chains, {k: f"{v:.2e}" for k, v in errs.items()})
     for k, v in errs.items():
         assert v <= _tol("bf16", k), (k, v)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_backward_token_major_gives_the_head_major_bits(libttt, dt):
+    """[B,L,H,64] activations and gradients (TTT_FLAG_TOKEN_MAJOR): the same arithmetic as the
+    head-major call, so the same bits."""
+    w = synth.workload(1, B=2, H=3, L=16 * 4 + 5, dtype=dt, seed=0xB6)
+    x, up = synth.linear_inputs(w), synth.upstream_grads(w)
+    XQ, XK, XV = (dev_act(x, n) for n in ("XQ", "XK", "XV"))
+    dout = dev_act(up, "d_out")
+    common = [dev_f32(x[k]) for k in ("lr", "W0", "b0", "ln_w", "ln_b")]
+    last = (dev_f32(up["dW_last"]), dev_f32(up["db_last"]))
+    gh = libttt.ttt_linear_backward(XQ, XK, XV, *common, dout, *last, mini_batch=w.K, eps=w.eps, ckpt_group=3)
+    tm = lambda t: t.transpose(1, 2).contiguous()
+    gt = libttt.ttt_linear_backward(tm(XQ), tm(XK), tm(XV), *common, tm(dout), *last, mini_batch=w.K, eps=w.eps,
+                                    ckpt_group=3, token_major=True)
+    torch.cuda.synchronize()
+    for k in ("dXQ", "dXK", "dXV"):
+        assert torch.equal(gt[k].transpose(1, 2), gh[k]), k
+    for k in ("dlr", "dW0", "db0", "dln_w", "dln_b"):
+        assert torch.equal(gt[k], gh[k]), k

@@ -305,12 +305,12 @@ def test_post_norm_o_proj_T0_is_a_no_op(libttt):
 
 def _bwd(lib, **kw):
     a = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W0=5 * A, b0=6 * A, stride=0, lnw=7 * A, lnb=8 * A, B=2,
-             H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, G=4, dout=9 * A, dWl=None, dbl=None, dXQ=10 * A, dXK=11 * A,
+             H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, flags=0, G=4, dout=9 * A, dWl=None, dbl=None, dXQ=10 * A, dXK=11 * A,
              dXV=12 * A, dlr=13 * A, dW0=14 * A, db0=15 * A, dlnw=16 * A, dlnb=17 * A, ws=1 << 32, wsb=1 << 30)
     a.update(kw)
     return lib.ttt_linear_backward(a["XQ"], a["XK"], a["XV"], a["lr"], a["te"], a["W0"], a["b0"], a["stride"],
                                    a["lnw"], a["lnb"], a["B"], a["H"], a["L"], a["d"], a["K"], a["eps"], a["dtype"],
-                                   a["G"], a["dout"], a["dWl"], a["dbl"], a["dXQ"], a["dXK"], a["dXV"], a["dlr"],
+                                   a["flags"], a["G"], a["dout"], a["dWl"], a["dbl"], a["dXQ"], a["dXK"], a["dXV"], a["dlr"],
                                    a["dW0"], a["db0"], a["dlnw"], a["dlnb"], a["ws"], a["wsb"], None)
 
 
@@ -320,6 +320,7 @@ def _bwd(lib, **kw):
     (dict(wsb=100), -1), (dict(ws=(1 << 32) + 16), -2), (dict(XK=2 * A + 2), -2), (dict(dXQ=10 * A + 8), -2),
     (dict(dlr=13 * A + 1), -2), (dict(dWl=18 * A + 4), -2), (dict(dXQ=A), -3), (dict(dXK=10 * A), -3),
     (dict(ws=5 * A), -3), (dict(dW0=9 * A), -3), (dict(dlnb=16 * A + 64), -3),
+    (dict(flags=1), -6), (dict(flags=4), -1), (dict(flags=2, dXQ=A), -3), (dict(flags=2, XK=2 * A + 2), -2),
 ])
 def test_linear_backward_rejects(libttt, kw, code):
     lib = libttt.lib()
