@@ -482,16 +482,31 @@ __global__ void linear_bwd_copy_kernel(const float* part, long long chains, floa
 
 // ---------------------------------------------------------------------------------------------
 // Tensor-core form (bf16 activations).  The 16 x 64 x 64 products and the rank-16 state updates
-// run as TF32 warp MMAs (m16n8k8, fp32 accumulation): the state W and its adjoint dW live as
-// accumulators, warp w holding rows 16 (w / 2) .. +15 and columns 32 (w % 2) .. +31 of each (four
-// 16 x 8 tiles), and their copies in shared memory serve as B operands, read plain or transposed.
-// A 16 x 64 product lands in a shared result tile, warp w computing columns 8w .. 8w + 7, and the
-// row-layout threads read it back.  The LayerNorm work and the 16 x 16 products are as above.
+// run as TF32 warp MMAs (m16n8k8, fp32 accumulation).
+//  * The state W lives as accumulators of W^T: warp w holds output features 16 (w % 4) .. +15
+//    (rows of W^T) and inputs 32 (w / 4) .. +31 (columns), four 16 x 8 tiles.  Read with the k
+//    slots t and t + 4 of an MMA step standing for the inputs k0 + 2t and k0 + 2t + 1, that
+//    accumulator layout is the B operand of Z = XK W, so a forward step multiplies by W straight
+//    from registers (each warp half of Z's inner dimension; the halves meet in shared memory with
+//    the LayerNorm's row exchange) and takes XK as bf16 pairs, one 32-bit load for two operands.
+//    The update W^T += (-t lr g)^T XK accumulates into the same registers, XK arriving by
+//    transposing ldmatrix loads.  W^T is written to shared memory only for the backward steps.
+//  * The adjoint dW lives as accumulators too, warp w holding rows 16 (w / 2) .. +15 and columns
+//    32 (w % 2) .. +31 (four 16 x 8 tiles); its shared copy serves as a B operand.
+//  * A 16 x 64 product of a backward step lands in a shared result tile, warp w computing columns
+//    8w .. 8w + 7, and the row-layout threads read it back.  The LayerNorm work and the 16 x 16
+//    products are as above.
+//  * A step's inputs are copied in (cp.async) during the step before it, into a ring of three
+//    buffers, so that a forward step needs no barrier at its top: the copy it reads was waited
+//    for before the last barrier of the step before, and the buffer it refills was last read two
+//    steps ago.
 // ---------------------------------------------------------------------------------------------
 constexpr int kSB = TTT_D + 8;  // row stride (bf16 elements) of the staged input tiles: 144 bytes
+constexpr int kSW = TTT_D + 8;  // row stride (floats) of W^T in shared memory
+constexpr int kStages = 3;      // staged steps in flight
 
 struct __align__(16) BwdTcSmem {
-    float W[TTT_D][kS];
+    float WT[TTT_D][kSW];  // W^T, [output feature][input feature], for the backward steps
     float dW[TTT_D][kS];
     float g[TTT_KMAX][kS];
     float dzb[TTT_KMAX][kS];
@@ -499,6 +514,7 @@ struct __align__(16) BwdTcSmem {
     float P0[TTT_KMAX][kS];  // product results
     float P1[TTT_KMAX][kS];
     float P2[TTT_KMAX][kS];
+    float Zp[TTT_KMAX][kS];  // a forward step's Z over inputs 32..63 (P2 holds it over 0..31)
     float A[TTT_KMAX][kS16];
     float M[TTT_KMAX][kS16];
     float MT[TTT_KMAX][kS16];
@@ -511,8 +527,8 @@ struct __align__(16) BwdTcSmem {
     float dlr_row[TTT_KMAX];
     // each step's inputs, copied in while the step before runs: [buffer][XQ, XK, XV, d_out]; the
     // MMAs and dot products read XQ and XK from here (bf16 values are exact TF32 operands)
-    __nv_bfloat16 stage[2][4][TTT_KMAX][kSB];
-    float stage_lr[2][TTT_KMAX];
+    __nv_bfloat16 stage[kStages][4][TTT_KMAX][kSB];
+    float stage_lr[kStages][TTT_KMAX];
 };
 
 // 16- and 4-byte cp.async with zero fill: src_bytes = size copies, 0 writes zeros without reading.
@@ -545,8 +561,15 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1
 // A TF32 operand from fp32 (rounded to nearest) or from bf16 (exact: the bits moved up).
 __device__ __forceinline__ uint32_t op32(float x) { return tf32(x); }
 __device__ __forceinline__ uint32_t op32(__nv_bfloat16 x) { return static_cast<uint32_t>(__bfloat16_as_ushort(x)) << 16; }
-__device__ __forceinline__ float f32(float x) { return x; }
 __device__ __forceinline__ float f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+// The two TF32 operands in a pair of bf16 values (low half: the first element).
+__device__ __forceinline__ uint32_t bf_lo(uint32_t p) { return p << 16; }
+__device__ __forceinline__ uint32_t bf_hi(uint32_t p) { return p & 0xffff0000u; }
+__device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+// 8-byte cp.async (the source and destination 8-byte aligned).
+__device__ __forceinline__ void cp_async_8(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 
 // acc += sum_{k < K} X[m][k] Y(k, n0 + n) for the 16 x 8 tile at columns n0: X rows of stride kSX;
 // Y(k, n) = Ymat[k][n], or Ymat[n][k] when kTrans (rows of stride kSY).  Even and odd k-steps
@@ -569,9 +592,9 @@ __device__ __forceinline__ void tc_tile(float (&acc)[4], const TX (*X)[kSX], con
 }
 
 // c0 += X0 Y and c1 += X1 Y over K = 64 for the tile at columns n0, sharing Y's fragments.
-template <bool kTrans, typename TX, int kSX>
+template <bool kTrans, typename TX, int kSX, int kSY>
 __device__ __forceinline__ void tc_tile2(float (&c0)[4], float (&c1)[4], const TX (*X0)[kSX], const TX (*X1)[kSX],
-                                         const float (*Y)[kS], int n0, int g, int t) {
+                                         const float (*Y)[kSY], int n0, int g, int t) {
 #pragma unroll
     for (int k0 = 0; k0 < TTT_D; k0 += 8) {
         const uint32_t b0 = tf32(kTrans ? Y[n0 + g][k0 + t] : Y[k0 + t][n0 + g]);
@@ -580,6 +603,23 @@ __device__ __forceinline__ void tc_tile2(float (&c0)[4], float (&c1)[4], const T
                  b0, b1);
         mma_tf32(c1, op32(X1[g][k0 + t]), op32(X1[g + 8][k0 + t]), op32(X1[g][k0 + t + 4]), op32(X1[g + 8][k0 + t + 4]),
                  b0, b1);
+    }
+}
+
+// c0 += X0 W and c1 += X1 W over K = 64 for the tile at columns n0, X0 and X1 bf16 tiles and W
+// given as W^T: the k slots t and t + 4 of each MMA step stand for the inputs k0 + 2t and
+// k0 + 2t + 1, so each operand pair is one 32-bit load of X and one 64-bit load of W^T.
+__device__ __forceinline__ void tc_tile2_wt(float (&c0)[4], float (&c1)[4], const __nv_bfloat16 (*X0)[kSB],
+                                            const __nv_bfloat16 (*X1)[kSB], const float (*WT)[kSW], int n0, int g,
+                                            int t) {
+#pragma unroll
+    for (int k0 = 0; k0 < TTT_D; k0 += 8) {
+        const float2 w2 = *reinterpret_cast<const float2*>(&WT[n0 + g][k0 + 2 * t]);
+        const uint32_t b0 = tf32(w2.x), b1 = tf32(w2.y);
+        const uint32_t p0 = ld_pair(&X0[g][k0 + 2 * t]), p1 = ld_pair(&X0[g + 8][k0 + 2 * t]);
+        const uint32_t q0 = ld_pair(&X1[g][k0 + 2 * t]), q1 = ld_pair(&X1[g + 8][k0 + 2 * t]);
+        mma_tf32(c0, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), b0, b1);
+        mma_tf32(c1, bf_lo(q0), bf_lo(q1), bf_hi(q0), bf_hi(q1), b0, b1);
     }
 }
 
@@ -620,7 +660,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int r = tid >> 4, c0 = 4 * (tid & 15);       // row layout: this thread's row and four features
-    const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);    // this warp's block of a 64 x 64 matrix
+    const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);    // this warp's block of dW
+    const int ni = 16 * (w & 3), kh = 32 * (w >> 2);    // this warp's block of W^T (outputs, inputs)
     const int nt = 8 * w;                               // this warp's columns of a 16 x 64 product
     const long long chain = blockIdx.x;
     const int h = static_cast<int>(chain % a.H);
@@ -672,9 +713,26 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             *reinterpret_cast<float2*>(&dst[m0 + g + 8][n0 + 8 * q + 2 * t]) = make_float2(acc[q][2], acc[q][3]);
         }
     };
+    // W^T in accumulators: tile j holds W[k][n] for inputs k = kh + 8j + 2t (elements 0, 2) and
+    // k + 1 (1, 3), outputs n = ni + g (0, 1) and ni + g + 8 (2, 3)
     float Wacc[4][4], dWacc[4][4];
-    load_acc(Wacc, W0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float* p = W0 + (kh + 8 * j + 2 * t) * TTT_D + ni + g;
+        Wacc[j][0] = p[0];
+        Wacc[j][1] = p[TTT_D];
+        Wacc[j][2] = p[8];
+        Wacc[j][3] = p[TTT_D + 8];
+    }
     if (tid < TTT_D) s.b[tid] = b0[tid];
+    // W^T into shared memory (each thread its own elements), for a backward step
+    auto publish_w = [&]() {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            *reinterpret_cast<float2*>(&s.WT[ni + g][kh + 8 * j + 2 * t]) = make_float2(Wacc[j][0], Wacc[j][1]);
+            *reinterpret_cast<float2*>(&s.WT[ni + g + 8][kh + 8 * j + 2 * t]) = make_float2(Wacc[j][2], Wacc[j][3]);
+        }
+    };
     // a state in the workspace: each thread's sixteen accumulators (its own layout), b from tid < 64
     auto save_state = [&](float* dst) {
 #pragma unroll
@@ -688,6 +746,16 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             Wacc[q][0] = v.x; Wacc[q][1] = v.y; Wacc[q][2] = v.z; Wacc[q][3] = v.w;
         }
         if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
+    };
+    // a saved state straight into s.WT and s.b, asynchronously (what publish_w would write after
+    // load_state): each thread copies the pairs it saved
+    auto fetch_state = [&](const float* src) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            cp_async_8(&s.WT[ni + g][kh + 8 * j + 2 * t], src + tid * 16 + 4 * j);
+            cp_async_8(&s.WT[ni + g + 8][kh + 8 * j + 2 * t], src + tid * 16 + 4 * j + 2);
+        }
+        if (tid < TTT_D) cp_async_4z(&s.b[tid], src + TTT_D * TTT_D + tid, 4u);
     };
 
     // The inputs of the step at t0 (Km tokens) into staging buffer buf, asynchronously: XK and XV
@@ -718,27 +786,34 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         long long t0;
         int Km;
     };
+    auto next_buf = [](int b) { return b == kStages - 1 ? 0 : b + 1; };
     auto start_next = [&](int buf, const Next& nx) {
-        if (nx.kind) prefetch(buf ^ 1, nx.t0, nx.Km, nx.kind == 2);
+        if (nx.kind) prefetch(next_buf(buf), nx.t0, nx.Km, nx.kind == 2);
     };
 
-    // One full mini-batch of the forward state recursion (W in Wacc and s.W, b in s.b), its inputs
-    // in staging buffer buf.
+    // One full mini-batch of the forward state recursion (W^T in Wacc, b in s.b), its inputs in
+    // staging buffer buf (copied and waited for during the step before).
     auto fwd_step = [&](long long t0, int buf, const Next& nx) {
         const bool live = r < K;
-        cp_async_wait_all();
-        __syncthreads();  // the staged inputs have landed, and the last step's readers of the tiles are done
         const float4 k4 = staged(buf, 1), v4 = staged(buf, 2);
         const __nv_bfloat16 (*xk)[kSB] = s.stage[buf][1];
         const float* lrs = s.stage_lr[buf];
         start_next(buf, nx);
-        {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile<TTT_D, false>(c, xk, s.W, nt, g, t);
-            put_tile(s.P0, c, nt, g, t);
+        {  // Z over this warp's inputs kh .. kh + 31, at outputs ni .. ni + 15
+            float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k0 = kh + 8 * j;
+                const uint32_t p0 = ld_pair(&xk[g][k0 + 2 * t]), p1 = ld_pair(&xk[g + 8][k0 + 2 * t]);
+                mma_tf32(z0, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), tf32(Wacc[j][0]), tf32(Wacc[j][1]));
+                mma_tf32(z1, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), tf32(Wacc[j][2]), tf32(Wacc[j][3]));
+            }
+            float (*Pz)[kS] = kh ? s.Zp : s.P2;
+            put_tile(Pz, z0, ni, g, t);
+            put_tile(Pz, z1, ni + 8, g, t);
         }
         __syncthreads();
-        const float4 z = ld4(&s.P0[r][c0]) + ld4(&s.b[c0]);
+        const float4 z = ld4(&s.P2[r][c0]) + ld4(&s.Zp[r][c0]) + ld4(&s.b[c0]);
         float4 xh;
         float sig;
         row_norm(z, eps, xh, sig);
@@ -746,24 +821,39 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
         const float4 gv = live ? (q - f4(mq) - xh * mqx) * (1.0f / sig) : f4(0.f);
         st4(&s.g[r][c0], gv);
+        cp_async_wait_all();  // the next step's inputs, copied since this step began
         __syncthreads();
         const float tl = s.te[K - 1];
-        tc_rank16(Wacc, xk, lrs, -tl, s.g, m0, n0, g, t);
-        if (tid < TTT_D) {
+        {  // W^T += (-tl lr g)^T XK over the tokens as k: token pairs 2t, 2t + 1 fill the slots t, t + 4
+            uint32_t xb[2][4];
+            ldmatrix_x4_trans(smem_u32(&xk[lane & 7][kh + 8 * (lane >> 3)]), xb[0][0], xb[0][1], xb[0][2], xb[0][3]);
+            ldmatrix_x4_trans(smem_u32(&xk[8 + (lane & 7)][kh + 8 * (lane >> 3)]), xb[1][0], xb[1][1], xb[1][2],
+                              xb[1][3]);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int j0 = 8 * hf + 2 * t;
+                const float se = -tl * lrs[j0], so = -tl * lrs[j0 + 1];
+                const uint32_t a0 = tf32(se * s.g[j0][ni + g]), a1 = tf32(se * s.g[j0][ni + g + 8]);
+                const uint32_t a2 = tf32(so * s.g[j0 + 1][ni + g]), a3 = tf32(so * s.g[j0 + 1][ni + g + 8]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) mma_tf32(Wacc[j], a0, a1, a2, a3, bf_lo(xb[hf][j]), bf_hi(xb[hf][j]));
+            }
+        }
+        if (tid < TTT_D) {  // rows past K hold zeros (g and the zero-filled lr): the fixed bound adds nothing
             float acc = 0.f;
-            for (int i = 0; i < K; ++i) acc = fmaf(tl * lrs[i], s.g[i][tid], acc);
+#pragma unroll
+            for (int i = 0; i < TTT_KMAX; ++i) acc = fmaf(tl * lrs[i], s.g[i][tid], acc);
             s.b[tid] -= acc;
         }
-        // the Z product, W's only reader, finished before the last barrier; each thread writes its own
-        // elements, and the next step rewrites xk, g and lr only after its first barrier
-        put_acc(s.W, Wacc);
     };
 
     float4 dgam = f4(0.f), dbet = f4(0.f);
 
     // The backward step of the mini-batch at t0 (as in linear_bwd_kernel), with its start state in
-    // Wacc / s.W / s.b, the adjoint after it in dWacc / s.dW / s.db, its inputs in staging buffer buf.
-    auto bwd_step = [&](long long t0, int Km, bool full, int buf, const Next& nx) {
+    // s.WT / s.b, the adjoint after it in dWacc / s.dW / s.db, its inputs in staging buffer buf;
+    // next_state (or null): the saved start state of the step after, copied into s.WT and s.b
+    // once this step has no more use for them.
+    auto bwd_step = [&](long long t0, int Km, bool full, int buf, const Next& nx, const float* next_state) {
         const bool live = r < Km;
         const long long row = (t0 + r) * ts + c0;
         cp_async_wait_all();
@@ -775,7 +865,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         start_next(buf, nx);
         {  // XK W and XQ W, sharing W's fragments
             float cz[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile2<false>(cz, cb, xk, xq, s.W, nt, g, t);
+            tc_tile2_wt(cz, cb, xk, xq, s.WT, nt, g, t);
             put_tile(s.P0, cz, nt, g, t);
             put_tile(s.P1, cb, nt, g, t);
         }
@@ -867,7 +957,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         __syncthreads();  // (7)
         {  // dZbar W^T + dA XK and dZ W^T + dA^T XQ; the adjoint of the start state
             float cq[4] = {0.f, 0.f, 0.f, 0.f}, ck[4] = {0.f, 0.f, 0.f, 0.f};
-            tc_tile2<true>(cq, ck, s.dzb, s.dz, s.W, nt, g, t);
+            tc_tile2<false>(cq, ck, s.dzb, s.dz, s.WT, nt, g, t);
             tc_tile<TTT_KMAX, false>(cq, s.dA, xk, nt, g, t);
             tc_tile<TTT_KMAX, false>(ck, s.dAT, xq, nt, g, t);
             put_tile(s.P0, cq, nt, g, t);
@@ -875,7 +965,9 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             tc_rank16(dWacc, xq, nullptr, 1.f, s.dzb, m0, n0, g, t);
             tc_rank16(dWacc, xk, nullptr, 1.f, s.dz, m0, n0, g, t);
         }
-        __syncthreads();  // (8)
+        cp_async_wait_all();  // the next step's inputs (a forward step after this one has no barrier at its top)
+        __syncthreads();      // (8)
+        if (next_state) fetch_state(next_state);  // s.WT's and s.b's readers are done
         if (live) {
             st4(dXQ + row, o4 + ld4(&s.P0[r][c0]));
             st4(dXK + row, dxk + ld4(&s.P1[r][c0]));
@@ -905,13 +997,14 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     int buf = 0;
 
     // ---- phase 1: the forward state recursion, a checkpoint every G full mini-batches --------
-    put_acc(s.W, Wacc);
     if (n_full > 0) prefetch(0, 0, K, false);
     else if (after_phase1.kind) prefetch(0, after_phase1.t0, after_phase1.Km, after_phase1.kind == 2);
+    cp_async_wait_all();
+    __syncthreads();  // the first step's inputs, b and the step coefficients in place for every thread
     for (long long m = 0; m < n_full; ++m) {
         if (m % G == 0) save_state(a.ckpt + (chain * a.n_ckpt + m / G) * kState);
         fwd_step(m * K, buf, m + 1 < n_full ? Next{1, (m + 1) * K, K} : after_phase1);
-        buf ^= 1;
+        buf = next_buf(buf);
     }
 
     // ---- the remainder tail, from the state after the full mini-batches -----------------------
@@ -924,30 +1017,28 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     if (tid < TTT_D) s.db[tid] = a.db_last ? a.db_last[chain * TTT_D + tid] : 0.f;
     put_acc(s.dW, dWacc);
     if (rem > 0) {
-        bwd_step(n_full * K, rem, false, buf, after_tail);
-        buf ^= 1;
+        publish_w();  // s.WT's last readers passed barriers long ago; the step's first barrier orders the rest
+        bwd_step(n_full * K, rem, false, buf, after_tail, nullptr);
+        buf = next_buf(buf);
     }
 
     // ---- phase 2: the groups from the last; rebuild each one's states, then step back ----------
     float* const slab = a.slab + chain * G * kState;
     for (long long c = a.n_ckpt - 1; c >= 0; --c) {
         const long long m0g = c * G, m1g = m0g + G < n_full ? m0g + G : n_full;
-        // no barrier: s.b's readers and s.W's readers of the last step passed its later barriers,
-        // and each thread rewrites only its own elements
+        // no barrier: s.b's readers of the last step passed its later barriers, and each thread
+        // rewrites only its own elements
         load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
-        put_acc(s.W, Wacc);
-        for (long long m = m0g; m < m1g; ++m) {
+        for (long long m = m0g; m + 1 < m1g; ++m) {  // the group's states but its last, kept in the slab
             save_state(slab + (m - m0g) * kState);
-            if (m + 1 < m1g) {
-                fwd_step(m * K, buf, m + 2 < m1g ? Next{1, (m + 1) * K, K} : Next{2, (m1g - 1) * K, K});
-                buf ^= 1;
-            }
+            fwd_step(m * K, buf, m + 2 < m1g ? Next{1, (m + 1) * K, K} : Next{2, (m1g - 1) * K, K});
+            buf = next_buf(buf);
         }
+        publish_w();  // the last state of the group is the first one its backward steps need
         for (long long m = m1g - 1; m >= m0g; --m) {
-            load_state(slab + (m - m0g) * kState);  // (no barrier, as above)
-            put_acc(s.W, Wacc);
-            bwd_step(m * K, K, true, buf, m > m0g ? Next{2, (m - 1) * K, K} : (c > 0 ? group_first(c - 1) : Next{0, 0, 0}));
-            buf ^= 1;
+            bwd_step(m * K, K, true, buf, m > m0g ? Next{2, (m - 1) * K, K} : (c > 0 ? group_first(c - 1) : Next{0, 0, 0}),
+                     m > m0g ? slab + (m - 1 - m0g) * kState : nullptr);
+            buf = next_buf(buf);
         }
     }
 
