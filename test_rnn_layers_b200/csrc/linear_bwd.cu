@@ -126,26 +126,6 @@ __device__ __forceinline__ float dot64(const float* p, const float* q) {
     return a0 + a1;
 }
 
-// dot64 of two bf16 rows (16-byte aligned), in the same order of accumulation.
-__device__ __forceinline__ float dot64_bf16(const __nv_bfloat16* p, const __nv_bfloat16* q) {
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll 2
-    for (int f = 0; f < TTT_D; f += 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(p + f), v = *reinterpret_cast<const uint4*>(q + f);
-        const uint32_t us[4] = {u.x, u.y, u.z, u.w}, vs[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; i += 2) {
-            const float2 x0 = unpack_bf16x2(us[i]), y0 = unpack_bf16x2(vs[i]);
-            const float2 x1 = unpack_bf16x2(us[i + 1]), y1 = unpack_bf16x2(vs[i + 1]);
-            a0 = fmaf(x0.x, y0.x, a0);
-            a1 = fmaf(x0.y, y0.y, a1);
-            a0 = fmaf(x1.x, y1.x, a0);
-            a1 = fmaf(x1.y, y1.y, a1);
-        }
-    }
-    return a0 + a1;
-}
-
 // LayerNorm statistics of a row whose four features z this thread holds: x_hat and sigma.
 __device__ __forceinline__ void row_norm(float4 z, float eps, float4& xh, float& sigma) {
     const float mu = row_sum(hsum4(z)) * (1.0f / TTT_D);
@@ -491,8 +471,9 @@ __global__ void linear_bwd_copy_kernel(const float* part, long long chains, floa
 //    the LayerNorm's row exchange) and takes XK as bf16 pairs, one 32-bit load for two operands.
 //    The update W^T += (-t lr g)^T XK accumulates into the same registers, XK arriving by
 //    transposing ldmatrix loads.  W^T is written to shared memory only for the backward steps.
-//  * The adjoint dW lives as accumulators too, warp w holding rows 16 (w / 2) .. +15 and columns
-//    32 (w % 2) .. +31 (four 16 x 8 tiles); its shared copy serves as a B operand.
+//  * The adjoint dW lives in the same layout (dW^T accumulators); its updates dW^T += dZbar^T XQ
+//    + dZ^T XK take XQ and XK by transposing ldmatrix loads as well, and its shared copy (dW^T)
+//    is a B operand of the next step's products.
 //  * A 16 x 64 product of a backward step lands in a shared result tile, warp w computing columns
 //    8w .. 8w + 7, and the row-layout threads read it back.  The LayerNorm work and the 16 x 16
 //    products are as above.
@@ -507,7 +488,7 @@ constexpr int kStages = 3;      // staged steps in flight
 
 struct __align__(16) BwdTcSmem {
     float WT[TTT_D][kSW];  // W^T, [output feature][input feature], for the backward steps
-    float dW[TTT_D][kS];
+    float dWT[TTT_D][kSW];  // dW^T, likewise
     float g[TTT_KMAX][kS];
     float dzb[TTT_KMAX][kS];
     float dz[TTT_KMAX][kS];
@@ -561,7 +542,6 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], uint32_t a0, uint32_t a1
 // A TF32 operand from fp32 (rounded to nearest) or from bf16 (exact: the bits moved up).
 __device__ __forceinline__ uint32_t op32(float x) { return tf32(x); }
 __device__ __forceinline__ uint32_t op32(__nv_bfloat16 x) { return static_cast<uint32_t>(__bfloat16_as_ushort(x)) << 16; }
-__device__ __forceinline__ float f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 // The two TF32 operands in a pair of bf16 values (low half: the first element).
 __device__ __forceinline__ uint32_t bf_lo(uint32_t p) { return p << 16; }
 __device__ __forceinline__ uint32_t bf_hi(uint32_t p) { return p & 0xffff0000u; }
@@ -623,34 +603,45 @@ __device__ __forceinline__ void tc_tile2_wt(float (&c0)[4], float (&c1)[4], cons
     }
 }
 
+// c += X W over K = 64 for the tile at columns n0, as tc_tile2_wt with one operand.
+__device__ __forceinline__ void tc_tile_wt(float (&c)[4], const __nv_bfloat16 (*X)[kSB], const float (*WT)[kSW], int n0,
+                                           int g, int t) {
+    float odd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k0 = 0; k0 < TTT_D; k0 += 8) {
+        const float2 w2 = *reinterpret_cast<const float2*>(&WT[n0 + g][k0 + 2 * t]);
+        const uint32_t p0 = ld_pair(&X[g][k0 + 2 * t]), p1 = ld_pair(&X[g + 8][k0 + 2 * t]);
+        if ((k0 >> 3) & 1) mma_tf32(odd, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), tf32(w2.x), tf32(w2.y));
+        else mma_tf32(c, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), tf32(w2.x), tf32(w2.y));
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[e] += odd[e];
+}
+
+// acc (a matrix's transpose in the W^T accumulator layout: tile j at rows ni .. ni + 15, columns
+// kh + 8j .. + 7) += sum over the 16 tokens j of s_j Gm[j][n] X[j][k], s_j = scale * lr[j] (lr
+// non-null) or 1: the rank-16 update of a state or its adjoint by a mini-batch.  The token pairs
+// 2t, 2t + 1 fill the k slots t, t + 4; X (bf16) arrives by transposing ldmatrix loads.
+__device__ __forceinline__ void tc_rank16_t(float (&acc)[4][4], const float (*Gm)[kS], const float* lr, float scale,
+                                            const __nv_bfloat16 (*X)[kSB], int ni, int kh, int lane, int g, int t) {
+    uint32_t xb[2][4];
+    ldmatrix_x4_trans(smem_u32(&X[lane & 7][kh + 8 * (lane >> 3)]), xb[0][0], xb[0][1], xb[0][2], xb[0][3]);
+    ldmatrix_x4_trans(smem_u32(&X[8 + (lane & 7)][kh + 8 * (lane >> 3)]), xb[1][0], xb[1][1], xb[1][2], xb[1][3]);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const int j0 = 8 * hf + 2 * t;
+        const float se = lr ? scale * lr[j0] : 1.f, so = lr ? scale * lr[j0 + 1] : 1.f;
+        const uint32_t a0 = tf32(se * Gm[j0][ni + g]), a1 = tf32(se * Gm[j0][ni + g + 8]);
+        const uint32_t a2 = tf32(so * Gm[j0 + 1][ni + g]), a3 = tf32(so * Gm[j0 + 1][ni + g + 8]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_tf32(acc[j], a0, a1, a2, a3, bf_lo(xb[hf][j]), bf_hi(xb[hf][j]));
+    }
+}
+
 // A 16 x 8 accumulator tile into rows 0..15, columns n0..n0+7 of a result tile.
 __device__ __forceinline__ void put_tile(float (*P)[kS], const float (&c)[4], int n0, int g, int t) {
     *reinterpret_cast<float2*>(&P[g][n0 + 2 * t]) = make_float2(c[0], c[1]);
     *reinterpret_cast<float2*>(&P[g + 8][n0 + 2 * t]) = make_float2(c[2], c[3]);
-}
-
-// acc (this warp's four 16 x 8 tiles of a 64 x 64 matrix at rows m0, columns n0 + 8q) +=
-// sum_{j < 16} s_j X[j][m] Y[j][n]: the rank-16 update by the tokens of a mini-batch, with
-// s_j = scale * lr[j] (lr non-null) or 1.
-template <typename TX, int kSX>
-__device__ __forceinline__ void tc_rank16(float (&acc)[4][4], const TX (*X)[kSX], const float* lr, float scale,
-                                          const float (*Y)[kS], int m0, int n0, int g, int t) {
-#pragma unroll
-    for (int k0 = 0; k0 < TTT_KMAX; k0 += 8) {
-        float x0 = f32(X[k0 + t][m0 + g]), x1 = f32(X[k0 + t][m0 + g + 8]);
-        float x2 = f32(X[k0 + t + 4][m0 + g]), x3 = f32(X[k0 + t + 4][m0 + g + 8]);
-        if (lr) {
-            const float s0 = scale * lr[k0 + t], s1 = scale * lr[k0 + t + 4];
-            x0 *= s0;
-            x1 *= s0;
-            x2 *= s1;
-            x3 *= s1;
-        }
-        const uint32_t a0 = tf32(x0), a1 = tf32(x1), a2 = tf32(x2), a3 = tf32(x3);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            mma_tf32(acc[q], a0, a1, a2, a3, tf32(Y[k0 + t][n0 + 8 * q + g]), tf32(Y[k0 + t + 4][n0 + 8 * q + g]));
-    }
 }
 
 template <typename T>
@@ -660,8 +651,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int r = tid >> 4, c0 = 4 * (tid & 15);       // row layout: this thread's row and four features
-    const int m0 = 16 * (w >> 1), n0 = 32 * (w & 1);    // this warp's block of dW
-    const int ni = 16 * (w & 3), kh = 32 * (w >> 2);    // this warp's block of W^T (outputs, inputs)
+    const int ni = 16 * (w & 3), kh = 32 * (w >> 2);    // this warp's block of W^T and dW^T (outputs, inputs)
     const int nt = 8 * w;                               // this warp's columns of a 16 x 64 product
     const long long chain = blockIdx.x;
     const int h = static_cast<int>(chain % a.H);
@@ -689,50 +679,42 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     const float* W0 = a.W0 + (a.w0_chain_stride ? chain * a.w0_chain_stride : static_cast<long long>(h) * TTT_D * TTT_D);
     const float* b0 = a.b0 + (a.w0_chain_stride ? chain * TTT_D : static_cast<long long>(h) * TTT_D);
 
-    // this warp's tiles of a [k][f] matrix in memory <-> accumulators: tile q holds rows m0 + g
-    // (elements 0, 1) and m0 + g + 8 (elements 2, 3), columns n0 + 8q + 2t, + 1
+    // A [k][n] matrix in memory <-> accumulators in the W^T layout: tile j holds entry (k, n) for
+    // inputs k = kh + 8j + 2t (elements 0, 2) and k + 1 (1, 3), outputs n = ni + g (0, 1) and
+    // ni + g + 8 (2, 3).
     auto load_acc = [&](float (&acc)[4][4], const float* src) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float2 u = *reinterpret_cast<const float2*>(src + (m0 + g) * TTT_D + n0 + 8 * q + 2 * t);
-            const float2 v = *reinterpret_cast<const float2*>(src + (m0 + g + 8) * TTT_D + n0 + 8 * q + 2 * t);
-            acc[q][0] = u.x; acc[q][1] = u.y; acc[q][2] = v.x; acc[q][3] = v.y;
+        for (int j = 0; j < 4; ++j) {
+            const float* p = src + (kh + 8 * j + 2 * t) * TTT_D + ni + g;
+            acc[j][0] = p[0];
+            acc[j][1] = p[TTT_D];
+            acc[j][2] = p[8];
+            acc[j][3] = p[TTT_D + 8];
         }
     };
     auto store_acc = [&](float* dst, const float (&acc)[4][4]) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            *reinterpret_cast<float2*>(dst + (m0 + g) * TTT_D + n0 + 8 * q + 2 * t) = make_float2(acc[q][0], acc[q][1]);
-            *reinterpret_cast<float2*>(dst + (m0 + g + 8) * TTT_D + n0 + 8 * q + 2 * t) = make_float2(acc[q][2], acc[q][3]);
+        for (int j = 0; j < 4; ++j) {
+            float* p = dst + (kh + 8 * j + 2 * t) * TTT_D + ni + g;
+            p[0] = acc[j][0];
+            p[TTT_D] = acc[j][1];
+            p[8] = acc[j][2];
+            p[TTT_D + 8] = acc[j][3];
         }
     };
-    auto put_acc = [&](float (*dst)[kS], const float (&acc)[4][4]) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            *reinterpret_cast<float2*>(&dst[m0 + g][n0 + 8 * q + 2 * t]) = make_float2(acc[q][0], acc[q][1]);
-            *reinterpret_cast<float2*>(&dst[m0 + g + 8][n0 + 8 * q + 2 * t]) = make_float2(acc[q][2], acc[q][3]);
-        }
-    };
-    // W^T in accumulators: tile j holds W[k][n] for inputs k = kh + 8j + 2t (elements 0, 2) and
-    // k + 1 (1, 3), outputs n = ni + g (0, 1) and ni + g + 8 (2, 3)
-    float Wacc[4][4], dWacc[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float* p = W0 + (kh + 8 * j + 2 * t) * TTT_D + ni + g;
-        Wacc[j][0] = p[0];
-        Wacc[j][1] = p[TTT_D];
-        Wacc[j][2] = p[8];
-        Wacc[j][3] = p[TTT_D + 8];
-    }
-    if (tid < TTT_D) s.b[tid] = b0[tid];
-    // W^T into shared memory (each thread its own elements), for a backward step
-    auto publish_w = [&]() {
+    // the transpose into shared memory ([n][k]), each thread its own elements
+    auto put_t = [&](float (*dst)[kSW], const float (&acc)[4][4]) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            *reinterpret_cast<float2*>(&s.WT[ni + g][kh + 8 * j + 2 * t]) = make_float2(Wacc[j][0], Wacc[j][1]);
-            *reinterpret_cast<float2*>(&s.WT[ni + g + 8][kh + 8 * j + 2 * t]) = make_float2(Wacc[j][2], Wacc[j][3]);
+            *reinterpret_cast<float2*>(&dst[ni + g][kh + 8 * j + 2 * t]) = make_float2(acc[j][0], acc[j][1]);
+            *reinterpret_cast<float2*>(&dst[ni + g + 8][kh + 8 * j + 2 * t]) = make_float2(acc[j][2], acc[j][3]);
         }
     };
+    // the state W and the adjoint dW, as W^T and dW^T
+    float Wacc[4][4], dWacc[4][4];
+    load_acc(Wacc, W0);
+    if (tid < TTT_D) s.b[tid] = b0[tid];
+    auto publish_w = [&]() { put_t(s.WT, Wacc); };  // for a backward step
     // a state in the workspace: each thread's sixteen accumulators (its own layout), b from tid < 64
     auto save_state = [&](float* dst) {
 #pragma unroll
@@ -824,21 +806,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         cp_async_wait_all();  // the next step's inputs, copied since this step began
         __syncthreads();
         const float tl = s.te[K - 1];
-        {  // W^T += (-tl lr g)^T XK over the tokens as k: token pairs 2t, 2t + 1 fill the slots t, t + 4
-            uint32_t xb[2][4];
-            ldmatrix_x4_trans(smem_u32(&xk[lane & 7][kh + 8 * (lane >> 3)]), xb[0][0], xb[0][1], xb[0][2], xb[0][3]);
-            ldmatrix_x4_trans(smem_u32(&xk[8 + (lane & 7)][kh + 8 * (lane >> 3)]), xb[1][0], xb[1][1], xb[1][2],
-                              xb[1][3]);
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int j0 = 8 * hf + 2 * t;
-                const float se = -tl * lrs[j0], so = -tl * lrs[j0 + 1];
-                const uint32_t a0 = tf32(se * s.g[j0][ni + g]), a1 = tf32(se * s.g[j0][ni + g + 8]);
-                const uint32_t a2 = tf32(so * s.g[j0 + 1][ni + g]), a3 = tf32(so * s.g[j0 + 1][ni + g + 8]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) mma_tf32(Wacc[j], a0, a1, a2, a3, bf_lo(xb[hf][j]), bf_hi(xb[hf][j]));
-            }
-        }
+        tc_rank16_t(Wacc, s.g, lrs, -tl, xk, ni, kh, lane, g, t);  // W^T += (-tl lr g)^T XK
         if (tid < TTT_D) {  // rows past K hold zeros (g and the zero-filled lr): the fixed bound adds nothing
             float acc = 0.f;
 #pragma unroll
@@ -850,7 +818,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     float4 dgam = f4(0.f), dbet = f4(0.f);
 
     // The backward step of the mini-batch at t0 (as in linear_bwd_kernel), with its start state in
-    // s.WT / s.b, the adjoint after it in dWacc / s.dW / s.db, its inputs in staging buffer buf;
+    // s.WT / s.b, the adjoint after it in dWacc / s.dWT / s.db, its inputs in staging buffer buf;
     // next_state (or null): the saved start state of the step after, copied into s.WT and s.b
     // once this step has no more use for them.
     auto bwd_step = [&](long long t0, int Km, bool full, int buf, const Next& nx, const float* next_state) {
@@ -869,13 +837,25 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             put_tile(s.P0, cz, nt, g, t);
             put_tile(s.P1, cb, nt, g, t);
         }
-        {  // A = XQ XK^T and M = eta * tril(A + 1) at (i, j) = (r, tid % 16)
-            const int i = r, j = tid & 15;
-            const float av = dot64_bf16(xq[i], xk[j]);
-            const float m = (j <= i && i < Km) ? s.te[i] * lrs[j] * (av + 1.0f) : 0.f;
-            s.A[i][j] = av;
-            s.M[i][j] = m;
-            s.MT[j][i] = m;
+        if (w < 2) {  // A = XQ XK^T at columns 8w .. 8w + 7 (bf16 products are exact), and M = eta * tril(A + 1)
+            float ca[4] = {0.f, 0.f, 0.f, 0.f}, odd[4] = {0.f, 0.f, 0.f, 0.f};
+            const int j0 = 8 * w;
+#pragma unroll
+            for (int k0 = 0; k0 < TTT_D; k0 += 8) {
+                const uint32_t p0 = ld_pair(&xq[g][k0 + 2 * t]), p1 = ld_pair(&xq[g + 8][k0 + 2 * t]);
+                const uint32_t kb = ld_pair(&xk[j0 + g][k0 + 2 * t]);
+                if ((k0 >> 3) & 1) mma_tf32(odd, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), bf_lo(kb), bf_hi(kb));
+                else mma_tf32(ca, bf_lo(p0), bf_lo(p1), bf_hi(p0), bf_hi(p1), bf_lo(kb), bf_hi(kb));
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {  // element (i, j): i = g (+ 8), j = j0 + 2t (+ 1)
+                const int i = g + 8 * (e >> 1), j = j0 + 2 * t + (e & 1);
+                const float av = ca[e] + odd[e];
+                const float m = (j <= i && i < Km) ? s.te[i] * lrs[j] * (av + 1.0f) : 0.f;
+                s.A[i][j] = av;
+                s.M[i][j] = m;
+                s.MT[j][i] = m;
+            }
         }
         __syncthreads();  // (2)
         const float4 bb = ld4(&s.b[c0]);
@@ -896,8 +876,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             put_tile(s.P0, cm, nt, g, t);
             if (full) {
                 float cu[4] = {0.f, 0.f, 0.f, 0.f}, cv[4] = {0.f, 0.f, 0.f, 0.f};
-                tc_tile<TTT_D, false>(cu, xk, s.dW, nt, g, t);
-                tc_tile<TTT_D, true>(cv, s.g, s.dW, nt, g, t);
+                tc_tile_wt(cu, xk, s.dWT, nt, g, t);
+                tc_tile<TTT_D, false>(cv, s.g, s.dWT, nt, g, t);
                 put_tile(s.P1, cu, nt, g, t);
                 put_tile(s.P2, cv, nt, g, t);
             }
@@ -920,13 +900,37 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             tc_tile<TTT_KMAX, false>(cg, s.MT, s.dzb, nt, g, t);
             put_tile(s.P0, cg, nt, g, t);
         }
-        {  // dM = -dZbar g^T on the lower triangle: its shares of dA and of dlr
-            const int i = r, j = tid & 15;
-            const float dm = (j <= i && i < Km) ? -dot64(s.dzb[i], s.g[j]) : 0.f;
-            s.dlr_eta[i][j] = s.te[i] * (s.A[i][j] + 1.0f) * dm;
-            const float da = dm * s.te[i] * lrs[j];
-            s.dA[i][j] = da;
-            s.dAT[j][i] = da;
+        if (w < 2) {  // dM = -dZbar g^T at columns 8w .. 8w + 7, lower triangle: its shares of dA and of dlr
+            // three TF32 products per step (hi hi + hi lo + lo hi, each operand split in two TF32
+            // parts), close to fp32 products
+            float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
+            const int j0 = 8 * w;
+            auto split = [](float x, uint32_t& hi, uint32_t& lo) {
+                hi = tf32(x);
+                lo = tf32(x - __uint_as_float(hi));
+            };
+#pragma unroll
+            for (int k0 = 0; k0 < TTT_D; k0 += 8) {
+                uint32_t ah[4], al[4], bh[2], bl[2];
+                split(s.dzb[g][k0 + t], ah[0], al[0]);
+                split(s.dzb[g + 8][k0 + t], ah[1], al[1]);
+                split(s.dzb[g][k0 + t + 4], ah[2], al[2]);
+                split(s.dzb[g + 8][k0 + t + 4], ah[3], al[3]);
+                split(s.g[j0 + g][k0 + t], bh[0], bl[0]);
+                split(s.g[j0 + g][k0 + t + 4], bh[1], bl[1]);
+                mma_tf32(ch, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+                mma_tf32(cl, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+                mma_tf32(cl, al[0], al[1], al[2], al[3], bh[0], bh[1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {  // element (i, j): i = g (+ 8), j = j0 + 2t (+ 1)
+                const int i = g + 8 * (e >> 1), j = j0 + 2 * t + (e & 1);
+                const float dm = (j <= i && i < Km) ? -(ch[e] + cl[e]) : 0.f;
+                s.dlr_eta[i][j] = s.te[i] * (s.A[i][j] + 1.0f) * dm;
+                const float da = dm * s.te[i] * lrs[j];
+                s.dA[i][j] = da;
+                s.dAT[j][i] = da;
+            }
         }
         __syncthreads();  // (6)
         float4 dg = f4(0.f) - ld4(&s.P0[r][c0]);
@@ -962,8 +966,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             tc_tile<TTT_KMAX, false>(ck, s.dAT, xq, nt, g, t);
             put_tile(s.P0, cq, nt, g, t);
             put_tile(s.P1, ck, nt, g, t);
-            tc_rank16(dWacc, xq, nullptr, 1.f, s.dzb, m0, n0, g, t);
-            tc_rank16(dWacc, xk, nullptr, 1.f, s.dz, m0, n0, g, t);
+            tc_rank16_t(dWacc, s.dzb, nullptr, 1.f, xq, ni, kh, lane, g, t);
+            tc_rank16_t(dWacc, s.dz, nullptr, 1.f, xk, ni, kh, lane, g, t);
         }
         cp_async_wait_all();  // the next step's inputs (a forward step after this one has no barrier at its top)
         __syncthreads();      // (8)
@@ -982,7 +986,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             for (int i = 0; i < Km; ++i) acc += s.dzb[i][tid] + s.dz[i][tid];
             s.db[tid] += acc;
         }
-        put_acc(s.dW, dWacc);  // s.dW's readers (the update's products) finished before barrier (4)
+        put_t(s.dWT, dWacc);  // s.dWT's readers (the update's products) finished before barrier (4)
     };
 
     // ---- the order of the steps, for the prefetch of each one's successor ----------------------
@@ -1015,7 +1019,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         for (int q = 0; q < 4; ++q) dWacc[q][0] = dWacc[q][1] = dWacc[q][2] = dWacc[q][3] = 0.f;
     }
     if (tid < TTT_D) s.db[tid] = a.db_last ? a.db_last[chain * TTT_D + tid] : 0.f;
-    put_acc(s.dW, dWacc);
+    put_t(s.dWT, dWacc);
     if (rem > 0) {
         publish_w();  // s.WT's last readers passed barriers long ago; the step's first barrier orders the rest
         bwd_step(n_full * K, rem, false, buf, after_tail, nullptr);
