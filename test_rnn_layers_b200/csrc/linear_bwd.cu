@@ -546,10 +546,6 @@ __device__ __forceinline__ uint32_t op32(__nv_bfloat16 x) { return static_cast<u
 __device__ __forceinline__ uint32_t bf_lo(uint32_t p) { return p << 16; }
 __device__ __forceinline__ uint32_t bf_hi(uint32_t p) { return p & 0xffff0000u; }
 __device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
-// 8-byte cp.async (the source and destination 8-byte aligned).
-__device__ __forceinline__ void cp_async_8(void* dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
 
 // acc += sum_{k < K} X[m][k] Y(k, n0 + n) for the 16 x 8 tile at columns n0: X rows of stride kSX;
 // Y(k, n) = Ymat[k][n], or Ymat[n][k] when kTrans (rows of stride kSY).  Even and odd k-steps
@@ -721,23 +717,16 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         for (int q = 0; q < 4; ++q) st4(dst + tid * 16 + 4 * q, make_float4(Wacc[q][0], Wacc[q][1], Wacc[q][2], Wacc[q][3]));
         if (tid < TTT_D) dst[TTT_D * TTT_D + tid] = s.b[tid];
     };
-    auto load_state = [&](const float* src) {
+    auto load_regs = [&](const float* src) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const float4 v = ld4(src + tid * 16 + 4 * q);
             Wacc[q][0] = v.x; Wacc[q][1] = v.y; Wacc[q][2] = v.z; Wacc[q][3] = v.w;
         }
-        if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
     };
-    // a saved state straight into s.WT and s.b, asynchronously (what publish_w would write after
-    // load_state): each thread copies the pairs it saved
-    auto fetch_state = [&](const float* src) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            cp_async_8(&s.WT[ni + g][kh + 8 * j + 2 * t], src + tid * 16 + 4 * j);
-            cp_async_8(&s.WT[ni + g + 8][kh + 8 * j + 2 * t], src + tid * 16 + 4 * j + 2);
-        }
-        if (tid < TTT_D) cp_async_4z(&s.b[tid], src + TTT_D * TTT_D + tid, 4u);
+    auto load_state = [&](const float* src) {
+        load_regs(src);
+        if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
     };
 
     // The inputs of the step at t0 (Km tokens) into staging buffer buf, asynchronously: XK and XV
@@ -819,8 +808,8 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
 
     // The backward step of the mini-batch at t0 (as in linear_bwd_kernel), with its start state in
     // s.WT / s.b, the adjoint after it in dWacc / s.dWT / s.db, its inputs in staging buffer buf;
-    // next_state (or null): the saved start state of the step after, copied into s.WT and s.b
-    // once this step has no more use for them.
+    // next_state (or null): the saved start state of the step after, loaded into the W registers
+    // early and written to s.WT and s.b once this step has no more use for them.
     auto bwd_step = [&](long long t0, int Km, bool full, int buf, const Next& nx, const float* next_state) {
         const bool live = r < Km;
         const long long row = (t0 + r) * ts + c0;
@@ -831,6 +820,11 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const __nv_bfloat16 (*xk)[kSB] = s.stage[buf][1];
         const float* lrs = s.stage_lr[buf];
         start_next(buf, nx);
+        float b_next = 0.f;
+        if (next_state) {  // the next step's start state into the idle W registers, a step ahead of its use
+            load_regs(next_state);
+            if (tid < TTT_D) b_next = next_state[TTT_D * TTT_D + tid];
+        }
         {  // XK W and XQ W, sharing W's fragments
             float cz[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
             tc_tile2_wt(cz, cb, xk, xq, s.WT, nt, g, t);
@@ -971,7 +965,10 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         }
         cp_async_wait_all();  // the next step's inputs (a forward step after this one has no barrier at its top)
         __syncthreads();      // (8)
-        if (next_state) fetch_state(next_state);  // s.WT's and s.b's readers are done
+        if (next_state) {  // s.WT's and s.b's readers are done
+            publish_w();
+            if (tid < TTT_D) s.b[tid] = b_next;
+        }
         if (live) {
             st4(dXQ + row, o4 + ld4(&s.P0[r][c0]));
             st4(dXK + row, dxk + ld4(&s.P1[r][c0]));
