@@ -91,6 +91,8 @@ CASES = [  # (name, dtype, B, H, L, K, G, token_eta)
     ("f32_K1_online", "f32", 1, 2, 9, 1, 4, None),
     ("bf16_tail", "bf16", 2, 2, 16 * 8 + 7, 16, 4, None),
     ("bf16_no_tail", "bf16", 1, 4, 16 * 6, 16, 6, None),
+    ("bf16_K8_tail", "bf16", 1, 3, 8 * 5 + 3, 8, 2, None),
+    ("bf16_K4_eta_table", "bf16", 2, 1, 37, 4, 3, [0.9, 0.5, 0.3, 0.2]),
 ]
 
 

@@ -145,3 +145,16 @@ def test_linear_row_mean_offset(libttt, offset, flags):
                for n, t in (("out", out), ("W_last", Wl), ("b_last", bl), ("W_grad_tail", Wg), ("b_grad_tail", bg))})
     print(f"\n[row mean offset {offset}, flags {flags}]:", {k: f"{v:.2e}" for k, v in e.items()})
     assert max(e.values()) <= TOL, e
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_backward_wide_inputs(libttt, dt):
+    """The TTT-Linear backward (tensor-core kernel for bf16, FFMA kernel for fp32) at the wide
+    scale, 2 x 2 chains with a tail and two checkpoint groups, against the backward oracle at each
+    kernel's own bar (bf16 1e-2, fp32 1e-5); upstream gradients N(0, 1)."""
+    from test_backward import _compare, _gpu, _oracle
+    w = synth.workload(1, B=2, H=2, L=16 * 6 + 5, dtype=dt, seed=0x5CA1F, **WIDE)
+    ids = list(range(w.chains))
+    ref = _oracle(w, synth.linear_inputs(w, chains=ids), synth.upstream_grads(w, chains=ids), ids)
+    g = _gpu(libttt, w, synth.linear_inputs(w), synth.upstream_grads(w), 3)
+    _compare(w, g, ref, tag=f"wide {dt}")
