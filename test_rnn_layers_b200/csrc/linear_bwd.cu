@@ -640,6 +640,21 @@ __device__ __forceinline__ void put_tile(float (*P)[kS], const float (&c)[4], in
     *reinterpret_cast<float2*>(&P[g + 8][n0 + 2 * t]) = make_float2(c[2], c[3]);
 }
 
+// row_norm with one-pass statistics: the sum and the sum of squares in one shuffle tree, the
+// variance as E[z^2] - mean^2 (its rounding grows with (mean / std)^2 of the row).
+__device__ __forceinline__ void row_norm1(float4 z, float eps, float4& xh, float& sigma) {
+    float s1 = hsum4(z), s2 = hsum4(z * z);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    const float mu = s1 * (1.0f / TTT_D);
+    const float v = fmaxf(s2 * (1.0f / TTT_D) - mu * mu, 0.f);
+    sigma = sqrtf(v + eps);
+    xh = (z - f4(mu)) * (1.0f / sigma);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -787,7 +802,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const float4 z = ld4(&s.P2[r][c0]) + ld4(&s.Zp[r][c0]) + ld4(&s.b[c0]);
         float4 xh;
         float sig;
-        row_norm(z, eps, xh, sig);
+        row_norm1(z, eps, xh, sig);
         const float4 q = lw * (lw * xh + lb - (v4 - k4));
         const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
         const float4 gv = live ? (q - f4(mq) - xh * mqx) * (1.0f / sig) : f4(0.f);
@@ -856,7 +871,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const float4 z = ld4(&s.P0[r][c0]) + bb;
         float4 xh;
         float sig;
-        row_norm(z, eps, xh, sig);
+        row_norm1(z, eps, xh, sig);
         const float4 res = lw * xh + lb - (v4 - k4);
         const float4 q = lw * res;
         const float mq = row_sum(hsum4(q)) * (1.0f / TTT_D), mqx = row_sum(hsum4(q * xh)) * (1.0f / TTT_D);
@@ -880,7 +895,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const float4 zb = zb0 - ld4(&s.P0[r][c0]);
         float4 xhb;
         float sigb;
-        row_norm(zb, eps, xhb, sigb);
+        row_norm1(zb, eps, xhb, sigb);
         const float4 p = lw * o4;
         const float mp = row_sum(hsum4(p)) * (1.0f / TTT_D), mpx = row_sum(hsum4(p * xhb)) * (1.0f / TTT_D);
         st4(&s.dzb[r][c0], (p - f4(mp) - xhb * mpx) * (1.0f / sigb));
@@ -978,10 +993,13 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
             for (int i = 0; i < TTT_KMAX; ++i) acc += s.dlr_eta[i][tid];
             dlr[t0 + tid] = acc;
         }
-        if (tid < TTT_D) {
+        if (tid >= TTT_D && tid < 2 * TTT_D) {  // db, on the third and fourth warps
+            const int f = tid - TTT_D;
             float acc = 0.f;
-            for (int i = 0; i < Km; ++i) acc += s.dzb[i][tid] + s.dz[i][tid];
-            s.db[tid] += acc;
+#pragma unroll
+            for (int i = 0; i < TTT_KMAX; ++i)
+                if (i < Km) acc += s.dzb[i][f] + s.dz[i][f];
+            s.db[f] += acc;
         }
         put_t(s.dWT, dWacc);  // s.dWT's readers (the update's products) finished before barrier (4)
     };

@@ -158,3 +158,24 @@ def test_backward_wide_inputs(libttt, dt):
     ref = _oracle(w, synth.linear_inputs(w, chains=ids), synth.upstream_grads(w, chains=ids), ids)
     g = _gpu(libttt, w, synth.linear_inputs(w), synth.upstream_grads(w), 3)
     _compare(w, g, ref, tag=f"wide {dt}")
+
+
+@pytest.mark.parametrize("offset,dt", [(0.25, "bf16"), (1.0, "bf16"), (0.25, "f32")],
+                         ids=["b0+0.25_bf16", "b0+1_bf16", "b0+0.25_f32"])
+def test_backward_row_mean_offset(libttt, offset, dt):
+    """The backward with a common offset in b0 (row means of Z and Zbar near `offset` against a
+    spread of about 0.02), 2 x 2 chains of 32 full mini-batches and a tail, checkpoint group 4, at
+    each kernel's own bar.  bf16 up to mean / std = 50, the bound the forward kernel states for its
+    one-pass statistics, which the tensor-core backward shares (3.1e-3 measured there).  fp32 (the
+    FFMA backward, two-pass statistics) to mean / std = 12: float32 itself loses about
+    eps * mean / std of each z before any arithmetic, so at 50 the 1e-5 bar is out of reach of any
+    float32 computation (1.1e-5 measured)."""
+    from test_backward import _compare, _gpu, _oracle
+    w = synth.workload(1, B=2, H=2, L=16 * 32 + 5, dtype=dt, seed=0x0FF6)
+    ids = list(range(w.chains))
+    x, xf = synth.linear_inputs(w, chains=ids), synth.linear_inputs(w)
+    for d in (x, xf):
+        d["b0"] = (d["b0"] + offset).astype(np.float32)
+    ref = _oracle(w, x, synth.upstream_grads(w, chains=ids), ids)
+    g = _gpu(libttt, w, xf, synth.upstream_grads(w), 4)
+    _compare(w, g, ref, tag=f"row mean offset {offset} {dt}")
