@@ -444,9 +444,12 @@ long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, 
  *   d_ln_w, d_ln_b  [H,d] float32, summed over the batch.
  *   workspace    device buffer of at least ttt_linear_backward_workspace_bytes, 256-byte aligned;
  *                its contents on entry do not matter and are overwritten.
- * One CTA per chain.  fp32 activations compute in float32 throughout; bf16 activations run the
- * products and state updates on the tensor cores with TF32 operands (11-bit significands, like
- * the forward's fp16 operands) and fp32 accumulation, state and adjoint.  The batch sums run in
+ * One CTA per chain.  fp32 activations compute in float32 throughout (two-pass LayerNorm
+ * statistics); bf16 activations run the products and state updates on the tensor cores with TF32
+ * operands (11-bit significands, like the forward's fp16 operands) and fp32 accumulation, state
+ * and adjoint, and take each LayerNorm variance in one pass, with the forward kernel's bound (rows
+ * of Z with |mean over features| below about 50x their spread; see ttt_linear_forward).  fp32
+ * activations serve states beyond it.  The batch sums run in
  * a fixed order, so results are reproducible bit for bit.  Asynchronous on `stream`; allocates nothing; has no
  * device-side waits.  Errors as ttt_linear_forward (flags aside), plus TTT_ERR_ARG for
  * ckpt_group < 1 or a workspace smaller than needed.  The call makes two launches (the scan's
