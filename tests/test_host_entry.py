@@ -92,3 +92,24 @@ def test_host_entry_L0_and_shared_workspace(libttt):
     torch.cuda.synchronize()
     for a, b in zip(r1, r2):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("token_major", [False, True], ids=["head_major", "token_major"])
+@pytest.mark.parametrize("chunk", [1, 2])
+def test_host_entry_odd_heads_both_layouts(libttt, token_major, chunk):
+    """Five heads and three batch rows in chunks of 1 or 2 rows (a ragged last chunk), head-major
+    and token-major activations: the same bits as the device entry point."""
+    w = synth.workload(1, B=3, H=5, L=16 * 3 + 4, seed=0x405A + chunk)
+    x = synth.linear_inputs(w)
+    tm = (lambda t: t.transpose(1, 2).contiguous()) if token_major else (lambda t: t)
+    acts = [n for n in ("XQ", "XK", "XV")]
+    dev = libttt.ttt_linear_forward(*[tm(dev_act(x, n)) for n in acts], dev_f32(x["lr"]), dev_f32(x["W0"]),
+                                    dev_f32(x["b0"]), dev_f32(x["ln_w"]), dev_f32(x["ln_b"]), mini_batch=w.K,
+                                    eps=w.eps, tail_grads=True, token_major=token_major)
+    host = libttt.ttt_linear_forward_host(*[tm(_host_act(x, n)).pin_memory() for n in acts], _host_f32(x["lr"]),
+                                          _host_f32(x["W0"]), _host_f32(x["b0"]), _host_f32(x["ln_w"]),
+                                          _host_f32(x["ln_b"]), mini_batch=w.K, eps=w.eps, tail_grads=True,
+                                          chunk_batches=chunk, token_major=token_major)
+    torch.cuda.synchronize()
+    for d, h in zip(dev, host):
+        assert torch.equal(d.cpu(), h)
