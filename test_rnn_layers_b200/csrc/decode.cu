@@ -144,16 +144,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(DecodeArgs
         if (warp == 0) {
             // g = ln_fused_l2_bwd(z, xv - xk)
             const float z0 = s.sz[lane], z1 = s.sz[lane + 32];
-            const float mu = warp_sum(z0 + z1) * (1.0f / TTT_D);
-            const float c0 = z0 - mu, c1 = z1 - mu;
-            const float rstd = rsqrtf(warp_sum(c0 * c0 + c1 * c1) * (1.0f / TTT_D) + a.eps);
-            const float xh0 = c0 * rstd, xh1 = c1 * rstd;
+            float mu, rstd;
+            warp_row_stats(z0, z1, a.eps, mu, rstd);
+            const float xh0 = (z0 - mu) * rstd, xh1 = (z1 - mu) * rstd;
             const float w0 = lnw[lane], w1 = lnw[lane + 32];
             const float xk0 = to_f32(s.x[bi][1][lane]), xk1 = to_f32(s.x[bi][1][lane + 32]);
             const float xq0 = to_f32(s.x[bi][0][lane]), xq1 = to_f32(s.x[bi][0][lane + 32]);
             const float q0 = w0 * (w0 * xh0 + lnb[lane] - (to_f32(s.x[bi][2][lane]) - xk0));
             const float q1 = w1 * (w1 * xh1 + lnb[lane + 32] - (to_f32(s.x[bi][2][lane + 32]) - xk1));
-            const float sq = warp_sum(q0 + q1), sqx = warp_sum(q0 * xh0 + q1 * xh1);
+            float sq = q0 + q1, sqx = fmaf(q0, xh0, q1 * xh1);
+            warp_sum2(sq, sqx);
             const float g0 = (TTT_D * q0 - sq - xh0 * sqx) * rstd * (1.0f / TTT_D);
             const float g1 = (TTT_D * q1 - sq - xh1 * sqx) * rstd * (1.0f / TTT_D);
             s.sg[lane] = g0;
@@ -165,9 +165,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(DecodeArgs
             // xq W_bar + b_bar
             const float u0 = s.sqw[lane] - t * (s.sqg[lane] + lr * s.sqk * g0) + bb0;
             const float u1 = s.sqw[lane + 32] - t * (s.sqg[lane + 32] + lr * s.sqk * g1) + bb1;
-            const float m2 = warp_sum(u0 + u1) * (1.0f / TTT_D);
+            float m2, r2;
+            warp_row_stats(u0, u1, a.eps, m2, r2);
             const float d0 = u0 - m2, d1 = u1 - m2;
-            const float r2 = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.0f / TTT_D) + a.eps);
             T* out = static_cast<T*>(a.out) + c * TTT_D;
             out[lane] = from_f32<T>(xq0 + w0 * d0 * r2 + lnb[lane]);
             out[lane + 32] = from_f32<T>(xq1 + w1 * d1 * r2 + lnb[lane + 32]);

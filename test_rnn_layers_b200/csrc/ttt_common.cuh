@@ -62,6 +62,23 @@ __device__ __forceinline__ float warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
+// Two warp sums side by side (one shuffle tree's depth for both).
+__device__ __forceinline__ void warp_sum2(float& u, float& v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        u += __shfl_xor_sync(0xffffffffu, u, o);
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    }
+}
+// Mean and 1/sqrt(var + eps) of a TTT_D-feature row held as (x0, x1) per lane, the variance in one
+// pass (E[x^2] - mean^2, clamped at zero): one shuffle tree instead of two dependent ones; its
+// rounding grows with (mean / std)^2 of the row.
+__device__ __forceinline__ void warp_row_stats(float x0, float x1, float eps, float& mu, float& rstd) {
+    float s1 = x0 + x1, s2 = fmaf(x0, x0, x1 * x1);
+    warp_sum2(s1, s2);
+    mu = s1 * (1.0f / TTT_D);
+    rstd = rsqrtf(fmaxf(fmaf(-mu, mu, s2 * (1.0f / TTT_D)), 0.f) + eps);
+}
 
 // ---------------------------------------------------------------------------------------------
 // status word: kernels OR in TTT_STATUS_* bits when they give up on a bounded wait
