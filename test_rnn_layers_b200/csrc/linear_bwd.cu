@@ -25,16 +25,16 @@
 //    backward step for each mini-batch of the group in reverse.  Both phases run the same
 //    forward-step code, so a rebuilt state has the bits of the first.
 //  * The LayerNorm work uses a row layout: thread (r, c0) = (tid / 16, 4 (tid % 16)) owns four
-//    consecutive features of one row of a 16 x 64 tile, so a row's sums are half-warp shuffles
-//    (two-pass statistics).  The 16 x 16 products XQ XK^T and dZbar g^T are per-thread dot
-//    products.
-//  * linear_bwd_tc_kernel (bf16 activations): the 16 x 64 x 64 products and the rank-16 state
-//    updates are TF32 warp MMAs (m16n8k8, fp32 accumulation) with the state and its adjoint held
-//    as accumulators and published to shared memory as B operands; each step's input tiles are
-//    copied in one step ahead by cp.async.
+//    consecutive features of one row of a 16 x 64 tile, so a row's sums are half-warp shuffles.
+//  * linear_bwd_tc_kernel (bf16 activations): the 16 x 64 x 64 products, the 16 x 16 products
+//    XQ XK^T and dZbar g^T, and the rank-16 state updates are TF32 warp MMAs (m16n8k8, fp32
+//    accumulation); the state and its adjoint live as accumulators (the layouts are described
+//    at the kernel), the LayerNorm statistics are taken in one pass, and each step's input tiles
+//    are copied in one step ahead by cp.async.
 //  * linear_bwd_kernel (fp32 activations): every product is one row of a tile times a 64-wide
-//    matrix read as float4 rows, fp32 throughout; the state and its adjoint live in shared
-//    memory as [k][f] and transposed, each thread owning a 4 x 4 block of both in registers.
+//    matrix read as float4 rows, fp32 throughout, the 16 x 16 products per-thread dot products
+//    and the LayerNorm statistics two-pass; the state and its adjoint live in shared memory as
+//    [k][f] and transposed, each thread owning a 4 x 4 block of both in registers.
 //  * No waits: nothing in either kernel can hang.
 #include "ttt_common.cuh"
 #include "ttt_internal.h"
@@ -126,7 +126,8 @@ __device__ __forceinline__ float dot64(const float* p, const float* q) {
     return a0 + a1;
 }
 
-// LayerNorm statistics of a row whose four features z this thread holds: x_hat and sigma.
+// LayerNorm statistics of a row whose four features z this thread holds, in two passes: x_hat
+// and sigma.
 __device__ __forceinline__ void row_norm(float4 z, float eps, float4& xh, float& sigma) {
     const float mu = row_sum(hsum4(z)) * (1.0f / TTT_D);
     const float4 c = z - f4(mu);
