@@ -529,6 +529,22 @@ def bench_linear_backward(args, world, peaks, G=16):
     ms_all = time_steps(step_all_states, K, 3, world)
     ws_all = ws.numel()
     del ws
+    # the training split: the forward's checkpoints (ttt_linear_forward_ckpt, written once before
+    # the timed region) and the backward from them (ttt_linear_backward_ckpt), which skips its own
+    # pass of the state recursion
+    ws = torch.empty(ttt.ttt_linear_backward_workspace_bytes(w.B, w.H, w.L, w.K, G), dtype=torch.uint8, device="cuda")
+    ckpt = torch.empty(ttt.ttt_linear_ckpt_bytes(w.B, w.H, w.L, w.K, G) // 4, device="cuda")
+    ttt.ttt_linear_forward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], mini_batch=w.K, eps=w.eps,
+                           ckpt=ckpt, ckpt_group=G)
+
+    def step_from_ckpt():
+        g = ttt.ttt_linear_backward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], dout, dWl, dbl,
+                                    mini_batch=w.K, eps=w.eps, ckpt_group=G, workspace=ws, ckpt=ckpt)
+        if world > 1:
+            allreduce_shared_grads(g)
+
+    ms_ck = time_steps(step_from_ckpt, K, 3, world)
+    del ws, ckpt
     flops, nbytes = linear_bwd_flops(w.B, w.H, w.L), linear_bwd_bytes(w.B, w.H, w.L)
     tfl = flops / (ms / 1e3) / 1e12
     gbs = nbytes / (ms / 1e3) / 1e9
@@ -541,6 +557,9 @@ def bench_linear_backward(args, world, peaks, G=16):
                            "bytes per step" if world > 1 else "none (one GPU)"),
             "every_state_kept": {"ckpt_group": 1, "ms_per_step": round(ms_all, 4),
                                  "value": round(world * w.B * w.L / (ms_all / 1e3), 1), "workspace_bytes": ws_all},
+            "from_forward_checkpoints": {"ckpt_group": G, "call": "ttt_linear_backward_ckpt",
+                                         "ms_per_step": round(ms_ck, 4),
+                                         "value": round(world * w.B * w.L / (ms_ck / 1e3), 1)},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "peak_source": f"{which} hbm_gbs",
                          "unit": "GB/s", "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
                          "floor_ms": round(nbytes / hbm / 1e6, 4), "algorithmic_flops": flops,

@@ -463,6 +463,56 @@ int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const fl
                         const float* db_last, void* dXQ, void* dXK, void* dXV, float* d_lr, float* dW0, float* db0,
                         float* d_ln_w, float* d_ln_b, void* workspace, long long workspace_bytes, void* stream);
 
+/* ---- checkpoints from the forward ------------------------------------------------------------
+ * [walkthrough] TTTLinear.ttt's scan keeps the carried state at the start of every checkpoint
+ * group during the forward pass and rebuilds the states inside a group during the backward.  The
+ * three calls below give training that split: the forward writes the group-boundary states, and
+ * the backward starts from them instead of running the state recursion once more (its phase 1). */
+
+/*
+ * ttt_linear_ckpt_bytes -- bytes of the checkpoint buffer of ttt_linear_forward_ckpt and
+ * ttt_linear_backward_ckpt: per chain, ceil(n_full / ckpt_group) + 1 states of (d*d + d) float32,
+ * n_full = L / K.  Host-only.  Returns the byte count (> 0) or a negative TTT_ERR_* code.
+ */
+long long ttt_linear_ckpt_bytes(int B, int H, long long L, int d, int mini_batch, int ckpt_group);
+
+/*
+ * ttt_linear_forward_ckpt -- ttt_linear_forward that also writes checkpoints for the backward.
+ * Arguments and results as ttt_linear_forward, plus
+ *   ckpt_group   G >= 1: a state is kept before every G-th full mini-batch (mini-batches 0, G, 2G, ...).
+ *   ckpt         device buffer of ttt_linear_ckpt_bytes, 16-byte aligned, written: chain c's entry i
+ *                (c * (n_ckpt + 1) + i, each d*d + d float32) is W as [k][n] then b before full
+ *                mini-batch i*G for i < n_ckpt, and the state after the last full mini-batch (equal
+ *                to W_last, b_last) at i = n_ckpt.  The states are the kernel's own fp32 state.
+ * Errors as ttt_linear_forward, plus TTT_ERR_ARG for a null ckpt or ckpt_group < 1, TTT_ERR_ALIGN,
+ * and TTT_ERR_ALIAS when ckpt overlaps another argument.
+ */
+int ttt_linear_forward_ckpt(const void* XQ, const void* XK, const void* XV, const float* lr,
+                            const float* token_eta, const float* W0, const float* b0,
+                            long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                            long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                            void* out, float* W_last, float* b_last, float* W_grad_tail,
+                            float* b_grad_tail, int ckpt_group, float* ckpt, void* stream);
+
+/*
+ * ttt_linear_backward_ckpt -- ttt_linear_backward from the checkpoints of ttt_linear_forward_ckpt
+ * (the same inputs and ckpt_group): the backward skips its own pass of the state recursion over
+ * the full mini-batches and rebuilds each group from the caller's state at its start.
+ * Arguments and results as ttt_linear_backward, plus
+ *   ckpt         the checkpoint buffer (read only), 16-byte aligned; the workspace keeps its size.
+ * The gradients are those of ttt_linear_backward up to rounding: the forward's fp16-operand
+ * state recursion and the backward's TF32 one differ in the last bits (bf16 activations), so
+ * unlike ttt_linear_backward the results depend on ckpt_group in those bits.
+ * Errors as ttt_linear_backward, plus TTT_ERR_ARG for a null ckpt, TTT_ERR_ALIGN, TTT_ERR_ALIAS.
+ */
+int ttt_linear_backward_ckpt(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                             const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
+                             const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps,
+                             int dtype, unsigned int flags, int ckpt_group, const float* ckpt, const void* d_out,
+                             const float* dW_last, const float* db_last, void* dXQ, void* dXK, void* dXV,
+                             float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b, void* workspace,
+                             long long workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

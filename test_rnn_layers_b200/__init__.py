@@ -36,7 +36,8 @@ EXPORTS = ("ttt_partition", "ttt_error_string", "ttt_last_error_message", "ttt_d
            "ttt_set_wait_limit", "ttt_linear_forward", "ttt_linear_forward_rope", "ttt_linear_host_workspace_bytes",
            "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward",
            "ttt_linear_decode_step", "ttt_linear_decode_step_hist", "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
-           "ttt_linear_backward_workspace_bytes", "ttt_linear_backward")
+           "ttt_linear_backward_workspace_bytes", "ttt_linear_backward", "ttt_linear_ckpt_bytes",
+           "ttt_linear_forward_ckpt", "ttt_linear_backward_ckpt")
 
 
 class TTTError(RuntimeError):
@@ -87,11 +88,18 @@ def lib():
         L.ttt_linear_backward_workspace_bytes.restype = ll
         L.ttt_linear_backward.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u, i, vp, fp,
                                           fp, vp, vp, vp, fp, fp, fp, fp, fp, vp, ll, vp]
+        L.ttt_linear_ckpt_bytes.argtypes = [i, i, ll, i, i, i]
+        L.ttt_linear_ckpt_bytes.restype = ll
+        L.ttt_linear_forward_ckpt.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u,
+                                              vp, fp, fp, fp, fp, i, fp, vp]
+        L.ttt_linear_backward_ckpt.argtypes = [vp, vp, vp, fp, fp, fp, fp, ll, fp, fp, i, i, ll, i, i, f, i, u, i, fp,
+                                               vp, fp, fp, vp, vp, vp, fp, fp, fp, fp, fp, vp, ll, vp]
         for name in ("ttt_partition", "ttt_device_status", "ttt_set_wait_limit", "ttt_linear_forward",
                      "ttt_o_proj_prepare", "ttt_post_norm_o_proj",
                      "ttt_linear_forward_rope",
                      "ttt_linear_forward_host", "ttt_linear_forward_host_static", "ttt_mlp_forward", "ttt_linear_decode_step",
-                     "ttt_linear_decode_step_hist", "ttt_linear_backward"):
+                     "ttt_linear_decode_step_hist", "ttt_linear_backward", "ttt_linear_forward_ckpt",
+                     "ttt_linear_backward_ckpt"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -167,14 +175,17 @@ def ttt_device_status(clear: bool = True, stream=None) -> int:
 def ttt_linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
                        token_eta=None, out=None, W_last=None, b_last=None, W_grad_tail=None,
                        b_grad_tail=None, tail_grads: bool = False, flags: int = 0, token_major: bool = False,
-                       stream=None):
+                       stream=None, ckpt=None, ckpt_group: int = 16):
     """TTT-Linear prefill over [B,H,L,64] activations, or [B,L,H,64] with token_major (see include/ttt.h).
 
     W0/b0: [H,64,64]/[H,64] shared over the batch, or [B,H,64,64]/[B,H,64] per chain.
+    ckpt: a float32 CUDA tensor of ttt_linear_ckpt_bytes(...) bytes to receive the checkpoints of
+    ttt_linear_backward (ttt_linear_forward_ckpt: the state before every ckpt_group-th full
+    mini-batch, then the state after the last), or None.
     Returns (out, W_last, b_last) or, with tail_grads, (out, W_last, b_last, W_grad_tail, b_grad_tail).
     """
     return _linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch, eps, token_eta, out, W_last, b_last,
-                           W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, None)
+                           W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, None, ckpt, ckpt_group)
 
 
 def ttt_linear_forward_rope(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int = 16, eps: float = 1e-6,
@@ -190,8 +201,17 @@ def ttt_linear_forward_rope(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch: int 
                            W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, rope_theta)
 
 
+def ttt_linear_ckpt_bytes(B: int, H: int, L: int, mini_batch: int = 16, ckpt_group: int = 16, d: int = 64) -> int:
+    """Bytes of the checkpoint buffer of ttt_linear_forward(..., ckpt=) and ttt_linear_backward(..., ckpt=)."""
+    n = lib().ttt_linear_ckpt_bytes(B, H, L, d, mini_batch, ckpt_group)
+    if n < 0:
+        _check(int(n))
+    return int(n)
+
+
 def _linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch, eps, token_eta, out, W_last, b_last,
-                    W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, rope_theta):
+                    W_grad_tail, b_grad_tail, tail_grads, flags, token_major, stream, rope_theta, ckpt=None,
+                    ckpt_group=16):
     _need(XQ, "XQ")
     B, H, L, d = _act_sizes(XQ, token_major)
     flags |= TTT_FLAG_TOKEN_MAJOR if token_major else 0
@@ -217,7 +237,12 @@ def _linear_forward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, mini_batch, eps, token_e
             H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch, eps)
     tail = (_dtype_code(XQ), flags, _ptr(out), _ptr(W_last), _ptr(b_last), _ptr(W_grad_tail), _ptr(b_grad_tail),
             _stream(stream))
-    if rope_theta is None:
+    if ckpt is not None:
+        _need(ckpt, "ckpt", torch.float32)
+        if ckpt.numel() * 4 < ttt_linear_ckpt_bytes(B, H, L, mini_batch, ckpt_group, d):
+            raise ValueError("ckpt is smaller than ttt_linear_ckpt_bytes(...)")
+        rc = lib().ttt_linear_forward_ckpt(*head, *tail[:-1], ckpt_group, _ptr(ckpt), tail[-1])
+    elif rope_theta is None:
         rc = lib().ttt_linear_forward(*head, *tail)
     else:
         rc = lib().ttt_linear_forward_rope(*head, rope_theta, *tail)
@@ -487,9 +512,12 @@ def ttt_linear_backward_workspace_bytes(B: int, H: int, L: int, mini_batch: int 
 
 def ttt_linear_backward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, d_out, dW_last=None, db_last=None,
                         mini_batch: int = 16, eps: float = 1e-6, token_eta=None, ckpt_group: int = 16,
-                        token_major: bool = False, workspace=None, stream=None):
+                        token_major: bool = False, workspace=None, stream=None, ckpt=None):
     """Gradients of <d_out, out> + <dW_last, W_last> + <db_last, b_last> for ttt_linear_forward's
     inputs ([B,H,L,64], or [B,L,H,64] with token_major; see include/ttt.h).
+    ckpt: the checkpoints ttt_linear_forward(..., ckpt=, ckpt_group=) wrote for the same inputs and
+    ckpt_group (ttt_linear_backward_ckpt: the backward then skips its own pass of the state
+    recursion), or None.
 
     Returns a dict: dXQ, dXK, dXV (the activations' dtype), dlr [B,H,L], dW0/db0 (per head when W0
     is [H,64,64], per chain when it is [B,H,64,64]), dln_w/dln_b [H,64].
@@ -521,11 +549,17 @@ def ttt_linear_backward(XQ, XK, XV, lr, W0, b0, ln_w, ln_b, d_out, dW_last=None,
          "dlr": torch.empty((B, H, L), device=dev),
          "dW0": torch.empty(W0.shape, device=dev), "db0": torch.empty(b0.shape, device=dev),
          "dln_w": torch.empty((H, d), device=dev), "dln_b": torch.empty((H, d), device=dev)}
-    _check(lib().ttt_linear_backward(_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
-                                     H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch,
-                                     eps, _dtype_code(XQ), TTT_FLAG_TOKEN_MAJOR if token_major else 0, ckpt_group,
-                                     _ptr(d_out), _ptr(dW_last), _ptr(db_last),
-                                     _ptr(g["dXQ"]), _ptr(g["dXK"]), _ptr(g["dXV"]), _ptr(g["dlr"]), _ptr(g["dW0"]),
-                                     _ptr(g["db0"]), _ptr(g["dln_w"]), _ptr(g["dln_b"]), _ptr(workspace),
-                                     workspace.numel(), _stream(stream)))
+    head = (_ptr(XQ), _ptr(XK), _ptr(XV), _ptr(lr), _ptr(token_eta), _ptr(W0), _ptr(b0),
+            H * d * d if per_chain else 0, _ptr(ln_w), _ptr(ln_b), B, H, L, d, mini_batch, eps, _dtype_code(XQ),
+            TTT_FLAG_TOKEN_MAJOR if token_major else 0, ckpt_group)
+    tail = (_ptr(d_out), _ptr(dW_last), _ptr(db_last), _ptr(g["dXQ"]), _ptr(g["dXK"]), _ptr(g["dXV"]), _ptr(g["dlr"]),
+            _ptr(g["dW0"]), _ptr(g["db0"]), _ptr(g["dln_w"]), _ptr(g["dln_b"]), _ptr(workspace), workspace.numel(),
+            _stream(stream))
+    if ckpt is None:
+        _check(lib().ttt_linear_backward(*head, *tail))
+    else:
+        _need(ckpt, "ckpt", torch.float32)
+        if ckpt.numel() * 4 < ttt_linear_ckpt_bytes(B, H, L, mini_batch, ckpt_group, d):
+            raise ValueError("ckpt is smaller than ttt_linear_ckpt_bytes(...)")
+        _check(lib().ttt_linear_backward_ckpt(*head, _ptr(ckpt), *tail))
     return g

@@ -368,11 +368,16 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_kernel(const LinearBwdArgs a
     };
 
     // ---- phase 1: the forward state recursion, a checkpoint every G full mini-batches --------
-    put_state(false);
-    __syncthreads();
-    for (long long m = 0; m < a.n_full; ++m) {
-        if (m % G == 0) save_state(a.ckpt + (chain * a.n_ckpt + m / G) * kState);
-        fwd_step(m * K);
+    // (with the caller's checkpoints, only the state after the full mini-batches: the last entry)
+    if (a.ckpt_given) {
+        load_state(a.ckpt + (chain * a.ckpt_stride + a.n_ckpt) * kState);
+    } else {
+        put_state(false);
+        __syncthreads();
+        for (long long m = 0; m < a.n_full; ++m) {
+            if (m % G == 0) save_state(a.ckpt + (chain * a.ckpt_stride + m / G) * kState);
+            fwd_step(m * K);
+        }
     }
 
     // ---- the remainder tail, from the state after the full mini-batches -----------------------
@@ -394,7 +399,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_kernel(const LinearBwdArgs a
     for (long long c = a.n_ckpt - 1; c >= 0; --c) {
         const long long m0 = c * G, m1 = m0 + G < a.n_full ? m0 + G : a.n_full;
         __syncthreads();
-        load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
+        load_state(a.ckpt + (chain * a.ckpt_stride + c) * kState);
         put_state(false);
         __syncthreads();
         for (long long m = m0; m < m1; ++m) {
@@ -733,16 +738,21 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         for (int q = 0; q < 4; ++q) st4(dst + tid * 16 + 4 * q, make_float4(Wacc[q][0], Wacc[q][1], Wacc[q][2], Wacc[q][3]));
         if (tid < TTT_D) dst[TTT_D * TTT_D + tid] = s.b[tid];
     };
+    // a checkpoint (W as [k][n], then b), the format the forward kernels write
+    auto save_ckpt = [&](float* dst) {
+        store_acc(dst, Wacc);
+        if (tid < TTT_D) dst[TTT_D * TTT_D + tid] = s.b[tid];
+    };
+    auto load_ckpt = [&](const float* src) {
+        load_acc(Wacc, src);
+        if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
+    };
     auto load_regs = [&](const float* src) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const float4 v = ld4(src + tid * 16 + 4 * q);
             Wacc[q][0] = v.x; Wacc[q][1] = v.y; Wacc[q][2] = v.z; Wacc[q][3] = v.w;
         }
-    };
-    auto load_state = [&](const float* src) {
-        load_regs(src);
-        if (tid < TTT_D) s.b[tid] = src[TTT_D * TTT_D + tid];
     };
 
     // The inputs of the step at t0 (Km tokens) into staging buffer buf, asynchronously: XK and XV
@@ -1017,12 +1027,19 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
     int buf = 0;
 
     // ---- phase 1: the forward state recursion, a checkpoint every G full mini-batches --------
-    if (n_full > 0) prefetch(0, 0, K, false);
-    else if (after_phase1.kind) prefetch(0, after_phase1.t0, after_phase1.Km, after_phase1.kind == 2);
+    // (with the caller's checkpoints, only the state after the full mini-batches: the last entry)
+    if (a.ckpt_given) {
+        if (after_phase1.kind) prefetch(0, after_phase1.t0, after_phase1.Km, after_phase1.kind == 2);
+        load_ckpt(a.ckpt + (chain * a.ckpt_stride + a.n_ckpt) * kState);
+    } else if (n_full > 0) {
+        prefetch(0, 0, K, false);
+    } else if (after_phase1.kind) {
+        prefetch(0, after_phase1.t0, after_phase1.Km, after_phase1.kind == 2);
+    }
     cp_async_wait_all();
     __syncthreads();  // the first step's inputs, b and the step coefficients in place for every thread
-    for (long long m = 0; m < n_full; ++m) {
-        if (m % G == 0) save_state(a.ckpt + (chain * a.n_ckpt + m / G) * kState);
+    for (long long m = 0; m < (a.ckpt_given ? 0 : n_full); ++m) {
+        if (m % G == 0) save_ckpt(a.ckpt + (chain * a.ckpt_stride + m / G) * kState);
         fwd_step(m * K, buf, m + 1 < n_full ? Next{1, (m + 1) * K, K} : after_phase1);
         buf = next_buf(buf);
     }
@@ -1048,7 +1065,7 @@ __global__ void __launch_bounds__(kT, 2) linear_bwd_tc_kernel(const LinearBwdArg
         const long long m0g = c * G, m1g = m0g + G < n_full ? m0g + G : n_full;
         // no barrier: s.b's readers of the last step passed its later barriers, and each thread
         // rewrites only its own elements
-        load_state(a.ckpt + (chain * a.n_ckpt + c) * kState);
+        load_ckpt(a.ckpt + (chain * a.ckpt_stride + c) * kState);
         for (long long m = m0g; m + 1 < m1g; ++m) {  // the group's states but its last, kept in the slab
             save_state(slab + (m - m0g) * kState);
             fwd_step(m * K, buf, m + 2 < m1g ? Next{1, (m + 1) * K, K} : Next{2, (m1g - 1) * K, K});

@@ -70,6 +70,11 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
         const bool full = m < a.n_full;
         const int Km = full ? a.K : static_cast<int>(a.rem);
         const long long t0 = m * a.K;
+        if (a.ckpt && full && m % a.ckpt_G == 0) {  // a checkpoint for the backward: the state before m
+            float* d = a.ckpt + (chain * a.ckpt_stride + m / a.ckpt_G) * (TTT_D * TTT_D + TTT_D);
+            for (int i = tid; i < TTT_D * TTT_D; i += kThreads) d[i] = s.W[i];
+            if (tid < TTT_D) d[TTT_D * TTT_D + tid] = s.b[tid];
+        }
 
         for (int i = tid; i < TTT_KMAX * TTT_D; i += kThreads) {
             int r = i / TTT_D, c = i % TTT_D;
@@ -182,6 +187,11 @@ __global__ void __launch_bounds__(kThreads) linear_simt_kernel(LinearArgs a) {
     float* Wl = a.W_last + chain * TTT_D * TTT_D;
     for (int i = tid; i < TTT_D * TTT_D; i += kThreads) Wl[i] = s.W[i];
     if (tid < TTT_D) a.b_last[chain * TTT_D + tid] = s.b[tid];
+    if (a.ckpt) {  // the state after the last full mini-batch, the last checkpoint entry
+        float* d = a.ckpt + (chain * a.ckpt_stride + a.ckpt_stride - 1) * (TTT_D * TTT_D + TTT_D);
+        for (int i = tid; i < TTT_D * TTT_D; i += kThreads) d[i] = s.W[i];
+        if (tid < TTT_D) d[TTT_D * TTT_D + tid] = s.b[tid];
+    }
     if (a.rem == 0) {
         if (a.W_grad_tail)
             for (int i = tid; i < TTT_D * TTT_D; i += kThreads) a.W_grad_tail[chain * TTT_D * TTT_D + i] = 0.f;
@@ -197,13 +207,17 @@ __global__ void linear_state_copy_kernel(LinearArgs a) {
                                                  : static_cast<long long>(h) * TTT_D * TTT_D);
     const float* b0 = a.b0 + (a.w0_chain_stride ? chain * TTT_D : static_cast<long long>(h) * TTT_D);
     float* Wl = a.W_last + chain * TTT_D * TTT_D;
+    // (no full mini-batch: the only checkpoint entry is the state after none, W0 and b0)
+    float* ck = a.ckpt ? a.ckpt + (chain * a.ckpt_stride + a.ckpt_stride - 1) * (TTT_D * TTT_D + TTT_D) : nullptr;
     for (int i = threadIdx.x; i < TTT_D * TTT_D; i += blockDim.x) {
         float w = W0[i];
         Wl[i] = w;
+        if (ck) ck[i] = w;
         if (a.W_grad_tail) a.W_grad_tail[chain * TTT_D * TTT_D + i] = 0.f;
     }
     if (threadIdx.x < TTT_D) {
         a.b_last[chain * TTT_D + threadIdx.x] = b0[threadIdx.x];
+        if (ck) ck[TTT_D * TTT_D + threadIdx.x] = b0[threadIdx.x];
         if (a.b_grad_tail) a.b_grad_tail[chain * TTT_D + threadIdx.x] = 0.f;
     }
 }

@@ -213,7 +213,7 @@ __device__ __forceinline__ void store_out(const float4 (*red)[2], const LinearAr
 // kTok: token-major activations ([B, L, H, 64], 4-D tensor maps) or head-major ([B, H, L, 64],
 // 3-D tensor maps over [B*H, L, 64]).  kRope: rotate XQ and XK, pairs (2k, 2k+1) (1) or
 // (k, k + d/2) (2); 0: no rotation.
-template <bool kTok, int kRope>
+template <bool kTok, int kRope, bool kCkpt>
 __global__ void __launch_bounds__(kBlock, 2)
 linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     // align by a byte offset from the shared array itself (an integer round trip of the pointer
@@ -323,6 +323,21 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         Bt[0] = a.b0[b0off + 16 * w + g];
         Bt[2] = a.b0[b0off + 16 * w + g + 8];
     }
+    // the state (W as [k][n] at Wd, b at bd) from the accumulators
+    auto store_state = [&](float* Wd, float* bd) {
+#pragma unroll
+        for (int jt = 0; jt < 8; ++jt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
+                Wd[j * TTT_D + f] = Wt[jt][e];
+            }
+        if (t == 0) {
+            bd[16 * w + g] = Bt[0];
+            bd[16 * w + g + 8] = Bt[2];
+        }
+    };
+    auto put_state = [&](float* dst) { store_state(dst, dst + TTT_D * TTT_D); };  // one checkpoint entry
     const uint32_t ones_b = (g == 0) ? 0x3c003c00u : 0u;  // fp16 B operand: ones in column 0
     float bc[2][2], lw[2][2], lb[2][2];  // per n-tile nt, feature 16w + 8nt + 2t + e
 #pragma unroll
@@ -410,7 +425,8 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
         const int Km = full_mb ? K : static_cast<int>(a.rem);
         const int st1 = st + 1 == kStages ? 0 : st + 1;
         const uint32_t par1 = par ^ (st1 == 0 ? 1u : 0u);
-        // the next stage: tested now, so that the test's latency hides behind the MMAs below
+        if (kCkpt && full_mb && m % a.ckpt_G == 0)  // a checkpoint for the backward: the state before m
+            put_state(a.ckpt + (static_cast<long long>(chain) * a.ckpt_stride + m / a.ckpt_G) * (TTT_D * TTT_D + TTT_D));
         // the next stage: tested now, so that the test's latency hides behind the MMAs below
         bool have_next = (m + 1 < n_mb) && mbar_test_wait(&s.full[st1], par1);
         const uint32_t xq_s = smem_u32(&s.xq[st][0]), xk_s = smem_u32(&s.xk[st][0]);
@@ -640,18 +656,9 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     }
 
     // ---- final state ------------------------------------------------------------------------
-    float* Wl = a.W_last + static_cast<long long>(chain) * TTT_D * TTT_D;
-#pragma unroll
-    for (int jt = 0; jt < 8; ++jt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
-            Wl[j * TTT_D + f] = Wt[jt][e];
-        }
-    if (t == 0) {
-        a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + g] = Bt[0];
-        a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + g + 8] = Bt[2];
-    }
+    store_state(a.W_last + static_cast<long long>(chain) * TTT_D * TTT_D, a.b_last + static_cast<long long>(chain) * TTT_D);
+    if (kCkpt)  // the state after the last full mini-batch, the last checkpoint entry
+        put_state(a.ckpt + (static_cast<long long>(chain) * a.ckpt_stride + a.ckpt_stride - 1) * (TTT_D * TTT_D + TTT_D));
     if (a.rem == 0) {
         if (a.W_grad_tail)
             for (int i = tid; i < TTT_D * TTT_D; i += kThreads)
@@ -664,9 +671,12 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
 
 cudaError_t launch_linear_tc(const LinearArgs& a, const LinearMaps& maps, cudaStream_t st) {
     const size_t smem = sizeof(TcSmem) + 1024;  // + alignment slack
-    auto kernel = a.rope == 2 ? (a.tok_major ? linear_tc_kernel<true, 2> : linear_tc_kernel<false, 2>)
-                : a.rope == 1 ? (a.tok_major ? linear_tc_kernel<true, 1> : linear_tc_kernel<false, 1>)
-                              : (a.tok_major ? linear_tc_kernel<true, 0> : linear_tc_kernel<false, 0>);
+    // (checkpoints are written by their own instantiations, so that the plain scan carries none of
+    // that code; the rotary forms take none)
+    auto kernel = a.rope == 2 ? (a.tok_major ? linear_tc_kernel<true, 2, false> : linear_tc_kernel<false, 2, false>)
+                : a.rope == 1 ? (a.tok_major ? linear_tc_kernel<true, 1, false> : linear_tc_kernel<false, 1, false>)
+                : a.ckpt      ? (a.tok_major ? linear_tc_kernel<true, 0, true> : linear_tc_kernel<false, 0, true>)
+                              : (a.tok_major ? linear_tc_kernel<true, 0, false> : linear_tc_kernel<false, 0, false>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     kernel<<<static_cast<unsigned>(a.B * a.H), kBlock, smem, st>>>(a, maps);

@@ -188,7 +188,7 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
                    const float* W0, const float* b0, long long w0_chain_stride, const float* ln_w, const float* ln_b,
                    int B, int H, long long L, int mini_batch, float eps, int dtype, unsigned int flags, void* out,
                    float* W_last, float* b_last, float* W_grad_tail, float* b_grad_tail, cudaStream_t st,
-                   int rope = 0, float rope_theta = 0.f) {
+                   int rope = 0, float rope_theta = 0.f, float* ckpt = nullptr, int ckpt_group = 0) {
     int rc;
     ttt::LinearArgs a{};
     a.XQ = XQ; a.XK = XK; a.XV = XV; a.lr = lr; a.token_eta = token_eta;
@@ -200,6 +200,9 @@ int enqueue_linear(const void* XQ, const void* XK, const void* XV, const float* 
     a.wait_limit = wait_limit();
     a.rope = rope;
     a.rope_theta = rope_theta;
+    a.ckpt = ckpt;
+    a.ckpt_G = ckpt_group;
+    a.ckpt_stride = ckpt ? (a.n_full + ckpt_group - 1) / ckpt_group + 1 : 0;
     const bool tm = (flags & TTT_FLAG_TOKEN_MAJOR) != 0;
     set_act_strides(a, H, L, tm);
 
@@ -348,9 +351,12 @@ static int linear_forward_checked(const void* XQ, const void* XK, const void* XV
                                   long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
                                   long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
                                   int rope, float rope_theta, void* out, float* W_last, float* b_last,
-                                  float* W_grad_tail, float* b_grad_tail, void* stream) {
+                                  float* W_grad_tail, float* b_grad_tail, void* stream, float* ckpt = nullptr,
+                                  int ckpt_group = 0) {
     int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
     if (rc) return rc;
+    if (ckpt && ckpt_group < 1) return fail(TTT_ERR_ARG, "ckpt_group must be >= 1 (got %d)", ckpt_group);
+    if (ckpt && !aligned(ckpt, 16)) return fail(TTT_ERR_ALIGN, "ckpt must be 16-byte aligned");
     const long long chains = static_cast<long long>(B) * H;
     const long long per_head = static_cast<long long>(kD) * kD;
     if (w0_batch_stride != 0 && w0_batch_stride != H * per_head)
@@ -375,17 +381,19 @@ static int linear_forward_checked(const void* XQ, const void* XK, const void* XV
                  {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4},
                  {"W0", W0, static_cast<size_t>(wrows * per_head) * 4}, {"b0", b0, static_cast<size_t>(wrows * kD) * 4},
                  {"ln_w", ln_w, static_cast<size_t>(H) * kD * 4}, {"ln_b", ln_b, static_cast<size_t>(H) * kD * 4}};
+    const size_t ckpt_bytes = ckpt ? static_cast<size_t>(chains) * ((L / mini_batch + ckpt_group - 1) / ckpt_group + 1) *
+                                         (per_head + kD) * 4 : 0;
     Span outs[] = {{"out", out, act}, {"W_last", W_last, static_cast<size_t>(chains * per_head) * 4},
                    {"b_last", b_last, static_cast<size_t>(chains * kD) * 4},
                    {"W_grad_tail", W_grad_tail, static_cast<size_t>(chains * per_head) * 4},
-                   {"b_grad_tail", b_grad_tail, static_cast<size_t>(chains * kD) * 4}};
+                   {"b_grad_tail", b_grad_tail, static_cast<size_t>(chains * kD) * 4}, {"ckpt", ckpt, ckpt_bytes}};
     const int same_ok[2][2] = {{1, 5}, {2, 6}};  // W_last == W0, b_last == b0 (per-chain state)
-    rc = check_aliasing(in, 9, outs, 5, same_ok, 2);
+    rc = check_aliasing(in, 9, outs, 6, same_ok, 2);
     if (rc) return rc;
 
     return enqueue_linear(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride ? per_head : 0, ln_w, ln_b, B, H, L,
                           mini_batch, eps, dtype, flags, out, W_last, b_last, W_grad_tail, b_grad_tail,
-                          static_cast<cudaStream_t>(stream), rope, rope_theta);
+                          static_cast<cudaStream_t>(stream), rope, rope_theta, ckpt, ckpt_group);
 }
 
 int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const float* lr,
@@ -397,6 +405,27 @@ int ttt_linear_forward(const void* XQ, const void* XK, const void* XV, const flo
     return linear_forward_checked(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d,
                                   mini_batch, eps, dtype, flags, 0, 0.f, out, W_last, b_last, W_grad_tail,
                                   b_grad_tail, stream);
+}
+
+long long ttt_linear_ckpt_bytes(int B, int H, long long L, int d, int mini_batch, int ckpt_group) {
+    int rc = check_common(B, H, L, d, mini_batch, 1.0f, TTT_F32, 0);
+    if (rc) return rc;
+    if (ckpt_group < 1) return fail(TTT_ERR_ARG, "ckpt_group must be >= 1 (got %d)", ckpt_group);
+    ok();
+    const long long n_ckpt = (L / mini_batch + ckpt_group - 1) / ckpt_group;
+    return static_cast<long long>(B) * H * (n_ckpt + 1) * (kD * kD + kD) * 4;
+}
+
+int ttt_linear_forward_ckpt(const void* XQ, const void* XK, const void* XV, const float* lr,
+                            const float* token_eta, const float* W0, const float* b0,
+                            long long w0_batch_stride, const float* ln_w, const float* ln_b, int B, int H,
+                            long long L, int d, int mini_batch, float eps, int dtype, unsigned int flags,
+                            void* out, float* W_last, float* b_last, float* W_grad_tail,
+                            float* b_grad_tail, int ckpt_group, float* ckpt, void* stream) {
+    if (!ckpt) return fail(TTT_ERR_ARG, "ckpt must be non-null");
+    return linear_forward_checked(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d,
+                                  mini_batch, eps, dtype, flags, 0, 0.f, out, W_last, b_last, W_grad_tail,
+                                  b_grad_tail, stream, ckpt, ckpt_group);
 }
 
 int ttt_linear_forward_rope(const void* XQ, const void* XK, const void* XV, const float* lr,
@@ -779,12 +808,14 @@ long long ttt_linear_backward_workspace_bytes(int B, int H, long long L, int d, 
     return static_cast<long long>(bwd_layout(B, H, L, mini_batch, ckpt_group).total);
 }
 
-int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
-                        const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
-                        const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps, int dtype,
-                        unsigned int flags, int ckpt_group, const void* d_out, const float* dW_last,
-                        const float* db_last, void* dXQ, void* dXK, void* dXV, float* d_lr, float* dW0, float* db0,
-                        float* d_ln_w, float* d_ln_b, void* workspace, long long workspace_bytes, void* stream) {
+// ttt_linear_backward and ttt_linear_backward_ckpt (ckpt_in: the forward's checkpoints, or null).
+static int linear_backward_impl(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                                const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
+                                const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps,
+                                int dtype, unsigned int flags, int ckpt_group, const float* ckpt_in,
+                                const void* d_out, const float* dW_last, const float* db_last, void* dXQ, void* dXK,
+                                void* dXV, float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b,
+                                void* workspace, long long workspace_bytes, void* stream) {
     int rc = check_common(B, H, L, d, mini_batch, eps, dtype, flags);
     if (rc) return rc;
     if (flags & TTT_FLAG_FP32_COMPUTE)
@@ -798,9 +829,10 @@ int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const fl
         return fail(TTT_ERR_ARG, "W0, b0, ln_w, ln_b, dW0, db0, d_ln_w, d_ln_b and workspace must be non-null");
     if (L > 0 && (!XQ || !XK || !XV || !lr || !d_out || !dXQ || !dXK || !dXV || !d_lr))
         return fail(TTT_ERR_ARG, "XQ, XK, XV, lr, d_out, dXQ, dXK, dXV and d_lr must be non-null when L > 0");
-    const void* a16[] = {XQ, XK, XV, d_out, dXQ, dXK, dXV, W0, b0, dW_last, db_last, dW0, db0};
-    const char* n16[] = {"XQ", "XK", "XV", "d_out", "dXQ", "dXK", "dXV", "W0", "b0", "dW_last", "db_last", "dW0", "db0"};
-    for (int i = 0; i < 13; ++i)
+    const void* a16[] = {XQ, XK, XV, d_out, dXQ, dXK, dXV, W0, b0, dW_last, db_last, dW0, db0, ckpt_in};
+    const char* n16[] = {"XQ", "XK", "XV", "d_out", "dXQ", "dXK", "dXV", "W0", "b0", "dW_last", "db_last", "dW0", "db0",
+                         "ckpt"};
+    for (int i = 0; i < 14; ++i)
         if (a16[i] && !aligned(a16[i], 16)) return fail(TTT_ERR_ALIGN, "%s must be 16-byte aligned", n16[i]);
     const void* a4[] = {lr, token_eta, ln_w, ln_b, d_lr, d_ln_w, d_ln_b};
     const char* n4[] = {"lr", "token_eta", "ln_w", "ln_b", "d_lr", "d_ln_w", "d_ln_b"};
@@ -821,11 +853,12 @@ int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const fl
                  {"token_eta", token_eta, static_cast<size_t>(mini_batch) * 4}, {"W0", W0, wbytes}, {"b0", b0, bbytes},
                  {"ln_w", ln_w, hbytes}, {"ln_b", ln_b, hbytes}, {"d_out", d_out, act},
                  {"dW_last", dW_last, static_cast<size_t>(chains * per_head) * 4},
-                 {"db_last", db_last, static_cast<size_t>(chains * kD) * 4}};
+                 {"db_last", db_last, static_cast<size_t>(chains * kD) * 4},
+                 {"ckpt", ckpt_in, ckpt_in ? static_cast<size_t>(chains) * (lay.n_ckpt + 1) * (per_head + kD) * 4 : 0}};
     Span outs[] = {{"dXQ", dXQ, act}, {"dXK", dXK, act}, {"dXV", dXV, act}, {"d_lr", d_lr, tok},
                    {"dW0", dW0, wbytes}, {"db0", db0, bbytes}, {"d_ln_w", d_ln_w, hbytes}, {"d_ln_b", d_ln_b, hbytes},
                    {"workspace", workspace, lay.total}};
-    rc = check_aliasing(in, 12, outs, 9);
+    rc = check_aliasing(in, 13, outs, 9);
     if (rc) return rc;
 
     ttt::LinearBwdArgs a{};
@@ -842,7 +875,9 @@ int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const fl
     a.eps = eps; a.G = ckpt_group; a.n_ckpt = lay.n_ckpt;
     a.dXQ = dXQ; a.dXK = dXK; a.dXV = dXV; a.d_lr = d_lr;
     char* ws = static_cast<char*>(workspace);
-    a.ckpt = reinterpret_cast<float*>(ws);
+    a.ckpt = ckpt_in ? const_cast<float*>(ckpt_in) : reinterpret_cast<float*>(ws);  // (read only when given)
+    a.ckpt_stride = ckpt_in ? lay.n_ckpt + 1 : lay.n_ckpt;
+    a.ckpt_given = ckpt_in ? 1 : 0;
     a.slab = reinterpret_cast<float*>(ws + lay.slab);
     a.part = reinterpret_cast<float*>(ws + lay.part);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -851,6 +886,30 @@ int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const fl
     e = ttt::launch_linear_bwd_reduce(a.part, B, H, w0_batch_stride ? 1 : 0, dW0, db0, d_ln_w, d_ln_b, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward reduction launch");
     return ok();
+}
+
+int ttt_linear_backward(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                        const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
+                        const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps, int dtype,
+                        unsigned int flags, int ckpt_group, const void* d_out, const float* dW_last,
+                        const float* db_last, void* dXQ, void* dXK, void* dXV, float* d_lr, float* dW0, float* db0,
+                        float* d_ln_w, float* d_ln_b, void* workspace, long long workspace_bytes, void* stream) {
+    return linear_backward_impl(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d,
+                                mini_batch, eps, dtype, flags, ckpt_group, nullptr, d_out, dW_last, db_last, dXQ, dXK,
+                                dXV, d_lr, dW0, db0, d_ln_w, d_ln_b, workspace, workspace_bytes, stream);
+}
+
+int ttt_linear_backward_ckpt(const void* XQ, const void* XK, const void* XV, const float* lr, const float* token_eta,
+                             const float* W0, const float* b0, long long w0_batch_stride, const float* ln_w,
+                             const float* ln_b, int B, int H, long long L, int d, int mini_batch, float eps,
+                             int dtype, unsigned int flags, int ckpt_group, const float* ckpt, const void* d_out,
+                             const float* dW_last, const float* db_last, void* dXQ, void* dXK, void* dXV,
+                             float* d_lr, float* dW0, float* db0, float* d_ln_w, float* d_ln_b, void* workspace,
+                             long long workspace_bytes, void* stream) {
+    if (!ckpt) return fail(TTT_ERR_ARG, "ckpt must be non-null");
+    return linear_backward_impl(XQ, XK, XV, lr, token_eta, W0, b0, w0_batch_stride, ln_w, ln_b, B, H, L, d,
+                                mini_batch, eps, dtype, flags, ckpt_group, ckpt, d_out, dW_last, db_last, dXQ, dXK,
+                                dXV, d_lr, dW0, db0, d_ln_w, d_ln_b, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -40,6 +40,11 @@ struct LinearArgs {
     float* b_grad_tail;
     unsigned int* status;     // device status word
     long long wait_limit;     // polls per bounded wait
+    // checkpoints for the backward (or nullptr): the state (W as [k][n], then b) before every
+    // ckpt_G-th full mini-batch, then the state after the last full one, ckpt_stride per chain
+    float* ckpt;
+    int ckpt_G;
+    long long ckpt_stride;
 };
 
 struct MlpArgs {
@@ -169,7 +174,10 @@ struct LinearBwdArgs {
     void* dXK;
     void* dXV;
     float* d_lr;
-    float* ckpt;                // [B*H][n_ckpt][d*d + d]
+    float* ckpt;                // [B*H][ckpt_stride][d*d + d]: W ([k][n]) and b before every G-th full mini-batch
+    long long ckpt_stride;      // states per chain in ckpt
+    int ckpt_given;             // 1: ckpt holds the caller's checkpoints, the state after the last full
+                                //    mini-batch at index n_ckpt; phase 1 is skipped
     float* slab;                // [B*H][G][d*d + d]
     float* part;                // [B*H][d*d + 3d]: dW0, db0, d ln_w, d ln_b of each chain
 };

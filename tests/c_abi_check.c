@@ -78,5 +78,19 @@ int main(void) {
     check(ttt_linear_backward(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0u, 0, out,
                               NULL, NULL, g[0], g[1], g[2], g[3], g[4], g[5], g[6], g[7], NULL, 0, NULL) == TTT_ERR_ARG,
           "backward rejects ckpt_group = 0");
+    const long long cks = ttt_linear_ckpt_bytes(8, 32, 8200, 64, 16, 16);
+    check(cks == 8LL * 32 * 33 * (64 * 64 + 64) * 4, "checkpoint buffer size");
+    check(ttt_linear_ckpt_bytes(8, 32, 8200, 64, 16, 0) == TTT_ERR_ARG, "checkpoint size rejects ckpt_group = 0");
+    float* ck = (float*)((uintptr_t)20 * A);  /* fake checkpoint buffer */
+    check(ttt_linear_forward_ckpt(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0u,
+                                  out, Wl, bl, NULL, NULL, 4, NULL, NULL) == TTT_ERR_ARG,
+          "forward with checkpoints rejects a null buffer");
+    check(ttt_linear_forward_ckpt(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0u,
+                                  out, Wl, bl, NULL, NULL, 0, ck, NULL) == TTT_ERR_ARG,
+          "forward with checkpoints rejects ckpt_group = 0");
+    check(ttt_linear_backward_ckpt(XQ, XK, XV, lr, NULL, W0, b0, 0, lnw, lnb, 2, 3, 64, 64, 16, 1e-6f, TTT_BF16, 0u, 4,
+                                   NULL, out, NULL, NULL, g[0], g[1], g[2], g[3], g[4], g[5], g[6], g[7], NULL, 0,
+                                   NULL) == TTT_ERR_ARG,
+          "backward from checkpoints rejects a null buffer");
     return failures == 0 ? 0 : 1;
 }

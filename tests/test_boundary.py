@@ -337,3 +337,58 @@ def test_linear_backward_workspace_bytes(libttt):
     assert libttt.ttt_linear_backward_workspace_bytes(2, 3, 0, 16, 16) == up(6 * 16 * state) + up(6 * (64 * 64 + 192) * 4)
     with pytest.raises(libttt.TTTError):
         libttt.ttt_linear_backward_workspace_bytes(2, 3, 100, 16, 0)
+
+
+def _fwd_ckpt(lib, G=4, ck=19 * A, **kw):
+    args = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W0=5 * A, b0=6 * A, stride=0, lnw=7 * A,
+                lnb=8 * A, B=2, H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, flags=0, out=9 * A,
+                Wl=10 * A, bl=11 * A, Wg=None, bg=None)
+    args.update(kw)
+    return lib.ttt_linear_forward_ckpt(args["XQ"], args["XK"], args["XV"], args["lr"], args["te"], args["W0"],
+                                       args["b0"], args["stride"], args["lnw"], args["lnb"], args["B"], args["H"],
+                                       args["L"], args["d"], args["K"], args["eps"], args["dtype"], args["flags"],
+                                       args["out"], args["Wl"], args["bl"], args["Wg"], args["bg"], G, ck, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ck=None), -1), (dict(G=0), -1), (dict(ck=19 * A + 8), -2), (dict(ck=9 * A), -3),
+    (dict(ck=10 * A + 64), -3), (dict(ck=A), -3), (dict(K=0), -1), (dict(d=32), -6),
+])
+def test_linear_forward_ckpt_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _fwd_ckpt(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
+def _bwd_ckpt(lib, ck=19 * A, **kw):
+    a = dict(XQ=A, XK=2 * A, XV=3 * A, lr=4 * A, te=None, W0=5 * A, b0=6 * A, stride=0, lnw=7 * A, lnb=8 * A, B=2,
+             H=3, L=64, d=64, K=16, eps=1e-6, dtype=1, flags=0, G=4, dout=9 * A, dWl=None, dbl=None, dXQ=10 * A,
+             dXK=11 * A, dXV=12 * A, dlr=13 * A, dW0=14 * A, db0=15 * A, dlnw=16 * A, dlnb=17 * A, ws=1 << 32,
+             wsb=1 << 30)
+    a.update(kw)
+    return lib.ttt_linear_backward_ckpt(a["XQ"], a["XK"], a["XV"], a["lr"], a["te"], a["W0"], a["b0"], a["stride"],
+                                        a["lnw"], a["lnb"], a["B"], a["H"], a["L"], a["d"], a["K"], a["eps"],
+                                        a["dtype"], a["flags"], a["G"], ck, a["dout"], a["dWl"], a["dbl"], a["dXQ"],
+                                        a["dXK"], a["dXV"], a["dlr"], a["dW0"], a["db0"], a["dlnw"], a["dlnb"],
+                                        a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ck=None), -1), (dict(G=0), -1), (dict(ck=19 * A + 4), -2), (dict(ck=10 * A), -3),
+    (dict(ck=(1 << 32) + 4096), -3), (dict(flags=1), -6), (dict(wsb=100), -1),
+])
+def test_linear_backward_ckpt_rejects(libttt, kw, code):
+    lib = libttt.lib()
+    assert _bwd_ckpt(lib, **kw) == code
+    assert lib.ttt_last_error_message()
+
+
+def test_linear_ckpt_bytes(libttt):
+    # per chain: ceil(n_full / G) group starts + the state after the last full mini-batch
+    state = (64 * 64 + 64) * 4
+    assert libttt.ttt_linear_ckpt_bytes(2, 3, 8200, 16, 16) == 6 * (32 + 1) * state
+    assert libttt.ttt_linear_ckpt_bytes(2, 3, 8200, 16, 5) == 6 * (103 + 1) * state
+    assert libttt.ttt_linear_ckpt_bytes(2, 3, 15, 16, 4) == 6 * 1 * state
+    assert libttt.ttt_linear_ckpt_bytes(2, 3, 0, 16, 4) == 6 * 1 * state
+    with pytest.raises(libttt.TTTError):
+        libttt.ttt_linear_ckpt_bytes(2, 3, 100, 16, 0)
