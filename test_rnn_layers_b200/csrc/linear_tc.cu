@@ -656,7 +656,22 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     }
 
     // ---- final state ------------------------------------------------------------------------
-    store_state(a.W_last + static_cast<long long>(chain) * TTT_D * TTT_D, a.b_last + static_cast<long long>(chain) * TTT_D);
+    if constexpr (kRope == 0) {
+        store_state(a.W_last + static_cast<long long>(chain) * TTT_D * TTT_D, a.b_last + static_cast<long long>(chain) * TTT_D);
+    } else {  // (the same stores, written out: the rotary forms allocate their registers better this way)
+        float* Wl = a.W_last + static_cast<long long>(chain) * TTT_D * TTT_D;
+#pragma unroll
+        for (int jt = 0; jt < 8; ++jt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 8 * jt + 2 * t + (e & 1), f = 16 * w + g + 8 * (e >> 1);
+                Wl[j * TTT_D + f] = Wt[jt][e];
+            }
+        if (t == 0) {
+            a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + g] = Bt[0];
+            a.b_last[static_cast<long long>(chain) * TTT_D + 16 * w + g + 8] = Bt[2];
+        }
+    }
     if (kCkpt)  // the state after the last full mini-batch, the last checkpoint entry
         put_state(a.ckpt + (static_cast<long long>(chain) * a.ckpt_stride + a.ckpt_stride - 1) * (TTT_D * TTT_D + TTT_D));
     if (a.rem == 0) {
