@@ -419,14 +419,23 @@ linear_tc_kernel(const LinearArgs a, const __grid_constant__ LinearMaps maps) {
     bool failed = false;
     int m = 0, st = 0;
     uint32_t par = 0;
+    // (checkpoint instantiations: the next entry to write, and the full mini-batches until then)
+    float* ck_next = kCkpt ? a.ckpt + static_cast<long long>(chain) * a.ckpt_stride * (TTT_D * TTT_D + TTT_D) : nullptr;
+    int ck_wait = 0;
 
     for (; m < n_mb; ++m, st = (st + 1 == kStages ? 0 : st + 1), par ^= (st == 0)) {
         const bool full_mb = m < n_full;
         const int Km = full_mb ? K : static_cast<int>(a.rem);
         const int st1 = st + 1 == kStages ? 0 : st + 1;
         const uint32_t par1 = par ^ (st1 == 0 ? 1u : 0u);
-        if (kCkpt && full_mb && m % a.ckpt_G == 0)  // a checkpoint for the backward: the state before m
-            put_state(a.ckpt + (static_cast<long long>(chain) * a.ckpt_stride + m / a.ckpt_G) * (TTT_D * TTT_D + TTT_D));
+        if (kCkpt && full_mb) {  // a checkpoint for the backward: the state before every G-th m
+            if (ck_wait == 0) {
+                put_state(ck_next);
+                ck_next += TTT_D * TTT_D + TTT_D;
+                ck_wait = a.ckpt_G;
+            }
+            --ck_wait;
+        }
         // the next stage: tested now, so that the test's latency hides behind the MMAs below
         bool have_next = (m + 1 < n_mb) && mbar_test_wait(&s.full[st1], par1);
         const uint32_t xq_s = smem_u32(&s.xq[st][0]), xk_s = smem_u32(&s.xk[st][0]);
