@@ -545,6 +545,26 @@ def bench_linear_backward(args, world, peaks, G=16):
 
     ms_ck = time_steps(step_from_ckpt, K, 3, world)
     del ws, ckpt
+    # a whole training step of the layer's scan at checkpoint groups G and 1 (every state kept):
+    # the forward with checkpoints, then the backward from them
+    train = {}
+    for Gt in (G, 1):
+        ws = torch.empty(ttt.ttt_linear_backward_workspace_bytes(w.B, w.H, w.L, w.K, Gt), dtype=torch.uint8,
+                         device="cuda")
+        ckpt = torch.empty(ttt.ttt_linear_ckpt_bytes(w.B, w.H, w.L, w.K, Gt) // 4, device="cuda")
+
+        def train_step(Gt=Gt, ws=ws, ckpt=ckpt):
+            ttt.ttt_linear_forward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], mini_batch=w.K,
+                                   eps=w.eps, ckpt=ckpt, ckpt_group=Gt)
+            g = ttt.ttt_linear_backward(XQ, XK, XV, t["lr"], t["W0"], t["b0"], t["ln_w"], t["ln_b"], dout, dWl, dbl,
+                                        mini_batch=w.K, eps=w.eps, ckpt_group=Gt, workspace=ws, ckpt=ckpt)
+            if world > 1:
+                allreduce_shared_grads(g)
+
+        ms_t = time_steps(train_step, K, 3, world)
+        train[f"ckpt_group_{Gt}"] = {"ms_per_step": round(ms_t, 4), "value": round(world * w.B * w.L / (ms_t / 1e3), 1),
+                                     "checkpoint_bytes": ckpt.numel() * 4}
+        del ws, ckpt
     flops, nbytes = linear_bwd_flops(w.B, w.H, w.L), linear_bwd_bytes(w.B, w.H, w.L)
     tfl = flops / (ms / 1e3) / 1e12
     gbs = nbytes / (ms / 1e3) / 1e9
@@ -560,6 +580,7 @@ def bench_linear_backward(args, world, peaks, G=16):
             "from_forward_checkpoints": {"ckpt_group": G, "call": "ttt_linear_backward_ckpt",
                                          "ms_per_step": round(ms_ck, 4),
                                          "value": round(world * w.B * w.L / (ms_ck / 1e3), 1)},
+            "training_step": dict(train, calls="ttt_linear_forward_ckpt then ttt_linear_backward_ckpt"),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "peak_source": f"{which} hbm_gbs",
                          "unit": "GB/s", "frac": round(gbs / hbm, 4), "algorithmic_bytes": nbytes,
                          "floor_ms": round(nbytes / hbm / 1e6, 4), "algorithmic_flops": flops,
