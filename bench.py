@@ -813,7 +813,7 @@ def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--rows", default="linear,linear_tm,linear_rope,oproj,backward,mlp,decode,decode_hist",
                     help="comma list: linear (the headline) plus mlp and decode rows in the same line")
